@@ -1,0 +1,257 @@
+"""The oracle: a plain, slow CPU encoder/decoder for the BF16RANS container.
+
+This package is TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import it. The GPU library never does, and the
+two share no code.
+
+What it computes: the method paragraph of the "Qwen3.8-27B-BF16-NVLC-Lossless" model
+card, which splits each BF16 word into sign, exponent and fraction, codes the
+sign+exponent symbol with a per-tensor rANS model, and lets that symbol select the
+fraction's distribution. The byte layout and every parameter come from FORMAT.md.
+The arithmetic lives in ``bsoracle.c``. This module only marshals arguments through
+ctypes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bsoracle.c")
+_LIB = os.path.join(_HERE, "libbsoracle.so")
+
+OK, E_ARG, E_FORMAT, E_VERSION, E_SIZE, E_CORRUPT, E_NOMEM = 0, 1, 2, 3, 4, 6, 7
+KIND_RANS, KIND_STORED, KIND_RAW = 0, 1, 2
+_NAMES = {1: "E_ARG", 2: "E_FORMAT", 3: "E_VERSION", 4: "E_SIZE", 6: "E_CORRUPT", 7: "E_NOMEM"}
+
+
+class OracleError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"oracle {what}: status {code} ({_NAMES.get(code, '?')})")
+        self.code = code
+
+
+def build(force: bool = False) -> str:
+    """Compile bsoracle.c into libbsoracle.so next to it (plain gcc, no GPU code)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-Wall", "-shared", "-fPIC", _SRC, "-o", tmp])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Item(ctypes.Structure):
+    _fields_ = [
+        ("kind", ctypes.c_uint32),
+        ("ndim", ctypes.c_uint32),
+        ("shape", ctypes.c_uint64 * 8),
+        ("n_elems", ctypes.c_uint64),
+        ("data", ctypes.c_void_p),
+        ("name", ctypes.c_char_p),
+        ("name_bytes", ctypes.c_uint32),
+        ("reserved", ctypes.c_uint32),
+    ]
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_uint32) for k in ("log2_chunk", "ns", "nf", "max_routes", "force_rans")]
+
+
+class _Info(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_uint32) for k in
+                ("kind", "ndim", "log2_chunk", "lanes", "ns", "nf", "n_routes", "name_offset", "name_bytes",
+                 "reserved")] + \
+               [(k, ctypes.c_uint64) for k in
+                ("n_elems", "n_chunks", "model_offset", "model_bytes", "data_offset", "data_bytes", "checksum")] + \
+               [("shape", ctypes.c_uint64 * 8), ("coded_bytes", ctypes.c_uint64)]
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        P, u32, u64, i64 = ctypes.c_void_p, ctypes.c_uint32, ctypes.c_uint64, ctypes.c_int64
+        L.bso_encode.argtypes = [ctypes.POINTER(_Item), u32, ctypes.POINTER(_Params), ctypes.POINTER(P),
+                                 ctypes.POINTER(u64)]
+        L.bso_free.argtypes = [P]
+        L.bso_free.restype = None
+        L.bso_validate.argtypes = [P, u64, ctypes.POINTER(u32)]
+        L.bso_tensor_info_get.argtypes = [P, u64, u32, ctypes.POINTER(_Info)]
+        L.bso_decode.argtypes = [P, u64, u32, P, u64, ctypes.POINTER(i64)]
+        L.bso_decode_chunks.argtypes = [P, u64, u32, u64, u64, P, u64, ctypes.POINTER(i64)]
+        L.bso_quantise.argtypes = [P, u32, u32, P]
+        L.bso_choose_routes.argtypes = [P, u32, P, ctypes.POINTER(u32), P]
+        L.bso_lane_encode.argtypes = [P, u32, P, P, u32, u32, P, u32, ctypes.POINTER(u64), P, P,
+                                      ctypes.POINTER(u32)]
+        L.bso_lane_decode.argtypes = [P, u32, P, P, u32, u32, u64, P, u32, u32, P, ctypes.POINTER(u64)]
+        L.bso_mix64.argtypes = [u64]
+        L.bso_mix64.restype = u64
+        L.bso_checksum.argtypes = [P, u64, u32]
+        L.bso_checksum.restype = u64
+        for fn in ("bso_encode", "bso_validate", "bso_tensor_info_get", "bso_decode", "bso_decode_chunks",
+                   "bso_quantise", "bso_choose_routes", "bso_lane_encode", "bso_lane_decode"):
+            getattr(L, fn).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data if a.size else 0
+
+
+def _buf(container) -> tuple[np.ndarray, int]:
+    arr = np.frombuffer(container, dtype=np.uint8) if not isinstance(container, np.ndarray) else container
+    assert arr.dtype == np.uint8 and arr.flags["C_CONTIGUOUS"]
+    return arr, arr.size
+
+
+def encode(items, log2_chunk: int = 16, ns: int = 12, nf: int = 10, max_routes: int = 7,
+           force_rans: bool = False) -> bytes:
+    """items: sequence of (name, array, kind) with kind "bf16" (uint16 words, any shape)
+    or "raw" (uint8 bytes). Returns the container bytes (FORMAT.md section 4.6)."""
+    keep = []
+    arr_items = (_Item * max(1, len(items)))()
+    for k, (name, a, kind) in enumerate(items):
+        a = np.ascontiguousarray(a)
+        if kind == "bf16":
+            assert a.dtype == np.uint16
+        else:
+            assert a.dtype == np.uint8
+        nb = name.encode()
+        keep += [a, nb]
+        it = arr_items[k]
+        it.kind = 0 if kind == "bf16" else 2
+        shape = a.shape
+        it.ndim = len(shape)
+        for d, v in enumerate(shape):
+            it.shape[d] = v
+        it.n_elems = a.size
+        it.data = _ptr(a)
+        it.name = nb
+        it.name_bytes = len(nb)
+    p = _Params(log2_chunk, ns, nf, max_routes, 1 if force_rans else 0)
+    out = ctypes.c_void_p()
+    n = ctypes.c_uint64()
+    st = lib().bso_encode(arr_items, len(items), ctypes.byref(p), ctypes.byref(out), ctypes.byref(n))
+    if st:
+        raise OracleError(st, "encode")
+    try:
+        return ctypes.string_at(out.value, n.value)
+    finally:
+        lib().bso_free(out)
+
+
+def validate(container) -> int:
+    arr, n = _buf(container)
+    nt = ctypes.c_uint32()
+    st = lib().bso_validate(_ptr(arr), n, ctypes.byref(nt))
+    if st:
+        raise OracleError(st, "validate")
+    return nt.value
+
+
+def info(container, idx: int) -> dict:
+    arr, n = _buf(container)
+    ti = _Info()
+    st = lib().bso_tensor_info_get(_ptr(arr), n, idx, ctypes.byref(ti))
+    if st:
+        raise OracleError(st, "info")
+    d = {k: getattr(ti, k) for k, _ in _Info._fields_ if k != "shape"}
+    d["shape"] = tuple(ti.shape[i] for i in range(ti.ndim))
+    off = int.from_bytes(bytes(arr[32:40]), "little")
+    d["name"] = bytes(arr[off + ti.name_offset: off + ti.name_offset + ti.name_bytes]).decode()
+    return d
+
+
+def decode(container, idx: int) -> np.ndarray:
+    """Whole tensor: uint16 words (RANS/STORED) or uint8 bytes (RAW)."""
+    arr, n = _buf(container)
+    ti = info(arr, idx)
+    out = np.zeros(ti["n_elems"], dtype=np.uint8 if ti["kind"] == KIND_RAW else np.uint16)
+    bad = ctypes.c_int64(-1)
+    st = lib().bso_decode(_ptr(arr), n, idx, _ptr(out), out.nbytes, ctypes.byref(bad))
+    if st:
+        e = OracleError(st, "decode")
+        e.bad_chunk = bad.value
+        raise e
+    return out.reshape(ti["shape"]) if ti["shape"] else out.reshape(())
+
+
+def decode_chunks(container, idx: int, c0: int, c1: int, out: np.ndarray) -> int:
+    """Decode chunks [c0, c1) of a RANS tensor into out (the whole tensor's uint16 array).
+    Returns the status (0 or E_CORRUPT...) instead of raising, for fault tests."""
+    arr, n = _buf(container)
+    bad = ctypes.c_int64(-1)
+    st = lib().bso_decode_chunks(_ptr(arr), n, idx, c0, c1, _ptr(out), out.nbytes, ctypes.byref(bad))
+    return st
+
+
+def quantise(counts, M: int) -> np.ndarray:
+    c = np.ascontiguousarray(counts, dtype=np.uint64)
+    q = np.zeros(c.size, dtype=np.uint32)
+    st = lib().bso_quantise(_ptr(c), c.size, M, _ptr(q))
+    if st:
+        raise OracleError(st, "quantise")
+    return q
+
+
+def choose_routes(cef, max_routes: int = 7):
+    c = np.ascontiguousarray(cef, dtype=np.uint64).reshape(256 * 128)
+    route = np.zeros(256, dtype=np.uint8)
+    route_e = np.zeros(256, dtype=np.uint32)
+    nr = ctypes.c_uint32()
+    st = lib().bso_choose_routes(_ptr(c), max_routes, _ptr(route), ctypes.byref(nr), _ptr(route_e))
+    if st:
+        raise OracleError(st, "choose_routes")
+    return route, route_e[: nr.value].copy()
+
+
+def _tables(Fs, route, Ff):
+    Fs = np.ascontiguousarray(Fs, dtype=np.uint32)
+    route = np.ascontiguousarray(route, dtype=np.uint8)
+    Ff = np.ascontiguousarray(Ff, dtype=np.uint32).reshape(-1)
+    assert Fs.size == 512 and route.size == 256 and Ff.size % 128 == 0
+    return Fs, route, Ff if Ff.size else np.zeros(128, np.uint32), Ff.size // 128
+
+
+def lane_encode(Fs, ns, route, Ff, nf, words):
+    """One lane (FORMAT.md sections 2-3): returns (start_state, words, tags)."""
+    Fs, route, Ffb, nr = _tables(Fs, route, Ff)
+    w = np.ascontiguousarray(words, dtype=np.uint16)
+    S = w.size
+    wo = np.zeros(max(S, 1), np.uint32)
+    tg = np.zeros(max(S, 1), np.uint32)
+    st_out = ctypes.c_uint64()
+    nw = ctypes.c_uint32()
+    st = lib().bso_lane_encode(_ptr(Fs), ns, _ptr(route), _ptr(Ffb), nr, nf, _ptr(w), S, ctypes.byref(st_out),
+                               _ptr(wo), _ptr(tg), ctypes.byref(nw))
+    if st:
+        raise OracleError(st, "lane_encode")
+    return st_out.value, wo[: nw.value].copy(), tg[: nw.value].copy()
+
+
+def lane_decode(Fs, ns, route, Ff, nf, state, words, S):
+    """Returns (status, decoded words, final state)."""
+    Fs, route, Ffb, nr = _tables(Fs, route, Ff)
+    wd = np.ascontiguousarray(words, dtype=np.uint32)
+    out = np.zeros(max(S, 1), np.uint16)
+    fin = ctypes.c_uint64()
+    st = lib().bso_lane_decode(_ptr(Fs), ns, _ptr(route), _ptr(Ffb), nr, nf, state, _ptr(wd), wd.size, S,
+                               _ptr(out), ctypes.byref(fin))
+    return st, out[:S].copy(), fin.value
+
+
+def mix64(v: int) -> int:
+    return int(lib().bso_mix64(v))
+
+
+def checksum(a: np.ndarray) -> int:
+    """FORMAT.md section 7 checksum of uint16 words or uint8 bytes."""
+    a = np.ascontiguousarray(a).reshape(-1)
+    return int(lib().bso_checksum(_ptr(a), a.size, 2 if a.dtype == np.uint8 else 0))

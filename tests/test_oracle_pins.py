@@ -1,0 +1,272 @@
+"""Pins of the oracle against facts that do not come from the oracle itself.
+
+* FORMAT.md section 8: a container derived by hand (tests/golden/one_weight.hex).
+* The NVLC model card's field split and bitwise reconstruction: every 16-bit pattern
+  round-trips (this covers +-0, subnormals, +-inf and NaN payloads).
+* rANS exactness: brute force over tiny alphabets, where the decode must invert the
+  encode and the end state must be L. The code length must equal the model's ideal
+  cost sum(log2(M/q)) plus the 32-bit start state, up to rANS rounding.
+* The quantiser: closed forms, plus optimality against exhaustive search on small cases.
+* The route rule: the Pearson-statistic threshold at its exact boundary.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+L = 1 << 32
+
+
+def _golden_bytes(path):
+    hexs = []
+    with open(path) as fh:
+        for line in fh:
+            hexs.append(line.split("#", 1)[0])
+    return bytes.fromhex("".join("".join(hexs).split()))
+
+
+# ---------------------------------------------------------------- golden container
+def test_golden_one_weight_encode(golden_dir):
+    want = _golden_bytes(os.path.join(golden_dir, "one_weight.hex"))
+    assert len(want) == 896
+    got = oracle.encode([("w", np.array([0x3F80], np.uint16), "bf16")], force_rans=True)
+    assert got == want
+
+
+def test_golden_one_weight_decode(golden_dir):
+    c = _golden_bytes(os.path.join(golden_dir, "one_weight.hex"))
+    assert oracle.validate(c) == 1
+    ti = oracle.info(c, 0)
+    assert (ti["kind"], ti["ns"], ti["nf"], ti["n_chunks"], ti["name"]) == (0, 12, 10, 1, "w")
+    assert oracle.decode(c, 0).tolist() == [0x3F80]
+
+
+def test_checksum_published_splitmix64_outputs():
+    # splitmix64 seeded with 0 produces e220a8397b1dcdaf, 6e789e6aa1b965f4, 06c45d188009454f
+    g = 0x9E3779B97F4A7C15
+    assert oracle.mix64(0) == 0xE220A8397B1DCDAF
+    assert oracle.mix64(g) == 0x6E789E6AA1B965F4
+    assert oracle.mix64((2 * g) % (1 << 64)) == 0x06C45D188009454F
+
+
+def test_checksum_is_position_sensitive_sum():
+    w = np.array([5, 7, 9], np.uint16)
+    parts = [oracle.mix64((i << 16) | int(v)) for i, v in enumerate(w)]
+    assert oracle.checksum(w) == sum(parts) % (1 << 64)
+    assert oracle.checksum(w[::-1].copy()) != oracle.checksum(w)
+    assert oracle.checksum(np.zeros(0, np.uint16)) == 0
+    b = np.array([1, 2], np.uint8)
+    assert oracle.checksum(b) == (oracle.mix64(1) + oracle.mix64((1 << 8) | 2)) % (1 << 64)
+
+
+def test_one_weight_defaults_to_stored():
+    c = oracle.encode([("w", np.array([0x3F80], np.uint16), "bf16")])
+    assert oracle.info(c, 0)["kind"] == oracle.KIND_STORED
+    assert oracle.decode(c, 0).tolist() == [0x3F80]
+
+
+# ---------------------------------------------------------------- every bit pattern
+def test_all_patterns_one_tensor():
+    w = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    c = oracle.encode([("all", w, "bf16")], force_rans=True)
+    assert oracle.info(c, 0)["kind"] == oracle.KIND_RANS
+    assert np.array_equal(oracle.decode(c, 0), w)
+
+
+def test_all_patterns_single_element_tensors():
+    # 65,536 one-weight tensors: each has a one-symbol s-model (zero-width s code).
+    w = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    items = [(f"p{k}", w[k:k + 1], "bf16") for k in range(65536)]
+    c = oracle.encode(items, force_rans=True)
+    arr = np.frombuffer(c, np.uint8)
+    assert oracle.validate(arr) == 65536
+    for k in range(0, 65536):
+        assert int(oracle.decode(arr, k)[0]) == k
+
+
+def test_field_split_closed_form():
+    # w == (s << 7) | f with s = w >> 7 (9 bits) and f = w & 0x7F (7 bits).
+    w = np.arange(65536, dtype=np.uint32)
+    s, f = w >> 7, w & 0x7F
+    assert s.max() == 511 and f.max() == 127
+    assert np.array_equal((s << 7) | f, w)
+    # sign is bit 8 of s, exponent its low 8 bits: 1.0 = 0x3F80 -> sign 0, exponent 127
+    assert (0x3F80 >> 7) == 127 and (0xBF80 >> 7) == 256 + 127
+
+
+# ---------------------------------------------------------------- brute force, one lane
+def _tables(fs_dict, ns, route=None, ff=None):
+    Fs = np.zeros(512, np.uint32)
+    for k, v in fs_dict.items():
+        Fs[k] = v
+    assert Fs.sum() == 1 << ns
+    r = np.full(256, 0xFF, np.uint8)
+    if route:
+        for e, idx in route.items():
+            r[e] = idx
+    Ff = np.zeros((0, 128), np.uint32) if ff is None else np.asarray(ff, np.uint32)
+    return Fs, r, Ff
+
+
+def _ideal_bits(words, Fs, ns, route, Ff, nf):
+    bits = 0.0
+    for w in words:
+        s, f = int(w) >> 7, int(w) & 0x7F
+        r = int(route[s & 0xFF])
+        qf = (1 << nf) // 128 if r == 0xFF else int(Ff[r][f])
+        bits += ns - math.log2(int(Fs[s])) + nf - math.log2(qf)
+    return bits
+
+
+TINY_MODELS = []
+# three s symbols (exponents 1, 2 and the sign-flipped 1), ns = 4
+_ff = np.zeros((1, 128), np.uint32)
+_ff[0, 0], _ff[0, 1], _ff[0, 5] = 100, 27, 1   # sums to 128 = 2^7, a skewed route for e = 2
+TINY_MODELS.append(dict(fs={1: 9, 2: 6, 257: 1}, ns=4, route={2: 0}, ff=_ff, nf=7,
+                        alphabet=[(1 << 7) | 3, (2 << 7) | 1, (257 << 7) | 0]))
+TINY_MODELS.append(dict(fs={1: 1, 2: 1, 3: 2}, ns=2, route=None, ff=None, nf=7,
+                        alphabet=[(1 << 7) | 0, (2 << 7) | 127, (3 << 7) | 64]))
+_ff2 = np.zeros((2, 128), np.uint32)
+_ff2[0, :] = 8            # flat over 128 values, sums to 1024
+_ff2[1, 7], _ff2[1, 9] = 1023, 1
+TINY_MODELS.append(dict(fs={10: 4095, 300: 1}, ns=12, route={10: 0, 300 & 0xFF: 1}, ff=_ff2, nf=10,
+                        alphabet=[(10 << 7) | 7, (300 << 7) | 9, (300 << 7) | 7]))
+
+
+@pytest.mark.parametrize("mi", range(len(TINY_MODELS)))
+def test_bruteforce_tiny_alphabets(mi):
+    m = TINY_MODELS[mi]
+    Fs, route, Ff = _tables(m["fs"], m["ns"], m["route"], m["ff"])
+    alphabet = m["alphabet"]
+    n_seq = 0
+    for S in range(0, 9):
+        for seq in itertools.product(alphabet, repeat=S):
+            words = np.array(seq, np.uint16)
+            x0, wd, tags = oracle.lane_encode(Fs, m["ns"], route, Ff, m["nf"], words)
+            assert L <= x0 < (1 << 64)
+            assert np.all(np.diff(tags.astype(np.int64)) > 0)   # at most one word per step
+            st, out, fin = oracle.lane_decode(Fs, m["ns"], route, Ff, m["nf"], x0, wd, S)
+            assert st == 0 and fin == L
+            assert np.array_equal(out, words)
+            # code length: log2(x0) + 32*n_words = 32 + ideal bits, up to rANS rounding
+            ideal = _ideal_bits(words, Fs, m["ns"], route, Ff, m["nf"])
+            got = math.log2(x0) + 32 * wd.size
+            assert abs(got - 32 - ideal) <= 1e-6 + S * 2 ** -(32 - m["ns"] - m["nf"]) * 2, (seq, got, ideal)
+            n_seq += 1
+    assert n_seq == sum(3 ** k for k in range(9))
+
+
+def test_lane_decode_detects_wrong_state():
+    m = TINY_MODELS[0]
+    Fs, route, Ff = _tables(m["fs"], m["ns"], m["route"], m["ff"])
+    words = np.array(m["alphabet"] * 3, np.uint16)
+    x0, wd, _ = oracle.lane_encode(Fs, m["ns"], route, Ff, m["nf"], words)
+    # Decoding is a bijection on (state, words): a different start state either fails the
+    # end check or decodes to a different message; it can never reproduce the original.
+    for delta in (1, 2, 3, 1 << 20, 1 << 40):
+        st, out, fin = oracle.lane_decode(Fs, m["ns"], route, Ff, m["nf"], x0 ^ delta, wd, words.size)
+        assert st == oracle.E_CORRUPT or not np.array_equal(out, words)
+        assert (st == oracle.E_CORRUPT) == (fin != L or st == oracle.E_CORRUPT)
+
+
+# ---------------------------------------------------------------- quantiser
+def test_quantise_exact_proportions():
+    assert oracle.quantise([1, 1, 2], 2048).tolist() == [512, 512, 1024]
+    assert oracle.quantise([0, 5, 0, 15], 16).tolist() == [0, 4, 0, 12]
+
+
+def test_quantise_single_symbol_gets_all():
+    assert oracle.quantise([0, 0, 7, 0], 4096).tolist() == [0, 0, 4096, 0]
+
+
+def test_quantise_tie_goes_to_lowest():
+    # floor((2*1*4 + 3) / 6) = 1 each; one slot left, all ratios 1/3 tie -> index 0
+    assert oracle.quantise([1, 1, 1], 4).tolist() == [2, 1, 1]
+
+
+def test_quantise_rare_symbols_keep_one_slot():
+    c = [10 ** 9, 1, 1, 1]
+    q = oracle.quantise(c, 16)
+    assert q.tolist() == [13, 1, 1, 1]
+
+
+def test_quantise_too_many_symbols():
+    with pytest.raises(oracle.OracleError):
+        oracle.quantise([1, 1, 1], 2)
+
+
+def _cost(c, q, M):
+    return sum(ci * (math.log2(M) - math.log2(qi)) for ci, qi in zip(c, q) if ci)
+
+
+def _best_cost(c, M):
+    K = len(c)
+    best = float("inf")
+    present = [k for k in range(K) if c[k]]
+    for parts in itertools.product(range(1, M + 1), repeat=len(present)):
+        if sum(parts) != M:
+            continue
+        q = [0] * K
+        for k, v in zip(present, parts):
+            q[k] = v
+        best = min(best, _cost(c, q, M))
+    return best
+
+
+def test_quantise_near_optimal_small_cases():
+    rng = np.random.default_rng(5)
+    for _ in range(40):
+        K = int(rng.integers(2, 5))
+        c = [int(v) for v in rng.integers(0, 60, K)]
+        if sum(1 for v in c if v) < 1:
+            continue
+        M = 16
+        q = oracle.quantise(c, M).tolist()
+        assert sum(q) == M and all((qi >= 1) == (ci > 0) for qi, ci in zip(q, c))
+        # greedy first-order moves reach the exhaustive optimum within 0.5% of total cost
+        assert _cost(c, q, M) <= _best_cost(c, M) * 1.005 + 1e-9
+
+
+def test_quantise_invariants_random():
+    rng = np.random.default_rng(1)
+    for M in (128, 1024, 4096):
+        for _ in range(20):
+            c = rng.integers(0, 1000, 512) * (rng.random(512) < 0.2)
+            if c.sum() == 0:
+                continue
+            q = oracle.quantise(c, M)
+            assert int(q.sum()) == M
+            assert np.array_equal(q > 0, c > 0)
+
+
+# ---------------------------------------------------------------- route rule
+def test_route_threshold_boundary():
+    # one exponent, n = 128: chi2*n = 128*S - n^2. Counts (1+a, 1-a, 1, ...) give S = 128 + 2a^2.
+    # The threshold is 128*S - n^2 > 4096*n, i.e. 256*a^2 > 4096*128, i.e. a^2 > 2048.
+    def cef_with(counts):
+        cef = np.zeros((256, 128), np.uint64)
+        cef[40, : len(counts)] = counts
+        return cef
+    # a flat 128-count row: chi2 = 0
+    r, re = oracle.choose_routes(cef_with([1] * 128))
+    assert r[40] == 0xFF and re.size == 0
+    # all mass on one fraction: chi2 = 127*n > 4096 when n > 4096/127
+    r, re = oracle.choose_routes(cef_with([33]))
+    assert r[40] == 0 and re.tolist() == [40]
+    r, re = oracle.choose_routes(cef_with([32]))          # 127*32 = 4064 < 4096
+    assert r[40] == 0xFF
+
+
+def test_route_ranking_and_limit():
+    cef = np.zeros((256, 128), np.uint64)
+    for e, k in ((10, 1000), (20, 3000), (30, 2000)):
+        cef[e, 0] = k            # one-hot rows: chi2 = 127 * n
+    r, re = oracle.choose_routes(cef, max_routes=2)
+    assert re.tolist() == [20, 30]                       # the two largest chi2, in ascending e
+    assert r[20] == 0 and r[30] == 1 and r[10] == 0xFF
+    r, re = oracle.choose_routes(cef, max_routes=0)
+    assert re.size == 0
