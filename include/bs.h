@@ -1,0 +1,195 @@
+/*
+ * bs.h -- C ABI of libbs, the B200 (sm_100a) decoder for BF16RANS containers.
+ *
+ * The method is the one the "Qwen3.8-27B-BF16-NVLC-Lossless" model card describes in the
+ * paragraph after its accounting table:
+ *   - each BF16 word is split into sign:1 | exponent:8 | fraction:7;
+ *   - the joint sign+exponent symbol is rANS-coded with a per-tensor model;
+ *   - the decoded symbol selects the distribution of the 7-bit fraction;
+ *   - the fields are recombined bitwise, so the output is byte-identical to the original.
+ * The container layout (interleaved 32-lane chunks, tables, raw spans, checksum) is
+ * specified in FORMAT.md in this repository.
+ *
+ * Conventions
+ *  - Every function returns a bs_status, and nothing throws across the ABI.
+ *  - The caller owns every device buffer: the container copy, the workspace and the
+ *    outputs. The library allocates no device memory. Its only allocation is host memory
+ *    inside a plan, which bs_plan_destroy frees.
+ *  - "stream" is a cudaStream_t passed as void*, so that this header needs no CUDA
+ *    header. 0 means the legacy default stream.
+ *  - A plan is immutable after bs_plan returns. Decodes of the same plan may run
+ *    concurrently on different streams into disjoint outputs. They share the plan's
+ *    device error word, which records corruption found by any of them.
+ *  - Corruption found on the device is reported asynchronously through bs_check.
+ *    Kernels never trap, and every device loop is bounded by the chunk's weight count.
+ */
+#ifndef BS_H
+#define BS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BS_OK = 0,
+    BS_E_ARG = 1,          /* null pointer, bad index, misaligned buffer, bad size */
+    BS_E_FORMAT = 2,       /* the container fails validation (FORMAT.md section 5) */
+    BS_E_VERSION = 3,      /* unknown magic version */
+    BS_E_SIZE = 4,         /* an output or workspace buffer is the wrong size */
+    BS_E_CUDA = 5,         /* a CUDA runtime call failed (the CUDA error is kept, see bs_last_cuda_error) */
+    BS_E_CORRUPT = 6,      /* a chunk failed its end check, or a checksum differs */
+    BS_E_NOMEM = 7,        /* host allocation failed */
+    BS_E_UNSUPPORTED = 8   /* a device without sm_100 support */
+} bs_status;
+
+enum { BS_KIND_RANS = 0, BS_KIND_STORED = 1, BS_KIND_RAW = 2 };
+
+typedef struct bs_plan_t bs_plan_t; /* opaque host object */
+
+typedef struct {
+    uint64_t n_elems;     /* weights (RANS, STORED) or bytes (RAW) */
+    uint64_t out_bytes;   /* size of the decoded tensor: 2*n_elems, or n_elems for RAW */
+    uint64_t coded_bytes; /* RANS: model + chunk table + chunk payloads (padded); else out_bytes */
+    uint64_t n_chunks;    /* RANS only */
+    uint64_t checksum;    /* FORMAT.md section 7, of the original tensor */
+    uint64_t shape[8];
+    uint32_t kind;        /* BS_KIND_* */
+    uint32_t ndim;
+    uint32_t ns, nf, n_routes, log2_chunk; /* RANS model parameters */
+    const char* name;     /* not NUL-terminated; points into the plan */
+    uint32_t name_bytes;
+    uint32_t reserved;
+} bs_tensor_info;
+
+/* Bytes of device workspace that bs_plan needs for this container: the decode
+ * tables of every RANS tensor plus a 256-byte error block. h_container must hold the
+ * whole container. Returns 0 if the container does not validate. */
+size_t bs_plan_workspace_bytes(const void* h_container, size_t container_bytes);
+
+/*
+ * bs_plan: parse and validate a container, build its decode tables and upload them.
+ *
+ *   h_container      host copy of the whole container (read only during the call), or
+ *                    NULL: the plan then reads the header, directory, models and chunk
+ *                    tables from d_container with synchronous copies on stream
+ *   container_bytes  its length, equal to the header's total_bytes
+ *   d_container      the same bytes in device memory, 16-byte aligned; it must stay
+ *                    alive and unchanged for the life of the plan
+ *   d_workspace      device buffer of at least bs_plan_workspace_bytes, 256-byte aligned;
+ *                    the plan owns its contents until bs_plan_destroy
+ *   stream           the tables are uploaded with cudaMemcpyAsync on this stream
+ *   out              receives the plan
+ *
+ * Validation follows FORMAT.md section 5: a bad header gives BS_E_FORMAT or
+ * BS_E_VERSION, and a short workspace gives BS_E_SIZE.
+ */
+bs_status bs_plan(const void* h_container, size_t container_bytes, const void* d_container, void* d_workspace,
+                  size_t workspace_bytes, void* stream, bs_plan_t** out);
+
+/* As bs_plan_workspace_bytes, reading the metadata from device memory (synchronous
+ * copies on stream). Returns 0 if the container does not validate. */
+size_t bs_plan_workspace_bytes_device(const void* d_container, size_t container_bytes, void* stream);
+
+void bs_plan_destroy(bs_plan_t* plan);
+
+bs_status bs_tensor_count(const bs_plan_t* plan, int32_t* n);
+bs_status bs_tensor_info_get(const bs_plan_t* plan, int32_t idx, bs_tensor_info* out);
+
+/*
+ * bs_decode_tensor: decode tensor idx into d_out (device, 16-byte aligned, out_bytes =
+ * the tensor's out_bytes; otherwise BS_E_SIZE / BS_E_ARG). The work is enqueued on stream
+ * and the call returns at once.
+ *  - RANS: the interleaved rANS decode kernel, with one warp per 32-lane chunk.
+ *  - STORED and RAW: a vectorised copy kernel.
+ */
+bs_status bs_decode_tensor(const bs_plan_t* plan, int32_t idx, void* d_out, size_t out_bytes, void* stream);
+
+/*
+ * bs_decode_batch: decode n tensors in one pass. All the RANS tensors go in a single
+ * kernel launch per CTA shape (more than 448 of them are split across launches), and STORED/RAW
+ * tensors in one copy launch. idx[k] goes to d_out[k], of out_bytes[k] bytes.
+ *  - The outputs must not overlap.
+ *  - idx, d_out and out_bytes are host arrays, read during the call.
+ */
+bs_status bs_decode_batch(const bs_plan_t* plan, const int32_t* idx, void* const* d_out, const size_t* out_bytes,
+                          int32_t n, void* stream);
+
+/*
+ * bs_verify_tensor: compute the FORMAT.md section 7 checksum of a decoded tensor on the
+ * device and compare it with the stored one. The check is the analogue of the per-tensor
+ * md5 that the "Gemma 2 9B Instruct -- Lossless Compressed" card ("What lossless
+ * means") runs at decompression.
+ *  - d_scratch: 16 device bytes, 8-byte aligned, owned by the caller.
+ *  - Synchronises stream. Returns BS_E_CORRUPT on a mismatch.
+ *  - *got may be NULL. Otherwise it receives the computed checksum.
+ */
+bs_status bs_verify_tensor(const bs_plan_t* plan, int32_t idx, const void* d_out, size_t out_bytes,
+                           void* d_scratch, void* stream, uint64_t* got);
+
+/*
+ * bs_check: synchronise stream, then read and clear the plan's device error word.
+ * Returns BS_E_CORRUPT if any decode since the last check found a corrupt chunk. In
+ * that case *first_bad (if not NULL) is (tensor_index << 40) | chunk_index of the
+ * smallest such pair, and -1 otherwise.
+ */
+bs_status bs_check(const bs_plan_t* plan, void* stream, int64_t* first_bad);
+
+/* ------------------------------------------------------------------------------------
+ * Encoder on the device. It produces the canonical container of FORMAT.md section 4.6,
+ * byte-identical to any other encoder that follows FORMAT.md section 6. The card's
+ * compressor ("bigsmall compress" on the "Gemma 2 9B Instruct -- Lossless Compressed"
+ * card, "Want to compress your own model?") is the user-facing counterpart.
+ *
+ *   1. bs_encoder_create  describes the tensors (device pointers to the originals)
+ *   2. bs_encoder_run     histograms, models and a counting pass on the device; returns
+ *                         the exact container size
+ *   3. bs_encoder_emit    writes the container into caller device memory (and, if asked,
+ *                         a host copy)
+ *   4. bs_encoder_destroy
+ * The originals must stay unchanged on the device from run to emit. All device memory
+ * belongs to the caller: the originals, the scratch buffer (bs_encoder_scratch_bytes) and
+ * the container.
+ * ------------------------------------------------------------------------------------ */
+typedef struct bs_encoder_t bs_encoder_t;
+
+typedef struct {
+    uint32_t kind;        /* 0: BF16 words (the encoder picks RANS or STORED); 2: RAW bytes */
+    uint32_t ndim;
+    uint64_t shape[8];
+    uint64_t n_elems;     /* words (kind 0) or bytes (kind 2); must equal the shape product */
+    const void* d_data;   /* device; 16-byte aligned for kind 0 */
+    const char* name;     /* copied at create time */
+    uint32_t name_bytes;
+    uint32_t reserved;
+} bs_enc_item;
+
+typedef struct {
+    uint32_t log2_chunk;  /* 8..24, default 16 */
+    uint32_t ns;          /* 1..12, default 12 */
+    uint32_t nf;          /* 7..11, default 10 */
+    uint32_t max_routes;  /* 0..15, default 7 */
+    uint32_t force_rans;  /* 1: never fall back to STORED (tests only) */
+} bs_enc_params;
+
+bs_status bs_encoder_create(const bs_enc_item* items, int32_t n, const bs_enc_params* params, bs_encoder_t** out);
+/* Device scratch for bs_encoder_run / bs_encoder_emit (histograms, tables, chunk sizes). */
+bs_status bs_encoder_scratch_bytes(const bs_encoder_t* enc, size_t* bytes);
+/* Synchronises stream. *container_bytes receives the size bs_encoder_emit will write. */
+bs_status bs_encoder_run(bs_encoder_t* enc, void* d_scratch, size_t scratch_bytes, void* stream,
+                         size_t* container_bytes);
+/* d_container: container_bytes of device memory, 16-byte aligned. h_container: NULL, or
+ * a host buffer of container_bytes that receives a copy. Synchronises stream. */
+bs_status bs_encoder_emit(bs_encoder_t* enc, void* d_scratch, void* d_container, size_t container_bytes,
+                          void* h_container, void* stream);
+void bs_encoder_destroy(bs_encoder_t* enc);
+
+const char* bs_status_str(bs_status s);
+int bs_last_cuda_error(void); /* the cudaError_t behind the last BS_E_CUDA on this thread */
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BS_H */

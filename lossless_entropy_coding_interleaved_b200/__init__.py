@@ -1,0 +1,283 @@
+"""Python binding of libbs, the sm_100a decoder for BF16RANS containers.
+
+The binding only marshals arguments. Every step of the decode runs in libbs's CUDA
+kernels (csrc/bs_kernels.cu), and its host planner is csrc/bs_plan.cpp. PyTorch
+supplies device memory and streams. There is no CPU fallback: importing this module
+without a built libbs.so raises, and so does planning without a CUDA device.
+
+The method is the one in the paragraph after the accounting table of the
+"Qwen3.8-27B-BF16-NVLC-Lossless" model card:
+  - each BF16 word is split into sign, exponent and fraction;
+  - the sign+exponent symbol is rANS-decoded with a per-tensor model;
+  - that symbol selects the 7-bit fraction's distribution;
+  - the fields are recombined bitwise.
+The byte layout is FORMAT.md.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbs.so")
+
+OK, E_ARG, E_FORMAT, E_VERSION, E_SIZE, E_CUDA, E_CORRUPT, E_NOMEM, E_UNSUPPORTED = range(9)
+KIND_RANS, KIND_STORED, KIND_RAW = 0, 1, 2
+
+
+class BsError(RuntimeError):
+    def __init__(self, code: int, what: str, msg: str = "", first_bad: int = -1):
+        super().__init__(f"libbs {what}: {msg or code} (status {code})")
+        self.code = code
+        self.first_bad = first_bad
+
+
+class _Info(ctypes.Structure):
+    _fields_ = [("n_elems", ctypes.c_uint64), ("out_bytes", ctypes.c_uint64), ("coded_bytes", ctypes.c_uint64),
+                ("n_chunks", ctypes.c_uint64), ("checksum", ctypes.c_uint64), ("shape", ctypes.c_uint64 * 8),
+                ("kind", ctypes.c_uint32), ("ndim", ctypes.c_uint32), ("ns", ctypes.c_uint32),
+                ("nf", ctypes.c_uint32), ("n_routes", ctypes.c_uint32), ("log2_chunk", ctypes.c_uint32),
+                ("name", ctypes.c_void_p), ("name_bytes", ctypes.c_uint32), ("reserved", ctypes.c_uint32)]
+
+
+class _EncItem(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_uint32), ("ndim", ctypes.c_uint32), ("shape", ctypes.c_uint64 * 8),
+                ("n_elems", ctypes.c_uint64), ("d_data", ctypes.c_void_p), ("name", ctypes.c_char_p),
+                ("name_bytes", ctypes.c_uint32), ("reserved", ctypes.c_uint32)]
+
+
+class _EncParams(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_uint32) for k in ("log2_chunk", "ns", "nf", "max_routes", "force_rans")]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libbs.so is not built ({LIB_PATH}); run `python -m "
+                          f"lossless_entropy_coding_interleaved_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, i32, u64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64, ctypes.c_size_t
+    L.bs_plan_workspace_bytes.argtypes = [P, sz]
+    L.bs_plan_workspace_bytes.restype = sz
+    L.bs_plan.argtypes = [P, sz, P, P, sz, P, ctypes.POINTER(P)]
+    L.bs_plan_destroy.argtypes = [P]
+    L.bs_plan_destroy.restype = None
+    L.bs_tensor_count.argtypes = [P, ctypes.POINTER(i32)]
+    L.bs_tensor_info_get.argtypes = [P, i32, ctypes.POINTER(_Info)]
+    L.bs_decode_tensor.argtypes = [P, i32, P, sz, P]
+    L.bs_decode_batch.argtypes = [P, P, P, P, i32, P]
+    L.bs_verify_tensor.argtypes = [P, i32, P, sz, P, P, ctypes.POINTER(u64)]
+    L.bs_check.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
+    L.bs_status_str.argtypes = [ctypes.c_int]
+    L.bs_status_str.restype = ctypes.c_char_p
+    L.bs_last_cuda_error.argtypes = []
+    L.bs_plan_workspace_bytes_device.argtypes = [P, sz, P]
+    L.bs_plan_workspace_bytes_device.restype = sz
+    L.bs_encoder_create.argtypes = [ctypes.POINTER(_EncItem), i32, ctypes.POINTER(_EncParams), ctypes.POINTER(P)]
+    L.bs_encoder_scratch_bytes.argtypes = [P, ctypes.POINTER(sz)]
+    L.bs_encoder_run.argtypes = [P, P, sz, P, ctypes.POINTER(sz)]
+    L.bs_encoder_emit.argtypes = [P, P, P, sz, P, P]
+    L.bs_encoder_destroy.argtypes = [P]
+    L.bs_encoder_destroy.restype = None
+    for fn in ("bs_plan", "bs_tensor_count", "bs_tensor_info_get", "bs_decode_tensor", "bs_decode_batch",
+               "bs_verify_tensor", "bs_check", "bs_last_cuda_error", "bs_encoder_create", "bs_encoder_scratch_bytes",
+               "bs_encoder_run", "bs_encoder_emit"):
+        getattr(L, fn).restype = ctypes.c_int
+    return L
+
+
+lib = _load()
+
+#: every symbol include/bs.h declares
+EXPORTS = ("bs_plan_workspace_bytes", "bs_plan_workspace_bytes_device", "bs_plan", "bs_plan_destroy",
+           "bs_tensor_count", "bs_tensor_info_get", "bs_decode_tensor", "bs_decode_batch", "bs_verify_tensor",
+           "bs_check", "bs_encoder_create", "bs_encoder_scratch_bytes", "bs_encoder_run", "bs_encoder_emit",
+           "bs_encoder_destroy", "bs_status_str", "bs_last_cuda_error")
+
+
+def _check(st: int, what: str):
+    if st != OK:
+        msg = lib.bs_status_str(st).decode()
+        if st == E_CUDA:
+            msg += f" (cudaError {lib.bs_last_cuda_error()})"
+        raise BsError(st, what, msg)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _host_bytes(container) -> np.ndarray:
+    if isinstance(container, np.ndarray):
+        a = np.ascontiguousarray(container.reshape(-1).view(np.uint8))
+    else:
+        a = np.frombuffer(container, dtype=np.uint8)
+    return a
+
+
+def workspace_bytes(container) -> int:
+    h = _host_bytes(container)
+    n = lib.bs_plan_workspace_bytes(h.ctypes.data, h.size)
+    if n == 0:
+        raise BsError(E_FORMAT, "workspace_bytes", "container fails validation")
+    return n
+
+
+def encode(tensors, log2_chunk: int = 16, ns: int = 12, nf: int = 10, max_routes: int = 7,
+           force_rans: bool = False, host_copy: bool = False, stream=None):
+    """Encode device tensors into a container on the device (bs_encoder_*).
+
+    tensors: sequence of (name, tensor) pairs; int16/bfloat16 CUDA tensors are BF16
+    words and uint8 CUDA tensors are opaque byte spans. Returns (d_container, h_container),
+    a uint8 CUDA tensor and, when host_copy, a uint8 numpy copy (else None).
+    """
+    keep = []
+    items = (_EncItem * max(1, len(tensors)))()
+    dev = None
+    for k, (name, t) in enumerate(tensors):
+        assert t.is_cuda and t.is_contiguous()
+        dev = t.device
+        if t.dtype == torch.bfloat16:
+            t = t.view(torch.int16)
+        assert t.dtype in (torch.int16, torch.uint8), t.dtype
+        nb = name.encode()
+        keep += [t, nb]
+        it = items[k]
+        it.kind = 0 if t.dtype == torch.int16 else 2
+        it.ndim = t.dim()
+        for d, v in enumerate(t.shape):
+            it.shape[d] = v
+        it.n_elems = t.numel()
+        it.d_data = t.data_ptr() if t.numel() else None
+        it.name = nb
+        it.name_bytes = len(nb)
+    if dev is None:
+        dev = torch.device("cuda")
+    prm = _EncParams(log2_chunk, ns, nf, max_routes, 1 if force_rans else 0)
+    enc = ctypes.c_void_p()
+    _check(lib.bs_encoder_create(items, len(tensors), ctypes.byref(prm), ctypes.byref(enc)), "encoder_create")
+    try:
+        sc = ctypes.c_size_t()
+        _check(lib.bs_encoder_scratch_bytes(enc, ctypes.byref(sc)), "encoder_scratch_bytes")
+        scratch = torch.empty(max(sc.value, 256), dtype=torch.uint8, device=dev)
+        total = ctypes.c_size_t()
+        st = _stream(stream)
+        with torch.cuda.device(dev):
+            _check(lib.bs_encoder_run(enc, scratch.data_ptr(), scratch.numel(), st, ctypes.byref(total)),
+                   "encoder_run")
+            d_container = torch.empty(total.value, dtype=torch.uint8, device=dev)
+            h = np.empty(total.value, dtype=np.uint8) if host_copy else None
+            _check(lib.bs_encoder_emit(enc, scratch.data_ptr(), d_container.data_ptr(), total.value,
+                                       h.ctypes.data if host_copy else None, st), "encoder_emit")
+    finally:
+        lib.bs_encoder_destroy(enc)
+    return d_container, h
+
+
+class Plan:
+    """A validated container resident in device memory, with its decode tables.
+
+    ``container`` holds the container's bytes on the host (bytes or a uint8 numpy
+    array), or is None when ``d_container`` is given: the plan then reads the metadata
+    from the device. ``d_container`` is an optional uint8 CUDA tensor that already holds
+    the container; without it, the host bytes are copied to ``device``.
+    """
+
+    def __init__(self, container=None, device="cuda", d_container: torch.Tensor | None = None, stream=None):
+        if not torch.cuda.is_available():
+            raise BsError(E_UNSUPPORTED, "plan", "no CUDA device")
+        if container is None and d_container is None:
+            raise BsError(E_ARG, "plan", "no container")
+        self.device = torch.device(device) if d_container is None else d_container.device
+        h = None if container is None else _host_bytes(container)
+        if d_container is None:
+            d_container = torch.from_numpy(h.copy()).to(self.device)
+        assert d_container.dtype == torch.uint8 and d_container.is_cuda
+        assert h is None or d_container.numel() == h.size
+        self.d_container = d_container
+        self.container_bytes = d_container.numel()
+        st = _stream(stream)
+        with torch.cuda.device(self.device):
+            if h is not None:
+                ws = workspace_bytes(h)
+            else:
+                ws = lib.bs_plan_workspace_bytes_device(d_container.data_ptr(), d_container.numel(), st)
+                if ws == 0:
+                    raise BsError(E_FORMAT, "workspace_bytes", "container fails validation")
+            self.workspace = torch.empty(ws, dtype=torch.uint8, device=self.device)
+            self._scratch = torch.zeros(2, dtype=torch.int64, device=self.device)
+            ptr = ctypes.c_void_p()
+            _check(lib.bs_plan(None if h is None else h.ctypes.data, self.container_bytes, d_container.data_ptr(),
+                               self.workspace.data_ptr(), ws, st, ctypes.byref(ptr)), "plan")
+        self._p = ptr
+        n = ctypes.c_int32()
+        _check(lib.bs_tensor_count(self._p, ctypes.byref(n)), "tensor_count")
+        self.n_tensors = n.value
+        self._info = [self._get_info(k) for k in range(self.n_tensors)]
+        self.names = [i["name"] for i in self._info]
+
+    def __del__(self):
+        p = getattr(self, "_p", None)
+        if p and lib is not None:
+            lib.bs_plan_destroy(p)
+            self._p = None
+
+    def _get_info(self, idx: int) -> dict:
+        ti = _Info()
+        _check(lib.bs_tensor_info_get(self._p, idx, ctypes.byref(ti)), "tensor_info")
+        d = {k: getattr(ti, k) for k, _ in _Info._fields_ if k not in ("shape", "name", "name_bytes", "reserved")}
+        d["shape"] = tuple(ti.shape[i] for i in range(ti.ndim))
+        d["name"] = ctypes.string_at(ti.name, ti.name_bytes).decode() if ti.name_bytes else ""
+        return d
+
+    def info(self, idx: int) -> dict:
+        return dict(self._info[idx])
+
+    def empty_output(self, idx: int) -> torch.Tensor:
+        """A device buffer of the right size and dtype for tensor idx: int16 words viewable
+        as bfloat16, or uint8 for RAW."""
+        i = self._info[idx]
+        if i["kind"] == KIND_RAW:
+            return torch.empty(i["n_elems"], dtype=torch.uint8, device=self.device)
+        return torch.empty(i["shape"] if i["shape"] else (), dtype=torch.int16, device=self.device)
+
+    def decode(self, idx: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        if out is None:
+            out = self.empty_output(idx)
+        _check(lib.bs_decode_tensor(self._p, idx, out.data_ptr(), out.numel() * out.element_size(),
+                                    _stream(stream)), "decode_tensor")
+        return out
+
+    def decode_batch(self, idxs, outs=None, stream=None):
+        idxs = list(idxs)
+        if outs is None:
+            outs = [self.empty_output(k) for k in idxs]
+        n = len(idxs)
+        ia = (ctypes.c_int32 * max(n, 1))(*idxs)
+        pa = (ctypes.c_void_p * max(n, 1))(*[o.data_ptr() for o in outs])
+        ba = (ctypes.c_size_t * max(n, 1))(*[o.numel() * o.element_size() for o in outs])
+        _check(lib.bs_decode_batch(self._p, ia, pa, ba, n, _stream(stream)), "decode_batch")
+        return outs
+
+    def verify(self, idx: int, out: torch.Tensor, stream=None) -> int:
+        """Checksum of a decoded tensor computed on the device; raises BsError(E_CORRUPT)
+        if it differs from the stored one. Synchronises the stream."""
+        got = ctypes.c_uint64()
+        st = lib.bs_verify_tensor(self._p, idx, out.data_ptr(), out.numel() * out.element_size(),
+                                  self._scratch.data_ptr(), _stream(stream), ctypes.byref(got))
+        _check(st, "verify_tensor")
+        return got.value
+
+    def check(self, stream=None) -> int:
+        """Synchronise and read the device error word: -1 if clean, else raises BsError with
+        first_bad = (tensor << 40) | chunk."""
+        fb = ctypes.c_int64()
+        st = lib.bs_check(self._p, _stream(stream), ctypes.byref(fb))
+        if st == E_CORRUPT:
+            raise BsError(st, "check", "corrupt chunk", first_bad=fb.value)
+        _check(st, "check")
+        return fb.value

@@ -1,0 +1,506 @@
+// bs_plan.cpp -- host side of libbs: container parsing and validation, decode-table
+// construction, and the C ABI of include/bs.h. The GPU work lives in bs_kernels.cu.
+//
+// The container is the one FORMAT.md specifies. This parser is written against that
+// document. It shares no code with the oracle (oracle/bsoracle.c).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+#include <memory>
+#include <new>
+#include <vector>
+
+#include "bs_internal.h"
+
+using namespace bs;
+
+struct bs_plan_t {
+    std::vector<Tensor> tensors;
+    const uint8_t* d_container = nullptr;
+    uint64_t container_bytes = 0;
+    uint8_t* d_ws = nullptr;
+    uint64_t ws_bytes = 0;
+    int device = 0;
+    std::vector<uint8_t> host_tables; // staging copy of the workspace tables (kept until destroy)
+};
+
+namespace {
+thread_local int g_last_cuda = 0;
+} // namespace
+
+void bs::record_cuda_error(int e) { g_last_cuda = e; }
+
+namespace {
+
+bs_status cuda_fail(cudaError_t e) {
+    g_last_cuda = static_cast<int>(e);
+    return BS_E_CUDA;
+}
+
+uint64_t get_u64(const uint8_t* p) {
+    uint64_t v;
+    std::memcpy(&v, p, 8);
+    return v;
+}
+uint32_t get_u32(const uint8_t* p) {
+    uint32_t v;
+    std::memcpy(&v, p, 4);
+    return v;
+}
+uint16_t get_u16(const uint8_t* p) {
+    uint16_t v;
+    std::memcpy(&v, p, 2);
+    return v;
+}
+bool inside(uint64_t off, uint64_t bytes, uint64_t len) { return off <= len && bytes <= len - off; }
+uint64_t up16(uint64_t v) { return (v + 15) & ~uint64_t(15); }
+uint64_t up256(uint64_t v) { return (v + 255) & ~uint64_t(255); }
+
+// Reads container bytes from a host copy or, without one, from device memory.
+struct Reader {
+    const uint8_t* host = nullptr;
+    const uint8_t* dev = nullptr;
+    cudaStream_t stream = nullptr;
+    uint64_t len = 0;
+    bool cuda_error = false;
+    bool read(uint64_t off, uint64_t n, void* dst) {
+        if (!inside(off, n, len)) return false;
+        if (n == 0) return true;
+        if (host) {
+            std::memcpy(dst, host + off, n);
+            return true;
+        }
+        cudaError_t e = cudaMemcpyAsync(dst, dev + off, n, cudaMemcpyDeviceToHost, stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+        if (e != cudaSuccess) {
+            g_last_cuda = static_cast<int>(e);
+            cuda_error = true;
+            return false;
+        }
+        return true;
+    }
+};
+
+// FORMAT.md sections 4-5. Fills `out` with every tensor, or returns the first error.
+bs_status parse(Reader& rd, std::vector<Tensor>& out) {
+    const uint64_t len = rd.len;
+    uint8_t hdr[kHeaderBytes];
+    auto fail = [&](bs_status st) { return rd.cuda_error ? BS_E_CUDA : st; };
+    if (len < kHeaderBytes || !rd.read(0, kHeaderBytes, hdr)) return fail(BS_E_FORMAT);
+    const uint8_t* b = hdr;
+    if (std::memcmp(b, "BF16RANS", 8) != 0) return BS_E_FORMAT;
+    if (get_u32(b + 8) != 1) return BS_E_VERSION;
+    if (get_u32(b + 12) != kHeaderBytes || get_u32(b + 20) != kDirEntryBytes || get_u64(b + 56) != 0)
+        return BS_E_FORMAT;
+    if (get_u64(b + 48) != len) return BS_E_SIZE;
+    const uint32_t nt = get_u32(b + 16);
+    const uint64_t dir = get_u64(b + 24), names = get_u64(b + 32), names_bytes = get_u64(b + 40);
+    if (dir % 16 || names % 16) return BS_E_FORMAT;
+    if (!inside(dir, uint64_t(kDirEntryBytes) * nt, len) || !inside(names, names_bytes, len)) return BS_E_FORMAT;
+    std::vector<uint8_t> dbuf, nbuf, tbuf;
+    try {
+        dbuf.resize(uint64_t(kDirEntryBytes) * nt);
+        nbuf.resize(names_bytes);
+    } catch (...) {
+        return BS_E_NOMEM;
+    }
+    if (!rd.read(dir, dbuf.size(), dbuf.data()) || !rd.read(names, names_bytes, nbuf.data())) return fail(BS_E_FORMAT);
+    out.clear();
+    out.reserve(nt);
+    for (uint32_t k = 0; k < nt; ++k) {
+        const uint8_t* d = dbuf.data() + uint64_t(kDirEntryBytes) * k;
+        Tensor t;
+        t.kind = d[0];
+        t.ndim = d[1];
+        t.log2_chunk = d[2];
+        t.lanes = d[3];
+        t.ns = d[4];
+        t.nf = d[5];
+        t.n_routes = d[6];
+        if (d[7] != 0 || get_u64(d + 72) != 0) return BS_E_FORMAT;
+        const uint32_t name_off = get_u32(d + 8), name_len = get_u32(d + 12);
+        t.n_elems = get_u64(d + 16);
+        t.n_chunks = get_u64(d + 24);
+        t.model_offset = get_u64(d + 32);
+        t.model_bytes = get_u64(d + 40);
+        t.data_offset = get_u64(d + 48);
+        t.data_bytes = get_u64(d + 56);
+        t.checksum = get_u64(d + 64);
+        for (int i = 0; i < 8; ++i) t.shape[i] = get_u64(d + 80 + 8 * i);
+        if (t.kind > BS_KIND_RAW || t.ndim > 8) return BS_E_FORMAT;
+        if (uint64_t(name_off) + name_len > names_bytes) return BS_E_FORMAT;
+        t.name.assign(reinterpret_cast<const char*>(nbuf.data() + name_off), name_len);
+        unsigned __int128 prod = 1;
+        for (uint32_t i = 0; i < t.ndim; ++i) {
+            prod *= t.shape[i];
+            if (prod > (static_cast<unsigned __int128>(1) << 64)) return BS_E_FORMAT;
+        }
+        for (uint32_t i = t.ndim; i < 8; ++i)
+            if (t.shape[i] != 0) return BS_E_FORMAT;
+        if (prod != t.n_elems) return BS_E_FORMAT;
+        if (t.data_offset % 16 || !inside(t.data_offset, t.data_bytes, len)) return BS_E_FORMAT;
+        if (t.kind != BS_KIND_RANS) {
+            if (t.kind == BS_KIND_STORED && t.n_elems > (1ull << 62)) return BS_E_FORMAT;
+            const uint64_t want = t.kind == BS_KIND_STORED ? 2 * t.n_elems : t.n_elems;
+            if (t.data_bytes != want) return BS_E_FORMAT;
+            t.coded_bytes = want;
+            out.push_back(std::move(t));
+            continue;
+        }
+        // RANS
+        if (t.lanes != kLanes || t.log2_chunk < 8 || t.log2_chunk > 24) return BS_E_FORMAT;
+        if (t.ns < 1 || t.ns > kMaxNs || t.nf < 7 || t.nf > kMaxNf || t.n_routes > kMaxRoutes) return BS_E_FORMAT;
+        if (t.n_elems == 0 || t.n_elems > (1ull << 40)) return BS_E_FORMAT;
+        const uint64_t C = 1ull << t.log2_chunk;
+        if (t.n_chunks != (t.n_elems + C - 1) / C || t.data_bytes != 16 * t.n_chunks) return BS_E_FORMAT;
+        if (t.model_offset % 16 || !inside(t.model_offset, t.model_bytes, len) || t.model_bytes < 264 ||
+            t.model_bytes > 260 + 4 * 512 + 256 * kMaxRoutes)
+            return BS_E_FORMAT;
+        t.model.resize(t.model_bytes);
+        if (!rd.read(t.model_offset, t.model_bytes, t.model.data())) return fail(BS_E_FORMAT);
+        const uint8_t* m = t.model.data();
+        const uint32_t n_present = get_u16(m);
+        if (n_present < 1 || n_present > 512) return BS_E_FORMAT;
+        if (t.model_bytes != 260 + 4ull * n_present + 256ull * t.n_routes) return BS_E_FORMAT;
+        uint64_t sum = 0;
+        int prev = -1;
+        for (uint32_t i = 0; i < n_present; ++i) {
+            const int s = get_u16(m + 4 + 4 * i);
+            const uint32_t q = get_u16(m + 6 + 4 * i);
+            if (s <= prev || s > 511 || q == 0) return BS_E_FORMAT;
+            prev = s;
+            sum += q;
+        }
+        if (sum != (1ull << t.ns)) return BS_E_FORMAT;
+        const uint8_t* route = m + 4 + 4 * n_present;
+        for (int e = 0; e < 256; ++e)
+            if (route[e] != 0xFF && route[e] >= t.n_routes) return BS_E_FORMAT;
+        for (uint32_t r = 0; r < t.n_routes; ++r) {
+            sum = 0;
+            for (int f = 0; f < 128; ++f) sum += get_u16(route + 256 + 256 * r + 2 * f);
+            if (sum != (1ull << t.nf)) return BS_E_FORMAT;
+        }
+        try {
+            tbuf.resize(t.data_bytes);
+        } catch (...) {
+            return BS_E_NOMEM;
+        }
+        if (!rd.read(t.data_offset, t.data_bytes, tbuf.data())) return fail(BS_E_FORMAT);
+        t.coded_bytes = t.model_bytes + t.data_bytes;
+        for (uint64_t c = 0; c < t.n_chunks; ++c) {
+            const uint8_t* e = tbuf.data() + 16 * c;
+            const uint64_t off = get_u64(e);
+            const uint32_t nw = get_u32(e + 8);
+            if (off % 16 || !inside(off, 256 + 4ull * nw, len)) return BS_E_FORMAT;
+            t.coded_bytes += up16(256 + 4ull * nw);
+        }
+        t.table_bytes = table_bytes_for(t.ns, t.nf, t.n_routes);
+        out.push_back(std::move(t));
+    }
+    return BS_OK;
+}
+
+// Expand one tensor's model into the decode tables (layout in bs_internal.h).
+void build_tables(const Tensor& t, uint8_t* dst) {
+    const uint8_t* m = t.model.data();
+    const uint32_t n_present = get_u16(m);
+    const uint8_t* route = m + 4 + 4 * n_present;
+    const uint32_t Mf = 1u << t.nf;
+    auto fbase = [&](uint32_t s) -> uint32_t {
+        const uint8_t r = route[s & 0xFF];
+        return (r == 0xFF ? t.n_routes : r) * Mf;
+    };
+    uint32_t* st = reinterpret_cast<uint32_t*>(dst);
+    uint32_t cum = 0;
+    for (uint32_t i = 0; i < n_present; ++i) {
+        const uint32_t s = get_u16(m + 4 + 4 * i), q = get_u16(m + 6 + 4 * i);
+        for (uint32_t k = 0; k < q; ++k) {
+            st[2 * (cum + k)] = q | (k << 16);
+            st[2 * (cum + k) + 1] = (s << 7) | (fbase(s) << 16);
+        }
+        cum += q;
+    }
+    uint32_t* ft = reinterpret_cast<uint32_t*>(dst + (8u << t.ns));
+    for (uint32_t r = 0; r <= t.n_routes; ++r) {
+        uint32_t* row = ft + r * Mf;
+        cum = 0;
+        for (uint32_t f = 0; f < 128; ++f) {
+            const uint32_t q = (r == t.n_routes) ? Mf / 128 : get_u16(route + 256 + 256 * r + 2 * f);
+            for (uint32_t k = 0; k < q; ++k) row[cum + k] = f | (q << 7) | (k << 19);
+            cum += q;
+        }
+    }
+}
+
+uint64_t workspace_for(const std::vector<Tensor>& ts) {
+    uint64_t ws = kErrBlockBytes;
+    for (const Tensor& t : ts)
+        if (t.kind == BS_KIND_RANS) ws += up256(t.table_bytes);
+    return ws;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+} // namespace
+
+extern "C" {
+
+size_t bs_plan_workspace_bytes(const void* h_container, size_t container_bytes) {
+    if (!h_container) return 0;
+    std::vector<Tensor> ts;
+    Reader rd;
+    rd.host = static_cast<const uint8_t*>(h_container);
+    rd.len = container_bytes;
+    if (parse(rd, ts) != BS_OK) return 0;
+    return workspace_for(ts);
+}
+
+size_t bs_plan_workspace_bytes_device(const void* d_container, size_t container_bytes, void* stream) {
+    if (!d_container) return 0;
+    std::vector<Tensor> ts;
+    Reader rd;
+    rd.dev = static_cast<const uint8_t*>(d_container);
+    rd.stream = static_cast<cudaStream_t>(stream);
+    rd.len = container_bytes;
+    if (parse(rd, ts) != BS_OK) return 0;
+    return workspace_for(ts);
+}
+
+bs_status bs_plan(const void* h_container, size_t container_bytes, const void* d_container, void* d_workspace,
+                  size_t workspace_bytes, void* stream, bs_plan_t** out) {
+    if (!out || !d_container || !d_workspace) return BS_E_ARG;
+    *out = nullptr;
+    if (!aligned(d_container, 16) || !aligned(d_workspace, 256)) return BS_E_ARG;
+    int dev = 0, major = 0, minor = 0;
+    cudaError_t ce = cudaGetDevice(&dev);
+    if (ce != cudaSuccess) return cuda_fail(ce);
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0) return BS_E_UNSUPPORTED;
+
+    std::unique_ptr<bs_plan_t> p(new (std::nothrow) bs_plan_t);
+    if (!p) return BS_E_NOMEM;
+    Reader rd;
+    rd.host = static_cast<const uint8_t*>(h_container);
+    rd.dev = static_cast<const uint8_t*>(d_container);
+    rd.stream = static_cast<cudaStream_t>(stream);
+    rd.len = container_bytes;
+    bs_status st = parse(rd, p->tensors);
+    if (st != BS_OK) return st;
+    const uint64_t ws = workspace_for(p->tensors);
+    if (workspace_bytes < ws) return BS_E_SIZE;
+    const int smem_cap = max_dynamic_smem();
+    try {
+        p->host_tables.assign(ws, 0);
+    } catch (...) {
+        return BS_E_NOMEM;
+    }
+    uint64_t pos = kErrBlockBytes;
+    for (Tensor& t : p->tensors) {
+        if (t.kind != BS_KIND_RANS) continue;
+        if (static_cast<int>(t.table_bytes + ring_bytes_per_cta(warps_for_tables(t.table_bytes))) > smem_cap)
+            return BS_E_UNSUPPORTED;
+        t.ws_offset = pos;
+        build_tables(t, p->host_tables.data() + pos);
+        pos += up256(t.table_bytes);
+    }
+    // error block: flags = 0, first_bad = all ones
+    std::memset(p->host_tables.data() + 8, 0xFF, 8);
+    ce = cudaMemcpyAsync(d_workspace, p->host_tables.data(), ws, cudaMemcpyHostToDevice,
+                         static_cast<cudaStream_t>(stream));
+    if (ce != cudaSuccess) return cuda_fail(ce);
+    p->d_container = static_cast<const uint8_t*>(d_container);
+    p->container_bytes = container_bytes;
+    p->d_ws = static_cast<uint8_t*>(d_workspace);
+    p->ws_bytes = ws;
+    p->device = dev;
+    *out = p.release();
+    return BS_OK;
+}
+
+void bs_plan_destroy(bs_plan_t* plan) { delete plan; }
+
+bs_status bs_tensor_count(const bs_plan_t* plan, int32_t* n) {
+    if (!plan || !n) return BS_E_ARG;
+    *n = static_cast<int32_t>(plan->tensors.size());
+    return BS_OK;
+}
+
+bs_status bs_tensor_info_get(const bs_plan_t* plan, int32_t idx, bs_tensor_info* o) {
+    if (!plan || !o || idx < 0 || idx >= static_cast<int32_t>(plan->tensors.size())) return BS_E_ARG;
+    const Tensor& t = plan->tensors[idx];
+    std::memset(o, 0, sizeof(*o));
+    o->n_elems = t.n_elems;
+    o->out_bytes = t.kind == BS_KIND_RAW ? t.n_elems : 2 * t.n_elems;
+    o->coded_bytes = t.coded_bytes;
+    o->n_chunks = t.n_chunks;
+    o->checksum = t.checksum;
+    for (int i = 0; i < 8; ++i) o->shape[i] = t.shape[i];
+    o->kind = t.kind;
+    o->ndim = t.ndim;
+    o->ns = t.ns;
+    o->nf = t.nf;
+    o->n_routes = t.n_routes;
+    o->log2_chunk = t.log2_chunk;
+    o->name = t.name.data();
+    o->name_bytes = static_cast<uint32_t>(t.name.size());
+    return BS_OK;
+}
+
+bs_status bs_decode_batch(const bs_plan_t* plan, const int32_t* idx, void* const* d_out, const size_t* out_bytes,
+                          int32_t n, void* stream) {
+    if (!plan || n < 0 || (n > 0 && (!idx || !d_out || !out_bytes))) return BS_E_ARG;
+    const int32_t nt = static_cast<int32_t>(plan->tensors.size());
+    for (int32_t k = 0; k < n; ++k) {
+        if (idx[k] < 0 || idx[k] >= nt) return BS_E_ARG;
+        const Tensor& t = plan->tensors[idx[k]];
+        const uint64_t want = t.kind == BS_KIND_RAW ? t.n_elems : 2 * t.n_elems;
+        if (out_bytes[k] != want) return BS_E_SIZE;
+        if (want && !d_out[k]) return BS_E_ARG;
+        if (t.kind == BS_KIND_RANS && !aligned(d_out[k], 16)) return BS_E_ARG;
+    }
+    // One parameter block per CTA shape (16 or 8 warps) and one for verbatim copies.
+    // (16 or 8 warps) x (default precisions ns=12/nf=10, or any)
+    struct Pending {
+        std::unique_ptr<DecodeParams> p;
+        int warps;
+        bool default_precision;
+        uint32_t smem = 0;
+    };
+    Pending dec[4] = {{nullptr, 16, true}, {nullptr, 16, false}, {nullptr, 8, true}, {nullptr, 8, false}};
+    for (Pending& d : dec) {
+        d.p.reset(new (std::nothrow) DecodeParams);
+        if (!d.p) return BS_E_NOMEM;
+    }
+    std::unique_ptr<CopyParams> cp(new (std::nothrow) CopyParams);
+    if (!cp) return BS_E_NOMEM;
+    for (Pending& d : dec) {
+        d.p->n_items = 0;
+        d.p->total_ctas = 0;
+        d.p->err = reinterpret_cast<unsigned long long*>(plan->d_ws);
+    }
+    cp->n_items = 0;
+    cp->total_blocks = 0;
+    auto flush_decode = [&](Pending& d) -> bs_status {
+        if (d.p->n_items == 0) return BS_OK;
+        const int e = launch_decode(*d.p, d.warps, d.default_precision, d.smem, stream);
+        d.p->n_items = 0;
+        d.p->total_ctas = 0;
+        d.smem = 0;
+        return e ? cuda_fail(static_cast<cudaError_t>(e)) : BS_OK;
+    };
+    auto flush_copy = [&]() -> bs_status {
+        if (cp->n_items == 0) return BS_OK;
+        const int e = launch_copy(*cp, stream);
+        cp->n_items = 0;
+        cp->total_blocks = 0;
+        return e ? cuda_fail(static_cast<cudaError_t>(e)) : BS_OK;
+    };
+    for (int32_t k = 0; k < n; ++k) {
+        const Tensor& t = plan->tensors[idx[k]];
+        if (t.kind == BS_KIND_RANS) {
+            const int warps = warps_for_tables(t.table_bytes);
+            const bool dflt = t.ns == 12 && t.nf == 10;
+            Pending& d = dec[(warps == 16 ? 0 : 2) + (dflt ? 0 : 1)];
+            const uint64_t per_cta = uint64_t(warps) * kChains;
+            const uint64_t ctas = (t.n_chunks + per_cta - 1) / per_cta;
+            if (d.p->n_items == kMaxDecodeItems || d.p->total_ctas + ctas > 0x7FFFFFFFull) {
+                bs_status s = flush_decode(d);
+                if (s) return s;
+            }
+            DecodeItem& it = d.p->item[d.p->n_items++];
+            std::memset(&it, 0, sizeof(it));
+            it.chunk_table = plan->d_container + t.data_offset;
+            it.container = plan->d_container;
+            it.tables = reinterpret_cast<const uint4*>(plan->d_ws + t.ws_offset);
+            it.out = static_cast<uint16_t*>(d_out[k]);
+            it.n_elems = t.n_elems;
+            it.cta_begin = d.p->total_ctas;
+            it.tensor_index = static_cast<uint32_t>(idx[k]);
+            it.table_bytes = t.table_bytes;
+            it.log2_chunk = static_cast<uint8_t>(t.log2_chunk);
+            it.ns = static_cast<uint8_t>(t.ns);
+            it.nf = static_cast<uint8_t>(t.nf);
+            d.p->total_ctas += static_cast<uint32_t>(ctas);
+            d.smem = std::max<uint32_t>(d.smem, t.table_bytes + ring_bytes_per_cta(warps));
+        } else if (t.n_elems) {
+            const uint64_t bytes = t.kind == BS_KIND_RAW ? t.n_elems : 2 * t.n_elems;
+            const uint64_t blks = (bytes + kCopyBlockBytes - 1) / kCopyBlockBytes;
+            if (cp->n_items == kMaxCopyItems || cp->total_blocks + blks > 0x7FFFFFFFull) {
+                bs_status s = flush_copy();
+                if (s) return s;
+            }
+            CopyItem& it = cp->item[cp->n_items++];
+            it.src = plan->d_container + t.data_offset;
+            it.dst = static_cast<uint8_t*>(d_out[k]);
+            it.bytes = bytes;
+            it.blk_begin = cp->total_blocks;
+            cp->total_blocks += blks;
+        }
+    }
+    for (Pending& d : dec) {
+        bs_status s = flush_decode(d);
+        if (s) return s;
+    }
+    return flush_copy();
+}
+
+bs_status bs_decode_tensor(const bs_plan_t* plan, int32_t idx, void* d_out, size_t out_bytes, void* stream) {
+    return bs_decode_batch(plan, &idx, &d_out, &out_bytes, 1, stream);
+}
+
+bs_status bs_verify_tensor(const bs_plan_t* plan, int32_t idx, const void* d_out, size_t out_bytes, void* d_scratch,
+                           void* stream, uint64_t* got) {
+    if (!plan || idx < 0 || idx >= static_cast<int32_t>(plan->tensors.size()) || !d_scratch ||
+        !aligned(d_scratch, 8))
+        return BS_E_ARG;
+    const Tensor& t = plan->tensors[idx];
+    const uint64_t want = t.kind == BS_KIND_RAW ? t.n_elems : 2 * t.n_elems;
+    if (out_bytes != want) return BS_E_SIZE;
+    if (want && !d_out) return BS_E_ARG;
+    auto* sum = static_cast<unsigned long long*>(d_scratch);
+    int e = launch_checksum(d_out, t.n_elems, t.kind == BS_KIND_RAW, sum, stream);
+    if (e) return cuda_fail(static_cast<cudaError_t>(e));
+    unsigned long long h = 0;
+    cudaError_t ce = cudaMemcpyAsync(&h, sum, 8, cudaMemcpyDeviceToHost, static_cast<cudaStream_t>(stream));
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (ce != cudaSuccess) return cuda_fail(ce);
+    if (got) *got = h;
+    return h == t.checksum ? BS_OK : BS_E_CORRUPT;
+}
+
+bs_status bs_check(const bs_plan_t* plan, void* stream, int64_t* first_bad) {
+    if (!plan) return BS_E_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned long long h[2] = {0, 0};
+    cudaError_t ce = cudaMemcpyAsync(h, plan->d_ws, 16, cudaMemcpyDeviceToHost, s);
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(s);
+    if (ce != cudaSuccess) return cuda_fail(ce);
+    if (first_bad) *first_bad = h[0] ? static_cast<int64_t>(h[1]) : -1;
+    if (!h[0]) return BS_OK;
+    static const unsigned long long reset[2] = {0, ~0ull};
+    ce = cudaMemcpyAsync(plan->d_ws, reset, 16, cudaMemcpyHostToDevice, s);
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(s);
+    if (ce != cudaSuccess) return cuda_fail(ce);
+    return BS_E_CORRUPT;
+}
+
+const char* bs_status_str(bs_status s) {
+    switch (s) {
+    case BS_OK: return "ok";
+    case BS_E_ARG: return "bad argument";
+    case BS_E_FORMAT: return "container fails validation";
+    case BS_E_VERSION: return "unknown container version";
+    case BS_E_SIZE: return "wrong buffer size";
+    case BS_E_CUDA: return "CUDA runtime error";
+    case BS_E_CORRUPT: return "corrupt chunk or checksum mismatch";
+    case BS_E_NOMEM: return "host allocation failed";
+    case BS_E_UNSUPPORTED: return "unsupported device or model size";
+    }
+    return "unknown status";
+}
+
+int bs_last_cuda_error(void) { return g_last_cuda; }
+
+} // extern "C"

@@ -1,0 +1,121 @@
+"""GPU encoder parity, and full-size decode parity in the bench's launch configuration.
+
+* The device encoder must write the same bytes as the oracle encoder (FORMAT.md section
+  6 fixes every choice with integer rules), and the oracle must decode them back to the
+  originals.
+* At full size (the 9B-shaped checkpoint and full-shape 27B-scale layers), every decoded
+  tensor is compared bit-exact with its regenerated original on the device. Sampled chunks
+  are also decoded by the oracle from a host copy of the same container.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+bs = pytest.importorskip("lossless_entropy_coding_interleaved_b200")
+
+
+def _gpu_items(specs, device="cuda:0"):
+    cpu = [S.generate(s, "cpu") for s in specs]
+    return cpu, [(s.name, t.to(device)) for s, t in zip(specs, cpu)]
+
+
+def _host_items(specs, cpu):
+    return [(s.name, S.words_numpy(t), "raw" if s.is_raw else "bf16") for s, t in zip(specs, cpu)]
+
+
+@pytest.mark.parametrize("name,kw", [("tensor_1m", {}), ("edge_mix", {}), ("edge_mix", {"force_rans": True}),
+                                     ("gemma2_layer", {})])
+def test_device_encoder_matches_oracle_bytes(name, kw):
+    specs = S.workload(name)
+    cpu, dev = _gpu_items(specs)
+    d_c, h_c = bs.encode(dev, host_copy=True, **kw)
+    want = oracle.encode(_host_items(specs, cpu), **kw)
+    assert h_c.size == len(want)
+    assert bytes(h_c.tobytes()) == want
+    assert torch.equal(d_c.cpu(), torch.from_numpy(h_c))
+
+
+@pytest.mark.parametrize("log2_chunk,ns,nf,max_routes", [(8, 12, 10, 7), (12, 9, 7, 2), (17, 12, 11, 15),
+                                                         (16, 11, 10, 0)])
+def test_device_encoder_parameters(log2_chunk, ns, nf, max_routes):
+    specs = S.workload("edge_mix")[:2] + S.workload("tensor_1m")
+    cpu, dev = _gpu_items(specs)
+    kw = dict(log2_chunk=log2_chunk, ns=ns, nf=nf, max_routes=max_routes)
+    _, h_c = bs.encode(dev, host_copy=True, **kw)
+    assert bytes(h_c.tobytes()) == oracle.encode(_host_items(specs, cpu), **kw)
+    for k, t in enumerate(cpu):
+        assert np.array_equal(oracle.decode(h_c, k), S.words_numpy(t))
+
+
+def test_device_encoder_sizes():
+    rng = np.random.default_rng(5)
+    sizes = [0, 1, 2, 7, 8, 255, 256, 257, 1000, 4097, 65535, 65536, 65537]
+    arrs = []
+    for n in sizes:
+        x = (rng.standard_normal(n) * 0.02).astype(np.float32)
+        arrs.append((x.view(np.uint32) >> 16).astype(np.uint16))
+    dev = [(f"n{n}", torch.from_numpy(a.view(np.int16)).cuda()) for n, a in zip(sizes, arrs)]
+    for force in (False, True):
+        _, h_c = bs.encode(dev, host_copy=True, force_rans=force)
+        assert bytes(h_c.tobytes()) == oracle.encode([(f"n{n}", a, "bf16") for n, a in zip(sizes, arrs)],
+                                                     force_rans=force)
+
+
+def test_plan_from_device_container():
+    specs = S.workload("edge_mix")
+    cpu, dev = _gpu_items(specs)
+    d_c, _ = bs.encode(dev)
+    plan = bs.Plan(d_container=d_c)                    # metadata read from the device
+    outs = plan.decode_batch(range(len(specs)))
+    plan.check()
+    for k, (s, t) in enumerate(zip(specs, dev)):
+        assert torch.equal(outs[k].view(-1), t[1].reshape(-1)), s.name
+
+
+def _full_size_check(specs, sample_chunks=3):
+    """Generate on the device, encode, decode in one batch, compare everything bit-exact,
+    then oracle-decode sampled chunks from a host copy."""
+    dev = [(s.name, S.generate(s, "cuda:0")) for s in specs]
+    d_c, h_c = bs.encode(dev, host_copy=True)
+    plan = bs.Plan(d_container=d_c)
+    outs = plan.decode_batch(range(len(specs)))
+    plan.check()
+    n = coded = 0
+    for k, (s, (_, t)) in enumerate(zip(specs, dev)):
+        assert torch.equal(outs[k].view(-1), t.view(-1)), s.name
+        i = plan.info(k)
+        n += i["n_elems"]
+        coded += i["coded_bytes"]
+    rng = np.random.default_rng(0)
+    for k in rng.choice(len(specs), size=min(4, len(specs)), replace=False):
+        i = plan.info(int(k))
+        if i["kind"] != bs.KIND_RANS:
+            continue
+        whole = np.zeros(i["n_elems"], np.uint16)
+        chunks = rng.choice(i["n_chunks"], size=min(sample_chunks, i["n_chunks"]), replace=False)
+        gpu = S.words_numpy(outs[int(k)]).reshape(-1)
+        C = 1 << i["log2_chunk"]
+        for c in chunks:
+            assert oracle.decode_chunks(h_c, int(k), int(c), int(c) + 1, whole) == 0
+            lo, hi = int(c) * C, min((int(c) + 1) * C, i["n_elems"])
+            assert np.array_equal(whole[lo:hi], gpu[lo:hi])
+    del outs, dev, plan, d_c
+    torch.cuda.empty_cache()
+    return n, coded
+
+
+def test_full_gemma2_9b_checkpoint():
+    n, coded = _full_size_check(S.workload("gemma2_9b"))
+    assert n == 9_241_702_400
+    assert coded * 8 / n < 10.6
+
+
+def test_full_shape_qwen27b_layers():
+    # two full-shape layers and the full embedding of the 27B-scale checkpoint
+    specs = S.workload("qwen_27b_scale", layers=2) + [S.workload("qwen_27b_scale")[-1]]
+    _full_size_check(specs)

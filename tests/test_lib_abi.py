@@ -1,0 +1,52 @@
+"""CPU checks of the boundary: libbs.so loads and exports every function include/bs.h
+declares. No compute call is made (there is no GPU here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "bs.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(bs_[a-z_0-9]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for want in ("bs_plan", "bs_decode_tensor", "bs_decode_batch", "bs_plan_workspace_bytes", "bs_check"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    import lossless_entropy_coding_interleaved_b200 as bs
+    lib = ctypes.CDLL(bs.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert set(bs.EXPORTS) == set(_declared())
+
+
+def test_status_strings_and_workspace_size_on_host():
+    import numpy as np
+    import lossless_entropy_coding_interleaved_b200 as bs
+    import oracle
+    assert bs.lib.bs_status_str(bs.E_CORRUPT).decode().startswith("corrupt")
+    w = np.arange(5000, dtype=np.uint16) % 300
+    c = oracle.encode([("a", w, "bf16")], force_rans=True)
+    n = bs.workspace_bytes(c)
+    assert n >= 256 + (8 << 12) + 4 * 1024
+    with pytest.raises(bs.BsError):
+        bs.workspace_bytes(c[:-16])
+
+
+def test_plan_without_gpu_fails_loudly():
+    import torch
+    import lossless_entropy_coding_interleaved_b200 as bs
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(bs.BsError):
+        bs.Plan(b"\0" * 64)
