@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Decode benchmark: full-model lossless BF16 decode on B200.
+
+One step decodes the whole 9B-shaped checkpoint, 9,241,702,400 BF16 weights in one
+container, with one bs_decode_batch call. The container and the outputs are resident in
+HBM. The synthetic weights are drawn on the device from the seeded recipe in
+synthetic/, encoded once with the device encoder (untimed), planned, and checked
+bit-exact against the originals before timing. The JSON line carries:
+
+* value      decompressed BF16 GB/s over all ranks (replicas: every rank decodes its
+             own copy of the checkpoint)
+* roofline   (compressed bytes read + BF16 bytes written) per decode step over the step's
+             CUDA-event time, against the measured HBM copy bandwidth
+* e2e        the same metric with the container copied in from pinned host memory and
+             every decoded tensor copied back out, inside the timed region
+* cpu_baseline  the oracle decoder on the host cores, on a bounded sample (layer 0)
+
+`--impl reference` times the oracle alone (host cores, rank 0) on the same sample.
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decompressed BF16 GB/s (full-model decode, 1 B200) and % HBM roofline; bits/weight"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gemma2_9b", help="a workload of synthetic/ (default: the 9B checkpoint)")
+    ap.add_argument("--layers", type=int, default=None, help="truncate a multi-layer workload (smaller cases)")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-threads", type=int, default=0, help="oracle threads (0: all host cores)")
+    return ap.parse_args()
+
+
+def _peak_hbm():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            return float(json.load(fh)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _traffic_per_weight():
+    """DRAM bytes per weight of decode_kernel from the committed ncu summary, if the kernel
+    sources still hash to what was profiled; else None."""
+    import hashlib
+    csrc = os.path.join(ROOT, "lossless_entropy_coding_interleaved_b200", "csrc")
+    try:
+        src = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("bs_kernels.cu", "bs_internal.h"))
+        lines = open(os.path.join(ROOT, "profiles", "decode_kernel_gemma2_9b.md")).read().splitlines()
+    except OSError:
+        return None
+    kv = dict(l.split(": ", 1) for l in lines if l.startswith(("kernel_sha256: ", "traffic_bytes_per_weight: ")))
+    if kv.get("kernel_sha256") != hashlib.sha256(src).hexdigest()[:16]:
+        return None
+    return float(kv["traffic_bytes_per_weight"])
+
+
+def _workload_desc(name, layers):
+    import synthetic as S
+    specs = S.workload(name, layers=layers)
+    n = sum(s.numel for s in specs if not s.is_raw)
+    d = {"gemma2_9b": "42 Gemma-2-9B-shaped decoder layers (q,k,v,o,gate,up,down + 4 RMSNorm vectors) "
+                      "+ 256000x3584 embedding",
+         "gemma2_layer": "one Gemma-2-9B-shaped decoder layer",
+         "qwen_27b_scale": "64 layers of hidden 5120 + 152064x5120 embedding",
+         "tensor_1m": "one 1024x1024 tensor", "edge_mix": "edge-case mix"}.get(name, name)
+    if layers is not None:
+        d += f" (first {layers} layers only)"
+    return specs, n, d
+
+
+# ------------------------------------------------------------------ oracle on host cores
+def _oracle_sample(workload, threads):
+    """The bounded CPU sample: layer 0 of the workload, generated and encoded on the host by
+    the oracle, then decoded by the oracle with `threads` threads over its chunks."""
+    import numpy as np
+    import oracle
+    import synthetic as S
+    specs = [s for s in S.workload(workload, layers=1) if not s.is_raw]
+    if workload in ("gemma2_9b", "qwen_27b_scale"):
+        specs = [s for s in specs if s.name.startswith("layers.0.")]
+    arrs = [S.words_numpy(S.generate(s, "cpu")) for s in specs]
+    c = np.frombuffer(oracle.encode([(s.name, a, "bf16") for s, a in zip(specs, arrs)]), np.uint8)
+    infos = [oracle.info(c, k) for k in range(len(specs))]
+    outs = [np.zeros(i["n_elems"], np.uint16) for i in infos]
+    tasks = []
+    for k, i in enumerate(infos):
+        if i["kind"] == oracle.KIND_RANS:
+            step = max(1, i["n_chunks"] // max(1, threads))
+            tasks += [(k, c0, min(c0 + step, i["n_chunks"])) for c0 in range(0, i["n_chunks"], step)]
+    n = sum(a.size for a in arrs)
+    desc = (f"oracle decode of layer 0 of {workload} ({len(specs)} tensors, {n} weights), "
+            f"{len(tasks)} chunk ranges over {threads} host threads")
+
+    def run_once(pool):
+        t0 = time.perf_counter()
+        futs = [pool.submit(oracle.decode_chunks, c, k, c0, c1, outs[k]) for k, c0, c1 in tasks]
+        for k, i in enumerate(infos):
+            if i["kind"] != oracle.KIND_RANS:
+                outs[k][:] = oracle.decode(c, k).reshape(-1)
+        assert all(f.result() == 0 for f in futs)
+        return time.perf_counter() - t0
+
+    def check():
+        for a, o in zip(arrs, outs):
+            assert np.array_equal(a.reshape(-1), o), "oracle sample decode mismatch"
+
+    return n, desc, run_once, check
+
+
+def _cpu_threads(req):
+    return req if req > 0 else (os.cpu_count() or 1)
+
+
+# ------------------------------------------------------------------ clocks during timing
+class _Clocks:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(index), "-lms", "100"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.count(",") >= 9]
+        load = [r for r in rows if r[2].strip().isdigit() and int(r[2]) > 600]
+        use = load or rows
+        sm = [int(r[2]) for r in use if r[2].strip().isdigit()]
+        mx = [int(r[3]) for r in use if r[3].strip().isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in use for i in range(4) if r[6 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(load),
+                "power_w_max": max((float(r[4]) for r in use if r[4].replace(".", "", 1).isdigit()), default=None)}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    threads = _cpu_threads(a.cpu_threads)
+    specs, n_all, desc = _workload_desc(a.workload, a.layers)
+    n, sample, run_once, check = _oracle_sample(a.workload, threads)
+    with cf.ThreadPoolExecutor(threads) as pool:
+        for _ in range(a.warmup):
+            run_once(pool)
+        check()
+        ts = [run_once(pool) for _ in range(a.steps)]
+    sec = sum(ts)
+    value = 2 * n * a.steps / sec / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(1e3 * sec / a.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u64",
+            "data": "synthetic", "config": {"workload": a.workload, "description": desc, "n_weights": n_all,
+                                            "step": "one bounded sample per step: " + sample},
+            "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(a):
+    import torch
+    import torch.distributed as dist
+
+    import lossless_entropy_coding_interleaved_b200 as bs
+    import synthetic as S
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    specs, n, desc = _workload_desc(a.workload, a.layers)
+    t0 = time.time()
+    originals = [(s.name, S.generate(s, dev)) for s in specs]
+    d_c, _ = bs.encode(originals)
+    torch.cuda.synchronize()
+    t_encode = time.time() - t0
+    plan = bs.Plan(d_container=d_c)
+    outs = [plan.empty_output(k) for k in range(plan.n_tensors)]
+    idx = list(range(plan.n_tensors))
+    infos = [plan.info(k) for k in idx]
+    coded = sum(i["coded_bytes"] for i in infos)
+    out_bytes = sum(i["out_bytes"] for i in infos)
+    bf16_n = sum(i["n_elems"] for i in infos if i["kind"] != bs.KIND_RAW)
+    bf16_coded = sum(i["coded_bytes"] for i in infos if i["kind"] != bs.KIND_RAW)
+
+    # empirical entropy H(s) + H(f|s) = H(w) of the originals, on the device
+    hbits = torch.zeros((), dtype=torch.float64, device=dev)
+    for (nm, t), s in zip(originals, specs):
+        if s.is_raw:
+            continue
+        flat = t.view(-1)
+        cnt = torch.zeros(65536, dtype=torch.int64, device=dev)
+        for lo in range(0, flat.numel(), 1 << 27):
+            cnt += torch.bincount(flat[lo:lo + (1 << 27)].to(torch.int32) & 0xFFFF, minlength=65536)
+        c = cnt[cnt > 0].to(torch.float64)
+        hbits += -(c * torch.log2(c / flat.numel())).sum()
+    h_per_w = float(hbits) / bf16_n
+
+    stream = torch.cuda.current_stream()
+    for _ in range(max(1, a.warmup)):
+        plan.decode_batch(idx, outs, stream=stream)
+    torch.cuda.synchronize()
+    plan.check()
+    parity = all(torch.equal(o.view(-1), t.view(-1)) for o, (_, t) in zip(outs, originals))
+    if not parity:
+        raise SystemExit("bench: decoded output differs from the originals")
+    del originals
+    torch.cuda.empty_cache()
+
+    # timed region: K steps, CUDA events per step on the launching stream
+    phys = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+    smi_index = phys[local] if local < len(phys) and phys[local].strip().isdigit() else str(local)
+    clocks = _Clocks(smi_index)
+    time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    l0 = bs.launch_counter()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for k in range(a.steps):
+        ev[k][0].record(stream)
+        plan.decode_batch(idx, outs, stream=stream)
+        ev[k][1].record(stream)
+    g1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = bs.launch_counter() - l0
+    clk = clocks.stop()
+    total_ms = g0.elapsed_time(g1)
+    step_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
+    plan.check()
+    t_max = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    total_ms = float(t_max)
+    value = world * a.steps * out_bytes / (total_ms * 1e-3) / 1e9
+    mean_step = statistics.mean(step_ms)
+    peak, peak_kind = _peak_hbm()
+    tpw = _traffic_per_weight()
+    achieved = (coded + out_bytes) / (mean_step * 1e-3) / 1e9
+
+    # end to end: container in from pinned host memory, every tensor back out, per step
+    e2e = None
+    if not a.no_e2e and a.e2e_steps > 0:
+        h_c = torch.empty(d_c.numel(), dtype=torch.uint8, pin_memory=True)
+        h_c.copy_(d_c)
+        h_outs = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(a.e2e_steps):
+            d_c.copy_(h_c, non_blocking=True)
+            plan.decode_batch(idx, outs, stream=stream)
+            for o, h in zip(outs, h_outs):
+                h.copy_(o, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        plan.check()
+        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e2e = {"value": round(world * a.e2e_steps * out_bytes / (float(e_ms) * 1e-3) / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": int(d_c.numel()), "d2h_bytes_per_step": int(out_bytes),
+               "steps": a.e2e_steps, "path": "Plan.decode_batch with the container copied in from pinned host "
+                                             "memory and every tensor copied back, per step"}
+        del h_c, h_outs
+
+    cpu = None
+    if rank == 0 and not a.no_cpu_baseline:
+        threads = _cpu_threads(a.cpu_threads)
+        n_s, sample, run_once, check = _oracle_sample(a.workload, threads)
+        with cf.ThreadPoolExecutor(threads) as pool:
+            run_once(pool)
+            check()
+            sec = run_once(pool)
+        cpu = {"value": round(2 * n_s / sec / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": sample}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": round(total_ms / a.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u64",
+        "data": "synthetic (seeded device draws, synthetic/ recipe)",
+        "config": {"workload": a.workload, "description": desc, "n_weights": n, "tensors": len(specs),
+                   "container_bytes": int(d_c.numel()), "coded_bytes": int(coded),
+                   "decoded_bytes": int(out_bytes),
+                   "bits_per_weight": round(bf16_coded * 8 / bf16_n, 5),
+                   "entropy_bits_per_weight": round(h_per_w, 5),
+                   "overhead_pct_vs_entropy": round(100 * (bf16_coded * 8 / bf16_n / h_per_w - 1), 4),
+                   "parallelism": f"replicas x{world} (no collective on the data path)",
+                   "l2": "no flush: inputs larger than L2 (container and outputs are GBs)",
+                   "parity": "bit-exact vs originals before timing", "encode_s": round(t_encode, 2),
+                   "words": "BF16 bit patterns; rANS state arithmetic in u64"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": (None if tpw is None else int(tpw * bf16_n)),
+                     "traffic_source": "profiles/decode_kernel_gemma2_9b.md (4-layer capture scaled by weights)",
+                     "kernel": "decode_kernel", "per_launch_bytes": int(coded + out_bytes),
+                     "launch_ms_mean": round(mean_step, 4)},
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    a = _args()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

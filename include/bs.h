@@ -109,7 +109,7 @@ bs_status bs_decode_tensor(const bs_plan_t* plan, int32_t idx, void* d_out, size
 
 /*
  * bs_decode_batch: decode n tensors in one pass. All the RANS tensors go in a single
- * kernel launch per CTA shape (more than 448 of them are split across launches), and STORED/RAW
+ * kernel launch per CTA shape (more than 500 of them are split across launches), and STORED/RAW
  * tensors in one copy launch. idx[k] goes to d_out[k], of out_bytes[k] bytes.
  *  - The outputs must not overlap.
  *  - idx, d_out and out_bytes are host arrays, read during the call.
@@ -188,6 +188,8 @@ void bs_encoder_destroy(bs_encoder_t* enc);
 
 const char* bs_status_str(bs_status s);
 int bs_last_cuda_error(void); /* the cudaError_t behind the last BS_E_CUDA on this thread */
+/* Kernel launches libbs has made in this process (all threads); a diagnostic counter. */
+uint64_t bs_launch_counter(void);
 
 #ifdef __cplusplus
 }

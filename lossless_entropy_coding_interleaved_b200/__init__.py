@@ -55,8 +55,8 @@ class _EncParams(ctypes.Structure):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libbs.so is not built ({LIB_PATH}); run `python -m "
-                          f"lossless_entropy_coding_interleaved_b200.build`")
+        raise ImportError(f"libbs.so is not built ({LIB_PATH}); run "
+                          f"`python lossless_entropy_coding_interleaved_b200/build.py`")
     L = ctypes.CDLL(LIB_PATH)
     P, i32, u64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64, ctypes.c_size_t
     L.bs_plan_workspace_bytes.argtypes = [P, sz]
@@ -73,6 +73,8 @@ def _load():
     L.bs_status_str.argtypes = [ctypes.c_int]
     L.bs_status_str.restype = ctypes.c_char_p
     L.bs_last_cuda_error.argtypes = []
+    L.bs_launch_counter.argtypes = []
+    L.bs_launch_counter.restype = u64
     L.bs_plan_workspace_bytes_device.argtypes = [P, sz, P]
     L.bs_plan_workspace_bytes_device.restype = sz
     L.bs_encoder_create.argtypes = [ctypes.POINTER(_EncItem), i32, ctypes.POINTER(_EncParams), ctypes.POINTER(P)]
@@ -94,7 +96,12 @@ lib = _load()
 EXPORTS = ("bs_plan_workspace_bytes", "bs_plan_workspace_bytes_device", "bs_plan", "bs_plan_destroy",
            "bs_tensor_count", "bs_tensor_info_get", "bs_decode_tensor", "bs_decode_batch", "bs_verify_tensor",
            "bs_check", "bs_encoder_create", "bs_encoder_scratch_bytes", "bs_encoder_run", "bs_encoder_emit",
-           "bs_encoder_destroy", "bs_status_str", "bs_last_cuda_error")
+           "bs_encoder_destroy", "bs_status_str", "bs_last_cuda_error", "bs_launch_counter")
+
+
+def launch_counter() -> int:
+    """Kernel launches libbs has made in this process."""
+    return int(lib.bs_launch_counter())
 
 
 def _check(st: int, what: str):

@@ -1,6 +1,9 @@
 """Build libbs.so (the sm_100a decoder library) in place, next to this file.
 
-    python -m lossless_entropy_coding_interleaved_b200.build [--verbose]
+    python lossless_entropy_coding_interleaved_b200/build.py [--verbose]
+
+Run it as a script (or load it by path, as __graft_entry__.build does). Importing it
+through the package would first load the library it is meant to rebuild.
 
 nvcc cross-compiles for sm_100a without a GPU, so this runs on any host with CUDA 12.9.
 """

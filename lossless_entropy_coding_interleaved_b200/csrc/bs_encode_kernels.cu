@@ -51,6 +51,7 @@ int launch_histogram(const uint16_t* in, uint64_t n, unsigned long long* d_hist,
     const uint64_t want = (n + 4095) / 4096;
     if (want < grid) grid = want;
     histogram_kernel<<<static_cast<unsigned>(grid), 512, smem, s>>>(in, n, d_hist);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -138,6 +139,7 @@ __global__ void __launch_bounds__(kEncWarps * 32) encode_kernel(const __grid_con
 int launch_encode(const EncParams& p, void* stream) {
     if (p.total_ctas == 0) return cudaSuccess;
     encode_kernel<<<p.total_ctas, kEncWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    count_launch();
     return cudaGetLastError();
 }
 

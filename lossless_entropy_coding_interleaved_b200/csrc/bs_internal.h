@@ -78,7 +78,7 @@ struct DecodeItem {
 };
 static_assert(sizeof(DecodeItem) == 64, "DecodeItem layout");
 
-constexpr int kMaxDecodeItems = 448;
+constexpr int kMaxDecodeItems = 500; // 64 B each: the parameters stay under 32 KiB
 struct DecodeParams {
     uint32_t n_items;
     uint32_t total_ctas;
@@ -139,6 +139,8 @@ int launch_encode(const EncParams& p, void* stream);
 
 // Keeps the cudaError_t behind a BS_E_CUDA for bs_last_cuda_error (bs_plan.cpp).
 void record_cuda_error(int e);
+// Counts kernel launches for bs_launch_counter (bs_plan.cpp).
+void count_launch();
 
 // Kernel launchers (bs_kernels.cu). They return a cudaError_t as int.
 int launch_decode(const DecodeParams& p, int warps, bool default_precision, uint32_t smem_bytes, void* stream);

@@ -313,6 +313,7 @@ static int launch_decode_t(const DecodeParams& p, uint32_t smem_bytes, cudaStrea
                                          static_cast<int>(smem_bytes));
     if (e != cudaSuccess) return e;
     decode_kernel<WARPS, NS, NF><<<p.total_ctas, WARPS * 32, smem_bytes, s>>>(p);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -327,6 +328,7 @@ int launch_decode(const DecodeParams& p, int warps, bool default_precision, uint
 int launch_copy(const CopyParams& p, void* stream) {
     if (p.total_blocks == 0) return cudaSuccess;
     copy_kernel<<<static_cast<unsigned>(p.total_blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -341,6 +343,7 @@ int launch_checksum(const void* data, uint64_t n, int raw_bytes, unsigned long l
     const uint64_t want = (n + 255) / 256;
     const unsigned grid = static_cast<unsigned>(want < static_cast<uint64_t>(sms) * 8 ? want : sms * 8ull);
     checksum_kernel<<<grid, 256, 0, s>>>(data, n, raw_bytes, d_sum);
+    count_launch();
     return cudaGetLastError();
 }
 

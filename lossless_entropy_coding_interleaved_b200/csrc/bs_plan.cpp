@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <memory>
 #include <new>
@@ -30,6 +31,9 @@ thread_local int g_last_cuda = 0;
 } // namespace
 
 void bs::record_cuda_error(int e) { g_last_cuda = e; }
+
+static std::atomic<unsigned long long> g_launches{0};
+void bs::count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 namespace {
 
@@ -502,5 +506,7 @@ const char* bs_status_str(bs_status s) {
 }
 
 int bs_last_cuda_error(void) { return g_last_cuda; }
+
+uint64_t bs_launch_counter(void) { return g_launches.load(std::memory_order_relaxed); }
 
 } // extern "C"

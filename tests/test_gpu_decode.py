@@ -66,7 +66,7 @@ def test_every_bit_pattern():
 
 
 def test_sizes_and_multiple_launches():
-    # 1033 tensors: more RANS tensors than one launch carries (448), every tail length
+    # 1033 tensors: more RANS tensors than one launch carries (500), every tail length
     rng = np.random.default_rng(11)
     sizes = list(range(1, 1026)) + [4095, 4096, 4097, 65535, 65536, 65537, 3 * 65536 + 255]
     items = []
