@@ -28,13 +28,10 @@ constexpr uint32_t kMaxNs = 12, kMaxNf = 11, kMaxRoutes = 15;
 constexpr int kChains = 2;
 constexpr int kRingWords = 1024;
 constexpr int kQuarterWords = kRingWords / 4;
-// The rings come first in dynamic shared memory, aligned to their 4 KiB size (so a ring
-// address is (offset & 4095) | base); kRingAlignSlack covers the alignment.
-constexpr uint32_t kRingAlignSlack = 4096;
-constexpr uint32_t ring_bytes_per_cta(int warps) {
-    return uint32_t(warps) * kChains * kRingWords * 4 + kRingAlignSlack;
-}
-constexpr uint32_t kBigCtaTableBytes = 92 * 1024;
+// The rings come first in dynamic shared memory, then the tables. The largest tables
+// (160 KiB) plus 8 warps of rings (64 KiB) fit the 227 KiB a CTA may use.
+constexpr uint32_t ring_bytes_per_cta(int warps) { return uint32_t(warps) * kChains * kRingWords * 4; }
+constexpr uint32_t kBigCtaTableBytes = 96 * 1024;
 inline int warps_for_tables(uint32_t table_bytes) { return table_bytes <= kBigCtaTableBytes ? 16 : 8; }
 
 // Workspace layout: a 256-byte error block, then 256-aligned tables per RANS tensor.

@@ -60,7 +60,7 @@ struct Chain {
     uint32_t posb;            // bytes of the word stream consumed (warp-uniform)
     uint32_t fq;              // ring quarters requested (warp-uniform)
     uint32_t total_q, n_words, stream_bytes, nc, n_blocks;
-    uint32_t ring;            // shared-memory address of the ring (4 KiB aligned)
+    uint32_t ring;            // shared-memory address of the ring
     const uint8_t* ring_ptr;  // the same ring as a pointer into the dynamic smem array
     const uint8_t* stream;
     uint16_t* out;
@@ -95,11 +95,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
         }
         s_item = lo;
     }
-    // dynamic smem: [pad to 4 KiB][rings][tables]
-    const uint32_t smem_base = smem_u32(smem);
-    const uint32_t ring_base = (smem_base + kRingAlignSlack - 1) & ~(kRingAlignSlack - 1);
-    const uint32_t tab_base = ring_base + WARPS * kChains * kRingWords * 4;
-    uint8_t* tab_ptr = smem + (tab_base - smem_base);
+    // dynamic smem: [rings][tables]
+    const uint32_t ring_base = smem_u32(smem);
+    uint8_t* tab_ptr = smem + WARPS * kChains * kRingWords * 4;
     __syncthreads();
     const DecodeItem& it = p.item[s_item];
 
@@ -126,7 +124,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
         h.chunk = chunk0 + k;
         h.live = h.chunk < n_chunks;
         h.ring = ring_base + (warp * kChains + k) * (kRingWords * 4);
-        h.ring_ptr = smem + (h.ring - smem_base);
+        h.ring_ptr = smem + (warp * kChains + k) * (kRingWords * 4);
         h.posb = 0;
         h.fq = 0;
         h.bad = false;
@@ -180,7 +178,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
                         const uint32_t piece = lane + 32u * e; // 64 pieces of 16 B per quarter
                         const uint32_t byte = h.fq * (kQuarterWords * 4u) + 16u * piece;
                         if (byte < h.stream_bytes)
-                            cp_async16(h.ring | (byte & (kRingWords * 4u - 1u)), h.stream + byte,
+                            cp_async16(h.ring + (byte & (kRingWords * 4u - 1u)), h.stream + byte,
                                        min(16u, h.stream_bytes - byte));
                     }
                     ++h.fq;

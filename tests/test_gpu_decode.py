@@ -90,6 +90,16 @@ def test_parameters(log2_chunk, ns, nf):
     assert np.array_equal(outs[0], w)
 
 
+@pytest.mark.parametrize("nf", [10, 11])
+def test_largest_tables(nf):
+    # 15 routes: 32 KiB + 16 rows x 2^nf x 4 B of tables (96 KiB / 160 KiB), the two CTA shapes
+    w = np.concatenate([((e << 7) | (np.arange(3000) % (3 + e % 5))).astype(np.uint16) for e in range(90, 110)])
+    c = oracle.encode([("skewed", w, "bf16")], nf=nf, max_routes=15)
+    assert oracle.info(c, 0)["n_routes"] == 15
+    _, outs = _decode_all(c, 1)
+    assert np.array_equal(outs[0], w)
+
+
 def test_gemma2_layer_bit_exact():
     specs = S.workload("gemma2_layer")
     arrs, items = _items(specs)
