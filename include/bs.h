@@ -137,6 +137,37 @@ bs_status bs_verify_tensor(const bs_plan_t* plan, int32_t idx, const void* d_out
  */
 bs_status bs_check(const bs_plan_t* plan, void* stream, int64_t* first_bad);
 
+/*
+ * bs_decode_tensor_noalloc: decode one tensor with no device memory from the caller beyond
+ * the container and the output. The paper has no counterpart: this is a convenience of
+ * this library.
+ *
+ * For callers that cannot allocate device memory: for example a plugin inside another
+ * runtime whose allocator owns all of the GPU's memory, or a callback where an allocation
+ * would synchronise the device or is not allowed.
+ *
+ * Instead of a caller workspace, the decode tables (at most 96 KiB) and the error block live
+ * in a static device array of 96 KiB + 256 bytes. Every GPU that loads libbs holds that array
+ * until the process exits.
+ *
+ *   h_container      host copy of the whole container; tensor idx is validated in place
+ *                    (no host allocation)
+ *   d_container      the same bytes on the device, 16-byte aligned
+ *   d_out, out_bytes as for bs_decode_tensor
+ *
+ * Behaviour:
+ *  - The first call on a device looks up the array's device address with
+ *    cudaGetSymbolAddress. Make that first call before any stream capture.
+ *  - Every call shares the array and rewrites it (the tables, and the error block is cleared).
+ *    Calls that overlap on the GPU race, so issue them on one stream or one after another.
+ *  - The call synchronises stream and returns BS_E_CORRUPT if a chunk fails its end check.
+ *  - Tables larger than 96 KiB give BS_E_SIZE. That means more routes or higher precisions
+ *    than the defaults with up to 15 routes.
+ *  - It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+bs_status bs_decode_tensor_noalloc(const void* h_container, size_t container_bytes, const void* d_container,
+                                   int32_t idx, void* d_out, size_t out_bytes, void* stream);
+
 /* ------------------------------------------------------------------------------------
  * Encoder on the device. It produces the canonical container of FORMAT.md section 4.6,
  * byte-identical to any other encoder that follows FORMAT.md section 6. The card's

@@ -73,6 +73,8 @@ def _load():
     L.bs_status_str.argtypes = [ctypes.c_int]
     L.bs_status_str.restype = ctypes.c_char_p
     L.bs_last_cuda_error.argtypes = []
+    L.bs_decode_tensor_noalloc.argtypes = [P, sz, P, i32, P, sz, P]
+    L.bs_decode_tensor_noalloc.restype = ctypes.c_int
     L.bs_launch_counter.argtypes = []
     L.bs_launch_counter.restype = u64
     L.bs_plan_workspace_bytes_device.argtypes = [P, sz, P]
@@ -96,7 +98,18 @@ lib = _load()
 EXPORTS = ("bs_plan_workspace_bytes", "bs_plan_workspace_bytes_device", "bs_plan", "bs_plan_destroy",
            "bs_tensor_count", "bs_tensor_info_get", "bs_decode_tensor", "bs_decode_batch", "bs_verify_tensor",
            "bs_check", "bs_encoder_create", "bs_encoder_scratch_bytes", "bs_encoder_run", "bs_encoder_emit",
-           "bs_encoder_destroy", "bs_status_str", "bs_last_cuda_error", "bs_launch_counter")
+           "bs_encoder_destroy", "bs_status_str", "bs_last_cuda_error", "bs_launch_counter",
+           "bs_decode_tensor_noalloc")
+
+
+def decode_noalloc(container, d_container: torch.Tensor, idx: int, out: torch.Tensor, stream=None) -> torch.Tensor:
+    """bs_decode_tensor_noalloc: decode tensor idx into out using libbs's static device
+    array instead of a workspace. For callers that cannot allocate device memory. It
+    synchronises the stream, and calls that overlap on the GPU race on the shared array."""
+    h = _host_bytes(container)
+    _check(lib.bs_decode_tensor_noalloc(h.ctypes.data, h.size, d_container.data_ptr(), idx, out.data_ptr(),
+                                        out.numel() * out.element_size(), _stream(stream)), "decode_tensor_noalloc")
+    return out
 
 
 def launch_counter() -> int:

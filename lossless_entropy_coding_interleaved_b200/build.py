@@ -17,7 +17,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libbs.so")
-SOURCES = ["bs_kernels.cu", "bs_encode_kernels.cu", "bs_plan.cpp", "bs_encode.cpp"]
+SOURCES = ["bs_kernels.cu", "bs_encode_kernels.cu", "bs_noalloc.cu", "bs_plan.cpp", "bs_encode.cpp"]
 HEADERS = ["bs_internal.h", os.path.join(ROOT, "include", "bs.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

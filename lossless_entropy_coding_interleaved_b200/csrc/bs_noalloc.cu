@@ -1,0 +1,275 @@
+// bs_noalloc.cu -- bs_decode_tensor_noalloc: decode one tensor without any device
+// memory from the caller beyond the container and the output.
+//
+// Who needs this: code that cannot call cudaMalloc or ask an allocator for a workspace.
+// Examples are a plugin running inside another runtime whose allocator owns every byte of
+// device memory, or a callback on a path where an allocation would synchronise the device
+// or is forbidden. Such callers still hand in the container and the output buffer. The
+// decode tables and the error block live in the static device array below instead of a
+// caller workspace.
+//
+// The array is file-scope device memory: every GPU that loads libbs holds it until the
+// process exits. Host code must not pass the symbol itself to a kernel, because on the host
+// it is only a stand-in. The device address is looked up once per device with
+// cudaGetSymbolAddress, on the first call made with that device current.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "bs_internal.h"
+
+namespace bs {
+
+// Largest decode tables the array holds: 96 KiB covers the default precisions (ns=12,
+// nf=10) with up to 15 fraction routes. Larger tables get BS_E_SIZE.
+constexpr uint32_t kNoAllocTableBytes = 96 * 1024;
+constexpr uint32_t kNoAllocBytes = 256 + kNoAllocTableBytes; // error block, then tables
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_addr_mutex;
+unsigned char* g_addr[kMaxDevices] = {nullptr};
+
+// Device address of g_noalloc_scratch for the current device (looked up once per device).
+cudaError_t scratch_address(unsigned char** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_addr_mutex);
+    if (!g_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_addr[dev] = static_cast<unsigned char*>(p);
+    }
+    *out = g_addr[dev];
+    return cudaSuccess;
+}
+
+uint64_t rd64(const uint8_t* p) {
+    uint64_t v;
+    std::memcpy(&v, p, 8);
+    return v;
+}
+uint32_t rd32(const uint8_t* p) {
+    uint32_t v;
+    std::memcpy(&v, p, 4);
+    return v;
+}
+uint16_t rd16(const uint8_t* p) {
+    uint16_t v;
+    std::memcpy(&v, p, 2);
+    return v;
+}
+bool in_range(uint64_t off, uint64_t n, uint64_t len) { return off <= len && n <= len - off; }
+
+} // namespace
+
+// Expand a tensor's model (read from the container on the device) into the decode-table
+// layout that decode_kernel stages (bs_internal.h): the s-table, then the fraction rows
+// with the UNIFORM row last. One CTA. It writes into the tables part of the array above.
+// The host validated the model in its own copy. The device copy is read defensively: the
+// caller zeroes the table region first, n_present comes from the host, every write is
+// bounded by its table, and a route index out of range reads as UNIFORM. So the decode
+// kernel's lookups stay inside the tables even if the two copies differ.
+__global__ void __launch_bounds__(512) noalloc_tables_kernel(const uint8_t* model, uint32_t n_present, uint32_t ns,
+                                                             uint32_t nf, uint32_t n_routes) {
+    __shared__ uint32_t s_cum[513];
+    __shared__ uint16_t f_cum[16][129];
+    unsigned char* tab = g_noalloc_scratch + 256;
+    const uint8_t* pairs = model + 4;
+    const uint8_t* route = model + 4 + 4 * n_present;
+    const uint8_t* rows = route + 256;
+    const uint32_t Mf = 1u << nf;
+    if (threadIdx.x == 0) {
+        uint32_t acc = 0;
+        for (uint32_t i = 0; i < n_present; ++i) {
+            s_cum[i] = acc;
+            acc += pairs[4 * i + 2] | (pairs[4 * i + 3] << 8);
+        }
+        s_cum[n_present] = acc;
+    }
+    if (threadIdx.x >= 32 && threadIdx.x < 32 + n_routes + 1) {
+        const uint32_t r = threadIdx.x - 32;
+        uint32_t acc = 0;
+        for (uint32_t f = 0; f < 128; ++f) {
+            f_cum[r][f] = static_cast<uint16_t>(acc);
+            acc += (r == n_routes) ? Mf / 128 : (rows[256 * r + 2 * f] | (rows[256 * r + 2 * f + 1] << 8));
+        }
+        f_cum[r][128] = static_cast<uint16_t>(acc);
+    }
+    __syncthreads();
+    uint32_t* st = reinterpret_cast<uint32_t*>(tab);
+    const uint32_t Ms = 1u << ns;
+    for (uint32_t i = threadIdx.x; i < n_present; i += blockDim.x) {
+        const uint32_t s = (pairs[4 * i] | (pairs[4 * i + 1] << 8)) & 0x1FFu;
+        const uint32_t q = s_cum[i + 1] - s_cum[i];
+        const uint8_t r = route[s & 0xFF];
+        const uint32_t fbase = (r < n_routes ? r : n_routes) * Mf;
+        for (uint32_t k = 0; k < q && s_cum[i] + k < Ms; ++k) {
+            st[2 * (s_cum[i] + k)] = q | (k << 16);
+            st[2 * (s_cum[i] + k) + 1] = (s << 7) | (fbase << 16);
+        }
+    }
+    uint32_t* ft = reinterpret_cast<uint32_t*>(tab + (8u << ns));
+    for (uint32_t j = threadIdx.x; j < (n_routes + 1) * 128; j += blockDim.x) {
+        const uint32_t r = j >> 7, f = j & 127u;
+        const uint32_t c0 = f_cum[r][f], q = static_cast<uint16_t>(f_cum[r][f + 1] - c0);
+        for (uint32_t k = 0; k < q && c0 + k < Mf; ++k) ft[r * Mf + c0 + k] = f | (q << 7) | (k << 19);
+    }
+}
+
+} // namespace bs
+
+using namespace bs;
+
+extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t len, const void* d_container_v,
+                                              int32_t idx, void* d_out, size_t out_bytes, void* stream_v) {
+    const uint8_t* b = static_cast<const uint8_t*>(h_container_v);
+    const uint8_t* d_container = static_cast<const uint8_t*>(d_container_v);
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    if (!b || !d_container || idx < 0) return BS_E_ARG;
+    if (reinterpret_cast<uintptr_t>(d_container) & 15u) return BS_E_ARG;
+    // --- validate the header and this tensor in place (FORMAT.md sections 4-5) ---
+    if (len < kHeaderBytes || std::memcmp(b, "BF16RANS", 8) != 0) return BS_E_FORMAT;
+    if (rd32(b + 8) != 1) return BS_E_VERSION;
+    if (rd32(b + 12) != kHeaderBytes || rd32(b + 20) != kDirEntryBytes || rd64(b + 56) != 0) return BS_E_FORMAT;
+    if (rd64(b + 48) != len) return BS_E_SIZE;
+    const uint32_t nt = rd32(b + 16);
+    const uint64_t dir = rd64(b + 24), names_bytes = rd64(b + 40);
+    if (dir % 16 || !in_range(dir, uint64_t(kDirEntryBytes) * nt, len) || !in_range(rd64(b + 32), names_bytes, len))
+        return BS_E_FORMAT;
+    if (static_cast<uint32_t>(idx) >= nt) return BS_E_ARG;
+    const uint8_t* d = b + dir + uint64_t(kDirEntryBytes) * idx;
+    const uint32_t kind = d[0], ndim = d[1], log2c = d[2], lanes = d[3], ns = d[4], nf = d[5], n_routes = d[6];
+    const uint64_t n = rd64(d + 16), n_chunks = rd64(d + 24), model_off = rd64(d + 32), model_bytes = rd64(d + 40);
+    const uint64_t data_off = rd64(d + 48), data_bytes = rd64(d + 56);
+    if (kind > BS_KIND_RAW || ndim > 8 || d[7] != 0 || rd64(d + 72) != 0) return BS_E_FORMAT;
+    if (uint64_t(rd32(d + 8)) + rd32(d + 12) > names_bytes) return BS_E_FORMAT;
+    unsigned __int128 prod = 1;
+    for (uint32_t i = 0; i < 8; ++i) {
+        const uint64_t v = rd64(d + 80 + 8 * i);
+        if (i >= ndim) {
+            if (v) return BS_E_FORMAT;
+            continue;
+        }
+        prod *= v;
+        if (prod > (static_cast<unsigned __int128>(1) << 64)) return BS_E_FORMAT;
+    }
+    if (prod != n || data_off % 16 || !in_range(data_off, data_bytes, len)) return BS_E_FORMAT;
+    const uint64_t want = kind == BS_KIND_RAW ? n : 2 * n;
+    if (kind == BS_KIND_STORED && n > (1ull << 62)) return BS_E_FORMAT;
+    if (out_bytes != want) return BS_E_SIZE;
+    if (want && (!d_out || (reinterpret_cast<uintptr_t>(d_out) & 15u))) return BS_E_ARG;
+
+    if (kind != BS_KIND_RANS) { // verbatim: no scratch needed, the copy kernel does it
+        if (data_bytes != want) return BS_E_FORMAT;
+        if (want == 0) return BS_OK;
+        CopyParams cp;
+        cp.n_items = 1;
+        cp.total_blocks = (want + kCopyBlockBytes - 1) / kCopyBlockBytes;
+        cp.item[0] = CopyItem{d_container + data_off, static_cast<uint8_t*>(d_out), want, 0};
+        int e = launch_copy(cp, stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+        if (e) {
+            record_cuda_error(e);
+            return BS_E_CUDA;
+        }
+        return BS_OK;
+    }
+    if (lanes != kLanes || log2c < 8 || log2c > 24 || ns < 1 || ns > kMaxNs || nf < 7 || nf > kMaxNf ||
+        n_routes > kMaxRoutes || n == 0 || n > (1ull << 40))
+        return BS_E_FORMAT;
+    if (n_chunks != ((n + (1ull << log2c) - 1) >> log2c) || data_bytes != 16 * n_chunks) return BS_E_FORMAT;
+    if (model_off % 16 || !in_range(model_off, model_bytes, len) || model_bytes < 264) return BS_E_FORMAT;
+    const uint8_t* m = b + model_off;
+    const uint32_t n_present = rd16(m);
+    if (n_present < 1 || n_present > 512 || model_bytes != 260 + 4ull * n_present + 256ull * n_routes)
+        return BS_E_FORMAT;
+    uint64_t sum = 0;
+    int prev = -1;
+    for (uint32_t i = 0; i < n_present; ++i) {
+        const int s = rd16(m + 4 + 4 * i);
+        const uint32_t q = rd16(m + 6 + 4 * i);
+        if (s <= prev || s > 511 || q == 0) return BS_E_FORMAT;
+        prev = s;
+        sum += q;
+    }
+    if (sum != (1ull << ns)) return BS_E_FORMAT;
+    const uint8_t* route = m + 4 + 4 * n_present;
+    for (int e = 0; e < 256; ++e)
+        if (route[e] != 0xFF && route[e] >= n_routes) return BS_E_FORMAT;
+    for (uint32_t r = 0; r < n_routes; ++r) {
+        sum = 0;
+        for (int f = 0; f < 128; ++f) sum += rd16(route + 256 + 256 * r + 2 * f);
+        if (sum != (1ull << nf)) return BS_E_FORMAT;
+    }
+    for (uint64_t c = 0; c < n_chunks; ++c) {
+        const uint8_t* e = b + data_off + 16 * c;
+        if (rd64(e) % 16 || !in_range(rd64(e), 256 + 4ull * rd32(e + 8), len)) return BS_E_FORMAT;
+    }
+    const uint32_t tb = table_bytes_for(ns, nf, n_routes);
+    if (tb > kNoAllocTableBytes) return BS_E_SIZE; // larger than the static array holds
+
+    // --- set-up: the array's device address on this device ---
+    unsigned char* scratch = nullptr;
+    cudaError_t ce = scratch_address(&scratch);
+    if (ce != cudaSuccess) {
+        record_cuda_error(ce);
+        return BS_E_CUDA;
+    }
+    // error block: flags = 0, first_bad = all ones; tables zeroed (the array keeps the
+    // previous call's bytes)
+    ce = cudaMemsetAsync(scratch, 0, 256 + tb, stream);
+    if (ce == cudaSuccess) ce = cudaMemsetAsync(scratch + 8, 0xFF, 8, stream);
+    if (ce != cudaSuccess) {
+        record_cuda_error(ce);
+        return BS_E_CUDA;
+    }
+    noalloc_tables_kernel<<<1, 512, 0, stream>>>(d_container + model_off, n_present, ns, nf, n_routes);
+    count_launch();
+    ce = cudaGetLastError();
+    if (ce != cudaSuccess) {
+        record_cuda_error(ce);
+        return BS_E_CUDA;
+    }
+    // --- the decode kernel, unchanged, with its tables and error block in the array ---
+    DecodeParams p; // about 31 KiB of launch parameters, on the stack (no heap use)
+    p.n_items = 1;
+    const int warps = warps_for_tables(tb);
+    const uint64_t per_cta = uint64_t(warps) * kChains;
+    p.total_ctas = static_cast<uint32_t>((n_chunks + per_cta - 1) / per_cta);
+    p.err = reinterpret_cast<unsigned long long*>(scratch);
+    DecodeItem& it = p.item[0];
+    std::memset(&it, 0, sizeof(it));
+    it.chunk_table = d_container + data_off;
+    it.container = d_container;
+    it.tables = reinterpret_cast<const uint4*>(scratch + 256);
+    it.out = static_cast<uint16_t*>(d_out);
+    it.n_elems = n;
+    it.cta_begin = 0;
+    it.tensor_index = static_cast<uint32_t>(idx);
+    it.table_bytes = tb;
+    it.log2_chunk = static_cast<uint8_t>(log2c);
+    it.ns = static_cast<uint8_t>(ns);
+    it.nf = static_cast<uint8_t>(nf);
+    int e = launch_decode(p, warps, ns == 12 && nf == 10, tb + ring_bytes_per_cta(warps), stream);
+    if (e) {
+        record_cuda_error(e);
+        return BS_E_CUDA;
+    }
+    unsigned long long flags = 0;
+    ce = cudaMemcpyAsync(&flags, scratch, 8, cudaMemcpyDeviceToHost, stream);
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(stream);
+    if (ce != cudaSuccess) {
+        record_cuda_error(ce);
+        return BS_E_CUDA;
+    }
+    return flags ? BS_E_CORRUPT : BS_OK;
+}

@@ -1,0 +1,77 @@
+"""bs_decode_tensor_noalloc: decoding without a caller workspace.
+
+Some callers cannot allocate device memory. Examples are a plugin inside another runtime
+whose allocator owns the whole GPU, or a callback where an allocation would synchronise the
+device. For them, libbs keeps the decode tables and the error block in a static device array
+instead of a workspace.
+
+This test calls that entry point through the C ABI and checks its output against the
+regular bs_decode_tensor on the same container, bit-exact (the tolerance of every decode
+test here), on two calls in a row. The file sorts last so that a run stopping at the first
+failure has already run everything else.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+bs = pytest.importorskip("lossless_entropy_coding_interleaved_b200")
+
+
+def _container():
+    specs = S.workload("tensor_1m") + [s for s in S.workload("edge_mix") if s.name in ("ragged", "one", "raw_span")]
+    arrs = [S.words_numpy(S.generate(s, "cpu")) for s in specs]
+    c = oracle.encode([(s.name, a, "raw" if s.is_raw else "bf16") for s, a in zip(specs, arrs)])
+    return specs, arrs, c
+
+
+def test_noalloc_matches_regular_decode_twice():
+    specs, arrs, c = _container()
+    plan = bs.Plan(c, device="cuda:0")
+    d_c = plan.d_container
+    for k in [0, 1, 0, 3]:       # two calls in a row on tensor 0, then others, then 0 again
+        want = plan.decode(k)
+        got = plan.empty_output(k)
+        got.fill_(0x55)
+        bs.decode_noalloc(c, d_c, k, got)
+        torch.cuda.synchronize()
+        assert torch.equal(got, want), specs[k].name
+        a = got.cpu().numpy()
+        a = a.view(np.uint16) if a.dtype == np.int16 else a
+        assert np.array_equal(a.reshape(arrs[k].shape), arrs[k])
+    plan.check()
+
+
+def test_noalloc_reports_corrupt_chunk_and_oversized_tables():
+    specs, arrs, c = _container()
+    bad = bytearray(c)
+    ti = oracle.info(c, 0)
+    e0 = ti["data_offset"] + 16 * 3
+    off = int.from_bytes(bad[e0:e0 + 8], "little")
+    bad[off + 8 * 7 + 6] ^= 0x20                       # chunk 3, lane 7's start state
+    d_bad = torch.from_numpy(np.frombuffer(bytes(bad), np.uint8).copy()).cuda()
+    out = torch.empty(arrs[0].shape, dtype=torch.int16, device="cuda:0")
+    with pytest.raises(bs.BsError) as e:
+        bs.decode_noalloc(bytes(bad), d_bad, 0, out)
+    assert e.value.code == bs.E_CORRUPT
+    # a clean call right after: the shared error block starts from zero again
+    d_c = torch.from_numpy(np.frombuffer(c, np.uint8).copy()).cuda()
+    bs.decode_noalloc(c, d_c, 0, out)
+    assert np.array_equal(out.cpu().numpy().view(np.uint16).reshape(arrs[0].shape), arrs[0])
+    # tables above the 96 KiB the static array holds: 16 exponents, each with a skewed
+    # fraction distribution, give 15 routes; at nf = 11 that is 32 KiB + 16 x 8 KiB
+    w = np.concatenate([((e << 7) | (np.arange(1000) % 3)).astype(np.uint16) for e in range(100, 116)])
+    big = oracle.encode([("skewed", w, "bf16")], nf=11, max_routes=15)
+    assert oracle.info(big, 0)["n_routes"] == 15
+    d_big = torch.from_numpy(np.frombuffer(big, np.uint8).copy()).cuda()
+    out = torch.empty(w.size, dtype=torch.int16, device="cuda:0")
+    with pytest.raises(bs.BsError) as e:
+        bs.decode_noalloc(big, d_big, 0, out)
+    assert e.value.code == bs.E_SIZE
+    # the same tensor through the regular path (workspace from the caller) decodes fine
+    plan = bs.Plan(big, device="cuda:0")
+    assert np.array_equal(plan.decode(0).cpu().numpy().view(np.uint16), w)
