@@ -23,7 +23,7 @@ constexpr uint32_t kMaxNs = 12, kMaxNf = 11, kMaxRoutes = 15;
 // chains per lane), and a CTA of kWarps warps covers kWarps*kChains chunks of one tensor.
 // Each chunk's word stream goes through its own shared-memory ring of kRingWords 32-bit
 // words, in quarters of kRingWords/4 words.
-// Two CTA shapes: 16 warps when the tensor's tables fit in kBigCtaTableBytes, else 8 warps
+// Three CTA shapes by table size: 20 warps up to 64 KiB of tables, 16 up to 96 KiB, else 8
 // (the largest tables, 160 KiB, plus 8 warps of rings fit in the 227 KiB a CTA may use).
 constexpr int kChains = 2;
 constexpr int kRingWords = 1024;
@@ -32,7 +32,10 @@ constexpr int kQuarterWords = kRingWords / 4;
 // (160 KiB) plus 8 warps of rings (64 KiB) fit the 227 KiB a CTA may use.
 constexpr uint32_t ring_bytes_per_cta(int warps) { return uint32_t(warps) * kChains * kRingWords * 4; }
 constexpr uint32_t kBigCtaTableBytes = 96 * 1024;
-inline int warps_for_tables(uint32_t table_bytes) { return table_bytes <= kBigCtaTableBytes ? 16 : 8; }
+constexpr uint32_t kHugeCtaTableBytes = 64 * 1024;  // 20 warps: 160 KiB of rings + 64 KiB
+inline int warps_for_tables(uint32_t table_bytes) {
+    return table_bytes <= kHugeCtaTableBytes ? 20 : table_bytes <= kBigCtaTableBytes ? 16 : 8;
+}
 
 // Workspace layout: a 256-byte error block, then 256-aligned tables per RANS tensor.
 constexpr uint64_t kErrBlockBytes = 256;
@@ -52,12 +55,18 @@ struct Tensor {
 // ---- Decode tables (built on the host, copied to the workspace, staged in smem) ----
 // s-table: 2^ns entries of 8 bytes, indexed by slot = x & (2^ns - 1):
 //   .x = freq | (bias << 16)        freq = Fs[s] (<= 4096), bias = slot - cum_s(s)
-//   .y = (s << 7) | (fbase << 16)   s already in its output position; fbase = first
-//                                   f-table word of the route that e = s & 0xFF selects
+//   .y = (s << 7) | (frow << 16)    s already in its output position; frow locates the
+//                                   f-table row of the route that e = s & 0xFF selects:
+//                                   its byte offset when nf <= 10, its word offset when
+//                                   nf = 11 (see frow_field)
 // f-table: (n_routes + 1) rows of 2^nf u32 entries (the last row is UNIFORM):
 //   bits 0-6 fraction, bits 7-18 freq, bits 19-30 bias
 inline uint32_t table_bytes_for(uint32_t ns, uint32_t nf, uint32_t n_routes) {
     return (8u << ns) + 4u * (n_routes + 1) * (1u << nf);
+}
+// The frow field of an s-entry for fraction row `row` (it must fit in 16 bits).
+__host__ __device__ inline uint32_t frow_field(uint32_t row, uint32_t nf) {
+    return nf <= 10 ? (row << (nf + 2)) : (row << nf);
 }
 
 // ---- Kernel launch parameters (passed by value, __grid_constant__) ----

@@ -15,8 +15,12 @@
 //    lane owns 8 contiguous output weights per 8 steps. Those leave as one 16-byte store,
 //    so a warp writes 512 contiguous bytes per chunk.
 //  * The tensor's decode tables (s-table 8 B/slot, f-table rows 4 B/slot) are staged once
-//    per CTA in shared memory. A CTA (16 warps, or 8 for the largest tables) decodes
-//    32 (16) chunks of the same tensor.
+//    per CTA in shared memory, at offset 0 so that table addresses fold into constants. A
+//    CTA of 20 warps (tables up to 64 KiB), 16 (up to 96 KiB) or 8 (up to 160 KiB) decodes
+//    40, 32 or 16 chunks of the same tensor; 20 warps x 2 chains is the most that the
+//    register file holds (96 registers per thread).
+//  * Full 256-weight blocks take a path without store bounds; the ragged tail and chunks
+//    of unequal length take a checked path.
 //  * The word stream of a chunk is prefetched into its own shared-memory ring with
 //    cp.async (16 B per lane, in quarters of 256 words), kept 2-3 quarters ahead; the
 //    upkeep runs every 16 steps.
@@ -82,6 +86,8 @@ __device__ __forceinline__ void rans_update(uint32_t& lo, uint32_t& hi, uint32_t
 // NS/NF > 0: compile-time precisions (the default container); 0: read from the item.
 template <int WARPS, int NS, int NF>
 __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
+    // dynamic smem: [s-table][f-rows][rings]; the tables start at offset 0 so that table
+    // addresses are an index times the entry size plus a constant
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ int s_item;
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
@@ -95,16 +101,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
         }
         s_item = lo;
     }
-    // dynamic smem: [rings][tables]
-    const uint32_t ring_base = smem_u32(smem);
-    uint8_t* tab_ptr = smem + WARPS * kChains * kRingWords * 4;
     __syncthreads();
     const DecodeItem& it = p.item[s_item];
 
     // stage the tables
     const uint32_t tb = it.table_bytes;
     {
-        uint4* dst = reinterpret_cast<uint4*>(tab_ptr);
+        uint4* dst = reinterpret_cast<uint4*>(smem);
         for (uint32_t k = tid; k < tb / 16u; k += blockDim.x) dst[k] = __ldg(it.tables + k);
     }
     __syncthreads();
@@ -116,6 +119,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
     const uint64_t chunk0 = static_cast<uint64_t>(blockIdx.x - it.cta_begin) * (WARPS * kChains) + warp * kChains;
     if (chunk0 >= n_chunks) return;
 
+    const uint32_t ring_off = tb + (warp * kChains) * (kRingWords * 4); // this warp's first ring
+    const uint32_t ring_base = smem_u32(smem) + ring_off;
     Chain c[kChains];
     uint32_t nb = 0;
 #pragma unroll
@@ -123,8 +128,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
         Chain& h = c[k];
         h.chunk = chunk0 + k;
         h.live = h.chunk < n_chunks;
-        h.ring = ring_base + (warp * kChains + k) * (kRingWords * 4);
-        h.ring_ptr = smem + (warp * kChains + k) * (kRingWords * 4);
+        h.ring = ring_base + k * (kRingWords * 4);
+        h.ring_ptr = smem + ring_off + k * (kRingWords * 4);
         h.posb = 0;
         h.fq = 0;
         h.bad = false;
@@ -156,14 +161,14 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
 
     const uint32_t ns = NS > 0 ? NS : it.ns, nf = NF > 0 ? NF : it.nf;
     const uint32_t smask = (1u << ns) - 1u, fmask = (1u << nf) - 1u;
-    const uint8_t* ftab = tab_ptr + (8u << ns);
+    const uint8_t* ftab = smem + (8u << ns);
     const uint32_t lt = lanemask_lt();
 
-    // blocks of 16 steps (two octets); the last may be a single octet
-    for (uint32_t blk = 0; blk < nb; blk += 2) {
-        // Ring upkeep: request up to quarter q+3 for each chain, where q holds the next
-        // word. The next 16 steps need at most quarters q..q+2. Wait for every copy, or
-        // for all but the newest group when those quarters were already requested.
+    // Ring upkeep before a block of 16 steps: request up to quarter q+3 for each chain,
+    // where q holds the next word. The next 16 steps need at most quarters q..q+2. Wait for
+    // every copy, or for all but the newest group when those were requested earlier.
+    // Quarters wholly inside the stream skip the per-piece bounds.
+    auto upkeep = [&](uint32_t blk) {
         __syncwarp();
         bool newest_needed = blk == 0;
 #pragma unroll
@@ -173,13 +178,21 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
                 const uint32_t q = h.posb / (kQuarterWords * 4u);
                 if (h.fq <= min(q + 2, h.total_q - 1)) newest_needed = true;
                 while (h.fq < q + 4 && h.fq < h.total_q) {
+                    const uint32_t qb = h.fq * (kQuarterWords * 4u);
+                    if (qb + kQuarterWords * 4u <= h.stream_bytes) {
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const uint32_t piece = lane + 32u * e; // 64 pieces of 16 B per quarter
-                        const uint32_t byte = h.fq * (kQuarterWords * 4u) + 16u * piece;
-                        if (byte < h.stream_bytes)
-                            cp_async16(h.ring + (byte & (kRingWords * 4u - 1u)), h.stream + byte,
-                                       min(16u, h.stream_bytes - byte));
+                        for (int e = 0; e < 2; ++e) {
+                            const uint32_t byte = qb + 16u * (lane + 32u * e);
+                            cp_async16(h.ring + (byte & (kRingWords * 4u - 1u)), h.stream + byte, 16u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const uint32_t byte = qb + 16u * (lane + 32u * e);
+                            if (byte < h.stream_bytes)
+                                cp_async16(h.ring + (byte & (kRingWords * 4u - 1u)), h.stream + byte,
+                                           min(16u, h.stream_bytes - byte));
+                        }
                     }
                     ++h.fq;
                 }
@@ -189,39 +202,72 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
         if (newest_needed) cp_async_wait<0>();
         else cp_async_wait<1>();
         __syncwarp();
+    };
 
+    // 8 steps of every chain, interleaved; o[k] receives chain k's 8 words as 4 pairs
+    auto octet = [&](uint32_t (&o)[kChains][4]) {
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+#pragma unroll
+            for (int k = 0; k < kChains; ++k) {
+                Chain& h = c[k];
+                // sign+exponent symbol
+                const uint2 se = *reinterpret_cast<const uint2*>(smem + ((h.lo & smask) << 3));
+                rans_update(h.lo, h.hi, se.x & 0xFFFFu, se.x >> 16, ns);
+                // fraction, from the row the symbol's exponent selects (frow_field)
+                const uint32_t fslot = h.lo & fmask;
+                const uint32_t fe = *reinterpret_cast<const uint32_t*>(
+                    ftab + (nf <= 10 ? (se.y >> 16) + (fslot << 2) : ((se.y >> 16) + fslot) << 2));
+                rans_update(h.lo, h.hi, (fe >> 7) & 0xFFFu, fe >> 19, nf);
+                // renormalise: lanes below 2^32 take the next words, in lane order
+                // (branch-free: every lane reads; the ones that need no word discard it)
+                const bool need = h.hi == 0;
+                const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
+                const uint32_t w = *reinterpret_cast<const uint32_t*>(
+                    h.ring_ptr + ((h.posb + (__popc(m & lt) << 2)) & (kRingWords * 4u - 1u)));
+                h.hi = need ? h.lo : h.hi;
+                h.lo = need ? w : h.lo;
+                h.posb += __popc(m) << 2;
+                // w = (s << 7) | f: s sits pre-shifted in se.y
+                const uint32_t word = (se.y & 0xFF80u) | (fe & 0x7Fu);
+                if (s & 1) o[k][s >> 1] = __byte_perm(o[k][s >> 1], word, 0x5410);
+                else o[k][s >> 1] = word;
+            }
+        }
+    };
+
+    // Full blocks first: every live chain has all 256 weights of the block, so the stores
+    // need no bounds; blocks are taken two at a time.
+    uint32_t nb_full = 0xFFFFFFFFu;
+#pragma unroll
+    for (int k = 0; k < kChains; ++k)
+        if (c[k].live) nb_full = min(nb_full, c[k].nc >> 8);
+    uint32_t blk = 0;
+    for (; blk + 2 <= nb_full; blk += 2) {
+        upkeep(blk);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            uint32_t o[kChains][4];
+            octet(o);
+            const uint32_t b = blk + half, i0 = (b << 8) + (lane << 3);
+#pragma unroll
+            for (int k = 0; k < kChains; ++k) {
+                Chain& h = c[k];
+                if (h.live) *reinterpret_cast<uint4*>(h.out + i0) = make_uint4(o[k][0], o[k][1], o[k][2], o[k][3]);
+                if (b + 1 == h.n_blocks) // end check: state back at L, every word consumed
+                    h.bad |= (h.lo != 0) | (h.hi != 1) | (h.posb != h.stream_bytes);
+            }
+        }
+    }
+    // The rest (ragged tails, chains of different lengths), with bounds, two blocks at a time.
+    for (; blk < nb; blk += 2) {
+        upkeep(blk);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             const uint32_t b = blk + half;
             if (b >= nb) break;
             uint32_t o[kChains][4];
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-#pragma unroll
-                for (int k = 0; k < kChains; ++k) {
-                    Chain& h = c[k];
-                    // sign+exponent symbol
-                    const uint2 se = *reinterpret_cast<const uint2*>(tab_ptr + ((h.lo & smask) << 3));
-                    rans_update(h.lo, h.hi, se.x & 0xFFFFu, se.x >> 16, ns);
-                    // fraction, from the table the symbol's exponent selects
-                    const uint32_t fe =
-                        *reinterpret_cast<const uint32_t*>(ftab + (((se.y >> 16) + (h.lo & fmask)) << 2));
-                    rans_update(h.lo, h.hi, (fe >> 7) & 0xFFFu, fe >> 19, nf);
-                    // renormalise: lanes below 2^32 take the next words, in lane order
-                    // (branch-free: every lane reads; the ones that need no word discard it)
-                    const bool need = h.hi == 0;
-                    const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
-                    const uint32_t w = *reinterpret_cast<const uint32_t*>(
-                        h.ring_ptr + ((h.posb + (__popc(m & lt) << 2)) & (kRingWords * 4u - 1u)));
-                    h.hi = need ? h.lo : h.hi;
-                    h.lo = need ? w : h.lo;
-                    h.posb += __popc(m) << 2;
-                    // w = (s << 7) | f: s sits pre-shifted in se.y
-                    const uint32_t word = (se.y & 0xFF80u) | (fe & 0x7Fu);
-                    if (s & 1) o[k][s >> 1] = __byte_perm(o[k][s >> 1], word, 0x5410);
-                    else o[k][s >> 1] = word;
-                }
-            }
+            octet(o);
 #pragma unroll
             for (int k = 0; k < kChains; ++k) {
                 Chain& h = c[k];
@@ -318,6 +364,8 @@ static int launch_decode_t(const DecodeParams& p, uint32_t smem_bytes, cudaStrea
 int launch_decode(const DecodeParams& p, int warps, bool default_precision, uint32_t smem_bytes, void* stream) {
     if (p.total_ctas == 0) return cudaSuccess;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (warps == 20)
+        return default_precision ? launch_decode_t<20, 12, 10>(p, smem_bytes, s) : launch_decode_t<20, 0, 0>(p, smem_bytes, s);
     if (warps == 16)
         return default_precision ? launch_decode_t<16, 12, 10>(p, smem_bytes, s) : launch_decode_t<16, 0, 0>(p, smem_bytes, s);
     return default_precision ? launch_decode_t<8, 12, 10>(p, smem_bytes, s) : launch_decode_t<8, 0, 0>(p, smem_bytes, s);

@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(512) noalloc_tables_kernel(const uint8_t* mode
         const uint32_t s = (pairs[4 * i] | (pairs[4 * i + 1] << 8)) & 0x1FFu;
         const uint32_t q = s_cum[i + 1] - s_cum[i];
         const uint8_t r = route[s & 0xFF];
-        const uint32_t fbase = (r < n_routes ? r : n_routes) * Mf;
+        const uint32_t fbase = frow_field(r < n_routes ? r : n_routes, nf);
         for (uint32_t k = 0; k < q && s_cum[i] + k < Ms; ++k) {
             st[2 * (s_cum[i] + k)] = q | (k << 16);
             st[2 * (s_cum[i] + k) + 1] = (s << 7) | (fbase << 16);

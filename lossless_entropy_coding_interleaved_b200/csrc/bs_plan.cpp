@@ -213,7 +213,7 @@ void build_tables(const Tensor& t, uint8_t* dst) {
     const uint32_t Mf = 1u << t.nf;
     auto fbase = [&](uint32_t s) -> uint32_t {
         const uint8_t r = route[s & 0xFF];
-        return (r == 0xFF ? t.n_routes : r) * Mf;
+        return frow_field(r == 0xFF ? t.n_routes : r, t.nf);
     };
     uint32_t* st = reinterpret_cast<uint32_t*>(dst);
     uint32_t cum = 0;
@@ -365,14 +365,15 @@ bs_status bs_decode_batch(const bs_plan_t* plan, const int32_t* idx, void* const
         if (t.kind == BS_KIND_RANS && !aligned(d_out[k], 16)) return BS_E_ARG;
     }
     // One parameter block per CTA shape (16 or 8 warps) and one for verbatim copies.
-    // (16 or 8 warps) x (default precisions ns=12/nf=10, or any)
+    // (20, 16 or 8 warps) x (default precisions ns=12/nf=10, or any)
     struct Pending {
         std::unique_ptr<DecodeParams> p;
         int warps;
         bool default_precision;
         uint32_t smem = 0;
     };
-    Pending dec[4] = {{nullptr, 16, true}, {nullptr, 16, false}, {nullptr, 8, true}, {nullptr, 8, false}};
+    Pending dec[6] = {{nullptr, 20, true}, {nullptr, 20, false}, {nullptr, 16, true},
+                      {nullptr, 16, false}, {nullptr, 8, true}, {nullptr, 8, false}};
     for (Pending& d : dec) {
         d.p.reset(new (std::nothrow) DecodeParams);
         if (!d.p) return BS_E_NOMEM;
@@ -406,7 +407,7 @@ bs_status bs_decode_batch(const bs_plan_t* plan, const int32_t* idx, void* const
         if (t.kind == BS_KIND_RANS) {
             const int warps = warps_for_tables(t.table_bytes);
             const bool dflt = t.ns == 12 && t.nf == 10;
-            Pending& d = dec[(warps == 16 ? 0 : 2) + (dflt ? 0 : 1)];
+            Pending& d = dec[(warps == 20 ? 0 : warps == 16 ? 2 : 4) + (dflt ? 0 : 1)];
             const uint64_t per_cta = uint64_t(warps) * kChains;
             const uint64_t ctas = (t.n_chunks + per_cta - 1) / per_cta;
             if (d.p->n_items == kMaxDecodeItems || d.p->total_ctas + ctas > 0x7FFFFFFFull) {
