@@ -165,6 +165,42 @@ class _Clocks:
                 "power_w_max": max((float(r[4]) for r in use if r[4].replace(".", "", 1).isdigit()), default=None)}
 
 
+# ------------------------------------------------------------------ ranks (replicas only)
+class _Ranks:
+    """One process per GPU, launched by torch.distributed.run. The ranks are independent
+    replicas: the only collectives are the barriers around the timed region and the max of
+    the ranks' times, none of them on the data path."""
+
+    def __init__(self, backend="nccl", device=None, timeout_s=300):
+        import datetime
+        import torch.distributed as dist
+        self.dist = dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.device = device
+        if self.world > 1:
+            kw = {"device_id": device} if backend == "nccl" and device is not None else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max(self, value: float) -> float:
+        """The largest value over all ranks (every rank gets it)."""
+        if self.world == 1:
+            return float(value)
+        import torch
+        t = torch.tensor([float(value)], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t)
+
+    def close(self):
+        if self.world > 1:
+            self.dist.destroy_process_group()
+
+
 # ------------------------------------------------------------------ reference arm
 def run_reference(a):
     rank = int(os.environ.get("RANK", "0"))
@@ -194,23 +230,16 @@ def run_reference(a):
 # ------------------------------------------------------------------ our arm
 def run_ours(a):
     import torch
-    import torch.distributed as dist
 
     import lossless_entropy_coding_interleaved_b200 as bs
     import synthetic as S
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    ranks = _Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    barrier = ranks.barrier
 
     specs, n, desc = _workload_desc(a.workload, a.layers)
     t0 = time.time()
@@ -274,10 +303,7 @@ def run_ours(a):
     total_ms = g0.elapsed_time(g1)
     step_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
     plan.check()
-    t_max = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    total_ms = float(t_max)
+    total_ms = ranks.max(total_ms)
     value = world * a.steps * out_bytes / (total_ms * 1e-3) / 1e9
     mean_step = statistics.mean(step_ms)
     peak, peak_kind = _peak_hbm()
@@ -303,10 +329,8 @@ def run_ours(a):
         torch.cuda.synchronize()
         barrier()
         plan.check()
-        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-        e2e = {"value": round(world * a.e2e_steps * out_bytes / (float(e_ms) * 1e-3) / 1e9, 3), "unit": "GB/s",
+        e_ms = ranks.max(e0.elapsed_time(e1))
+        e2e = {"value": round(world * a.e2e_steps * out_bytes / (e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
                "h2d_bytes_per_step": int(d_c.numel()), "d2h_bytes_per_step": int(out_bytes),
                "steps": a.e2e_steps, "path": "Plan.decode_batch with the container copied in from pinned host "
                                              "memory and every tensor copied back, per step"}
@@ -323,8 +347,7 @@ def run_ours(a):
         cpu = {"value": round(2 * n_s / sec / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": sample}
 
-    if world > 1:
-        dist.destroy_process_group()
+    ranks.close()
     if rank != 0:
         return
     line = {
