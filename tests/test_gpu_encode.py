@@ -119,3 +119,26 @@ def test_full_shape_qwen27b_layers():
     # two full-shape layers and the full embedding of the 27B-scale checkpoint
     specs = S.workload("qwen_27b_scale", layers=2) + [S.workload("qwen_27b_scale")[-1]]
     _full_size_check(specs)
+
+
+def test_every_tensor_of_the_27b_scale_checkpoint():
+    # all 64 layers and the embedding, each layer encoded and decoded as its own container
+    specs = S.workload("qwen_27b_scale")
+    layers = {}
+    for s in specs:
+        layers.setdefault(s.name.split(".")[1] if s.name.startswith("layers.") else "embed", []).append(s)
+    n = coded = 0
+    for key, group in layers.items():
+        dev = [(s.name, S.generate(s, "cuda:0")) for s in group]
+        d_c, _ = bs.encode(dev)
+        plan = bs.Plan(d_container=d_c)
+        outs = plan.decode_batch(range(len(group)))
+        plan.check()
+        for k, (s, (_, t)) in enumerate(zip(group, dev)):
+            assert torch.equal(outs[k].view(-1), t.view(-1)), s.name
+            n += plan.info(k)["n_elems"]
+            coded += plan.info(k)["coded_bytes"]
+        del dev, outs, plan, d_c
+    torch.cuda.empty_cache()
+    assert n == 30_642_012_160
+    assert coded * 8 / n < 10.7
