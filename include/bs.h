@@ -217,6 +217,83 @@ bs_status bs_encoder_emit(bs_encoder_t* enc, void* d_scratch, void* d_container,
                           void* h_container, void* stream);
 void bs_encoder_destroy(bs_encoder_t* enc);
 
+/* ------------------------------------------------------------------------------------
+ * Layer streaming: decode groups of tensors on demand from a container in HOST memory
+ * into a bounded device cache, with least-recently-used eviction. This is the device
+ * counterpart of the low-VRAM streaming loader on the "Gemma 2 9B Instruct -- Lossless
+ * Compressed" card (section "Low-VRAM streaming"): layers are decompressed as they are
+ * needed, under a cap on device memory (the card's lru_max_vram_gb). The card gives only
+ * that API, so the policy and the memory layout below are this library's.
+ *
+ * group_of_tensor[k] is the group of tensor k (directory order). Group numbers run
+ * 0..G-1 and each is used at least once; a group is typically one layer.
+ * d_arena is the whole device budget, owned by the caller (256-byte aligned). It holds:
+ *   - two staging slots, each the size of the largest group's compressed byte range;
+ *   - then the cache of decoded groups.
+ * Eviction is least-recently-used among unpinned groups. A prefetched group is kept until it
+ * has been acquired once, unless nothing else can make room.
+ * Loading a group runs on the stream given to prefetch or acquire, in three steps:
+ *   1. one cudaMemcpyAsync host-to-device of the group's compressed bytes into a slot;
+ *   2. the decode kernels (the same as bs_decode_batch) into a cache block;
+ *   3. events that order the later reuse of the slot and of the block.
+ * No call blocks the host, except create (which uploads the tables) and check.
+ * For the copies to overlap other work, h_container should be page-locked.
+ * h_container must stay valid and unchanged until bs_streamer_destroy.
+ * Device memory is never allocated. The library's host memory is freed by destroy.
+ * The object is internally locked: calls from several host threads are serialised.
+ * After a BS_E_CUDA from prefetch or acquire the cache may have lost the block being loaded
+ * (the block is never reused while work may still write into it); destroy and recreate.
+ * ------------------------------------------------------------------------------------ */
+typedef struct bs_streamer_t bs_streamer_t;
+
+typedef struct {
+    uint64_t loads;            /* groups staged and decoded */
+    uint64_t hits;             /* acquires that found their group resident */
+    uint64_t evictions;        /* groups dropped from the cache to make room */
+    uint64_t h2d_bytes;        /* compressed bytes copied host-to-device */
+    uint64_t decoded_bytes;    /* bytes of decoded cache blocks written */
+    uint64_t resident_groups;  /* groups in the cache now */
+    uint64_t cache_bytes;      /* size of the cache part of the arena */
+    uint64_t cache_bytes_used; /* bytes of it held by resident groups now */
+    uint64_t stage_bytes;      /* size of one staging slot */
+} bs_streamer_stats_t;
+
+/* Device workspace bytes (decode tables and error block); 0 if the container fails validation. */
+size_t bs_streamer_workspace_bytes(const void* h_container, size_t container_bytes);
+/* The smallest arena for this grouping: two staging slots plus the largest decoded group.
+ * 0 if the container fails validation or the grouping is invalid. */
+size_t bs_streamer_min_arena_bytes(const void* h_container, size_t container_bytes, const int32_t* group_of_tensor);
+/* Validate the container (as bs_plan does) and upload the decode tables into d_workspace on
+ * stream, then synchronise it. Returns:
+ *   BS_E_SIZE when the workspace or the arena is too small;
+ *   BS_E_ARG for a bad grouping;
+ *   BS_E_UNSUPPORTED off sm_100.
+ * The streamer is bound to the current device. */
+bs_status bs_streamer_create(const void* h_container, size_t container_bytes, const int32_t* group_of_tensor,
+                             void* d_workspace, size_t workspace_bytes, void* d_arena, size_t arena_bytes,
+                             void* stream, bs_streamer_t** out);
+bs_status bs_streamer_group_count(const bs_streamer_t* s, int32_t* n);
+/* As bs_tensor_info_get; the name stays valid until bs_streamer_destroy. */
+bs_status bs_streamer_tensor_info_get(const bs_streamer_t* s, int32_t idx, bs_tensor_info* info);
+/* Queue the load of a group that is not resident. Returns BS_OK at once if it is resident.
+ * Returns BS_E_SIZE when the groups now acquired leave no room for it. */
+bs_status bs_streamer_prefetch(bs_streamer_t* s, int32_t group, void* stream);
+/* Make the group resident (loading it on `stream` if needed) and pin it.
+ * d_ptrs[0..n_ptrs) receives the device address of each of its tensors, in ascending
+ * tensor index. RANS/STORED tensors are BF16 words, RAW tensors are bytes, and every
+ * address is 256-byte aligned. n_ptrs must equal the group's tensor count (else BS_E_SIZE).
+ * Work queued on `stream` after this call sees the decoded data, including a load started
+ * on another stream by prefetch. Every acquire needs a matching release. */
+bs_status bs_streamer_acquire(bs_streamer_t* s, int32_t group, void** d_ptrs, int32_t n_ptrs, void* stream);
+/* Unpin after the work queued on `stream` so far. The group may then be evicted, and its
+ * memory is reused only after that work. */
+bs_status bs_streamer_release(bs_streamer_t* s, int32_t group, void* stream);
+bs_status bs_streamer_get_stats(bs_streamer_t* s, bs_streamer_stats_t* out);
+/* As bs_check, for the streamer's error word: synchronises stream. */
+bs_status bs_streamer_check(bs_streamer_t* s, void* stream, int64_t* first_bad);
+/* Frees host state only. It does not synchronise: finish the streams before freeing the arena. */
+void bs_streamer_destroy(bs_streamer_t* s);
+
 const char* bs_status_str(bs_status s);
 int bs_last_cuda_error(void); /* the cudaError_t behind the last BS_E_CUDA on this thread */
 /* Kernel launches libbs has made in this process (all threads); a diagnostic counter. */

@@ -49,6 +49,12 @@ class _EncItem(ctypes.Structure):
                 ("name_bytes", ctypes.c_uint32), ("reserved", ctypes.c_uint32)]
 
 
+class _StreamStats(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_uint64) for k in ("loads", "hits", "evictions", "h2d_bytes", "decoded_bytes",
+                                                "resident_groups", "cache_bytes", "cache_bytes_used",
+                                                "stage_bytes")]
+
+
 class _EncParams(ctypes.Structure):
     _fields_ = [(k, ctypes.c_uint32) for k in ("log2_chunk", "ns", "nf", "max_routes", "force_rans")]
 
@@ -85,6 +91,23 @@ def _load():
     L.bs_encoder_emit.argtypes = [P, P, P, sz, P, P]
     L.bs_encoder_destroy.argtypes = [P]
     L.bs_encoder_destroy.restype = None
+    L.bs_streamer_workspace_bytes.argtypes = [P, sz]
+    L.bs_streamer_workspace_bytes.restype = sz
+    L.bs_streamer_min_arena_bytes.argtypes = [P, sz, P]
+    L.bs_streamer_min_arena_bytes.restype = sz
+    L.bs_streamer_create.argtypes = [P, sz, P, P, sz, P, sz, P, ctypes.POINTER(P)]
+    L.bs_streamer_group_count.argtypes = [P, ctypes.POINTER(i32)]
+    L.bs_streamer_tensor_info_get.argtypes = [P, i32, ctypes.POINTER(_Info)]
+    L.bs_streamer_prefetch.argtypes = [P, i32, P]
+    L.bs_streamer_acquire.argtypes = [P, i32, P, i32, P]
+    L.bs_streamer_release.argtypes = [P, i32, P]
+    L.bs_streamer_get_stats.argtypes = [P, ctypes.POINTER(_StreamStats)]
+    L.bs_streamer_check.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
+    L.bs_streamer_destroy.argtypes = [P]
+    L.bs_streamer_destroy.restype = None
+    for fn in ("bs_streamer_create", "bs_streamer_group_count", "bs_streamer_tensor_info_get", "bs_streamer_prefetch", "bs_streamer_acquire",
+               "bs_streamer_release", "bs_streamer_get_stats", "bs_streamer_check"):
+        getattr(L, fn).restype = ctypes.c_int
     for fn in ("bs_plan", "bs_tensor_count", "bs_tensor_info_get", "bs_decode_tensor", "bs_decode_batch",
                "bs_verify_tensor", "bs_check", "bs_last_cuda_error", "bs_encoder_create", "bs_encoder_scratch_bytes",
                "bs_encoder_run", "bs_encoder_emit"):
@@ -99,7 +122,10 @@ EXPORTS = ("bs_plan_workspace_bytes", "bs_plan_workspace_bytes_device", "bs_plan
            "bs_tensor_count", "bs_tensor_info_get", "bs_decode_tensor", "bs_decode_batch", "bs_verify_tensor",
            "bs_check", "bs_encoder_create", "bs_encoder_scratch_bytes", "bs_encoder_run", "bs_encoder_emit",
            "bs_encoder_destroy", "bs_status_str", "bs_last_cuda_error", "bs_launch_counter",
-           "bs_decode_tensor_noalloc")
+           "bs_decode_tensor_noalloc", "bs_streamer_workspace_bytes", "bs_streamer_min_arena_bytes",
+           "bs_streamer_create", "bs_streamer_group_count", "bs_streamer_tensor_info_get", "bs_streamer_prefetch",
+           "bs_streamer_acquire",
+           "bs_streamer_release", "bs_streamer_get_stats", "bs_streamer_check", "bs_streamer_destroy")
 
 
 def decode_noalloc(container, d_container: torch.Tensor, idx: int, out: torch.Tensor, stream=None) -> torch.Tensor:
@@ -137,6 +163,28 @@ def _host_bytes(container) -> np.ndarray:
     else:
         a = np.frombuffer(container, dtype=np.uint8)
     return a
+
+
+def _info_dict(ti: _Info) -> dict:
+    d = {k: getattr(ti, k) for k, _ in _Info._fields_ if k not in ("shape", "name", "name_bytes", "reserved")}
+    d["shape"] = tuple(ti.shape[i] for i in range(ti.ndim))
+    d["name"] = ctypes.string_at(ti.name, ti.name_bytes).decode() if ti.name_bytes else ""
+    return d
+
+
+def _container_names(h: np.ndarray) -> list:
+    """Tensor names in directory order, read from a container that already passed
+    validation (FORMAT.md 4.1: n_tensors at 16, dir_offset at 24, names_offset at 32;
+    4.2: 144-byte entries with name_offset at 8 and name_bytes at 12)."""
+    hdr = h[:64].tobytes()
+    nt = int.from_bytes(hdr[16:20], "little")
+    d0, n0 = int.from_bytes(hdr[24:32], "little"), int.from_bytes(hdr[32:40], "little")
+    names = []
+    for k in range(nt):
+        e = h[d0 + 144 * k: d0 + 144 * k + 16].tobytes()
+        off, nb = int.from_bytes(e[8:12], "little"), int.from_bytes(e[12:16], "little")
+        names.append(h[n0 + off: n0 + off + nb].tobytes().decode())
+    return names
 
 
 def workspace_bytes(container) -> int:
@@ -249,10 +297,7 @@ class Plan:
     def _get_info(self, idx: int) -> dict:
         ti = _Info()
         _check(lib.bs_tensor_info_get(self._p, idx, ctypes.byref(ti)), "tensor_info")
-        d = {k: getattr(ti, k) for k, _ in _Info._fields_ if k not in ("shape", "name", "name_bytes", "reserved")}
-        d["shape"] = tuple(ti.shape[i] for i in range(ti.ndim))
-        d["name"] = ctypes.string_at(ti.name, ti.name_bytes).decode() if ti.name_bytes else ""
-        return d
+        return _info_dict(ti)
 
     def info(self, idx: int) -> dict:
         return dict(self._info[idx])
@@ -300,4 +345,127 @@ class Plan:
         if st == E_CORRUPT:
             raise BsError(st, "check", "corrupt chunk", first_bad=fb.value)
         _check(st, "check")
+        return fb.value
+
+
+def _group_list(groups, names) -> list:
+    if callable(groups):
+        keys = {}
+        groups = [keys.setdefault(groups(n), len(keys)) for n in names]
+    groups = [int(g) for g in groups]
+    if len(groups) != len(names):
+        raise BsError(E_ARG, "streamer", "one group number per tensor")
+    return groups
+
+
+def streamer_min_arena_bytes(container, groups) -> int:
+    """bs_streamer_min_arena_bytes: the smallest device budget for this grouping (two
+    staging slots plus the largest decoded group)."""
+    h = container.numpy() if isinstance(container, torch.Tensor) else _host_bytes(container)
+    if lib.bs_streamer_workspace_bytes(h.ctypes.data, h.size) == 0:
+        raise BsError(E_FORMAT, "streamer", "container fails validation")
+    g = _group_list(groups, _container_names(h))
+    ga = (ctypes.c_int32 * max(1, len(g)))(*g)
+    n = lib.bs_streamer_min_arena_bytes(h.ctypes.data, h.size, ga)
+    if n == 0:
+        raise BsError(E_ARG, "streamer", "invalid grouping")
+    return n
+
+
+class Streamer:
+    """Layer streaming (bs_streamer_*): decode groups of tensors on demand from a container
+    in host memory into a device cache of ``arena_bytes`` with least-recently-used eviction.
+
+    ``groups`` gives each tensor's group number in directory order: a list of ints, or a
+    callable name -> hashable key, whose distinct keys are numbered in order of first use.
+    The host bytes are copied once into page-locked memory, so the host-to-device copies
+    can overlap other work; a page-locked uint8 CPU tensor is used in place instead. ``arena_bytes`` is the whole device budget: two staging slots
+    plus the cache (at least ``min_arena_bytes``).
+    """
+
+    def __init__(self, container, groups, arena_bytes: int | None = None, device="cuda", stream=None):
+        if not torch.cuda.is_available():
+            raise BsError(E_UNSUPPORTED, "streamer", "no CUDA device")
+        self.device = torch.device(device)
+        if isinstance(container, torch.Tensor) and container.dtype == torch.uint8 and container.is_pinned():
+            self.host = container.reshape(-1)          # used in place: it must stay unchanged
+        else:
+            h = _host_bytes(container)
+            self.host = torch.empty(h.size, dtype=torch.uint8, pin_memory=True)
+            self.host.numpy()[:] = h
+        hp, hn = self.host.data_ptr(), self.host.numel()
+        ws = lib.bs_streamer_workspace_bytes(hp, hn)
+        if ws == 0:
+            raise BsError(E_FORMAT, "streamer", "container fails validation")
+        self.names = _container_names(self.host.numpy())
+        groups = _group_list(groups, self.names)
+        self._groups = (ctypes.c_int32 * max(1, len(groups)))(*groups)
+        self.min_arena_bytes = lib.bs_streamer_min_arena_bytes(hp, hn, self._groups)
+        if self.min_arena_bytes == 0:
+            raise BsError(E_ARG, "streamer", "invalid grouping")
+        if arena_bytes is None:
+            arena_bytes = self.min_arena_bytes
+        with torch.cuda.device(self.device):
+            self.workspace = torch.empty(ws, dtype=torch.uint8, device=self.device)
+            self.arena = torch.empty(arena_bytes, dtype=torch.uint8, device=self.device)
+            ptr = ctypes.c_void_p()
+            _check(lib.bs_streamer_create(hp, hn, self._groups, self.workspace.data_ptr(), ws,
+                                          self.arena.data_ptr(), arena_bytes, _stream(stream), ctypes.byref(ptr)),
+                   "streamer_create")
+        self._s = ptr
+        n = ctypes.c_int32()
+        _check(lib.bs_streamer_group_count(self._s, ctypes.byref(n)), "streamer_group_count")
+        self.n_groups = n.value
+        self.members = [[k for k, g in enumerate(groups) if g == j] for j in range(self.n_groups)]
+        self._info = []
+        for k in range(len(self.names)):
+            ti = _Info()
+            _check(lib.bs_streamer_tensor_info_get(self._s, k, ctypes.byref(ti)), "streamer_tensor_info")
+            self._info.append(_info_dict(ti))
+
+    def info(self, idx: int) -> dict:
+        return dict(self._info[idx])
+
+    def __del__(self):
+        s = getattr(self, "_s", None)
+        if s and lib is not None:
+            torch.cuda.synchronize(self.device)
+            lib.bs_streamer_destroy(s)
+            self._s = None
+
+    def prefetch(self, group: int, stream=None):
+        _check(lib.bs_streamer_prefetch(self._s, group, _stream(stream)), "streamer_prefetch")
+
+    def acquire(self, group: int, stream=None) -> list:
+        """Pin the group and return its tensors as views into the arena (int16 words shaped
+        like the originals, uint8 for RAW), valid until release."""
+        m = self.members[group] if 0 <= group < self.n_groups else []
+        ptrs = (ctypes.c_void_p * max(1, len(m)))()
+        _check(lib.bs_streamer_acquire(self._s, group, ptrs, len(m), _stream(stream)), "streamer_acquire")
+        base = self.arena.data_ptr()
+        out = []
+        for k, p in zip(m, ptrs):
+            i = self._info[k]
+            off = (p or base) - base
+            if i["kind"] == KIND_RAW:
+                out.append(self.arena[off:off + i["n_elems"]])
+            else:
+                v = self.arena[off:off + 2 * i["n_elems"]].view(torch.int16)
+                out.append(v.view(i["shape"]) if i["shape"] else v.view(()))
+        return out
+
+    def release(self, group: int, stream=None):
+        _check(lib.bs_streamer_release(self._s, group, _stream(stream)), "streamer_release")
+
+    def stats(self) -> dict:
+        st = _StreamStats()
+        _check(lib.bs_streamer_get_stats(self._s, ctypes.byref(st)), "streamer_stats")
+        return {k: getattr(st, k) for k, _ in _StreamStats._fields_}
+
+    def check(self, stream=None) -> int:
+        fb = ctypes.c_int64()
+        st = lib.bs_streamer_check(self._s, _stream(stream), ctypes.byref(fb))
+        if st == E_CORRUPT:
+            raise BsError(st, "streamer_check", "corrupt chunk", first_bad=fb.value)
+        _check(st, "streamer_check")
         return fb.value

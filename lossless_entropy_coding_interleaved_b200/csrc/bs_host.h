@@ -1,0 +1,62 @@
+// bs_host.h -- host-side pieces of libbs shared by the planner (bs_plan.cpp) and the layer
+// streamer (bs_stream.cpp): container parsing, the workspace image, and the batching of
+// decode and copy work into kernel launches.
+#pragma once
+
+#include <cstdint>
+#include <memory>
+#include <vector>
+
+#include "bs_internal.h"
+
+namespace bs {
+
+inline uint64_t up256(uint64_t v) { return (v + 255) & ~uint64_t(255); }
+
+// Parse and validate a container held in host memory (FORMAT.md sections 4-5).
+bs_status parse_host_container(const uint8_t* h, uint64_t len, std::vector<Tensor>& out);
+
+// Bytes of the decode workspace: the error block, then each RANS tensor's tables.
+uint64_t workspace_bytes_for(const std::vector<Tensor>& ts);
+
+// Assign each RANS tensor its ws_offset and write the workspace image. The image holds
+// the error block (no flag set, first_bad = all ones) and the decode tables.
+// Returns BS_E_UNSUPPORTED when a tensor's tables and rings exceed the device's shared
+// memory per block.
+bs_status build_workspace(std::vector<Tensor>& ts, std::vector<uint8_t>& image);
+
+// Bins decode work by CTA shape (20, 16 or 8 warps) and precision (default ns=12/nf=10,
+// or any), and verbatim copies into one copy list. It launches a bin when the bin is full,
+// and launches every bin on flush().
+class DecodeBatch {
+  public:
+    // d_err: the workspace's error block.
+    explicit DecodeBatch(unsigned long long* d_err) : err_(d_err) {}
+    bs_status init(); // allocates the parameter blocks (about 220 KB of host memory)
+    // Queue tensor t, whose chunk offsets are relative to d_container, for decoding into d_out.
+    // Launches on `stream` when a bin fills up.
+    bs_status add(const Tensor& t, uint32_t tensor_index, const uint8_t* d_container, const uint8_t* d_ws,
+                  void* d_out, void* stream);
+    bs_status flush(void* stream);
+
+  private:
+    struct Bin {
+        std::unique_ptr<DecodeParams> p;
+        int warps = 0;
+        bool default_precision = false;
+        uint32_t smem = 0;
+    };
+    bs_status flush_bin(Bin& b, void* stream);
+    bs_status flush_copy(void* stream);
+    unsigned long long* err_;
+    Bin bins_[6];
+    std::unique_ptr<CopyParams> cp_;
+};
+
+// bs_tensor_info for tensor t; the name points into t.
+void fill_tensor_info(const Tensor& t, bs_tensor_info* o);
+
+// Records e for bs_last_cuda_error and returns BS_E_CUDA.
+bs_status cuda_status(int e);
+
+} // namespace bs

@@ -12,7 +12,7 @@
 #include <new>
 #include <vector>
 
-#include "bs_internal.h"
+#include "bs_host.h"
 
 using namespace bs;
 
@@ -37,10 +37,7 @@ void bs::count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 namespace {
 
-bs_status cuda_fail(cudaError_t e) {
-    g_last_cuda = static_cast<int>(e);
-    return BS_E_CUDA;
-}
+bs_status cuda_fail(cudaError_t e) { return cuda_status(static_cast<int>(e)); }
 
 uint64_t get_u64(const uint8_t* p) {
     uint64_t v;
@@ -59,7 +56,6 @@ uint16_t get_u16(const uint8_t* p) {
 }
 bool inside(uint64_t off, uint64_t bytes, uint64_t len) { return off <= len && bytes <= len - off; }
 uint64_t up16(uint64_t v) { return (v + 15) & ~uint64_t(15); }
-uint64_t up256(uint64_t v) { return (v + 255) & ~uint64_t(255); }
 
 // Reads container bytes from a host copy or, without one, from device memory.
 struct Reader {
@@ -237,12 +233,154 @@ void build_tables(const Tensor& t, uint8_t* dst) {
     }
 }
 
-uint64_t workspace_for(const std::vector<Tensor>& ts) {
+} // namespace
+
+uint64_t bs::workspace_bytes_for(const std::vector<Tensor>& ts) {
     uint64_t ws = kErrBlockBytes;
     for (const Tensor& t : ts)
         if (t.kind == BS_KIND_RANS) ws += up256(t.table_bytes);
     return ws;
 }
+
+bs_status bs::cuda_status(int e) {
+    g_last_cuda = e;
+    return BS_E_CUDA;
+}
+
+bs_status bs::parse_host_container(const uint8_t* h, uint64_t len, std::vector<Tensor>& out) {
+    if (!h) return BS_E_ARG;
+    Reader rd;
+    rd.host = h;
+    rd.len = len;
+    return parse(rd, out);
+}
+
+bs_status bs::build_workspace(std::vector<Tensor>& ts, std::vector<uint8_t>& image) {
+    const int smem_cap = max_dynamic_smem();
+    try {
+        image.assign(workspace_bytes_for(ts), 0);
+    } catch (...) {
+        return BS_E_NOMEM;
+    }
+    uint64_t pos = kErrBlockBytes;
+    for (Tensor& t : ts) {
+        if (t.kind != BS_KIND_RANS) continue;
+        if (static_cast<int>(t.table_bytes + ring_bytes_per_cta(warps_for_tables(t.table_bytes))) > smem_cap)
+            return BS_E_UNSUPPORTED;
+        t.ws_offset = pos;
+        build_tables(t, image.data() + pos);
+        pos += up256(t.table_bytes);
+    }
+    std::memset(image.data() + 8, 0xFF, 8); // error block: flags = 0, first_bad = all ones
+    return BS_OK;
+}
+
+void bs::fill_tensor_info(const Tensor& t, bs_tensor_info* o) {
+    std::memset(o, 0, sizeof(*o));
+    o->n_elems = t.n_elems;
+    o->out_bytes = t.kind == BS_KIND_RAW ? t.n_elems : 2 * t.n_elems;
+    o->coded_bytes = t.coded_bytes;
+    o->n_chunks = t.n_chunks;
+    o->checksum = t.checksum;
+    for (int i = 0; i < 8; ++i) o->shape[i] = t.shape[i];
+    o->kind = t.kind;
+    o->ndim = t.ndim;
+    o->ns = t.ns;
+    o->nf = t.nf;
+    o->n_routes = t.n_routes;
+    o->log2_chunk = t.log2_chunk;
+    o->name = t.name.data();
+    o->name_bytes = static_cast<uint32_t>(t.name.size());
+}
+
+bs_status DecodeBatch::init() {
+    const int shapes[3] = {20, 16, 8};
+    for (int k = 0; k < 6; ++k) {
+        bins_[k].p.reset(new (std::nothrow) DecodeParams);
+        if (!bins_[k].p) return BS_E_NOMEM;
+        bins_[k].warps = shapes[k / 2];
+        bins_[k].default_precision = k % 2 == 0;
+        bins_[k].p->n_items = 0;
+        bins_[k].p->total_ctas = 0;
+        bins_[k].p->err = err_;
+    }
+    cp_.reset(new (std::nothrow) CopyParams);
+    if (!cp_) return BS_E_NOMEM;
+    cp_->n_items = 0;
+    cp_->total_blocks = 0;
+    return BS_OK;
+}
+
+bs_status DecodeBatch::flush_bin(Bin& b, void* stream) {
+    if (b.p->n_items == 0) return BS_OK;
+    const int e = launch_decode(*b.p, b.warps, b.default_precision, b.smem, stream);
+    b.p->n_items = 0;
+    b.p->total_ctas = 0;
+    b.smem = 0;
+    return e ? cuda_status(e) : BS_OK;
+}
+
+bs_status DecodeBatch::flush_copy(void* stream) {
+    if (cp_->n_items == 0) return BS_OK;
+    const int e = launch_copy(*cp_, stream);
+    cp_->n_items = 0;
+    cp_->total_blocks = 0;
+    return e ? cuda_status(e) : BS_OK;
+}
+
+bs_status DecodeBatch::add(const Tensor& t, uint32_t tensor_index, const uint8_t* d_container,
+                           const uint8_t* d_ws, void* d_out, void* stream) {
+    if (t.kind == BS_KIND_RANS) {
+        const int warps = warps_for_tables(t.table_bytes);
+        const bool dflt = t.ns == 12 && t.nf == 10;
+        Bin& b = bins_[(warps == 20 ? 0 : warps == 16 ? 2 : 4) + (dflt ? 0 : 1)];
+        const uint64_t per_cta = uint64_t(warps) * kChains;
+        const uint64_t ctas = (t.n_chunks + per_cta - 1) / per_cta;
+        if (b.p->n_items == kMaxDecodeItems || b.p->total_ctas + ctas > 0x7FFFFFFFull) {
+            bs_status s = flush_bin(b, stream);
+            if (s) return s;
+        }
+        DecodeItem& it = b.p->item[b.p->n_items++];
+        std::memset(&it, 0, sizeof(it));
+        it.chunk_table = d_container + t.data_offset;
+        it.container = d_container;
+        it.tables = reinterpret_cast<const uint4*>(d_ws + t.ws_offset);
+        it.out = static_cast<uint16_t*>(d_out);
+        it.n_elems = t.n_elems;
+        it.cta_begin = b.p->total_ctas;
+        it.tensor_index = tensor_index;
+        it.table_bytes = t.table_bytes;
+        it.log2_chunk = static_cast<uint8_t>(t.log2_chunk);
+        it.ns = static_cast<uint8_t>(t.ns);
+        it.nf = static_cast<uint8_t>(t.nf);
+        b.p->total_ctas += static_cast<uint32_t>(ctas);
+        b.smem = std::max<uint32_t>(b.smem, t.table_bytes + ring_bytes_per_cta(warps));
+    } else if (t.n_elems) {
+        const uint64_t bytes = t.kind == BS_KIND_RAW ? t.n_elems : 2 * t.n_elems;
+        const uint64_t blks = (bytes + kCopyBlockBytes - 1) / kCopyBlockBytes;
+        if (cp_->n_items == kMaxCopyItems || cp_->total_blocks + blks > 0x7FFFFFFFull) {
+            bs_status s = flush_copy(stream);
+            if (s) return s;
+        }
+        CopyItem& it = cp_->item[cp_->n_items++];
+        it.src = d_container + t.data_offset;
+        it.dst = static_cast<uint8_t*>(d_out);
+        it.bytes = bytes;
+        it.blk_begin = cp_->total_blocks;
+        cp_->total_blocks += blks;
+    }
+    return BS_OK;
+}
+
+bs_status DecodeBatch::flush(void* stream) {
+    for (Bin& b : bins_) {
+        bs_status s = flush_bin(b, stream);
+        if (s) return s;
+    }
+    return flush_copy(stream);
+}
+
+namespace {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -257,7 +395,7 @@ size_t bs_plan_workspace_bytes(const void* h_container, size_t container_bytes) 
     rd.host = static_cast<const uint8_t*>(h_container);
     rd.len = container_bytes;
     if (parse(rd, ts) != BS_OK) return 0;
-    return workspace_for(ts);
+    return workspace_bytes_for(ts);
 }
 
 size_t bs_plan_workspace_bytes_device(const void* d_container, size_t container_bytes, void* stream) {
@@ -268,7 +406,7 @@ size_t bs_plan_workspace_bytes_device(const void* d_container, size_t container_
     rd.stream = static_cast<cudaStream_t>(stream);
     rd.len = container_bytes;
     if (parse(rd, ts) != BS_OK) return 0;
-    return workspace_for(ts);
+    return workspace_bytes_for(ts);
 }
 
 bs_status bs_plan(const void* h_container, size_t container_bytes, const void* d_container, void* d_workspace,
@@ -292,25 +430,10 @@ bs_status bs_plan(const void* h_container, size_t container_bytes, const void* d
     rd.len = container_bytes;
     bs_status st = parse(rd, p->tensors);
     if (st != BS_OK) return st;
-    const uint64_t ws = workspace_for(p->tensors);
+    const uint64_t ws = workspace_bytes_for(p->tensors);
     if (workspace_bytes < ws) return BS_E_SIZE;
-    const int smem_cap = max_dynamic_smem();
-    try {
-        p->host_tables.assign(ws, 0);
-    } catch (...) {
-        return BS_E_NOMEM;
-    }
-    uint64_t pos = kErrBlockBytes;
-    for (Tensor& t : p->tensors) {
-        if (t.kind != BS_KIND_RANS) continue;
-        if (static_cast<int>(t.table_bytes + ring_bytes_per_cta(warps_for_tables(t.table_bytes))) > smem_cap)
-            return BS_E_UNSUPPORTED;
-        t.ws_offset = pos;
-        build_tables(t, p->host_tables.data() + pos);
-        pos += up256(t.table_bytes);
-    }
-    // error block: flags = 0, first_bad = all ones
-    std::memset(p->host_tables.data() + 8, 0xFF, 8);
+    st = build_workspace(p->tensors, p->host_tables);
+    if (st != BS_OK) return st;
     ce = cudaMemcpyAsync(d_workspace, p->host_tables.data(), ws, cudaMemcpyHostToDevice,
                          static_cast<cudaStream_t>(stream));
     if (ce != cudaSuccess) return cuda_fail(ce);
@@ -333,22 +456,7 @@ bs_status bs_tensor_count(const bs_plan_t* plan, int32_t* n) {
 
 bs_status bs_tensor_info_get(const bs_plan_t* plan, int32_t idx, bs_tensor_info* o) {
     if (!plan || !o || idx < 0 || idx >= static_cast<int32_t>(plan->tensors.size())) return BS_E_ARG;
-    const Tensor& t = plan->tensors[idx];
-    std::memset(o, 0, sizeof(*o));
-    o->n_elems = t.n_elems;
-    o->out_bytes = t.kind == BS_KIND_RAW ? t.n_elems : 2 * t.n_elems;
-    o->coded_bytes = t.coded_bytes;
-    o->n_chunks = t.n_chunks;
-    o->checksum = t.checksum;
-    for (int i = 0; i < 8; ++i) o->shape[i] = t.shape[i];
-    o->kind = t.kind;
-    o->ndim = t.ndim;
-    o->ns = t.ns;
-    o->nf = t.nf;
-    o->n_routes = t.n_routes;
-    o->log2_chunk = t.log2_chunk;
-    o->name = t.name.data();
-    o->name_bytes = static_cast<uint32_t>(t.name.size());
+    fill_tensor_info(plan->tensors[idx], o);
     return BS_OK;
 }
 
@@ -364,91 +472,15 @@ bs_status bs_decode_batch(const bs_plan_t* plan, const int32_t* idx, void* const
         if (want && !d_out[k]) return BS_E_ARG;
         if (t.kind == BS_KIND_RANS && !aligned(d_out[k], 16)) return BS_E_ARG;
     }
-    // One parameter block per CTA shape (16 or 8 warps) and one for verbatim copies.
-    // (20, 16 or 8 warps) x (default precisions ns=12/nf=10, or any)
-    struct Pending {
-        std::unique_ptr<DecodeParams> p;
-        int warps;
-        bool default_precision;
-        uint32_t smem = 0;
-    };
-    Pending dec[6] = {{nullptr, 20, true}, {nullptr, 20, false}, {nullptr, 16, true},
-                      {nullptr, 16, false}, {nullptr, 8, true}, {nullptr, 8, false}};
-    for (Pending& d : dec) {
-        d.p.reset(new (std::nothrow) DecodeParams);
-        if (!d.p) return BS_E_NOMEM;
-    }
-    std::unique_ptr<CopyParams> cp(new (std::nothrow) CopyParams);
-    if (!cp) return BS_E_NOMEM;
-    for (Pending& d : dec) {
-        d.p->n_items = 0;
-        d.p->total_ctas = 0;
-        d.p->err = reinterpret_cast<unsigned long long*>(plan->d_ws);
-    }
-    cp->n_items = 0;
-    cp->total_blocks = 0;
-    auto flush_decode = [&](Pending& d) -> bs_status {
-        if (d.p->n_items == 0) return BS_OK;
-        const int e = launch_decode(*d.p, d.warps, d.default_precision, d.smem, stream);
-        d.p->n_items = 0;
-        d.p->total_ctas = 0;
-        d.smem = 0;
-        return e ? cuda_fail(static_cast<cudaError_t>(e)) : BS_OK;
-    };
-    auto flush_copy = [&]() -> bs_status {
-        if (cp->n_items == 0) return BS_OK;
-        const int e = launch_copy(*cp, stream);
-        cp->n_items = 0;
-        cp->total_blocks = 0;
-        return e ? cuda_fail(static_cast<cudaError_t>(e)) : BS_OK;
-    };
+    DecodeBatch batch(reinterpret_cast<unsigned long long*>(plan->d_ws));
+    bs_status st = batch.init();
+    if (st) return st;
     for (int32_t k = 0; k < n; ++k) {
-        const Tensor& t = plan->tensors[idx[k]];
-        if (t.kind == BS_KIND_RANS) {
-            const int warps = warps_for_tables(t.table_bytes);
-            const bool dflt = t.ns == 12 && t.nf == 10;
-            Pending& d = dec[(warps == 20 ? 0 : warps == 16 ? 2 : 4) + (dflt ? 0 : 1)];
-            const uint64_t per_cta = uint64_t(warps) * kChains;
-            const uint64_t ctas = (t.n_chunks + per_cta - 1) / per_cta;
-            if (d.p->n_items == kMaxDecodeItems || d.p->total_ctas + ctas > 0x7FFFFFFFull) {
-                bs_status s = flush_decode(d);
-                if (s) return s;
-            }
-            DecodeItem& it = d.p->item[d.p->n_items++];
-            std::memset(&it, 0, sizeof(it));
-            it.chunk_table = plan->d_container + t.data_offset;
-            it.container = plan->d_container;
-            it.tables = reinterpret_cast<const uint4*>(plan->d_ws + t.ws_offset);
-            it.out = static_cast<uint16_t*>(d_out[k]);
-            it.n_elems = t.n_elems;
-            it.cta_begin = d.p->total_ctas;
-            it.tensor_index = static_cast<uint32_t>(idx[k]);
-            it.table_bytes = t.table_bytes;
-            it.log2_chunk = static_cast<uint8_t>(t.log2_chunk);
-            it.ns = static_cast<uint8_t>(t.ns);
-            it.nf = static_cast<uint8_t>(t.nf);
-            d.p->total_ctas += static_cast<uint32_t>(ctas);
-            d.smem = std::max<uint32_t>(d.smem, t.table_bytes + ring_bytes_per_cta(warps));
-        } else if (t.n_elems) {
-            const uint64_t bytes = t.kind == BS_KIND_RAW ? t.n_elems : 2 * t.n_elems;
-            const uint64_t blks = (bytes + kCopyBlockBytes - 1) / kCopyBlockBytes;
-            if (cp->n_items == kMaxCopyItems || cp->total_blocks + blks > 0x7FFFFFFFull) {
-                bs_status s = flush_copy();
-                if (s) return s;
-            }
-            CopyItem& it = cp->item[cp->n_items++];
-            it.src = plan->d_container + t.data_offset;
-            it.dst = static_cast<uint8_t*>(d_out[k]);
-            it.bytes = bytes;
-            it.blk_begin = cp->total_blocks;
-            cp->total_blocks += blks;
-        }
+        st = batch.add(plan->tensors[idx[k]], static_cast<uint32_t>(idx[k]), plan->d_container, plan->d_ws,
+                       d_out[k], stream);
+        if (st) return st;
     }
-    for (Pending& d : dec) {
-        bs_status s = flush_decode(d);
-        if (s) return s;
-    }
-    return flush_copy();
+    return batch.flush(stream);
 }
 
 bs_status bs_decode_tensor(const bs_plan_t* plan, int32_t idx, void* d_out, size_t out_bytes, void* stream) {
