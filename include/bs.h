@@ -5,7 +5,8 @@
  * paragraph after its accounting table:
  *   - each BF16 word is split into sign:1 | exponent:8 | fraction:7;
  *   - the joint sign+exponent symbol is rANS-coded with a per-tensor model;
- *   - the decoded symbol selects the distribution of the 7-bit fraction;
+ *   - the decoded symbol selects the distribution of the 7-bit fraction (here a table over
+ *     its top three bits; the low four bits are kept verbatim);
  *   - the fields are recombined bitwise, so the output is byte-identical to the original.
  * The container layout (interleaved 32-lane chunks, tables, raw spans, checksum) is
  * specified in FORMAT.md in this repository.
@@ -58,10 +59,10 @@ typedef struct {
     uint64_t shape[8];
     uint32_t kind;        /* BS_KIND_* */
     uint32_t ndim;
-    uint32_t ns, nf, n_routes, log2_chunk; /* RANS model parameters */
+    uint32_t ns, nh, n_routes, log2_chunk; /* RANS model parameters (FORMAT.md section 2) */
     const char* name;     /* not NUL-terminated; points into the plan */
     uint32_t name_bytes;
-    uint32_t reserved;
+    uint32_t nib_mode;    /* RANS: 0 = nibbles stored, 0x10 + c = every low nibble is c */
 } bs_tensor_info;
 
 /* Bytes of device workspace that bs_plan needs for this container: the decode
@@ -146,8 +147,8 @@ bs_status bs_check(const bs_plan_t* plan, void* stream, int64_t* first_bad);
  * runtime whose allocator owns all of the GPU's memory, or a callback where an allocation
  * would synchronise the device or is not allowed.
  *
- * Instead of a caller workspace, the decode tables (at most 96 KiB) and the error block live
- * in a static device array of 96 KiB + 256 bytes. Every GPU that loads libbs holds that array
+ * Instead of a caller workspace, the decode tables (at most 66 KiB) and the error block live
+ * in a static device array of 66 KiB + 256 bytes. Every GPU that loads libbs holds that array
  * until the process exits.
  *
  *   h_container      host copy of the whole container; tensor idx is validated in place
@@ -161,8 +162,8 @@ bs_status bs_check(const bs_plan_t* plan, void* stream, int64_t* first_bad);
  *  - Every call shares the array and rewrites it (the tables, and the error block is cleared).
  *    Calls that overlap on the GPU race, so issue them on one stream or one after another.
  *  - The call synchronises stream and returns BS_E_CORRUPT if a chunk fails its end check.
- *  - Tables larger than 96 KiB give BS_E_SIZE. That means more routes or higher precisions
- *    than the defaults with up to 15 routes.
+ *  - Tables larger than 66 KiB give BS_E_SIZE. No valid container has such a tensor: 66 KiB
+ *    is the s-table at ns = 13 plus 16 fraction rows at nh = 5.
  *  - It calls no cudaMalloc, cudaFree or other allocating routine.
  */
 bs_status bs_decode_tensor_noalloc(const void* h_container, size_t container_bytes, const void* d_container,
@@ -199,9 +200,9 @@ typedef struct {
 
 typedef struct {
     uint32_t log2_chunk;  /* 8..24, default 16 */
-    uint32_t ns;          /* 1..12, default 12 */
-    uint32_t nf;          /* 7..11, default 10 */
-    uint32_t max_routes;  /* 0..15, default 7 */
+    uint32_t ns;          /* 1..13, default 11 */
+    uint32_t nh;          /* 3..5 with ns + nh <= 16, default 5 */
+    uint32_t max_routes;  /* 0..15, default 15 */
     uint32_t force_rans;  /* 1: never fall back to STORED (tests only) */
 } bs_enc_params;
 

@@ -39,8 +39,8 @@ class _Info(ctypes.Structure):
     _fields_ = [("n_elems", ctypes.c_uint64), ("out_bytes", ctypes.c_uint64), ("coded_bytes", ctypes.c_uint64),
                 ("n_chunks", ctypes.c_uint64), ("checksum", ctypes.c_uint64), ("shape", ctypes.c_uint64 * 8),
                 ("kind", ctypes.c_uint32), ("ndim", ctypes.c_uint32), ("ns", ctypes.c_uint32),
-                ("nf", ctypes.c_uint32), ("n_routes", ctypes.c_uint32), ("log2_chunk", ctypes.c_uint32),
-                ("name", ctypes.c_void_p), ("name_bytes", ctypes.c_uint32), ("reserved", ctypes.c_uint32)]
+                ("nh", ctypes.c_uint32), ("n_routes", ctypes.c_uint32), ("log2_chunk", ctypes.c_uint32),
+                ("name", ctypes.c_void_p), ("name_bytes", ctypes.c_uint32), ("nib_mode", ctypes.c_uint32)]
 
 
 class _EncItem(ctypes.Structure):
@@ -56,7 +56,7 @@ class _StreamStats(ctypes.Structure):
 
 
 class _EncParams(ctypes.Structure):
-    _fields_ = [(k, ctypes.c_uint32) for k in ("log2_chunk", "ns", "nf", "max_routes", "force_rans")]
+    _fields_ = [(k, ctypes.c_uint32) for k in ("log2_chunk", "ns", "nh", "max_routes", "force_rans")]
 
 
 def _load():
@@ -166,7 +166,7 @@ def _host_bytes(container) -> np.ndarray:
 
 
 def _info_dict(ti: _Info) -> dict:
-    d = {k: getattr(ti, k) for k, _ in _Info._fields_ if k not in ("shape", "name", "name_bytes", "reserved")}
+    d = {k: getattr(ti, k) for k, _ in _Info._fields_ if k not in ("shape", "name", "name_bytes")}
     d["shape"] = tuple(ti.shape[i] for i in range(ti.ndim))
     d["name"] = ctypes.string_at(ti.name, ti.name_bytes).decode() if ti.name_bytes else ""
     return d
@@ -195,7 +195,7 @@ def workspace_bytes(container) -> int:
     return n
 
 
-def encode(tensors, log2_chunk: int = 16, ns: int = 12, nf: int = 10, max_routes: int = 7,
+def encode(tensors, log2_chunk: int = 16, ns: int = 11, nh: int = 5, max_routes: int = 15,
            force_rans: bool = False, host_copy: bool = False, stream=None):
     """Encode device tensors into a container on the device (bs_encoder_*).
 
@@ -225,7 +225,7 @@ def encode(tensors, log2_chunk: int = 16, ns: int = 12, nf: int = 10, max_routes
         it.name_bytes = len(nb)
     if dev is None:
         dev = torch.device("cuda")
-    prm = _EncParams(log2_chunk, ns, nf, max_routes, 1 if force_rans else 0)
+    prm = _EncParams(log2_chunk, ns, nh, max_routes, 1 if force_rans else 0)
     enc = ctypes.c_void_p()
     _check(lib.bs_encoder_create(items, len(tensors), ctypes.byref(prm), ctypes.byref(enc)), "encoder_create")
     try:

@@ -73,10 +73,11 @@ bool quantise(const uint64_t* c, int K, uint32_t M, uint32_t* q) {
     return true;
 }
 
-// FORMAT.md section 6, routes: Pearson's statistic against the uniform fraction
-// distribution, chi2 * n_e = 128 * sum c^2 - n_e^2. Exponents with chi2 > 4096 compete, the
-// largest chi2 (lower exponent on ties) win up to max_routes, numbered in ascending exponent.
-void choose_routes(const uint64_t* cef, uint32_t max_routes, uint8_t* route, std::vector<int>& route_e) {
+// FORMAT.md section 6, routes: Pearson's statistic of the fraction's top three bits against
+// the uniform distribution, chi2 * n_e = 8 * sum c^2 - n_e^2. Exponents with chi2 > 256
+// compete, the largest chi2 (lower exponent on ties) win up to max_routes, numbered in
+// ascending exponent.
+void choose_routes(const uint64_t* ceh, uint32_t max_routes, uint8_t* route, std::vector<int>& route_e) {
     using u128 = unsigned __int128;
     u128 num[256];
     uint64_t ne[256];
@@ -84,13 +85,13 @@ void choose_routes(const uint64_t* cef, uint32_t max_routes, uint8_t* route, std
     for (int e = 0; e < 256; ++e) {
         u128 sq = 0;
         uint64_t n = 0;
-        for (int f = 0; f < 128; ++f) {
-            n += cef[e * 128 + f];
-            sq += u128(cef[e * 128 + f]) * cef[e * 128 + f];
+        for (int h = 0; h < 8; ++h) {
+            n += ceh[e * 8 + h];
+            sq += u128(ceh[e * 8 + h]) * ceh[e * 8 + h];
         }
         ne[e] = n;
-        num[e] = u128(128) * sq - u128(n) * n;
-        cand[e] = n > 0 && num[e] > u128(4096) * n;
+        num[e] = u128(8) * sq - u128(n) * n;
+        cand[e] = n > 0 && num[e] > u128(256) * n;
         taken[e] = false;
         route[e] = 0xFF;
     }
@@ -118,6 +119,7 @@ struct EncTensor {
     bool candidate = false;         // a BF16 tensor with weights: try RANS
     uint64_t n_chunks = 0;
     uint32_t n_routes = 0;
+    uint32_t nib_mode = 0;          // FORMAT.md section 3: 0 = stored, 0x10 + c = constant c
     uint16_t pad_word = 0;
     std::vector<uint8_t> model;     // FORMAT.md 4.3
     std::vector<uint32_t> tables;   // encode tables (bs_internal.h)
@@ -145,34 +147,43 @@ namespace {
 
 // Build the model bytes and the encode tables of one tensor from its histogram.
 bool build_model(EncTensor& T, const bs_enc_params& P, const unsigned long long* hist) {
-    uint64_t cs[512], cef[256 * 128];
+    uint64_t cs[512], ceh[256 * 8];
     for (int s = 0; s < 512; ++s) cs[s] = hist[s];
-    for (int k = 0; k < 256 * 128; ++k) cef[k] = hist[512 + k];
+    for (int k = 0; k < 256 * 8; ++k) ceh[k] = hist[512 + k];
+    const unsigned long long* cnib = hist + 512 + 256 * 8;
     uint32_t Fs[512];
     if (!quantise(cs, 512, 1u << P.ns, Fs)) return false;
     uint8_t route[256];
     std::vector<int> route_e;
-    choose_routes(cef, P.max_routes, route, route_e);
+    choose_routes(ceh, P.max_routes, route, route_e);
     const uint32_t R = static_cast<uint32_t>(route_e.size());
-    std::vector<uint32_t> Ff(128 * R);
+    std::vector<uint32_t> Fh(8 * R);
     for (uint32_t r = 0; r < R; ++r)
-        if (!quantise(cef + 128 * route_e[r], 128, 1u << P.nf, Ff.data() + 128 * r)) return false;
+        if (!quantise(ceh + 8 * route_e[r], 8, 1u << P.nh, Fh.data() + 8 * r)) return false;
     T.n_routes = R;
-    // pad word: most frequent s (lowest on ties), then its table's most frequent fraction
+    // pad word: most frequent s (lowest on ties), then its table's most frequent h
     int s_pad = 0;
     for (int s = 1; s < 512; ++s)
         if (cs[s] > cs[s_pad]) s_pad = s;
-    int f_pad = 0;
+    int h_pad = 0;
     if (route[s_pad & 0xFF] != 0xFF) {
-        const uint32_t* row = Ff.data() + 128 * route[s_pad & 0xFF];
-        for (int f = 1; f < 128; ++f)
-            if (row[f] > row[f_pad]) f_pad = f;
+        const uint32_t* row = Fh.data() + 8 * route[s_pad & 0xFF];
+        for (int h = 1; h < 8; ++h)
+            if (row[h] > row[h_pad]) h_pad = h;
     }
-    T.pad_word = static_cast<uint16_t>((s_pad << 7) | f_pad);
+    T.pad_word = static_cast<uint16_t>((s_pad << 7) | (h_pad << 4));
+    // nibble mode: constant when only one low nibble occurs
+    int seen = 0, only = 0;
+    for (int u = 0; u < 16; ++u)
+        if (cnib[u]) {
+            ++seen;
+            only = u;
+        }
+    T.nib_mode = seen == 1 ? 0x10u | static_cast<uint32_t>(only) : 0u;
     // model bytes (FORMAT.md 4.3)
     uint32_t n_present = 0;
     for (int s = 0; s < 512; ++s) n_present += Fs[s] != 0;
-    T.model.assign(260 + 4ull * n_present + 256ull * R, 0);
+    T.model.assign(260 + 4ull * n_present + 16ull * R, 0);
     uint8_t* m = T.model.data();
     put_u16(m, static_cast<uint16_t>(n_present));
     uint64_t o = 4;
@@ -184,7 +195,7 @@ bool build_model(EncTensor& T, const bs_enc_params& P, const unsigned long long*
         }
     std::memcpy(m + o, route, 256);
     o += 256;
-    for (uint32_t k = 0; k < 128 * R; ++k, o += 2) put_u16(m + o, static_cast<uint16_t>(Ff[k]));
+    for (uint32_t k = 0; k < 8 * R; ++k, o += 2) put_u16(m + o, static_cast<uint16_t>(Fh[k]));
     // encode tables
     T.tables.assign(enc_table_words(R), 0);
     uint32_t cum = 0;
@@ -192,16 +203,16 @@ bool build_model(EncTensor& T, const bs_enc_params& P, const unsigned long long*
         T.tables[s] = Fs[s] | (cum << 16);
         cum += Fs[s];
     }
-    const uint32_t Mf = 1u << P.nf;
+    const uint32_t Mh = 1u << P.nh;
     for (uint32_t r = 0; r <= R; ++r) {
         cum = 0;
-        for (int f = 0; f < 128; ++f) {
-            const uint32_t q = r == R ? Mf / 128 : Ff[128 * r + f];
-            T.tables[512 + 128 * r + f] = q | (cum << 16);
+        for (int h = 0; h < 8; ++h) {
+            const uint32_t q = r == R ? Mh / 8 : Fh[8 * r + h];
+            T.tables[512 + 8 * r + h] = q | (cum << 16);
             cum += q;
         }
     }
-    uint8_t* rt = reinterpret_cast<uint8_t*>(T.tables.data() + 512 + 128 * (R + 1));
+    uint8_t* rt = reinterpret_cast<uint8_t*>(T.tables.data() + 512 + 8 * (R + 1));
     for (int e = 0; e < 256; ++e) rt[e] = route[e] == 0xFF ? static_cast<uint8_t>(R) : route[e];
     return true;
 }
@@ -242,8 +253,9 @@ bs_status run_encode_launches(bs_encoder_t* enc, uint8_t* d_scratch, uint8_t* d_
         it.pad_word = T.pad_word;
         it.log2_chunk = static_cast<uint8_t>(enc->prm.log2_chunk);
         it.ns = static_cast<uint8_t>(enc->prm.ns);
-        it.nf = static_cast<uint8_t>(enc->prm.nf);
+        it.nh = static_cast<uint8_t>(enc->prm.nh);
         it.n_routes = static_cast<uint8_t>(T.n_routes);
+        it.nib_stored = T.nib_mode == 0;
         p->total_ctas += static_cast<uint32_t>(ctas);
     }
     return flush();
@@ -257,8 +269,8 @@ bs_status bs_encoder_create(const bs_enc_item* items, int32_t n, const bs_enc_pa
     if (!out || n < 0 || (n && !items) || !prm) return BS_E_ARG;
     *out = nullptr;
     const bs_enc_params& P = *prm;
-    if (P.log2_chunk < 8 || P.log2_chunk > 24 || P.ns < 1 || P.ns > kMaxNs || P.nf < 7 || P.nf > kMaxNf ||
-        P.max_routes > kMaxRoutes)
+    if (P.log2_chunk < 8 || P.log2_chunk > 24 || P.ns < 1 || P.ns > kMaxNs || P.nh < kMinNh || P.nh > kMaxNh ||
+        P.ns + P.nh > kMaxPrecision || P.max_routes > kMaxRoutes)
         return BS_E_ARG;
     std::unique_ptr<bs_encoder_t> enc(new (std::nothrow) bs_encoder_t);
     if (!enc) return BS_E_NOMEM;
@@ -367,7 +379,9 @@ bs_status bs_encoder_run(bs_encoder_t* enc, void* d_scratch_v, size_t scratch_by
         names_bytes += T.name.size();
         if (!T.candidate) continue;
         T.coded = T.model.size() + 16 * T.n_chunks;
-        for (uint32_t nw : T.n_words) T.coded += up16(256 + 4ull * nw);
+        const uint64_t C = 1ull << P.log2_chunk;
+        for (uint64_t c = 0; c < T.n_chunks; ++c)
+            T.coded += payload_bytes(std::min(C, T.item.n_elems - c * C), T.n_words[c], T.nib_mode == 0);
         T.kind = (!P.force_rans && T.coded >= 2 * T.item.n_elems) ? BS_KIND_STORED : BS_KIND_RANS;
     }
     enc->dir_offset = kHeaderBytes;
@@ -381,9 +395,10 @@ bs_status bs_encoder_run(bs_encoder_t* enc, void* d_scratch_v, size_t scratch_by
             T.data_offset = pos;
             pos = up16(pos + 16 * T.n_chunks);
             T.chunk_off.resize(T.n_chunks);
+            const uint64_t C = 1ull << enc->prm.log2_chunk;
             for (uint64_t c = 0; c < T.n_chunks; ++c) {
                 T.chunk_off[c] = pos;
-                pos += up16(256 + 4ull * T.n_words[c]);
+                pos += payload_bytes(std::min(C, T.item.n_elems - c * C), T.n_words[c], T.nib_mode == 0);
             }
         } else {
             const uint64_t bytes = T.kind == BS_KIND_STORED ? 2 * T.item.n_elems : T.item.n_elems;
@@ -427,7 +442,7 @@ bs_status bs_encoder_emit(bs_encoder_t* enc, void* d_scratch_v, void* d_containe
     std::vector<uint8_t> head(enc->names_offset + enc->names_bytes, 0);
     uint8_t* h = head.data();
     std::memcpy(h, "BF16RANS", 8);
-    put_u32(h + 8, 1);
+    put_u32(h + 8, kFormatVersion);
     put_u32(h + 12, kHeaderBytes);
     put_u32(h + 16, static_cast<uint32_t>(enc->t.size()));
     put_u32(h + 20, kDirEntryBytes);
@@ -454,8 +469,9 @@ bs_status bs_encoder_emit(bs_encoder_t* enc, void* d_scratch_v, void* d_containe
             d[2] = static_cast<uint8_t>(P.log2_chunk);
             d[3] = kLanes;
             d[4] = static_cast<uint8_t>(P.ns);
-            d[5] = static_cast<uint8_t>(P.nf);
+            d[5] = static_cast<uint8_t>(P.nh);
             d[6] = static_cast<uint8_t>(T.n_routes);
+            d[7] = static_cast<uint8_t>(T.nib_mode);
             put_u64(d + 24, T.n_chunks);
             put_u64(d + 32, T.model_offset);
             put_u64(d + 40, T.model.size());

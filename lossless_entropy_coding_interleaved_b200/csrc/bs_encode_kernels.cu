@@ -1,16 +1,17 @@
 // bs_encode_kernels.cu -- sm_100a kernels of the container encoder (FORMAT.md sections 3, 6).
 //
-// histogram_kernel: per-tensor counts of the sign+exponent symbol s = w >> 7 and of
-// (exponent, fraction) pairs. These are the statistics the quantiser and the route rule
-// of FORMAT.md section 6 need. The counts go into per-CTA shared memory, then into global
-// 64-bit bins.
+// histogram_kernel: per-tensor counts of the sign+exponent symbol s = w >> 7, of
+// (exponent, h) pairs (h = the fraction's top three bits) and of the low nibbles. These are
+// the statistics the quantiser, the route rule and the nibble mode of FORMAT.md section 6
+// need. The counts go into per-CTA shared memory, then into global 64-bit bins.
 //
-// encode_kernel: one warp per chunk, lane j holds rANS state j (64-bit). It walks its
-// steps backwards from L = 2^32 as FORMAT.md section 2 specifies. Each weight renormalises
-// at most once, encodes the fraction first and then s. The count pass records how many
-// words each chunk emits. The write pass places the words of step t (lane order) just
-// before those of step t+1, starting from the end of the chunk's word area. That is the
-// interleaved order of FORMAT.md section 3, with no staging buffer.
+// encode_kernel: one warp per chunk, lane j holds rANS state j (32-bit). It walks its
+// steps backwards from L = 2^16 as FORMAT.md section 2 specifies: each weight renormalises
+// at most once (one 16-bit word) and is one step of the product alphabet (s, h). The count
+// pass records how many words each chunk emits. The write pass places the words of step t
+// (lane order) just before those of step t+1, starting from the end of the chunk's word
+// area. That is the interleaved order of FORMAT.md section 3, with no staging buffer. The
+// write pass also stores the nibble words when the tensor keeps them.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -28,7 +29,8 @@ __global__ void __launch_bounds__(512) histogram_kernel(const uint16_t* __restri
     for (uint64_t i = blockIdx.x * static_cast<uint64_t>(blockDim.x) + threadIdx.x; i < n; i += stride) {
         const uint32_t w = in[i];
         atomicAdd(&h[w >> 7], 1u);
-        atomicAdd(&h[512 + (w & 0x7FFFu)], 1u); // ((s & 0xFF) << 7) | f
+        atomicAdd(&h[512 + ((w >> 4) & 0x7FFu)], 1u); // ((s & 0xFF) << 3) | h
+        atomicAdd(&h[512 + 2048 + (w & 15u)], 1u);
     }
     __syncthreads();
     for (uint32_t k = threadIdx.x; k < kHistBins; k += blockDim.x)
@@ -57,7 +59,7 @@ int launch_histogram(const uint16_t* in, uint64_t n, unsigned long long* d_hist,
 
 __global__ void __launch_bounds__(kEncWarps * 32) encode_kernel(const __grid_constant__ EncParams p) {
     __shared__ int s_item;
-    __shared__ uint32_t tab[512 + 128 * 16 + 64];
+    __shared__ uint32_t tab[512 + 8 * 16 + 64];
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
     if (tid == 0) {
         int lo = 0, hi = static_cast<int>(p.n_items) - 1;
@@ -82,18 +84,22 @@ __global__ void __launch_bounds__(kEncWarps * 32) encode_kernel(const __grid_con
     const uint64_t base = chunk << log2c;
     const uint32_t nc = static_cast<uint32_t>(min(C, n - base));
     const uint32_t n_blocks = (nc + 255u) >> 8;
-    const uint32_t ns = it.ns, nf = it.nf, shift = 64 - ns - nf;
+    const uint32_t ns = it.ns, nh = it.nh, P = ns + nh;
     const uint32_t* stab = tab;
-    const uint32_t* frows = tab + 512;
-    const uint8_t* route = reinterpret_cast<const uint8_t*>(tab + 512 + 128 * (it.n_routes + 1));
+    const uint32_t* hrows = tab + 512;
+    const uint8_t* route = reinterpret_cast<const uint8_t*>(tab + 512 + 8 * (it.n_routes + 1));
     const uint16_t* in = it.in + base;
     const uint32_t lt = (1u << lane) - 1u;
 
-    uint64_t x = kStateL;
+    uint32_t x = kStateL;
     uint32_t cnt = 0;                                     // count pass
     uint32_t end = p.write ? it.n_words[chunk] : 0;       // write pass: next free word, from the end
-    uint32_t* words = nullptr;
-    if (p.write) words = reinterpret_cast<uint32_t*>(p.container + it.chunk_off[chunk] + 256);
+    uint8_t* payload = nullptr;
+    uint16_t* words = nullptr;
+    if (p.write) {
+        payload = p.container + it.chunk_off[chunk];
+        words = reinterpret_cast<uint16_t*>(payload + 128 + (it.nib_stored ? 128u * n_blocks : 0u));
+    }
 
     for (uint32_t b = n_blocks; b-- > 0;) {
         const uint32_t i0 = (b << 8) + (lane << 3);
@@ -107,27 +113,34 @@ __global__ void __launch_bounds__(kEncWarps * 32) encode_kernel(const __grid_con
 #pragma unroll
             for (int k = 0; k < 8; ++k) v[k] = (i0 + k < nc) ? in[i0 + k] : it.pad_word;
         }
+        if (p.write && it.nib_stored) { // FORMAT.md section 3: step k's nibble at 4*(k >> 1) + 16*(k & 1)
+            uint32_t nib = 0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) nib |= static_cast<uint32_t>(v[k] & 15u) << (4 * (k >> 1) + 16 * (k & 1));
+            reinterpret_cast<uint32_t*>(payload + 128)[32u * b + lane] = nib;
+        }
 #pragma unroll
         for (int k = 7; k >= 0; --k) {
-            const uint32_t w = v[k], s = w >> 7, e = s & 0xFFu, f = w & 0x7Fu;
-            const uint32_t se = stab[s], fe = frows[route[e] * 128u + f];
-            const uint32_t qs = se & 0xFFFFu, cs = se >> 16, qf = fe & 0xFFFFu, cf = fe >> 16;
-            const bool emit = (x >> shift) >= static_cast<uint64_t>(qs) * qf;
+            const uint32_t w = v[k], s = w >> 7, e = s & 0xFFu, h = (w >> 4) & 7u;
+            const uint32_t se = stab[s], he = hrows[route[e] * 8u + h];
+            const uint32_t qs = se & 0xFFFFu, cs = se >> 16, qh = he & 0xFFFFu, ch = he >> 16;
+            const uint32_t Q = qs * qh;
+            const bool emit = static_cast<uint64_t>(x) >= (static_cast<uint64_t>(Q) << (32 - P));
             if (p.write) {
                 const uint32_t m = __ballot_sync(0xFFFFFFFFu, emit);
                 const uint32_t k_t = __popc(m);
-                if (emit) words[end - k_t + __popc(m & lt)] = static_cast<uint32_t>(x);
+                if (emit) words[end - k_t + __popc(m & lt)] = static_cast<uint16_t>(x);
                 end -= k_t;
             } else {
                 cnt += emit;
             }
-            if (emit) x >>= 32;
-            x = ((x / qf) << nf) + cf + (x % qf);
-            x = ((x / qs) << ns) + cs + (x % qs);
+            if (emit) x >>= 16;
+            const uint32_t r = x % Q;
+            x = ((x / Q) << P) + ((cs + r / qh) << nh) + ch + r % qh;
         }
     }
     if (p.write) {
-        reinterpret_cast<unsigned long long*>(p.container + it.chunk_off[chunk])[lane] = x;
+        reinterpret_cast<uint32_t*>(payload)[lane] = x;
         if (lane == 0 && end != 0) atomicOr(p.err, 1u);
     } else {
 #pragma unroll

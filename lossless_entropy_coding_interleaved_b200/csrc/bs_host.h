@@ -25,8 +25,8 @@ uint64_t workspace_bytes_for(const std::vector<Tensor>& ts);
 // memory per block.
 bs_status build_workspace(std::vector<Tensor>& ts, std::vector<uint8_t>& image);
 
-// Bins decode work by CTA shape (20, 16 or 8 warps) and precision (default ns=12/nf=10,
-// or any), and verbatim copies into one copy list. It launches a bin when the bin is full,
+// Bins decode work by precision (default ns=11/nh=5, or any), and verbatim copies into one
+// copy list. It launches a bin when the bin is full,
 // and launches every bin on flush().
 class DecodeBatch {
   public:
@@ -42,14 +42,13 @@ class DecodeBatch {
   private:
     struct Bin {
         std::unique_ptr<DecodeParams> p;
-        int warps = 0;
         bool default_precision = false;
         uint32_t smem = 0;
     };
     bs_status flush_bin(Bin& b, void* stream);
     bs_status flush_copy(void* stream);
     unsigned long long* err_;
-    Bin bins_[6];
+    Bin bins_[2];
     std::unique_ptr<CopyParams> cp_;
 };
 

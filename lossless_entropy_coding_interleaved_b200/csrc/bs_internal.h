@@ -12,61 +12,71 @@
 
 namespace bs {
 
-// FORMAT.md sections 2-4
+// FORMAT.md sections 2-4 (version 2)
+constexpr uint32_t kFormatVersion = 2;
 constexpr uint32_t kLanes = 32;
-constexpr uint64_t kStateL = 1ull << 32;
+constexpr uint32_t kStateL = 1u << 16;
 constexpr uint32_t kHeaderBytes = 64;
 constexpr uint32_t kDirEntryBytes = 144;
-constexpr uint32_t kMaxNs = 12, kMaxNf = 11, kMaxRoutes = 15;
+constexpr uint32_t kMaxNs = 13, kMinNh = 3, kMaxNh = 5, kMaxPrecision = 16, kMaxRoutes = 15;
+// Bytes of a chunk payload: 32 start states, the nibble words when stored, the 16-bit
+// words, padded to 16 (FORMAT.md section 4.5).
+inline uint64_t payload_bytes(uint64_t n_c, uint32_t n_words, bool nib_stored) {
+    const uint64_t blocks = (n_c + 255) / 256;
+    return (128 + (nib_stored ? 128 * blocks : 0) + 2ull * n_words + 15) & ~uint64_t(15);
+}
 
 // Decode-kernel geometry: a warp decodes kChains chunks at once (two independent state
 // chains per lane), and a CTA of kWarps warps covers kWarps*kChains chunks of one tensor.
-// Each chunk's word stream goes through its own shared-memory ring of kRingWords 32-bit
-// words, in quarters of kRingWords/4 words.
-// Three CTA shapes by table size: 20 warps up to 64 KiB of tables, 16 up to 96 KiB, else 8
-// (the largest tables, 160 KiB, plus 8 warps of rings fit in the 227 KiB a CTA may use).
+// Each chunk's 16-bit word stream goes through its own shared-memory ring of kRingBytes,
+// in quarters of kQuarterBytes (one 16-byte cp.async per lane fills a quarter).
+constexpr int kWarps = 20;
 constexpr int kChains = 2;
-constexpr int kRingWords = 1024;
-constexpr int kQuarterWords = kRingWords / 4;
-// The rings come first in dynamic shared memory, then the tables. The largest tables
-// (160 KiB) plus 8 warps of rings (64 KiB) fit the 227 KiB a CTA may use.
-constexpr uint32_t ring_bytes_per_cta(int warps) { return uint32_t(warps) * kChains * kRingWords * 4; }
-constexpr uint32_t kBigCtaTableBytes = 96 * 1024;
-constexpr uint32_t kHugeCtaTableBytes = 64 * 1024;  // 20 warps: 160 KiB of rings + 64 KiB
-inline int warps_for_tables(uint32_t table_bytes) {
-    return table_bytes <= kHugeCtaTableBytes ? 20 : table_bytes <= kBigCtaTableBytes ? 16 : 8;
-}
+constexpr uint32_t kRingBytes = 2048;
+constexpr uint32_t kQuarterBytes = kRingBytes / 4;
+static_assert(kQuarterBytes == 32 * 16, "one cp.async of 16 bytes per lane fills a quarter");
+// Shared memory of a CTA:
+//   [0, kHRegion)                 fraction rows, one copy per lane (row r, slot j, lane c at
+//                                 byte ((r << nh) + j) * 128 + 4c): conflict-free lookups
+//   [kHRegion, + 8 << ns)         s-table
+//   then the rings, kWarps * kChains * kRingBytes
+// The fraction region is reserved at its largest (16 rows of 2^5 slots) so that the s-table
+// sits at a constant offset. With ns = 13 the total is 128 KiB + 80 KiB of rings.
+constexpr uint32_t kHRegion = 16u * 32u * 128u;
+constexpr uint32_t kRingRegion = uint32_t(kWarps) * kChains * kRingBytes;
+inline uint32_t smem_bytes_for(uint32_t ns) { return kHRegion + (8u << ns) + kRingRegion; }
 
 // Workspace layout: a 256-byte error block, then 256-aligned tables per RANS tensor.
 constexpr uint64_t kErrBlockBytes = 256;
 
 // One tensor of the container as parsed by the planner.
 struct Tensor {
-    uint32_t kind = 0, ndim = 0, log2_chunk = 0, lanes = 0, ns = 0, nf = 0, n_routes = 0;
+    uint32_t kind = 0, ndim = 0, log2_chunk = 0, lanes = 0, ns = 0, nh = 0, n_routes = 0, nib_mode = 0;
     uint64_t n_elems = 0, n_chunks = 0, model_offset = 0, model_bytes = 0, data_offset = 0, data_bytes = 0;
     uint64_t checksum = 0, coded_bytes = 0;
     uint64_t shape[8] = {0};
     std::string name;
     std::vector<uint8_t> model; // RANS: the model section (FORMAT.md 4.3)
     uint64_t ws_offset = 0;   // RANS: byte offset of the decode tables in the workspace
-    uint32_t table_bytes = 0; // RANS: bytes of s-table + f-tables (multiple of 16)
+    uint32_t table_bytes = 0; // RANS: bytes of s-table + compact fraction rows (multiple of 16)
 };
 
 // ---- Decode tables (built on the host, copied to the workspace, staged in smem) ----
-// s-table: 2^ns entries of 8 bytes, indexed by slot = x & (2^ns - 1):
-//   .x = freq | (bias << 16)        freq = Fs[s] (<= 4096), bias = slot - cum_s(s)
-//   .y = (s << 7) | (frow << 16)    s already in its output position; frow locates the
-//                                   f-table row of the route that e = s & 0xFF selects:
-//                                   its byte offset when nf <= 10, its word offset when
-//                                   nf = 11 (see frow_field)
-// f-table: (n_routes + 1) rows of 2^nf u32 entries (the last row is UNIFORM):
-//   bits 0-6 fraction, bits 7-18 freq, bits 19-30 bias
-inline uint32_t table_bytes_for(uint32_t ns, uint32_t nf, uint32_t n_routes) {
-    return (8u << ns) + 4u * (n_routes + 1) * (1u << nf);
+// s-table: 2^ns entries of 8 bytes, indexed by js, the high ns bits of the P-bit slot:
+//   .x = Fs | (bs << 16)            Fs = Fs[s] (<= 8192), bs = js - cum_s(s)
+//   .y = (s << 7) | (frow << 16)    s already in its output position; frow = the byte
+//                                   offset in shared memory of the fraction row that
+//                                   e = s & 0xFF selects: row * (2^nh * 128)
+// fraction rows (compact in the workspace, one copy per lane in shared memory):
+//   (n_routes + 1) rows of 2^nh u32 entries (the last row is UNIFORM), indexed by jh:
+//   bits 4-6 h, bits 16-23 Fh, bits 24-31 bh = jh - cum_h(h); bits 0-3 and 7-15 are zero,
+//   so (s << 7) | (h << 4) is one bitwise select of the two entries
+inline uint32_t table_bytes_for(uint32_t ns, uint32_t nh, uint32_t n_routes) {
+    return (8u << ns) + 4u * (n_routes + 1) * (1u << nh);
 }
-// The frow field of an s-entry for fraction row `row` (it must fit in 16 bits).
-__host__ __device__ inline uint32_t frow_field(uint32_t row, uint32_t nf) {
-    return nf <= 10 ? (row << (nf + 2)) : (row << nf);
+__host__ __device__ inline uint32_t frow_field(uint32_t row, uint32_t nh) { return row << (nh + 7); }
+__host__ __device__ inline uint32_t h_entry(uint32_t h, uint32_t Fh, uint32_t bh) {
+    return (h << 4) | (Fh << 16) | (bh << 24);
 }
 
 // ---- Kernel launch parameters (passed by value, __grid_constant__) ----
@@ -79,8 +89,9 @@ struct DecodeItem {
     uint32_t cta_begin;         // first CTA of this tensor in the launch
     uint32_t tensor_index;      // for error reports
     uint32_t table_bytes;
-    uint8_t log2_chunk, ns, nf, pad0;
-    uint32_t pad1[2];
+    uint8_t log2_chunk, ns, nh, n_routes;
+    uint8_t nib_mode, pad0[3];
+    uint32_t pad1;
 };
 static_assert(sizeof(DecodeItem) == 64, "DecodeItem layout");
 
@@ -110,9 +121,9 @@ struct CopyParams {
 // ---- Encoder (bs_encode.cpp, bs_encode_kernels.cu) ----
 // Encode tables of one tensor, in u32 words:
 //   [0, 512)                s-table: qs | (cum_s << 16)
-//   [512, 512 + 128*rows)   fraction rows (the last one UNIFORM): qf | (cum_f << 16)
+//   [512, 512 + 8*rows)     fraction rows over h (the last one UNIFORM): qh | (cum_h << 16)
 //   [.., + 64)              route: 256 bytes, row index per exponent
-inline uint32_t enc_table_words(uint32_t n_routes) { return 512 + 128 * (n_routes + 1) + 64; }
+inline uint32_t enc_table_words(uint32_t n_routes) { return 512 + 8 * (n_routes + 1) + 64; }
 
 struct EncItem {
     const uint16_t* in;         // device: original words
@@ -123,7 +134,7 @@ struct EncItem {
     uint32_t cta_begin;
     uint32_t table_words;
     uint16_t pad_word;
-    uint8_t log2_chunk, ns, nf, n_routes, pad0, pad1;
+    uint8_t log2_chunk, ns, nh, n_routes, nib_stored, pad1;
 };
 static_assert(sizeof(EncItem) == 56, "EncItem layout");
 
@@ -139,7 +150,7 @@ struct EncParams {
     EncItem item[kMaxEncItems];
 };
 
-constexpr uint32_t kHistBins = 512 + 256 * 128; // s counts, then (exponent, fraction) counts
+constexpr uint32_t kHistBins = 512 + 256 * 8 + 16; // s counts, (exponent, h) counts, low-nibble counts
 int launch_histogram(const uint16_t* in, uint64_t n, unsigned long long* d_hist, void* stream);
 int launch_encode(const EncParams& p, void* stream);
 
@@ -149,7 +160,7 @@ void record_cuda_error(int e);
 void count_launch();
 
 // Kernel launchers (bs_kernels.cu). They return a cudaError_t as int.
-int launch_decode(const DecodeParams& p, int warps, bool default_precision, uint32_t smem_bytes, void* stream);
+int launch_decode(const DecodeParams& p, bool default_precision, uint32_t smem_bytes, void* stream);
 int launch_copy(const CopyParams& p, void* stream);
 int launch_checksum(const void* data, uint64_t n, int raw_bytes, unsigned long long* d_sum, void* stream);
 int max_dynamic_smem();

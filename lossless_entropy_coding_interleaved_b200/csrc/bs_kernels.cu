@@ -4,28 +4,32 @@
 // is the one the "Qwen3.8-27B-BF16-NVLC-Lossless" model card describes in the paragraph
 // after its accounting table:
 //   - the sign+exponent symbol s is decoded with the tensor's rANS model;
-//   - s selects the fraction's distribution and the 7-bit fraction f is decoded with it;
-//   - w = (s << 7) | f is rebuilt bitwise.
-// Layout and parameters: FORMAT.md sections 2-3.
+//   - s selects the fraction's distribution (here over the fraction's top three bits h;
+//     the low four bits u are stored verbatim) and h is decoded with it;
+//   - w = (s << 7) | (h << 4) | u is rebuilt bitwise.
+// Layout and parameters: FORMAT.md (version 2) sections 2-4.
 //
 // Mapping onto the B200:
 //  * One warp decodes two 32-lane chunks at once (two independent dependency chains per
-//    lane hide the latency of the table lookups). Lane j holds rANS state j of each chunk
-//    (64-bit, kept as two 32-bit halves). Under the octet map of FORMAT.md section 3, a
-//    lane owns 8 contiguous output weights per 8 steps. Those leave as one 16-byte store,
-//    so a warp writes 512 contiguous bytes per chunk.
-//  * The tensor's decode tables (s-table 8 B/slot, f-table rows 4 B/slot) are staged once
-//    per CTA in shared memory, at offset 0 so that table addresses fold into constants. A
-//    CTA of 20 warps (tables up to 64 KiB), 16 (up to 96 KiB) or 8 (up to 160 KiB) decodes
-//    40, 32 or 16 chunks of the same tensor; 20 warps x 2 chains is the most that the
-//    register file holds (96 registers per thread).
+//    lane hide the latency of the table lookups). Lane j holds rANS state j of each chunk,
+//    a 32-bit state. Under the octet map of FORMAT.md section 3, a lane owns 8 contiguous
+//    output weights per 8 steps. Those leave as one 16-byte store, so a warp writes 512
+//    contiguous bytes per chunk.
+//  * One weight is one state update: the P-bit slot gives the s-entry (its high ns bits)
+//    and the fraction entry (its low nh bits) at once, and x = Q*(x >> P) + B with
+//    Q = Fs*Fh and B = bs*Fh + bh. No 64-bit arithmetic, no second update.
+//  * The s-table (8 B/entry) is staged in shared memory once per CTA. The fraction rows
+//    are staged with one copy per lane, so lane c always reads bank c: that lookup never
+//    conflicts. The fraction region sits at offset 0 and the s-table at a constant offset,
+//    so table addresses fold into constants.
 //  * Full 256-weight blocks take a path without store bounds; the ragged tail and chunks
 //    of unequal length take a checked path.
-//  * The word stream of a chunk is prefetched into its own shared-memory ring with
-//    cp.async (16 B per lane, in quarters of 256 words), kept 2-3 quarters ahead; the
-//    upkeep runs every 16 steps.
-//  * The default precisions (ns=12, nf=10) get an instantiation with constant shifts.
-//  * Renormalisation reads (at most one 32-bit word per lane per weight) are assigned in
+//  * The 16-bit word stream of a chunk is prefetched into its own 2 KiB shared-memory ring
+//    with cp.async (16 B per lane, in quarters of 512 B), kept 2-3 quarters ahead; the
+//    upkeep runs every 16 steps. The nibble words are loaded one block ahead into
+//    registers (one coalesced 128-byte load per chunk and block).
+//  * The default precisions (ns=11, nh=5) get an instantiation with constant shifts.
+//  * Renormalisation reads (at most one 16-bit word per lane per weight) are assigned in
 //    lane order by ballot + prefix popcount. The words a step consumes are contiguous, so
 //    the ring read is conflict-free.
 //  * No tensor cores: nothing here is a contraction.
@@ -58,36 +62,27 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
-// One chunk in flight on a warp: lane j holds state j as two 32-bit halves.
+// One chunk in flight on a warp: lane j holds state j.
 struct Chain {
-    uint32_t lo, hi;          // rANS state x = hi:lo, in [2^32, 2^64) between weights
+    uint32_t x;               // rANS state, in [2^16, 2^32) between weights
     uint32_t posb;            // bytes of the word stream consumed (warp-uniform)
     uint32_t fq;              // ring quarters requested (warp-uniform)
-    uint32_t total_q, n_words, stream_bytes, nc, n_blocks;
+    uint32_t total_q, stream_bytes, nc, n_blocks;
     uint32_t ring;            // shared-memory address of the ring
-    const uint8_t* ring_ptr;  // the same ring as a pointer into the dynamic smem array
+    uint32_t ring_off;        // the same ring as an offset into the dynamic smem array
+    uint32_t raw;             // nibble word of the current block (constant mode: c in every nibble)
     const uint8_t* stream;
+    const uint32_t* nib;      // nibble words (block-major), or null in constant mode
     uint16_t* out;
     uint64_t chunk;
     bool live;                // a real chunk (false: a filler chain that is never stored)
     bool bad;
 };
 
-// x = freq * (x >> n) + bias on the split state, for 1 <= n <= 31.
-__device__ __forceinline__ void rans_update(uint32_t& lo, uint32_t& hi, uint32_t freq, uint32_t bias, uint32_t n) {
-    const uint32_t t_lo = __funnelshift_r(lo, hi, n);
-    const uint32_t t_hi = hi >> n;
-    const uint64_t p = static_cast<uint64_t>(freq) * t_lo + bias;
-    lo = static_cast<uint32_t>(p);
-    hi = static_cast<uint32_t>(p >> 32) + freq * t_hi;
-}
-
-
-// NS/NF > 0: compile-time precisions (the default container); 0: read from the item.
-template <int WARPS, int NS, int NF>
-__global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
-    // dynamic smem: [s-table][f-rows][rings]; the tables start at offset 0 so that table
-    // addresses are an index times the entry size plus a constant
+// NS/NH > 0: compile-time precisions (the default container); 0: read from the item.
+template <int NS, int NH>
+__global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
+    // dynamic smem: [fraction rows, one copy per lane][s-table][rings]
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ int s_item;
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
@@ -103,12 +98,17 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
     }
     __syncthreads();
     const DecodeItem& it = p.item[s_item];
+    const uint32_t ns = NS > 0 ? NS : it.ns, nh = NH > 0 ? NH : it.nh, P = ns + nh;
 
-    // stage the tables
-    const uint32_t tb = it.table_bytes;
+    // stage the tables: the s-table as it is, each fraction entry once per lane
     {
-        uint4* dst = reinterpret_cast<uint4*>(smem);
-        for (uint32_t k = tid; k < tb / 16u; k += blockDim.x) dst[k] = __ldg(it.tables + k);
+        const uint32_t sb = 8u << ns;
+        uint4* sdst = reinterpret_cast<uint4*>(smem + kHRegion);
+        for (uint32_t k = tid; k < sb / 16u; k += blockDim.x) sdst[k] = __ldg(it.tables + k);
+        const uint32_t* hsrc = reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(it.tables) + sb);
+        uint32_t* hdst = reinterpret_cast<uint32_t*>(smem);
+        const uint32_t hwords = (uint32_t(it.n_routes) + 1u) << (nh + 5);
+        for (uint32_t k = tid; k < hwords; k += blockDim.x) hdst[k] = __ldg(hsrc + (k >> 5));
     }
     __syncthreads();
 
@@ -116,10 +116,12 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
     const uint64_t C = 1ull << log2c;
     const uint64_t n_elems = it.n_elems;
     const uint64_t n_chunks = (n_elems + C - 1) >> log2c;
-    const uint64_t chunk0 = static_cast<uint64_t>(blockIdx.x - it.cta_begin) * (WARPS * kChains) + warp * kChains;
+    const uint64_t chunk0 = static_cast<uint64_t>(blockIdx.x - it.cta_begin) * (kWarps * kChains) + warp * kChains;
     if (chunk0 >= n_chunks) return;
 
-    const uint32_t ring_off = tb + (warp * kChains) * (kRingWords * 4); // this warp's first ring
+    const bool nib_stored = it.nib_mode == 0;
+    const uint32_t raw_const = (it.nib_mode & 15u) * 0x11111111u;
+    const uint32_t ring_off = kHRegion + (8u << ns) + (warp * kChains) * kRingBytes; // this warp's first ring
     const uint32_t ring_base = smem_u32(smem) + ring_off;
     Chain c[kChains];
     uint32_t nb = 0;
@@ -128,46 +130,45 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
         Chain& h = c[k];
         h.chunk = chunk0 + k;
         h.live = h.chunk < n_chunks;
-        h.ring = ring_base + k * (kRingWords * 4);
-        h.ring_ptr = smem + ring_off + k * (kRingWords * 4);
+        h.ring = ring_base + k * kRingBytes;
+        h.ring_off = ring_off + k * kRingBytes;
         h.posb = 0;
         h.fq = 0;
         h.bad = false;
+        h.raw = raw_const;
+        h.nib = nullptr;
         if (h.live) {
             const uint8_t* ent = it.chunk_table + 16 * h.chunk;
             const uint64_t off = __ldg(reinterpret_cast<const unsigned long long*>(ent));
-            h.n_words = __ldg(reinterpret_cast<const unsigned int*>(ent + 8));
+            const uint32_t n_words = __ldg(reinterpret_cast<const unsigned int*>(ent + 8));
             const uint8_t* payload = it.container + off;
-            h.stream = payload + 256;
-            h.stream_bytes = 4u * h.n_words;
-            h.total_q = (h.n_words + kQuarterWords - 1) / kQuarterWords;
             const uint64_t base = h.chunk << log2c;
             h.nc = static_cast<uint32_t>(min(C, n_elems - base));
             h.n_blocks = (h.nc + 255u) >> 8; // blocks of 8 steps
+            if (nib_stored) h.nib = reinterpret_cast<const uint32_t*>(payload + 128);
+            h.stream = payload + 128 + (nib_stored ? 128u * h.n_blocks : 0u);
+            h.stream_bytes = 2u * n_words;
+            h.total_q = (h.stream_bytes + kQuarterBytes - 1) / kQuarterBytes;
             h.out = it.out + base;
-            const uint64_t x = __ldg(reinterpret_cast<const unsigned long long*>(payload) + lane);
-            h.lo = static_cast<uint32_t>(x);
-            h.hi = static_cast<uint32_t>(x >> 32);
-            h.bad = h.hi == 0;
+            h.x = __ldg(reinterpret_cast<const unsigned int*>(payload) + lane);
+            h.bad = h.x < kStateL;
         } else { // filler: decodes from L and its own (unfilled) ring; nothing is stored
-            h.n_words = h.stream_bytes = h.total_q = h.nc = h.n_blocks = 0;
+            h.stream_bytes = h.total_q = h.nc = h.n_blocks = 0;
             h.stream = nullptr;
             h.out = nullptr;
-            h.lo = 0;
-            h.hi = 1;
+            h.x = kStateL;
         }
         nb = max(nb, h.n_blocks);
     }
 
-    const uint32_t ns = NS > 0 ? NS : it.ns, nf = NF > 0 ? NF : it.nf;
-    const uint32_t smask = (1u << ns) - 1u, fmask = (1u << nf) - 1u;
-    const uint8_t* ftab = smem + (8u << ns);
-    const uint32_t lt = lanemask_lt();
+    const uint32_t smask8 = ((1u << ns) - 1u) << 3, hmask7 = ((1u << nh) - 1u) << 7;
+    const uint32_t lt = lanemask_lt(), lane4 = lane << 2;
 
     // Ring upkeep before a block of 16 steps: request up to quarter q+3 for each chain,
-    // where q holds the next word. The next 16 steps need at most quarters q..q+2. Wait for
-    // every copy, or for all but the newest group when those were requested earlier.
-    // Quarters wholly inside the stream skip the per-piece bounds.
+    // where q holds the next word. The next 16 steps need at most quarters q..q+2 (at most
+    // 32 lanes x 16 steps x 2 bytes = 1 KiB). Wait for every copy, or for all but the
+    // newest group when those were requested earlier. Quarters wholly inside the stream
+    // skip the per-piece bounds.
     auto upkeep = [&](uint32_t blk) {
         __syncwarp();
         bool newest_needed = blk == 0;
@@ -175,25 +176,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
         for (int k = 0; k < kChains; ++k) {
             Chain& h = c[k];
             if (blk < h.n_blocks) {
-                const uint32_t q = h.posb / (kQuarterWords * 4u);
+                const uint32_t q = h.posb / kQuarterBytes;
                 if (h.fq <= min(q + 2, h.total_q - 1)) newest_needed = true;
                 while (h.fq < q + 4 && h.fq < h.total_q) {
-                    const uint32_t qb = h.fq * (kQuarterWords * 4u);
-                    if (qb + kQuarterWords * 4u <= h.stream_bytes) {
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const uint32_t byte = qb + 16u * (lane + 32u * e);
-                            cp_async16(h.ring + (byte & (kRingWords * 4u - 1u)), h.stream + byte, 16u);
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const uint32_t byte = qb + 16u * (lane + 32u * e);
-                            if (byte < h.stream_bytes)
-                                cp_async16(h.ring + (byte & (kRingWords * 4u - 1u)), h.stream + byte,
-                                           min(16u, h.stream_bytes - byte));
-                        }
-                    }
+                    const uint32_t byte = h.fq * kQuarterBytes + 16u * lane;
+                    const uint32_t dst = h.ring + (byte & (kRingBytes - 1u));
+                    if ((h.fq + 1) * kQuarterBytes <= h.stream_bytes) cp_async16(dst, h.stream + byte, 16u);
+                    else if (byte < h.stream_bytes) cp_async16(dst, h.stream + byte, min(16u, h.stream_bytes - byte));
                     ++h.fq;
                 }
             }
@@ -204,6 +193,19 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
         __syncwarp();
     };
 
+    // Nibble words: the current block's is in h.raw; the next one is loaded ahead.
+    uint32_t raw_next[kChains];
+#pragma unroll
+    for (int k = 0; k < kChains; ++k) raw_next[k] = (c[k].nib && c[k].n_blocks > 0) ? __ldg(c[k].nib + lane) : raw_const;
+    auto next_raw = [&](uint32_t b) {
+#pragma unroll
+        for (int k = 0; k < kChains; ++k) {
+            Chain& h = c[k];
+            h.raw = raw_next[k];
+            if (h.nib && b + 1 < h.n_blocks) raw_next[k] = __ldg(h.nib + 32u * (b + 1) + lane);
+        }
+    };
+
     // 8 steps of every chain, interleaved; o[k] receives chain k's 8 words as 4 pairs
     auto octet = [&](uint32_t (&o)[kChains][4]) {
 #pragma unroll
@@ -211,29 +213,34 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
 #pragma unroll
             for (int k = 0; k < kChains; ++k) {
                 Chain& h = c[k];
-                // sign+exponent symbol
-                const uint2 se = *reinterpret_cast<const uint2*>(smem + ((h.lo & smask) << 3));
-                rans_update(h.lo, h.hi, se.x & 0xFFFFu, se.x >> 16, ns);
-                // fraction, from the row the symbol's exponent selects (frow_field)
-                const uint32_t fslot = h.lo & fmask;
-                const uint32_t fe = *reinterpret_cast<const uint32_t*>(
-                    ftab + (nf <= 10 ? (se.y >> 16) + (fslot << 2) : ((se.y >> 16) + fslot) << 2));
-                rans_update(h.lo, h.hi, (fe >> 7) & 0xFFFu, fe >> 19, nf);
-                // renormalise: lanes below 2^32 take the next words, in lane order
+                const uint32_t x = h.x;
+                const uint32_t t = x >> P;
+                // the s-entry from the slot's high ns bits, the fraction entry from its low nh bits
+                const uint2 se = *reinterpret_cast<const uint2*>(smem + kHRegion + ((x >> (nh - 3)) & smask8));
+                const uint32_t u = ((x << 7) & hmask7) | lane4;
+                const uint32_t fe = *reinterpret_cast<const uint32_t*>(smem + (se.y >> 16) + u);
+                const uint32_t Fs = se.x & 0xFFFFu, bs = se.x >> 16;
+                const uint32_t Fh = __byte_perm(fe, 0u, 0x4442), bh = fe >> 24;
+                uint32_t xn = (Fs * Fh) * t + (bs * Fh + bh);
+                // renormalise: lanes below 2^16 take the next words, in lane order
                 // (branch-free: every lane reads; the ones that need no word discard it)
-                const bool need = h.hi == 0;
+                const bool need = xn < kStateL;
                 const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
-                const uint32_t w = *reinterpret_cast<const uint32_t*>(
-                    h.ring_ptr + ((h.posb + (__popc(m & lt) << 2)) & (kRingWords * 4u - 1u)));
-                h.hi = need ? h.lo : h.hi;
-                h.lo = need ? w : h.lo;
-                h.posb += __popc(m) << 2;
-                // w = (s << 7) | f: s sits pre-shifted in se.y
-                const uint32_t word = (se.y & 0xFF80u) | (fe & 0x7Fu);
+                const uint32_t w = *reinterpret_cast<const uint16_t*>(
+                    smem + h.ring_off + ((h.posb + (__popc(m & lt) << 1)) & (kRingBytes - 1u)));
+                h.x = need ? ((xn << 16) | w) : xn;
+                h.posb += __popc(m) << 1;
+                // (s << 7) | (h << 4): s sits pre-shifted in se.y, h in bits 4-6 of fe
+                const uint32_t word = (se.y & 0xFF80u) | (fe & 0x70u);
                 if (s & 1) o[k][s >> 1] = __byte_perm(o[k][s >> 1], word, 0x5410);
                 else o[k][s >> 1] = word;
             }
         }
+        // the low nibbles of the pairs (FORMAT.md section 3: pair p at bits 4p and 16+4p)
+#pragma unroll
+        for (int k = 0; k < kChains; ++k)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) o[k][q] |= (c[k].raw >> (4 * q)) & 0x000F000Fu;
     };
 
     // Full blocks first: every live chain has all 256 weights of the block, so the stores
@@ -247,15 +254,16 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
         upkeep(blk);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
+            const uint32_t b = blk + half, i0 = (b << 8) + (lane << 3);
+            next_raw(b);
             uint32_t o[kChains][4];
             octet(o);
-            const uint32_t b = blk + half, i0 = (b << 8) + (lane << 3);
 #pragma unroll
             for (int k = 0; k < kChains; ++k) {
                 Chain& h = c[k];
                 if (h.live) *reinterpret_cast<uint4*>(h.out + i0) = make_uint4(o[k][0], o[k][1], o[k][2], o[k][3]);
                 if (b + 1 == h.n_blocks) // end check: state back at L, every word consumed
-                    h.bad |= (h.lo != 0) | (h.hi != 1) | (h.posb != h.stream_bytes);
+                    h.bad |= (h.x != kStateL) | (h.posb != h.stream_bytes);
             }
         }
     }
@@ -266,6 +274,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
         for (int half = 0; half < 2; ++half) {
             const uint32_t b = blk + half;
             if (b >= nb) break;
+            next_raw(b);
             uint32_t o[kChains][4];
             octet(o);
 #pragma unroll
@@ -281,7 +290,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
                             if (i0 + e < h.nc) h.out[i0 + e] = static_cast<uint16_t>(o[k][e >> 1] >> (16 * (e & 1)));
                     }
                     if (b + 1 == h.n_blocks) // end check: state back at L, every word consumed
-                        h.bad |= (h.lo != 0) | (h.hi != 1) | (h.posb != h.stream_bytes);
+                        h.bad |= (h.x != kStateL) | (h.posb != h.stream_bytes);
                 }
             }
         }
@@ -351,24 +360,20 @@ int max_dynamic_smem() {
     return v;
 }
 
-template <int WARPS, int NS, int NF>
+template <int NS, int NH>
 static int launch_decode_t(const DecodeParams& p, uint32_t smem_bytes, cudaStream_t s) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<WARPS, NS, NF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<NS, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem_bytes));
     if (e != cudaSuccess) return e;
-    decode_kernel<WARPS, NS, NF><<<p.total_ctas, WARPS * 32, smem_bytes, s>>>(p);
+    decode_kernel<NS, NH><<<p.total_ctas, kWarps * 32, smem_bytes, s>>>(p);
     count_launch();
     return cudaGetLastError();
 }
 
-int launch_decode(const DecodeParams& p, int warps, bool default_precision, uint32_t smem_bytes, void* stream) {
+int launch_decode(const DecodeParams& p, bool default_precision, uint32_t smem_bytes, void* stream) {
     if (p.total_ctas == 0) return cudaSuccess;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (warps == 20)
-        return default_precision ? launch_decode_t<20, 12, 10>(p, smem_bytes, s) : launch_decode_t<20, 0, 0>(p, smem_bytes, s);
-    if (warps == 16)
-        return default_precision ? launch_decode_t<16, 12, 10>(p, smem_bytes, s) : launch_decode_t<16, 0, 0>(p, smem_bytes, s);
-    return default_precision ? launch_decode_t<8, 12, 10>(p, smem_bytes, s) : launch_decode_t<8, 0, 0>(p, smem_bytes, s);
+    return default_precision ? launch_decode_t<11, 5>(p, smem_bytes, s) : launch_decode_t<0, 0>(p, smem_bytes, s);
 }
 
 int launch_copy(const CopyParams& p, void* stream) {

@@ -22,9 +22,10 @@
 
 namespace bs {
 
-// Largest decode tables the array holds: 96 KiB covers the default precisions (ns=12,
-// nf=10) with up to 15 fraction routes. Larger tables get BS_E_SIZE.
-constexpr uint32_t kNoAllocTableBytes = 96 * 1024;
+// Largest decode tables the array holds: the s-table at ns = 13 (64 KiB) plus 16 compact
+// fraction rows of 2^5 entries (2 KiB). That is every tensor a valid container can hold;
+// larger tables would get BS_E_SIZE.
+constexpr uint32_t kNoAllocTableBytes = (8u << kMaxNs) + 4u * (kMaxRoutes + 1) * (1u << kMaxNh);
 constexpr uint32_t kNoAllocBytes = 256 + kNoAllocTableBytes; // error block, then tables
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
@@ -72,21 +73,21 @@ bool in_range(uint64_t off, uint64_t n, uint64_t len) { return off <= len && n <
 } // namespace
 
 // Expand a tensor's model (read from the container on the device) into the decode-table
-// layout that decode_kernel stages (bs_internal.h): the s-table, then the fraction rows
-// with the UNIFORM row last. One CTA. It writes into the tables part of the array above.
+// layout that decode_kernel stages (bs_internal.h): the s-table, then the compact fraction
+// rows with the UNIFORM row last. One CTA. It writes into the tables part of the array above.
 // The host validated the model in its own copy. The device copy is read defensively: the
 // caller zeroes the table region first, n_present comes from the host, every write is
 // bounded by its table, and a route index out of range reads as UNIFORM. So the decode
 // kernel's lookups stay inside the tables even if the two copies differ.
 __global__ void __launch_bounds__(512) noalloc_tables_kernel(const uint8_t* model, uint32_t n_present, uint32_t ns,
-                                                             uint32_t nf, uint32_t n_routes) {
+                                                             uint32_t nh, uint32_t n_routes) {
     __shared__ uint32_t s_cum[513];
-    __shared__ uint16_t f_cum[16][129];
+    __shared__ uint16_t h_cum[16][9];
     unsigned char* tab = g_noalloc_scratch + 256;
     const uint8_t* pairs = model + 4;
     const uint8_t* route = model + 4 + 4 * n_present;
     const uint8_t* rows = route + 256;
-    const uint32_t Mf = 1u << nf;
+    const uint32_t Mh = 1u << nh;
     if (threadIdx.x == 0) {
         uint32_t acc = 0;
         for (uint32_t i = 0; i < n_present; ++i) {
@@ -98,11 +99,11 @@ __global__ void __launch_bounds__(512) noalloc_tables_kernel(const uint8_t* mode
     if (threadIdx.x >= 32 && threadIdx.x < 32 + n_routes + 1) {
         const uint32_t r = threadIdx.x - 32;
         uint32_t acc = 0;
-        for (uint32_t f = 0; f < 128; ++f) {
-            f_cum[r][f] = static_cast<uint16_t>(acc);
-            acc += (r == n_routes) ? Mf / 128 : (rows[256 * r + 2 * f] | (rows[256 * r + 2 * f + 1] << 8));
+        for (uint32_t h = 0; h < 8; ++h) {
+            h_cum[r][h] = static_cast<uint16_t>(acc);
+            acc += (r == n_routes) ? Mh / 8 : (rows[16 * r + 2 * h] | (rows[16 * r + 2 * h + 1] << 8));
         }
-        f_cum[r][128] = static_cast<uint16_t>(acc);
+        h_cum[r][8] = static_cast<uint16_t>(acc);
     }
     __syncthreads();
     uint32_t* st = reinterpret_cast<uint32_t*>(tab);
@@ -111,17 +112,17 @@ __global__ void __launch_bounds__(512) noalloc_tables_kernel(const uint8_t* mode
         const uint32_t s = (pairs[4 * i] | (pairs[4 * i + 1] << 8)) & 0x1FFu;
         const uint32_t q = s_cum[i + 1] - s_cum[i];
         const uint8_t r = route[s & 0xFF];
-        const uint32_t fbase = frow_field(r < n_routes ? r : n_routes, nf);
+        const uint32_t frow = frow_field(r < n_routes ? r : n_routes, nh);
         for (uint32_t k = 0; k < q && s_cum[i] + k < Ms; ++k) {
             st[2 * (s_cum[i] + k)] = q | (k << 16);
-            st[2 * (s_cum[i] + k) + 1] = (s << 7) | (fbase << 16);
+            st[2 * (s_cum[i] + k) + 1] = (s << 7) | (frow << 16);
         }
     }
-    uint32_t* ft = reinterpret_cast<uint32_t*>(tab + (8u << ns));
-    for (uint32_t j = threadIdx.x; j < (n_routes + 1) * 128; j += blockDim.x) {
-        const uint32_t r = j >> 7, f = j & 127u;
-        const uint32_t c0 = f_cum[r][f], q = static_cast<uint16_t>(f_cum[r][f + 1] - c0);
-        for (uint32_t k = 0; k < q && c0 + k < Mf; ++k) ft[r * Mf + c0 + k] = f | (q << 7) | (k << 19);
+    uint32_t* ht = reinterpret_cast<uint32_t*>(tab + (8u << ns));
+    for (uint32_t j = threadIdx.x; j < (n_routes + 1) * 8; j += blockDim.x) {
+        const uint32_t r = j >> 3, h = j & 7u;
+        const uint32_t c0 = h_cum[r][h], q = static_cast<uint16_t>(h_cum[r][h + 1] - c0);
+        for (uint32_t k = 0; k < q && c0 + k < Mh; ++k) ht[r * Mh + c0 + k] = h_entry(h, q, k);
     }
 }
 
@@ -138,7 +139,7 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
     if (reinterpret_cast<uintptr_t>(d_container) & 15u) return BS_E_ARG;
     // --- validate the header and this tensor in place (FORMAT.md sections 4-5) ---
     if (len < kHeaderBytes || std::memcmp(b, "BF16RANS", 8) != 0) return BS_E_FORMAT;
-    if (rd32(b + 8) != 1) return BS_E_VERSION;
+    if (rd32(b + 8) != kFormatVersion) return BS_E_VERSION;
     if (rd32(b + 12) != kHeaderBytes || rd32(b + 20) != kDirEntryBytes || rd64(b + 56) != 0) return BS_E_FORMAT;
     if (rd64(b + 48) != len) return BS_E_SIZE;
     const uint32_t nt = rd32(b + 16);
@@ -147,10 +148,12 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
         return BS_E_FORMAT;
     if (static_cast<uint32_t>(idx) >= nt) return BS_E_ARG;
     const uint8_t* d = b + dir + uint64_t(kDirEntryBytes) * idx;
-    const uint32_t kind = d[0], ndim = d[1], log2c = d[2], lanes = d[3], ns = d[4], nf = d[5], n_routes = d[6];
+    const uint32_t kind = d[0], ndim = d[1], log2c = d[2], lanes = d[3], ns = d[4], nh = d[5], n_routes = d[6];
+    const uint32_t nib_mode = d[7];
     const uint64_t n = rd64(d + 16), n_chunks = rd64(d + 24), model_off = rd64(d + 32), model_bytes = rd64(d + 40);
     const uint64_t data_off = rd64(d + 48), data_bytes = rd64(d + 56);
-    if (kind > BS_KIND_RAW || ndim > 8 || d[7] != 0 || rd64(d + 72) != 0) return BS_E_FORMAT;
+    if (kind > BS_KIND_RAW || ndim > 8 || rd64(d + 72) != 0) return BS_E_FORMAT;
+    if (kind != BS_KIND_RANS && nib_mode != 0) return BS_E_FORMAT;
     if (uint64_t(rd32(d + 8)) + rd32(d + 12) > names_bytes) return BS_E_FORMAT;
     unsigned __int128 prod = 1;
     for (uint32_t i = 0; i < 8; ++i) {
@@ -183,14 +186,15 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
         }
         return BS_OK;
     }
-    if (lanes != kLanes || log2c < 8 || log2c > 24 || ns < 1 || ns > kMaxNs || nf < 7 || nf > kMaxNf ||
-        n_routes > kMaxRoutes || n == 0 || n > (1ull << 40))
+    if (lanes != kLanes || log2c < 8 || log2c > 24 || ns < 1 || ns > kMaxNs || nh < kMinNh || nh > kMaxNh ||
+        ns + nh > kMaxPrecision || n_routes > kMaxRoutes || n == 0 || n > (1ull << 40))
         return BS_E_FORMAT;
+    if (nib_mode != 0 && (nib_mode & 0xF0u) != 0x10u) return BS_E_FORMAT;
     if (n_chunks != ((n + (1ull << log2c) - 1) >> log2c) || data_bytes != 16 * n_chunks) return BS_E_FORMAT;
     if (model_off % 16 || !in_range(model_off, model_bytes, len) || model_bytes < 264) return BS_E_FORMAT;
     const uint8_t* m = b + model_off;
     const uint32_t n_present = rd16(m);
-    if (n_present < 1 || n_present > 512 || model_bytes != 260 + 4ull * n_present + 256ull * n_routes)
+    if (n_present < 1 || n_present > 512 || model_bytes != 260 + 4ull * n_present + 16ull * n_routes)
         return BS_E_FORMAT;
     uint64_t sum = 0;
     int prev = -1;
@@ -207,14 +211,17 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
         if (route[e] != 0xFF && route[e] >= n_routes) return BS_E_FORMAT;
     for (uint32_t r = 0; r < n_routes; ++r) {
         sum = 0;
-        for (int f = 0; f < 128; ++f) sum += rd16(route + 256 + 256 * r + 2 * f);
-        if (sum != (1ull << nf)) return BS_E_FORMAT;
+        for (int h = 0; h < 8; ++h) sum += rd16(route + 256 + 16 * r + 2 * h);
+        if (sum != (1ull << nh)) return BS_E_FORMAT;
     }
+    const uint64_t C = 1ull << log2c;
     for (uint64_t c = 0; c < n_chunks; ++c) {
         const uint8_t* e = b + data_off + 16 * c;
-        if (rd64(e) % 16 || !in_range(rd64(e), 256 + 4ull * rd32(e + 8), len)) return BS_E_FORMAT;
+        const uint64_t nc = (n - c * C < C) ? n - c * C : C;
+        if (rd64(e) % 16 || rd32(e + 12) != 0 || !in_range(rd64(e), payload_bytes(nc, rd32(e + 8), nib_mode == 0), len))
+            return BS_E_FORMAT;
     }
-    const uint32_t tb = table_bytes_for(ns, nf, n_routes);
+    const uint32_t tb = table_bytes_for(ns, nh, n_routes);
     if (tb > kNoAllocTableBytes) return BS_E_SIZE; // larger than the static array holds
 
     // --- set-up: the array's device address on this device ---
@@ -232,7 +239,7 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
         record_cuda_error(ce);
         return BS_E_CUDA;
     }
-    noalloc_tables_kernel<<<1, 512, 0, stream>>>(d_container + model_off, n_present, ns, nf, n_routes);
+    noalloc_tables_kernel<<<1, 512, 0, stream>>>(d_container + model_off, n_present, ns, nh, n_routes);
     count_launch();
     ce = cudaGetLastError();
     if (ce != cudaSuccess) {
@@ -242,8 +249,7 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
     // --- the decode kernel, unchanged, with its tables and error block in the array ---
     DecodeParams p; // about 31 KiB of launch parameters, on the stack (no heap use)
     p.n_items = 1;
-    const int warps = warps_for_tables(tb);
-    const uint64_t per_cta = uint64_t(warps) * kChains;
+    const uint64_t per_cta = uint64_t(kWarps) * kChains;
     p.total_ctas = static_cast<uint32_t>((n_chunks + per_cta - 1) / per_cta);
     p.err = reinterpret_cast<unsigned long long*>(scratch);
     DecodeItem& it = p.item[0];
@@ -258,8 +264,10 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
     it.table_bytes = tb;
     it.log2_chunk = static_cast<uint8_t>(log2c);
     it.ns = static_cast<uint8_t>(ns);
-    it.nf = static_cast<uint8_t>(nf);
-    int e = launch_decode(p, warps, ns == 12 && nf == 10, tb + ring_bytes_per_cta(warps), stream);
+    it.nh = static_cast<uint8_t>(nh);
+    it.n_routes = static_cast<uint8_t>(n_routes);
+    it.nib_mode = static_cast<uint8_t>(nib_mode);
+    int e = launch_decode(p, ns == 11 && nh == 5, smem_bytes_for(ns), stream);
     if (e) {
         record_cuda_error(e);
         return BS_E_CUDA;

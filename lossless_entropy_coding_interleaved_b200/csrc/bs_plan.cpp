@@ -90,7 +90,7 @@ bs_status parse(Reader& rd, std::vector<Tensor>& out) {
     if (len < kHeaderBytes || !rd.read(0, kHeaderBytes, hdr)) return fail(BS_E_FORMAT);
     const uint8_t* b = hdr;
     if (std::memcmp(b, "BF16RANS", 8) != 0) return BS_E_FORMAT;
-    if (get_u32(b + 8) != 1) return BS_E_VERSION;
+    if (get_u32(b + 8) != kFormatVersion) return BS_E_VERSION;
     if (get_u32(b + 12) != kHeaderBytes || get_u32(b + 20) != kDirEntryBytes || get_u64(b + 56) != 0)
         return BS_E_FORMAT;
     if (get_u64(b + 48) != len) return BS_E_SIZE;
@@ -116,9 +116,10 @@ bs_status parse(Reader& rd, std::vector<Tensor>& out) {
         t.log2_chunk = d[2];
         t.lanes = d[3];
         t.ns = d[4];
-        t.nf = d[5];
+        t.nh = d[5];
         t.n_routes = d[6];
-        if (d[7] != 0 || get_u64(d + 72) != 0) return BS_E_FORMAT;
+        t.nib_mode = d[7];
+        if (get_u64(d + 72) != 0) return BS_E_FORMAT;
         const uint32_t name_off = get_u32(d + 8), name_len = get_u32(d + 12);
         t.n_elems = get_u64(d + 16);
         t.n_chunks = get_u64(d + 24);
@@ -129,6 +130,7 @@ bs_status parse(Reader& rd, std::vector<Tensor>& out) {
         t.checksum = get_u64(d + 64);
         for (int i = 0; i < 8; ++i) t.shape[i] = get_u64(d + 80 + 8 * i);
         if (t.kind > BS_KIND_RAW || t.ndim > 8) return BS_E_FORMAT;
+        if (t.kind != BS_KIND_RANS && t.nib_mode != 0) return BS_E_FORMAT;
         if (uint64_t(name_off) + name_len > names_bytes) return BS_E_FORMAT;
         t.name.assign(reinterpret_cast<const char*>(nbuf.data() + name_off), name_len);
         unsigned __int128 prod = 1;
@@ -150,19 +152,22 @@ bs_status parse(Reader& rd, std::vector<Tensor>& out) {
         }
         // RANS
         if (t.lanes != kLanes || t.log2_chunk < 8 || t.log2_chunk > 24) return BS_E_FORMAT;
-        if (t.ns < 1 || t.ns > kMaxNs || t.nf < 7 || t.nf > kMaxNf || t.n_routes > kMaxRoutes) return BS_E_FORMAT;
+        if (t.ns < 1 || t.ns > kMaxNs || t.nh < kMinNh || t.nh > kMaxNh || t.ns + t.nh > kMaxPrecision ||
+            t.n_routes > kMaxRoutes)
+            return BS_E_FORMAT;
+        if (t.nib_mode != 0 && (t.nib_mode & 0xF0u) != 0x10u) return BS_E_FORMAT;
         if (t.n_elems == 0 || t.n_elems > (1ull << 40)) return BS_E_FORMAT;
         const uint64_t C = 1ull << t.log2_chunk;
         if (t.n_chunks != (t.n_elems + C - 1) / C || t.data_bytes != 16 * t.n_chunks) return BS_E_FORMAT;
         if (t.model_offset % 16 || !inside(t.model_offset, t.model_bytes, len) || t.model_bytes < 264 ||
-            t.model_bytes > 260 + 4 * 512 + 256 * kMaxRoutes)
+            t.model_bytes > 260 + 4 * 512 + 16 * kMaxRoutes)
             return BS_E_FORMAT;
         t.model.resize(t.model_bytes);
         if (!rd.read(t.model_offset, t.model_bytes, t.model.data())) return fail(BS_E_FORMAT);
         const uint8_t* m = t.model.data();
         const uint32_t n_present = get_u16(m);
         if (n_present < 1 || n_present > 512) return BS_E_FORMAT;
-        if (t.model_bytes != 260 + 4ull * n_present + 256ull * t.n_routes) return BS_E_FORMAT;
+        if (t.model_bytes != 260 + 4ull * n_present + 16ull * t.n_routes) return BS_E_FORMAT;
         uint64_t sum = 0;
         int prev = -1;
         for (uint32_t i = 0; i < n_present; ++i) {
@@ -178,8 +183,8 @@ bs_status parse(Reader& rd, std::vector<Tensor>& out) {
             if (route[e] != 0xFF && route[e] >= t.n_routes) return BS_E_FORMAT;
         for (uint32_t r = 0; r < t.n_routes; ++r) {
             sum = 0;
-            for (int f = 0; f < 128; ++f) sum += get_u16(route + 256 + 256 * r + 2 * f);
-            if (sum != (1ull << t.nf)) return BS_E_FORMAT;
+            for (int h = 0; h < 8; ++h) sum += get_u16(route + 256 + 16 * r + 2 * h);
+            if (sum != (1ull << t.nh)) return BS_E_FORMAT;
         }
         try {
             tbuf.resize(t.data_bytes);
@@ -192,24 +197,27 @@ bs_status parse(Reader& rd, std::vector<Tensor>& out) {
             const uint8_t* e = tbuf.data() + 16 * c;
             const uint64_t off = get_u64(e);
             const uint32_t nw = get_u32(e + 8);
-            if (off % 16 || !inside(off, 256 + 4ull * nw, len)) return BS_E_FORMAT;
-            t.coded_bytes += up16(256 + 4ull * nw);
+            const uint64_t nc = std::min<uint64_t>(C, t.n_elems - c * C);
+            const uint64_t bytes = payload_bytes(nc, nw, t.nib_mode == 0);
+            if (off % 16 || get_u32(e + 12) != 0 || !inside(off, bytes, len)) return BS_E_FORMAT;
+            t.coded_bytes += bytes;
         }
-        t.table_bytes = table_bytes_for(t.ns, t.nf, t.n_routes);
+        t.table_bytes = table_bytes_for(t.ns, t.nh, t.n_routes);
         out.push_back(std::move(t));
     }
     return BS_OK;
 }
 
-// Expand one tensor's model into the decode tables (layout in bs_internal.h).
+// Expand one tensor's model into the decode tables (layout in bs_internal.h): the s-table,
+// then the compact fraction rows with the UNIFORM row last.
 void build_tables(const Tensor& t, uint8_t* dst) {
     const uint8_t* m = t.model.data();
     const uint32_t n_present = get_u16(m);
     const uint8_t* route = m + 4 + 4 * n_present;
-    const uint32_t Mf = 1u << t.nf;
-    auto fbase = [&](uint32_t s) -> uint32_t {
+    const uint32_t Mh = 1u << t.nh;
+    auto frow = [&](uint32_t s) -> uint32_t {
         const uint8_t r = route[s & 0xFF];
-        return frow_field(r == 0xFF ? t.n_routes : r, t.nf);
+        return frow_field(r == 0xFF ? t.n_routes : r, t.nh);
     };
     uint32_t* st = reinterpret_cast<uint32_t*>(dst);
     uint32_t cum = 0;
@@ -217,17 +225,17 @@ void build_tables(const Tensor& t, uint8_t* dst) {
         const uint32_t s = get_u16(m + 4 + 4 * i), q = get_u16(m + 6 + 4 * i);
         for (uint32_t k = 0; k < q; ++k) {
             st[2 * (cum + k)] = q | (k << 16);
-            st[2 * (cum + k) + 1] = (s << 7) | (fbase(s) << 16);
+            st[2 * (cum + k) + 1] = (s << 7) | (frow(s) << 16);
         }
         cum += q;
     }
-    uint32_t* ft = reinterpret_cast<uint32_t*>(dst + (8u << t.ns));
+    uint32_t* ht = reinterpret_cast<uint32_t*>(dst + (8u << t.ns));
     for (uint32_t r = 0; r <= t.n_routes; ++r) {
-        uint32_t* row = ft + r * Mf;
+        uint32_t* row = ht + r * Mh;
         cum = 0;
-        for (uint32_t f = 0; f < 128; ++f) {
-            const uint32_t q = (r == t.n_routes) ? Mf / 128 : get_u16(route + 256 + 256 * r + 2 * f);
-            for (uint32_t k = 0; k < q; ++k) row[cum + k] = f | (q << 7) | (k << 19);
+        for (uint32_t h = 0; h < 8; ++h) {
+            const uint32_t q = (r == t.n_routes) ? Mh / 8 : get_u16(route + 256 + 16 * r + 2 * h);
+            for (uint32_t k = 0; k < q; ++k) row[cum + k] = h_entry(h, q, k);
             cum += q;
         }
     }
@@ -265,8 +273,7 @@ bs_status bs::build_workspace(std::vector<Tensor>& ts, std::vector<uint8_t>& ima
     uint64_t pos = kErrBlockBytes;
     for (Tensor& t : ts) {
         if (t.kind != BS_KIND_RANS) continue;
-        if (static_cast<int>(t.table_bytes + ring_bytes_per_cta(warps_for_tables(t.table_bytes))) > smem_cap)
-            return BS_E_UNSUPPORTED;
+        if (static_cast<int>(smem_bytes_for(t.ns)) > smem_cap) return BS_E_UNSUPPORTED;
         t.ws_offset = pos;
         build_tables(t, image.data() + pos);
         pos += up256(t.table_bytes);
@@ -286,7 +293,8 @@ void bs::fill_tensor_info(const Tensor& t, bs_tensor_info* o) {
     o->kind = t.kind;
     o->ndim = t.ndim;
     o->ns = t.ns;
-    o->nf = t.nf;
+    o->nh = t.nh;
+    o->nib_mode = t.nib_mode;
     o->n_routes = t.n_routes;
     o->log2_chunk = t.log2_chunk;
     o->name = t.name.data();
@@ -294,12 +302,10 @@ void bs::fill_tensor_info(const Tensor& t, bs_tensor_info* o) {
 }
 
 bs_status DecodeBatch::init() {
-    const int shapes[3] = {20, 16, 8};
-    for (int k = 0; k < 6; ++k) {
+    for (int k = 0; k < 2; ++k) {
         bins_[k].p.reset(new (std::nothrow) DecodeParams);
         if (!bins_[k].p) return BS_E_NOMEM;
-        bins_[k].warps = shapes[k / 2];
-        bins_[k].default_precision = k % 2 == 0;
+        bins_[k].default_precision = k == 0;
         bins_[k].p->n_items = 0;
         bins_[k].p->total_ctas = 0;
         bins_[k].p->err = err_;
@@ -313,7 +319,7 @@ bs_status DecodeBatch::init() {
 
 bs_status DecodeBatch::flush_bin(Bin& b, void* stream) {
     if (b.p->n_items == 0) return BS_OK;
-    const int e = launch_decode(*b.p, b.warps, b.default_precision, b.smem, stream);
+    const int e = launch_decode(*b.p, b.default_precision, b.smem, stream);
     b.p->n_items = 0;
     b.p->total_ctas = 0;
     b.smem = 0;
@@ -331,10 +337,9 @@ bs_status DecodeBatch::flush_copy(void* stream) {
 bs_status DecodeBatch::add(const Tensor& t, uint32_t tensor_index, const uint8_t* d_container,
                            const uint8_t* d_ws, void* d_out, void* stream) {
     if (t.kind == BS_KIND_RANS) {
-        const int warps = warps_for_tables(t.table_bytes);
-        const bool dflt = t.ns == 12 && t.nf == 10;
-        Bin& b = bins_[(warps == 20 ? 0 : warps == 16 ? 2 : 4) + (dflt ? 0 : 1)];
-        const uint64_t per_cta = uint64_t(warps) * kChains;
+        const bool dflt = t.ns == 11 && t.nh == 5;
+        Bin& b = bins_[dflt ? 0 : 1];
+        const uint64_t per_cta = uint64_t(kWarps) * kChains;
         const uint64_t ctas = (t.n_chunks + per_cta - 1) / per_cta;
         if (b.p->n_items == kMaxDecodeItems || b.p->total_ctas + ctas > 0x7FFFFFFFull) {
             bs_status s = flush_bin(b, stream);
@@ -352,9 +357,11 @@ bs_status DecodeBatch::add(const Tensor& t, uint32_t tensor_index, const uint8_t
         it.table_bytes = t.table_bytes;
         it.log2_chunk = static_cast<uint8_t>(t.log2_chunk);
         it.ns = static_cast<uint8_t>(t.ns);
-        it.nf = static_cast<uint8_t>(t.nf);
+        it.nh = static_cast<uint8_t>(t.nh);
+        it.n_routes = static_cast<uint8_t>(t.n_routes);
+        it.nib_mode = static_cast<uint8_t>(t.nib_mode);
         b.p->total_ctas += static_cast<uint32_t>(ctas);
-        b.smem = std::max<uint32_t>(b.smem, t.table_bytes + ring_bytes_per_cta(warps));
+        b.smem = std::max<uint32_t>(b.smem, smem_bytes_for(t.ns));
     } else if (t.n_elems) {
         const uint64_t bytes = t.kind == BS_KIND_RAW ? t.n_elems : 2 * t.n_elems;
         const uint64_t blks = (bytes + kCopyBlockBytes - 1) / kCopyBlockBytes;

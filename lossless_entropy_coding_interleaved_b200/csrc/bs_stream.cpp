@@ -96,18 +96,19 @@ struct Group {
 uint64_t out_bytes_of(const Tensor& t) { return t.kind == BS_KIND_RAW ? t.n_elems : 2 * t.n_elems; }
 
 // The container bytes that tensor t's decode reads: [begin, end), begin 16-byte aligned.
-// For RANS: the chunk table and each chunk's states and words (the model is expanded into
-// the workspace at create time and is not read again).
+// For RANS: the chunk table and each chunk's payload: states, nibble words and words (the
+// model is expanded into the workspace at create time and is not read again).
 void coded_range(const Tensor& t, const uint8_t* h, uint64_t* begin, uint64_t* end) {
     uint64_t b = t.data_offset, e = t.data_offset + t.data_bytes;
     if (t.kind == BS_KIND_RANS) {
+        const uint64_t C = 1ull << t.log2_chunk;
         for (uint64_t c = 0; c < t.n_chunks; ++c) {
             uint64_t off;
             uint32_t nw;
             std::memcpy(&off, h + t.data_offset + 16 * c, 8);
             std::memcpy(&nw, h + t.data_offset + 16 * c + 8, 4);
             b = std::min(b, off);
-            e = std::max<uint64_t>(e, off + 256 + 4ull * nw);
+            e = std::max<uint64_t>(e, off + payload_bytes(std::min(C, t.n_elems - c * C), nw, t.nib_mode == 0));
         }
     }
     *begin = b & ~uint64_t(15);

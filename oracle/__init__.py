@@ -7,7 +7,8 @@ two share no code.
 What it computes: the method paragraph of the "Qwen3.8-27B-BF16-NVLC-Lossless" model
 card, which splits each BF16 word into sign, exponent and fraction, codes the
 sign+exponent symbol with a per-tensor rANS model, and lets that symbol select the
-fraction's distribution. The byte layout and every parameter come from FORMAT.md.
+fraction's distribution. The byte layout and every parameter come from FORMAT.md
+(version 2: the fraction's top three bits are coded, its low four bits kept verbatim).
 The arithmetic lives in ``bsoracle.c``. This module only marshals arguments through
 ctypes.
 """
@@ -57,13 +58,13 @@ class _Item(ctypes.Structure):
 
 
 class _Params(ctypes.Structure):
-    _fields_ = [(k, ctypes.c_uint32) for k in ("log2_chunk", "ns", "nf", "max_routes", "force_rans")]
+    _fields_ = [(k, ctypes.c_uint32) for k in ("log2_chunk", "ns", "nh", "max_routes", "force_rans")]
 
 
 class _Info(ctypes.Structure):
     _fields_ = [(k, ctypes.c_uint32) for k in
-                ("kind", "ndim", "log2_chunk", "lanes", "ns", "nf", "n_routes", "name_offset", "name_bytes",
-                 "reserved")] + \
+                ("kind", "ndim", "log2_chunk", "lanes", "ns", "nh", "n_routes", "name_offset", "name_bytes",
+                 "nib_mode")] + \
                [(k, ctypes.c_uint64) for k in
                 ("n_elems", "n_chunks", "model_offset", "model_bytes", "data_offset", "data_bytes", "checksum")] + \
                [("shape", ctypes.c_uint64 * 8), ("coded_bytes", ctypes.c_uint64)]
@@ -87,9 +88,9 @@ def lib():
         L.bso_decode_chunks.argtypes = [P, u64, u32, u64, u64, P, u64, ctypes.POINTER(i64)]
         L.bso_quantise.argtypes = [P, u32, u32, P]
         L.bso_choose_routes.argtypes = [P, u32, P, ctypes.POINTER(u32), P]
-        L.bso_lane_encode.argtypes = [P, u32, P, P, u32, u32, P, u32, ctypes.POINTER(u64), P, P,
+        L.bso_lane_encode.argtypes = [P, u32, P, P, u32, u32, P, u32, ctypes.POINTER(u32), P, P,
                                       ctypes.POINTER(u32)]
-        L.bso_lane_decode.argtypes = [P, u32, P, P, u32, u32, u64, P, u32, u32, P, ctypes.POINTER(u64)]
+        L.bso_lane_decode.argtypes = [P, u32, P, P, u32, u32, u32, P, u32, P, u32, P, ctypes.POINTER(u32)]
         L.bso_mix64.argtypes = [u64]
         L.bso_mix64.restype = u64
         L.bso_checksum.argtypes = [P, u64, u32]
@@ -111,7 +112,7 @@ def _buf(container) -> tuple[np.ndarray, int]:
     return arr, arr.size
 
 
-def encode(items, log2_chunk: int = 16, ns: int = 12, nf: int = 10, max_routes: int = 7,
+def encode(items, log2_chunk: int = 16, ns: int = 11, nh: int = 5, max_routes: int = 15,
            force_rans: bool = False) -> bytes:
     """items: sequence of (name, array, kind) with kind "bf16" (uint16 words, any shape)
     or "raw" (uint8 bytes). Returns the container bytes (FORMAT.md section 4.6)."""
@@ -135,7 +136,7 @@ def encode(items, log2_chunk: int = 16, ns: int = 12, nf: int = 10, max_routes: 
         it.data = _ptr(a)
         it.name = nb
         it.name_bytes = len(nb)
-    p = _Params(log2_chunk, ns, nf, max_routes, 1 if force_rans else 0)
+    p = _Params(log2_chunk, ns, nh, max_routes, 1 if force_rans else 0)
     out = ctypes.c_void_p()
     n = ctypes.c_uint64()
     st = lib().bso_encode(arr_items, len(items), ctypes.byref(p), ctypes.byref(out), ctypes.byref(n))
@@ -201,8 +202,9 @@ def quantise(counts, M: int) -> np.ndarray:
     return q
 
 
-def choose_routes(cef, max_routes: int = 7):
-    c = np.ascontiguousarray(cef, dtype=np.uint64).reshape(256 * 128)
+def choose_routes(ceh, max_routes: int = 15):
+    """ceh: 256 x 8 counts of the fraction's top three bits per exponent."""
+    c = np.ascontiguousarray(ceh, dtype=np.uint64).reshape(256 * 8)
     route = np.zeros(256, dtype=np.uint8)
     route_e = np.zeros(256, dtype=np.uint32)
     nr = ctypes.c_uint32()
@@ -212,37 +214,42 @@ def choose_routes(cef, max_routes: int = 7):
     return route, route_e[: nr.value].copy()
 
 
-def _tables(Fs, route, Ff):
+def _tables(Fs, route, Fh):
     Fs = np.ascontiguousarray(Fs, dtype=np.uint32)
     route = np.ascontiguousarray(route, dtype=np.uint8)
-    Ff = np.ascontiguousarray(Ff, dtype=np.uint32).reshape(-1)
-    assert Fs.size == 512 and route.size == 256 and Ff.size % 128 == 0
-    return Fs, route, Ff if Ff.size else np.zeros(128, np.uint32), Ff.size // 128
+    Fh = np.ascontiguousarray(Fh, dtype=np.uint32).reshape(-1)
+    assert Fs.size == 512 and route.size == 256 and Fh.size % 8 == 0
+    return Fs, route, Fh if Fh.size else np.zeros(8, np.uint32), Fh.size // 8
 
 
-def lane_encode(Fs, ns, route, Ff, nf, words):
-    """One lane (FORMAT.md sections 2-3): returns (start_state, words, tags)."""
-    Fs, route, Ffb, nr = _tables(Fs, route, Ff)
+def lane_encode(Fs, ns, route, Fh, nh, words):
+    """One lane (FORMAT.md sections 2-3): returns (start_state, words, tags). The low
+    nibbles of ``words`` do not enter the state; the caller keeps them."""
+    Fs, route, Fhb, nr = _tables(Fs, route, Fh)
     w = np.ascontiguousarray(words, dtype=np.uint16)
     S = w.size
-    wo = np.zeros(max(S, 1), np.uint32)
+    wo = np.zeros(max(S, 1), np.uint16)
     tg = np.zeros(max(S, 1), np.uint32)
-    st_out = ctypes.c_uint64()
+    st_out = ctypes.c_uint32()
     nw = ctypes.c_uint32()
-    st = lib().bso_lane_encode(_ptr(Fs), ns, _ptr(route), _ptr(Ffb), nr, nf, _ptr(w), S, ctypes.byref(st_out),
+    st = lib().bso_lane_encode(_ptr(Fs), ns, _ptr(route), _ptr(Fhb), nr, nh, _ptr(w), S, ctypes.byref(st_out),
                                _ptr(wo), _ptr(tg), ctypes.byref(nw))
     if st:
         raise OracleError(st, "lane_encode")
     return st_out.value, wo[: nw.value].copy(), tg[: nw.value].copy()
 
 
-def lane_decode(Fs, ns, route, Ff, nf, state, words, S):
-    """Returns (status, decoded words, final state)."""
-    Fs, route, Ffb, nr = _tables(Fs, route, Ff)
-    wd = np.ascontiguousarray(words, dtype=np.uint32)
+def lane_decode(Fs, ns, route, Fh, nh, state, words, nibbles, S):
+    """Returns (status, decoded words, final state). ``nibbles[t]`` is weight t's low nibble."""
+    Fs, route, Fhb, nr = _tables(Fs, route, Fh)
+    wd = np.ascontiguousarray(words, dtype=np.uint16)
+    nb = np.ascontiguousarray(nibbles, dtype=np.uint8)
+    assert nb.size >= S
+    if nb.size == 0:
+        nb = np.zeros(1, np.uint8)
     out = np.zeros(max(S, 1), np.uint16)
-    fin = ctypes.c_uint64()
-    st = lib().bso_lane_decode(_ptr(Fs), ns, _ptr(route), _ptr(Ffb), nr, nf, state, _ptr(wd), wd.size, S,
+    fin = ctypes.c_uint32()
+    st = lib().bso_lane_decode(_ptr(Fs), ns, _ptr(route), _ptr(Fhb), nr, nh, state, _ptr(wd), wd.size, _ptr(nb), S,
                                _ptr(out), ctypes.byref(fin))
     return st, out[:S].copy(), fin.value
 

@@ -8,16 +8,17 @@
  * paragraph after its accounting table:
  *   - each BF16 word is split into its exact sign:1 | exponent:8 | fraction:7 fields;
  *   - the joint sign+exponent symbol is coded with a per-tensor rANS model;
- *   - the decoded symbol selects the distribution for the 7-bit fraction;
+ *   - the decoded symbol selects the distribution for the 7-bit fraction (here: a
+ *     table over the fraction's top three bits, with the low four bits verbatim);
  *   - the fields are recombined bitwise;
  *   - a residual stream keeps non-BF16 bytes verbatim (RAW kind here).
  * The card gives no byte layout, rANS parameters, interleaving or quantiser. Those
- * come from FORMAT.md, and each function says which section it follows.
+ * come from FORMAT.md (version 2), and each function says which section it follows.
  *
  * Pins (tests/test_oracle_*.py):
  *   - round trip on every 16-bit pattern;
  *   - brute force over tiny alphabets;
- *   - the hand-derived container in FORMAT.md section 7;
+ *   - the hand-derived container in FORMAT.md section 8;
  *   - Gibbs' inequality and a stated overhead bound against the empirical entropy;
  *   - closed forms of the quantiser.
  *
@@ -44,7 +45,8 @@ enum { KIND_RANS = 0, KIND_STORED = 1, KIND_RAW = 2 };
 #define LANES 32
 #define HEADER_BYTES 64
 #define DIR_ENTRY_BYTES 144
-#define STATE_L 4294967296ULL /* 2^32, FORMAT.md section 2 */
+#define STATE_L 65536u /* 2^16, FORMAT.md section 2 */
+#define FORMAT_VERSION 2
 
 /* ------------------------------------------------------------------ */
 /* little-endian helpers                                              */
@@ -134,28 +136,30 @@ int bso_quantise(const uint64_t* c, uint32_t K, uint32_t M, uint32_t* q) {
     return BSO_OK;
 }
 
+
 /* ------------------------------------------------------------------ */
 /* Route choice, FORMAT.md section 6                                  */
 /* ------------------------------------------------------------------ */
-/* cef: 256*128 counts, row e = exponent. Writes route[256] and the ascending
- * exponent list route_e[0..n_routes-1]. */
-int bso_choose_routes(const uint64_t* cef, uint32_t max_routes, uint8_t* route, uint32_t* n_routes_out,
+/* ceh: 256*8 counts of the fraction's top three bits, row e = exponent. Writes
+ * route[256] and the ascending exponent list route_e[0..n_routes-1]. */
+int bso_choose_routes(const uint64_t* ceh, uint32_t max_routes, uint8_t* route, uint32_t* n_routes_out,
                       uint32_t* route_e) {
-    unsigned __int128 num[256]; /* chi2_e * n_e = 128*S_e - n_e^2 */
+    unsigned __int128 num[256]; /* chi2_e * n_e = 8*S_e - n_e^2 */
     uint64_t ne[256];
     int cand[256];
+    if (max_routes > 15) return BSO_E_ARG;
     for (int e = 0; e < 256; e++) {
         unsigned __int128 S = 0;
         uint64_t n = 0;
-        for (int f = 0; f < 128; f++) {
-            uint64_t v = cef[e * 128 + f];
+        for (int h = 0; h < 8; h++) {
+            uint64_t v = ceh[e * 8 + h];
             n += v;
             S += (unsigned __int128)v * v;
         }
         ne[e] = n;
-        num[e] = 128 * S - (unsigned __int128)n * n;
-        /* candidate: chi2 > 4096  <=>  128 S - n^2 > 4096 n */
-        cand[e] = (n > 0) && (num[e] > (unsigned __int128)4096 * n);
+        num[e] = 8 * S - (unsigned __int128)n * n;
+        /* candidate: chi2 > 256  <=>  8 S - n^2 > 256 n */
+        cand[e] = (n > 0) && (num[e] > (unsigned __int128)256 * n);
         route[e] = 0xFF;
     }
     /* take candidates by decreasing chi2 (= num/n), ties to lower e */
@@ -182,24 +186,24 @@ int bso_choose_routes(const uint64_t* cef, uint32_t max_routes, uint8_t* route, 
 }
 
 /* ------------------------------------------------------------------ */
-/* Per-tensor model                                                   */
+/* Per-tensor model, FORMAT.md sections 1-2                           */
 /* ------------------------------------------------------------------ */
 typedef struct {
-    uint32_t ns, nf, n_routes;
+    uint32_t ns, nh, n_routes;
     uint32_t Fs[512], cum_s[512];
     uint8_t route[256];
-    uint32_t Ff[16][128], cum_f[16][128]; /* route tables; row index = route */
-    uint32_t Fu, n_present;                 /* UNIFORM frequency = Mf/128 */
+    uint32_t Fh[16][8], cum_h[16][8]; /* route tables over h; row index = route */
+    uint32_t Fu, n_present;           /* UNIFORM frequency = Mh/8 */
     /* decode lookups (slot -> symbol) */
     uint16_t* s_of_slot; /* Ms entries */
-    uint8_t* f_of_slot;  /* (n_routes + 1) * Mf entries, last row = UNIFORM */
+    uint8_t* h_of_slot;  /* (n_routes + 1) * Mh entries, last row = UNIFORM */
 } model_t;
 
 static void model_free(model_t* m) {
     free(m->s_of_slot);
-    free(m->f_of_slot);
+    free(m->h_of_slot);
     m->s_of_slot = NULL;
-    m->f_of_slot = NULL;
+    m->h_of_slot = NULL;
 }
 
 static void model_cums(model_t* m) {
@@ -207,32 +211,32 @@ static void model_cums(model_t* m) {
     for (int s = 0; s < 512; s++) { m->cum_s[s] = acc; acc += m->Fs[s]; }
     for (uint32_t r = 0; r < m->n_routes; r++) {
         acc = 0;
-        for (int f = 0; f < 128; f++) { m->cum_f[r][f] = acc; acc += m->Ff[r][f]; }
+        for (int h = 0; h < 8; h++) { m->cum_h[r][h] = acc; acc += m->Fh[r][h]; }
     }
-    m->Fu = (1u << m->nf) / 128u;
+    m->Fu = (1u << m->nh) / 8u;
 }
 
-/* frequency and cumulative of fraction f under the table that exponent e selects */
-static void frac_model(const model_t* m, uint32_t e, uint32_t f, uint32_t* q, uint32_t* cum) {
+/* frequency and cumulative of top bits h under the table that exponent e selects */
+static void frac_model(const model_t* m, uint32_t e, uint32_t h, uint32_t* q, uint32_t* cum) {
     uint8_t r = m->route[e];
-    if (r == 0xFF) { *q = m->Fu; *cum = m->Fu * f; }
-    else { *q = m->Ff[r][f]; *cum = m->cum_f[r][f]; }
+    if (r == 0xFF) { *q = m->Fu; *cum = m->Fu * h; }
+    else { *q = m->Fh[r][h]; *cum = m->cum_h[r][h]; }
 }
 
 static int model_build_lookups(model_t* m) {
-    uint32_t Ms = 1u << m->ns, Mf = 1u << m->nf;
+    uint32_t Ms = 1u << m->ns, Mh = 1u << m->nh;
     m->s_of_slot = (uint16_t*)malloc(sizeof(uint16_t) * Ms);
-    m->f_of_slot = (uint8_t*)malloc((size_t)(m->n_routes + 1) * Mf);
-    if (!m->s_of_slot || !m->f_of_slot) return BSO_E_NOMEM;
+    m->h_of_slot = (uint8_t*)malloc((size_t)(m->n_routes + 1) * Mh);
+    if (!m->s_of_slot || !m->h_of_slot) return BSO_E_NOMEM;
     for (int s = 0; s < 512; s++)
         for (uint32_t k = 0; k < m->Fs[s]; k++) m->s_of_slot[m->cum_s[s] + k] = (uint16_t)s;
     for (uint32_t r = 0; r <= m->n_routes; r++) {
-        uint8_t* row = m->f_of_slot + (size_t)r * Mf;
-        for (int f = 0; f < 128; f++) {
+        uint8_t* row = m->h_of_slot + (size_t)r * Mh;
+        for (int h = 0; h < 8; h++) {
             uint32_t q, cum;
-            if (r == m->n_routes) { q = m->Fu; cum = m->Fu * (uint32_t)f; }
-            else { q = m->Ff[r][f]; cum = m->cum_f[r][f]; }
-            for (uint32_t k = 0; k < q; k++) row[cum + k] = (uint8_t)f;
+            if (r == m->n_routes) { q = m->Fu; cum = m->Fu * (uint32_t)h; }
+            else { q = m->Fh[r][h]; cum = m->cum_h[r][h]; }
+            for (uint32_t k = 0; k < q; k++) row[cum + k] = (uint8_t)h;
         }
     }
     return BSO_OK;
@@ -241,24 +245,25 @@ static int model_build_lookups(model_t* m) {
 /* ------------------------------------------------------------------ */
 /* One lane, FORMAT.md sections 2-3                                   */
 /* ------------------------------------------------------------------ */
-/* Encode the lane's S weights (given in decode order) backwards from x = L.
+/* Encode the lane's S weights (given in decode order) backwards from x = L. Only the
+ * fields s and h go through the state; the nibbles are stored apart.
  * emitted[t] = 1 and word[t] = the word if the lane emitted while encoding step t. */
-static uint64_t lane_encode(const model_t* m, const uint16_t* w, uint32_t S, uint8_t* emitted, uint32_t* word) {
-    uint64_t x = STATE_L;
-    uint32_t Ms = 1u << m->ns, Mf = 1u << m->nf;
+static uint32_t lane_encode(const model_t* m, const uint16_t* w, uint32_t S, uint8_t* emitted, uint16_t* word) {
+    uint32_t x = STATE_L;
+    uint32_t P = m->ns + m->nh;
     for (uint32_t tt = S; tt-- > 0;) {
-        uint32_t s = w[tt] >> 7, f = w[tt] & 0x7F, e = s & 0xFF;
-        uint32_t qs = m->Fs[s], cs = m->cum_s[s], qf, cf;
-        frac_model(m, e, f, &qf, &cf);
-        uint64_t Q = (uint64_t)qs * qf;
+        uint32_t s = w[tt] >> 7, h = (w[tt] >> 4) & 7u, e = s & 0xFF;
+        uint32_t qs = m->Fs[s], cs = m->cum_s[s], qh, ch;
+        frac_model(m, e, h, &qh, &ch);
+        uint64_t Q = (uint64_t)qs * qh;
         emitted[tt] = 0;
-        if ((x >> (64 - m->ns - m->nf)) >= Q) { /* renormalise: one word at most */
+        if ((uint64_t)x >= (Q << (32 - P))) { /* renormalise: one word at most */
             emitted[tt] = 1;
-            word[tt] = (uint32_t)(x & 0xFFFFFFFFu);
-            x >>= 32;
+            word[tt] = (uint16_t)(x & 0xFFFFu);
+            x >>= 16;
         }
-        x = (x / qf) * Mf + cf + (x % qf); /* fraction first */
-        x = (x / qs) * Ms + cs + (x % qs); /* then the sign+exponent symbol */
+        uint64_t k = x % Q;
+        x = (uint32_t)(((uint64_t)x / Q << P) + ((cs + k / qh) << m->nh) + ch + k % qh);
     }
     return x;
 }
@@ -266,12 +271,12 @@ static uint64_t lane_encode(const model_t* m, const uint16_t* w, uint32_t S, uin
 /* ------------------------------------------------------------------ */
 /* Single-lane entry points for the brute-force pins                  */
 /* ------------------------------------------------------------------ */
-/* Tables are given directly: Fs[512] (sum 2^ns), route[256], Ff[n_routes][128]. */
-static int model_from_tables(model_t* m, const uint32_t* Fs, uint32_t ns, const uint8_t* route, const uint32_t* Ff,
-                             uint32_t n_routes, uint32_t nf) {
+/* Tables are given directly: Fs[512] (sum 2^ns), route[256], Fh[n_routes][8]. */
+static int model_from_tables(model_t* m, const uint32_t* Fs, uint32_t ns, const uint8_t* route, const uint32_t* Fh,
+                             uint32_t n_routes, uint32_t nh) {
     memset(m, 0, sizeof(*m));
-    if (ns < 1 || ns > 12 || nf < 7 || nf > 11 || n_routes > 15) return BSO_E_ARG;
-    m->ns = ns; m->nf = nf; m->n_routes = n_routes;
+    if (ns < 1 || ns > 13 || nh < 3 || nh > 5 || ns + nh > 16 || n_routes > 15) return BSO_E_ARG;
+    m->ns = ns; m->nh = nh; m->n_routes = n_routes;
     uint64_t sum = 0;
     for (int s = 0; s < 512; s++) { m->Fs[s] = Fs[s]; sum += Fs[s]; }
     if (sum != (1u << ns)) return BSO_E_ARG;
@@ -281,28 +286,28 @@ static int model_from_tables(model_t* m, const uint32_t* Fs, uint32_t ns, const 
     }
     for (uint32_t r = 0; r < n_routes; r++) {
         sum = 0;
-        for (int f = 0; f < 128; f++) { m->Ff[r][f] = Ff[r * 128 + f]; sum += Ff[r * 128 + f]; }
-        if (sum != (1u << nf)) return BSO_E_ARG;
+        for (int h = 0; h < 8; h++) { m->Fh[r][h] = Fh[r * 8 + h]; sum += Fh[r * 8 + h]; }
+        if (sum != (1u << nh)) return BSO_E_ARG;
     }
     model_cums(m);
     return BSO_OK;
 }
 
 /* Every word must have a nonzero frequency under the tables. */
-int bso_lane_encode(const uint32_t* Fs, uint32_t ns, const uint8_t* route, const uint32_t* Ff, uint32_t n_routes,
-                    uint32_t nf, const uint16_t* w, uint32_t S, uint64_t* state_out, uint32_t* words_out,
+int bso_lane_encode(const uint32_t* Fs, uint32_t ns, const uint8_t* route, const uint32_t* Fh, uint32_t n_routes,
+                    uint32_t nh, const uint16_t* w, uint32_t S, uint32_t* state_out, uint16_t* words_out,
                     uint32_t* tags_out, uint32_t* n_words_out) {
     model_t* m = (model_t*)calloc(1, sizeof(model_t));
     if (!m) return BSO_E_NOMEM;
-    int st = model_from_tables(m, Fs, ns, route, Ff, n_routes, nf);
+    int st = model_from_tables(m, Fs, ns, route, Fh, n_routes, nh);
     if (st) { free(m); return st; }
     for (uint32_t t = 0; t < S; t++) {
-        uint32_t s = w[t] >> 7, qf, cf;
-        frac_model(m, s & 0xFF, w[t] & 0x7F, &qf, &cf);
-        if (m->Fs[s] == 0 || qf == 0) { free(m); return BSO_E_ARG; }
+        uint32_t s = w[t] >> 7, qh, ch;
+        frac_model(m, s & 0xFF, (w[t] >> 4) & 7u, &qh, &ch);
+        if (m->Fs[s] == 0 || qh == 0) { free(m); return BSO_E_ARG; }
     }
     uint8_t* em = (uint8_t*)malloc(S ? S : 1);
-    uint32_t* wd = (uint32_t*)malloc(sizeof(uint32_t) * (S ? S : 1));
+    uint16_t* wd = (uint16_t*)malloc(sizeof(uint16_t) * (S ? S : 1));
     if (!em || !wd) { free(em); free(wd); free(m); return BSO_E_NOMEM; }
     *state_out = lane_encode(m, w, S, em, wd);
     uint32_t k = 0;
@@ -315,37 +320,37 @@ int bso_lane_encode(const uint32_t* Fs, uint32_t ns, const uint8_t* route, const
     return BSO_OK;
 }
 
-/* Decode S weights of one lane; words are consumed in order. Returns BSO_E_CORRUPT
- * if the end state is not L or the word count does not match. */
-int bso_lane_decode(const uint32_t* Fs, uint32_t ns, const uint8_t* route, const uint32_t* Ff, uint32_t n_routes,
-                    uint32_t nf, uint64_t state, const uint32_t* words, uint32_t n_words, uint32_t S, uint16_t* out,
-                    uint64_t* final_state) {
+/* Decode S weights of one lane; words are consumed in order, nib[t] is the stored low
+ * nibble of weight t. Returns BSO_E_CORRUPT if the end state is not L or the word count
+ * does not match. */
+int bso_lane_decode(const uint32_t* Fs, uint32_t ns, const uint8_t* route, const uint32_t* Fh, uint32_t n_routes,
+                    uint32_t nh, uint32_t state, const uint16_t* words, uint32_t n_words, const uint8_t* nib,
+                    uint32_t S, uint16_t* out, uint32_t* final_state) {
     model_t* mp = (model_t*)calloc(1, sizeof(model_t));
     if (!mp) return BSO_E_NOMEM;
-    int st = model_from_tables(mp, Fs, ns, route, Ff, n_routes, nf);
+    int st = model_from_tables(mp, Fs, ns, route, Fh, n_routes, nh);
     if (st) { free(mp); return st; }
     if ((st = model_build_lookups(mp))) { model_free(mp); free(mp); return st; }
     const model_t* m = mp;
-    uint64_t x = state;
-    uint32_t pos = 0, Ms = 1u << ns, Mf = 1u << nf;
-    int bad = (x >> 32) == 0;
+    uint32_t x = state, P = ns + nh;
+    uint32_t pos = 0, Mh = 1u << nh;
+    int bad = x < STATE_L;
     for (uint32_t t = 0; t < S; t++) {
-        uint32_t slot = (uint32_t)(x & (Ms - 1));
-        uint32_t s = m->s_of_slot[slot];
-        x = (uint64_t)m->Fs[s] * (x >> ns) + slot - m->cum_s[s];
+        uint32_t slot = x & ((1u << P) - 1u);
+        uint32_t js = slot >> nh, jh = slot & (Mh - 1u);
+        uint32_t s = m->s_of_slot[js];
         uint8_t r = m->route[s & 0xFF];
-        uint32_t row = (r == 0xFF) ? m->n_routes : r;
-        slot = (uint32_t)(x & (Mf - 1));
-        uint32_t f = m->f_of_slot[(size_t)row * Mf + slot], qf, cf;
-        frac_model(m, s & 0xFF, f, &qf, &cf);
-        x = (uint64_t)qf * (x >> nf) + slot - cf;
+        uint32_t row = (r == 0xFF) ? m->n_routes : r, qh, ch;
+        uint32_t h = m->h_of_slot[(size_t)row * Mh + jh];
+        frac_model(m, s & 0xFF, h, &qh, &ch);
+        x = m->Fs[s] * qh * (x >> P) + (js - m->cum_s[s]) * qh + (jh - ch);
         if (x < STATE_L) {
             uint32_t wd = 0;
             if (pos < n_words) wd = words[pos]; else bad = 1;
             pos++;
-            x = (x << 32) | wd;
+            x = (x << 16) | wd;
         }
-        out[t] = (uint16_t)((s << 7) | f);
+        out[t] = (uint16_t)((s << 7) | (h << 4) | (nib[t] & 15u));
     }
     *final_state = x;
     model_free(mp);
@@ -366,6 +371,7 @@ typedef struct {
     uint32_t* chunk_words;
     uint64_t coded_total; /* model + 16*n_chunks + sum chunk bytes */
     uint32_t n_routes;
+    uint32_t nib_mode; /* FORMAT.md section 3: 0 = stored, 0x10 + c = constant c */
 } rans_blob_t;
 
 static void blob_free(rans_blob_t* b) {
@@ -381,46 +387,54 @@ static void blob_free(rans_blob_t* b) {
 /* local weight index of (step t, lane j): FORMAT.md section 3 */
 static uint64_t octet_index(uint32_t t, uint32_t j) { return ((uint64_t)(t >> 3) << 8) + 8u * j + (t & 7u); }
 
-static int encode_rans(const uint16_t* w, uint64_t n, uint32_t log2_chunk, uint32_t ns, uint32_t nf,
+/* bit position of the nibble of step t inside its lane's block word: FORMAT.md section 3 */
+static uint32_t nibble_shift(uint32_t t) { return 4u * ((t & 7u) >> 1) + 16u * (t & 1u); }
+
+static int encode_rans(const uint16_t* w, uint64_t n, uint32_t log2_chunk, uint32_t ns, uint32_t nh,
                        uint32_t max_routes, rans_blob_t* out) {
     memset(out, 0, sizeof(*out));
     model_t* m = (model_t*)calloc(1, sizeof(model_t));
     uint64_t* cs = (uint64_t*)calloc(512, sizeof(uint64_t));
-    uint64_t* cef = (uint64_t*)calloc(256 * 128, sizeof(uint64_t));
+    uint64_t* ceh = (uint64_t*)calloc(256 * 8, sizeof(uint64_t));
     int st = BSO_E_NOMEM;
-    if (!m || !cs || !cef) goto done;
-    m->ns = ns; m->nf = nf;
+    if (!m || !cs || !ceh) goto done;
+    m->ns = ns; m->nh = nh;
     /* counts */
     for (uint64_t i = 0; i < n; i++) {
         uint32_t s = w[i] >> 7;
         cs[s]++;
-        cef[(s & 0xFF) * 128 + (w[i] & 0x7F)]++;
+        ceh[(s & 0xFF) * 8 + ((w[i] >> 4) & 7u)]++;
     }
     /* s-model */
     if ((st = bso_quantise(cs, 512, 1u << ns, m->Fs))) goto done;
     /* routes and fraction tables */
     uint32_t route_e[256];
-    if ((st = bso_choose_routes(cef, max_routes, m->route, &m->n_routes, route_e))) goto done;
+    if ((st = bso_choose_routes(ceh, max_routes, m->route, &m->n_routes, route_e))) goto done;
     for (uint32_t r = 0; r < m->n_routes; r++)
-        if ((st = bso_quantise(cef + route_e[r] * 128, 128, 1u << nf, m->Ff[r]))) goto done;
+        if ((st = bso_quantise(ceh + route_e[r] * 8, 8, 1u << nh, m->Fh[r]))) goto done;
     model_cums(m);
     out->n_routes = m->n_routes;
     /* pad word */
     uint32_t s_pad = 0;
     for (uint32_t s = 1; s < 512; s++)
         if (cs[s] > cs[s_pad]) s_pad = s;
-    uint32_t f_pad = 0;
+    uint32_t h_pad = 0;
     if (m->route[s_pad & 0xFF] != 0xFF) {
-        const uint32_t* row = m->Ff[m->route[s_pad & 0xFF]];
-        for (uint32_t f = 1; f < 128; f++)
-            if (row[f] > row[f_pad]) f_pad = f;
+        const uint32_t* row = m->Fh[m->route[s_pad & 0xFF]];
+        for (uint32_t h = 1; h < 8; h++)
+            if (row[h] > row[h_pad]) h_pad = h;
     }
-    uint16_t pad = (uint16_t)((s_pad << 7) | f_pad);
+    uint16_t pad = (uint16_t)((s_pad << 7) | (h_pad << 4));
+    /* nibble mode: constant when every weight has the same low nibble */
+    out->nib_mode = 0x10u | (w[0] & 15u);
+    for (uint64_t i = 1; i < n; i++)
+        if ((w[i] & 15u) != (w[0] & 15u)) { out->nib_mode = 0; break; }
+    const uint32_t nib_stored = out->nib_mode == 0;
 
     /* serialize the model (4.3) */
     uint32_t n_present = 0;
     for (int s = 0; s < 512; s++) if (m->Fs[s]) n_present++;
-    out->model_bytes = 260 + 4ull * n_present + 256ull * m->n_routes;
+    out->model_bytes = 260 + 4ull * n_present + 16ull * m->n_routes;
     out->model = (uint8_t*)calloc(1, out->model_bytes);
     if (!out->model) { st = BSO_E_NOMEM; goto done; }
     wr_u16(out->model, (uint16_t)n_present);
@@ -430,7 +444,7 @@ static int encode_rans(const uint16_t* w, uint64_t n, uint32_t log2_chunk, uint3
     memcpy(out->model + o, m->route, 256);
     o += 256;
     for (uint32_t r = 0; r < m->n_routes; r++)
-        for (int f = 0; f < 128; f++) { wr_u16(out->model + o, (uint16_t)m->Ff[r][f]); o += 2; }
+        for (int h = 0; h < 8; h++) { wr_u16(out->model + o, (uint16_t)m->Fh[r][h]); o += 2; }
 
     /* chunks */
     uint64_t C = 1ull << log2_chunk;
@@ -442,16 +456,18 @@ static int encode_rans(const uint16_t* w, uint64_t n, uint32_t log2_chunk, uint3
     out->coded_total = out->model_bytes + 16 * out->n_chunks;
     for (uint64_t c = 0; c < out->n_chunks; c++) {
         uint64_t base = c * C, nc = (n - base < C) ? n - base : C;
-        uint32_t S = (uint32_t)(8 * ((nc + 255) / 256));
+        uint32_t B = (uint32_t)((nc + 255) / 256), S = 8 * B;
         uint16_t* lw = (uint16_t*)malloc(sizeof(uint16_t) * S);
         uint8_t* em = (uint8_t*)malloc((size_t)LANES * S);
-        uint32_t* wd = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)LANES * S);
-        uint64_t states[LANES];
-        if (!lw || !em || !wd) { free(lw); free(em); free(wd); st = BSO_E_NOMEM; goto done; }
+        uint16_t* wd = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)LANES * S);
+        uint32_t* nib = (uint32_t*)calloc((size_t)LANES * B, sizeof(uint32_t));
+        uint32_t states[LANES];
+        if (!lw || !em || !wd || !nib) { free(lw); free(em); free(wd); free(nib); st = BSO_E_NOMEM; goto done; }
         for (uint32_t j = 0; j < LANES; j++) {
             for (uint32_t t = 0; t < S; t++) {
                 uint64_t i = octet_index(t, j);
                 lw[t] = (i < nc) ? w[base + i] : pad;
+                nib[(size_t)(t >> 3) * LANES + j] |= (uint32_t)(lw[t] & 15u) << nibble_shift(t);
             }
             states[j] = lane_encode(m, lw, S, em + (size_t)j * S, wd + (size_t)j * S);
         }
@@ -459,23 +475,25 @@ static int encode_rans(const uint16_t* w, uint64_t n, uint32_t log2_chunk, uint3
         uint32_t nw = 0;
         for (uint32_t t = 0; t < S; t++)
             for (uint32_t j = 0; j < LANES; j++) nw += em[(size_t)j * S + t];
-        uint64_t bytes = align16(256 + 4ull * nw);
+        uint64_t bytes = align16(128 + 128ull * B * nib_stored + 2ull * nw);
         uint8_t* p = (uint8_t*)calloc(1, bytes);
-        if (!p) { free(lw); free(em); free(wd); st = BSO_E_NOMEM; goto done; }
-        for (uint32_t j = 0; j < LANES; j++) wr_u64(p + 8 * j, states[j]);
-        uint64_t q = 256;
+        if (!p) { free(lw); free(em); free(wd); free(nib); st = BSO_E_NOMEM; goto done; }
+        for (uint32_t j = 0; j < LANES; j++) wr_u32(p + 4 * j, states[j]);
+        if (nib_stored)
+            for (uint64_t k = 0; k < (uint64_t)LANES * B; k++) wr_u32(p + 128 + 4 * k, nib[k]);
+        uint64_t q = 128 + 128ull * B * nib_stored;
         for (uint32_t t = 0; t < S; t++)
             for (uint32_t j = 0; j < LANES; j++)
-                if (em[(size_t)j * S + t]) { wr_u32(p + q, wd[(size_t)j * S + t]); q += 4; }
+                if (em[(size_t)j * S + t]) { wr_u16(p + q, wd[(size_t)j * S + t]); q += 2; }
         out->chunk[c] = p;
         out->chunk_bytes[c] = bytes;
         out->chunk_words[c] = nw;
         out->coded_total += bytes;
-        free(lw); free(em); free(wd);
+        free(lw); free(em); free(wd); free(nib);
     }
     st = BSO_OK;
 done:
-    free(m); free(cs); free(cef);
+    free(m); free(cs); free(ceh);
     if (st) blob_free(out);
     return st;
 }
@@ -495,14 +513,14 @@ typedef struct {
 } bso_item;
 
 typedef struct {
-    uint32_t log2_chunk, ns, nf, max_routes, force_rans;
+    uint32_t log2_chunk, ns, nh, max_routes, force_rans;
 } bso_params;
 
 int bso_encode(const bso_item* items, uint32_t n_items, const bso_params* p, uint8_t** out, uint64_t* out_len) {
     if (!items && n_items) return BSO_E_ARG;
     if (!p || !out || !out_len) return BSO_E_ARG;
-    if (p->log2_chunk < 8 || p->log2_chunk > 24 || p->ns < 1 || p->ns > 12 || p->nf < 7 || p->nf > 11 ||
-        p->max_routes > 15)
+    if (p->log2_chunk < 8 || p->log2_chunk > 24 || p->ns < 1 || p->ns > 13 || p->nh < 3 || p->nh > 5 ||
+        p->ns + p->nh > 16 || p->max_routes > 15)
         return BSO_E_ARG;
     int st = BSO_OK;
     rans_blob_t* blobs = (rans_blob_t*)calloc(n_items ? n_items : 1, sizeof(rans_blob_t));
@@ -519,7 +537,7 @@ int bso_encode(const bso_item* items, uint32_t n_items, const bso_params* p, uin
         if (it->kind == 2) { kinds[k] = KIND_RAW; continue; }
         if (it->n_elems > (1ull << 40)) { st = BSO_E_ARG; goto fail; }
         if (it->n_elems == 0) { kinds[k] = KIND_STORED; continue; }
-        if ((st = encode_rans((const uint16_t*)it->data, it->n_elems, p->log2_chunk, p->ns, p->nf, p->max_routes,
+        if ((st = encode_rans((const uint16_t*)it->data, it->n_elems, p->log2_chunk, p->ns, p->nh, p->max_routes,
                               &blobs[k])))
             goto fail;
         if (!p->force_rans && blobs[k].coded_total >= 2 * it->n_elems) { kinds[k] = KIND_STORED; blob_free(&blobs[k]); }
@@ -551,7 +569,7 @@ int bso_encode(const bso_item* items, uint32_t n_items, const bso_params* p, uin
     uint8_t* buf = (uint8_t*)calloc(1, total);
     if (!buf) { st = BSO_E_NOMEM; goto fail2; }
     memcpy(buf, "BF16RANS", 8);
-    wr_u32(buf + 8, 1);
+    wr_u32(buf + 8, FORMAT_VERSION);
     wr_u32(buf + 12, HEADER_BYTES);
     wr_u32(buf + 16, n_items);
     wr_u32(buf + 20, DIR_ENTRY_BYTES);
@@ -577,8 +595,9 @@ int bso_encode(const bso_item* items, uint32_t n_items, const bso_params* p, uin
             d[2] = (uint8_t)p->log2_chunk;
             d[3] = LANES;
             d[4] = (uint8_t)p->ns;
-            d[5] = (uint8_t)p->nf;
+            d[5] = (uint8_t)p->nh;
             d[6] = (uint8_t)b->n_routes;
+            d[7] = (uint8_t)b->nib_mode;
             wr_u64(d + 24, b->n_chunks);
             wr_u64(d + 32, model_off[k]);
             wr_u64(d + 40, b->model_bytes);
@@ -621,7 +640,7 @@ void bso_free(void* p) { free(p); }
 /* Parser and validation, FORMAT.md sections 4-5                      */
 /* ------------------------------------------------------------------ */
 typedef struct {
-    uint32_t kind, ndim, log2_chunk, lanes, ns, nf, n_routes, name_offset, name_bytes, reserved;
+    uint32_t kind, ndim, log2_chunk, lanes, ns, nh, n_routes, name_offset, name_bytes, nib_mode;
     uint64_t n_elems, n_chunks, model_offset, model_bytes, data_offset, data_bytes, checksum;
     uint64_t shape[8];
     uint64_t coded_bytes; /* RANS: model + chunk table + chunk payloads (padded); else data bytes */
@@ -632,7 +651,7 @@ static int in_bounds(uint64_t off, uint64_t bytes, uint64_t len) { return off <=
 static int parse_header(const uint8_t* b, uint64_t len, uint32_t* n_tensors) {
     if (!b || len < HEADER_BYTES) return BSO_E_FORMAT;
     if (memcmp(b, "BF16RANS", 8) != 0) return BSO_E_FORMAT;
-    if (rd_u32(b + 8) != 1) return BSO_E_VERSION;
+    if (rd_u32(b + 8) != FORMAT_VERSION) return BSO_E_VERSION;
     if (rd_u32(b + 12) != HEADER_BYTES || rd_u32(b + 20) != DIR_ENTRY_BYTES || rd_u64(b + 56) != 0) return BSO_E_FORMAT;
     if (rd_u64(b + 48) != len) return BSO_E_SIZE;
     uint32_t nt = rd_u32(b + 16);
@@ -652,7 +671,7 @@ static int parse_entry(const uint8_t* b, uint64_t len, uint32_t idx, bso_tensor_
     const uint8_t* d = b + rd_u64(b + 24) + (uint64_t)DIR_ENTRY_BYTES * idx;
     memset(ti, 0, sizeof(*ti));
     ti->kind = d[0]; ti->ndim = d[1]; ti->log2_chunk = d[2]; ti->lanes = d[3];
-    ti->ns = d[4]; ti->nf = d[5]; ti->n_routes = d[6];
+    ti->ns = d[4]; ti->nh = d[5]; ti->n_routes = d[6]; ti->nib_mode = d[7];
     ti->name_offset = rd_u32(d + 8); ti->name_bytes = rd_u32(d + 12);
     ti->n_elems = rd_u64(d + 16); ti->n_chunks = rd_u64(d + 24);
     ti->model_offset = rd_u64(d + 32); ti->model_bytes = rd_u64(d + 40);
@@ -660,7 +679,8 @@ static int parse_entry(const uint8_t* b, uint64_t len, uint32_t idx, bso_tensor_
     ti->checksum = rd_u64(d + 64);
     for (int k = 0; k < 8; k++) ti->shape[k] = rd_u64(d + 80 + 8 * k);
     if (ti->ndim > 8 || ti->kind > 2) return BSO_E_FORMAT;
-    if (d[7] != 0 || rd_u64(d + 72) != 0) return BSO_E_FORMAT;
+    if (rd_u64(d + 72) != 0) return BSO_E_FORMAT;
+    if (ti->kind != KIND_RANS && ti->nib_mode != 0) return BSO_E_FORMAT;
     for (uint32_t k = ti->ndim; k < 8; k++)
         if (ti->shape[k] != 0) return BSO_E_FORMAT;
     if ((uint64_t)ti->name_offset + ti->name_bytes > rd_u64(b + 40)) return BSO_E_FORMAT;
@@ -677,7 +697,9 @@ static int parse_entry(const uint8_t* b, uint64_t len, uint32_t idx, bso_tensor_
     }
     /* RANS */
     if (ti->lanes != LANES || ti->log2_chunk < 8 || ti->log2_chunk > 24) return BSO_E_FORMAT;
-    if (ti->ns < 1 || ti->ns > 12 || ti->nf < 7 || ti->nf > 11 || ti->n_routes > 15) return BSO_E_FORMAT;
+    if (ti->ns < 1 || ti->ns > 13 || ti->nh < 3 || ti->nh > 5 || ti->ns + ti->nh > 16 || ti->n_routes > 15)
+        return BSO_E_FORMAT;
+    if (ti->nib_mode != 0 && (ti->nib_mode & 0xF0u) != 0x10u) return BSO_E_FORMAT;
     if (ti->n_elems == 0 || ti->n_elems > (1ull << 40)) return BSO_E_FORMAT;
     uint64_t C = 1ull << ti->log2_chunk;
     if (ti->n_chunks != (ti->n_elems + C - 1) / C || ti->data_bytes != 16 * ti->n_chunks) return BSO_E_FORMAT;
@@ -686,7 +708,7 @@ static int parse_entry(const uint8_t* b, uint64_t len, uint32_t idx, bso_tensor_
     const uint8_t* mm = b + ti->model_offset;
     uint32_t n_present = rd_u16(mm);
     if (n_present < 1 || n_present > 512) return BSO_E_FORMAT;
-    if (ti->model_bytes != 260 + 4ull * n_present + 256ull * ti->n_routes) return BSO_E_FORMAT;
+    if (ti->model_bytes != 260 + 4ull * n_present + 16ull * ti->n_routes) return BSO_E_FORMAT;
     uint64_t sum = 0;
     int prev = -1;
     for (uint32_t k = 0; k < n_present; k++) {
@@ -702,16 +724,18 @@ static int parse_entry(const uint8_t* b, uint64_t len, uint32_t idx, bso_tensor_
         if (route[e] != 0xFF && route[e] >= ti->n_routes) return BSO_E_FORMAT;
     for (uint32_t r = 0; r < ti->n_routes; r++) {
         sum = 0;
-        for (int f = 0; f < 128; f++) sum += rd_u16(route + 256 + 256 * r + 2 * f);
-        if (sum != (1ull << ti->nf)) return BSO_E_FORMAT;
+        for (int h = 0; h < 8; h++) sum += rd_u16(route + 256 + 16 * r + 2 * h);
+        if (sum != (1ull << ti->nh)) return BSO_E_FORMAT;
     }
     ti->coded_bytes = ti->model_bytes + ti->data_bytes;
     for (uint64_t c = 0; c < ti->n_chunks; c++) {
         const uint8_t* e = b + ti->data_offset + 16 * c;
         uint64_t off = rd_u64(e);
         uint32_t nw = rd_u32(e + 8);
-        if (off % 16 || !in_bounds(off, 256 + 4ull * nw, len)) return BSO_E_FORMAT;
-        ti->coded_bytes += align16(256 + 4ull * nw);
+        uint64_t nc = (ti->n_elems - c * C < C) ? ti->n_elems - c * C : C;
+        uint64_t bytes = align16(128 + 128 * ((nc + 255) / 256) * (ti->nib_mode == 0) + 2ull * nw);
+        if (off % 16 || rd_u32(e + 12) != 0 || !in_bounds(off, bytes, len)) return BSO_E_FORMAT;
+        ti->coded_bytes += bytes;
     }
     return BSO_OK;
 }
@@ -735,7 +759,7 @@ int bso_tensor_info_get(const uint8_t* b, uint64_t len, uint32_t idx, bso_tensor
 
 static int load_model(const uint8_t* b, const bso_tensor_info* ti, model_t* m) {
     memset(m, 0, sizeof(*m));
-    m->ns = ti->ns; m->nf = ti->nf; m->n_routes = ti->n_routes;
+    m->ns = ti->ns; m->nh = ti->nh; m->n_routes = ti->n_routes;
     const uint8_t* mm = b + ti->model_offset;
     uint32_t n_present = rd_u16(mm);
     m->n_present = n_present;
@@ -743,7 +767,7 @@ static int load_model(const uint8_t* b, const bso_tensor_info* ti, model_t* m) {
     const uint8_t* route = mm + 4 + 4 * n_present;
     memcpy(m->route, route, 256);
     for (uint32_t r = 0; r < ti->n_routes; r++)
-        for (int f = 0; f < 128; f++) m->Ff[r][f] = rd_u16(route + 256 + 256 * r + 2 * f);
+        for (int h = 0; h < 8; h++) m->Fh[r][h] = rd_u16(route + 256 + 16 * r + 2 * h);
     model_cums(m);
     return model_build_lookups(m);
 }
@@ -759,35 +783,39 @@ static int decode_chunk(const uint8_t* b, const bso_tensor_info* ti, const model
     uint32_t nw = rd_u32(e + 8);
     uint64_t C = 1ull << ti->log2_chunk, base = c * C;
     uint64_t nc = (ti->n_elems - base < C) ? ti->n_elems - base : C;
-    uint32_t S = (uint32_t)(8 * ((nc + 255) / 256));
-    uint32_t Ms = 1u << m->ns, Mf = 1u << m->nf;
-    uint64_t x[LANES];
+    uint32_t B = (uint32_t)((nc + 255) / 256), S = 8 * B;
+    uint32_t P = m->ns + m->nh, Mh = 1u << m->nh;
+    const int nib_stored = ti->nib_mode == 0;
+    const uint8_t* nib = p + 128;
+    const uint8_t* words = p + 128 + 128ull * B * nib_stored;
+    uint32_t x[LANES];
     int bad = 0;
     for (int j = 0; j < LANES; j++) {
-        x[j] = rd_u64(p + 8 * j);
-        if ((x[j] >> 32) == 0) bad = 1;
+        x[j] = rd_u32(p + 4 * j);
+        if (x[j] < STATE_L) bad = 1;
     }
     if (bad) return BSO_E_CORRUPT;
     uint32_t pos = 0;
     for (uint32_t t = 0; t < S; t++) {
         for (uint32_t j = 0; j < LANES; j++) { /* lanes in ascending order take words */
-            uint32_t slot = (uint32_t)(x[j] & (Ms - 1));
-            uint32_t s = m->s_of_slot[slot];
-            x[j] = (uint64_t)m->Fs[s] * (x[j] >> m->ns) + slot - m->cum_s[s];
+            uint32_t slot = x[j] & ((1u << P) - 1u);
+            uint32_t js = slot >> m->nh, jh = slot & (Mh - 1u);
+            uint32_t s = m->s_of_slot[js];
             uint8_t r = m->route[s & 0xFF];
-            uint32_t row = (r == 0xFF) ? m->n_routes : r, qf, cf;
-            slot = (uint32_t)(x[j] & (Mf - 1));
-            uint32_t f = m->f_of_slot[(size_t)row * Mf + slot];
-            frac_model(m, s & 0xFF, f, &qf, &cf);
-            x[j] = (uint64_t)qf * (x[j] >> m->nf) + slot - cf;
+            uint32_t row = (r == 0xFF) ? m->n_routes : r, qh, ch;
+            uint32_t h = m->h_of_slot[(size_t)row * Mh + jh];
+            frac_model(m, s & 0xFF, h, &qh, &ch);
+            x[j] = m->Fs[s] * qh * (x[j] >> P) + (js - m->cum_s[s]) * qh + (jh - ch);
             if (x[j] < STATE_L) {
                 uint32_t wd = 0;
-                if (pos < nw) wd = rd_u32(p + 256 + 4ull * pos); else bad = 1;
+                if (pos < nw) wd = rd_u16(words + 2ull * pos); else bad = 1;
                 pos++;
-                x[j] = (x[j] << 32) | wd;
+                x[j] = (x[j] << 16) | wd;
             }
+            uint32_t u = nib_stored ? (rd_u32(nib + 4ull * ((t >> 3) * LANES + j)) >> nibble_shift(t)) & 15u
+                                    : ti->nib_mode & 15u;
             uint64_t i = octet_index(t, j);
-            if (i < nc) out[base + i] = (uint16_t)((s << 7) | f);
+            if (i < nc) out[base + i] = (uint16_t)((s << 7) | (h << 4) | u);
         }
     }
     for (int j = 0; j < LANES; j++)

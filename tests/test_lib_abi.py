@@ -38,7 +38,11 @@ def test_status_strings_and_workspace_size_on_host():
     w = np.arange(5000, dtype=np.uint16) % 300
     c = oracle.encode([("a", w, "bf16")], force_rans=True)
     n = bs.workspace_bytes(c)
-    assert n >= 256 + (8 << 12) + 4 * 1024
+    # the error block, then the s-table (8 B x 2^ns) and the compact fraction rows
+    # (4 B x 2^nh per route, plus the UNIFORM row), rounded up to 256 bytes
+    ti = oracle.info(c, 0)
+    tables = (8 << ti["ns"]) + 4 * (ti["n_routes"] + 1) * (1 << ti["nh"])
+    assert n == 256 + (tables + 255) // 256 * 256
     with pytest.raises(bs.BsError):
         bs.workspace_bytes(c[:-16])
 

@@ -1,11 +1,13 @@
 """Pins of the oracle against facts that do not come from the oracle itself.
 
-* FORMAT.md section 8: a container derived by hand (tests/golden/one_weight.hex).
+* FORMAT.md section 8: two containers derived by hand (tests/golden/one_weight.hex with
+  constant nibbles, tests/golden/two_weights.hex with stored nibbles).
 * The NVLC model card's field split and bitwise reconstruction: every 16-bit pattern
   round-trips (this covers +-0, subnormals, +-inf and NaN payloads).
 * rANS exactness: brute force over tiny alphabets, where the decode must invert the
   encode and the end state must be L. The code length must equal the model's ideal
-  cost sum(log2(M/q)) plus the 32-bit start state, up to rANS rounding.
+  cost sum(log2(2^P/Q)) plus the 16 bits of the start state L, within the rANS rounding
+  bound of log2(1 + 2^(P-16)) bits per step.
 * The quantiser: closed forms, plus optimality against exhaustive search on small cases.
 * The route rule: the Pearson-statistic threshold at its exact boundary.
 """
@@ -18,7 +20,7 @@ import pytest
 
 import oracle
 
-L = 1 << 32
+L = 1 << 16
 
 
 def _golden_bytes(path):
@@ -30,19 +32,24 @@ def _golden_bytes(path):
 
 
 # ---------------------------------------------------------------- golden container
-def test_golden_one_weight_encode(golden_dir):
-    want = _golden_bytes(os.path.join(golden_dir, "one_weight.hex"))
-    assert len(want) == 896
-    got = oracle.encode([("w", np.array([0x3F80], np.uint16), "bf16")], force_rans=True)
+GOLDEN = [("one_weight.hex", [0x3F80], 704, 0x10), ("two_weights.hex", [0x3F80, 0x3F81], 832, 0x00)]
+
+
+@pytest.mark.parametrize("fname,words,size,nib_mode", GOLDEN)
+def test_golden_encode(golden_dir, fname, words, size, nib_mode):
+    want = _golden_bytes(os.path.join(golden_dir, fname))
+    assert len(want) == size
+    got = oracle.encode([("w", np.array(words, np.uint16), "bf16")], force_rans=True)
     assert got == want
 
 
-def test_golden_one_weight_decode(golden_dir):
-    c = _golden_bytes(os.path.join(golden_dir, "one_weight.hex"))
+@pytest.mark.parametrize("fname,words,size,nib_mode", GOLDEN)
+def test_golden_decode(golden_dir, fname, words, size, nib_mode):
+    c = _golden_bytes(os.path.join(golden_dir, fname))
     assert oracle.validate(c) == 1
     ti = oracle.info(c, 0)
-    assert (ti["kind"], ti["ns"], ti["nf"], ti["n_chunks"], ti["name"]) == (0, 12, 10, 1, "w")
-    assert oracle.decode(c, 0).tolist() == [0x3F80]
+    assert (ti["kind"], ti["ns"], ti["nh"], ti["n_chunks"], ti["name"], ti["nib_mode"]) == (0, 11, 5, 1, "w", nib_mode)
+    assert oracle.decode(c, 0).tolist() == words
 
 
 def test_checksum_published_splitmix64_outputs():
@@ -99,7 +106,7 @@ def test_field_split_closed_form():
 
 
 # ---------------------------------------------------------------- brute force, one lane
-def _tables(fs_dict, ns, route=None, ff=None):
+def _tables(fs_dict, ns, route=None, fh=None):
     Fs = np.zeros(512, np.uint32)
     for k, v in fs_dict.items():
         Fs[k] = v
@@ -108,67 +115,81 @@ def _tables(fs_dict, ns, route=None, ff=None):
     if route:
         for e, idx in route.items():
             r[e] = idx
-    Ff = np.zeros((0, 128), np.uint32) if ff is None else np.asarray(ff, np.uint32)
-    return Fs, r, Ff
+    Fh = np.zeros((0, 8), np.uint32) if fh is None else np.asarray(fh, np.uint32)
+    return Fs, r, Fh
 
 
-def _ideal_bits(words, Fs, ns, route, Ff, nf):
+def _ideal_bits(words, Fs, ns, route, Fh, nh):
+    """sum over weights of log2(2^P / Q), Q = Fs[s] * qh: the model's cost of (s, h)."""
     bits = 0.0
     for w in words:
-        s, f = int(w) >> 7, int(w) & 0x7F
+        s, h = int(w) >> 7, (int(w) >> 4) & 7
         r = int(route[s & 0xFF])
-        qf = (1 << nf) // 128 if r == 0xFF else int(Ff[r][f])
-        bits += ns - math.log2(int(Fs[s])) + nf - math.log2(qf)
+        qh = (1 << nh) // 8 if r == 0xFF else int(Fh[r][h])
+        bits += ns + nh - math.log2(int(Fs[s]) * qh)
     return bits
 
 
 TINY_MODELS = []
-# three s symbols (exponents 1, 2 and the sign-flipped 1), ns = 4
-_ff = np.zeros((1, 128), np.uint32)
-_ff[0, 0], _ff[0, 1], _ff[0, 5] = 100, 27, 1   # sums to 128 = 2^7, a skewed route for e = 2
-TINY_MODELS.append(dict(fs={1: 9, 2: 6, 257: 1}, ns=4, route={2: 0}, ff=_ff, nf=7,
-                        alphabet=[(1 << 7) | 3, (2 << 7) | 1, (257 << 7) | 0]))
-TINY_MODELS.append(dict(fs={1: 1, 2: 1, 3: 2}, ns=2, route=None, ff=None, nf=7,
-                        alphabet=[(1 << 7) | 0, (2 << 7) | 127, (3 << 7) | 64]))
-_ff2 = np.zeros((2, 128), np.uint32)
-_ff2[0, :] = 8            # flat over 128 values, sums to 1024
-_ff2[1, 7], _ff2[1, 9] = 1023, 1
-TINY_MODELS.append(dict(fs={10: 4095, 300: 1}, ns=12, route={10: 0, 300 & 0xFF: 1}, ff=_ff2, nf=10,
-                        alphabet=[(10 << 7) | 7, (300 << 7) | 9, (300 << 7) | 7]))
+# three s symbols (exponents 1, 2 and the sign-flipped 1), ns = 4, nh = 5
+_fh = np.zeros((1, 8), np.uint32)
+_fh[0, 0], _fh[0, 1], _fh[0, 5], _fh[0, 6] = 20, 9, 2, 1   # sums to 32 = 2^5, a skewed route for e = 2
+TINY_MODELS.append(dict(fs={1: 9, 2: 6, 257: 1}, ns=4, route={2: 0}, fh=_fh, nh=5,
+                        alphabet=[(1 << 7) | (3 << 4) | 5, (2 << 7) | (1 << 4) | 9, (257 << 7) | 0]))
+TINY_MODELS.append(dict(fs={1: 1, 2: 1, 3: 2}, ns=2, route=None, fh=None, nh=3,
+                        alphabet=[(1 << 7) | 0, (2 << 7) | (7 << 4) | 15, (3 << 7) | (4 << 4) | 1]))
+# P = 16, the largest precision: one symbol of frequency 1 at ns = 13 and a table with a
+# frequency-1 entry, so Q = 1 costs 16 bits and every step of it emits a word
+_fh2 = np.zeros((2, 8), np.uint32)
+_fh2[0, :] = 1            # flat over the eight values, sums to 8
+_fh2[1, 3], _fh2[1, 7] = 7, 1
+TINY_MODELS.append(dict(fs={10: 8191, 300: 1}, ns=13, route={10: 0, 300 & 0xFF: 1}, fh=_fh2, nh=3,
+                        alphabet=[(10 << 7) | (3 << 4) | 7, (300 << 7) | (3 << 4) | 9, (300 << 7) | (7 << 4)]))
 
 
 @pytest.mark.parametrize("mi", range(len(TINY_MODELS)))
 def test_bruteforce_tiny_alphabets(mi):
     m = TINY_MODELS[mi]
-    Fs, route, Ff = _tables(m["fs"], m["ns"], m["route"], m["ff"])
+    Fs, route, Fh = _tables(m["fs"], m["ns"], m["route"], m["fh"])
     alphabet = m["alphabet"]
+    P = m["ns"] + m["nh"]
     n_seq = 0
     for S in range(0, 9):
         for seq in itertools.product(alphabet, repeat=S):
             words = np.array(seq, np.uint16)
-            x0, wd, tags = oracle.lane_encode(Fs, m["ns"], route, Ff, m["nf"], words)
-            assert L <= x0 < (1 << 64)
+            x0, wd, tags = oracle.lane_encode(Fs, m["ns"], route, Fh, m["nh"], words)
+            assert L <= x0 < (1 << 32)
             assert np.all(np.diff(tags.astype(np.int64)) > 0)   # at most one word per step
-            st, out, fin = oracle.lane_decode(Fs, m["ns"], route, Ff, m["nf"], x0, wd, S)
+            st, out, fin = oracle.lane_decode(Fs, m["ns"], route, Fh, m["nh"], x0, wd, words & 15, S)
             assert st == 0 and fin == L
             assert np.array_equal(out, words)
-            # code length: log2(x0) + 32*n_words = 32 + ideal bits, up to rANS rounding
-            ideal = _ideal_bits(words, Fs, m["ns"], route, Ff, m["nf"])
-            got = math.log2(x0) + 32 * wd.size
-            assert abs(got - 32 - ideal) <= 1e-6 + S * 2 ** -(32 - m["ns"] - m["nf"]) * 2, (seq, got, ideal)
+            # code length: log2(x0) + 16*n_words = 16 + ideal bits, up to rANS rounding
+            ideal = _ideal_bits(words, Fs, m["ns"], route, Fh, m["nh"])
+            got = math.log2(x0) + 16 * wd.size
+            assert abs(got - 16 - ideal) <= 1e-6 + S * math.log2(1 + 2.0 ** (P - 16)), (seq, got, ideal)
             n_seq += 1
     assert n_seq == sum(3 ** k for k in range(9))
 
 
+def test_bruteforce_code_length_is_tight_at_low_precision():
+    # With P = 6 the rounding bound is S*log2(1 + 2^-10): the length must match the model.
+    m = TINY_MODELS[1]
+    Fs, route, Fh = _tables(m["fs"], m["ns"], m["route"], m["fh"])
+    words = np.array(m["alphabet"] * 20, np.uint16)
+    x0, wd, _ = oracle.lane_encode(Fs, m["ns"], route, Fh, m["nh"], words)
+    ideal = _ideal_bits(words, Fs, m["ns"], route, Fh, m["nh"])
+    assert abs(math.log2(x0) + 16 * wd.size - 16 - ideal) < 0.1
+
+
 def test_lane_decode_detects_wrong_state():
     m = TINY_MODELS[0]
-    Fs, route, Ff = _tables(m["fs"], m["ns"], m["route"], m["ff"])
+    Fs, route, Fh = _tables(m["fs"], m["ns"], m["route"], m["fh"])
     words = np.array(m["alphabet"] * 3, np.uint16)
-    x0, wd, _ = oracle.lane_encode(Fs, m["ns"], route, Ff, m["nf"], words)
+    x0, wd, _ = oracle.lane_encode(Fs, m["ns"], route, Fh, m["nh"], words)
     # Decoding is a bijection on (state, words): a different start state either fails the
     # end check or decodes to a different message; it can never reproduce the original.
-    for delta in (1, 2, 3, 1 << 20, 1 << 40):
-        st, out, fin = oracle.lane_decode(Fs, m["ns"], route, Ff, m["nf"], x0 ^ delta, wd, words.size)
+    for delta in (1, 2, 3, 1 << 12, 1 << 20):
+        st, out, fin = oracle.lane_decode(Fs, m["ns"], route, Fh, m["nh"], x0 ^ delta, wd, words & 15, words.size)
         assert st == oracle.E_CORRUPT or not np.array_equal(out, words)
         assert (st == oracle.E_CORRUPT) == (fin != L or st == oracle.E_CORRUPT)
 
@@ -244,29 +265,50 @@ def test_quantise_invariants_random():
 
 
 # ---------------------------------------------------------------- route rule
+def _ceh_with(counts, e=40):
+    ceh = np.zeros((256, 8), np.uint64)
+    ceh[e, : len(counts)] = counts
+    return ceh
+
+
 def test_route_threshold_boundary():
-    # one exponent, n = 128: chi2*n = 128*S - n^2. Counts (1+a, 1-a, 1, ...) give S = 128 + 2a^2.
-    # The threshold is 128*S - n^2 > 4096*n, i.e. 256*a^2 > 4096*128, i.e. a^2 > 2048.
-    def cef_with(counts):
-        cef = np.zeros((256, 128), np.uint64)
-        cef[40, : len(counts)] = counts
-        return cef
-    # a flat 128-count row: chi2 = 0
-    r, re = oracle.choose_routes(cef_with([1] * 128))
+    # chi2*n = 8*S - n^2 over the eight top-bit counts; candidate iff 8*S - n^2 > 256*n.
+    r, re = oracle.choose_routes(_ceh_with([16] * 8))      # flat: chi2 = 0
     assert r[40] == 0xFF and re.size == 0
-    # all mass on one fraction: chi2 = 127*n > 4096 when n > 4096/127
-    r, re = oracle.choose_routes(cef_with([33]))
+    # all mass on one value: 8*n^2 - n^2 = 7*n^2 > 256*n iff n > 36.57
+    r, re = oracle.choose_routes(_ceh_with([37]))
     assert r[40] == 0 and re.tolist() == [40]
-    r, re = oracle.choose_routes(cef_with([32]))          # 127*32 = 4064 < 4096
+    r, re = oracle.choose_routes(_ceh_with([36]))          # 7*36 = 252 < 256
     assert r[40] == 0xFF
+    # exactly on the boundary is not a candidate: n = 64, S = 48^2 + 16^2 = 2560,
+    # 8*2560 - 64^2 = 16384 = 256*64
+    r, _ = oracle.choose_routes(_ceh_with([48, 16]))
+    assert r[40] == 0xFF
+    r, _ = oracle.choose_routes(_ceh_with([49, 15]))       # 8*2626 - 4096 = 16912 > 16384
+    assert r[40] == 0
 
 
 def test_route_ranking_and_limit():
-    cef = np.zeros((256, 128), np.uint64)
+    ceh = np.zeros((256, 8), np.uint64)
     for e, k in ((10, 1000), (20, 3000), (30, 2000)):
-        cef[e, 0] = k            # one-hot rows: chi2 = 127 * n
-    r, re = oracle.choose_routes(cef, max_routes=2)
+        ceh[e, 0] = k            # one-hot rows: chi2 = 7 * n
+    r, re = oracle.choose_routes(ceh, max_routes=2)
     assert re.tolist() == [20, 30]                       # the two largest chi2, in ascending e
     assert r[20] == 0 and r[30] == 1 and r[10] == 0xFF
-    r, re = oracle.choose_routes(cef, max_routes=0)
+    r, re = oracle.choose_routes(ceh, max_routes=0)
     assert re.size == 0
+    with pytest.raises(oracle.OracleError):
+        oracle.choose_routes(ceh, max_routes=16)
+
+
+# ---------------------------------------------------------------- nibble modes
+def test_nibble_modes():
+    # constant low nibble -> no nibble words; any other -> stored, and both round-trip
+    for words, mode in (([0x3F85] * 300, 0x15), ([0x3F80, 0x3F8F] * 150, 0x00)):
+        w = np.array(words, np.uint16)
+        c = oracle.encode([("w", w, "bf16")], force_rans=True)
+        ti = oracle.info(c, 0)
+        assert ti["nib_mode"] == mode
+        assert np.array_equal(oracle.decode(c, 0), w)
+        nib_bytes = 0 if mode else 128 * 2     # n_c = 300 weights -> B = 2 blocks
+        assert ti["coded_bytes"] >= ti["model_bytes"] + 16 + 128 + nib_bytes

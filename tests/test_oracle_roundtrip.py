@@ -51,12 +51,18 @@ def test_chunk_sizes(log2_chunk):
     _roundtrip([("w", w, "bf16")], log2_chunk=log2_chunk)
 
 
-@pytest.mark.parametrize("ns,nf", [(1, 7), (8, 7), (11, 10), (12, 11), (12, 7)])
-def test_precisions(ns, nf):
+@pytest.mark.parametrize("ns,nh", [(1, 3), (8, 3), (8, 5), (11, 5), (12, 4), (13, 3), (11, 3)])
+def test_precisions(ns, nh):
     w = _words(S.workload("tensor_1m")[0]).reshape(-1)[:70_000]
     if ns < 9:   # fewer than 512 slots: keep the alphabet small enough to fit
-        w = np.where(np.arange(w.size) % 2 == 0, 0x3C00, 0xBC01).astype(np.uint16)
-    _roundtrip([("w", w, "bf16")], ns=ns, nf=nf, force_rans=True)
+        w = np.where(np.arange(w.size) % 2 == 0, 0x3C00, 0xBC31).astype(np.uint16)
+    _roundtrip([("w", w, "bf16")], ns=ns, nh=nh, force_rans=True)
+
+
+@pytest.mark.parametrize("ns,nh", [(14, 3), (12, 5), (11, 6), (11, 2), (0, 5)])
+def test_precisions_out_of_range(ns, nh):
+    with pytest.raises(oracle.OracleError):
+        oracle.encode([("w", np.ones(10, np.uint16), "bf16")], ns=ns, nh=nh)
 
 
 def test_edge_mix_roundtrip_and_kinds():
@@ -67,9 +73,11 @@ def test_edge_mix_roundtrip_and_kinds():
     assert kinds["uniform16"] == oracle.KIND_STORED       # incompressible -> stored
     assert kinds["raw_span"] == oracle.KIND_RAW
     assert kinds["t3"] == kinds["outliers"] == kinds["zeros"] == kinds["ones"] == oracle.KIND_RANS
-    # degenerate tensors: only the lane flush remains (32 states + at most a word per step)
+    # degenerate tensors: only the lane flush remains (32 states + at most a word per step);
+    # their nibbles are constant, so no nibble words are stored
     for nm in ("zeros", "ones"):
         ti = oracle.info(arr, [s.name for s in specs].index(nm))
+        assert ti["nib_mode"] == 0x10
         assert ti["coded_bytes"] < 0.02 * 2 * ti["n_elems"]
 
 
@@ -149,11 +157,12 @@ def test_fault_truncation_and_header():
     with pytest.raises(oracle.OracleError) as e:
         oracle.validate(bytes(bad))
     assert e.value.code == oracle.E_FORMAT
-    bad = bytearray(c)
-    bad[8] = 2
-    with pytest.raises(oracle.OracleError) as e:
-        oracle.validate(bytes(bad))
-    assert e.value.code == oracle.E_VERSION
+    for version in (1, 3):           # version 1 (64-bit states) is not read by version-2 decoders
+        bad = bytearray(c)
+        bad[8] = version
+        with pytest.raises(oracle.OracleError) as e:
+            oracle.validate(bytes(bad))
+        assert e.value.code == oracle.E_VERSION
 
 
 def test_fault_table_sum_and_offsets():

@@ -26,15 +26,20 @@ def _u64(h, off):
 
 def _coded_range(h, k):
     """[begin, end) of the bytes tensor k's decode reads, from the FORMAT.md directory and
-    chunk table: the chunk table or raw data, and every chunk's states and words."""
+    chunk table: the chunk table or raw data, and every chunk's payload (section 4.5:
+    128 bytes of states, 128 bytes of nibble words per 256-weight block when stored, the
+    16-bit words, padded to 16 bytes)."""
     e = _u64(h, 24) + 144 * k
     kind, data_off, data_bytes, n_chunks = int(h[e]), _u64(h, e + 48), _u64(h, e + 56), _u64(h, e + 24)
+    n, log2c, nib_stored = _u64(h, e + 16), int(h[e + 2]), int(h[e + 7]) == 0
     b, end = data_off, data_off + data_bytes
     if kind == 0:
         for c in range(n_chunks):
             off = _u64(h, data_off + 16 * c)
             nw = int(h[data_off + 16 * c + 8:data_off + 16 * c + 12].view(np.uint32)[0])
-            b, end = min(b, off), max(end, off + 256 + 4 * nw)
+            nc = min(1 << log2c, n - (c << log2c))
+            size = 128 + (128 * -(-nc // 256) if nib_stored else 0) + 2 * nw
+            b, end = min(b, off), max(end, off + (size + 15) // 16 * 16)
     return b & ~15, end
 
 
