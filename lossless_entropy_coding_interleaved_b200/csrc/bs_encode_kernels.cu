@@ -129,8 +129,13 @@ __global__ void __launch_bounds__(kEncWarps * 32) encode_kernel(const __grid_con
             if (p.write) {
                 const uint32_t m = __ballot_sync(0xFFFFFFFFu, emit);
                 const uint32_t k_t = __popc(m);
-                if (emit) words[end - k_t + __popc(m & lt)] = static_cast<uint16_t>(x);
-                end -= k_t;
+                if (k_t <= end) {
+                    if (emit) words[end - k_t + __popc(m & lt)] = static_cast<uint16_t>(x);
+                    end -= k_t;
+                } else { // more words than the count pass saw: report, never write out of range
+                    if (lane == 0) atomicOr(p.err, 1u);
+                    end = 0;
+                }
             } else {
                 cnt += emit;
             }

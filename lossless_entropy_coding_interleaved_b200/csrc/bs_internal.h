@@ -18,7 +18,7 @@ constexpr uint32_t kLanes = 32;
 constexpr uint32_t kStateL = 1u << 16;
 constexpr uint32_t kHeaderBytes = 64;
 constexpr uint32_t kDirEntryBytes = 144;
-constexpr uint32_t kMaxNs = 13, kMinNh = 3, kMaxNh = 5, kMaxPrecision = 16, kMaxRoutes = 15;
+constexpr uint32_t kMaxNs = 12, kMinNh = 3, kMaxNh = 5, kMaxPrecision = 16, kMaxRoutes = 15;
 // Bytes of a chunk payload: 32 start states, the nibble words when stored, the 16-bit
 // words, padded to 16 (FORMAT.md section 4.5).
 inline uint64_t payload_bytes(uint64_t n_c, uint32_t n_words, bool nib_stored) {
@@ -29,22 +29,27 @@ inline uint64_t payload_bytes(uint64_t n_c, uint32_t n_words, bool nib_stored) {
 // Decode-kernel geometry: a warp decodes kChains chunks at once (two independent state
 // chains per lane), and a CTA of kWarps warps covers kWarps*kChains chunks of one tensor.
 // Each chunk's 16-bit word stream goes through its own shared-memory ring of kRingBytes,
-// in quarters of kQuarterBytes (one 16-byte cp.async per lane fills a quarter).
+// in quarters of kQuarterBytes (one 16-byte cp.async per lane fills a quarter), and its
+// nibble words through a ring of kNibRingBlocks blocks (128 bytes each).
 constexpr int kWarps = 20;
 constexpr int kChains = 2;
 constexpr uint32_t kRingBytes = 2048;
 constexpr uint32_t kQuarterBytes = kRingBytes / 4;
 static_assert(kQuarterBytes == 32 * 16, "one cp.async of 16 bytes per lane fills a quarter");
+constexpr uint32_t kNibRingBlocks = 8;
+constexpr uint32_t kNibRingBytes = kNibRingBlocks * 128;
 // Shared memory of a CTA:
 //   [0, kHRegion)                 fraction rows, one copy per lane (row r, slot j, lane c at
 //                                 byte ((r << nh) + j) * 128 + 4c): conflict-free lookups
-//   [kHRegion, + 8 << ns)         s-table
-//   then the rings, kWarps * kChains * kRingBytes
+//   [kHRegion, + 8 << ns)         s-table (its size rounded up to 2 KiB)
+//   then the word rings (kRingBytes each, so each starts at a multiple of kRingBytes) and
+//   the nibble rings
 // The fraction region is reserved at its largest (16 rows of 2^5 slots) so that the s-table
-// sits at a constant offset. With ns = 13 the total is 128 KiB + 80 KiB of rings.
+// sits at a constant offset. With ns = 12 the total is 96 KiB + 120 KiB of rings.
 constexpr uint32_t kHRegion = 16u * 32u * 128u;
-constexpr uint32_t kRingRegion = uint32_t(kWarps) * kChains * kRingBytes;
-inline uint32_t smem_bytes_for(uint32_t ns) { return kHRegion + (8u << ns) + kRingRegion; }
+constexpr uint32_t kRingRegion = uint32_t(kWarps) * kChains * (kRingBytes + kNibRingBytes);
+__host__ __device__ inline uint32_t s_region_bytes(uint32_t ns) { return ((8u << ns) + kRingBytes - 1) & ~(kRingBytes - 1); }
+inline uint32_t smem_bytes_for(uint32_t ns) { return kHRegion + s_region_bytes(ns) + kRingRegion; }
 
 // Workspace layout: a 256-byte error block, then 256-aligned tables per RANS tensor.
 constexpr uint64_t kErrBlockBytes = 256;
@@ -100,6 +105,10 @@ struct DecodeParams {
     uint32_t n_items;
     uint32_t total_ctas;
     unsigned long long* err; // [0]: flags, [1]: smallest (tensor << 40 | chunk) that failed
+    // Multipliers the decode loop uses in multiply-adds. Read from the parameters, they stay
+    // opaque to the compiler, so those steps run as IMAD on the FMA pipe (which has spare
+    // issue slots) instead of becoming shifts on the integer ALU pipe, the kernel's bound.
+    uint32_t mul2 = 2, mul65536 = 65536;
     DecodeItem item[kMaxDecodeItems];
 };
 

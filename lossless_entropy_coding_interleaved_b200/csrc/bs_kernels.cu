@@ -26,8 +26,8 @@
 //    of unequal length take a checked path.
 //  * The 16-bit word stream of a chunk is prefetched into its own 2 KiB shared-memory ring
 //    with cp.async (16 B per lane, in quarters of 512 B), kept 2-3 quarters ahead; the
-//    upkeep runs every 16 steps. The nibble words are loaded one block ahead into
-//    registers (one coalesced 128-byte load per chunk and block).
+//    upkeep runs every 16 steps. The same upkeep copies the nibble words (128 B per block)
+//    four blocks ahead into a 1 KiB ring, so no global load sits on the decode loop.
 //  * The default precisions (ns=11, nh=5) get an instantiation with constant shifts.
 //  * Renormalisation reads (at most one 16-bit word per lane per weight) are assigned in
 //    lane order by ballot + prefix popcount. The words a step consumes are contiguous, so
@@ -68,11 +68,13 @@ struct Chain {
     uint32_t posb;            // bytes of the word stream consumed (warp-uniform)
     uint32_t fq;              // ring quarters requested (warp-uniform)
     uint32_t total_q, stream_bytes, nc, n_blocks;
-    uint32_t ring;            // shared-memory address of the ring
+    uint32_t ring;            // shared-memory address of the word ring
     uint32_t ring_off;        // the same ring as an offset into the dynamic smem array
+    uint32_t nring;           // shared-memory address of the nibble ring
+    uint32_t nring_off;       // the same ring as an offset into the dynamic smem array
     uint32_t raw;             // nibble word of the current block (constant mode: c in every nibble)
     const uint8_t* stream;
-    const uint32_t* nib;      // nibble words (block-major), or null in constant mode
+    const uint8_t* nib;       // nibble words (block-major), or null in constant mode
     uint16_t* out;
     uint64_t chunk;
     bool live;                // a real chunk (false: a filler chain that is never stored)
@@ -121,8 +123,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(const __grid_con
 
     const bool nib_stored = it.nib_mode == 0;
     const uint32_t raw_const = (it.nib_mode & 15u) * 0x11111111u;
-    const uint32_t ring_off = kHRegion + (8u << ns) + (warp * kChains) * kRingBytes; // this warp's first ring
-    const uint32_t ring_base = smem_u32(smem) + ring_off;
+    const uint32_t rings = kHRegion + s_region_bytes(ns);                  // a multiple of kRingBytes
+    const uint32_t ring_off = rings + (warp * kChains) * kRingBytes;       // this warp's first word ring
+    const uint32_t nring_off = rings + kWarps * kChains * kRingBytes + (warp * kChains) * kNibRingBytes;
+    const uint32_t ring_base = smem_u32(smem) + ring_off, nring_base = smem_u32(smem) + nring_off;
     Chain c[kChains];
     uint32_t nb = 0;
 #pragma unroll
@@ -132,6 +136,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(const __grid_con
         h.live = h.chunk < n_chunks;
         h.ring = ring_base + k * kRingBytes;
         h.ring_off = ring_off + k * kRingBytes;
+        h.nring = nring_base + k * kNibRingBytes;
+        h.nring_off = nring_off + k * kNibRingBytes;
         h.posb = 0;
         h.fq = 0;
         h.bad = false;
@@ -145,7 +151,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(const __grid_con
             const uint64_t base = h.chunk << log2c;
             h.nc = static_cast<uint32_t>(min(C, n_elems - base));
             h.n_blocks = (h.nc + 255u) >> 8; // blocks of 8 steps
-            if (nib_stored) h.nib = reinterpret_cast<const uint32_t*>(payload + 128);
+            if (nib_stored) h.nib = payload + 128;
             h.stream = payload + 128 + (nib_stored ? 128u * h.n_blocks : 0u);
             h.stream_bytes = 2u * n_words;
             h.total_q = (h.stream_bytes + kQuarterBytes - 1) / kQuarterBytes;
@@ -163,18 +169,29 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(const __grid_con
 
     const uint32_t smask8 = ((1u << ns) - 1u) << 3, hmask7 = ((1u << nh) - 1u) << 7;
     const uint32_t lt = lanemask_lt(), lane4 = lane << 2;
+    const uint32_t mul2 = p.mul2, mul65536 = p.mul65536;
 
     // Ring upkeep before a block of 16 steps: request up to quarter q+3 for each chain,
     // where q holds the next word. The next 16 steps need at most quarters q..q+2 (at most
     // 32 lanes x 16 steps x 2 bytes = 1 KiB). Wait for every copy, or for all but the
     // newest group when those were requested earlier. Quarters wholly inside the stream
     // skip the per-piece bounds.
+    // Nibble words: at block blk (even) the ring must hold blocks blk and blk+1, which were
+    // requested two upkeeps earlier; this upkeep requests blocks blk+4 and blk+5 (16 lanes x
+    // 16 bytes). The first upkeep requests blocks 0-5 and waits for all of them.
     auto upkeep = [&](uint32_t blk) {
         __syncwarp();
         bool newest_needed = blk == 0;
 #pragma unroll
         for (int k = 0; k < kChains; ++k) {
             Chain& h = c[k];
+            if (h.nib && blk < h.n_blocks) {
+                for (uint32_t b = (blk == 0 ? 0u : blk + 4u); b < blk + 6u; b += 2u) {
+                    const uint32_t byte = 128u * b + 16u * lane; // lanes 0-15: blocks b and b+1
+                    if (lane < 16 && byte < 128u * h.n_blocks)
+                        cp_async16(h.nring + (byte & (kNibRingBytes - 1u)), h.nib + byte, 16u);
+                }
+            }
             if (blk < h.n_blocks) {
                 const uint32_t q = h.posb / kQuarterBytes;
                 if (h.fq <= min(q + 2, h.total_q - 1)) newest_needed = true;
@@ -193,16 +210,13 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(const __grid_con
         __syncwarp();
     };
 
-    // Nibble words: the current block's is in h.raw; the next one is loaded ahead.
-    uint32_t raw_next[kChains];
-#pragma unroll
-    for (int k = 0; k < kChains; ++k) raw_next[k] = (c[k].nib && c[k].n_blocks > 0) ? __ldg(c[k].nib + lane) : raw_const;
+    // The current block's nibble word of each chain, from its ring (or the constant).
     auto next_raw = [&](uint32_t b) {
 #pragma unroll
         for (int k = 0; k < kChains; ++k) {
             Chain& h = c[k];
-            h.raw = raw_next[k];
-            if (h.nib && b + 1 < h.n_blocks) raw_next[k] = __ldg(h.nib + 32u * (b + 1) + lane);
+            if (h.nib && b < h.n_blocks)
+                h.raw = *reinterpret_cast<const uint32_t*>(smem + h.nring_off + ((128u * b) & (kNibRingBytes - 1u)) + lane4);
         }
     };
 
@@ -227,9 +241,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(const __grid_con
                 const bool need = xn < kStateL;
                 const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
                 const uint32_t w = *reinterpret_cast<const uint16_t*>(
-                    smem + h.ring_off + ((h.posb + (__popc(m & lt) << 1)) & (kRingBytes - 1u)));
-                h.x = need ? ((xn << 16) | w) : xn;
-                h.posb += __popc(m) << 1;
+                    smem + (((h.posb + __popc(m & lt) * mul2) & (kRingBytes - 1u)) | h.ring_off));
+                const uint32_t xr = xn * mul65536 + w; // (xn << 16) | w as one IMAD, computed by every lane
+                h.x = need ? xr : xn;
+                h.posb += __popc(m) * mul2;
                 // (s << 7) | (h << 4): s sits pre-shifted in se.y, h in bits 4-6 of fe
                 const uint32_t word = (se.y & 0xFF80u) | (fe & 0x70u);
                 if (s & 1) o[k][s >> 1] = __byte_perm(o[k][s >> 1], word, 0x5410);

@@ -22,7 +22,7 @@
 
 namespace bs {
 
-// Largest decode tables the array holds: the s-table at ns = 13 (64 KiB) plus 16 compact
+// Largest decode tables the array holds: the s-table at ns = 12 (32 KiB) plus 16 compact
 // fraction rows of 2^5 entries (2 KiB). That is every tensor a valid container can hold;
 // larger tables would get BS_E_SIZE.
 constexpr uint32_t kNoAllocTableBytes = (8u << kMaxNs) + 4u * (kMaxRoutes + 1) * (1u << kMaxNh);

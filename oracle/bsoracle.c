@@ -275,7 +275,7 @@ static uint32_t lane_encode(const model_t* m, const uint16_t* w, uint32_t S, uin
 static int model_from_tables(model_t* m, const uint32_t* Fs, uint32_t ns, const uint8_t* route, const uint32_t* Fh,
                              uint32_t n_routes, uint32_t nh) {
     memset(m, 0, sizeof(*m));
-    if (ns < 1 || ns > 13 || nh < 3 || nh > 5 || ns + nh > 16 || n_routes > 15) return BSO_E_ARG;
+    if (ns < 1 || ns > 12 || nh < 3 || nh > 5 || ns + nh > 16 || n_routes > 15) return BSO_E_ARG;
     m->ns = ns; m->nh = nh; m->n_routes = n_routes;
     uint64_t sum = 0;
     for (int s = 0; s < 512; s++) { m->Fs[s] = Fs[s]; sum += Fs[s]; }
@@ -519,7 +519,7 @@ typedef struct {
 int bso_encode(const bso_item* items, uint32_t n_items, const bso_params* p, uint8_t** out, uint64_t* out_len) {
     if (!items && n_items) return BSO_E_ARG;
     if (!p || !out || !out_len) return BSO_E_ARG;
-    if (p->log2_chunk < 8 || p->log2_chunk > 24 || p->ns < 1 || p->ns > 13 || p->nh < 3 || p->nh > 5 ||
+    if (p->log2_chunk < 8 || p->log2_chunk > 24 || p->ns < 1 || p->ns > 12 || p->nh < 3 || p->nh > 5 ||
         p->ns + p->nh > 16 || p->max_routes > 15)
         return BSO_E_ARG;
     int st = BSO_OK;
@@ -697,7 +697,7 @@ static int parse_entry(const uint8_t* b, uint64_t len, uint32_t idx, bso_tensor_
     }
     /* RANS */
     if (ti->lanes != LANES || ti->log2_chunk < 8 || ti->log2_chunk > 24) return BSO_E_FORMAT;
-    if (ti->ns < 1 || ti->ns > 13 || ti->nh < 3 || ti->nh > 5 || ti->ns + ti->nh > 16 || ti->n_routes > 15)
+    if (ti->ns < 1 || ti->ns > 12 || ti->nh < 3 || ti->nh > 5 || ti->ns + ti->nh > 16 || ti->n_routes > 15)
         return BSO_E_FORMAT;
     if (ti->nib_mode != 0 && (ti->nib_mode & 0xF0u) != 0x10u) return BSO_E_FORMAT;
     if (ti->n_elems == 0 || ti->n_elems > (1ull << 40)) return BSO_E_FORMAT;

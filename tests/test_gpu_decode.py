@@ -79,22 +79,24 @@ def test_sizes_and_multiple_launches():
         assert np.array_equal(outs[k], a), sizes[k]
 
 
-@pytest.mark.parametrize("log2_chunk,ns,nf", [(8, 12, 10), (12, 11, 7), (16, 1, 7), (16, 8, 11), (17, 12, 11),
-                                               (20, 12, 10)])
-def test_parameters(log2_chunk, ns, nf):
+@pytest.mark.parametrize("log2_chunk,ns,nh", [(8, 11, 5), (12, 11, 3), (16, 1, 3), (16, 8, 5), (17, 12, 3),
+                                               (20, 11, 5), (16, 12, 4)])
+def test_parameters(log2_chunk, ns, nh):
     w = S.words_numpy(S.generate(S.workload("tensor_1m")[0], "cpu")).reshape(-1)[:700_001].copy()
     if ns < 9:
-        w = np.where(np.arange(w.size) % 3 == 0, 0x3C00, 0xBC01).astype(np.uint16)
-    c = oracle.encode([("w", w, "bf16")], log2_chunk=log2_chunk, ns=ns, nf=nf, force_rans=True)
+        w = np.where(np.arange(w.size) % 3 == 0, 0x3C00, 0xBC31).astype(np.uint16)
+    c = oracle.encode([("w", w, "bf16")], log2_chunk=log2_chunk, ns=ns, nh=nh, force_rans=True)
     _, outs = _decode_all(c, 1)
     assert np.array_equal(outs[0], w)
 
 
-@pytest.mark.parametrize("nf", [10, 11])
-def test_largest_tables(nf):
-    # 15 routes: 32 KiB + 16 rows x 2^nf x 4 B of tables (96 KiB / 160 KiB), the two CTA shapes
-    w = np.concatenate([((e << 7) | (np.arange(3000) % (3 + e % 5))).astype(np.uint16) for e in range(90, 110)])
-    c = oracle.encode([("skewed", w, "bf16")], nf=nf, max_routes=15)
+@pytest.mark.parametrize("ns,nh", [(11, 5), (12, 4)])
+def test_largest_tables(ns, nh):
+    # 15 routes (16 fraction rows with UNIFORM) and, at ns = 12, the largest s-table (32 KiB):
+    # the most shared memory any valid container asks for
+    w = np.concatenate([((e << 7) | ((np.arange(3000) % (3 + e % 5)) << 4) | (np.arange(3000) % 16)).astype(np.uint16)
+                        for e in range(90, 110)])
+    c = oracle.encode([("skewed", w, "bf16")], ns=ns, nh=nh, max_routes=15)
     assert oracle.info(c, 0)["n_routes"] == 15
     _, outs = _decode_all(c, 1)
     assert np.array_equal(outs[0], w)
@@ -132,7 +134,7 @@ def test_corrupt_chunk_is_reported():
     ti = oracle.info(bytes(c), 0)
     e2 = ti["data_offset"] + 16 * 2
     off2 = int.from_bytes(c[e2:e2 + 8], "little")
-    c[off2 + 8 * 5 + 6] ^= 0x10                        # lane 5's state, bit 52
+    c[off2 + 4 * 5 + 2] ^= 0x10                        # lane 5's state, bit 20
     plan = bs.Plan(bytes(c), device="cuda:0")
     plan.decode(0)
     with pytest.raises(bs.BsError) as e:
@@ -143,19 +145,20 @@ def test_corrupt_chunk_is_reported():
 
 
 def test_in_sync_flip_caught_by_checksum():
-    # a flip inside a UNIFORM fraction changes one weight without desync: checksum catches it
+    # a flip in a stored nibble changes one weight without any desync: the checksum catches it
     w = np.full(70_000, 0x3C00, np.uint16) | (np.arange(70_000, dtype=np.uint16) & 0x7F)   # one exponent, flat
     c = bytearray(oracle.encode([("w", w, "bf16")], force_rans=True))
     ti = oracle.info(bytes(c), 0)
+    assert ti["nib_mode"] == 0
     e0 = ti["data_offset"]
     off0 = int.from_bytes(c[e0:e0 + 8], "little")
-    c[off0 + 256 + 4 * 40 + 1] ^= 0x04                  # a stream word's bit 10: raw fraction bits
+    c[off0 + 128 + 4 * 40 + 1] ^= 0x04                  # nibble word 40 (block 1, lane 8), bit 10
     plan = bs.Plan(bytes(c), device="cuda:0")
     out = plan.decode(0)
     plan.check()
     got = _host(out)
-    if np.array_equal(got, w):
-        pytest.skip("flip landed on bits that decode identically")
+    assert int(np.count_nonzero(got != w)) == 1         # weight 256 + 8*8 + 4: its nibble's bit 2
+    assert int(got[256 + 64 + 4]) == int(w[256 + 64 + 4]) ^ 0x4
     with pytest.raises(bs.BsError) as e:
         plan.verify(0, out)
     assert e.value.code == bs.E_CORRUPT

@@ -40,12 +40,12 @@ def test_device_encoder_matches_oracle_bytes(name, kw):
     assert torch.equal(d_c.cpu(), torch.from_numpy(h_c))
 
 
-@pytest.mark.parametrize("log2_chunk,ns,nf,max_routes", [(8, 12, 10, 7), (12, 9, 7, 2), (17, 12, 11, 15),
-                                                         (16, 11, 10, 0)])
-def test_device_encoder_parameters(log2_chunk, ns, nf, max_routes):
+@pytest.mark.parametrize("log2_chunk,ns,nh,max_routes", [(8, 11, 5, 7), (12, 9, 3, 2), (17, 12, 4, 15),
+                                                         (16, 12, 4, 0)])
+def test_device_encoder_parameters(log2_chunk, ns, nh, max_routes):
     specs = S.workload("edge_mix")[:2] + S.workload("tensor_1m")
     cpu, dev = _gpu_items(specs)
-    kw = dict(log2_chunk=log2_chunk, ns=ns, nf=nf, max_routes=max_routes)
+    kw = dict(log2_chunk=log2_chunk, ns=ns, nh=nh, max_routes=max_routes)
     _, h_c = bs.encode(dev, host_copy=True, **kw)
     assert bytes(h_c.tobytes()) == oracle.encode(_host_items(specs, cpu), **kw)
     for k, t in enumerate(cpu):

@@ -138,12 +138,12 @@ TINY_MODELS.append(dict(fs={1: 9, 2: 6, 257: 1}, ns=4, route={2: 0}, fh=_fh, nh=
                         alphabet=[(1 << 7) | (3 << 4) | 5, (2 << 7) | (1 << 4) | 9, (257 << 7) | 0]))
 TINY_MODELS.append(dict(fs={1: 1, 2: 1, 3: 2}, ns=2, route=None, fh=None, nh=3,
                         alphabet=[(1 << 7) | 0, (2 << 7) | (7 << 4) | 15, (3 << 7) | (4 << 4) | 1]))
-# P = 16, the largest precision: one symbol of frequency 1 at ns = 13 and a table with a
+# P = 16, the largest precision: one symbol of frequency 1 at ns = 12 and a table with a
 # frequency-1 entry, so Q = 1 costs 16 bits and every step of it emits a word
 _fh2 = np.zeros((2, 8), np.uint32)
-_fh2[0, :] = 1            # flat over the eight values, sums to 8
-_fh2[1, 3], _fh2[1, 7] = 7, 1
-TINY_MODELS.append(dict(fs={10: 8191, 300: 1}, ns=13, route={10: 0, 300 & 0xFF: 1}, fh=_fh2, nh=3,
+_fh2[0, :] = 2            # flat over the eight values, sums to 16
+_fh2[1, 3], _fh2[1, 7] = 15, 1
+TINY_MODELS.append(dict(fs={10: 4095, 300: 1}, ns=12, route={10: 0, 300 & 0xFF: 1}, fh=_fh2, nh=4,
                         alphabet=[(10 << 7) | (3 << 4) | 7, (300 << 7) | (3 << 4) | 9, (300 << 7) | (7 << 4)]))
 
 

@@ -52,7 +52,7 @@ def test_noalloc_reports_corrupt_chunk_and_oversized_tables():
     ti = oracle.info(c, 0)
     e0 = ti["data_offset"] + 16 * 3
     off = int.from_bytes(bad[e0:e0 + 8], "little")
-    bad[off + 8 * 7 + 6] ^= 0x20                       # chunk 3, lane 7's start state
+    bad[off + 4 * 7 + 2] ^= 0x20                       # chunk 3, lane 7's start state, bit 21
     d_bad = torch.from_numpy(np.frombuffer(bytes(bad), np.uint8).copy()).cuda()
     out = torch.empty(arrs[0].shape, dtype=torch.int16, device="cuda:0")
     with pytest.raises(bs.BsError) as e:
@@ -62,16 +62,20 @@ def test_noalloc_reports_corrupt_chunk_and_oversized_tables():
     d_c = torch.from_numpy(np.frombuffer(c, np.uint8).copy()).cuda()
     bs.decode_noalloc(c, d_c, 0, out)
     assert np.array_equal(out.cpu().numpy().view(np.uint16).reshape(arrs[0].shape), arrs[0])
-    # tables above the 96 KiB the static array holds: 16 exponents, each with a skewed
-    # fraction distribution, give 15 routes; at nf = 11 that is 32 KiB + 16 x 8 KiB
-    w = np.concatenate([((e << 7) | (np.arange(1000) % 3)).astype(np.uint16) for e in range(100, 116)])
-    big = oracle.encode([("skewed", w, "bf16")], nf=11, max_routes=15)
+    # the largest tables a valid container has (ns = 12 and 15 routes: 32 KiB + 2 KiB) fit
+    # the static array: 16 exponents, each with a skewed top-bit distribution
+    w = np.concatenate([((e << 7) | ((np.arange(1000) % 3) << 4) | (np.arange(1000) % 16)).astype(np.uint16)
+                        for e in range(100, 116)])
+    big = oracle.encode([("skewed", w, "bf16")], ns=12, nh=4, max_routes=15)
     assert oracle.info(big, 0)["n_routes"] == 15
     d_big = torch.from_numpy(np.frombuffer(big, np.uint8).copy()).cuda()
     out = torch.empty(w.size, dtype=torch.int16, device="cuda:0")
+    bs.decode_noalloc(big, d_big, 0, out)
+    assert np.array_equal(out.cpu().numpy().view(np.uint16), w)
+    # a directory entry with ns = 13 is refused before any device work
+    bad = bytearray(big)
+    dir_off = int.from_bytes(bad[24:32], "little")
+    bad[dir_off + 4] = 13
     with pytest.raises(bs.BsError) as e:
-        bs.decode_noalloc(big, d_big, 0, out)
-    assert e.value.code == bs.E_SIZE
-    # the same tensor through the regular path (workspace from the caller) decodes fine
-    plan = bs.Plan(big, device="cuda:0")
-    assert np.array_equal(plan.decode(0).cpu().numpy().view(np.uint16), w)
+        bs.decode_noalloc(bytes(bad), d_big, 0, out)
+    assert e.value.code == bs.E_FORMAT
