@@ -27,12 +27,15 @@ inline uint64_t payload_bytes(uint64_t n_c, uint32_t n_words, bool nib_stored) {
 }
 
 // Decode-kernel geometry: a warp decodes kChains chunks at once (two independent state
-// chains per lane), and a CTA of kWarps warps covers kWarps*kChains chunks of one tensor.
+// chains per lane), and a CTA of `warps` warps covers warps*kChains chunks of one tensor:
+// 24 warps for the default precisions, 20 otherwise (ns = 12 tables leave room for 20).
 // Each chunk's 16-bit word stream goes through its own shared-memory ring of kRingBytes,
 // in quarters of kQuarterBytes (one 16-byte cp.async per lane fills a quarter), and its
 // nibble words through a ring of kNibRingBlocks blocks (128 bytes each).
-constexpr int kWarps = 20;
+constexpr int kWarpsDefault = 24, kWarpsGeneric = 20;
 constexpr int kChains = 2;
+inline bool is_default_precision(uint32_t ns, uint32_t nh) { return ns == 11 && nh == 5; }
+inline int warps_for(uint32_t ns, uint32_t nh) { return is_default_precision(ns, nh) ? kWarpsDefault : kWarpsGeneric; }
 constexpr uint32_t kRingBytes = 2048;
 constexpr uint32_t kQuarterBytes = kRingBytes / 4;
 static_assert(kQuarterBytes == 32 * 16, "one cp.async of 16 bytes per lane fills a quarter");
@@ -45,11 +48,13 @@ constexpr uint32_t kNibRingBytes = kNibRingBlocks * 128;
 //   then the word rings (kRingBytes each, so each starts at a multiple of kRingBytes) and
 //   the nibble rings
 // The fraction region is reserved at its largest (16 rows of 2^5 slots) so that the s-table
-// sits at a constant offset. With ns = 12 the total is 96 KiB + 120 KiB of rings.
+// sits at a constant offset. Default precisions: 80 KiB of tables + 144 KiB of rings for 24
+// warps; ns = 12: 96 KiB + 120 KiB for 20 warps.
 constexpr uint32_t kHRegion = 16u * 32u * 128u;
-constexpr uint32_t kRingRegion = uint32_t(kWarps) * kChains * (kRingBytes + kNibRingBytes);
 __host__ __device__ inline uint32_t s_region_bytes(uint32_t ns) { return ((8u << ns) + kRingBytes - 1) & ~(kRingBytes - 1); }
-inline uint32_t smem_bytes_for(uint32_t ns) { return kHRegion + s_region_bytes(ns) + kRingRegion; }
+inline uint32_t smem_bytes_for(uint32_t ns, int warps) {
+    return kHRegion + s_region_bytes(ns) + uint32_t(warps) * kChains * (kRingBytes + kNibRingBytes);
+}
 
 // Workspace layout: a 256-byte error block, then 256-aligned tables per RANS tensor.
 constexpr uint64_t kErrBlockBytes = 256;

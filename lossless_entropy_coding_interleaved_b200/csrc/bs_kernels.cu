@@ -82,8 +82,8 @@ struct Chain {
 };
 
 // NS/NH > 0: compile-time precisions (the default container); 0: read from the item.
-template <int NS, int NH>
-__global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
+template <int WARPS, int NS, int NH>
+__global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
     // dynamic smem: [fraction rows, one copy per lane][s-table][rings]
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ int s_item;
@@ -118,14 +118,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(const __grid_con
     const uint64_t C = 1ull << log2c;
     const uint64_t n_elems = it.n_elems;
     const uint64_t n_chunks = (n_elems + C - 1) >> log2c;
-    const uint64_t chunk0 = static_cast<uint64_t>(blockIdx.x - it.cta_begin) * (kWarps * kChains) + warp * kChains;
+    const uint64_t chunk0 = static_cast<uint64_t>(blockIdx.x - it.cta_begin) * (WARPS * kChains) + warp * kChains;
     if (chunk0 >= n_chunks) return;
 
     const bool nib_stored = it.nib_mode == 0;
     const uint32_t raw_const = (it.nib_mode & 15u) * 0x11111111u;
     const uint32_t rings = kHRegion + s_region_bytes(ns);                  // a multiple of kRingBytes
     const uint32_t ring_off = rings + (warp * kChains) * kRingBytes;       // this warp's first word ring
-    const uint32_t nring_off = rings + kWarps * kChains * kRingBytes + (warp * kChains) * kNibRingBytes;
+    const uint32_t nring_off = rings + WARPS * kChains * kRingBytes + (warp * kChains) * kNibRingBytes;
     const uint32_t ring_base = smem_u32(smem) + ring_off, nring_base = smem_u32(smem) + nring_off;
     Chain c[kChains];
     uint32_t nb = 0;
@@ -210,12 +210,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(const __grid_con
         __syncwarp();
     };
 
-    // The current block's nibble word of each chain, from its ring (or the constant).
-    auto next_raw = [&](uint32_t b) {
+    // The current block's nibble word of each chain, from its ring (or the constant). In the
+    // full-block loop every live chain has block b; in the tail a chain past its end keeps
+    // its last word (its output is not stored).
+    auto next_raw = [&](uint32_t b, bool full) {
 #pragma unroll
         for (int k = 0; k < kChains; ++k) {
             Chain& h = c[k];
-            if (h.nib && b < h.n_blocks)
+            if (h.nib && (full || b < h.n_blocks))
                 h.raw = *reinterpret_cast<const uint32_t*>(smem + h.nring_off + ((128u * b) & (kNibRingBytes - 1u)) + lane4);
         }
     };
@@ -259,7 +261,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(const __grid_con
     };
 
     // Full blocks first: every live chain has all 256 weights of the block, so the stores
-    // need no bounds; blocks are taken two at a time.
+    // need no bounds; blocks are taken two at a time. A chain whose last block is the last
+    // one of this loop gets its end check after the loop.
     uint32_t nb_full = 0xFFFFFFFFu;
 #pragma unroll
     for (int k = 0; k < kChains; ++k)
@@ -270,18 +273,19 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(const __grid_con
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             const uint32_t b = blk + half, i0 = (b << 8) + (lane << 3);
-            next_raw(b);
+            next_raw(b, true);
             uint32_t o[kChains][4];
             octet(o);
 #pragma unroll
             for (int k = 0; k < kChains; ++k) {
                 Chain& h = c[k];
                 if (h.live) *reinterpret_cast<uint4*>(h.out + i0) = make_uint4(o[k][0], o[k][1], o[k][2], o[k][3]);
-                if (b + 1 == h.n_blocks) // end check: state back at L, every word consumed
-                    h.bad |= (h.x != kStateL) | (h.posb != h.stream_bytes);
             }
         }
     }
+#pragma unroll
+    for (int k = 0; k < kChains; ++k) // end check: state back at L, every word consumed
+        if (c[k].live && c[k].n_blocks == blk) c[k].bad |= (c[k].x != kStateL) | (c[k].posb != c[k].stream_bytes);
     // The rest (ragged tails, chains of different lengths), with bounds, two blocks at a time.
     for (; blk < nb; blk += 2) {
         upkeep(blk);
@@ -289,7 +293,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(const __grid_con
         for (int half = 0; half < 2; ++half) {
             const uint32_t b = blk + half;
             if (b >= nb) break;
-            next_raw(b);
+            next_raw(b, false);
             uint32_t o[kChains][4];
             octet(o);
 #pragma unroll
@@ -375,12 +379,12 @@ int max_dynamic_smem() {
     return v;
 }
 
-template <int NS, int NH>
+template <int WARPS, int NS, int NH>
 static int launch_decode_t(const DecodeParams& p, uint32_t smem_bytes, cudaStream_t s) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<NS, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<WARPS, NS, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem_bytes));
     if (e != cudaSuccess) return e;
-    decode_kernel<NS, NH><<<p.total_ctas, kWarps * 32, smem_bytes, s>>>(p);
+    decode_kernel<WARPS, NS, NH><<<p.total_ctas, WARPS * 32, smem_bytes, s>>>(p);
     count_launch();
     return cudaGetLastError();
 }
@@ -388,7 +392,8 @@ static int launch_decode_t(const DecodeParams& p, uint32_t smem_bytes, cudaStrea
 int launch_decode(const DecodeParams& p, bool default_precision, uint32_t smem_bytes, void* stream) {
     if (p.total_ctas == 0) return cudaSuccess;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return default_precision ? launch_decode_t<11, 5>(p, smem_bytes, s) : launch_decode_t<0, 0>(p, smem_bytes, s);
+    return default_precision ? launch_decode_t<kWarpsDefault, 11, 5>(p, smem_bytes, s)
+                             : launch_decode_t<kWarpsGeneric, 0, 0>(p, smem_bytes, s);
 }
 
 int launch_copy(const CopyParams& p, void* stream) {
