@@ -244,7 +244,7 @@ def run_reference(a):
     value = 2 * n * a.steps / sec / 1e9
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": a.gpus,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(1e3 * sec / a.steps, 3),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u64",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32",
             "data": "synthetic", "config": {"workload": a.workload, "description": desc, "n_weights": n_all,
                                             "step": "one bounded sample per step: " + sample},
             "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
@@ -387,7 +387,7 @@ def run_ours(a):
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": round(total_ms / a.steps, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "u64",
+        "scaling": "weak", "vs_baseline": None, "dtype": "u32",
         "data": "synthetic (seeded device draws, synthetic/ recipe)",
         "config": {"workload": a.workload, "description": desc, "n_weights": n, "tensors": len(specs),
                    "container_bytes": int(d_c.numel()), "coded_bytes": int(coded),
@@ -398,7 +398,7 @@ def run_ours(a):
                    "parallelism": f"replicas x{world} (no collective on the data path)",
                    "l2": "no flush: inputs larger than L2 (container and outputs are GBs)",
                    "parity": parity_how, "encode_s": round(t_encode, 2),
-                   "words": "BF16 bit patterns; rANS state arithmetic in u64"},
+                   "words": "BF16 bit patterns; rANS state arithmetic in u32"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": (None if tpw is None else int(tpw * bf16_n)),
@@ -508,7 +508,7 @@ def run_layerwise(a):
         "metric": "decompressed BF16 GB/s, layer by layer (one bs_decode_batch per layer)",
         "value": round(ranks.world * a.steps * out_bytes / (ms * 1e-3) / 1e9, 3), "unit": "GB/s",
         "n_gpus": ranks.world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms / a.steps, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u64", "data": "synthetic",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
         "config": {"workload": a.workload, "description": desc, "n_weights": n, "groups": len(members),
                    "decoded_bytes": int(out_bytes), "coded_bytes": int(coded),
                    "entropy_bits_per_weight": round(h_per_w, 5), "encode_s": round(t_encode, 2),
@@ -622,7 +622,7 @@ def run_stream(a):
                   "LRU device cache",
         "value": round(ranks.world * a.steps * out_bytes / (ms * 1e-3) / 1e9, 3), "unit": "GB/s",
         "n_gpus": ranks.world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms / a.steps, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u64", "data": "synthetic",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
         "config": {"workload": a.workload, "description": desc, "n_weights": n, "groups": n_groups,
                    "arena_bytes": int(arena), "stage_bytes": s1["stage_bytes"],
                    "decoded_bytes_per_pass": int(out_bytes), "h2d_bytes_per_pass": int(h2d),
