@@ -26,16 +26,18 @@ inline uint64_t payload_bytes(uint64_t n_c, uint32_t n_words, bool nib_stored) {
     return (128 + (nib_stored ? 128 * blocks : 0) + 2ull * n_words + 15) & ~uint64_t(15);
 }
 
-// Decode-kernel geometry: a warp decodes kChains chunks at once (two independent state
-// chains per lane), and a CTA of `warps` warps covers warps*kChains chunks of one tensor:
-// 24 warps for the default precisions, 20 otherwise (ns = 12 tables leave room for 20).
+// Decode-kernel geometry: a warp decodes `chains` chunks at once (independent state chains
+// per lane), and a CTA of `warps` warps covers warps*chains chunks of one tensor. The
+// default precisions use 24 warps of 2 chains; the others 20 warps of 2 (ns = 12 tables
+// leave room for 40 rings).
 // Each chunk's 16-bit word stream goes through its own shared-memory ring of kRingBytes,
 // in quarters of kQuarterBytes (one 16-byte cp.async per lane fills a quarter), and its
 // nibble words through a ring of kNibRingBlocks blocks (128 bytes each).
-constexpr int kWarpsDefault = 24, kWarpsGeneric = 20;
-constexpr int kChains = 2;
+constexpr int kWarpsDefault = 24, kChainsDefault = 2, kWarpsGeneric = 20, kChainsGeneric = 2;
 inline bool is_default_precision(uint32_t ns, uint32_t nh) { return ns == 11 && nh == 5; }
 inline int warps_for(uint32_t ns, uint32_t nh) { return is_default_precision(ns, nh) ? kWarpsDefault : kWarpsGeneric; }
+inline int chains_for(uint32_t ns, uint32_t nh) { return is_default_precision(ns, nh) ? kChainsDefault : kChainsGeneric; }
+inline uint64_t chunks_per_cta(uint32_t ns, uint32_t nh) { return uint64_t(warps_for(ns, nh)) * chains_for(ns, nh); }
 constexpr uint32_t kRingBytes = 2048;
 constexpr uint32_t kQuarterBytes = kRingBytes / 4;
 static_assert(kQuarterBytes == 32 * 16, "one cp.async of 16 bytes per lane fills a quarter");
@@ -48,12 +50,12 @@ constexpr uint32_t kNibRingBytes = kNibRingBlocks * 128;
 //   then the word rings (kRingBytes each, so each starts at a multiple of kRingBytes) and
 //   the nibble rings
 // The fraction region is reserved at its largest (16 rows of 2^5 slots) so that the s-table
-// sits at a constant offset. Default precisions: 80 KiB of tables + 144 KiB of rings for 24
-// warps; ns = 12: 96 KiB + 120 KiB for 20 warps.
+// sits at a constant offset. Default precisions: 80 KiB of tables + 144 KiB of rings for 48
+// chains; ns = 12: 96 KiB + 120 KiB for 40 chains.
 constexpr uint32_t kHRegion = 16u * 32u * 128u;
 __host__ __device__ inline uint32_t s_region_bytes(uint32_t ns) { return ((8u << ns) + kRingBytes - 1) & ~(kRingBytes - 1); }
-inline uint32_t smem_bytes_for(uint32_t ns, int warps) {
-    return kHRegion + s_region_bytes(ns) + uint32_t(warps) * kChains * (kRingBytes + kNibRingBytes);
+inline uint32_t smem_bytes_for(uint32_t ns, uint32_t nh) {
+    return kHRegion + s_region_bytes(ns) + uint32_t(chunks_per_cta(ns, nh)) * (kRingBytes + kNibRingBytes);
 }
 
 // Workspace layout: a 256-byte error block, then 256-aligned tables per RANS tensor.

@@ -82,8 +82,9 @@ struct Chain {
 };
 
 // NS/NH > 0: compile-time precisions (the default container); 0: read from the item.
-template <int WARPS, int NS, int NH>
+template <int WARPS, int CHAINS, int NS, int NH>
 __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
+    constexpr int kChains = CHAINS;
     // dynamic smem: [fraction rows, one copy per lane][s-table][rings]
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ int s_item;
@@ -222,33 +223,47 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
         }
     };
 
-    // 8 steps of every chain, interleaved; o[k] receives chain k's 8 words as 4 pairs
+    // 8 steps of every chain; o[k] receives chain k's 8 words as 4 pairs. Within a step the
+    // chains advance phase by phase (lookups, update, ballot, word read, select), so the
+    // independent work of the two chains sits side by side between the warp-wide votes.
     auto octet = [&](uint32_t (&o)[kChains][4]) {
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
+            uint2 se[kChains];
+            uint32_t fe[kChains], xn[kChains], m[kChains], w[kChains];
+            bool need[kChains];
+#pragma unroll
+            for (int k = 0; k < kChains; ++k) // the s-entry from the slot's high ns bits
+                se[k] = *reinterpret_cast<const uint2*>(smem + kHRegion + ((c[k].x >> (nh - 3)) & smask8));
+#pragma unroll
+            for (int k = 0; k < kChains; ++k) { // the fraction entry from its low nh bits
+                const uint32_t u = ((c[k].x << 7) & hmask7) | lane4;
+                fe[k] = *reinterpret_cast<const uint32_t*>(smem + (se[k].y >> 16) + u);
+            }
+#pragma unroll
+            for (int k = 0; k < kChains; ++k) {
+                const uint32_t t = c[k].x >> P;
+                const uint32_t Fs = se[k].x & 0xFFFFu, bs = se[k].x >> 16;
+                const uint32_t Fh = __byte_perm(fe[k], 0u, 0x4442), bh = fe[k] >> 24;
+                xn[k] = (Fs * Fh) * t + (bs * Fh + bh);
+                need[k] = xn[k] < kStateL;
+            }
+            // renormalise: lanes below 2^16 take the next words, in lane order
+            // (branch-free: every lane reads; the ones that need no word discard it)
+#pragma unroll
+            for (int k = 0; k < kChains; ++k) m[k] = __ballot_sync(0xFFFFFFFFu, need[k]);
+#pragma unroll
+            for (int k = 0; k < kChains; ++k)
+                w[k] = *reinterpret_cast<const uint16_t*>(
+                    smem + (((c[k].posb + __popc(m[k] & lt) * mul2) & (kRingBytes - 1u)) | c[k].ring_off));
 #pragma unroll
             for (int k = 0; k < kChains; ++k) {
                 Chain& h = c[k];
-                const uint32_t x = h.x;
-                const uint32_t t = x >> P;
-                // the s-entry from the slot's high ns bits, the fraction entry from its low nh bits
-                const uint2 se = *reinterpret_cast<const uint2*>(smem + kHRegion + ((x >> (nh - 3)) & smask8));
-                const uint32_t u = ((x << 7) & hmask7) | lane4;
-                const uint32_t fe = *reinterpret_cast<const uint32_t*>(smem + (se.y >> 16) + u);
-                const uint32_t Fs = se.x & 0xFFFFu, bs = se.x >> 16;
-                const uint32_t Fh = __byte_perm(fe, 0u, 0x4442), bh = fe >> 24;
-                uint32_t xn = (Fs * Fh) * t + (bs * Fh + bh);
-                // renormalise: lanes below 2^16 take the next words, in lane order
-                // (branch-free: every lane reads; the ones that need no word discard it)
-                const bool need = xn < kStateL;
-                const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
-                const uint32_t w = *reinterpret_cast<const uint16_t*>(
-                    smem + (((h.posb + __popc(m & lt) * mul2) & (kRingBytes - 1u)) | h.ring_off));
-                const uint32_t xr = xn * mul65536 + w; // (xn << 16) | w as one IMAD, computed by every lane
-                h.x = need ? xr : xn;
-                h.posb += __popc(m) * mul2;
+                const uint32_t xr = xn[k] * mul65536 + w[k]; // (xn << 16) | w as one IMAD, computed by every lane
+                h.x = need[k] ? xr : xn[k];
+                h.posb += __popc(m[k]) * mul2;
                 // (s << 7) | (h << 4): s sits pre-shifted in se.y, h in bits 4-6 of fe
-                const uint32_t word = (se.y & 0xFF80u) | (fe & 0x70u);
+                const uint32_t word = (se[k].y & 0xFF80u) | (fe[k] & 0x70u);
                 if (s & 1) o[k][s >> 1] = __byte_perm(o[k][s >> 1], word, 0x5410);
                 else o[k][s >> 1] = word;
             }
@@ -379,12 +394,12 @@ int max_dynamic_smem() {
     return v;
 }
 
-template <int WARPS, int NS, int NH>
+template <int WARPS, int CHAINS, int NS, int NH>
 static int launch_decode_t(const DecodeParams& p, uint32_t smem_bytes, cudaStream_t s) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<WARPS, NS, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem_bytes));
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<WARPS, CHAINS, NS, NH>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes));
     if (e != cudaSuccess) return e;
-    decode_kernel<WARPS, NS, NH><<<p.total_ctas, WARPS * 32, smem_bytes, s>>>(p);
+    decode_kernel<WARPS, CHAINS, NS, NH><<<p.total_ctas, WARPS * 32, smem_bytes, s>>>(p);
     count_launch();
     return cudaGetLastError();
 }
@@ -392,8 +407,8 @@ static int launch_decode_t(const DecodeParams& p, uint32_t smem_bytes, cudaStrea
 int launch_decode(const DecodeParams& p, bool default_precision, uint32_t smem_bytes, void* stream) {
     if (p.total_ctas == 0) return cudaSuccess;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return default_precision ? launch_decode_t<kWarpsDefault, 11, 5>(p, smem_bytes, s)
-                             : launch_decode_t<kWarpsGeneric, 0, 0>(p, smem_bytes, s);
+    return default_precision ? launch_decode_t<kWarpsDefault, kChainsDefault, 11, 5>(p, smem_bytes, s)
+                             : launch_decode_t<kWarpsGeneric, kChainsGeneric, 0, 0>(p, smem_bytes, s);
 }
 
 int launch_copy(const CopyParams& p, void* stream) {

@@ -273,7 +273,7 @@ bs_status bs::build_workspace(std::vector<Tensor>& ts, std::vector<uint8_t>& ima
     uint64_t pos = kErrBlockBytes;
     for (Tensor& t : ts) {
         if (t.kind != BS_KIND_RANS) continue;
-        if (static_cast<int>(smem_bytes_for(t.ns, warps_for(t.ns, t.nh))) > smem_cap) return BS_E_UNSUPPORTED;
+        if (static_cast<int>(smem_bytes_for(t.ns, t.nh)) > smem_cap) return BS_E_UNSUPPORTED;
         t.ws_offset = pos;
         build_tables(t, image.data() + pos);
         pos += up256(t.table_bytes);
@@ -339,8 +339,7 @@ bs_status DecodeBatch::add(const Tensor& t, uint32_t tensor_index, const uint8_t
     if (t.kind == BS_KIND_RANS) {
         const bool dflt = is_default_precision(t.ns, t.nh);
         Bin& b = bins_[dflt ? 0 : 1];
-        const int warps = warps_for(t.ns, t.nh);
-        const uint64_t per_cta = uint64_t(warps) * kChains;
+        const uint64_t per_cta = chunks_per_cta(t.ns, t.nh);
         const uint64_t ctas = (t.n_chunks + per_cta - 1) / per_cta;
         if (b.p->n_items == kMaxDecodeItems || b.p->total_ctas + ctas > 0x7FFFFFFFull) {
             bs_status s = flush_bin(b, stream);
@@ -362,7 +361,7 @@ bs_status DecodeBatch::add(const Tensor& t, uint32_t tensor_index, const uint8_t
         it.n_routes = static_cast<uint8_t>(t.n_routes);
         it.nib_mode = static_cast<uint8_t>(t.nib_mode);
         b.p->total_ctas += static_cast<uint32_t>(ctas);
-        b.smem = std::max<uint32_t>(b.smem, smem_bytes_for(t.ns, warps));
+        b.smem = std::max<uint32_t>(b.smem, smem_bytes_for(t.ns, t.nh));
     } else if (t.n_elems) {
         const uint64_t bytes = t.kind == BS_KIND_RAW ? t.n_elems : 2 * t.n_elems;
         const uint64_t blks = (bytes + kCopyBlockBytes - 1) / kCopyBlockBytes;
