@@ -43,11 +43,13 @@ class DecodeBatch {
     struct Bin {
         std::unique_ptr<DecodeParams> p;
         bool default_precision = false;
-        uint32_t smem = 0;
+        uint32_t s_region = 0;  // largest s-table region of the queued tensors
+        uint64_t chunks = 0;    // chunks queued; the CTA shape is chosen at flush
     };
     bs_status flush_bin(Bin& b, void* stream);
     bs_status flush_copy(void* stream);
     unsigned long long* err_;
+    uint32_t sms_ = 148;
     Bin bins_[2];
     std::unique_ptr<CopyParams> cp_;
 };

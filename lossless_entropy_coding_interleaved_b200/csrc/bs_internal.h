@@ -38,6 +38,15 @@ inline bool is_default_precision(uint32_t ns, uint32_t nh) { return ns == 11 && 
 inline int warps_for(uint32_t ns, uint32_t nh) { return is_default_precision(ns, nh) ? kWarpsDefault : kWarpsGeneric; }
 inline int chains_for(uint32_t ns, uint32_t nh) { return is_default_precision(ns, nh) ? kChainsDefault : kChainsGeneric; }
 inline uint64_t chunks_per_cta(uint32_t ns, uint32_t nh) { return uint64_t(warps_for(ns, nh)) * chains_for(ns, nh); }
+// Warps per CTA for one launch of `chunks` chunks: the largest shape when the grid covers the
+// SMs several times over; fewer warps when a small launch (one layer, one tensor) would
+// otherwise leave SMs idle, so that its CTAs spread over every SM in one wave.
+constexpr uint32_t kMinWarps = 4;
+inline uint32_t launch_warps(uint64_t chunks, uint32_t max_warps, uint32_t chains, uint32_t sms) {
+    const uint64_t per_sm = (chunks + sms - 1) / sms;
+    const uint64_t w = (per_sm + chains - 1) / chains;
+    return static_cast<uint32_t>(w < kMinWarps ? kMinWarps : w > max_warps ? max_warps : w);
+}
 constexpr uint32_t kRingBytes = 2048;
 constexpr uint32_t kQuarterBytes = kRingBytes / 4;
 static_assert(kQuarterBytes == 32 * 16, "one cp.async of 16 bytes per lane fills a quarter");
@@ -56,6 +65,9 @@ constexpr uint32_t kHRegion = 16u * 32u * 128u;
 __host__ __device__ inline uint32_t s_region_bytes(uint32_t ns) { return ((8u << ns) + kRingBytes - 1) & ~(kRingBytes - 1); }
 inline uint32_t smem_bytes_for(uint32_t ns, uint32_t nh) {
     return kHRegion + s_region_bytes(ns) + uint32_t(chunks_per_cta(ns, nh)) * (kRingBytes + kNibRingBytes);
+}
+inline uint32_t smem_bytes_for(uint32_t ns, uint32_t warps, uint32_t chains) {
+    return kHRegion + s_region_bytes(ns) + warps * chains * (kRingBytes + kNibRingBytes);
 }
 
 // Workspace layout: a 256-byte error block, then 256-aligned tables per RANS tensor.
@@ -116,6 +128,7 @@ struct DecodeParams {
     // opaque to the compiler, so those steps run as IMAD on the FMA pipe (which has spare
     // issue slots) instead of becoming shifts on the integer ALU pipe, the kernel's bound.
     uint32_t mul2 = 2, mul65536 = 65536;
+    uint32_t warps = 0; // warps per CTA of this launch (at most the kernel's WARPS)
     DecodeItem item[kMaxDecodeItems];
 };
 

@@ -249,7 +249,14 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
     // --- the decode kernel, unchanged, with its tables and error block in the array ---
     DecodeParams p; // about 31 KiB of launch parameters, on the stack (no heap use)
     p.n_items = 1;
-    const uint64_t per_cta = chunks_per_cta(ns, nh);
+    const bool dflt = is_default_precision(ns, nh);
+    const uint32_t chains = dflt ? kChainsDefault : kChainsGeneric;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        sms = 148;
+    p.warps = launch_warps(n_chunks, dflt ? kWarpsDefault : kWarpsGeneric, chains, static_cast<uint32_t>(sms));
+    const uint64_t per_cta = uint64_t(p.warps) * chains;
     p.total_ctas = static_cast<uint32_t>((n_chunks + per_cta - 1) / per_cta);
     p.err = reinterpret_cast<unsigned long long*>(scratch);
     DecodeItem& it = p.item[0];
@@ -267,7 +274,7 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
     it.nh = static_cast<uint8_t>(nh);
     it.n_routes = static_cast<uint8_t>(n_routes);
     it.nib_mode = static_cast<uint8_t>(nib_mode);
-    int e = launch_decode(p, is_default_precision(ns, nh), smem_bytes_for(ns, nh), stream);
+    int e = launch_decode(p, dflt, smem_bytes_for(ns, p.warps, chains), stream);
     if (e) {
         record_cuda_error(e);
         return BS_E_CUDA;

@@ -310,6 +310,10 @@ bs_status DecodeBatch::init() {
         bins_[k].p->total_ctas = 0;
         bins_[k].p->err = err_;
     }
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+        sms_ = static_cast<uint32_t>(sms);
     cp_.reset(new (std::nothrow) CopyParams);
     if (!cp_) return BS_E_NOMEM;
     cp_->n_items = 0;
@@ -317,12 +321,28 @@ bs_status DecodeBatch::init() {
     return BS_OK;
 }
 
+// Chooses the CTA shape for the queued chunks, assigns each item its CTA range and launches.
 bs_status DecodeBatch::flush_bin(Bin& b, void* stream) {
-    if (b.p->n_items == 0) return BS_OK;
-    const int e = launch_decode(*b.p, b.default_precision, b.smem, stream);
-    b.p->n_items = 0;
-    b.p->total_ctas = 0;
-    b.smem = 0;
+    DecodeParams& p = *b.p;
+    if (p.n_items == 0) return BS_OK;
+    const uint32_t max_warps = b.default_precision ? kWarpsDefault : kWarpsGeneric;
+    const uint32_t chains = b.default_precision ? kChainsDefault : kChainsGeneric;
+    p.warps = launch_warps(b.chunks, max_warps, chains, sms_);
+    const uint64_t per_cta = uint64_t(p.warps) * chains;
+    uint64_t ctas = 0;
+    for (uint32_t k = 0; k < p.n_items; ++k) {
+        DecodeItem& it = p.item[k];
+        const uint64_t C = 1ull << it.log2_chunk, n_chunks = (it.n_elems + C - 1) / C;
+        it.cta_begin = static_cast<uint32_t>(ctas);
+        ctas += (n_chunks + per_cta - 1) / per_cta;
+    }
+    p.total_ctas = static_cast<uint32_t>(ctas); // at most 2^31 / 8 + kMaxDecodeItems (see add)
+    const int e = launch_decode(p, b.default_precision, kHRegion + b.s_region + p.warps * chains * (kRingBytes + kNibRingBytes),
+                                stream);
+    p.n_items = 0;
+    p.total_ctas = 0;
+    b.s_region = 0;
+    b.chunks = 0;
     return e ? cuda_status(e) : BS_OK;
 }
 
@@ -339,9 +359,8 @@ bs_status DecodeBatch::add(const Tensor& t, uint32_t tensor_index, const uint8_t
     if (t.kind == BS_KIND_RANS) {
         const bool dflt = is_default_precision(t.ns, t.nh);
         Bin& b = bins_[dflt ? 0 : 1];
-        const uint64_t per_cta = chunks_per_cta(t.ns, t.nh);
-        const uint64_t ctas = (t.n_chunks + per_cta - 1) / per_cta;
-        if (b.p->n_items == kMaxDecodeItems || b.p->total_ctas + ctas > 0x7FFFFFFFull) {
+        // the smallest CTA holds kMinWarps * 2 chunks, so 2^31 chunks keep the grid below 2^31 CTAs
+        if (b.p->n_items == kMaxDecodeItems || b.chunks + t.n_chunks > (1ull << 31)) {
             bs_status s = flush_bin(b, stream);
             if (s) return s;
         }
@@ -352,7 +371,6 @@ bs_status DecodeBatch::add(const Tensor& t, uint32_t tensor_index, const uint8_t
         it.tables = reinterpret_cast<const uint4*>(d_ws + t.ws_offset);
         it.out = static_cast<uint16_t*>(d_out);
         it.n_elems = t.n_elems;
-        it.cta_begin = b.p->total_ctas;
         it.tensor_index = tensor_index;
         it.table_bytes = t.table_bytes;
         it.log2_chunk = static_cast<uint8_t>(t.log2_chunk);
@@ -360,8 +378,8 @@ bs_status DecodeBatch::add(const Tensor& t, uint32_t tensor_index, const uint8_t
         it.nh = static_cast<uint8_t>(t.nh);
         it.n_routes = static_cast<uint8_t>(t.n_routes);
         it.nib_mode = static_cast<uint8_t>(t.nib_mode);
-        b.p->total_ctas += static_cast<uint32_t>(ctas);
-        b.smem = std::max<uint32_t>(b.smem, smem_bytes_for(t.ns, t.nh));
+        b.chunks += t.n_chunks;
+        b.s_region = std::max<uint32_t>(b.s_region, s_region_bytes(t.ns));
     } else if (t.n_elems) {
         const uint64_t bytes = t.kind == BS_KIND_RAW ? t.n_elems : 2 * t.n_elems;
         const uint64_t blks = (bytes + kCopyBlockBytes - 1) / kCopyBlockBytes;
