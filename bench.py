@@ -12,7 +12,8 @@ bit-exact against the originals before timing. The JSON line carries:
 * roofline   (compressed bytes read + BF16 bytes written) per decode step over the step's
              CUDA-event time, against the measured HBM copy bandwidth
 * e2e        the same metric with the container copied in from pinned host memory and
-             every decoded tensor copied back out, inside the timed region
+             every decoded tensor copied back out, inside the timed region; the copies
+             and decodes of successive layer groups overlap on three streams
 * cpu_baseline  the oracle decoder on the host cores, on a bounded sample (layer 0)
 
 `--impl reference` times the oracle alone (host cores, rank 0) on the same sample.
@@ -344,30 +345,58 @@ def run_ours(a):
     tpw = _traffic_per_weight()
     achieved = (coded + out_bytes) / (mean_step * 1e-3) / 1e9
 
-    # end to end: container in from pinned host memory, every tensor back out, per step
+    # end to end: container in from pinned host memory, every tensor back out, per step,
+    # pipelined per layer group over three streams (the public Plan.decode_batch per group)
     e2e = None
     if not a.no_e2e and a.e2e_steps > 0:
         h_c = torch.empty(d_c.numel(), dtype=torch.uint8, pin_memory=True)
         h_c.copy_(d_c)
         h_outs = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+        ranges, members = _group_ranges(h_c.numpy(), plan.names)
         torch.cuda.synchronize()
         barrier()
+        s_in, s_dec, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        n_g = len(members)
+        done_out = [None] * n_g     # event: the previous step's copy-out of group g finished
+        done_dec = [None] * n_g     # event: the previous step's decode of group g finished
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
+        for st in (s_in, s_dec, s_out):
+            st.wait_event(e0)
         for _ in range(a.e2e_steps):
-            d_c.copy_(h_c, non_blocking=True)
-            plan.decode_batch(idx, outs, stream=stream)
-            for o, h in zip(outs, h_outs):
-                h.copy_(o, non_blocking=True)
+            for g in range(n_g):
+                lo, hi = ranges[g]
+                if done_dec[g] is not None:   # do not overwrite bytes a decode may still read
+                    s_in.wait_event(done_dec[g])
+                with torch.cuda.stream(s_in):
+                    d_c[lo:hi].copy_(h_c[lo:hi], non_blocking=True)
+                    arrived = torch.cuda.Event()
+                    arrived.record(s_in)
+                s_dec.wait_event(arrived)
+                if done_out[g] is not None:
+                    s_dec.wait_event(done_out[g])
+                plan.decode_batch(members[g], [outs[k] for k in members[g]], stream=s_dec)
+                decoded = torch.cuda.Event()
+                decoded.record(s_dec)
+                done_dec[g] = decoded
+                s_out.wait_event(decoded)
+                with torch.cuda.stream(s_out):
+                    for k in members[g]:
+                        h_outs[k].copy_(outs[k], non_blocking=True)
+                    done_out[g] = torch.cuda.Event()
+                    done_out[g].record(s_out)
+        for st in (s_in, s_dec, s_out):
+            stream.wait_stream(st)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
         plan.check()
         e_ms = ranks.max(e0.elapsed_time(e1))
         e2e = {"value": round(world * a.e2e_steps * out_bytes / (e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
-               "h2d_bytes_per_step": int(d_c.numel()), "d2h_bytes_per_step": int(out_bytes),
-               "steps": a.e2e_steps, "path": "Plan.decode_batch with the container copied in from pinned host "
-                                             "memory and every tensor copied back, per step"}
+               "h2d_bytes_per_step": int(sum(hi - lo for lo, hi in ranges)), "d2h_bytes_per_step": int(out_bytes),
+               "steps": a.e2e_steps, "groups": n_g,
+               "path": "per layer group: its container bytes copied in from pinned host memory, "
+                       "Plan.decode_batch, its tensors copied back out; three streams overlap the groups"}
         del h_c, h_outs
 
     cpu = None
@@ -422,6 +451,38 @@ def _group_of(name: str):
 def _groups(names):
     keys = {}
     return [keys.setdefault(_group_of(n), len(keys)) for n in names]
+
+
+def _group_ranges(h: "np.ndarray", names):
+    """Per layer group, the contiguous container bytes its tensors use and its member indices.
+
+    FORMAT.md 4.2 and 4.6: the canonical layout writes each tensor's sections (RANS: model,
+    chunk table, chunks; else the data) in directory order, each tensor starting at its
+    model_offset (RANS) or data_offset. A group's tensors are consecutive, so its bytes run
+    from its first tensor's start to the next group's start (or the end of the container)."""
+    import numpy as np
+    hdr = h[:64].tobytes()
+    nt = int.from_bytes(hdr[16:20], "little")
+    d0 = int.from_bytes(hdr[24:32], "little")
+    total = int.from_bytes(hdr[48:56], "little")
+    starts = []
+    for k in range(nt):
+        e = h[d0 + 144 * k: d0 + 144 * k + 144].tobytes()
+        kind = e[0]
+        model_off, data_off = int.from_bytes(e[32:40], "little"), int.from_bytes(e[48:56], "little")
+        starts.append(model_off if kind == 0 else data_off)
+    gid = _groups(names)
+    members, ranges = [], []
+    for k in range(nt):
+        if k == 0 or gid[k] != gid[k - 1]:
+            members.append([])
+        members[-1].append(k)
+    for g, m in enumerate(members):
+        lo = starts[m[0]]
+        hi = starts[members[g + 1][0]] if g + 1 < len(members) else total
+        assert all(starts[k] >= lo for k in m) and hi >= lo
+        ranges.append((lo, hi))
+    return ranges, members
 
 
 def _setup(a, dev):

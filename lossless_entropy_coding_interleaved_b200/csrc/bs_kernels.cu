@@ -265,8 +265,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
                 const uint32_t xr = xn[k] * mul65536 + w[k]; // (xn << 16) | w as one IMAD, computed by every lane
                 h.x = need[k] ? xr : xn[k];
                 h.posb += __popc(m[k]) * mul2;
-                // (s << 7) | (h << 4): s sits pre-shifted in se.y, h in bits 4-6 of fe
-                const uint32_t word = (se[k].y & 0xFF80u) | (fe[k] & 0x70u);
+                // (s << 7) | (h << 4): s sits pre-shifted in se.y, h in bits 4-6 of fe, and the
+                // rest of fe's low half is zero, so one masked select builds the low half (the
+                // high half is dropped when the pair is packed)
+                const uint32_t word = (se[k].y & 0xFF80u) | fe[k];
                 if (s & 1) o[k][s >> 1] = __byte_perm(o[k][s >> 1], word, 0x5410);
                 else o[k][s >> 1] = word;
             }
