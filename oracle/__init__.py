@@ -22,6 +22,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "bsoracle.c")
+_SRCS = (_SRC, os.path.join(_HERE, "fworacle.c"))
 _LIB = os.path.join(_HERE, "libbsoracle.so")
 
 OK, E_ARG, E_FORMAT, E_VERSION, E_SIZE, E_CORRUPT, E_NOMEM = 0, 1, 2, 3, 4, 6, 7
@@ -36,10 +37,11 @@ class OracleError(RuntimeError):
 
 
 def build(force: bool = False) -> str:
-    """Compile bsoracle.c into libbsoracle.so next to it (plain gcc, no GPU code)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    """Compile bsoracle.c and fworacle.c into libbsoracle.so next to them (plain gcc, no GPU code)."""
+    stale = not os.path.exists(_LIB) or any(os.path.getmtime(_LIB) < os.path.getmtime(f) for f in _SRCS)
+    if force or stale:
         tmp = _LIB + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", "-O2", "-std=c11", "-Wall", "-shared", "-fPIC", _SRC, "-o", tmp])
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-Wall", "-shared", "-fPIC", *_SRCS, "-o", tmp])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -70,6 +72,11 @@ class _Info(ctypes.Structure):
                [("shape", ctypes.c_uint64 * 8), ("coded_bytes", ctypes.c_uint64)]
 
 
+class _FwInfo(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_uint64) for k in ("n_elems", "n_tiles", "n_exc", "total_bytes")] + \
+               [("table", ctypes.c_uint16 * 16)]
+
+
 _lib = None
 
 
@@ -91,12 +98,19 @@ def lib():
         L.bso_lane_encode.argtypes = [P, u32, P, P, u32, u32, P, u32, ctypes.POINTER(u32), P, P,
                                       ctypes.POINTER(u32)]
         L.bso_lane_decode.argtypes = [P, u32, P, P, u32, u32, u32, P, u32, P, u32, P, ctypes.POINTER(u32)]
+        L.bso_fw_bytes.argtypes = [u64, u64]
+        L.bso_fw_bytes.restype = u64
+        L.bso_fw_table.argtypes = [P, u64, P, ctypes.POINTER(u32)]
+        L.bso_fw_encode.argtypes = [P, u64, P, u64, ctypes.POINTER(u64)]
+        L.bso_fw_parse.argtypes = [P, u64, ctypes.POINTER(_FwInfo)]
+        L.bso_fw_decode.argtypes = [P, u64, P, u64]
         L.bso_mix64.argtypes = [u64]
         L.bso_mix64.restype = u64
         L.bso_checksum.argtypes = [P, u64, u32]
         L.bso_checksum.restype = u64
         for fn in ("bso_encode", "bso_validate", "bso_tensor_info_get", "bso_decode", "bso_decode_chunks",
-                   "bso_quantise", "bso_choose_routes", "bso_lane_encode", "bso_lane_decode"):
+                   "bso_quantise", "bso_choose_routes", "bso_lane_encode", "bso_lane_decode", "bso_fw_table",
+                   "bso_fw_encode", "bso_fw_parse", "bso_fw_decode"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -262,3 +276,60 @@ def checksum(a: np.ndarray) -> int:
     """FORMAT.md section 7 checksum of uint16 words or uint8 bytes."""
     a = np.ascontiguousarray(a).reshape(-1)
     return int(lib().bso_checksum(_ptr(a), a.size, 2 if a.dtype == np.uint8 else 0))
+
+
+# ------------------------------------------------------------ fixed-width lane layout
+# FORMAT.md section 10; the arithmetic is in fworacle.c.
+def fw_bytes(n_elems: int, n_exc: int) -> int:
+    """Size of the FW layout of n_elems weights with n_exc escapes."""
+    return int(lib().bso_fw_bytes(n_elems, n_exc))
+
+
+def fw_table(words) -> tuple[list[int], int]:
+    """(code table of 16 entries, number of codes used) for uint16 words."""
+    w = np.ascontiguousarray(words, dtype=np.uint16).reshape(-1)
+    t = np.zeros(16, np.uint16)
+    k = ctypes.c_uint32()
+    st = lib().bso_fw_table(_ptr(w), w.size, _ptr(t), ctypes.byref(k))
+    if st:
+        raise OracleError(st, "fw_table")
+    return [int(v) for v in t], k.value
+
+
+def fw_encode(words) -> bytes:
+    """The FW layout of uint16 words (any shape, flattened)."""
+    w = np.ascontiguousarray(words, dtype=np.uint16).reshape(-1)
+    size = ctypes.c_uint64()
+    st = lib().bso_fw_encode(_ptr(w), w.size, None, 0, ctypes.byref(size))
+    if st:
+        raise OracleError(st, "fw_encode")
+    out = np.zeros(max(size.value, 1), np.uint8)
+    st = lib().bso_fw_encode(_ptr(w), w.size, _ptr(out), out.size, ctypes.byref(size))
+    if st:
+        raise OracleError(st, "fw_encode")
+    return out[: size.value].tobytes()
+
+
+def fw_info(blob) -> dict:
+    """Header fields of an FW layout (validated against its size)."""
+    arr, n = _buf(blob)
+    info = _FwInfo()
+    st = lib().bso_fw_parse(_ptr(arr), n, ctypes.byref(info))
+    if st:
+        raise OracleError(st, "fw_parse")
+    return {"n_elems": info.n_elems, "n_tiles": info.n_tiles, "n_exc": info.n_exc,
+            "total_bytes": info.total_bytes, "table": [int(v) for v in info.table]}
+
+
+def fw_decode(blob) -> np.ndarray:
+    """Decode an FW layout into uint16 words; raises OracleError on a malformed one."""
+    arr, n = _buf(blob)
+    info = _FwInfo()
+    st = lib().bso_fw_parse(_ptr(arr), n, ctypes.byref(info))
+    if st:
+        raise OracleError(st, "fw_parse")
+    out = np.zeros(max(info.n_elems, 1), np.uint16)
+    st = lib().bso_fw_decode(_ptr(arr), n, _ptr(out), info.n_elems)
+    if st:
+        raise OracleError(st, "fw_decode")
+    return out[: info.n_elems].copy()
