@@ -53,10 +53,11 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-threads", type=int, default=0, help="oracle threads (0: all host cores)")
-    ap.add_argument("--mode", choices=["model", "layerwise", "stream"], default="model",
+    ap.add_argument("--mode", choices=["model", "layerwise", "stream", "fw"], default="model",
                     help="model: one bs_decode_batch of every tensor per step (the default line); "
                          "layerwise: one bs_decode_batch per layer (group) per step; "
-                         "stream: layer streaming from a host container through the LRU device cache")
+                         "stream: layer streaming from a host container through the LRU device cache; "
+                         "fw: one bs_fw_decode of every tensor's fixed-width lane layout per step")
     ap.add_argument("--vram-gb", type=float, default=None,
                     help="stream mode: device budget (arena) in GB; default: the smallest arena that "
                          "double-buffers the largest group")
@@ -71,14 +72,14 @@ def _peak_hbm():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def _traffic_per_weight():
-    """DRAM bytes per weight of decode_kernel from the committed ncu summary, if the kernel
+def _traffic_per_weight(profile="decode_kernel_gemma2_9b.md", sources=("bs_kernels.cu", "bs_internal.h")):
+    """DRAM bytes per weight of a kernel from its committed ncu summary, if the kernel
     sources still hash to what was profiled; else None."""
     import hashlib
     csrc = os.path.join(ROOT, "lossless_entropy_coding_interleaved_b200", "csrc")
     try:
-        src = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("bs_kernels.cu", "bs_internal.h"))
-        lines = open(os.path.join(ROOT, "profiles", "decode_kernel_gemma2_9b.md")).read().splitlines()
+        src = b"".join(open(os.path.join(csrc, f), "rb").read() for f in sources)
+        lines = open(os.path.join(ROOT, "profiles", profile)).read().splitlines()
     except OSError:
         return None
     kv = dict(l.split(": ", 1) for l in lines if l.startswith(("kernel_sha256: ", "traffic_bytes_per_weight: ")))
@@ -252,6 +253,30 @@ def run_reference(a):
                              "sample": sample},
             "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def run_fw_reference(a):
+    """--impl reference --mode fw: the oracle's FW decode alone on the host cores (rank 0)."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    threads = _cpu_threads(a.cpu_threads)
+    _, n_all, desc = _workload_desc(a.workload, a.layers)
+    n, sample, run_once = _fw_oracle_sample(a.workload, threads)
+    with cf.ThreadPoolExecutor(threads) as pool:
+        for _ in range(a.warmup):
+            run_once(pool)
+        sec = sum(run_once(pool) for _ in range(a.steps))
+    value = 2 * n * a.steps / sec / 1e9
+    print(json.dumps({
+        "impl": "reference", "metric": FW_METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": a.gpus,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(1e3 * sec / a.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
+        "config": {"workload": a.workload, "description": desc, "n_weights": n_all,
+                   "step": "one bounded sample per step: " + sample},
+        "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+        flush=True)
 
 
 # ------------------------------------------------------------------ our arm
@@ -704,10 +729,196 @@ def run_stream(a):
         "gpu_launches": int(launches), "clocks": clk}), flush=True)
 
 
+# ------------------------------------------------------------------ fixed-width lane layout
+FW_METRIC = "decompressed BF16 GB/s from the fixed-width lane layout (full model, 1 B200) and % HBM roofline"
+
+
+def _fw_oracle_sample(workload, threads):
+    """The bounded CPU sample of the FW mode: layer 0 of the workload, laid out and decoded
+    by the oracle (one tensor per task on `threads` host threads)."""
+    import numpy as np
+    import oracle
+    import synthetic as S
+    specs = [s for s in S.workload(workload, layers=1) if not s.is_raw]
+    if workload in ("gemma2_9b", "qwen_27b_scale"):
+        specs = [s for s in specs if s.name.startswith("layers.0.")]
+    arrs = [S.words_numpy(S.generate(s, "cpu")).reshape(-1) for s in specs]
+    with cf.ThreadPoolExecutor(threads) as pool:
+        blobs = list(pool.map(oracle.fw_encode, arrs))
+    n = sum(a.size for a in arrs)
+    desc = f"oracle FW decode of layer 0 of {workload} ({len(specs)} tensors, {n} weights) on {threads} host threads"
+
+    def run_once(pool):
+        t0 = time.perf_counter()
+        outs = list(pool.map(oracle.fw_decode, blobs))
+        sec = time.perf_counter() - t0
+        assert all(np.array_equal(a, o) for a, o in zip(arrs, outs)), "oracle FW sample mismatch"
+        return sec
+
+    return n, desc, run_once
+
+
+def run_fw(a):
+    """Decode every BF16 tensor of the workload from its fixed-width lane layout (one
+    bs_fw_decode per step); layouts and outputs resident in HBM."""
+    import torch
+
+    import lossless_entropy_coding_interleaved_b200 as bs
+    import synthetic as S
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = _Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    specs, _, desc = _workload_desc(a.workload, a.layers)
+    specs = [s for s in specs if not s.is_raw]
+    originals = [S.generate(s, dev).reshape(-1) for s in specs]
+    torch.cuda.synchronize()
+    t0 = time.time()
+    built = [bs.fw_transcode(w) for w in originals]
+    torch.cuda.synchronize()
+    t_transcode = time.time() - t0
+    fws = [f for f, _ in built]
+    infos = [i for _, i in built]
+    n = sum(i.n_elems for i in infos)
+    n_exc = sum(i.n_exc for i in infos)
+    fw_bytes = sum(i.total_bytes for i in infos)
+    out_bytes = 2 * n
+    outs = [torch.empty_like(w) for w in originals]
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(1, a.warmup)):
+        bs.fw_decode(fws, infos, outs, err, stream=stream)
+    torch.cuda.synchronize()
+    if int(err.item()) != 0 or not all(torch.equal(o, w) for o, w in zip(outs, originals)):
+        raise SystemExit("bench: FW decode differs from the originals")
+    del originals
+    torch.cuda.empty_cache()
+
+    phys = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+    smi_index = phys[local] if local < len(phys) and phys[local].strip().isdigit() else str(local)
+    clocks = _Clocks(smi_index)
+    time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+    l0 = bs.launch_counter()
+    it = iter(ev)
+
+    def step():
+        e0, e1 = next(it)
+        e0.record(stream)
+        bs.fw_decode(fws, infos, outs, err, stream=stream)
+        e1.record(stream)
+
+    total_ms = ranks.max(_timed(stream, a.steps, step, ranks.barrier))
+    launches = bs.launch_counter() - l0
+    clk = clocks.stop()
+    if int(err.item()) != 0:
+        raise SystemExit("bench: FW decode raised its error flag")
+    mean_step = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    value = world * a.steps * out_bytes / (total_ms * 1e-3) / 1e9
+    peak, peak_kind = _peak_hbm()
+    achieved = (fw_bytes + out_bytes) / (mean_step * 1e-3) / 1e9
+    tpw = _traffic_per_weight("fw_decode_kernel_gemma2_9b.md", ("bs_fw.cu",))
+
+    # end to end: every layout copied in from pinned host memory and every output copied back,
+    # per layer group on three streams so that the copies of one group overlap the others
+    e2e = None
+    if not a.no_e2e and a.e2e_steps > 0:
+        h_fw = [torch.empty(f.shape, dtype=f.dtype, pin_memory=True) for f in fws]
+        for h, f in zip(h_fw, fws):
+            h.copy_(f)
+        h_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+        gid = _groups([s.name for s in specs])
+        members = {}
+        for k, g in enumerate(gid):
+            members.setdefault(g, []).append(k)
+        members = list(members.values())
+        torch.cuda.synchronize()
+        ranks.barrier()
+        s_in, s_dec, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        done_dec, done_out = [None] * len(members), [None] * len(members)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for st in (s_in, s_dec, s_out):
+            st.wait_event(e0)
+        for _ in range(a.e2e_steps):
+            for g, m in enumerate(members):
+                if done_dec[g] is not None:
+                    s_in.wait_event(done_dec[g])
+                with torch.cuda.stream(s_in):
+                    for k in m:
+                        fws[k].copy_(h_fw[k], non_blocking=True)
+                    arrived = torch.cuda.Event()
+                    arrived.record(s_in)
+                s_dec.wait_event(arrived)
+                if done_out[g] is not None:
+                    s_dec.wait_event(done_out[g])
+                bs.fw_decode([fws[k] for k in m], [infos[k] for k in m], [outs[k] for k in m], err, stream=s_dec)
+                decoded = torch.cuda.Event()
+                decoded.record(s_dec)
+                done_dec[g] = decoded
+                s_out.wait_event(decoded)
+                with torch.cuda.stream(s_out):
+                    for k in m:
+                        h_out[k].copy_(outs[k], non_blocking=True)
+                    done_out[g] = torch.cuda.Event()
+                    done_out[g].record(s_out)
+        for st in (s_in, s_dec, s_out):
+            stream.wait_stream(st)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ranks.barrier()
+        if int(err.item()) != 0:
+            raise SystemExit("bench: FW decode raised its error flag (e2e)")
+        e_ms = ranks.max(e0.elapsed_time(e1))
+        e2e = {"value": round(world * a.e2e_steps * out_bytes / (e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": int(fw_bytes), "d2h_bytes_per_step": int(out_bytes), "steps": a.e2e_steps,
+               "groups": len(members),
+               "path": "per layer group: its layouts copied in from pinned host memory, bs_fw_decode, "
+                       "its tensors copied back out; three streams overlap the groups"}
+        del h_fw, h_out
+
+    cpu = None
+    if rank == 0 and not a.no_cpu_baseline:
+        threads = _cpu_threads(a.cpu_threads)
+        n_s, sample, run_once = _fw_oracle_sample(a.workload, threads)
+        with cf.ThreadPoolExecutor(threads) as pool:
+            run_once(pool)
+            sec = run_once(pool)
+        cpu = {"value": round(2 * n_s / sec / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": sample}
+    ranks.close()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": FW_METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": round(total_ms / a.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u32",
+        "data": "synthetic (seeded device draws, synthetic/ recipe)",
+        "config": {"workload": a.workload, "description": desc, "n_weights": n, "tensors": len(specs),
+                   "layout": "fixed-width lane layout (FORMAT.md section 10)",
+                   "fw_bytes": int(fw_bytes), "decoded_bytes": int(out_bytes), "escapes": int(n_exc),
+                   "bits_per_weight": round(8 * fw_bytes / n, 5), "transcode_s": round(t_transcode, 3),
+                   "parallelism": f"replicas x{world} (no collective on the data path)",
+                   "l2": "no flush: inputs larger than L2 (layouts and outputs are GBs)",
+                   "parity": "bit-exact vs originals before timing; error word checked after"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": (None if tpw is None else int(tpw * n)),
+                     "traffic_source": "profiles/fw_decode_kernel_gemma2_9b.md (capture scaled by weights)",
+                     "kernel": "fw_decode_kernel", "per_launch_bytes": int(fw_bytes + out_bytes),
+                     "launch_ms_mean": round(mean_step, 4)},
+        "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": int(launches), "clocks": clk}), flush=True)
+
+
 def main():
     a = _args()
-    if a.impl == "reference":
+    if a.impl == "reference" and a.mode == "fw":
+        run_fw_reference(a)
+    elif a.impl == "reference":
         run_reference(a)
+    elif a.mode == "fw":
+        run_fw(a)
     elif a.mode == "layerwise":
         run_layerwise(a)
     elif a.mode == "stream":

@@ -295,6 +295,61 @@ bs_status bs_streamer_check(bs_streamer_t* s, void* stream, int64_t* first_bad);
 /* Frees host state only. It does not synchronise: finish the streams before freeing the arena. */
 void bs_streamer_destroy(bs_streamer_t* s);
 
+/* ------------------------------------------------------------------------------------
+ * Fixed-width lane layout ("FW layout", FORMAT.md section 10): a runtime form of one BF16
+ * tensor whose decode is a few bitwise operations per weight. The "Qwen3.8-27B-BF16-NVLC-
+ * Lossless" card says its GPU runtime derives fixed-width, lane-oriented streams from the
+ * rANS files once at initialisation (its Fixed7/Compact11 runtime, about 11.36 bits per
+ * weight resident). The card gives no layout; section 10 is this library's:
+ *   - a 4-bit code per weight for the tensor's 16 most frequent sign+exponent symbols;
+ *   - the 7-bit fraction in two planes;
+ *   - an exception list of (position, word) for the other symbols.
+ * Tiles of 256 weights: lane j of a warp owns 8 consecutive weights. The size is 11.125
+ * bits per weight plus 24 bits per escape, about 11.4 on Gaussian-shaped weights.
+ *
+ * Building one (on the device, from BF16 words that stay unchanged between the calls):
+ *   1. bs_fw_measure: statistics, code table and escape counts into caller scratch;
+ *      synchronises the stream and returns the layout's size in info->total_bytes;
+ *   2. bs_fw_write: writes the layout into caller device memory; synchronises the stream.
+ * Decoding: bs_fw_decode, enqueued on the stream without a sync. All device memory belongs
+ * to the caller. The library allocates none.
+ * ------------------------------------------------------------------------------------ */
+typedef struct {
+    uint64_t n_elems;     /* weights */
+    uint64_t n_tiles;     /* ceil(n_elems / 256) */
+    uint64_t n_exc;       /* escaped weights, below 2^32 */
+    uint64_t total_bytes; /* size of the layout in bytes (a multiple of 16) */
+    uint16_t table[16];   /* the sign+exponent symbol of each code */
+} bs_fw_info;
+
+/* Device scratch bytes of bs_fw_measure / bs_fw_write for n_elems weights (0 if n_elems > 2^40). */
+size_t bs_fw_scratch_bytes(uint64_t n_elems);
+/* d_in: n_elems BF16 words on the device, 16-byte aligned. d_scratch: 256-byte aligned,
+ * at least bs_fw_scratch_bytes(n_elems). Synchronises stream and fills *info.
+ * BS_E_SIZE if the scratch is short, n_elems > 2^40, or 2^32 or more weights would escape.
+ * BS_E_UNSUPPORTED off sm_100. */
+bs_status bs_fw_measure(const void* d_in, uint64_t n_elems, void* d_scratch, size_t scratch_bytes, void* stream,
+                        bs_fw_info* info);
+/* Writes the layout described by *info (from bs_fw_measure on the same d_in and d_scratch)
+ * into d_fw: fw_bytes == info->total_bytes bytes of device memory, 16-byte aligned.
+ * Synchronises stream. BS_E_CORRUPT if the input changed since bs_fw_measure. */
+bs_status bs_fw_write(const void* d_in, uint64_t n_elems, void* d_scratch, size_t scratch_bytes,
+                      const bs_fw_info* info, void* d_fw, size_t fw_bytes, void* stream);
+/* Validates a host copy of a layout's first 96 bytes (header and code table) against the
+ * layout's size fw_bytes, and fills *info. BS_E_FORMAT or BS_E_VERSION on a bad header. */
+bs_status bs_fw_parse(const void* h_head, size_t head_bytes, size_t fw_bytes, bs_fw_info* info);
+/* Decodes n layouts in as few launches as possible (up to 480 layouts per launch).
+ *   d_fw[k]: layout k on the device, 16-byte aligned, infos[k] its header (from
+ *            bs_fw_measure or bs_fw_parse);
+ *   d_out[k]: infos[k].n_elems words, 16-byte aligned, out_bytes[k] == 2 * n_elems;
+ *   d_err: a device word the caller zeroes before and reads after. An exception list that
+ *          fails its checks sets bit 0: tile_exc not ascending or past n_exc within a group of
+ *          4 tiles (the group's exceptions are then skipped), or a position past the tensor
+ *          (that exception is skipped). Nothing is written outside d_out[k].
+ * Enqueued on stream; returns BS_E_ARG / BS_E_SIZE for bad arguments before any launch. */
+bs_status bs_fw_decode(int32_t n, const void* const* d_fw, const bs_fw_info* infos, void* const* d_out,
+                       const size_t* out_bytes, uint32_t* d_err, void* stream);
+
 const char* bs_status_str(bs_status s);
 int bs_last_cuda_error(void); /* the cudaError_t behind the last BS_E_CUDA on this thread */
 /* Kernel launches libbs has made in this process (all threads); a diagnostic counter. */

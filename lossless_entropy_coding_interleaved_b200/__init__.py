@@ -59,6 +59,16 @@ class _EncParams(ctypes.Structure):
     _fields_ = [(k, ctypes.c_uint32) for k in ("log2_chunk", "ns", "nh", "max_routes", "force_rans")]
 
 
+class FwInfo(ctypes.Structure):
+    """bs_fw_info: the header of a fixed-width lane layout (FORMAT.md section 10)."""
+    _fields_ = [("n_elems", ctypes.c_uint64), ("n_tiles", ctypes.c_uint64), ("n_exc", ctypes.c_uint64),
+                ("total_bytes", ctypes.c_uint64), ("table", ctypes.c_uint16 * 16)]
+
+    def __repr__(self):
+        return (f"FwInfo(n_elems={self.n_elems}, n_tiles={self.n_tiles}, n_exc={self.n_exc}, "
+                f"total_bytes={self.total_bytes}, table={list(self.table)})")
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libbs.so is not built ({LIB_PATH}); run "
@@ -105,6 +115,14 @@ def _load():
     L.bs_streamer_check.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
     L.bs_streamer_destroy.argtypes = [P]
     L.bs_streamer_destroy.restype = None
+    L.bs_fw_scratch_bytes.argtypes = [u64]
+    L.bs_fw_scratch_bytes.restype = sz
+    L.bs_fw_measure.argtypes = [P, u64, P, sz, P, ctypes.POINTER(FwInfo)]
+    L.bs_fw_write.argtypes = [P, u64, P, sz, ctypes.POINTER(FwInfo), P, sz, P]
+    L.bs_fw_parse.argtypes = [P, sz, sz, ctypes.POINTER(FwInfo)]
+    L.bs_fw_decode.argtypes = [i32, P, P, P, P, P, P]
+    for fn in ("bs_fw_measure", "bs_fw_write", "bs_fw_parse", "bs_fw_decode"):
+        getattr(L, fn).restype = ctypes.c_int
     for fn in ("bs_streamer_create", "bs_streamer_group_count", "bs_streamer_tensor_info_get", "bs_streamer_prefetch", "bs_streamer_acquire",
                "bs_streamer_release", "bs_streamer_get_stats", "bs_streamer_check"):
         getattr(L, fn).restype = ctypes.c_int
@@ -125,7 +143,8 @@ EXPORTS = ("bs_plan_workspace_bytes", "bs_plan_workspace_bytes_device", "bs_plan
            "bs_decode_tensor_noalloc", "bs_streamer_workspace_bytes", "bs_streamer_min_arena_bytes",
            "bs_streamer_create", "bs_streamer_group_count", "bs_streamer_tensor_info_get", "bs_streamer_prefetch",
            "bs_streamer_acquire",
-           "bs_streamer_release", "bs_streamer_get_stats", "bs_streamer_check", "bs_streamer_destroy")
+           "bs_streamer_release", "bs_streamer_get_stats", "bs_streamer_check", "bs_streamer_destroy",
+           "bs_fw_scratch_bytes", "bs_fw_measure", "bs_fw_write", "bs_fw_parse", "bs_fw_decode")
 
 
 def decode_noalloc(container, d_container: torch.Tensor, idx: int, out: torch.Tensor, stream=None) -> torch.Tensor:
@@ -469,3 +488,55 @@ class Streamer:
             raise BsError(st, "streamer_check", "corrupt chunk", first_bad=fb.value)
         _check(st, "streamer_check")
         return fb.value
+
+
+# ------------------------------------------------------------ fixed-width lane layout
+def _words(t: torch.Tensor) -> torch.Tensor:
+    assert t.is_cuda and t.is_contiguous() and t.element_size() == 2, "BF16 words: a contiguous 2-byte CUDA tensor"
+    return t
+
+
+def fw_scratch_bytes(n_elems: int) -> int:
+    return int(lib.bs_fw_scratch_bytes(n_elems))
+
+
+def fw_transcode(words: torch.Tensor, stream=None) -> tuple[torch.Tensor, FwInfo]:
+    """Build the fixed-width lane layout of BF16 words on their device (bs_fw_measure, then
+    bs_fw_write). Returns (layout as a uint8 CUDA tensor, its FwInfo). Synchronises the stream."""
+    w = _words(words)
+    n = w.numel()
+    scratch = torch.empty(max(fw_scratch_bytes(n), 256), dtype=torch.uint8, device=w.device)
+    info = FwInfo()
+    st = _stream(stream)
+    with torch.cuda.device(w.device):
+        _check(lib.bs_fw_measure(w.data_ptr() if n else None, n, scratch.data_ptr(), scratch.numel(), st,
+                                 ctypes.byref(info)), "fw_measure")
+        fw = torch.empty(info.total_bytes, dtype=torch.uint8, device=w.device)
+        _check(lib.bs_fw_write(w.data_ptr() if n else None, n, scratch.data_ptr(), scratch.numel(),
+                               ctypes.byref(info), fw.data_ptr(), fw.numel(), st), "fw_write")
+    return fw, info
+
+
+def fw_parse(head, fw_bytes: int) -> FwInfo:
+    """bs_fw_parse of a host copy of a layout's first 96 bytes (or more)."""
+    h = _host_bytes(head)
+    info = FwInfo()
+    _check(lib.bs_fw_parse(h.ctypes.data, h.size, fw_bytes, ctypes.byref(info)), "fw_parse")
+    return info
+
+
+def fw_decode(fws, infos, outs, err: torch.Tensor, stream=None):
+    """bs_fw_decode: decode layouts fws[k] (uint8 CUDA tensors, headers infos[k]) into outs[k]
+    (2-byte CUDA tensors of n_elems). err: a zeroed int32 CUDA tensor of one element that
+    receives the error flags. Enqueued on the stream."""
+    n = len(fws)
+    assert len(infos) == n and len(outs) == n
+    P = ctypes.c_void_p
+    p_fw = (P * max(n, 1))(*[f.data_ptr() for f in fws])
+    p_out = (P * max(n, 1))(*[_words(o).data_ptr() if o.numel() else None for o in outs])
+    sizes = (ctypes.c_size_t * max(n, 1))(*[o.numel() * 2 for o in outs])
+    inf = (FwInfo * max(n, 1))(*infos)
+    assert err.is_cuda and err.dtype == torch.int32 and err.numel() >= 1
+    with torch.cuda.device(err.device):
+        _check(lib.bs_fw_decode(n, p_fw, inf, p_out, sizes, err.data_ptr(), _stream(stream)), "fw_decode")
+    return outs

@@ -17,7 +17,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libbs.so")
-SOURCES = ["bs_kernels.cu", "bs_encode_kernels.cu", "bs_noalloc.cu", "bs_plan.cpp", "bs_encode.cpp", "bs_stream.cpp"]
+SOURCES = ["bs_kernels.cu", "bs_encode_kernels.cu", "bs_noalloc.cu", "bs_fw.cu", "bs_plan.cpp", "bs_encode.cpp",
+           "bs_stream.cpp"]
 HEADERS = ["bs_internal.h", "bs_host.h", os.path.join(ROOT, "include", "bs.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
