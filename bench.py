@@ -53,11 +53,14 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-threads", type=int, default=0, help="oracle threads (0: all host cores)")
-    ap.add_argument("--mode", choices=["model", "layerwise", "stream", "fw"], default="model",
+    ap.add_argument("--batch", type=int, default=1, help="gemv mode: tokens per product (1..8)")
+    ap.add_argument("--mode", choices=["model", "layerwise", "stream", "fw", "gemv"], default="model",
                     help="model: one bs_decode_batch of every tensor per step (the default line); "
                          "layerwise: one bs_decode_batch per layer (group) per step; "
                          "stream: layer streaming from a host container through the LRU device cache; "
-                         "fw: one bs_fw_decode of every tensor's fixed-width lane layout per step")
+                         "fw: one bs_fw_decode of every tensor's fixed-width lane layout per step; "
+                         "gemv: y = W x for every weight matrix from its layout (bs_fw_gemv), one "
+                         "forward-shaped pass per step, against dense cuBLAS products")
     ap.add_argument("--vram-gb", type=float, default=None,
                     help="stream mode: device budget (arena) in GB; default: the smallest arena that "
                          "double-buffers the largest group")
@@ -911,6 +914,179 @@ def run_fw(a):
         "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": int(launches), "clocks": clk}), flush=True)
 
 
+# ------------------------------------------------------------------ fused GEMV on the layout
+GEMV_METRIC = "BF16-equivalent weight GB/s of y = W x from the fixed-width lane layout (every matrix, 1 B200)"
+
+
+def _gemv_calls(specs):
+    """The products of one forward-shaped pass, grouped as a decoder step issues them: per layer
+    (q, k, v) on one x, o, (gate, up) on one x, down; then the LM head on the embedding.
+    The synthetic matrices are iid, so each layer tensor is multiplied as the [out, in] matrix
+    of its projection (rows = its second dimension) and the embedding as [vocab, hidden]."""
+    by = {s.name: k for k, s in enumerate(specs)}
+    calls = []
+    layers = sorted({int(s.name.split(".")[1]) for s in specs if s.name.startswith("layers.")})
+    for L in layers:
+        for grp in (("q", "k", "v"), ("o",), ("gate", "up"), ("down",)):
+            ks = [by[f"layers.{L}.{m}"] for m in grp if f"layers.{L}.{m}" in by]
+            if ks:
+                calls.append([(k, specs[k].shape[1], specs[k].shape[0]) for k in ks])
+    if "embed" in by:
+        k = by["embed"]
+        calls.append([(k, specs[k].shape[0], specs[k].shape[1])])
+    return calls
+
+
+def run_gemv(a):
+    """One step = every weight matrix's product y = W x, straight from its FW layout, grouped as
+    a decoder pass issues them (169 calls for the 9B checkpoint), captured in a CUDA graph."""
+    import torch
+
+    import lossless_entropy_coding_interleaved_b200 as bs
+    import synthetic as S
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = _Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    batch = a.batch
+    specs_all, _, desc = _workload_desc(a.workload, a.layers)
+    specs = [s for s in specs_all if not s.is_raw and len(s.shape) == 2]
+    dense = [S.generate(s, dev).reshape(-1) for s in specs]
+    built = [bs.fw_transcode(w) for w in dense]
+    torch.cuda.synchronize()
+    calls = _gemv_calls(specs)
+    n_w = sum(rows * cols for c in calls for _, rows, cols in c)
+    fw_bytes = sum(built[k][1].total_bytes for c in calls for k, _, _ in c)
+    g = torch.Generator(device=dev).manual_seed(1234)
+    xs, ys, yd, items = [], [], [], []
+    for c in calls:
+        cols = c[0][2]
+        x = torch.randn(batch, cols, device=dev, generator=g).to(torch.bfloat16)
+        xs.append(x)
+        y = [torch.empty(batch, rows, dtype=torch.float32, device=dev) for _, rows, _ in c]
+        ys.append(y)
+        yd.append([torch.empty(batch, rows, dtype=torch.bfloat16, device=dev) for _, rows, _ in c])
+        items.append([(built[k][0], built[k][1], rows, cols, x.view(torch.int16), yy) for (k, rows, _), yy in zip(c, y)])
+    xy_bytes = sum(2 * batch * c[0][2] + 4 * batch * sum(r for _, r, _ in c) for c in calls)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def fused_pass():
+        for it in items:
+            bs.fw_gemv(it, err, stream=torch.cuda.current_stream())
+
+    def dense_pass():
+        for c, x, yy in zip(calls, xs, yd):
+            for (k, rows, cols), y in zip(c, yy):
+                torch.matmul(x, dense[k].view(torch.bfloat16).view(rows, cols).t(), out=y)
+
+    # parity before timing: every product against a float64 product of the originals on the
+    # device, within 2 * K * 2^-24 * (sum |w x| + 64 max|x|) per output (escapes included)
+    fused_pass()
+    torch.cuda.synchronize()
+    worst = 0.0
+    for c, x, yy in zip(calls, xs, ys):
+        xf = x.double()
+        for (k, rows, cols), y in zip(c, yy):
+            wf = dense[k].view(torch.bfloat16).view(rows, cols).double()
+            ref = xf @ wf.t()
+            tol = 2.0 * cols * 2.0 ** -24 * (xf.abs() @ wf.abs().t() + 64.0 * xf.abs().max())
+            worst = max(worst, float(((y.double() - ref).abs() / tol).max()))
+    if int(err.item()) != 0 or not worst <= 1.0:
+        raise SystemExit(f"bench: fused GEMV out of tolerance (worst {worst:.3g} of the bound) or error flag set")
+
+    def graph_of(fn):
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for _ in range(max(1, a.warmup)):
+                fn()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            fn()
+        torch.cuda.synchronize()
+        return gr
+
+    l0 = bs.launch_counter()
+    g_fused = graph_of(fused_pass)
+    launches_per_pass = (bs.launch_counter() - l0) // (max(1, a.warmup) + 1)
+    g_dense = graph_of(dense_pass)
+
+    phys = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+    smi_index = phys[local] if local < len(phys) and phys[local].strip().isdigit() else str(local)
+    clocks = _Clocks(smi_index)
+    time.sleep(0.3)
+    ms_fused = ranks.max(_timed(stream, a.steps, g_fused.replay, ranks.barrier))
+    clk = clocks.stop()
+    ms_dense = ranks.max(_timed(stream, a.steps, g_dense.replay, ranks.barrier))
+    if int(err.item()) != 0:
+        raise SystemExit("bench: fused GEMV raised its error flag")
+    step_ms = ms_fused / a.steps
+    value = world * a.steps * 2 * n_w / (ms_fused * 1e-3) / 1e9
+    peak, peak_kind = _peak_hbm()
+    achieved = (fw_bytes + xy_bytes) / (step_ms * 1e-3) / 1e9
+
+    # end to end: x in from pinned host memory and y back out, per call, inside the timed region
+    e2e = None
+    if not a.no_e2e and a.e2e_steps > 0:
+        hx = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True).copy_(x) for x in xs]
+        hy = [[torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in yy] for yy in ys]
+
+        def e2e_pass():
+            for it, x, h, yy, hh in zip(items, xs, hx, ys, hy):
+                x.copy_(h, non_blocking=True)
+                bs.fw_gemv(it, err, stream=torch.cuda.current_stream())
+                for y, hy1 in zip(yy, hh):
+                    hy1.copy_(y, non_blocking=True)
+
+        e_ms = ranks.max(_timed(stream, a.e2e_steps, e2e_pass, ranks.barrier))
+        e2e = {"value": round(world * a.e2e_steps * 2 * n_w / (e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": int(sum(x.numel() * 2 for x in xs)),
+               "d2h_bytes_per_step": int(sum(y.numel() * 4 for yy in ys for y in yy)), "steps": a.e2e_steps,
+               "path": "per call: x copied in from pinned host memory, bs_fw_gemv, y copied back; "
+                       "the layouts stay resident (the weights of a served model)"}
+
+    cpu = None
+    if rank == 0 and not a.no_cpu_baseline:
+        import numpy as np
+        import oracle
+        c = calls[0]
+        k, rows, cols = c[0]
+        w = dense[k].cpu().numpy().view(np.uint16)
+        blob = oracle.fw_encode(w)
+        x = xs[0].view(torch.int16).cpu().numpy().view(np.uint16)
+        t0 = time.perf_counter()
+        oracle.fw_gemv(blob, rows, cols, x)
+        sec = time.perf_counter() - t0
+        cpu = {"value": round(2 * rows * cols / sec / 1e9, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"oracle decode + float64 numpy product of {specs[k].name} ({rows} x {cols}), batch {batch}"}
+    ranks.close()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": GEMV_METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded device draws, synthetic/ recipe)",
+        "config": {"workload": a.workload, "description": desc, "batch": batch, "matrices": len(specs),
+                   "calls_per_step": len(calls), "n_weights": int(n_w), "fw_bytes": int(fw_bytes),
+                   "bits_per_weight": round(8 * fw_bytes / n_w, 5),
+                   "dense_cublas_ms_per_step": round(ms_dense / a.steps, 4),
+                   "speedup_vs_dense": round(ms_dense / ms_fused, 4),
+                   "graph": "each step replays one CUDA graph of the pass's calls",
+                   "parity": f"every product within its fp32 bound before timing (worst {worst:.3g} of it)",
+                   "parallelism": f"replicas x{world} (no collective on the data path)",
+                   "l2": "no flush: the layouts (GBs) are larger than L2"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": "fw_gemv_kernel", "per_step_bytes": int(fw_bytes + xy_bytes),
+                     "launches_per_step": int(launches_per_pass)},
+        "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": int(launches_per_pass * a.steps), "clocks": clk}),
+        flush=True)
+
+
 def main():
     a = _args()
     if a.impl == "reference" and a.mode == "fw":
@@ -919,6 +1095,8 @@ def main():
         run_reference(a)
     elif a.mode == "fw":
         run_fw(a)
+    elif a.mode == "gemv":
+        run_gemv(a)
     elif a.mode == "layerwise":
         run_layerwise(a)
     elif a.mode == "stream":

@@ -350,6 +350,27 @@ bs_status bs_fw_parse(const void* h_head, size_t head_bytes, size_t fw_bytes, bs
 bs_status bs_fw_decode(int32_t n, const void* const* d_fw, const bs_fw_info* infos, void* const* d_out,
                        const size_t* out_bytes, uint32_t* d_err, void* stream);
 
+/* y = W x with W in the FW layout, decoded in registers on its way to the multiply: no dense
+ * copy of W is written. This is the operand path of the NVLC card's runtime (compressed
+ * weights resident, no persistent decoded-weight cache). For batch 1..8 the product is bound
+ * by the bytes of W, so it runs on the CUDA cores with fp32 accumulation.
+ *   d_fw, info: W's layout, rows x cols row-major (rows * cols == info.n_elems), with cols
+ *               a multiple of 256 (each row is whole tiles); 16-byte aligned;
+ *   d_x:        BF16 [batch][cols], 16-byte aligned;
+ *   d_y:        FP32 [batch][rows]; each entry is written once (no accumulation into it).
+ * Summation order is fixed, so results are deterministic. Escaped weights enter as the
+ * decoded placeholder plus a correction (w_true - w_placeholder) * x. */
+typedef struct {
+    const void* d_fw;
+    bs_fw_info info;
+    uint32_t rows, cols;
+    const void* d_x;
+    float* d_y;
+} bs_fw_gemv_item;
+/* Computes every item's product, up to 384 items per launch; batch is 1..8 for all items.
+ * d_err as for bs_fw_decode. Enqueued on stream. */
+bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_t batch, uint32_t* d_err, void* stream);
+
 const char* bs_status_str(bs_status s);
 int bs_last_cuda_error(void); /* the cudaError_t behind the last BS_E_CUDA on this thread */
 /* Kernel launches libbs has made in this process (all threads); a diagnostic counter. */

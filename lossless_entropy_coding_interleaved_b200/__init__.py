@@ -69,6 +69,12 @@ class FwInfo(ctypes.Structure):
                 f"total_bytes={self.total_bytes}, table={list(self.table)})")
 
 
+class FwGemvItem(ctypes.Structure):
+    """bs_fw_gemv_item: one product y = W x (W in the FW layout)."""
+    _fields_ = [("d_fw", ctypes.c_void_p), ("info", FwInfo), ("rows", ctypes.c_uint32), ("cols", ctypes.c_uint32),
+                ("d_x", ctypes.c_void_p), ("d_y", ctypes.c_void_p)]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libbs.so is not built ({LIB_PATH}); run "
@@ -121,7 +127,8 @@ def _load():
     L.bs_fw_write.argtypes = [P, u64, P, sz, ctypes.POINTER(FwInfo), P, sz, P]
     L.bs_fw_parse.argtypes = [P, sz, sz, ctypes.POINTER(FwInfo)]
     L.bs_fw_decode.argtypes = [i32, P, P, P, P, P, P]
-    for fn in ("bs_fw_measure", "bs_fw_write", "bs_fw_parse", "bs_fw_decode"):
+    L.bs_fw_gemv.argtypes = [i32, ctypes.POINTER(FwGemvItem), ctypes.c_uint32, P, P]
+    for fn in ("bs_fw_measure", "bs_fw_write", "bs_fw_parse", "bs_fw_decode", "bs_fw_gemv"):
         getattr(L, fn).restype = ctypes.c_int
     for fn in ("bs_streamer_create", "bs_streamer_group_count", "bs_streamer_tensor_info_get", "bs_streamer_prefetch", "bs_streamer_acquire",
                "bs_streamer_release", "bs_streamer_get_stats", "bs_streamer_check"):
@@ -144,7 +151,7 @@ EXPORTS = ("bs_plan_workspace_bytes", "bs_plan_workspace_bytes_device", "bs_plan
            "bs_streamer_create", "bs_streamer_group_count", "bs_streamer_tensor_info_get", "bs_streamer_prefetch",
            "bs_streamer_acquire",
            "bs_streamer_release", "bs_streamer_get_stats", "bs_streamer_check", "bs_streamer_destroy",
-           "bs_fw_scratch_bytes", "bs_fw_measure", "bs_fw_write", "bs_fw_parse", "bs_fw_decode")
+           "bs_fw_scratch_bytes", "bs_fw_measure", "bs_fw_write", "bs_fw_parse", "bs_fw_decode", "bs_fw_gemv")
 
 
 def decode_noalloc(container, d_container: torch.Tensor, idx: int, out: torch.Tensor, stream=None) -> torch.Tensor:
@@ -540,3 +547,28 @@ def fw_decode(fws, infos, outs, err: torch.Tensor, stream=None):
     with torch.cuda.device(err.device):
         _check(lib.bs_fw_decode(n, p_fw, inf, p_out, sizes, err.data_ptr(), _stream(stream)), "fw_decode")
     return outs
+
+
+def fw_gemv(products, err: torch.Tensor, stream=None):
+    """bs_fw_gemv: products is a sequence of (fw, info, rows, cols, x, y) with fw the layout of
+    W (rows x cols), x a BF16 CUDA tensor [batch, cols] (or [cols]) and y a float32 CUDA
+    tensor [batch, rows] (or [rows]); every x has the same batch (1..8). err: a zeroed int32
+    CUDA tensor of one element. Enqueued on the stream."""
+    n = len(products)
+    arr = (FwGemvItem * max(n, 1))()
+    batch = None
+    for k, (fw, info, rows, cols, x, y) in enumerate(products):
+        b = 1 if x.dim() == 1 else x.shape[0]
+        assert batch in (None, b), "every product of one call has the same batch"
+        batch = b
+        assert x.is_cuda and x.is_contiguous() and x.element_size() == 2 and x.numel() == b * cols
+        assert y.is_cuda and y.is_contiguous() and y.dtype == torch.float32 and y.numel() == b * rows
+        arr[k].d_fw = fw.data_ptr()
+        arr[k].info = info
+        arr[k].rows, arr[k].cols = rows, cols
+        arr[k].d_x = x.data_ptr()
+        arr[k].d_y = y.data_ptr()
+    assert err.is_cuda and err.dtype == torch.int32 and err.numel() >= 1
+    with torch.cuda.device(err.device):
+        _check(lib.bs_fw_gemv(n, arr, batch or 1, err.data_ptr(), _stream(stream)), "fw_gemv")
+    return [p[5] for p in products]

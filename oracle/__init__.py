@@ -333,3 +333,14 @@ def fw_decode(blob) -> np.ndarray:
     if st:
         raise OracleError(st, "fw_decode")
     return out[: info.n_elems].copy()
+
+
+def fw_gemv(blob, rows: int, cols: int, x) -> np.ndarray:
+    """y = W x in float64, with W (rows x cols, row-major) decoded from an FW layout and x
+    BF16 words [batch, cols] (or [cols]). The weights and x are exact in float64; the product
+    is numpy's matmul. Returns [batch, rows] (or [rows])."""
+    w = fw_decode(blob).reshape(rows, cols)
+    wf = (w.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    xa = np.ascontiguousarray(x, dtype=np.uint16)
+    xf = (xa.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return xf @ wf.T

@@ -209,3 +209,38 @@ def test_refuses_bad_exception_lists():
         with pytest.raises(oracle.OracleError) as e:
             oracle.fw_decode(b)
         assert e.value.code == oracle.E_CORRUPT
+
+
+# ---------------------------------------------------------------- y = W x on the layout
+def _bf(v):
+    return (np.asarray(v, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_gemv_oracle_closed_form():
+    # rows: all 1.0; all 2.0; 1.0 except one weight of 2^20; and 1.0 except 2^(k-8) at
+    # column k < 20. Row 3 has 20 + 1 distinct exponents in all, so some of its weights
+    # escape. x = 1, 2, ..., 256 (exact in BF16) for the first three rows, and all ones for
+    # row 3 in a second product.
+    cols = 256
+    w = np.full((4, cols), 0x3F80, np.uint16)
+    w[1, :] = 0x4000
+    w[2, 99] = _bf(2.0 ** 20)
+    w[3, :20] = _bf(2.0 ** (np.arange(20) - 8))
+    blob = oracle.fw_encode(w)
+    assert oracle.fw_info(blob)["n_exc"] >= 1
+    x = _bf(np.arange(1, cols + 1))
+    y = oracle.fw_gemv(blob, 4, cols, x)
+    assert y[:3].tolist() == [32896.0, 65792.0, 32896.0 + (2.0 ** 20 - 1) * 100]
+    ones = np.full(cols, 0x3F80, np.uint16)
+    y1 = oracle.fw_gemv(blob, 4, cols, ones)
+    assert y1[3] == (2.0 ** 20 - 1) * 2.0 ** -8 + (cols - 20)
+
+
+def test_gemv_oracle_matches_definition_on_the_originals():
+    rows, cols = 37, 512
+    w = _gaussian_bf16(rows * cols, seed=4, scale=1.0).reshape(rows, cols)
+    x = _gaussian_bf16(3 * cols, seed=5).reshape(3, cols)
+    blob = oracle.fw_encode(w)
+    assert oracle.fw_info(blob)["n_exc"] > 0
+    f = lambda a: (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.array_equal(oracle.fw_gemv(blob, rows, cols, x), f(x) @ f(w).T)
