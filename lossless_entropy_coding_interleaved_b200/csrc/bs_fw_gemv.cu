@@ -87,7 +87,7 @@ constexpr uint32_t gemv_smem() { return 1024 + kGemvWarps * kFwStages * GemvSlot
 template <int GROUP>
 struct GemvExc {
     uint32_t cnt = 0, e0 = 0, gpos = 0, word = 0;
-    uint32_t d[GROUP / 2] = {};
+    uint32_t d[(GROUP + 1) / 2] = {};
     __device__ uint32_t tile_of(uint32_t e) const {
         uint32_t t = 0;
 #pragma unroll
@@ -96,8 +96,9 @@ struct GemvExc {
     }
 };
 
+// Batches above 2 are held to 2 CTAs per SM (at most 128 registers); 1-2 need fewer anyway.
 template <int BATCH, int GROUP>
-__global__ void __launch_bounds__(kGemvWarps * 32) fw_gemv_kernel(const __grid_constant__ FwGemvParams p) {
+__global__ void __launch_bounds__(kGemvWarps * 32, BATCH <= 2 ? 1 : 2) fw_gemv_kernel(const __grid_constant__ FwGemvParams p) {
     using Slot = GemvSlot<GROUP>;
     extern __shared__ __align__(16) uint8_t smem[];
     uint32_t* pair_tab = reinterpret_cast<uint32_t*>(smem);
@@ -247,21 +248,24 @@ __global__ void __launch_bounds__(kGemvWarps * 32) fw_gemv_kernel(const __grid_c
         const uint32_t* sc0 = reinterpret_cast<const uint32_t*>(sl + Slot::C) + cw0;
         const uint32_t* sc1 = reinterpret_cast<const uint32_t*>(sl + Slot::C) + cw1;
         const uint16_t* xg = xl + col0;
+        auto tile = [&](int g) {
+            const uint4 w = fw_octet(pair_tab, sa[32 * g], sb[32 * g], sc0[24 * g], sc1[24 * g], csh);
 #pragma unroll
-        for (int g = 0; g < GROUP; ++g) {
-            if (static_cast<uint32_t>(g) < ng) {
-                const uint4 w = fw_octet(pair_tab, sa[32 * g], sb[32 * g], sc0[24 * g], sc1[24 * g], csh);
-#pragma unroll
-                for (int b = 0; b < BATCH; ++b) {
-                    const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xg + b * cols + 256 * g));
-                    float s = acc[b];
-                    s = fma_bf16x2(w.x, xv.x, s);
-                    s = fma_bf16x2(w.y, xv.y, s);
-                    s = fma_bf16x2(w.z, xv.z, s);
-                    s = fma_bf16x2(w.w, xv.w, s);
-                    acc[b] = s;
-                }
+            for (int b = 0; b < BATCH; ++b) {
+                const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xg + b * cols + 256 * g));
+                float s = acc[b];
+                s = fma_bf16x2(w.x, xv.x, s);
+                s = fma_bf16x2(w.y, xv.y, s);
+                s = fma_bf16x2(w.z, xv.z, s);
+                s = fma_bf16x2(w.w, xv.w, s);
+                acc[b] = s;
             }
+        };
+        if (ng == GROUP) { // a whole group: no per-tile test
+#pragma unroll
+            for (int g = 0; g < GROUP; ++g) tile(g);
+        } else {
+            for (uint32_t g = 0; g < ng; ++g) tile(static_cast<int>(g));
         }
         if (lane < cur.cnt) correct(acc, col0 + cur.gpos, cur.word);
         for (uint32_t e = lane + 32; e < cur.cnt; e += 32) // a group with more than 32 escapes
@@ -288,54 +292,37 @@ __global__ void __launch_bounds__(kGemvWarps * 32) fw_gemv_kernel(const __grid_c
     fw_wait<0>();
 }
 
-// tiles per group of the GEMV kernel
-#ifndef BS_GEMV_GROUP
-#define BS_GEMV_GROUP 8
-#endif
-constexpr int kGemvGroup = BS_GEMV_GROUP;
-
-// CTAs of fw_gemv_kernel<BATCH> that fit on one SM (after allowing its shared memory).
-template <int BATCH>
-cudaError_t gemv_ctas_per_sm(int* n) {
-    constexpr uint32_t smem = gemv_smem<kGemvGroup>();
-    cudaError_t e = cudaFuncSetAttribute(fw_gemv_kernel<BATCH, kGemvGroup>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, fw_gemv_kernel<BATCH, kGemvGroup>, kGemvWarps * 32, smem);
+// The group size of a product: the largest of 8, 7 and 4 that divides the row's tile count,
+// so that every group is whole (else 8, with a shorter last group per row).
+inline int gemv_group_for(uint32_t cols) {
+    const uint32_t tpr = cols / 256;
+    return tpr % 8 == 0 ? 8 : tpr % 7 == 0 ? 7 : tpr % 4 == 0 ? 4 : 8;
 }
 
-cudaError_t gemv_ctas_per_sm_batch(uint32_t batch, int* n) {
+// The kernel instance for (batch, group), its shared memory, and the CTAs that fit on an SM.
+struct GemvKernel {
+    void (*fn)(const FwGemvParams);
+    uint32_t smem;
+};
+template <int BATCH, int GROUP>
+GemvKernel gemv_kernel_of() {
+    return {fw_gemv_kernel<BATCH, GROUP>, gemv_smem<GROUP>()};
+}
+template <int GROUP>
+GemvKernel gemv_kernel_b(uint32_t batch) {
     switch (batch) {
-    case 1: return gemv_ctas_per_sm<1>(n);
-    case 2: return gemv_ctas_per_sm<2>(n);
-    case 3: return gemv_ctas_per_sm<3>(n);
-    case 4: return gemv_ctas_per_sm<4>(n);
-    case 5: return gemv_ctas_per_sm<5>(n);
-    case 6: return gemv_ctas_per_sm<6>(n);
-    case 7: return gemv_ctas_per_sm<7>(n);
-    default: return gemv_ctas_per_sm<8>(n);
+    case 1: return gemv_kernel_of<1, GROUP>();
+    case 2: return gemv_kernel_of<2, GROUP>();
+    case 3: return gemv_kernel_of<3, GROUP>();
+    case 4: return gemv_kernel_of<4, GROUP>();
+    case 5: return gemv_kernel_of<5, GROUP>();
+    case 6: return gemv_kernel_of<6, GROUP>();
+    case 7: return gemv_kernel_of<7, GROUP>();
+    default: return gemv_kernel_of<8, GROUP>();
     }
 }
-
-template <int BATCH>
-cudaError_t launch_gemv(const FwGemvParams& p, uint32_t ctas, cudaStream_t s) {
-    constexpr uint32_t smem = gemv_smem<kGemvGroup>();
-    fw_gemv_kernel<BATCH, kGemvGroup><<<ctas, kGemvWarps * 32, smem, s>>>(p);
-    count_launch();
-    return cudaGetLastError();
-}
-
-cudaError_t launch_gemv_batch(uint32_t batch, const FwGemvParams& p, uint32_t ctas, cudaStream_t s) {
-    switch (batch) {
-    case 1: return launch_gemv<1>(p, ctas, s);
-    case 2: return launch_gemv<2>(p, ctas, s);
-    case 3: return launch_gemv<3>(p, ctas, s);
-    case 4: return launch_gemv<4>(p, ctas, s);
-    case 5: return launch_gemv<5>(p, ctas, s);
-    case 6: return launch_gemv<6>(p, ctas, s);
-    case 7: return launch_gemv<7>(p, ctas, s);
-    default: return launch_gemv<8>(p, ctas, s);
-    }
+GemvKernel gemv_kernel(uint32_t batch, int group) {
+    return group == 7 ? gemv_kernel_b<7>(batch) : group == 4 ? gemv_kernel_b<4>(batch) : gemv_kernel_b<8>(batch);
 }
 
 } // namespace
@@ -360,43 +347,60 @@ extern "C" bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    // One wave: as many CTAs as fit on the GPU at once, shared among the launch's items in
-    // proportion to their rows (a warp per row at a time, at least one row per warp), so that
-    // every warp walks many rows and its copy ring stays full.
-    int per_sm = 0;
-    const cudaError_t oe = gemv_ctas_per_sm_batch(batch, &per_sm);
-    if (oe != cudaSuccess) return cuda_status(oe);
-    const uint64_t wave = uint64_t(std::max(per_sm, 1)) * static_cast<uint64_t>(sms);
+    // One wave per group size: as many CTAs as fit on the GPU at once, shared among the
+    // items in proportion to their rows (a warp per row at a time, at least one row per warp),
+    // so that every warp walks many rows and its copy ring stays full. Items whose rows split
+    // differently into groups run as separate launches.
     std::vector<FwGemvParams> params(1);
     FwGemvParams& p = params[0];
     p.err = d_err;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    int32_t k = 0;
-    while (k < n) {
-        p.n_items = 0;
-        uint64_t ctas = 0, rows_here = 0;
-        for (int32_t q = k; q < n && q < k + kGemvMaxItems; ++q) rows_here += items[q].rows;
-        for (; k < n && p.n_items < static_cast<uint32_t>(kGemvMaxItems); ++k) {
-            const bs_fw_gemv_item& g = items[k];
-            if (g.info.n_elems == 0) continue;
-            const uint64_t share = std::max<uint64_t>(1, wave * g.rows / std::max<uint64_t>(rows_here, 1));
-            const uint32_t c = static_cast<uint32_t>(std::min<uint64_t>(share, (g.rows + kGemvWarps - 1) / kGemvWarps));
-            if (ctas + c >= (1ull << 31)) break;
-            FwGemvItem& it = p.item[p.n_items++];
-            it.fw = static_cast<const uint8_t*>(g.d_fw);
-            it.x = static_cast<const uint16_t*>(g.d_x);
-            it.y = g.d_y;
-            it.rows = g.rows;
-            it.cols = g.cols;
-            it.n_exc = static_cast<uint32_t>(g.info.n_exc);
-            it.cta_begin = static_cast<uint32_t>(ctas);
-            it.ctas = c;
-            std::memcpy(it.table, g.info.table, sizeof(it.table));
-            ctas += c;
-        }
-        if (p.n_items == 0) continue;
-        const cudaError_t e = launch_gemv_batch(batch, p, static_cast<uint32_t>(ctas), s);
+    for (int group : {8, 7, 4}) {
+        const GemvKernel kern = gemv_kernel(batch, group);
+        bool any = false;
+        for (int32_t k = 0; k < n && !any; ++k) any = items[k].info.n_elems && gemv_group_for(items[k].cols) == group;
+        if (!any) continue;
+        cudaError_t e = cudaFuncSetAttribute(kern.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kern.smem));
+        int per_sm = 0;
+        if (e == cudaSuccess)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern.fn, kGemvWarps * 32, kern.smem);
         if (e != cudaSuccess) return cuda_status(e);
+        const uint64_t wave = uint64_t(std::max(per_sm, 1)) * static_cast<uint64_t>(sms);
+        int32_t k = 0;
+        while (k < n) {
+            p.n_items = 0;
+            uint64_t ctas = 0, rows_here = 0;
+            for (int32_t q = k, m = 0; q < n && m < kGemvMaxItems; ++q)
+                if (items[q].info.n_elems && gemv_group_for(items[q].cols) == group) {
+                    rows_here += items[q].rows;
+                    ++m;
+                }
+            for (; k < n && p.n_items < static_cast<uint32_t>(kGemvMaxItems); ++k) {
+                const bs_fw_gemv_item& g = items[k];
+                if (g.info.n_elems == 0 || gemv_group_for(g.cols) != group) continue;
+                const uint64_t share = std::max<uint64_t>(1, wave * g.rows / std::max<uint64_t>(rows_here, 1));
+                const uint32_t c =
+                    static_cast<uint32_t>(std::min<uint64_t>(share, (g.rows + kGemvWarps - 1) / kGemvWarps));
+                if (ctas + c >= (1ull << 31)) break;
+                FwGemvItem& it = p.item[p.n_items++];
+                it.fw = static_cast<const uint8_t*>(g.d_fw);
+                it.x = static_cast<const uint16_t*>(g.d_x);
+                it.y = g.d_y;
+                it.rows = g.rows;
+                it.cols = g.cols;
+                it.n_exc = static_cast<uint32_t>(g.info.n_exc);
+                it.cta_begin = static_cast<uint32_t>(ctas);
+                it.ctas = c;
+                std::memcpy(it.table, g.info.table, sizeof(it.table));
+                ctas += c;
+            }
+            if (p.n_items == 0) continue;
+            kern.fn<<<static_cast<uint32_t>(ctas), kGemvWarps * 32, kern.smem, s>>>(p);
+            count_launch();
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return cuda_status(e);
+        }
     }
     return BS_OK;
 }
