@@ -821,7 +821,7 @@ def run_fw(a):
     value = world * a.steps * out_bytes / (total_ms * 1e-3) / 1e9
     peak, peak_kind = _peak_hbm()
     achieved = (fw_bytes + out_bytes) / (mean_step * 1e-3) / 1e9
-    tpw = _traffic_per_weight("fw_decode_kernel_gemma2_9b.md", ("bs_fw.cu",))
+    tpw = _traffic_per_weight("fw_decode_kernel_gemma2_9b.md", ("bs_fw.cu", "bs_fw.cuh"))
 
     # end to end: every layout copied in from pinned host memory and every output copied back,
     # per layer group on three streams so that the copies of one group overlap the others
