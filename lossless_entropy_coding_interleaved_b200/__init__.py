@@ -354,6 +354,23 @@ class Plan:
         _check(lib.bs_decode_batch(self._p, ia, pa, ba, n, _stream(stream)), "decode_batch")
         return outs
 
+    def to_fw(self, idx: int, scratch: torch.Tensor | None = None, stream=None):
+        """The fixed-width lane layout (FORMAT.md section 10) of BF16 tensor idx, built on the
+        device from the container, as the runtime of the NVLC card derives its streams from
+        the rANS files at start-up. The tensor is decoded (bs_decode_tensor) into `scratch`
+        (or a temporary), checked (bs_check), then transcoded (bs_fw_measure, bs_fw_write).
+        Returns (layout, FwInfo). Synchronises the stream."""
+        i = self._info[idx]
+        if i["kind"] == KIND_RAW:
+            raise BsError(E_ARG, "to_fw", "a RAW tensor has no BF16 words")
+        n = i["n_elems"]
+        if scratch is None or scratch.numel() < n:
+            scratch = torch.empty(max(n, 1), dtype=torch.int16, device=self.device)
+        words = scratch.view(-1)[:n]
+        self.decode(idx, words, stream=stream)
+        self.check(stream=stream)
+        return fw_transcode(words, stream=stream)
+
     def verify(self, idx: int, out: torch.Tensor, stream=None) -> int:
         """Checksum of a decoded tensor computed on the device; raises BsError(E_CORRUPT)
         if it differs from the stored one. Synchronises the stream."""

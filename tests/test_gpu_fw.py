@@ -175,3 +175,14 @@ def test_position_past_tensor_is_flagged_and_contained():
     big = bigs[0].cpu().numpy().view(np.uint16)
     assert (big[:64] == 0x5A5A).all() and (big[-64:] == 0x5A5A).all()
     assert np.array_equal(got[:256 * 4], w[:256 * 4])
+
+
+def test_layout_from_container_matches_oracle():
+    # the runtime path: rANS container -> decode on the device -> FW layout on the device
+    specs = [s for s in S.workload("edge_mix") if not s.is_raw]
+    arrs = [S.words_numpy(S.generate(s, "cpu")) for s in specs]
+    c = oracle.encode([(s.name, a, "bf16") for s, a in zip(specs, arrs)])
+    plan = bs.Plan(c, device="cuda:0")
+    for k, a in enumerate(arrs):
+        fw, info = plan.to_fw(k)
+        assert fw.cpu().numpy().tobytes() == oracle.fw_encode(a.reshape(-1)), specs[k].name

@@ -151,3 +151,25 @@ def test_gemv_corrupt_tile_exc_is_flagged():
     torch.cuda.synchronize()
     assert int(err.item()) & 1
     assert torch.isfinite(y).all()
+
+
+def test_gemv_special_weights_follow_ieee():
+    # inf, -inf and NaN weights (rare exponents, so they escape): each output must match the
+    # float64 product's class (nan, +inf, -inf) and, where finite, its value
+    rows, cols = 24, 512
+    w = _gauss(rows * cols, seed=13).reshape(rows, cols)
+    w[3, 7] = 0x7F80             # +inf
+    w[5, 100] = 0xFF80           # -inf
+    w[9, 300] = 0x7FC1           # NaN
+    w[11, 0] = 0x7F80
+    w[11, 1] = 0xFF80            # inf + -inf in one row: NaN
+    x = _gauss(cols, seed=14, scale=1.0).reshape(1, cols)
+    x[0, 300] = 0x3F80
+    (y,), err, _ = _run([(w, x)], 1)
+    assert err == 0
+    ref = oracle.fw_gemv(oracle.fw_encode(w), rows, cols, x)
+    assert np.array_equal(np.isnan(y), np.isnan(ref))
+    assert np.array_equal(np.isposinf(y), np.isposinf(ref)) and np.array_equal(np.isneginf(y), np.isneginf(ref))
+    fin = np.isfinite(ref)
+    tol = _tolerance(w, x, oracle.fw_info(oracle.fw_encode(w))["table"][0])
+    assert np.all(np.abs(y[fin] - ref[fin]) <= tol[fin])
