@@ -26,7 +26,7 @@ _SRCS = (_SRC, os.path.join(_HERE, "fworacle.c"))
 _LIB = os.path.join(_HERE, "libbsoracle.so")
 
 OK, E_ARG, E_FORMAT, E_VERSION, E_SIZE, E_CORRUPT, E_NOMEM = 0, 1, 2, 3, 4, 6, 7
-KIND_RANS, KIND_STORED, KIND_RAW = 0, 1, 2
+KIND_RANS, KIND_STORED, KIND_RAW, KIND_JOINT = 0, 1, 2, 3
 _NAMES = {1: "E_ARG", 2: "E_FORMAT", 3: "E_VERSION", 4: "E_SIZE", 6: "E_CORRUPT", 7: "E_NOMEM"}
 
 
@@ -60,7 +60,7 @@ class _Item(ctypes.Structure):
 
 
 class _Params(ctypes.Structure):
-    _fields_ = [(k, ctypes.c_uint32) for k in ("log2_chunk", "ns", "nh", "max_routes", "force_rans")]
+    _fields_ = [(k, ctypes.c_uint32) for k in ("log2_chunk", "ns", "nh", "max_routes", "force_rans", "joint", "nj")]
 
 
 class _Info(ctypes.Structure):
@@ -127,9 +127,12 @@ def _buf(container) -> tuple[np.ndarray, int]:
 
 
 def encode(items, log2_chunk: int = 16, ns: int = 11, nh: int = 5, max_routes: int = 15,
-           force_rans: bool = False) -> bytes:
+           force_rans: bool = False, model: str = "factored", nj: int = 13) -> bytes:
     """items: sequence of (name, array, kind) with kind "bf16" (uint16 words, any shape)
-    or "raw" (uint8 bytes). Returns the container bytes (FORMAT.md section 4.6)."""
+    or "raw" (uint8 bytes). model "factored" codes BF16 tensors as kind RANS (ns, nh, routes),
+    "joint" as kind JOINT (one table over (s, h) of precision nj). Returns the container
+    bytes (FORMAT.md section 4.6)."""
+    assert model in ("factored", "joint")
     keep = []
     arr_items = (_Item * max(1, len(items)))()
     for k, (name, a, kind) in enumerate(items):
@@ -150,7 +153,7 @@ def encode(items, log2_chunk: int = 16, ns: int = 11, nh: int = 5, max_routes: i
         it.data = _ptr(a)
         it.name = nb
         it.name_bytes = len(nb)
-    p = _Params(log2_chunk, ns, nh, max_routes, 1 if force_rans else 0)
+    p = _Params(log2_chunk, ns, nh, max_routes, 1 if force_rans else 0, 1 if model == "joint" else 0, nj)
     out = ctypes.c_void_p()
     n = ctypes.c_uint64()
     st = lib().bso_encode(arr_items, len(items), ctypes.byref(p), ctypes.byref(out), ctypes.byref(n))

@@ -15,6 +15,9 @@
  * The card gives no byte layout, rANS parameters, interleaving or quantiser. Those
  * come from FORMAT.md (version 2), and each function says which section it follows.
  *
+ * The JOINT kind (FORMAT.md sections 1-2, 4.3b) codes the pair (s, h) with one table
+ * instead of the factored s-model and routes; model_t.joint selects it.
+ *
  * Pins (tests/test_oracle_*.py):
  *   - round trip on every 16-bit pattern;
  *   - brute force over tiny alphabets;
@@ -40,7 +43,11 @@ enum {
     BSO_E_NOMEM = 7
 };
 
-enum { KIND_RANS = 0, KIND_STORED = 1, KIND_RAW = 2 };
+enum { KIND_RANS = 0, KIND_STORED = 1, KIND_RAW = 2, KIND_JOINT = 3 };
+#define JOINT_PAIRS 4096 /* (s << 3) | h, FORMAT.md section 1 */
+
+/* RANS and JOINT tensors carry chunks of interleaved rANS lanes. */
+static int is_coded(uint32_t kind) { return kind == KIND_RANS || kind == KIND_JOINT; }
 
 #define LANES 32
 #define HEADER_BYTES 64
@@ -197,13 +204,30 @@ typedef struct {
     /* decode lookups (slot -> symbol) */
     uint16_t* s_of_slot; /* Ms entries */
     uint8_t* h_of_slot;  /* (n_routes + 1) * Mh entries, last row = UNIFORM */
+    /* the joint model (kind JOINT): one table over the pairs j = (s << 3) | h */
+    uint32_t joint, nj;
+    uint32_t Fj[JOINT_PAIRS], cum_j[JOINT_PAIRS];
+    uint16_t* j_of_slot; /* 2^nj entries */
 } model_t;
 
 static void model_free(model_t* m) {
     free(m->s_of_slot);
     free(m->h_of_slot);
+    free(m->j_of_slot);
     m->s_of_slot = NULL;
     m->h_of_slot = NULL;
+    m->j_of_slot = NULL;
+}
+
+/* FORMAT.md section 1, joint model: cumulative frequencies and the slot -> pair lookup */
+static int joint_build(model_t* m) {
+    uint32_t acc = 0;
+    for (int j = 0; j < JOINT_PAIRS; j++) { m->cum_j[j] = acc; acc += m->Fj[j]; }
+    m->j_of_slot = (uint16_t*)malloc(sizeof(uint16_t) << m->nj);
+    if (!m->j_of_slot) return BSO_E_NOMEM;
+    for (int j = 0; j < JOINT_PAIRS; j++)
+        for (uint32_t k = 0; k < m->Fj[j]; k++) m->j_of_slot[m->cum_j[j] + k] = (uint16_t)j;
+    return BSO_OK;
 }
 
 static void model_cums(model_t* m) {
@@ -251,6 +275,20 @@ static int model_build_lookups(model_t* m) {
 static uint32_t lane_encode(const model_t* m, const uint16_t* w, uint32_t S, uint8_t* emitted, uint16_t* word) {
     uint32_t x = STATE_L;
     uint32_t P = m->ns + m->nh;
+    if (m->joint) { /* FORMAT.md section 2, the JOINT kind: Q = Fj[j] out of 2^nj */
+        for (uint32_t tt = S; tt-- > 0;) {
+            uint32_t j = w[tt] >> 4;
+            uint64_t Q = m->Fj[j];
+            emitted[tt] = 0;
+            if ((uint64_t)x >= (Q << (32 - m->nj))) {
+                emitted[tt] = 1;
+                word[tt] = (uint16_t)(x & 0xFFFFu);
+                x >>= 16;
+            }
+            x = (uint32_t)(((uint64_t)x / Q << m->nj) + m->cum_j[j] + (uint64_t)x % Q);
+        }
+        return x;
+    }
     for (uint32_t tt = S; tt-- > 0;) {
         uint32_t s = w[tt] >> 7, h = (w[tt] >> 4) & 7u, e = s & 0xFF;
         uint32_t qs = m->Fs[s], cs = m->cum_s[s], qh, ch;
@@ -391,19 +429,42 @@ static uint64_t octet_index(uint32_t t, uint32_t j) { return ((uint64_t)(t >> 3)
 static uint32_t nibble_shift(uint32_t t) { return 4u * ((t & 7u) >> 1) + 16u * (t & 1u); }
 
 static int encode_rans(const uint16_t* w, uint64_t n, uint32_t log2_chunk, uint32_t ns, uint32_t nh,
-                       uint32_t max_routes, rans_blob_t* out) {
+                       uint32_t max_routes, uint32_t joint, uint32_t nj, rans_blob_t* out) {
     memset(out, 0, sizeof(*out));
     model_t* m = (model_t*)calloc(1, sizeof(model_t));
     uint64_t* cs = (uint64_t*)calloc(512, sizeof(uint64_t));
     uint64_t* ceh = (uint64_t*)calloc(256 * 8, sizeof(uint64_t));
+    uint64_t* cj = (uint64_t*)calloc(JOINT_PAIRS, sizeof(uint64_t));
     int st = BSO_E_NOMEM;
-    if (!m || !cs || !ceh) goto done;
+    if (!m || !cs || !ceh || !cj) goto done;
     m->ns = ns; m->nh = nh;
     /* counts */
     for (uint64_t i = 0; i < n; i++) {
         uint32_t s = w[i] >> 7;
         cs[s]++;
         ceh[(s & 0xFF) * 8 + ((w[i] >> 4) & 7u)]++;
+        cj[w[i] >> 4]++;
+    }
+    uint16_t pad;
+    if (joint) { /* FORMAT.md section 6, joint model; section 3, its pad word */
+        m->joint = 1;
+        m->nj = nj;
+        if ((st = bso_quantise(cj, JOINT_PAIRS, 1u << nj, m->Fj))) goto done;
+        if ((st = joint_build(m))) goto done;
+        uint32_t j_pad = 0;
+        for (uint32_t j = 1; j < JOINT_PAIRS; j++)
+            if (m->Fj[j] > m->Fj[j_pad]) j_pad = j;
+        pad = (uint16_t)(j_pad << 4);
+        uint32_t n_pairs = 0;
+        for (int j = 0; j < JOINT_PAIRS; j++) if (m->Fj[j]) n_pairs++;
+        out->model_bytes = 4 + 4ull * n_pairs; /* FORMAT.md section 4.3b */
+        out->model = (uint8_t*)calloc(1, out->model_bytes);
+        if (!out->model) { st = BSO_E_NOMEM; goto done; }
+        wr_u16(out->model, (uint16_t)n_pairs);
+        uint64_t o = 4;
+        for (int j = 0; j < JOINT_PAIRS; j++)
+            if (m->Fj[j]) { wr_u16(out->model + o, (uint16_t)j); wr_u16(out->model + o + 2, (uint16_t)m->Fj[j]); o += 4; }
+        goto chunks;
     }
     /* s-model */
     if ((st = bso_quantise(cs, 512, 1u << ns, m->Fs))) goto done;
@@ -424,12 +485,7 @@ static int encode_rans(const uint16_t* w, uint64_t n, uint32_t log2_chunk, uint3
         for (uint32_t h = 1; h < 8; h++)
             if (row[h] > row[h_pad]) h_pad = h;
     }
-    uint16_t pad = (uint16_t)((s_pad << 7) | (h_pad << 4));
-    /* nibble mode: constant when every weight has the same low nibble */
-    out->nib_mode = 0x10u | (w[0] & 15u);
-    for (uint64_t i = 1; i < n; i++)
-        if ((w[i] & 15u) != (w[0] & 15u)) { out->nib_mode = 0; break; }
-    const uint32_t nib_stored = out->nib_mode == 0;
+    pad = (uint16_t)((s_pad << 7) | (h_pad << 4));
 
     /* serialize the model (4.3) */
     uint32_t n_present = 0;
@@ -445,6 +501,13 @@ static int encode_rans(const uint16_t* w, uint64_t n, uint32_t log2_chunk, uint3
     o += 256;
     for (uint32_t r = 0; r < m->n_routes; r++)
         for (int h = 0; h < 8; h++) { wr_u16(out->model + o, (uint16_t)m->Fh[r][h]); o += 2; }
+
+chunks:;
+    /* nibble mode: constant when every weight has the same low nibble */
+    out->nib_mode = 0x10u | (w[0] & 15u);
+    for (uint64_t i = 1; i < n; i++)
+        if ((w[i] & 15u) != (w[0] & 15u)) { out->nib_mode = 0; break; }
+    const uint32_t nib_stored = out->nib_mode == 0;
 
     /* chunks */
     uint64_t C = 1ull << log2_chunk;
@@ -493,7 +556,8 @@ static int encode_rans(const uint16_t* w, uint64_t n, uint32_t log2_chunk, uint3
     }
     st = BSO_OK;
 done:
-    free(m); free(cs); free(ceh);
+    if (m) model_free(m);
+    free(m); free(cs); free(ceh); free(cj);
     if (st) blob_free(out);
     return st;
 }
@@ -514,15 +578,18 @@ typedef struct {
 
 typedef struct {
     uint32_t log2_chunk, ns, nh, max_routes, force_rans;
+    uint32_t joint; /* 1: the JOINT kind instead of the factored RANS model */
+    uint32_t nj;    /* JOINT precision, 8..13 */
 } bso_params;
 
 int bso_encode(const bso_item* items, uint32_t n_items, const bso_params* p, uint8_t** out, uint64_t* out_len) {
     if (!items && n_items) return BSO_E_ARG;
     if (!p || !out || !out_len) return BSO_E_ARG;
     if (p->log2_chunk < 8 || p->log2_chunk > 24 || p->ns < 1 || p->ns > 12 || p->nh < 3 || p->nh > 5 ||
-        p->ns + p->nh > 16 || p->max_routes > 15)
+        p->ns + p->nh > 16 || p->max_routes > 15 || p->joint > 1 || (p->joint && (p->nj < 8 || p->nj > 13)))
         return BSO_E_ARG;
     int st = BSO_OK;
+    const uint32_t coded_kind = p->joint ? KIND_JOINT : KIND_RANS;
     rans_blob_t* blobs = (rans_blob_t*)calloc(n_items ? n_items : 1, sizeof(rans_blob_t));
     uint8_t* kinds = (uint8_t*)calloc(n_items ? n_items : 1, 1);
     if (!blobs || !kinds) { free(blobs); free(kinds); return BSO_E_NOMEM; }
@@ -538,10 +605,10 @@ int bso_encode(const bso_item* items, uint32_t n_items, const bso_params* p, uin
         if (it->n_elems > (1ull << 40)) { st = BSO_E_ARG; goto fail; }
         if (it->n_elems == 0) { kinds[k] = KIND_STORED; continue; }
         if ((st = encode_rans((const uint16_t*)it->data, it->n_elems, p->log2_chunk, p->ns, p->nh, p->max_routes,
-                              &blobs[k])))
+                              p->joint, p->nj, &blobs[k])))
             goto fail;
         if (!p->force_rans && blobs[k].coded_total >= 2 * it->n_elems) { kinds[k] = KIND_STORED; blob_free(&blobs[k]); }
-        else kinds[k] = KIND_RANS;
+        else kinds[k] = (uint8_t)coded_kind;
     }
     /* layout */
     uint64_t dir_off = HEADER_BYTES, names_off = align16(dir_off + (uint64_t)DIR_ENTRY_BYTES * n_items);
@@ -551,7 +618,7 @@ int bso_encode(const bso_item* items, uint32_t n_items, const bso_params* p, uin
     uint64_t** chunk_off = (uint64_t**)calloc(n_items ? n_items : 1, sizeof(uint64_t*));
     if (!data_off || !model_off || !chunk_off) { st = BSO_E_NOMEM; goto fail2; }
     for (uint32_t k = 0; k < n_items; k++) {
-        if (kinds[k] == KIND_RANS) {
+        if (is_coded(kinds[k])) {
             model_off[k] = pos;
             pos = align16(pos + blobs[k].model_bytes);
             data_off[k] = pos;
@@ -590,12 +657,12 @@ int bso_encode(const bso_item* items, uint32_t n_items, const bso_params* p, uin
         for (uint32_t dd = 0; dd < it->ndim; dd++) wr_u64(d + 80 + 8 * dd, it->shape[dd]);
         if (it->name_bytes) memcpy(buf + names_off + name_pos, it->name, it->name_bytes);
         name_pos += it->name_bytes;
-        if (kinds[k] == KIND_RANS) {
+        if (is_coded(kinds[k])) {
             const rans_blob_t* b = &blobs[k];
             d[2] = (uint8_t)p->log2_chunk;
             d[3] = LANES;
-            d[4] = (uint8_t)p->ns;
-            d[5] = (uint8_t)p->nh;
+            d[4] = (uint8_t)(p->joint ? p->nj : p->ns);
+            d[5] = (uint8_t)(p->joint ? 0 : p->nh);
             d[6] = (uint8_t)b->n_routes;
             d[7] = (uint8_t)b->nib_mode;
             wr_u64(d + 24, b->n_chunks);
@@ -678,9 +745,9 @@ static int parse_entry(const uint8_t* b, uint64_t len, uint32_t idx, bso_tensor_
     ti->data_offset = rd_u64(d + 48); ti->data_bytes = rd_u64(d + 56);
     ti->checksum = rd_u64(d + 64);
     for (int k = 0; k < 8; k++) ti->shape[k] = rd_u64(d + 80 + 8 * k);
-    if (ti->ndim > 8 || ti->kind > 2) return BSO_E_FORMAT;
+    if (ti->ndim > 8 || ti->kind > 3) return BSO_E_FORMAT;
     if (rd_u64(d + 72) != 0) return BSO_E_FORMAT;
-    if (ti->kind != KIND_RANS && ti->nib_mode != 0) return BSO_E_FORMAT;
+    if (!is_coded(ti->kind) && ti->nib_mode != 0) return BSO_E_FORMAT;
     for (uint32_t k = ti->ndim; k < 8; k++)
         if (ti->shape[k] != 0) return BSO_E_FORMAT;
     if ((uint64_t)ti->name_offset + ti->name_bytes > rd_u64(b + 40)) return BSO_E_FORMAT;
@@ -695,17 +762,37 @@ static int parse_entry(const uint8_t* b, uint64_t len, uint32_t idx, bso_tensor_
         ti->coded_bytes = want;
         return BSO_OK;
     }
-    /* RANS */
+    /* RANS and JOINT */
     if (ti->lanes != LANES || ti->log2_chunk < 8 || ti->log2_chunk > 24) return BSO_E_FORMAT;
-    if (ti->ns < 1 || ti->ns > 12 || ti->nh < 3 || ti->nh > 5 || ti->ns + ti->nh > 16 || ti->n_routes > 15)
+    if (ti->kind == KIND_JOINT) {
+        if (ti->ns < 8 || ti->ns > 13 || ti->nh != 0 || ti->n_routes != 0) return BSO_E_FORMAT;
+    } else if (ti->ns < 1 || ti->ns > 12 || ti->nh < 3 || ti->nh > 5 || ti->ns + ti->nh > 16 || ti->n_routes > 15) {
         return BSO_E_FORMAT;
+    }
     if (ti->nib_mode != 0 && (ti->nib_mode & 0xF0u) != 0x10u) return BSO_E_FORMAT;
     if (ti->n_elems == 0 || ti->n_elems > (1ull << 40)) return BSO_E_FORMAT;
     uint64_t C = 1ull << ti->log2_chunk;
     if (ti->n_chunks != (ti->n_elems + C - 1) / C || ti->data_bytes != 16 * ti->n_chunks) return BSO_E_FORMAT;
-    if (ti->model_offset % 16 || !in_bounds(ti->model_offset, ti->model_bytes, len) || ti->model_bytes < 264)
-        return BSO_E_FORMAT;
+    if (ti->model_offset % 16 || !in_bounds(ti->model_offset, ti->model_bytes, len)) return BSO_E_FORMAT;
     const uint8_t* mm = b + ti->model_offset;
+    if (ti->kind == KIND_JOINT) { /* FORMAT.md section 4.3b */
+        if (ti->model_bytes < 8) return BSO_E_FORMAT;
+        uint32_t n_pairs = rd_u16(mm);
+        if (n_pairs < 1 || n_pairs > JOINT_PAIRS || rd_u16(mm + 2) != 0) return BSO_E_FORMAT;
+        if (ti->model_bytes != 4 + 4ull * n_pairs) return BSO_E_FORMAT;
+        uint64_t sumj = 0;
+        int prevj = -1;
+        for (uint32_t k = 0; k < n_pairs; k++) {
+            int j = rd_u16(mm + 4 + 4 * k);
+            uint32_t q = rd_u16(mm + 6 + 4 * k);
+            if (j <= prevj || j >= JOINT_PAIRS || q == 0) return BSO_E_FORMAT;
+            prevj = j;
+            sumj += q;
+        }
+        if (sumj != (1ull << ti->ns)) return BSO_E_FORMAT;
+        goto chunk_table;
+    }
+    if (ti->model_bytes < 264) return BSO_E_FORMAT;
     uint32_t n_present = rd_u16(mm);
     if (n_present < 1 || n_present > 512) return BSO_E_FORMAT;
     if (ti->model_bytes != 260 + 4ull * n_present + 16ull * ti->n_routes) return BSO_E_FORMAT;
@@ -727,6 +814,7 @@ static int parse_entry(const uint8_t* b, uint64_t len, uint32_t idx, bso_tensor_
         for (int h = 0; h < 8; h++) sum += rd_u16(route + 256 + 16 * r + 2 * h);
         if (sum != (1ull << ti->nh)) return BSO_E_FORMAT;
     }
+chunk_table:
     ti->coded_bytes = ti->model_bytes + ti->data_bytes;
     for (uint64_t c = 0; c < ti->n_chunks; c++) {
         const uint8_t* e = b + ti->data_offset + 16 * c;
@@ -759,8 +847,15 @@ int bso_tensor_info_get(const uint8_t* b, uint64_t len, uint32_t idx, bso_tensor
 
 static int load_model(const uint8_t* b, const bso_tensor_info* ti, model_t* m) {
     memset(m, 0, sizeof(*m));
-    m->ns = ti->ns; m->nh = ti->nh; m->n_routes = ti->n_routes;
     const uint8_t* mm = b + ti->model_offset;
+    if (ti->kind == KIND_JOINT) {
+        m->joint = 1;
+        m->nj = ti->ns;
+        uint32_t n_pairs = rd_u16(mm);
+        for (uint32_t k = 0; k < n_pairs; k++) m->Fj[rd_u16(mm + 4 + 4 * k)] = rd_u16(mm + 6 + 4 * k);
+        return joint_build(m);
+    }
+    m->ns = ti->ns; m->nh = ti->nh; m->n_routes = ti->n_routes;
     uint32_t n_present = rd_u16(mm);
     m->n_present = n_present;
     for (uint32_t k = 0; k < n_present; k++) m->Fs[rd_u16(mm + 4 + 4 * k)] = rd_u16(mm + 6 + 4 * k);
@@ -798,14 +893,23 @@ static int decode_chunk(const uint8_t* b, const bso_tensor_info* ti, const model
     uint32_t pos = 0;
     for (uint32_t t = 0; t < S; t++) {
         for (uint32_t j = 0; j < LANES; j++) { /* lanes in ascending order take words */
-            uint32_t slot = x[j] & ((1u << P) - 1u);
-            uint32_t js = slot >> m->nh, jh = slot & (Mh - 1u);
-            uint32_t s = m->s_of_slot[js];
-            uint8_t r = m->route[s & 0xFF];
-            uint32_t row = (r == 0xFF) ? m->n_routes : r, qh, ch;
-            uint32_t h = m->h_of_slot[(size_t)row * Mh + jh];
-            frac_model(m, s & 0xFF, h, &qh, &ch);
-            x[j] = m->Fs[s] * qh * (x[j] >> P) + (js - m->cum_s[s]) * qh + (jh - ch);
+            uint32_t s, h;
+            if (m->joint) { /* FORMAT.md section 2, the JOINT kind */
+                uint32_t slot = x[j] & ((1u << m->nj) - 1u);
+                uint32_t pj = m->j_of_slot[slot];
+                s = pj >> 3;
+                h = pj & 7u;
+                x[j] = m->Fj[pj] * (x[j] >> m->nj) + (slot - m->cum_j[pj]);
+            } else {
+                uint32_t slot = x[j] & ((1u << P) - 1u);
+                uint32_t js = slot >> m->nh, jh = slot & (Mh - 1u);
+                s = m->s_of_slot[js];
+                uint8_t r = m->route[s & 0xFF];
+                uint32_t row = (r == 0xFF) ? m->n_routes : r, qh, ch;
+                h = m->h_of_slot[(size_t)row * Mh + jh];
+                frac_model(m, s & 0xFF, h, &qh, &ch);
+                x[j] = m->Fs[s] * qh * (x[j] >> P) + (js - m->cum_s[s]) * qh + (jh - ch);
+            }
             if (x[j] < STATE_L) {
                 uint32_t wd = 0;
                 if (pos < nw) wd = rd_u16(words + 2ull * pos); else bad = 1;
@@ -835,7 +939,7 @@ int bso_decode_chunks(const uint8_t* b, uint64_t len, uint32_t idx, uint64_t c0,
     if (st) return st;
     uint64_t want = (ti.kind == KIND_RAW) ? ti.n_elems : 2 * ti.n_elems;
     if (out_bytes != want || (want && !out)) return BSO_E_SIZE;
-    if (ti.kind != KIND_RANS) {
+    if (!is_coded(ti.kind)) {
         if (ti.kind == KIND_STORED) {
             uint16_t* w = (uint16_t*)out;
             for (uint64_t i = 0; i < ti.n_elems; i++) w[i] = rd_u16(b + ti.data_offset + 2 * i);
@@ -863,7 +967,7 @@ int bso_decode(const uint8_t* b, uint64_t len, uint32_t idx, void* out, uint64_t
     bso_tensor_info ti;
     int st = parse_entry(b, len, idx, &ti);
     if (st) return st;
-    st = bso_decode_chunks(b, len, idx, 0, ti.kind == KIND_RANS ? ti.n_chunks : 0, out, out_bytes, bad_chunk);
+    st = bso_decode_chunks(b, len, idx, 0, is_coded(ti.kind) ? ti.n_chunks : 0, out, out_bytes, bad_chunk);
     if (st) return st;
     if (bso_checksum(out, ti.n_elems, ti.kind == KIND_RAW ? 2 : 0) != ti.checksum) return BSO_E_CORRUPT;
     return BSO_OK;

@@ -1,0 +1,166 @@
+"""Pins of the oracle's JOINT kind (FORMAT.md sections 1-2, 4.3b, 8.3): one quantised table
+over the pairs j = (s << 3) | h, decoded with one lookup per weight.
+
+What pins it:
+* the container of section 8.3, derived by hand (tests/golden/joint_two_weights.hex);
+* every 16-bit pattern and a size sweep round-trip;
+* a closed form: pairs with power-of-two frequencies cost exactly log2(2^nj / F) bits each,
+  so the word count is fixed up to the lanes' start and end states;
+* Gibbs' inequality and the 0.5% overhead gate against the empirical entropy;
+* every malformed JOINT field is refused.
+"""
+import os
+import struct
+
+import numpy as np
+import pytest
+
+import oracle
+import synthetic as S
+from tests.entropy import conditional_entropy_bits
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    hexs = []
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for line in fh:
+            hexs.append(line.split("#", 1)[0])
+    return bytes.fromhex("".join("".join(hexs).split()))
+
+
+def _words(spec):
+    return S.words_numpy(S.generate(spec, "cpu"))
+
+
+def _roundtrip(items, **kw):
+    c = oracle.encode(items, model="joint", **kw)
+    arr = np.frombuffer(c, np.uint8)
+    assert oracle.validate(arr) == len(items)
+    for k, (_, a, _) in enumerate(items):
+        assert np.array_equal(oracle.decode(arr, k), a), items[k][0]
+    return arr
+
+
+def test_golden_encode_and_decode():
+    want = _golden("joint_two_weights.hex")
+    w = np.array([0x3F80, 0x3F90], np.uint16)
+    got = oracle.encode([("w", w, "bf16")], model="joint", force_rans=True)
+    assert got == want
+    assert np.array_equal(oracle.decode(want, 0), w)
+    ti = oracle.info(want, 0)
+    assert (ti["kind"], ti["ns"], ti["nh"], ti["n_routes"], ti["nib_mode"]) == (oracle.KIND_JOINT, 13, 0, 0, 0x10)
+
+
+def test_every_pattern_round_trips():
+    w = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    rng = np.random.default_rng(3)
+    arr = _roundtrip([("all", w, "bf16"), ("shuffled", rng.permutation(w), "bf16")], force_rans=True)
+    assert oracle.info(arr, 0)["kind"] == oracle.KIND_JOINT
+
+
+def test_sizes_and_edges():
+    rng = np.random.default_rng(11)
+    sizes = list(range(1, 300)) + [1023, 1024, 1025, 65535, 65536, 65537, 2 * 65536 + 255]
+    items = []
+    for n in sizes:
+        x = (rng.standard_normal(n) * 0.02).astype(np.float32)
+        items.append((f"n{n}", (x.view(np.uint32) >> 16).astype(np.uint16), "bf16"))
+    arr = _roundtrip(items, force_rans=True)
+    for k, n in enumerate(sizes):
+        assert oracle.info(arr, k)["n_chunks"] == -(-n // 65536)
+
+
+@pytest.mark.parametrize("nj", [8, 10, 12, 13])
+@pytest.mark.parametrize("log2_chunk", [8, 16])
+def test_precisions_and_chunks(nj, log2_chunk):
+    w = _words(S.workload("tensor_1m")[0]).reshape(-1)[:90_001]
+    if nj < 10:   # keep the pair alphabet below 2^nj
+        w = np.where(np.arange(w.size) % 3 == 0, 0x3C00, 0xBC31).astype(np.uint16)
+    arr = _roundtrip([("w", w, "bf16")], nj=nj, log2_chunk=log2_chunk, force_rans=True)
+    assert oracle.info(arr, 0)["ns"] == nj
+
+
+@pytest.mark.parametrize("nj", [7, 14, 0])
+def test_precision_out_of_range(nj):
+    with pytest.raises(oracle.OracleError):
+        oracle.encode([("w", np.ones(10, np.uint16), "bf16")], model="joint", nj=nj)
+
+
+def test_power_of_two_frequencies_closed_form():
+    # four pairs with counts in proportion 1/2, 1/4, 1/8, 1/8 quantise exactly (4096, 2048,
+    # 1024, 1024 of 8192). Each weight then multiplies the state by exactly 2, 4, 8 or 8, i.e.
+    # costs exactly 1, 2, 3 or 3 bits: 1.75 bits per weight. Over the chunk's 65536 slots the
+    # 32 lanes take 2048 steps each and start from 2^16, so lane j's word count is
+    # floor((16 + bits_j - 16) / 16) within one word: the total is 65536 * 1.75 / 16 = 7168
+    # words, up to 32 (one partial word per lane).
+    n = 65536
+    pattern = np.array([0x3F80] * 4 + [0x3F90] * 2 + [0x3FA0, 0x3FB0], np.uint16)
+    w = np.tile(pattern, n // 8)
+    arr = _roundtrip([("w", w, "bf16")], force_rans=True)
+    ti = oracle.info(arr, 0)
+    n_words = int.from_bytes(arr[ti["data_offset"] + 8: ti["data_offset"] + 12].tobytes(), "little")
+    assert 7168 - 32 <= n_words <= 7168
+
+
+def test_gibbs_and_half_percent_gate():
+    total_bits = total_h = 0.0
+    for name in ("tensor_1m", "gemma2_layer"):
+        for s in S.workload(name):
+            w = _words(s)
+            c = oracle.encode([(s.name, w, "bf16")], model="joint", force_rans=True)
+            ti = oracle.info(c, 0)
+            h = conditional_entropy_bits(w)                   # total bits of the tensor
+            bits = 8.0 * ti["coded_bytes"]
+            assert bits >= h, s.name                          # Gibbs' inequality
+            total_bits += bits
+            total_h += h
+    assert total_bits / total_h - 1 < 0.005, total_bits / total_h - 1
+
+
+def test_edge_mix_kinds():
+    specs = S.workload("edge_mix")
+    items = [(s.name, _words(s), "raw" if s.is_raw else "bf16") for s in specs]
+    arr = _roundtrip(items)
+    kinds = {s.name: oracle.info(arr, k)["kind"] for k, s in enumerate(specs)}
+    assert kinds["uniform16"] == oracle.KIND_STORED
+    assert kinds["raw_span"] == oracle.KIND_RAW
+    assert kinds["t3"] == kinds["outliers"] == kinds["zeros"] == kinds["ones"] == oracle.KIND_JOINT
+
+
+def _bad(c, off, fmt, v):
+    b = bytearray(c)
+    struct.pack_into(fmt, b, off, v)
+    return np.frombuffer(bytes(b), np.uint8)
+
+
+def test_refuses_malformed_joint_fields():
+    c = _golden("joint_two_weights.hex")
+    d, m = 64, 224
+    bad = [
+        _bad(c, d + 4, "<B", 7),             # nj below 8
+        _bad(c, d + 4, "<B", 14),            # nj above 13
+        _bad(c, d + 5, "<B", 3),             # nh must be 0
+        _bad(c, d + 6, "<B", 1),             # n_routes must be 0
+        _bad(c, d + 0, "<B", 4),             # unknown kind
+        _bad(c, m + 0, "<H", 0),             # no pairs
+        _bad(c, m + 2, "<H", 1),             # reserved
+        _bad(c, m + 8, "<H", 1016),          # pairs not ascending
+        _bad(c, m + 4, "<H", 4096),          # pair out of range
+        _bad(c, m + 6, "<H", 0),             # zero frequency
+        _bad(c, m + 6, "<H", 4095),          # does not sum to 2^nj
+        _bad(c, d + 40, "<Q", 16),           # model_bytes != 4 + 4 * n_pairs
+    ]
+    for k, b in enumerate(bad):
+        with pytest.raises(oracle.OracleError) as e:
+            oracle.validate(b)
+        assert e.value.code == oracle.E_FORMAT, k
+
+
+def test_corrupt_state_is_detected():
+    c = bytearray(_golden("joint_two_weights.hex"))
+    c[256] ^= 0x10                           # lane 0's start state
+    with pytest.raises(oracle.OracleError) as e:
+        oracle.decode(np.frombuffer(bytes(c), np.uint8), 0)
+    assert e.value.code == oracle.E_CORRUPT
