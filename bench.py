@@ -54,6 +54,9 @@ def _args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-threads", type=int, default=0, help="oracle threads (0: all host cores)")
     ap.add_argument("--batch", type=int, default=1, help="gemv mode: tokens per product (1..8)")
+    ap.add_argument("--model", choices=["joint", "factored"], default="joint",
+                    help="rANS model of the container: joint (one table over (s, h), FORMAT.md kind JOINT; "
+                         "the default) or factored (s-model plus exponent routes, kind RANS)")
     ap.add_argument("--mode", choices=["model", "layerwise", "stream", "fw", "gemv"], default="model",
                     help="model: one bs_decode_batch of every tensor per step (the default line); "
                          "layerwise: one bs_decode_batch per layer (group) per step; "
@@ -121,7 +124,7 @@ def _word_histograms(originals, specs, dev):
 
 
 # ------------------------------------------------------------------ oracle on host cores
-def _oracle_sample(workload, threads):
+def _oracle_sample(workload, threads, model="joint"):
     """The bounded CPU sample: layer 0 of the workload, generated and encoded on the host by
     the oracle, then decoded by the oracle with `threads` threads over its chunks."""
     import numpy as np
@@ -131,12 +134,12 @@ def _oracle_sample(workload, threads):
     if workload in ("gemma2_9b", "qwen_27b_scale"):
         specs = [s for s in specs if s.name.startswith("layers.0.")]
     arrs = [S.words_numpy(S.generate(s, "cpu")) for s in specs]
-    c = np.frombuffer(oracle.encode([(s.name, a, "bf16") for s, a in zip(specs, arrs)]), np.uint8)
+    c = np.frombuffer(oracle.encode([(s.name, a, "bf16") for s, a in zip(specs, arrs)], model=model), np.uint8)
     infos = [oracle.info(c, k) for k in range(len(specs))]
     outs = [np.zeros(i["n_elems"], np.uint16) for i in infos]
     tasks = []
     for k, i in enumerate(infos):
-        if i["kind"] == oracle.KIND_RANS:
+        if i["kind"] in (oracle.KIND_RANS, oracle.KIND_JOINT):
             step = max(1, i["n_chunks"] // max(1, threads))
             tasks += [(k, c0, min(c0 + step, i["n_chunks"])) for c0 in range(0, i["n_chunks"], step)]
     n = sum(a.size for a in arrs)
@@ -147,7 +150,7 @@ def _oracle_sample(workload, threads):
         t0 = time.perf_counter()
         futs = [pool.submit(oracle.decode_chunks, c, k, c0, c1, outs[k]) for k, c0, c1 in tasks]
         for k, i in enumerate(infos):
-            if i["kind"] != oracle.KIND_RANS:
+            if i["kind"] not in (oracle.KIND_RANS, oracle.KIND_JOINT):
                 outs[k][:] = oracle.decode(c, k).reshape(-1)
         assert all(f.result() == 0 for f in futs)
         return time.perf_counter() - t0
@@ -239,7 +242,7 @@ def run_reference(a):
         return
     threads = _cpu_threads(a.cpu_threads)
     specs, n_all, desc = _workload_desc(a.workload, a.layers)
-    n, sample, run_once, check = _oracle_sample(a.workload, threads)
+    n, sample, run_once, check = _oracle_sample(a.workload, threads, a.model)
     with cf.ThreadPoolExecutor(threads) as pool:
         for _ in range(a.warmup):
             run_once(pool)
@@ -299,7 +302,7 @@ def run_ours(a):
     specs, n, desc = _workload_desc(a.workload, a.layers)
     t0 = time.time()
     originals = [(s.name, S.generate(s, dev)) for s in specs]
-    d_c, _ = bs.encode(originals)
+    d_c, _ = bs.encode(originals, model=a.model)
     torch.cuda.synchronize()
     t_encode = time.time() - t0
     hist_words = None
@@ -370,7 +373,7 @@ def run_ours(a):
     value = world * a.steps * out_bytes / (total_ms * 1e-3) / 1e9
     mean_step = statistics.mean(step_ms)
     peak, peak_kind = _peak_hbm()
-    tpw = _traffic_per_weight()
+    tpw = _traffic_per_weight() if a.model == "joint" else None
     achieved = (coded + out_bytes) / (mean_step * 1e-3) / 1e9
 
     # end to end: container in from pinned host memory, every tensor back out, per step,
@@ -430,7 +433,7 @@ def run_ours(a):
     cpu = None
     if rank == 0 and not a.no_cpu_baseline:
         threads = _cpu_threads(a.cpu_threads)
-        n_s, sample, run_once, check = _oracle_sample(a.workload, threads)
+        n_s, sample, run_once, check = _oracle_sample(a.workload, threads, a.model)
         with cf.ThreadPoolExecutor(threads) as pool:
             run_once(pool)
             check()
@@ -455,7 +458,10 @@ def run_ours(a):
                    "parallelism": f"replicas x{world} (no collective on the data path)",
                    "l2": "no flush: inputs larger than L2 (container and outputs are GBs)",
                    "parity": parity_how, "encode_s": round(t_encode, 2),
-                   "words": "BF16 bit patterns; rANS state arithmetic in u32"},
+                   "words": "BF16 bit patterns; rANS state arithmetic in u32",
+                   "model": ("joint: one rANS table over (sign+exponent, top 3 fraction bits), nj = 13 "
+                             "(FORMAT.md kind JOINT)" if a.model == "joint" else
+                             "factored: s-model (ns = 11) and exponent routes (nh = 5) (FORMAT.md kind RANS)")},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": (None if tpw is None else int(tpw * bf16_n)),
@@ -522,7 +528,7 @@ def _setup(a, dev):
     specs, n, desc = _workload_desc(a.workload, a.layers)
     t0 = time.time()
     originals = [(s.name, S.generate(s, dev)) for s in specs]
-    d_c, h_c = bs.encode(originals, host_copy=a.mode == "stream")
+    d_c, h_c = bs.encode(originals, host_copy=a.mode == "stream", model=a.model)
     torch.cuda.synchronize()
     t_encode = time.time() - t0
     hist = _word_histograms(originals, specs, dev)

@@ -46,7 +46,7 @@ typedef enum {
     BS_E_UNSUPPORTED = 8   /* a device without sm_100 support */
 } bs_status;
 
-enum { BS_KIND_RANS = 0, BS_KIND_STORED = 1, BS_KIND_RAW = 2 };
+enum { BS_KIND_RANS = 0, BS_KIND_STORED = 1, BS_KIND_RAW = 2, BS_KIND_JOINT = 3 };
 
 typedef struct bs_plan_t bs_plan_t; /* opaque host object */
 
@@ -59,7 +59,7 @@ typedef struct {
     uint64_t shape[8];
     uint32_t kind;        /* BS_KIND_* */
     uint32_t ndim;
-    uint32_t ns, nh, n_routes, log2_chunk; /* RANS model parameters (FORMAT.md section 2) */
+    uint32_t ns, nh, n_routes, log2_chunk; /* RANS model parameters (FORMAT.md section 2); JOINT: ns = nj, nh = n_routes = 0 */
     const char* name;     /* not NUL-terminated; points into the plan */
     uint32_t name_bytes;
     uint32_t nib_mode;    /* RANS: 0 = nibbles stored, 0x10 + c = every low nibble is c */
@@ -204,6 +204,8 @@ typedef struct {
     uint32_t nh;          /* 3..5 with ns + nh <= 16, default 5 */
     uint32_t max_routes;  /* 0..15, default 15 */
     uint32_t force_rans;  /* 1: never fall back to STORED (tests only) */
+    uint32_t model;       /* 0: factored RANS model (ns, nh, routes); 1: JOINT (FORMAT.md section 1) */
+    uint32_t nj;          /* JOINT precision, 8..13, default 13 */
 } bs_enc_params;
 
 bs_status bs_encoder_create(const bs_enc_item* items, int32_t n, const bs_enc_params* params, bs_encoder_t** out);

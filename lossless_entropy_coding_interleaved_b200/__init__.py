@@ -25,7 +25,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbs.so")
 
 OK, E_ARG, E_FORMAT, E_VERSION, E_SIZE, E_CUDA, E_CORRUPT, E_NOMEM, E_UNSUPPORTED = range(9)
-KIND_RANS, KIND_STORED, KIND_RAW = 0, 1, 2
+KIND_RANS, KIND_STORED, KIND_RAW, KIND_JOINT = 0, 1, 2, 3
 
 
 class BsError(RuntimeError):
@@ -56,7 +56,7 @@ class _StreamStats(ctypes.Structure):
 
 
 class _EncParams(ctypes.Structure):
-    _fields_ = [(k, ctypes.c_uint32) for k in ("log2_chunk", "ns", "nh", "max_routes", "force_rans")]
+    _fields_ = [(k, ctypes.c_uint32) for k in ("log2_chunk", "ns", "nh", "max_routes", "force_rans", "model", "nj")]
 
 
 class FwInfo(ctypes.Structure):
@@ -222,11 +222,13 @@ def workspace_bytes(container) -> int:
 
 
 def encode(tensors, log2_chunk: int = 16, ns: int = 11, nh: int = 5, max_routes: int = 15,
-           force_rans: bool = False, host_copy: bool = False, stream=None):
+           force_rans: bool = False, host_copy: bool = False, stream=None, model: str = "factored", nj: int = 13):
     """Encode device tensors into a container on the device (bs_encoder_*).
 
     tensors: sequence of (name, tensor) pairs; int16/bfloat16 CUDA tensors are BF16
-    words and uint8 CUDA tensors are opaque byte spans. Returns (d_container, h_container),
+    words and uint8 CUDA tensors are opaque byte spans. model "factored" codes BF16 tensors
+    as kind RANS (ns, nh, routes), "joint" as kind JOINT (one table of precision nj; faster
+    to decode). Returns (d_container, h_container),
     a uint8 CUDA tensor and, when host_copy, a uint8 numpy copy (else None).
     """
     keep = []
@@ -251,7 +253,8 @@ def encode(tensors, log2_chunk: int = 16, ns: int = 11, nh: int = 5, max_routes:
         it.name_bytes = len(nb)
     if dev is None:
         dev = torch.device("cuda")
-    prm = _EncParams(log2_chunk, ns, nh, max_routes, 1 if force_rans else 0)
+    assert model in ("factored", "joint")
+    prm = _EncParams(log2_chunk, ns, nh, max_routes, 1 if force_rans else 0, 1 if model == "joint" else 0, nj)
     enc = ctypes.c_void_p()
     _check(lib.bs_encoder_create(items, len(tensors), ctypes.byref(prm), ctypes.byref(enc)), "encoder_create")
     try:

@@ -1,6 +1,7 @@
 // bs_encode.cpp -- host side of the device encoder (include/bs.h, bs_encoder_*).
 //
-// It implements FORMAT.md section 6 (quantiser, route rule, pad word, STORED fallback)
+// It implements FORMAT.md section 6 (quantiser, route rule, joint model, pad word, STORED
+// fallback)
 // and the canonical layout of section 4.6 from that document. It shares no code with the
 // oracle. The statistics come from histogram_kernel and the per-chunk word counts from the
 // count pass of encode_kernel (bs_encode_kernels.cu). The write pass then places every
@@ -145,12 +146,51 @@ struct bs_encoder_t {
 
 namespace {
 
-// Build the model bytes and the encode tables of one tensor from its histogram.
+// Build the model bytes and the encode tables of one tensor from its histogram (pair
+// counts j = (s << 3) | h, then low-nibble counts).
 bool build_model(EncTensor& T, const bs_enc_params& P, const unsigned long long* hist) {
-    uint64_t cs[512], ceh[256 * 8];
-    for (int s = 0; s < 512; ++s) cs[s] = hist[s];
-    for (int k = 0; k < 256 * 8; ++k) ceh[k] = hist[512 + k];
-    const unsigned long long* cnib = hist + 512 + 256 * 8;
+    const unsigned long long* cnib = hist + 4096;
+    // nibble mode: constant when only one low nibble occurs
+    int seen = 0, only = 0;
+    for (int u = 0; u < 16; ++u)
+        if (cnib[u]) {
+            ++seen;
+            only = u;
+        }
+    T.nib_mode = seen == 1 ? 0x10u | static_cast<uint32_t>(only) : 0u;
+    if (P.model == 1) { // FORMAT.md section 6, joint model; section 3, its pad word
+        std::vector<uint64_t> cj(hist, hist + kJointPairs);
+        std::vector<uint32_t> Fj(kJointPairs);
+        if (!quantise(cj.data(), kJointPairs, 1u << P.nj, Fj.data())) return false;
+        uint32_t j_pad = 0, n_pairs = 0;
+        for (uint32_t j = 0; j < kJointPairs; ++j) {
+            if (Fj[j] > Fj[j_pad]) j_pad = j;
+            n_pairs += Fj[j] != 0;
+        }
+        T.pad_word = static_cast<uint16_t>(j_pad << 4);
+        T.n_routes = 0;
+        T.model.assign(4 + 4ull * n_pairs, 0); // FORMAT.md 4.3b
+        uint8_t* m = T.model.data();
+        put_u16(m, static_cast<uint16_t>(n_pairs));
+        uint64_t o = 4;
+        T.tables.assign(kEncJointWords, 0);
+        uint32_t cum = 0;
+        for (uint32_t j = 0; j < kJointPairs; ++j) {
+            T.tables[j] = Fj[j] | (cum << 16);
+            cum += Fj[j];
+            if (Fj[j]) {
+                put_u16(m + o, static_cast<uint16_t>(j));
+                put_u16(m + o + 2, static_cast<uint16_t>(Fj[j]));
+                o += 4;
+            }
+        }
+        return true;
+    }
+    uint64_t cs[512] = {}, ceh[256 * 8] = {};
+    for (uint32_t j = 0; j < kJointPairs; ++j) {
+        cs[j >> 3] += hist[j];
+        ceh[((j >> 3) & 0xFFu) * 8 + (j & 7u)] += hist[j]; // the sign is folded
+    }
     uint32_t Fs[512];
     if (!quantise(cs, 512, 1u << P.ns, Fs)) return false;
     uint8_t route[256];
@@ -172,14 +212,6 @@ bool build_model(EncTensor& T, const bs_enc_params& P, const unsigned long long*
             if (row[h] > row[h_pad]) h_pad = h;
     }
     T.pad_word = static_cast<uint16_t>((s_pad << 7) | (h_pad << 4));
-    // nibble mode: constant when only one low nibble occurs
-    int seen = 0, only = 0;
-    for (int u = 0; u < 16; ++u)
-        if (cnib[u]) {
-            ++seen;
-            only = u;
-        }
-    T.nib_mode = seen == 1 ? 0x10u | static_cast<uint32_t>(only) : 0u;
     // model bytes (FORMAT.md 4.3)
     uint32_t n_present = 0;
     for (int s = 0; s < 512; ++s) n_present += Fs[s] != 0;
@@ -251,11 +283,13 @@ bs_status run_encode_launches(bs_encoder_t* enc, uint8_t* d_scratch, uint8_t* d_
         it.cta_begin = p->total_ctas;
         it.table_words = static_cast<uint32_t>(T.tables.size());
         it.pad_word = T.pad_word;
+        const bool joint = enc->prm.model == 1;
         it.log2_chunk = static_cast<uint8_t>(enc->prm.log2_chunk);
-        it.ns = static_cast<uint8_t>(enc->prm.ns);
-        it.nh = static_cast<uint8_t>(enc->prm.nh);
+        it.ns = static_cast<uint8_t>(joint ? enc->prm.nj : enc->prm.ns);
+        it.nh = static_cast<uint8_t>(joint ? 0 : enc->prm.nh);
         it.n_routes = static_cast<uint8_t>(T.n_routes);
         it.nib_stored = T.nib_mode == 0;
+        it.joint = joint;
         p->total_ctas += static_cast<uint32_t>(ctas);
     }
     return flush();
@@ -270,7 +304,8 @@ bs_status bs_encoder_create(const bs_enc_item* items, int32_t n, const bs_enc_pa
     *out = nullptr;
     const bs_enc_params& P = *prm;
     if (P.log2_chunk < 8 || P.log2_chunk > 24 || P.ns < 1 || P.ns > kMaxNs || P.nh < kMinNh || P.nh > kMaxNh ||
-        P.ns + P.nh > kMaxPrecision || P.max_routes > kMaxRoutes)
+        P.ns + P.nh > kMaxPrecision || P.max_routes > kMaxRoutes || P.model > 1 ||
+        (P.model == 1 && (P.nj < kMinNj || P.nj > kMaxNj)))
         return BS_E_ARG;
     std::unique_ptr<bs_encoder_t> enc(new (std::nothrow) bs_encoder_t);
     if (!enc) return BS_E_NOMEM;
@@ -310,7 +345,7 @@ bs_status bs_encoder_create(const bs_enc_item* items, int32_t n, const bs_enc_pa
         if (!T.candidate) continue;
         T.n_chunks = (it.n_elems + (1ull << P.log2_chunk) - 1) >> P.log2_chunk;
         T.sc_tables = sc;
-        sc += up256(4ull * enc_table_words(kMaxRoutes));
+        sc += up256(4ull * kEncTableWordsMax);
         T.sc_words = sc;
         sc += up256(4ull * T.n_chunks);
         T.sc_offs = sc;
@@ -349,6 +384,15 @@ bs_status bs_encoder_run(bs_encoder_t* enc, void* d_scratch_v, size_t scratch_by
         ce = cudaMemcpyAsync(hist.data(), d_hist, 8ull * kHistBins, cudaMemcpyDeviceToHost, s);
         if (ce == cudaSuccess) ce = cudaStreamSynchronize(s);
         if (ce != cudaSuccess) return enc_cuda(ce);
+        if (P.model == 1) { // FORMAT.md section 6: more distinct pairs than 2^nj slots -> STORED
+            uint32_t n_pairs = 0;
+            for (uint32_t j = 0; j < kJointPairs; ++j) n_pairs += hist[j] != 0;
+            if (n_pairs > (1u << P.nj)) {
+                T.candidate = false;
+                T.kind = BS_KIND_STORED;
+                continue;
+            }
+        }
         if (!build_model(T, P, hist.data())) return BS_E_ARG;
         ce = cudaMemcpyAsync(d_scratch + T.sc_tables, T.tables.data(), 4ull * T.tables.size(), cudaMemcpyHostToDevice, s);
         if (ce != cudaSuccess) return enc_cuda(ce);
@@ -382,14 +426,16 @@ bs_status bs_encoder_run(bs_encoder_t* enc, void* d_scratch_v, size_t scratch_by
         const uint64_t C = 1ull << P.log2_chunk;
         for (uint64_t c = 0; c < T.n_chunks; ++c)
             T.coded += payload_bytes(std::min(C, T.item.n_elems - c * C), T.n_words[c], T.nib_mode == 0);
-        T.kind = (!P.force_rans && T.coded >= 2 * T.item.n_elems) ? BS_KIND_STORED : BS_KIND_RANS;
+        T.kind = (!P.force_rans && T.coded >= 2 * T.item.n_elems) ? BS_KIND_STORED
+                 : P.model == 1                                       ? BS_KIND_JOINT
+                                                                      : BS_KIND_RANS;
     }
     enc->dir_offset = kHeaderBytes;
     enc->names_offset = up16(enc->dir_offset + uint64_t(kDirEntryBytes) * enc->t.size());
     enc->names_bytes = names_bytes;
     uint64_t pos = up16(enc->names_offset + names_bytes);
     for (EncTensor& T : enc->t) {
-        if (T.kind == BS_KIND_RANS) {
+        if (is_coded(T.kind)) {
             T.model_offset = pos;
             pos = up16(pos + T.model.size());
             T.data_offset = pos;
@@ -424,16 +470,16 @@ bs_status bs_encoder_emit(bs_encoder_t* enc, void* d_scratch_v, void* d_containe
     if (ce != cudaSuccess) return enc_cuda(ce);
     // chunk offsets for the write pass
     for (EncTensor& T : enc->t) {
-        if (T.kind != BS_KIND_RANS) continue;
+        if (!is_coded(T.kind)) continue;
         ce = cudaMemcpyAsync(d_scratch + T.sc_offs, T.chunk_off.data(), 8ull * T.n_chunks, cudaMemcpyHostToDevice, s);
         if (ce != cudaSuccess) return enc_cuda(ce);
     }
     bs_status st = run_encode_launches(enc, d_scratch, d_container, 1, stream,
-                                       [](const EncTensor& T) { return T.kind == BS_KIND_RANS; });
+                                       [](const EncTensor& T) { return is_coded(T.kind); });
     if (st) return st;
     // verbatim data
     for (EncTensor& T : enc->t) {
-        if (T.kind == BS_KIND_RANS || T.item.n_elems == 0) continue;
+        if (is_coded(T.kind) || T.item.n_elems == 0) continue;
         const uint64_t bytes = T.kind == BS_KIND_STORED ? 2 * T.item.n_elems : T.item.n_elems;
         ce = cudaMemcpyAsync(d_container + T.data_offset, T.item.d_data, bytes, cudaMemcpyDeviceToDevice, s);
         if (ce != cudaSuccess) return enc_cuda(ce);
@@ -465,11 +511,11 @@ bs_status bs_encoder_emit(bs_encoder_t* enc, void* d_scratch_v, void* d_containe
         for (uint32_t i = 0; i < T.item.ndim; ++i) put_u64(d + 80 + 8 * i, T.item.shape[i]);
         std::memcpy(h + enc->names_offset + name_pos, T.name.data(), T.name.size());
         name_pos += T.name.size();
-        if (T.kind == BS_KIND_RANS) {
+        if (is_coded(T.kind)) {
             d[2] = static_cast<uint8_t>(P.log2_chunk);
             d[3] = kLanes;
-            d[4] = static_cast<uint8_t>(P.ns);
-            d[5] = static_cast<uint8_t>(P.nh);
+            d[4] = static_cast<uint8_t>(T.kind == BS_KIND_JOINT ? P.nj : P.ns);
+            d[5] = static_cast<uint8_t>(T.kind == BS_KIND_JOINT ? 0 : P.nh);
             d[6] = static_cast<uint8_t>(T.n_routes);
             d[7] = static_cast<uint8_t>(T.nib_mode);
             put_u64(d + 24, T.n_chunks);

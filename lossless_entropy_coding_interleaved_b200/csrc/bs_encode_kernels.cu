@@ -1,9 +1,10 @@
 // bs_encode_kernels.cu -- sm_100a kernels of the container encoder (FORMAT.md sections 3, 6).
 //
-// histogram_kernel: per-tensor counts of the sign+exponent symbol s = w >> 7, of
-// (exponent, h) pairs (h = the fraction's top three bits) and of the low nibbles. These are
-// the statistics the quantiser, the route rule and the nibble mode of FORMAT.md section 6
-// need. The counts go into per-CTA shared memory, then into global 64-bit bins.
+// histogram_kernel: per-tensor counts of the pairs j = w >> 4 = (s << 3) | h (sign+exponent
+// symbol s, the fraction's top three bits h) and of the low nibbles. The s counts and the
+// (exponent, h) counts that the factored model needs are sums of pair counts, and the JOINT
+// model uses the pair counts as they are (FORMAT.md section 6). The counts go into per-CTA
+// shared memory, then into global 64-bit bins.
 //
 // encode_kernel: one warp per chunk, lane j holds rANS state j (32-bit). It walks its
 // steps backwards from L = 2^16 as FORMAT.md section 2 specifies: each weight renormalises
@@ -28,9 +29,8 @@ __global__ void __launch_bounds__(512) histogram_kernel(const uint16_t* __restri
     const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
     for (uint64_t i = blockIdx.x * static_cast<uint64_t>(blockDim.x) + threadIdx.x; i < n; i += stride) {
         const uint32_t w = in[i];
-        atomicAdd(&h[w >> 7], 1u);
-        atomicAdd(&h[512 + ((w >> 4) & 0x7FFu)], 1u); // ((s & 0xFF) << 3) | h
-        atomicAdd(&h[512 + 2048 + (w & 15u)], 1u);
+        atomicAdd(&h[w >> 4], 1u);
+        atomicAdd(&h[4096 + (w & 15u)], 1u);
     }
     __syncthreads();
     for (uint32_t k = threadIdx.x; k < kHistBins; k += blockDim.x)
@@ -59,7 +59,7 @@ int launch_histogram(const uint16_t* in, uint64_t n, unsigned long long* d_hist,
 
 __global__ void __launch_bounds__(kEncWarps * 32) encode_kernel(const __grid_constant__ EncParams p) {
     __shared__ int s_item;
-    __shared__ uint32_t tab[512 + 8 * 16 + 64];
+    __shared__ uint32_t tab[kEncTableWordsMax]; // factored tables, or the JOINT table
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
     if (tid == 0) {
         int lo = 0, hi = static_cast<int>(p.n_items) - 1;
@@ -122,9 +122,19 @@ __global__ void __launch_bounds__(kEncWarps * 32) encode_kernel(const __grid_con
 #pragma unroll
         for (int k = 7; k >= 0; --k) {
             const uint32_t w = v[k], s = w >> 7, e = s & 0xFFu, h = (w >> 4) & 7u;
-            const uint32_t se = stab[s], he = hrows[route[e] * 8u + h];
-            const uint32_t qs = se & 0xFFFFu, cs = se >> 16, qh = he & 0xFFFFu, ch = he >> 16;
-            const uint32_t Q = qs * qh;
+            uint32_t Q, qh = 1, cs = 0, ch = 0; // JOINT: Q = Fj[j], cs = cum(j)
+            if (it.joint) {
+                const uint32_t je = tab[w >> 4];
+                Q = je & 0xFFFFu;
+                cs = je >> 16;
+            } else {
+                const uint32_t se = stab[s], he = hrows[route[e] * 8u + h];
+                const uint32_t qs = se & 0xFFFFu;
+                cs = se >> 16;
+                qh = he & 0xFFFFu;
+                ch = he >> 16;
+                Q = qs * qh;
+            }
             const bool emit = static_cast<uint64_t>(x) >= (static_cast<uint64_t>(Q) << (32 - P));
             if (p.write) {
                 const uint32_t m = __ballot_sync(0xFFFFFFFFu, emit);
@@ -141,7 +151,8 @@ __global__ void __launch_bounds__(kEncWarps * 32) encode_kernel(const __grid_con
             }
             if (emit) x >>= 16;
             const uint32_t r = x % Q;
-            x = ((x / Q) << P) + ((cs + r / qh) << nh) + ch + r % qh;
+            if (it.joint) x = ((x / Q) << P) + cs + r; // FORMAT.md section 2, the JOINT kind
+            else x = ((x / Q) << P) + ((cs + r / qh) << nh) + ch + r % qh;
         }
     }
     if (p.write) {

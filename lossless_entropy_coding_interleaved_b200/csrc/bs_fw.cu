@@ -65,12 +65,15 @@ inline FwScratch fw_scratch(uint64_t n) {
 
 // ------------------------------------------------------------------ transcode kernels
 // Section 10, code table: rank every present symbol by (count down, s up); the first 16
-// get codes. One CTA of 512 threads, thread s for symbol s.
+// get codes. One CTA of 512 threads, thread s for symbol s, whose count is the sum of its
+// eight (s, h) pair bins in the histogram.
 __global__ void __launch_bounds__(512) fw_select_kernel(const unsigned long long* __restrict__ hist,
                                                         uint8_t* __restrict__ sel) {
     __shared__ unsigned long long cnt[512];
     const uint32_t s = threadIdx.x;
-    cnt[s] = hist[s];
+    unsigned long long c8 = 0;
+    for (uint32_t h = 0; h < 8; ++h) c8 += hist[(s << 3) | h];
+    cnt[s] = c8;
     uint16_t* table = reinterpret_cast<uint16_t*>(sel + kSelTable);
     if (s < 16) table[s] = 0;
     __syncthreads();

@@ -25,7 +25,9 @@ uint64_t workspace_bytes_for(const std::vector<Tensor>& ts);
 // memory per block.
 bs_status build_workspace(std::vector<Tensor>& ts, std::vector<uint8_t>& image);
 
-// Bins decode work by precision (default ns=11/nh=5, or any), and verbatim copies into one
+// Bins decode work by kernel instance (factored at the default precisions or any other,
+// JOINT at nj = 13 or any other), and
+// verbatim copies into one
 // copy list. It launches a bin when the bin is full,
 // and launches every bin on flush().
 class DecodeBatch {
@@ -42,7 +44,7 @@ class DecodeBatch {
   private:
     struct Bin {
         std::unique_ptr<DecodeParams> p;
-        bool default_precision = false;
+        DecodeMode mode = DecodeMode::Default;
         uint32_t s_region = 0;  // largest s-table region of the queued tensors
         uint64_t chunks = 0;    // chunks queued; the CTA shape is chosen at flush
     };
@@ -50,7 +52,7 @@ class DecodeBatch {
     bs_status flush_copy(void* stream);
     unsigned long long* err_;
     uint32_t sms_ = 148;
-    Bin bins_[2];
+    Bin bins_[4];
     std::unique_ptr<CopyParams> cp_;
 };
 

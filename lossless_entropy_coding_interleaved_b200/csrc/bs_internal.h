@@ -19,6 +19,14 @@ constexpr uint32_t kStateL = 1u << 16;
 constexpr uint32_t kHeaderBytes = 64;
 constexpr uint32_t kDirEntryBytes = 144;
 constexpr uint32_t kMaxNs = 12, kMinNh = 3, kMaxNh = 5, kMaxPrecision = 16, kMaxRoutes = 15;
+// The JOINT kind (FORMAT.md sections 1-2): one table over the 4096 pairs j = (s << 3) | h,
+// precision nj. Its decode table (2^nj entries of 8 bytes) sits at offset 0 of shared
+// memory, and the rings follow at kJointRegion.
+constexpr uint32_t kJointPairs = 4096, kMinNj = 8, kMaxNj = 13;
+constexpr uint32_t kJointRegion = 8u << kMaxNj;
+inline bool is_coded(uint32_t kind) { return kind == BS_KIND_RANS || kind == BS_KIND_JOINT; }
+// joint table entry for slot (cum(j) + k): .x = F | (word << 16) with word = j << 4, .y = k
+inline uint32_t joint_table_bytes(uint32_t nj) { return 8u << nj; }
 // Bytes of a chunk payload: 32 start states, the nibble words when stored, the 16-bit
 // words, padded to 16 (FORMAT.md section 4.5).
 inline uint64_t payload_bytes(uint64_t n_c, uint32_t n_words, bool nib_stored) {
@@ -34,6 +42,8 @@ inline uint64_t payload_bytes(uint64_t n_c, uint32_t n_words, bool nib_stored) {
 // in quarters of kQuarterBytes (one 16-byte cp.async per lane fills a quarter), and its
 // nibble words through a ring of kNibRingBlocks blocks (128 bytes each).
 constexpr int kWarpsDefault = 24, kChainsDefault = 2, kWarpsGeneric = 20, kChainsGeneric = 2;
+// JOINT at the default precision (nj = 13): the table takes the first 64 KiB, then the rings.
+constexpr int kWarpsJoint = 24, kChainsJoint = 2;
 inline bool is_default_precision(uint32_t ns, uint32_t nh) { return ns == 11 && nh == 5; }
 inline int warps_for(uint32_t ns, uint32_t nh) { return is_default_precision(ns, nh) ? kWarpsDefault : kWarpsGeneric; }
 inline int chains_for(uint32_t ns, uint32_t nh) { return is_default_precision(ns, nh) ? kChainsDefault : kChainsGeneric; }
@@ -68,6 +78,10 @@ inline uint32_t smem_bytes_for(uint32_t ns, uint32_t nh) {
 }
 inline uint32_t smem_bytes_for(uint32_t ns, uint32_t warps, uint32_t chains) {
     return kHRegion + s_region_bytes(ns) + warps * chains * (kRingBytes + kNibRingBytes);
+}
+// JOINT: the table region (kJointRegion, the largest table), then the same rings.
+inline uint32_t joint_smem_bytes(uint32_t warps, uint32_t chains) {
+    return kJointRegion + warps * chains * (kRingBytes + kNibRingBytes);
 }
 
 // Workspace layout: a 256-byte error block, then 256-aligned tables per RANS tensor.
@@ -153,6 +167,9 @@ struct CopyParams {
 //   [512, 512 + 8*rows)     fraction rows over h (the last one UNIFORM): qh | (cum_h << 16)
 //   [.., + 64)              route: 256 bytes, row index per exponent
 inline uint32_t enc_table_words(uint32_t n_routes) { return 512 + 8 * (n_routes + 1) + 64; }
+// JOINT encode table: Fj | (cum << 16) per pair j
+constexpr uint32_t kEncJointWords = 4096;
+constexpr uint32_t kEncTableWordsMax = kEncJointWords; // larger than enc_table_words(kMaxRoutes)
 
 struct EncItem {
     const uint16_t* in;         // device: original words
@@ -163,7 +180,7 @@ struct EncItem {
     uint32_t cta_begin;
     uint32_t table_words;
     uint16_t pad_word;
-    uint8_t log2_chunk, ns, nh, n_routes, nib_stored, pad1;
+    uint8_t log2_chunk, ns, nh, n_routes, nib_stored, joint; // JOINT: ns = nj, nh = n_routes = 0
 };
 static_assert(sizeof(EncItem) == 56, "EncItem layout");
 
@@ -179,7 +196,9 @@ struct EncParams {
     EncItem item[kMaxEncItems];
 };
 
-constexpr uint32_t kHistBins = 512 + 256 * 8 + 16; // s counts, (exponent, h) counts, low-nibble counts
+// (s, h) pair counts (j = w >> 4, from which the s and (exponent, h) counts follow), then
+// the low-nibble counts
+constexpr uint32_t kHistBins = 4096 + 16;
 int launch_histogram(const uint16_t* in, uint64_t n, unsigned long long* d_hist, void* stream);
 int launch_encode(const EncParams& p, void* stream);
 
@@ -189,7 +208,19 @@ void record_cuda_error(int e);
 void count_launch();
 
 // Kernel launchers (bs_kernels.cu). They return a cudaError_t as int.
-int launch_decode(const DecodeParams& p, bool default_precision, uint32_t smem_bytes, void* stream);
+// Which decode_kernel instance a launch uses: the default precisions (ns 11, nh 5), any
+// other factored precisions, or the JOINT kind.
+// JOINT at nj = 13 (the default) has a compile-time instance; other nj use a generic one.
+enum class DecodeMode { Default = 0, Generic = 1, Joint = 2, JointGeneric = 3 };
+constexpr uint32_t kDefaultNj = 13;
+// The largest CTA shape of each mode (small launches take fewer warps, see launch_warps).
+inline uint32_t max_warps_of(DecodeMode m) {
+    return m == DecodeMode::Default ? kWarpsDefault : m == DecodeMode::Joint ? kWarpsJoint : kWarpsGeneric;
+}
+inline uint32_t chains_of(DecodeMode m) {
+    return m == DecodeMode::Default ? kChainsDefault : m == DecodeMode::Joint ? kChainsJoint : kChainsGeneric;
+}
+int launch_decode(const DecodeParams& p, DecodeMode mode, uint32_t smem_bytes, void* stream);
 int launch_copy(const CopyParams& p, void* stream);
 int launch_checksum(const void* data, uint64_t n, int raw_bytes, unsigned long long* d_sum, void* stream);
 int max_dynamic_smem();

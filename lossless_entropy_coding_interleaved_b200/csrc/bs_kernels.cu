@@ -63,20 +63,18 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
 // One chunk in flight on a warp: lane j holds state j.
+// Only what the step loop needs stays in registers; the rest (the rings' shared-memory
+// addresses, the quarter count, the stream and nibble pointers, the chunk index) is derived
+// where it is used.
 struct Chain {
     uint32_t x;               // rANS state, in [2^16, 2^32) between weights
     uint32_t posb;            // bytes of the word stream consumed (warp-uniform)
     uint32_t fq;              // ring quarters requested (warp-uniform)
-    uint32_t total_q, stream_bytes, nc, n_blocks;
-    uint32_t ring;            // shared-memory address of the word ring
-    uint32_t ring_off;        // the same ring as an offset into the dynamic smem array
-    uint32_t nring;           // shared-memory address of the nibble ring
-    uint32_t nring_off;       // the same ring as an offset into the dynamic smem array
+    uint32_t stream_bytes, nc, n_blocks;
+    uint32_t ring_off;        // the word ring, as an offset into the dynamic smem array
+    uint32_t nring_off;       // the nibble ring, as an offset into the dynamic smem array
     uint32_t raw;             // nibble word of the current block (constant mode: c in every nibble)
-    const uint8_t* stream;
-    const uint8_t* nib;       // nibble words (block-major), or null in constant mode
-    uint16_t* out;
-    uint64_t chunk;
+    const uint8_t* payload;   // the chunk's payload: start states, nibble words (if stored), words
     bool live;                // a real chunk (false: a filler chain that is never stored)
     bool bad;
 };
@@ -84,10 +82,13 @@ struct Chain {
 // NS/NH > 0: compile-time precisions (the default container); 0: read from the item.
 // SHAPE_FROM_PARAMS: the launch's warps per CTA come from the parameters (small launches);
 // otherwise the CTA has WARPS warps, a compile-time constant (measured 3% faster).
-template <int WARPS, int CHAINS, int NS, int NH, bool SHAPE_FROM_PARAMS>
+// JOINT: the JOINT kind (FORMAT.md sections 1-2): one table of 2^nj slots (nj = item.ns),
+// one lookup and one multiply-add per weight.
+template <int WARPS, int CHAINS, int NS, int NH, bool SHAPE_FROM_PARAMS, bool JOINT>
 __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int kChains = CHAINS;
-    // dynamic smem: [fraction rows, one copy per lane][s-table][rings]
+    // dynamic smem: [fraction rows, one copy per lane][s-table][rings], or for JOINT
+    // [joint table][rings]
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ int s_item;
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
@@ -105,8 +106,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
     const DecodeItem& it = p.item[s_item];
     const uint32_t ns = NS > 0 ? NS : it.ns, nh = NH > 0 ? NH : it.nh, P = ns + nh;
 
-    // stage the tables: the s-table as it is, each fraction entry once per lane
-    {
+    if (JOINT) { // stage the joint table as it is
+        const uint32_t jb = 8u << ns;
+        uint4* jdst = reinterpret_cast<uint4*>(smem);
+        for (uint32_t k = tid; k < jb / 16u; k += blockDim.x) jdst[k] = __ldg(it.tables + k);
+    } else { // stage the tables: the s-table as it is, each fraction entry once per lane
         const uint32_t sb = 8u << ns;
         uint4* sdst = reinterpret_cast<uint4*>(smem + kHRegion);
         for (uint32_t k = tid; k < sb / 16u; k += blockDim.x) sdst[k] = __ldg(it.tables + k);
@@ -127,51 +131,44 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
 
     const bool nib_stored = it.nib_mode == 0;
     const uint32_t raw_const = (it.nib_mode & 15u) * 0x11111111u;
-    const uint32_t rings = kHRegion + s_region_bytes(ns);                  // a multiple of kRingBytes
+    const uint32_t rings = JOINT ? kJointRegion : kHRegion + s_region_bytes(ns); // a multiple of kRingBytes
     const uint32_t ring_off = rings + (warp * kChains) * kRingBytes;       // this warp's first word ring
     const uint32_t nring_off = rings + warps * kChains * kRingBytes + (warp * kChains) * kNibRingBytes;
-    const uint32_t ring_base = smem_u32(smem) + ring_off, nring_base = smem_u32(smem) + nring_off;
+    const uint32_t smem_base = smem_u32(smem);
+    uint16_t* const out0 = it.out + (chunk0 << log2c); // chain k writes from out0 + k * C
     Chain c[kChains];
     uint32_t nb = 0;
 #pragma unroll
     for (int k = 0; k < kChains; ++k) {
         Chain& h = c[k];
-        h.chunk = chunk0 + k;
-        h.live = h.chunk < n_chunks;
-        h.ring = ring_base + k * kRingBytes;
+        const uint64_t chunk = chunk0 + k;
+        h.live = chunk < n_chunks;
         h.ring_off = ring_off + k * kRingBytes;
-        h.nring = nring_base + k * kNibRingBytes;
         h.nring_off = nring_off + k * kNibRingBytes;
         h.posb = 0;
         h.fq = 0;
         h.bad = false;
         h.raw = raw_const;
-        h.nib = nullptr;
         if (h.live) {
-            const uint8_t* ent = it.chunk_table + 16 * h.chunk;
+            const uint8_t* ent = it.chunk_table + 16 * chunk;
             const uint64_t off = __ldg(reinterpret_cast<const unsigned long long*>(ent));
             const uint32_t n_words = __ldg(reinterpret_cast<const unsigned int*>(ent + 8));
-            const uint8_t* payload = it.container + off;
-            const uint64_t base = h.chunk << log2c;
+            h.payload = it.container + off;
+            const uint64_t base = chunk << log2c;
             h.nc = static_cast<uint32_t>(min(C, n_elems - base));
             h.n_blocks = (h.nc + 255u) >> 8; // blocks of 8 steps
-            if (nib_stored) h.nib = payload + 128;
-            h.stream = payload + 128 + (nib_stored ? 128u * h.n_blocks : 0u);
             h.stream_bytes = 2u * n_words;
-            h.total_q = (h.stream_bytes + kQuarterBytes - 1) / kQuarterBytes;
-            h.out = it.out + base;
-            h.x = __ldg(reinterpret_cast<const unsigned int*>(payload) + lane);
+            h.x = __ldg(reinterpret_cast<const unsigned int*>(h.payload) + lane);
             h.bad = h.x < kStateL;
         } else { // filler: decodes from L and its own (unfilled) ring; nothing is stored
-            h.stream_bytes = h.total_q = h.nc = h.n_blocks = 0;
-            h.stream = nullptr;
-            h.out = nullptr;
+            h.stream_bytes = h.nc = h.n_blocks = 0;
+            h.payload = nullptr;
             h.x = kStateL;
         }
         nb = max(nb, h.n_blocks);
     }
 
-    const uint32_t smask8 = ((1u << ns) - 1u) << 3, hmask7 = ((1u << nh) - 1u) << 7;
+    const uint32_t smask8 = ((1u << ns) - 1u) << 3, hmask7 = ((1u << nh) - 1u) << 7; // JOINT: smask8 masks the slot
     const uint32_t lt = lanemask_lt(), lane4 = lane << 2;
     const uint32_t mul2 = p.mul2, mul65536 = p.mul65536;
 
@@ -189,21 +186,23 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
 #pragma unroll
         for (int k = 0; k < kChains; ++k) {
             Chain& h = c[k];
-            if (h.nib && blk < h.n_blocks) {
+            if (nib_stored && blk < h.n_blocks) { // nibble words start after the 128-byte states
                 for (uint32_t b = (blk == 0 ? 0u : blk + 4u); b < blk + 6u; b += 2u) {
                     const uint32_t byte = 128u * b + 16u * lane; // lanes 0-15: blocks b and b+1
                     if (lane < 16 && byte < 128u * h.n_blocks)
-                        cp_async16(h.nring + (byte & (kNibRingBytes - 1u)), h.nib + byte, 16u);
+                        cp_async16(smem_base + h.nring_off + (byte & (kNibRingBytes - 1u)), h.payload + 128 + byte, 16u);
                 }
             }
             if (blk < h.n_blocks) {
                 const uint32_t q = h.posb / kQuarterBytes;
-                if (h.fq <= min(q + 2, h.total_q - 1)) newest_needed = true;
-                while (h.fq < q + 4 && h.fq < h.total_q) {
+                const uint32_t total_q = (h.stream_bytes + kQuarterBytes - 1) / kQuarterBytes;
+                const uint8_t* stream = h.payload + 128 + (nib_stored ? 128u * h.n_blocks : 0u);
+                if (h.fq <= min(q + 2, total_q - 1)) newest_needed = true;
+                while (h.fq < q + 4 && h.fq < total_q) {
                     const uint32_t byte = h.fq * kQuarterBytes + 16u * lane;
-                    const uint32_t dst = h.ring + (byte & (kRingBytes - 1u));
-                    if ((h.fq + 1) * kQuarterBytes <= h.stream_bytes) cp_async16(dst, h.stream + byte, 16u);
-                    else if (byte < h.stream_bytes) cp_async16(dst, h.stream + byte, min(16u, h.stream_bytes - byte));
+                    const uint32_t dst = smem_base + h.ring_off + (byte & (kRingBytes - 1u));
+                    if ((h.fq + 1) * kQuarterBytes <= h.stream_bytes) cp_async16(dst, stream + byte, 16u);
+                    else if (byte < h.stream_bytes) cp_async16(dst, stream + byte, min(16u, h.stream_bytes - byte));
                     ++h.fq;
                 }
             }
@@ -221,7 +220,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
 #pragma unroll
         for (int k = 0; k < kChains; ++k) {
             Chain& h = c[k];
-            if (h.nib && (full || b < h.n_blocks))
+            if (nib_stored && h.live && (full || b < h.n_blocks))
                 h.raw = *reinterpret_cast<const uint32_t*>(smem + h.nring_off + ((128u * b) & (kNibRingBytes - 1u)) + lane4);
         }
     };
@@ -235,6 +234,17 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
             uint2 se[kChains];
             uint32_t fe[kChains], xn[kChains], m[kChains], w[kChains];
             bool need[kChains];
+            if (JOINT) { // the slot's entry: F and the word's (s, h) part in .x, the rank in .y
+#pragma unroll
+                for (int k = 0; k < kChains; ++k)
+                    se[k] = *reinterpret_cast<const uint2*>(smem + ((c[k].x << 3) & smask8));
+#pragma unroll
+                for (int k = 0; k < kChains; ++k) {
+                    xn[k] = (se[k].x & 0xFFFFu) * (c[k].x >> ns) + se[k].y;
+                    need[k] = xn[k] < kStateL;
+                    fe[k] = 0;
+                }
+            } else {
 #pragma unroll
             for (int k = 0; k < kChains; ++k) // the s-entry from the slot's high ns bits
                 se[k] = *reinterpret_cast<const uint2*>(smem + kHRegion + ((c[k].x >> (nh - 3)) & smask8));
@@ -250,6 +260,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
                 const uint32_t Fh = __byte_perm(fe[k], 0u, 0x4442), bh = fe[k] >> 24;
                 xn[k] = (Fs * Fh) * t + (bs * Fh + bh);
                 need[k] = xn[k] < kStateL;
+            }
             }
             // renormalise: lanes below 2^16 take the next words, in lane order
             // (branch-free: every lane reads; the ones that need no word discard it)
@@ -268,9 +279,14 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
                 // (s << 7) | (h << 4): s sits pre-shifted in se.y, h in bits 4-6 of fe, and the
                 // rest of fe's low half is zero, so one masked select builds the low half (the
                 // high half is dropped when the pair is packed)
-                const uint32_t word = (se[k].y & 0xFF80u) | fe[k];
-                if (s & 1) o[k][s >> 1] = __byte_perm(o[k][s >> 1], word, 0x5410);
-                else o[k][s >> 1] = word;
+                if (JOINT) { // the words sit in the high halves of the entries
+                    if (s & 1) o[k][s >> 1] = __byte_perm(o[k][s >> 1], se[k].x, 0x7632);
+                    else o[k][s >> 1] = se[k].x;
+                } else {
+                    const uint32_t word = (se[k].y & 0xFF80u) | fe[k];
+                    if (s & 1) o[k][s >> 1] = __byte_perm(o[k][s >> 1], word, 0x5410);
+                    else o[k][s >> 1] = word;
+                }
             }
         }
         // the low nibbles of the pairs (FORMAT.md section 3: pair p at bits 4p and 16+4p)
@@ -299,7 +315,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
 #pragma unroll
             for (int k = 0; k < kChains; ++k) {
                 Chain& h = c[k];
-                if (h.live) *reinterpret_cast<uint4*>(h.out + i0) = make_uint4(o[k][0], o[k][1], o[k][2], o[k][3]);
+                if (h.live) *reinterpret_cast<uint4*>(out0 + k * C + i0) = make_uint4(o[k][0], o[k][1], o[k][2], o[k][3]);
             }
         }
     }
@@ -322,11 +338,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
                 if (b < h.n_blocks) {
                     const uint32_t i0 = (b << 8) + (lane << 3);
                     if (i0 + 8 <= h.nc) {
-                        *reinterpret_cast<uint4*>(h.out + i0) = make_uint4(o[k][0], o[k][1], o[k][2], o[k][3]);
+                        *reinterpret_cast<uint4*>(out0 + k * C + i0) = make_uint4(o[k][0], o[k][1], o[k][2], o[k][3]);
                     } else {
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
-                            if (i0 + e < h.nc) h.out[i0 + e] = static_cast<uint16_t>(o[k][e >> 1] >> (16 * (e & 1)));
+                            if (i0 + e < h.nc) out0[k * C + i0 + e] = static_cast<uint16_t>(o[k][e >> 1] >> (16 * (e & 1)));
                     }
                     if (b + 1 == h.n_blocks) // end check: state back at L, every word consumed
                         h.bad |= (h.x != kStateL) | (h.posb != h.stream_bytes);
@@ -340,7 +356,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
     for (int k = 0; k < kChains; ++k) {
         if (c[k].live && __any_sync(0xFFFFFFFFu, c[k].bad) && lane == 0) {
             atomicOr(p.err, 1ull);
-            atomicMin(p.err + 1, (static_cast<unsigned long long>(it.tensor_index) << 40) | c[k].chunk);
+            atomicMin(p.err + 1, (static_cast<unsigned long long>(it.tensor_index) << 40) | (chunk0 + k));
         }
     }
 }
@@ -399,9 +415,9 @@ int max_dynamic_smem() {
     return v;
 }
 
-template <int WARPS, int CHAINS, int NS, int NH, bool SHAPE_FROM_PARAMS>
+template <int WARPS, int CHAINS, int NS, int NH, bool SHAPE_FROM_PARAMS, bool JOINT>
 static int launch_decode_shape(const DecodeParams& p, uint32_t smem_bytes, cudaStream_t s) {
-    auto kernel = decode_kernel<WARPS, CHAINS, NS, NH, SHAPE_FROM_PARAMS>;
+    auto kernel = decode_kernel<WARPS, CHAINS, NS, NH, SHAPE_FROM_PARAMS, JOINT>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes));
     if (e != cudaSuccess) return e;
     kernel<<<p.total_ctas, p.warps * 32, smem_bytes, s>>>(p);
@@ -409,18 +425,22 @@ static int launch_decode_shape(const DecodeParams& p, uint32_t smem_bytes, cudaS
     return cudaGetLastError();
 }
 
-template <int WARPS, int CHAINS, int NS, int NH>
+template <int WARPS, int CHAINS, int NS, int NH, bool JOINT>
 static int launch_decode_t(const DecodeParams& p, uint32_t smem_bytes, cudaStream_t s) {
     if (p.warps < 1 || p.warps > WARPS) return cudaErrorInvalidValue;
-    return p.warps == WARPS ? launch_decode_shape<WARPS, CHAINS, NS, NH, false>(p, smem_bytes, s)
-                            : launch_decode_shape<WARPS, CHAINS, NS, NH, true>(p, smem_bytes, s);
+    return p.warps == WARPS ? launch_decode_shape<WARPS, CHAINS, NS, NH, false, JOINT>(p, smem_bytes, s)
+                            : launch_decode_shape<WARPS, CHAINS, NS, NH, true, JOINT>(p, smem_bytes, s);
 }
 
-int launch_decode(const DecodeParams& p, bool default_precision, uint32_t smem_bytes, void* stream) {
+int launch_decode(const DecodeParams& p, DecodeMode mode, uint32_t smem_bytes, void* stream) {
     if (p.total_ctas == 0) return cudaSuccess;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return default_precision ? launch_decode_t<kWarpsDefault, kChainsDefault, 11, 5>(p, smem_bytes, s)
-                             : launch_decode_t<kWarpsGeneric, kChainsGeneric, 0, 0>(p, smem_bytes, s);
+    switch (mode) {
+    case DecodeMode::Default: return launch_decode_t<kWarpsDefault, kChainsDefault, 11, 5, false>(p, smem_bytes, s);
+    case DecodeMode::Joint: return launch_decode_t<kWarpsJoint, kChainsJoint, 13, 5, true>(p, smem_bytes, s);
+    case DecodeMode::JointGeneric: return launch_decode_t<kWarpsGeneric, kChainsGeneric, 0, 5, true>(p, smem_bytes, s);
+    default: return launch_decode_t<kWarpsGeneric, kChainsGeneric, 0, 0, false>(p, smem_bytes, s);
+    }
 }
 
 int launch_copy(const CopyParams& p, void* stream) {

@@ -22,10 +22,12 @@
 
 namespace bs {
 
-// Largest decode tables the array holds: the s-table at ns = 12 (32 KiB) plus 16 compact
-// fraction rows of 2^5 entries (2 KiB). That is every tensor a valid container can hold;
-// larger tables would get BS_E_SIZE.
-constexpr uint32_t kNoAllocTableBytes = (8u << kMaxNs) + 4u * (kMaxRoutes + 1) * (1u << kMaxNh);
+// Largest decode tables the array holds: the JOINT table at nj = 13 (64 KiB), which is
+// larger than any factored one (the s-table at ns = 12, 32 KiB, plus 16 compact fraction
+// rows of 2^5 entries, 2 KiB). That is every tensor a valid container can hold; larger
+// tables would get BS_E_SIZE.
+constexpr uint32_t kNoAllocFactoredBytes = (8u << kMaxNs) + 4u * (kMaxRoutes + 1) * (1u << kMaxNh);
+constexpr uint32_t kNoAllocTableBytes = (8u << kMaxNj) > kNoAllocFactoredBytes ? (8u << kMaxNj) : kNoAllocFactoredBytes;
 constexpr uint32_t kNoAllocBytes = 256 + kNoAllocTableBytes; // error block, then tables
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
@@ -126,6 +128,34 @@ __global__ void __launch_bounds__(512) noalloc_tables_kernel(const uint8_t* mode
     }
 }
 
+// The JOINT table (bs_internal.h): for the pair of slot cum(j) + k, .x = F | ((j << 4) << 16)
+// and .y = k. One CTA; thread 0 takes the running sums, then every thread fills pairs.
+// Writes are bounded by 2^nj slots, so a device copy that differs from the host's validated
+// one cannot write outside the table.
+__global__ void __launch_bounds__(512) noalloc_joint_kernel(const uint8_t* model, uint32_t n_pairs, uint32_t nj) {
+    __shared__ uint32_t cum[kJointPairs + 1];
+    uint32_t* jt = reinterpret_cast<uint32_t*>(g_noalloc_scratch + 256);
+    const uint8_t* pairs = model + 4;
+    if (threadIdx.x == 0) {
+        uint32_t acc = 0;
+        for (uint32_t i = 0; i < n_pairs; ++i) {
+            cum[i] = acc;
+            acc += pairs[4 * i + 2] | (pairs[4 * i + 3] << 8);
+        }
+        cum[n_pairs] = acc;
+    }
+    __syncthreads();
+    const uint32_t M = 1u << nj;
+    for (uint32_t i = threadIdx.x; i < n_pairs; i += blockDim.x) {
+        const uint32_t j = (pairs[4 * i] | (pairs[4 * i + 1] << 8)) & (kJointPairs - 1u);
+        const uint32_t q = cum[i + 1] - cum[i];
+        for (uint32_t k = 0; k < q && cum[i] + k < M; ++k) {
+            jt[2 * (cum[i] + k)] = (q & 0xFFFFu) | ((j << 4) << 16);
+            jt[2 * (cum[i] + k) + 1] = k;
+        }
+    }
+}
+
 } // namespace bs
 
 using namespace bs;
@@ -152,8 +182,8 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
     const uint32_t nib_mode = d[7];
     const uint64_t n = rd64(d + 16), n_chunks = rd64(d + 24), model_off = rd64(d + 32), model_bytes = rd64(d + 40);
     const uint64_t data_off = rd64(d + 48), data_bytes = rd64(d + 56);
-    if (kind > BS_KIND_RAW || ndim > 8 || rd64(d + 72) != 0) return BS_E_FORMAT;
-    if (kind != BS_KIND_RANS && nib_mode != 0) return BS_E_FORMAT;
+    if (kind > BS_KIND_JOINT || ndim > 8 || rd64(d + 72) != 0) return BS_E_FORMAT;
+    if (!is_coded(kind) && nib_mode != 0) return BS_E_FORMAT;
     if (uint64_t(rd32(d + 8)) + rd32(d + 12) > names_bytes) return BS_E_FORMAT;
     unsigned __int128 prod = 1;
     for (uint32_t i = 0; i < 8; ++i) {
@@ -171,7 +201,7 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
     if (out_bytes != want) return BS_E_SIZE;
     if (want && (!d_out || (reinterpret_cast<uintptr_t>(d_out) & 15u))) return BS_E_ARG;
 
-    if (kind != BS_KIND_RANS) { // verbatim: no scratch needed, the copy kernel does it
+    if (!is_coded(kind)) { // verbatim: no scratch needed, the copy kernel does it
         if (data_bytes != want) return BS_E_FORMAT;
         if (want == 0) return BS_OK;
         CopyParams cp;
@@ -186,14 +216,33 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
         }
         return BS_OK;
     }
-    if (lanes != kLanes || log2c < 8 || log2c > 24 || ns < 1 || ns > kMaxNs || nh < kMinNh || nh > kMaxNh ||
-        ns + nh > kMaxPrecision || n_routes > kMaxRoutes || n == 0 || n > (1ull << 40))
+    const bool joint = kind == BS_KIND_JOINT;
+    if (lanes != kLanes || log2c < 8 || log2c > 24 || n == 0 || n > (1ull << 40)) return BS_E_FORMAT;
+    if (joint ? (ns < kMinNj || ns > kMaxNj || nh != 0 || n_routes != 0)
+              : (ns < 1 || ns > kMaxNs || nh < kMinNh || nh > kMaxNh || ns + nh > kMaxPrecision || n_routes > kMaxRoutes))
         return BS_E_FORMAT;
     if (nib_mode != 0 && (nib_mode & 0xF0u) != 0x10u) return BS_E_FORMAT;
     if (n_chunks != ((n + (1ull << log2c) - 1) >> log2c) || data_bytes != 16 * n_chunks) return BS_E_FORMAT;
-    if (model_off % 16 || !in_range(model_off, model_bytes, len) || model_bytes < 264) return BS_E_FORMAT;
+    if (model_off % 16 || !in_range(model_off, model_bytes, len) || model_bytes < (joint ? 8u : 264u))
+        return BS_E_FORMAT;
     const uint8_t* m = b + model_off;
-    const uint32_t n_present = rd16(m);
+    const uint32_t n_present = joint ? 0 : rd16(m);
+    uint32_t n_pairs = 0;
+    if (joint) { // FORMAT.md section 4.3b
+        n_pairs = rd16(m);
+        if (n_pairs < 1 || n_pairs > kJointPairs || rd16(m + 2) != 0 || model_bytes != 4 + 4ull * n_pairs)
+            return BS_E_FORMAT;
+        uint64_t sumj = 0;
+        int prevj = -1;
+        for (uint32_t i = 0; i < n_pairs; ++i) {
+            const int j = rd16(m + 4 + 4 * i);
+            const uint32_t q = rd16(m + 6 + 4 * i);
+            if (j <= prevj || j >= static_cast<int>(kJointPairs) || q == 0) return BS_E_FORMAT;
+            prevj = j;
+            sumj += q;
+        }
+        if (sumj != (1ull << ns)) return BS_E_FORMAT;
+    } else {
     if (n_present < 1 || n_present > 512 || model_bytes != 260 + 4ull * n_present + 16ull * n_routes)
         return BS_E_FORMAT;
     uint64_t sum = 0;
@@ -214,6 +263,7 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
         for (int h = 0; h < 8; ++h) sum += rd16(route + 256 + 16 * r + 2 * h);
         if (sum != (1ull << nh)) return BS_E_FORMAT;
     }
+    }
     const uint64_t C = 1ull << log2c;
     for (uint64_t c = 0; c < n_chunks; ++c) {
         const uint8_t* e = b + data_off + 16 * c;
@@ -221,7 +271,7 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
         if (rd64(e) % 16 || rd32(e + 12) != 0 || !in_range(rd64(e), payload_bytes(nc, rd32(e + 8), nib_mode == 0), len))
             return BS_E_FORMAT;
     }
-    const uint32_t tb = table_bytes_for(ns, nh, n_routes);
+    const uint32_t tb = joint ? joint_table_bytes(ns) : table_bytes_for(ns, nh, n_routes);
     if (tb > kNoAllocTableBytes) return BS_E_SIZE; // larger than the static array holds
 
     // --- set-up: the array's device address on this device ---
@@ -239,7 +289,8 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
         record_cuda_error(ce);
         return BS_E_CUDA;
     }
-    noalloc_tables_kernel<<<1, 512, 0, stream>>>(d_container + model_off, n_present, ns, nh, n_routes);
+    if (joint) noalloc_joint_kernel<<<1, 512, 0, stream>>>(d_container + model_off, n_pairs, ns);
+    else noalloc_tables_kernel<<<1, 512, 0, stream>>>(d_container + model_off, n_present, ns, nh, n_routes);
     count_launch();
     ce = cudaGetLastError();
     if (ce != cudaSuccess) {
@@ -249,13 +300,15 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
     // --- the decode kernel, unchanged, with its tables and error block in the array ---
     DecodeParams p; // about 31 KiB of launch parameters, on the stack (no heap use)
     p.n_items = 1;
-    const bool dflt = is_default_precision(ns, nh);
-    const uint32_t chains = dflt ? kChainsDefault : kChainsGeneric;
+    const bool dflt = joint ? ns == kDefaultNj : is_default_precision(ns, nh); // the larger shape
+    const DecodeMode mode = joint ? (dflt ? DecodeMode::Joint : DecodeMode::JointGeneric)
+                                  : dflt ? DecodeMode::Default : DecodeMode::Generic;
+    const uint32_t chains = chains_of(mode);
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
         sms = 148;
-    p.warps = launch_warps(n_chunks, dflt ? kWarpsDefault : kWarpsGeneric, chains, static_cast<uint32_t>(sms));
+    p.warps = launch_warps(n_chunks, max_warps_of(mode), chains, static_cast<uint32_t>(sms));
     const uint64_t per_cta = uint64_t(p.warps) * chains;
     p.total_ctas = static_cast<uint32_t>((n_chunks + per_cta - 1) / per_cta);
     p.err = reinterpret_cast<unsigned long long*>(scratch);
@@ -274,7 +327,7 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
     it.nh = static_cast<uint8_t>(nh);
     it.n_routes = static_cast<uint8_t>(n_routes);
     it.nib_mode = static_cast<uint8_t>(nib_mode);
-    int e = launch_decode(p, dflt, smem_bytes_for(ns, p.warps, chains), stream);
+    int e = launch_decode(p, mode, joint ? joint_smem_bytes(p.warps, chains) : smem_bytes_for(ns, p.warps, chains), stream);
     if (e) {
         record_cuda_error(e);
         return BS_E_CUDA;

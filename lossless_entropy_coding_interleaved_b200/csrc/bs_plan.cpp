@@ -129,8 +129,8 @@ bs_status parse(Reader& rd, std::vector<Tensor>& out) {
         t.data_bytes = get_u64(d + 56);
         t.checksum = get_u64(d + 64);
         for (int i = 0; i < 8; ++i) t.shape[i] = get_u64(d + 80 + 8 * i);
-        if (t.kind > BS_KIND_RAW || t.ndim > 8) return BS_E_FORMAT;
-        if (t.kind != BS_KIND_RANS && t.nib_mode != 0) return BS_E_FORMAT;
+        if (t.kind > BS_KIND_JOINT || t.ndim > 8) return BS_E_FORMAT;
+        if (!is_coded(t.kind) && t.nib_mode != 0) return BS_E_FORMAT;
         if (uint64_t(name_off) + name_len > names_bytes) return BS_E_FORMAT;
         t.name.assign(reinterpret_cast<const char*>(nbuf.data() + name_off), name_len);
         unsigned __int128 prod = 1;
@@ -142,7 +142,7 @@ bs_status parse(Reader& rd, std::vector<Tensor>& out) {
             if (t.shape[i] != 0) return BS_E_FORMAT;
         if (prod != t.n_elems) return BS_E_FORMAT;
         if (t.data_offset % 16 || !inside(t.data_offset, t.data_bytes, len)) return BS_E_FORMAT;
-        if (t.kind != BS_KIND_RANS) {
+        if (!is_coded(t.kind)) {
             if (t.kind == BS_KIND_STORED && t.n_elems > (1ull << 62)) return BS_E_FORMAT;
             const uint64_t want = t.kind == BS_KIND_STORED ? 2 * t.n_elems : t.n_elems;
             if (t.data_bytes != want) return BS_E_FORMAT;
@@ -150,22 +150,43 @@ bs_status parse(Reader& rd, std::vector<Tensor>& out) {
             out.push_back(std::move(t));
             continue;
         }
-        // RANS
+        // RANS and JOINT
+        const bool joint = t.kind == BS_KIND_JOINT;
         if (t.lanes != kLanes || t.log2_chunk < 8 || t.log2_chunk > 24) return BS_E_FORMAT;
-        if (t.ns < 1 || t.ns > kMaxNs || t.nh < kMinNh || t.nh > kMaxNh || t.ns + t.nh > kMaxPrecision ||
-            t.n_routes > kMaxRoutes)
+        if (joint) {
+            if (t.ns < kMinNj || t.ns > kMaxNj || t.nh != 0 || t.n_routes != 0) return BS_E_FORMAT;
+        } else if (t.ns < 1 || t.ns > kMaxNs || t.nh < kMinNh || t.nh > kMaxNh || t.ns + t.nh > kMaxPrecision ||
+                   t.n_routes > kMaxRoutes) {
             return BS_E_FORMAT;
+        }
         if (t.nib_mode != 0 && (t.nib_mode & 0xF0u) != 0x10u) return BS_E_FORMAT;
         if (t.n_elems == 0 || t.n_elems > (1ull << 40)) return BS_E_FORMAT;
         const uint64_t C = 1ull << t.log2_chunk;
         if (t.n_chunks != (t.n_elems + C - 1) / C || t.data_bytes != 16 * t.n_chunks) return BS_E_FORMAT;
-        if (t.model_offset % 16 || !inside(t.model_offset, t.model_bytes, len) || t.model_bytes < 264 ||
-            t.model_bytes > 260 + 4 * 512 + 16 * kMaxRoutes)
+        const uint64_t model_min = joint ? 8 : 264, model_max = joint ? 4 + 4 * kJointPairs : 260 + 4 * 512 + 16 * kMaxRoutes;
+        if (t.model_offset % 16 || !inside(t.model_offset, t.model_bytes, len) || t.model_bytes < model_min ||
+            t.model_bytes > model_max)
             return BS_E_FORMAT;
         t.model.resize(t.model_bytes);
         if (!rd.read(t.model_offset, t.model_bytes, t.model.data())) return fail(BS_E_FORMAT);
         const uint8_t* m = t.model.data();
-        const uint32_t n_present = get_u16(m);
+        if (joint) { // FORMAT.md section 4.3b
+            const uint32_t n_pairs = get_u16(m);
+            if (n_pairs < 1 || n_pairs > kJointPairs || get_u16(m + 2) != 0) return BS_E_FORMAT;
+            if (t.model_bytes != 4 + 4ull * n_pairs) return BS_E_FORMAT;
+            uint64_t sumj = 0;
+            int prevj = -1;
+            for (uint32_t i = 0; i < n_pairs; ++i) {
+                const int j = get_u16(m + 4 + 4 * i);
+                const uint32_t q = get_u16(m + 6 + 4 * i);
+                if (j <= prevj || j >= static_cast<int>(kJointPairs) || q == 0) return BS_E_FORMAT;
+                prevj = j;
+                sumj += q;
+            }
+            if (sumj != (1ull << t.ns)) return BS_E_FORMAT;
+        }
+        const uint32_t n_present = joint ? 0 : get_u16(m);
+        if (!joint) {
         if (n_present < 1 || n_present > 512) return BS_E_FORMAT;
         if (t.model_bytes != 260 + 4ull * n_present + 16ull * t.n_routes) return BS_E_FORMAT;
         uint64_t sum = 0;
@@ -186,6 +207,8 @@ bs_status parse(Reader& rd, std::vector<Tensor>& out) {
             for (int h = 0; h < 8; ++h) sum += get_u16(route + 256 + 16 * r + 2 * h);
             if (sum != (1ull << t.nh)) return BS_E_FORMAT;
         }
+        }
+        (void)n_present;
         try {
             tbuf.resize(t.data_bytes);
         } catch (...) {
@@ -202,16 +225,31 @@ bs_status parse(Reader& rd, std::vector<Tensor>& out) {
             if (off % 16 || get_u32(e + 12) != 0 || !inside(off, bytes, len)) return BS_E_FORMAT;
             t.coded_bytes += bytes;
         }
-        t.table_bytes = table_bytes_for(t.ns, t.nh, t.n_routes);
+        t.table_bytes = joint ? joint_table_bytes(t.ns) : table_bytes_for(t.ns, t.nh, t.n_routes);
         out.push_back(std::move(t));
     }
     return BS_OK;
 }
 
 // Expand one tensor's model into the decode tables (layout in bs_internal.h): the s-table,
-// then the compact fraction rows with the UNIFORM row last.
+// then the compact fraction rows with the UNIFORM row last. For JOINT, one entry per slot:
+// .x = F | ((j << 4) << 16), .y = the slot's rank k within its pair.
 void build_tables(const Tensor& t, uint8_t* dst) {
     const uint8_t* m = t.model.data();
+    if (t.kind == BS_KIND_JOINT) {
+        const uint32_t n_pairs = get_u16(m);
+        uint32_t* jt = reinterpret_cast<uint32_t*>(dst);
+        uint32_t cum = 0;
+        for (uint32_t i = 0; i < n_pairs; ++i) {
+            const uint32_t j = get_u16(m + 4 + 4 * i), q = get_u16(m + 6 + 4 * i);
+            for (uint32_t k = 0; k < q; ++k) {
+                jt[2 * (cum + k)] = q | ((j << 4) << 16);
+                jt[2 * (cum + k) + 1] = k;
+            }
+            cum += q;
+        }
+        return;
+    }
     const uint32_t n_present = get_u16(m);
     const uint8_t* route = m + 4 + 4 * n_present;
     const uint32_t Mh = 1u << t.nh;
@@ -246,7 +284,7 @@ void build_tables(const Tensor& t, uint8_t* dst) {
 uint64_t bs::workspace_bytes_for(const std::vector<Tensor>& ts) {
     uint64_t ws = kErrBlockBytes;
     for (const Tensor& t : ts)
-        if (t.kind == BS_KIND_RANS) ws += up256(t.table_bytes);
+        if (is_coded(t.kind)) ws += up256(t.table_bytes);
     return ws;
 }
 
@@ -272,8 +310,10 @@ bs_status bs::build_workspace(std::vector<Tensor>& ts, std::vector<uint8_t>& ima
     }
     uint64_t pos = kErrBlockBytes;
     for (Tensor& t : ts) {
-        if (t.kind != BS_KIND_RANS) continue;
-        if (static_cast<int>(smem_bytes_for(t.ns, t.nh)) > smem_cap) return BS_E_UNSUPPORTED;
+        if (!is_coded(t.kind)) continue;
+        const uint32_t need = t.kind == BS_KIND_JOINT ? joint_smem_bytes(kWarpsJoint, kChainsJoint)
+                                                      : smem_bytes_for(t.ns, t.nh);
+        if (static_cast<int>(need) > smem_cap) return BS_E_UNSUPPORTED;
         t.ws_offset = pos;
         build_tables(t, image.data() + pos);
         pos += up256(t.table_bytes);
@@ -302,10 +342,10 @@ void bs::fill_tensor_info(const Tensor& t, bs_tensor_info* o) {
 }
 
 bs_status DecodeBatch::init() {
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < 4; ++k) {
         bins_[k].p.reset(new (std::nothrow) DecodeParams);
         if (!bins_[k].p) return BS_E_NOMEM;
-        bins_[k].default_precision = k == 0;
+        bins_[k].mode = static_cast<DecodeMode>(k);
         bins_[k].p->n_items = 0;
         bins_[k].p->total_ctas = 0;
         bins_[k].p->err = err_;
@@ -325,9 +365,8 @@ bs_status DecodeBatch::init() {
 bs_status DecodeBatch::flush_bin(Bin& b, void* stream) {
     DecodeParams& p = *b.p;
     if (p.n_items == 0) return BS_OK;
-    const uint32_t max_warps = b.default_precision ? kWarpsDefault : kWarpsGeneric;
-    const uint32_t chains = b.default_precision ? kChainsDefault : kChainsGeneric;
-    p.warps = launch_warps(b.chunks, max_warps, chains, sms_);
+    const uint32_t chains = chains_of(b.mode);
+    p.warps = launch_warps(b.chunks, max_warps_of(b.mode), chains, sms_);
     const uint64_t per_cta = uint64_t(p.warps) * chains;
     uint64_t ctas = 0;
     for (uint32_t k = 0; k < p.n_items; ++k) {
@@ -337,8 +376,10 @@ bs_status DecodeBatch::flush_bin(Bin& b, void* stream) {
         ctas += (n_chunks + per_cta - 1) / per_cta;
     }
     p.total_ctas = static_cast<uint32_t>(ctas); // at most 2^31 / 8 + kMaxDecodeItems (see add)
-    const int e = launch_decode(p, b.default_precision, kHRegion + b.s_region + p.warps * chains * (kRingBytes + kNibRingBytes),
-                                stream);
+    const bool joint = b.mode == DecodeMode::Joint || b.mode == DecodeMode::JointGeneric;
+    const uint32_t smem = joint ? joint_smem_bytes(p.warps, chains)
+                                                      : kHRegion + b.s_region + p.warps * chains * (kRingBytes + kNibRingBytes);
+    const int e = launch_decode(p, b.mode, smem, stream);
     p.n_items = 0;
     p.total_ctas = 0;
     b.s_region = 0;
@@ -356,9 +397,12 @@ bs_status DecodeBatch::flush_copy(void* stream) {
 
 bs_status DecodeBatch::add(const Tensor& t, uint32_t tensor_index, const uint8_t* d_container,
                            const uint8_t* d_ws, void* d_out, void* stream) {
-    if (t.kind == BS_KIND_RANS) {
-        const bool dflt = is_default_precision(t.ns, t.nh);
-        Bin& b = bins_[dflt ? 0 : 1];
+    if (is_coded(t.kind)) {
+        const DecodeMode mode = t.kind == BS_KIND_JOINT
+                                    ? (t.ns == kDefaultNj ? DecodeMode::Joint : DecodeMode::JointGeneric)
+                                : is_default_precision(t.ns, t.nh) ? DecodeMode::Default
+                                                                   : DecodeMode::Generic;
+        Bin& b = bins_[static_cast<int>(mode)];
         // the smallest CTA holds kMinWarps * 2 chunks, so 2^31 chunks keep the grid below 2^31 CTAs
         if (b.p->n_items == kMaxDecodeItems || b.chunks + t.n_chunks > (1ull << 31)) {
             bs_status s = flush_bin(b, stream);

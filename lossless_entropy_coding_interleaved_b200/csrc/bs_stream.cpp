@@ -96,11 +96,11 @@ struct Group {
 uint64_t out_bytes_of(const Tensor& t) { return t.kind == BS_KIND_RAW ? t.n_elems : 2 * t.n_elems; }
 
 // The container bytes that tensor t's decode reads: [begin, end), begin 16-byte aligned.
-// For RANS: the chunk table and each chunk's payload: states, nibble words and words (the
+// For RANS and JOINT: the chunk table and each chunk's payload: states, nibble words and words (the
 // model is expanded into the workspace at create time and is not read again).
 void coded_range(const Tensor& t, const uint8_t* h, uint64_t* begin, uint64_t* end) {
     uint64_t b = t.data_offset, e = t.data_offset + t.data_bytes;
-    if (t.kind == BS_KIND_RANS) {
+    if (is_coded(t.kind)) {
         const uint64_t C = 1ull << t.log2_chunk;
         for (uint64_t c = 0; c < t.n_chunks; ++c) {
             uint64_t off;

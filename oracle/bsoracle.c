@@ -604,6 +604,16 @@ int bso_encode(const bso_item* items, uint32_t n_items, const bso_params* p, uin
         if (it->kind == 2) { kinds[k] = KIND_RAW; continue; }
         if (it->n_elems > (1ull << 40)) { st = BSO_E_ARG; goto fail; }
         if (it->n_elems == 0) { kinds[k] = KIND_STORED; continue; }
+        if (p->joint) { /* FORMAT.md section 6: more distinct pairs than 2^nj slots -> STORED */
+            const uint16_t* w = (const uint16_t*)it->data;
+            uint8_t* seen = (uint8_t*)calloc(JOINT_PAIRS, 1);
+            uint32_t n_pairs = 0;
+            if (!seen) { st = BSO_E_NOMEM; goto fail; }
+            for (uint64_t i = 0; i < it->n_elems; i++)
+                if (!seen[w[i] >> 4]) { seen[w[i] >> 4] = 1; n_pairs++; }
+            free(seen);
+            if (n_pairs > (1u << p->nj)) { kinds[k] = KIND_STORED; continue; }
+        }
         if ((st = encode_rans((const uint16_t*)it->data, it->n_elems, p->log2_chunk, p->ns, p->nh, p->max_routes,
                               p->joint, p->nj, &blobs[k])))
             goto fail;

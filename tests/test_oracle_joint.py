@@ -164,3 +164,12 @@ def test_corrupt_state_is_detected():
     with pytest.raises(oracle.OracleError) as e:
         oracle.decode(np.frombuffer(bytes(c), np.uint8), 0)
     assert e.value.code == oracle.E_CORRUPT
+
+
+def test_too_many_pairs_for_the_precision_is_stored():
+    # 1100 distinct pairs do not fit the 1024 slots of nj = 10, so the tensor is STORED even
+    # when the encoder is told never to fall back; nj = 11 has room and codes it JOINT
+    w = ((np.arange(1100 * 3) % 1100).astype(np.uint16) << 4) | 5
+    for nj, kind in ((10, oracle.KIND_STORED), (11, oracle.KIND_JOINT)):
+        arr = _roundtrip([("w", w, "bf16")], nj=nj, force_rans=True)
+        assert oracle.info(arr, 0)["kind"] == kind, nj
