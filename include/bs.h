@@ -147,8 +147,8 @@ bs_status bs_check(const bs_plan_t* plan, void* stream, int64_t* first_bad);
  * runtime whose allocator owns all of the GPU's memory, or a callback where an allocation
  * would synchronise the device or is not allowed.
  *
- * Instead of a caller workspace, the decode tables (at most 34 KiB) and the error block live
- * in a static device array of 34 KiB + 256 bytes. Every GPU that loads libbs holds that array
+ * Instead of a caller workspace, the decode tables (at most 64 KiB) and the error block live
+ * in a static device array of 64 KiB + 256 bytes. Every GPU that loads libbs holds that array
  * until the process exits.
  *
  *   h_container      host copy of the whole container; tensor idx is validated in place
@@ -162,8 +162,9 @@ bs_status bs_check(const bs_plan_t* plan, void* stream, int64_t* first_bad);
  *  - Every call shares the array and rewrites it (the tables, and the error block is cleared).
  *    Calls that overlap on the GPU race, so issue them on one stream or one after another.
  *  - The call synchronises stream and returns BS_E_CORRUPT if a chunk fails its end check.
- *  - Tables larger than 34 KiB give BS_E_SIZE. No valid container has such a tensor: 34 KiB
- *    is the s-table at ns = 12 plus 16 fraction rows at nh = 5.
+ *  - Tables larger than 64 KiB give BS_E_SIZE. No valid container has such a tensor: 64 KiB
+ *    is the JOINT table at nj = 13; the largest RANS tables (the s-table at ns = 12 plus 16
+ *    fraction rows at nh = 5) take 34 KiB.
  *  - It calls no cudaMalloc, cudaFree or other allocating routine.
  */
 bs_status bs_decode_tensor_noalloc(const void* h_container, size_t container_bytes, const void* d_container,
