@@ -64,6 +64,11 @@ def _args():
                          "fw: one bs_fw_decode of every tensor's fixed-width lane layout per step; "
                          "gemv: y = W x for every weight matrix from its layout (bs_fw_gemv), one "
                          "forward-shaped pass per step, against dense cuBLAS products")
+    ap.add_argument("--batch-gb", type=float, default=None,
+                    help="model mode: decode in batches of whole chunks of about this many GB of output, "
+                         "one bs_decode_ranges call per batch (batches split tensors); default: one "
+                         "bs_decode_batch of every tensor")
+    ap.add_argument("--log2-chunk", type=int, default=16, help="weights per chunk, as a power of two (8..24)")
     ap.add_argument("--vram-gb", type=float, default=None,
                     help="stream mode: device budget (arena) in GB; default: the smallest arena that "
                          "double-buffers the largest group")
@@ -302,7 +307,7 @@ def run_ours(a):
     specs, n, desc = _workload_desc(a.workload, a.layers)
     t0 = time.time()
     originals = [(s.name, S.generate(s, dev)) for s in specs]
-    d_c, _ = bs.encode(originals, model=a.model)
+    d_c, _ = bs.encode(originals, model=a.model, log2_chunk=a.log2_chunk)
     torch.cuda.synchronize()
     t_encode = time.time() - t0
     hist_words = None
@@ -330,8 +335,25 @@ def run_ours(a):
     h_per_w = hbits / bf16_n
 
     stream = torch.cuda.current_stream()
+    batches = _chunk_batches(plan, infos, outs, a.batch_gb) if a.batch_gb else None
+    # batches go to two streams in turn, so one batch's last CTAs overlap the next one's first
+    side = [torch.cuda.Stream(device=dev) for _ in range(2)] if batches else []
+
+    def step():
+        if batches is None:
+            plan.decode_batch(idx, outs, stream=stream)
+            return
+        start = torch.cuda.Event()
+        start.record(stream)
+        for s_ in side:
+            s_.wait_event(start)
+        for i, b in enumerate(batches):
+            plan.decode_ranges(b, stream=side[i % 2])
+        for s_ in side:
+            stream.wait_stream(s_)
+
     for _ in range(max(1, a.warmup)):
-        plan.decode_batch(idx, outs, stream=stream)
+        step()
     torch.cuda.synchronize()
     plan.check()
     if originals is not None:
@@ -359,7 +381,7 @@ def run_ours(a):
     g0.record(stream)
     for k in range(a.steps):
         ev[k][0].record(stream)
-        plan.decode_batch(idx, outs, stream=stream)
+        step()
         ev[k][1].record(stream)
     g1.record(stream)
     torch.cuda.synchronize()
@@ -458,6 +480,10 @@ def run_ours(a):
                    "parallelism": f"replicas x{world} (no collective on the data path)",
                    "l2": "no flush: inputs larger than L2 (container and outputs are GBs)",
                    "parity": parity_how, "encode_s": round(t_encode, 2),
+                   "log2_chunk": a.log2_chunk,
+                   "batches": ("one bs_decode_batch of every tensor" if batches is None else
+                               f"{len(batches)} bs_decode_ranges calls of about {a.batch_gb} GB of output each "
+                               "(whole chunks, in container order; batches split tensors), on two streams in turn"),
                    "words": "BF16 bit patterns; rANS state arithmetic in u32",
                    "model": ("joint: one rANS table over (sign+exponent, top 3 fraction bits), nj = 13 "
                              "(FORMAT.md kind JOINT)" if a.model == "joint" else
@@ -553,6 +579,37 @@ def _timed(stream, steps, body, barrier):
     torch.cuda.synchronize()
     barrier()
     return g0.elapsed_time(g1)
+
+
+def _chunk_batches(plan, infos, outs, batch_gb):
+    """The checkpoint's chunks in tensor order, cut into batches of about batch_gb GB of
+    output: each batch is a list of (idx, begin, count, out view) ranges for
+    Plan.decode_ranges. STORED and RAW tensors go whole into the batch that reaches them."""
+    import lossless_entropy_coding_interleaved_b200 as bs
+    cap = int(batch_gb * 1e9)
+    batches, cur, room = [], [], cap
+    for k, i in enumerate(infos):
+        n = i["n_elems"]
+        coded = i["kind"] in (bs.KIND_RANS, bs.KIND_JOINT)
+        unit = 1 << i["log2_chunk"] if coded else max(n, 1)
+        per = 1 if i["kind"] == bs.KIND_RAW else 2
+        b = 0
+        while b < n:
+            take = max(unit, room // (per * unit) * unit)     # whole chunks that fit, at least one
+            cnt = min(take, n - b)
+            if cur and cur[-1][0] == k:                     # continues this tensor's last range
+                b0, c0 = cur[-1][1], cur[-1][2] + cnt
+                cur[-1] = (k, b0, c0, outs[k].view(-1)[b0:b0 + c0])
+            else:
+                cur.append((k, b, cnt, outs[k].view(-1)[b:b + cnt]))
+            b += cnt
+            room -= per * cnt
+            if room <= 0:
+                batches.append(cur)
+                cur, room = [], cap
+    if cur:
+        batches.append(cur)
+    return batches
 
 
 def run_layerwise(a):

@@ -119,6 +119,33 @@ bs_status bs_decode_batch(const bs_plan_t* plan, const int32_t* idx, void* const
                           int32_t n, void* stream);
 
 /*
+ * bs_decode_ranges: decode parts of tensors, in whole chunks, in one pass (the launches of
+ * bs_decode_batch). It serves callers that decode a checkpoint in batches of a fixed size,
+ * say 1 GB of output at a time, where one batch may end inside a tensor and the next one
+ * continue it.
+ *  - Range k decodes elements [begin, begin + count) of tensor idx (bytes for RAW) into
+ *    d_out, which receives exactly those words: out_bytes = 2 * count (RAW: count).
+ *  - RANS and JOINT tensors: begin must be a multiple of the tensor's chunk size
+ *    (2^log2_chunk) and the range must end on a chunk boundary or at the tensor's end,
+ *    else BS_E_ARG. d_out must then be 16-byte aligned. STORED and RAW ranges may start
+ *    and end anywhere.
+ *  - A range past the tensor's end, a negative or unknown idx or a nonzero reserved field
+ *    gives BS_E_ARG; a wrong out_bytes gives BS_E_SIZE. Nothing is launched then.
+ *  - Outputs must not overlap. ranges is a host array, read during the call.
+ *  - A corrupt chunk is reported by bs_check with the tensor's own chunk index.
+ */
+typedef struct {
+    int32_t idx;        /* tensor */
+    uint32_t reserved;  /* 0 */
+    uint64_t begin;     /* first element (RAW: byte) */
+    uint64_t count;     /* elements (RAW: bytes) */
+    void* d_out;        /* device, caller-owned */
+    size_t out_bytes;
+} bs_range;
+
+bs_status bs_decode_ranges(const bs_plan_t* plan, const bs_range* ranges, int32_t n, void* stream);
+
+/*
  * bs_verify_tensor: compute the FORMAT.md section 7 checksum of a decoded tensor on the
  * device and compare it with the stored one. The check is the analogue of the per-tensor
  * md5 that the "Gemma 2 9B Instruct -- Lossless Compressed" card ("What lossless

@@ -35,6 +35,11 @@ class BsError(RuntimeError):
         self.first_bad = first_bad
 
 
+class _Range(ctypes.Structure):
+    _fields_ = [("idx", ctypes.c_int32), ("reserved", ctypes.c_uint32), ("begin", ctypes.c_uint64),
+                ("count", ctypes.c_uint64), ("d_out", ctypes.c_void_p), ("out_bytes", ctypes.c_size_t)]
+
+
 class _Info(ctypes.Structure):
     _fields_ = [("n_elems", ctypes.c_uint64), ("out_bytes", ctypes.c_uint64), ("coded_bytes", ctypes.c_uint64),
                 ("n_chunks", ctypes.c_uint64), ("checksum", ctypes.c_uint64), ("shape", ctypes.c_uint64 * 8),
@@ -90,6 +95,7 @@ def _load():
     L.bs_tensor_info_get.argtypes = [P, i32, ctypes.POINTER(_Info)]
     L.bs_decode_tensor.argtypes = [P, i32, P, sz, P]
     L.bs_decode_batch.argtypes = [P, P, P, P, i32, P]
+    L.bs_decode_ranges.argtypes = [P, ctypes.POINTER(_Range), i32, P]
     L.bs_verify_tensor.argtypes = [P, i32, P, sz, P, P, ctypes.POINTER(u64)]
     L.bs_check.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
     L.bs_status_str.argtypes = [ctypes.c_int]
@@ -134,7 +140,7 @@ def _load():
                "bs_streamer_release", "bs_streamer_get_stats", "bs_streamer_check"):
         getattr(L, fn).restype = ctypes.c_int
     for fn in ("bs_plan", "bs_tensor_count", "bs_tensor_info_get", "bs_decode_tensor", "bs_decode_batch",
-               "bs_verify_tensor", "bs_check", "bs_last_cuda_error", "bs_encoder_create", "bs_encoder_scratch_bytes",
+               "bs_decode_ranges", "bs_verify_tensor", "bs_check", "bs_last_cuda_error", "bs_encoder_create", "bs_encoder_scratch_bytes",
                "bs_encoder_run", "bs_encoder_emit"):
         getattr(L, fn).restype = ctypes.c_int
     return L
@@ -144,7 +150,8 @@ lib = _load()
 
 #: every symbol include/bs.h declares
 EXPORTS = ("bs_plan_workspace_bytes", "bs_plan_workspace_bytes_device", "bs_plan", "bs_plan_destroy",
-           "bs_tensor_count", "bs_tensor_info_get", "bs_decode_tensor", "bs_decode_batch", "bs_verify_tensor",
+           "bs_tensor_count", "bs_tensor_info_get", "bs_decode_tensor", "bs_decode_batch", "bs_decode_ranges",
+           "bs_verify_tensor",
            "bs_check", "bs_encoder_create", "bs_encoder_scratch_bytes", "bs_encoder_run", "bs_encoder_emit",
            "bs_encoder_destroy", "bs_status_str", "bs_last_cuda_error", "bs_launch_counter",
            "bs_decode_tensor_noalloc", "bs_streamer_workspace_bytes", "bs_streamer_min_arena_bytes",
@@ -356,6 +363,20 @@ class Plan:
         ba = (ctypes.c_size_t * max(n, 1))(*[o.numel() * o.element_size() for o in outs])
         _check(lib.bs_decode_batch(self._p, ia, pa, ba, n, _stream(stream)), "decode_batch")
         return outs
+
+    def decode_ranges(self, ranges, stream=None):
+        """bs_decode_ranges: ranges is a sequence of (idx, begin, count, out). Elements
+        [begin, begin + count) of tensor idx (bytes for RAW) are decoded into out; for coded
+        kinds the range covers whole chunks (it may end at the tensor's end)."""
+        ranges = list(ranges)
+        n = len(ranges)
+        ra = (_Range * max(n, 1))()
+        for k, (idx, begin, count, out) in enumerate(ranges):
+            ra[k].idx, ra[k].reserved, ra[k].begin, ra[k].count = idx, 0, begin, count
+            ra[k].d_out = out.data_ptr() if out.numel() else None
+            ra[k].out_bytes = out.numel() * out.element_size()
+        _check(lib.bs_decode_ranges(self._p, ra, n, _stream(stream)), "decode_ranges")
+        return [r[3] for r in ranges]
 
     def to_fw(self, idx: int, scratch: torch.Tensor | None = None, stream=None):
         """The fixed-width lane layout (FORMAT.md section 10) of BF16 tensor idx, built on the

@@ -36,9 +36,11 @@ class DecodeBatch {
     explicit DecodeBatch(unsigned long long* d_err) : err_(d_err) {}
     bs_status init(); // allocates the parameter blocks (about 220 KB of host memory)
     // Queue tensor t, whose chunk offsets are relative to d_container, for decoding into d_out.
-    // Launches on `stream` when a bin fills up.
+    // Launches on `stream` when a bin fills up. [begin, begin + count) selects a range of the
+    // tensor's elements (bytes for RAW); for coded kinds begin is a multiple of the chunk size
+    // and the range ends on a chunk boundary or at the tensor's end (checked by the caller).
     bs_status add(const Tensor& t, uint32_t tensor_index, const uint8_t* d_container, const uint8_t* d_ws,
-                  void* d_out, void* stream);
+                  void* d_out, void* stream, uint64_t begin = 0, uint64_t count = ~0ull);
     bs_status flush(void* stream);
 
   private:

@@ -129,7 +129,7 @@ struct DecodeItem {
     uint32_t table_bytes;
     uint8_t log2_chunk, ns, nh, n_routes;
     uint8_t nib_mode, pad0[3];
-    uint32_t pad1;
+    uint32_t chunk_base;        // a range of a tensor: its first chunk (error reports add it)
 };
 static_assert(sizeof(DecodeItem) == 64, "DecodeItem layout");
 

@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
     for (int k = 0; k < kChains; ++k) {
         if (c[k].live && __any_sync(0xFFFFFFFFu, c[k].bad) && lane == 0) {
             atomicOr(p.err, 1ull);
-            atomicMin(p.err + 1, (static_cast<unsigned long long>(it.tensor_index) << 40) | (chunk0 + k));
+            atomicMin(p.err + 1, (static_cast<unsigned long long>(it.tensor_index) << 40) | (it.chunk_base + chunk0 + k));
         }
     }
 }

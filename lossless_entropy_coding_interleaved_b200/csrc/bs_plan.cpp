@@ -396,43 +396,52 @@ bs_status DecodeBatch::flush_copy(void* stream) {
 }
 
 bs_status DecodeBatch::add(const Tensor& t, uint32_t tensor_index, const uint8_t* d_container,
-                           const uint8_t* d_ws, void* d_out, void* stream) {
+                           const uint8_t* d_ws, void* d_out, void* stream, uint64_t begin, uint64_t count) {
+    const uint64_t n_units = t.n_elems; // elements, or bytes for RAW
+    if (begin > n_units) begin = n_units;
+    if (count > n_units - begin) count = n_units - begin;
     if (is_coded(t.kind)) {
+        // a range is decoded as a tensor of its own: its chunk entries, its length, its output
+        const uint64_t c0 = begin >> t.log2_chunk;
+        const uint64_t range_chunks = (count + (1ull << t.log2_chunk) - 1) >> t.log2_chunk;
         const DecodeMode mode = t.kind == BS_KIND_JOINT
                                     ? (t.ns == kDefaultNj ? DecodeMode::Joint : DecodeMode::JointGeneric)
                                 : is_default_precision(t.ns, t.nh) ? DecodeMode::Default
                                                                    : DecodeMode::Generic;
         Bin& b = bins_[static_cast<int>(mode)];
         // the smallest CTA holds kMinWarps * 2 chunks, so 2^31 chunks keep the grid below 2^31 CTAs
-        if (b.p->n_items == kMaxDecodeItems || b.chunks + t.n_chunks > (1ull << 31)) {
+        if (range_chunks == 0) return BS_OK;
+        if (b.p->n_items == kMaxDecodeItems || b.chunks + range_chunks > (1ull << 31)) {
             bs_status s = flush_bin(b, stream);
             if (s) return s;
         }
         DecodeItem& it = b.p->item[b.p->n_items++];
         std::memset(&it, 0, sizeof(it));
-        it.chunk_table = d_container + t.data_offset;
+        it.chunk_table = d_container + t.data_offset + 16 * c0;
         it.container = d_container;
         it.tables = reinterpret_cast<const uint4*>(d_ws + t.ws_offset);
         it.out = static_cast<uint16_t*>(d_out);
-        it.n_elems = t.n_elems;
+        it.n_elems = count;
         it.tensor_index = tensor_index;
+        it.chunk_base = static_cast<uint32_t>(c0); // c0 < n_chunks <= 2^32
         it.table_bytes = t.table_bytes;
         it.log2_chunk = static_cast<uint8_t>(t.log2_chunk);
         it.ns = static_cast<uint8_t>(t.ns);
         it.nh = static_cast<uint8_t>(t.nh);
         it.n_routes = static_cast<uint8_t>(t.n_routes);
         it.nib_mode = static_cast<uint8_t>(t.nib_mode);
-        b.chunks += t.n_chunks;
+        b.chunks += range_chunks;
         b.s_region = std::max<uint32_t>(b.s_region, s_region_bytes(t.ns));
-    } else if (t.n_elems) {
-        const uint64_t bytes = t.kind == BS_KIND_RAW ? t.n_elems : 2 * t.n_elems;
+    } else if (count) {
+        const uint64_t unit = t.kind == BS_KIND_RAW ? 1 : 2;
+        const uint64_t bytes = unit * count;
         const uint64_t blks = (bytes + kCopyBlockBytes - 1) / kCopyBlockBytes;
         if (cp_->n_items == kMaxCopyItems || cp_->total_blocks + blks > 0x7FFFFFFFull) {
             bs_status s = flush_copy(stream);
             if (s) return s;
         }
         CopyItem& it = cp_->item[cp_->n_items++];
-        it.src = d_container + t.data_offset;
+        it.src = d_container + t.data_offset + unit * begin;
         it.dst = static_cast<uint8_t*>(d_out);
         it.bytes = bytes;
         it.blk_begin = cp_->total_blocks;
@@ -539,7 +548,7 @@ bs_status bs_decode_batch(const bs_plan_t* plan, const int32_t* idx, void* const
         const uint64_t want = t.kind == BS_KIND_RAW ? t.n_elems : 2 * t.n_elems;
         if (out_bytes[k] != want) return BS_E_SIZE;
         if (want && !d_out[k]) return BS_E_ARG;
-        if (t.kind == BS_KIND_RANS && !aligned(d_out[k], 16)) return BS_E_ARG;
+        if (is_coded(t.kind) && !aligned(d_out[k], 16)) return BS_E_ARG;
     }
     DecodeBatch batch(reinterpret_cast<unsigned long long*>(plan->d_ws));
     bs_status st = batch.init();
@@ -547,6 +556,35 @@ bs_status bs_decode_batch(const bs_plan_t* plan, const int32_t* idx, void* const
     for (int32_t k = 0; k < n; ++k) {
         st = batch.add(plan->tensors[idx[k]], static_cast<uint32_t>(idx[k]), plan->d_container, plan->d_ws,
                        d_out[k], stream);
+        if (st) return st;
+    }
+    return batch.flush(stream);
+}
+
+bs_status bs_decode_ranges(const bs_plan_t* plan, const bs_range* ranges, int32_t n, void* stream) {
+    if (!plan || n < 0 || (n > 0 && !ranges)) return BS_E_ARG;
+    const int32_t nt = static_cast<int32_t>(plan->tensors.size());
+    for (int32_t k = 0; k < n; ++k) {
+        const bs_range& r = ranges[k];
+        if (r.idx < 0 || r.idx >= nt || r.reserved) return BS_E_ARG;
+        const Tensor& t = plan->tensors[r.idx];
+        if (r.begin > t.n_elems || r.count > t.n_elems - r.begin) return BS_E_ARG;
+        if (is_coded(t.kind)) { // whole chunks: the start and the end on chunk boundaries (or the tensor's end)
+            const uint64_t mask = (1ull << t.log2_chunk) - 1;
+            if ((r.begin & mask) || (r.begin + r.count != t.n_elems && (r.count & mask))) return BS_E_ARG;
+            if (r.count && !aligned(r.d_out, 16)) return BS_E_ARG;
+        }
+        const uint64_t want = t.kind == BS_KIND_RAW ? r.count : 2 * r.count;
+        if (r.out_bytes != want) return BS_E_SIZE;
+        if (want && !r.d_out) return BS_E_ARG;
+    }
+    DecodeBatch batch(reinterpret_cast<unsigned long long*>(plan->d_ws));
+    bs_status st = batch.init();
+    if (st) return st;
+    for (int32_t k = 0; k < n; ++k) {
+        const bs_range& r = ranges[k];
+        st = batch.add(plan->tensors[r.idx], static_cast<uint32_t>(r.idx), plan->d_container, plan->d_ws, r.d_out,
+                       stream, r.begin, r.count);
         if (st) return st;
     }
     return batch.flush(stream);
