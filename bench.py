@@ -68,6 +68,8 @@ def _args():
                     help="model mode: decode in batches of whole chunks of about this many GB of output, "
                          "one bs_decode_ranges call per batch (batches split tensors); default: one "
                          "bs_decode_batch of every tensor")
+    ap.add_argument("--batch-streams", type=int, default=1,
+                    help="model mode with --batch-gb: streams the batches go to in turn (1: one stream)")
     ap.add_argument("--log2-chunk", type=int, default=16, help="weights per chunk, as a power of two (8..24)")
     ap.add_argument("--vram-gb", type=float, default=None,
                     help="stream mode: device budget (arena) in GB; default: the smallest arena that "
@@ -336,8 +338,8 @@ def run_ours(a):
 
     stream = torch.cuda.current_stream()
     batches = _chunk_batches(plan, infos, outs, a.batch_gb) if a.batch_gb else None
-    # batches go to two streams in turn, so one batch's last CTAs overlap the next one's first
-    side = [torch.cuda.Stream(device=dev) for _ in range(2)] if batches else []
+    # with several streams, one batch's last CTAs may overlap the next one's first
+    side = [torch.cuda.Stream(device=dev) for _ in range(max(1, a.batch_streams))] if batches else []
 
     def step():
         if batches is None:
@@ -348,7 +350,7 @@ def run_ours(a):
         for s_ in side:
             s_.wait_event(start)
         for i, b in enumerate(batches):
-            plan.decode_ranges(b, stream=side[i % 2])
+            plan.decode_ranges(b, stream=side[i % len(side)])
         for s_ in side:
             stream.wait_stream(s_)
 
@@ -482,8 +484,9 @@ def run_ours(a):
                    "parity": parity_how, "encode_s": round(t_encode, 2),
                    "log2_chunk": a.log2_chunk,
                    "batches": ("one bs_decode_batch of every tensor" if batches is None else
-                               f"{len(batches)} bs_decode_ranges calls of about {a.batch_gb} GB of output each "
-                               "(whole chunks, in container order; batches split tensors), on two streams in turn"),
+                               f"{len(batches)} bs_decode_ranges calls of at most {a.batch_gb} GB of output and one "
+                               "kernel wave each (whole chunks, in container order; batches split tensors), on "
+                               f"{max(1, a.batch_streams)} stream(s) in turn"),
                    "words": "BF16 bit patterns; rANS state arithmetic in u32",
                    "model": ("joint: one rANS table over (sign+exponent, top 3 fraction bits), nj = 13 "
                              "(FORMAT.md kind JOINT)" if a.model == "joint" else
@@ -582,33 +585,56 @@ def _timed(stream, steps, body, barrier):
 
 
 def _chunk_batches(plan, infos, outs, batch_gb):
-    """The checkpoint's chunks in tensor order, cut into batches of about batch_gb GB of
-    output: each batch is a list of (idx, begin, count, out view) ranges for
-    Plan.decode_ranges. STORED and RAW tensors go whole into the batch that reaches them."""
+    """The checkpoint's chunks in tensor order, cut into batches of at most batch_gb GB of
+    output that each fill at most one wave of the decode kernel (bs_decode_geometry): each
+    batch is a list of (idx, begin, count, out view) ranges for Plan.decode_ranges. A
+    tensor's ranges are whole CTAs' worth of chunks except its last, so no range leaves a
+    part-filled CTA in the middle of a tensor. STORED and RAW tensors go whole into the
+    batch that reaches them."""
     import lossless_entropy_coding_interleaved_b200 as bs
     cap = int(batch_gb * 1e9)
-    batches, cur, room = [], [], cap
+    batches, cur = [], []
+    room, ctas_free = cap, None
+
+    def close():
+        nonlocal cur, room, ctas_free
+        if cur:
+            batches.append(cur)
+        cur, room, ctas_free = [], cap, None
+
     for k, i in enumerate(infos):
         n = i["n_elems"]
-        coded = i["kind"] in (bs.KIND_RANS, bs.KIND_JOINT)
-        unit = 1 << i["log2_chunk"] if coded else max(n, 1)
-        per = 1 if i["kind"] == bs.KIND_RAW else 2
-        b = 0
-        while b < n:
-            take = max(unit, room // (per * unit) * unit)     # whole chunks that fit, at least one
-            cnt = min(take, n - b)
-            if cur and cur[-1][0] == k:                     # continues this tensor's last range
-                b0, c0 = cur[-1][1], cur[-1][2] + cnt
-                cur[-1] = (k, b0, c0, outs[k].view(-1)[b0:b0 + c0])
-            else:
-                cur.append((k, b, cnt, outs[k].view(-1)[b:b + cnt]))
-            b += cnt
-            room -= per * cnt
-            if room <= 0:
-                batches.append(cur)
-                cur, room = [], cap
-    if cur:
-        batches.append(cur)
+        if i["kind"] not in (bs.KIND_RANS, bs.KIND_JOINT):
+            per = 1 if i["kind"] == bs.KIND_RAW else 2
+            if n and room < per * n:
+                close()
+            cur.append((k, 0, n, outs[k].view(-1)))
+            room -= per * n
+            continue
+        cpc, wave = plan.decode_geometry(k)
+        C = 1 << i["log2_chunk"]
+        n_chunks = -(-n // C)
+        c = 0
+        while c < n_chunks:
+            if ctas_free is None:
+                ctas_free = wave
+            fit = min(n_chunks - c, ctas_free * cpc, room // (2 * C))
+            if fit < n_chunks - c:
+                fit -= fit % cpc                          # whole CTAs unless it ends the tensor
+            if fit <= 0:
+                if not cur:                               # an empty batch takes one CTA's worth
+                    fit = min(cpc, n_chunks - c)
+                else:
+                    close()
+                    continue
+            b, cnt = c * C, min(fit * C, n - c * C)
+            cur.append((k, b, cnt, outs[k].view(-1)[b:b + cnt]))
+            c += fit
+            room -= 2 * cnt
+            ctas_free -= -(-fit // cpc)
+            if ctas_free <= 0 or room < 2 * C:
+                close()
+    close()
     return batches
 
 

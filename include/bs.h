@@ -146,6 +146,21 @@ typedef struct {
 bs_status bs_decode_ranges(const bs_plan_t* plan, const bs_range* ranges, int32_t n, void* stream);
 
 /*
+ * bs_decode_geometry: how the decode kernel splits tensor idx on the current device, for
+ * callers that cut their decode into batches (bs_decode_ranges).
+ *  - *chunks_per_cta receives the chunks one CTA takes at the kernel's largest shape. All of
+ *    a CTA's chunks come from one tensor, so a range whose chunk count is not a multiple of
+ *    it leaves its last CTA part-filled. STORED and RAW tensors give 0.
+ *  - *ctas_per_wave receives the CTAs that run at once on the device: one per SM.
+ * A launch of more CTAs than one wave runs in several waves, and a last wave with few CTAs
+ * costs as much time as a full one. A batch whose ranges take at most ctas_per_wave CTAs
+ * (each range taking ceil(chunks / chunks_per_cta)) runs as a single wave.
+ * Returns BS_E_ARG for a bad idx or a NULL output pointer, BS_E_CUDA if the device cannot
+ * be queried.
+ */
+bs_status bs_decode_geometry(const bs_plan_t* plan, int32_t idx, uint32_t* chunks_per_cta, uint32_t* ctas_per_wave);
+
+/*
  * bs_verify_tensor: compute the FORMAT.md section 7 checksum of a decoded tensor on the
  * device and compare it with the stored one. The check is the analogue of the per-tensor
  * md5 that the "Gemma 2 9B Instruct -- Lossless Compressed" card ("What lossless

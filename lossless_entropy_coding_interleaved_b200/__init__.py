@@ -96,6 +96,7 @@ def _load():
     L.bs_decode_tensor.argtypes = [P, i32, P, sz, P]
     L.bs_decode_batch.argtypes = [P, P, P, P, i32, P]
     L.bs_decode_ranges.argtypes = [P, ctypes.POINTER(_Range), i32, P]
+    L.bs_decode_geometry.argtypes = [P, i32, ctypes.POINTER(ctypes.c_uint32), ctypes.POINTER(ctypes.c_uint32)]
     L.bs_verify_tensor.argtypes = [P, i32, P, sz, P, P, ctypes.POINTER(u64)]
     L.bs_check.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
     L.bs_status_str.argtypes = [ctypes.c_int]
@@ -140,7 +141,7 @@ def _load():
                "bs_streamer_release", "bs_streamer_get_stats", "bs_streamer_check"):
         getattr(L, fn).restype = ctypes.c_int
     for fn in ("bs_plan", "bs_tensor_count", "bs_tensor_info_get", "bs_decode_tensor", "bs_decode_batch",
-               "bs_decode_ranges", "bs_verify_tensor", "bs_check", "bs_last_cuda_error", "bs_encoder_create", "bs_encoder_scratch_bytes",
+               "bs_decode_ranges", "bs_decode_geometry", "bs_verify_tensor", "bs_check", "bs_last_cuda_error", "bs_encoder_create", "bs_encoder_scratch_bytes",
                "bs_encoder_run", "bs_encoder_emit"):
         getattr(L, fn).restype = ctypes.c_int
     return L
@@ -151,6 +152,7 @@ lib = _load()
 #: every symbol include/bs.h declares
 EXPORTS = ("bs_plan_workspace_bytes", "bs_plan_workspace_bytes_device", "bs_plan", "bs_plan_destroy",
            "bs_tensor_count", "bs_tensor_info_get", "bs_decode_tensor", "bs_decode_batch", "bs_decode_ranges",
+           "bs_decode_geometry",
            "bs_verify_tensor",
            "bs_check", "bs_encoder_create", "bs_encoder_scratch_bytes", "bs_encoder_run", "bs_encoder_emit",
            "bs_encoder_destroy", "bs_status_str", "bs_last_cuda_error", "bs_launch_counter",
@@ -377,6 +379,12 @@ class Plan:
             ra[k].out_bytes = out.numel() * out.element_size()
         _check(lib.bs_decode_ranges(self._p, ra, n, _stream(stream)), "decode_ranges")
         return [r[3] for r in ranges]
+
+    def decode_geometry(self, idx: int):
+        """bs_decode_geometry: (chunks one CTA of tensor idx's decode takes, CTAs per wave)."""
+        cpc, wave = ctypes.c_uint32(), ctypes.c_uint32()
+        _check(lib.bs_decode_geometry(self._p, idx, ctypes.byref(cpc), ctypes.byref(wave)), "decode_geometry")
+        return cpc.value, wave.value
 
     def to_fw(self, idx: int, scratch: torch.Tensor | None = None, stream=None):
         """The fixed-width lane layout (FORMAT.md section 10) of BF16 tensor idx, built on the

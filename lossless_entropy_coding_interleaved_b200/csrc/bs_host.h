@@ -30,6 +30,12 @@ bs_status build_workspace(std::vector<Tensor>& ts, std::vector<uint8_t>& image);
 // verbatim copies into one
 // copy list. It launches a bin when the bin is full,
 // and launches every bin on flush().
+// The decode kernel instance (and CTA shape) of a coded tensor.
+inline DecodeMode decode_mode_of(const Tensor& t) {
+    if (t.kind == BS_KIND_JOINT) return t.ns == kDefaultNj ? DecodeMode::Joint : DecodeMode::JointGeneric;
+    return is_default_precision(t.ns, t.nh) ? DecodeMode::Default : DecodeMode::Generic;
+}
+
 class DecodeBatch {
   public:
     // d_err: the workspace's error block.

@@ -42,8 +42,9 @@ inline uint64_t payload_bytes(uint64_t n_c, uint32_t n_words, bool nib_stored) {
 // in quarters of kQuarterBytes (one 16-byte cp.async per lane fills a quarter), and its
 // nibble words through a ring of kNibRingBlocks blocks (128 bytes each).
 constexpr int kWarpsDefault = 24, kChainsDefault = 2, kWarpsGeneric = 20, kChainsGeneric = 2;
-// JOINT at the default precision (nj = 13): the table takes the first 64 KiB, then the rings.
-constexpr int kWarpsJoint = 24, kChainsJoint = 2;
+// JOINT at the default precision (nj = 13): the table takes the first 64 KiB, then 56 rings of
+// each kind (204 KiB in all). 28 warps hold 72 registers a thread, the most that fits.
+constexpr int kWarpsJoint = 28, kChainsJoint = 2;
 inline bool is_default_precision(uint32_t ns, uint32_t nh) { return ns == 11 && nh == 5; }
 inline int warps_for(uint32_t ns, uint32_t nh) { return is_default_precision(ns, nh) ? kWarpsDefault : kWarpsGeneric; }
 inline int chains_for(uint32_t ns, uint32_t nh) { return is_default_precision(ns, nh) ? kChainsDefault : kChainsGeneric; }
@@ -60,7 +61,7 @@ inline uint32_t launch_warps(uint64_t chunks, uint32_t max_warps, uint32_t chain
 constexpr uint32_t kRingBytes = 2048;
 constexpr uint32_t kQuarterBytes = kRingBytes / 4;
 static_assert(kQuarterBytes == 32 * 16, "one cp.async of 16 bytes per lane fills a quarter");
-constexpr uint32_t kNibRingBlocks = 8;
+constexpr uint32_t kNibRingBlocks = 4;
 constexpr uint32_t kNibRingBytes = kNibRingBlocks * 128;
 // Shared memory of a CTA:
 //   [0, kHRegion)                 fraction rows, one copy per lane (row r, slot j, lane c at

@@ -63,16 +63,15 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
 // One chunk in flight on a warp: lane j holds state j.
-// Only what the step loop needs stays in registers; the rest (the rings' shared-memory
-// addresses, the quarter count, the stream and nibble pointers, the chunk index) is derived
-// where it is used.
+// Only what the step loop needs stays in registers; the rest (the rings' offsets, the block
+// and quarter counts, the stream and nibble pointers, the chunk index) is derived where it is
+// used. Chain k's word ring sits at ring_off + k * kRingBytes and its nibble ring at
+// nring_off + k * kNibRingBytes, from the warp's two offsets.
 struct Chain {
     uint32_t x;               // rANS state, in [2^16, 2^32) between weights
     uint32_t posb;            // bytes of the word stream consumed (warp-uniform)
     uint32_t fq;              // ring quarters requested (warp-uniform)
-    uint32_t stream_bytes, nc, n_blocks;
-    uint32_t ring_off;        // the word ring, as an offset into the dynamic smem array
-    uint32_t nring_off;       // the nibble ring, as an offset into the dynamic smem array
+    uint32_t stream_bytes, nc; // blocks of 8 steps: (nc + 255) >> 8
     uint32_t raw;             // nibble word of the current block (constant mode: c in every nibble)
     const uint8_t* payload;   // the chunk's payload: start states, nibble words (if stored), words
     bool live;                // a real chunk (false: a filler chain that is never stored)
@@ -143,8 +142,6 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
         Chain& h = c[k];
         const uint64_t chunk = chunk0 + k;
         h.live = chunk < n_chunks;
-        h.ring_off = ring_off + k * kRingBytes;
-        h.nring_off = nring_off + k * kNibRingBytes;
         h.posb = 0;
         h.fq = 0;
         h.bad = false;
@@ -156,16 +153,15 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
             h.payload = it.container + off;
             const uint64_t base = chunk << log2c;
             h.nc = static_cast<uint32_t>(min(C, n_elems - base));
-            h.n_blocks = (h.nc + 255u) >> 8; // blocks of 8 steps
             h.stream_bytes = 2u * n_words;
             h.x = __ldg(reinterpret_cast<const unsigned int*>(h.payload) + lane);
             h.bad = h.x < kStateL;
         } else { // filler: decodes from L and its own (unfilled) ring; nothing is stored
-            h.stream_bytes = h.nc = h.n_blocks = 0;
+            h.stream_bytes = h.nc = 0;
             h.payload = nullptr;
             h.x = kStateL;
         }
-        nb = max(nb, h.n_blocks);
+        nb = max(nb, (h.nc + 255u) >> 8);
     }
 
     const uint32_t smask8 = ((1u << ns) - 1u) << 3, hmask7 = ((1u << nh) - 1u) << 7; // JOINT: smask8 masks the slot
@@ -178,29 +174,33 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
     // newest group when those were requested earlier. Quarters wholly inside the stream
     // skip the per-piece bounds.
     // Nibble words: at block blk (even) the ring must hold blocks blk and blk+1, which were
-    // requested two upkeeps earlier; this upkeep requests blocks blk+4 and blk+5 (16 lanes x
-    // 16 bytes). The first upkeep requests blocks 0-5 and waits for all of them.
+    // requested one upkeep earlier (the group before the newest); this upkeep requests blocks
+    // blk+2 and blk+3 (16 lanes x 16 bytes) into the other half of the 4-block ring. Sixteen
+    // steps separate two upkeeps, several microseconds, far longer than a DRAM read. The
+    // first upkeep requests blocks 0-3 and waits for all of them.
     auto upkeep = [&](uint32_t blk) {
         __syncwarp();
         bool newest_needed = blk == 0;
 #pragma unroll
         for (int k = 0; k < kChains; ++k) {
             Chain& h = c[k];
-            if (nib_stored && blk < h.n_blocks) { // nibble words start after the 128-byte states
-                for (uint32_t b = (blk == 0 ? 0u : blk + 4u); b < blk + 6u; b += 2u) {
+            const uint32_t n_blocks = (h.nc + 255u) >> 8;
+            if (nib_stored && blk < n_blocks) { // nibble words start after the 128-byte states
+                for (uint32_t b = (blk == 0 ? 0u : blk + 2u); b < blk + 4u; b += 2u) {
                     const uint32_t byte = 128u * b + 16u * lane; // lanes 0-15: blocks b and b+1
-                    if (lane < 16 && byte < 128u * h.n_blocks)
-                        cp_async16(smem_base + h.nring_off + (byte & (kNibRingBytes - 1u)), h.payload + 128 + byte, 16u);
+                    if (lane < 16 && byte < 128u * n_blocks)
+                        cp_async16(smem_base + nring_off + k * kNibRingBytes + (byte & (kNibRingBytes - 1u)),
+                                   h.payload + 128 + byte, 16u);
                 }
             }
-            if (blk < h.n_blocks) {
+            if (blk < n_blocks) {
                 const uint32_t q = h.posb / kQuarterBytes;
                 const uint32_t total_q = (h.stream_bytes + kQuarterBytes - 1) / kQuarterBytes;
-                const uint8_t* stream = h.payload + 128 + (nib_stored ? 128u * h.n_blocks : 0u);
+                const uint8_t* stream = h.payload + 128 + (nib_stored ? 128u * n_blocks : 0u);
                 if (h.fq <= min(q + 2, total_q - 1)) newest_needed = true;
                 while (h.fq < q + 4 && h.fq < total_q) {
                     const uint32_t byte = h.fq * kQuarterBytes + 16u * lane;
-                    const uint32_t dst = smem_base + h.ring_off + (byte & (kRingBytes - 1u));
+                    const uint32_t dst = smem_base + ring_off + k * kRingBytes + (byte & (kRingBytes - 1u));
                     if ((h.fq + 1) * kQuarterBytes <= h.stream_bytes) cp_async16(dst, stream + byte, 16u);
                     else if (byte < h.stream_bytes) cp_async16(dst, stream + byte, min(16u, h.stream_bytes - byte));
                     ++h.fq;
@@ -220,8 +220,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
 #pragma unroll
         for (int k = 0; k < kChains; ++k) {
             Chain& h = c[k];
-            if (nib_stored && h.live && (full || b < h.n_blocks))
-                h.raw = *reinterpret_cast<const uint32_t*>(smem + h.nring_off + ((128u * b) & (kNibRingBytes - 1u)) + lane4);
+            if (nib_stored && h.live && (full || b < ((h.nc + 255u) >> 8)))
+                h.raw = *reinterpret_cast<const uint32_t*>(smem + nring_off + k * kNibRingBytes +
+                                                           ((128u * b) & (kNibRingBytes - 1u)) + lane4);
         }
     };
 
@@ -269,7 +270,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
 #pragma unroll
             for (int k = 0; k < kChains; ++k)
                 w[k] = *reinterpret_cast<const uint16_t*>(
-                    smem + (((c[k].posb + __popc(m[k] & lt) * mul2) & (kRingBytes - 1u)) | c[k].ring_off));
+                    smem + (((c[k].posb + __popc(m[k] & lt) * mul2) & (kRingBytes - 1u)) | (ring_off + k * kRingBytes)));
 #pragma unroll
             for (int k = 0; k < kChains; ++k) {
                 Chain& h = c[k];
@@ -321,7 +322,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
     }
 #pragma unroll
     for (int k = 0; k < kChains; ++k) // end check: state back at L, every word consumed
-        if (c[k].live && c[k].n_blocks == blk) c[k].bad |= (c[k].x != kStateL) | (c[k].posb != c[k].stream_bytes);
+        if (c[k].live && ((c[k].nc + 255u) >> 8) == blk) c[k].bad |= (c[k].x != kStateL) | (c[k].posb != c[k].stream_bytes);
     // The rest (ragged tails, chains of different lengths), with bounds, two blocks at a time.
     for (; blk < nb; blk += 2) {
         upkeep(blk);
@@ -335,7 +336,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
 #pragma unroll
             for (int k = 0; k < kChains; ++k) {
                 Chain& h = c[k];
-                if (b < h.n_blocks) {
+                const uint32_t n_blocks = (h.nc + 255u) >> 8;
+                if (b < n_blocks) {
                     const uint32_t i0 = (b << 8) + (lane << 3);
                     if (i0 + 8 <= h.nc) {
                         *reinterpret_cast<uint4*>(out0 + k * C + i0) = make_uint4(o[k][0], o[k][1], o[k][2], o[k][3]);
@@ -344,7 +346,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
                         for (int e = 0; e < 8; ++e)
                             if (i0 + e < h.nc) out0[k * C + i0 + e] = static_cast<uint16_t>(o[k][e >> 1] >> (16 * (e & 1)));
                     }
-                    if (b + 1 == h.n_blocks) // end check: state back at L, every word consumed
+                    if (b + 1 == n_blocks) // end check: state back at L, every word consumed
                         h.bad |= (h.x != kStateL) | (h.posb != h.stream_bytes);
                 }
             }
@@ -356,7 +358,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
     for (int k = 0; k < kChains; ++k) {
         if (c[k].live && __any_sync(0xFFFFFFFFu, c[k].bad) && lane == 0) {
             atomicOr(p.err, 1ull);
-            atomicMin(p.err + 1, (static_cast<unsigned long long>(it.tensor_index) << 40) | (it.chunk_base + chunk0 + k));
+            atomicMin(p.err + 1, (static_cast<unsigned long long>(it.tensor_index) << 40) |
+                                     (it.chunk_base + static_cast<uint64_t>(blockIdx.x - it.cta_begin) * (warps * kChains) +
+                                      warp * kChains + k)); // chunk0 + k, recomputed
         }
     }
 }

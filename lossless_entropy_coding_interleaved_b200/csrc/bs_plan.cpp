@@ -365,8 +365,20 @@ bs_status DecodeBatch::init() {
 bs_status DecodeBatch::flush_bin(Bin& b, void* stream) {
     DecodeParams& p = *b.p;
     if (p.n_items == 0) return BS_OK;
-    const uint32_t chains = chains_of(b.mode);
-    p.warps = launch_warps(b.chunks, max_warps_of(b.mode), chains, sms_);
+    const uint32_t chains = chains_of(b.mode), max_warps = max_warps_of(b.mode);
+    p.warps = launch_warps(b.chunks, max_warps, chains, sms_);
+    // Every item rounds up to whole CTAs. If that pushes a launch that would fit one wave into
+    // a second one, widen the CTAs until it fits again (or the shape is the largest).
+    auto ctas_at = [&](uint32_t warps) {
+        uint64_t n = 0;
+        for (uint32_t k = 0; k < p.n_items; ++k) {
+            const DecodeItem& it = p.item[k];
+            const uint64_t C = 1ull << it.log2_chunk, n_chunks = (it.n_elems + C - 1) / C;
+            n += (n_chunks + uint64_t(warps) * chains - 1) / (uint64_t(warps) * chains);
+        }
+        return n;
+    };
+    while (p.warps < max_warps && ctas_at(p.warps) > sms_) ++p.warps;
     const uint64_t per_cta = uint64_t(p.warps) * chains;
     uint64_t ctas = 0;
     for (uint32_t k = 0; k < p.n_items; ++k) {
@@ -404,10 +416,7 @@ bs_status DecodeBatch::add(const Tensor& t, uint32_t tensor_index, const uint8_t
         // a range is decoded as a tensor of its own: its chunk entries, its length, its output
         const uint64_t c0 = begin >> t.log2_chunk;
         const uint64_t range_chunks = (count + (1ull << t.log2_chunk) - 1) >> t.log2_chunk;
-        const DecodeMode mode = t.kind == BS_KIND_JOINT
-                                    ? (t.ns == kDefaultNj ? DecodeMode::Joint : DecodeMode::JointGeneric)
-                                : is_default_precision(t.ns, t.nh) ? DecodeMode::Default
-                                                                   : DecodeMode::Generic;
+        const DecodeMode mode = decode_mode_of(t);
         Bin& b = bins_[static_cast<int>(mode)];
         // the smallest CTA holds kMinWarps * 2 chunks, so 2^31 chunks keep the grid below 2^31 CTAs
         if (range_chunks == 0) return BS_OK;
@@ -588,6 +597,19 @@ bs_status bs_decode_ranges(const bs_plan_t* plan, const bs_range* ranges, int32_
         if (st) return st;
     }
     return batch.flush(stream);
+}
+
+bs_status bs_decode_geometry(const bs_plan_t* plan, int32_t idx, uint32_t* chunks_per_cta, uint32_t* ctas_per_wave) {
+    if (!plan || !chunks_per_cta || !ctas_per_wave || idx < 0 || idx >= static_cast<int32_t>(plan->tensors.size()))
+        return BS_E_ARG;
+    const Tensor& t = plan->tensors[idx];
+    *chunks_per_cta = is_coded(t.kind) ? max_warps_of(decode_mode_of(t)) * chains_of(decode_mode_of(t)) : 0;
+    int dev = 0, sms = 0;
+    cudaError_t ce = cudaGetDevice(&dev);
+    if (ce == cudaSuccess) ce = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (ce != cudaSuccess || sms <= 0) return cuda_fail(ce == cudaSuccess ? cudaErrorInvalidDevice : ce);
+    *ctas_per_wave = static_cast<uint32_t>(sms); // every decode shape takes over half an SM's shared memory
+    return BS_OK;
 }
 
 bs_status bs_decode_tensor(const bs_plan_t* plan, int32_t idx, void* d_out, size_t out_bytes, void* stream) {

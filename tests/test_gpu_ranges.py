@@ -153,3 +153,20 @@ def test_corrupt_chunk_reported_with_its_tensor_index():
     plan.decode_ranges([(0, 0, 32 * C, o)])
     plan.check()
     assert np.array_equal(_host(o), arrs[0][:32 * C])
+
+
+def test_decode_geometry():
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    w = S.words_numpy(S.generate(S.workload("tensor_1m")[0], "cpu")).reshape(-1)
+    items = [("joint", w, "bf16"), ("u", np.arange(1 << 16, dtype=np.uint32).astype(np.uint16), "bf16")]
+    plan = bs.Plan(oracle.encode(items, model="joint"), device="cuda:0")
+    assert plan.info(1)["kind"] == bs.KIND_STORED
+    assert plan.decode_geometry(0) == (56, sms)       # JOINT: 28 warps of 2 chunks, one CTA per SM
+    assert plan.decode_geometry(1) == (0, sms)
+    fplan = bs.Plan(oracle.encode(items[:1]), device="cuda:0")
+    assert fplan.decode_geometry(0) == (48, sms)      # RANS, default precisions: 24 warps of 2
+    gplan = bs.Plan(oracle.encode(items[:1], ns=10, nh=4), device="cuda:0")
+    assert gplan.decode_geometry(0) == (40, sms)      # other precisions: 20 warps of 2
+    with pytest.raises(bs.BsError) as e:
+        plan.decode_geometry(2)
+    assert e.value.code == bs.E_ARG
