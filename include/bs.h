@@ -127,8 +127,8 @@ bs_status bs_decode_batch(const bs_plan_t* plan, const int32_t* idx, void* const
  *    d_out, which receives exactly those words: out_bytes = 2 * count (RAW: count).
  *  - RANS and JOINT tensors: begin must be a multiple of the tensor's chunk size
  *    (2^log2_chunk) and the range must end on a chunk boundary or at the tensor's end,
- *    else BS_E_ARG. d_out must then be 16-byte aligned. STORED and RAW ranges may start
- *    and end anywhere.
+ *    else BS_E_ARG. d_out must then be 16-byte aligned. STORED and RAW ranges, and empty
+ *    ranges of any kind, may start and end anywhere inside the tensor.
  *  - A range past the tensor's end, a negative or unknown idx or a nonzero reserved field
  *    gives BS_E_ARG; a wrong out_bytes gives BS_E_SIZE. Nothing is launched then.
  *  - Outputs must not overlap. ranges is a host array, read during the call.

@@ -578,10 +578,10 @@ bs_status bs_decode_ranges(const bs_plan_t* plan, const bs_range* ranges, int32_
         if (r.idx < 0 || r.idx >= nt || r.reserved) return BS_E_ARG;
         const Tensor& t = plan->tensors[r.idx];
         if (r.begin > t.n_elems || r.count > t.n_elems - r.begin) return BS_E_ARG;
-        if (is_coded(t.kind)) { // whole chunks: the start and the end on chunk boundaries (or the tensor's end)
+        if (is_coded(t.kind) && r.count) { // whole chunks: the start and the end on chunk boundaries (or the tensor's end)
             const uint64_t mask = (1ull << t.log2_chunk) - 1;
             if ((r.begin & mask) || (r.begin + r.count != t.n_elems && (r.count & mask))) return BS_E_ARG;
-            if (r.count && !aligned(r.d_out, 16)) return BS_E_ARG;
+            if (!aligned(r.d_out, 16)) return BS_E_ARG;
         }
         const uint64_t want = t.kind == BS_KIND_RAW ? r.count : 2 * r.count;
         if (r.out_bytes != want) return BS_E_SIZE;

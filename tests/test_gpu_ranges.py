@@ -126,9 +126,10 @@ def test_refused_requests():
     with pytest.raises(bs.BsError) as e:
         plan.decode(0, big[1:n + 1])
     assert e.value.code == bs.E_ARG
-    # empty ranges are fine, RAW ranges may start anywhere
+    # empty ranges are fine anywhere inside the tensor, RAW ranges may start anywhere
     o = _out(plan, 1, 30)
-    plan.decode_ranges([(0, C, 0, _out(plan, 0, 0)), (1, 37, 30, o)])
+    plan.decode_ranges([(0, C, 0, _out(plan, 0, 0)), (0, 77, 0, _out(plan, 0, 0)), (0, n, 0, _out(plan, 0, 0)),
+                        (1, 37, 30, o)])
     plan.check()
     assert np.array_equal(_host(o), np.arange(37, 67, dtype=np.uint8))
 
