@@ -70,6 +70,8 @@ def _args():
                          "bs_decode_batch of every tensor")
     ap.add_argument("--batch-streams", type=int, default=1,
                     help="model mode with --batch-gb: streams the batches go to in turn (1: one stream)")
+    ap.add_argument("--layer-streams", type=int, default=1,
+                    help="layerwise mode: streams consecutive layers go to in turn (1: one stream)")
     ap.add_argument("--log2-chunk", type=int, default=16, help="weights per chunk, as a power of two (8..24)")
     ap.add_argument("--vram-gb", type=float, default=None,
                     help="stream mode: device budget (arena) in GB; default: the smallest arena that "
@@ -656,10 +658,23 @@ def run_layerwise(a):
     coded = sum(i["coded_bytes"] for i in infos)
     out_bytes = sum(i["out_bytes"] for i in infos)
     stream = torch.cuda.current_stream()
+    # with --layer-streams 2, consecutive layers alternate between two streams, as a consumer
+    # that double-buffers layers would decode them: two layers' chunks share the SMs
+    side = [torch.cuda.Stream(device=dev) for _ in range(max(1, a.layer_streams))]
 
     def step():
-        for m in members:
-            plan.decode_batch(m, [outs[k] for k in m], stream=stream)
+        if len(side) == 1:
+            for m in members:
+                plan.decode_batch(m, [outs[k] for k in m], stream=stream)
+            return
+        start = torch.cuda.Event()
+        start.record(stream)
+        for s_ in side:
+            s_.wait_event(start)
+        for i, m in enumerate(members):
+            plan.decode_batch(m, [outs[k] for k in m], stream=side[i % len(side)])
+        for s_ in side:
+            stream.wait_stream(s_)
 
     for _ in range(max(3, a.warmup)):
         step()
@@ -688,6 +703,7 @@ def run_layerwise(a):
         "n_gpus": ranks.world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms / a.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
         "config": {"workload": a.workload, "description": desc, "n_weights": n, "groups": len(members),
+                   "layer_streams": len(side),
                    "decoded_bytes": int(out_bytes), "coded_bytes": int(coded),
                    "entropy_bits_per_weight": round(h_per_w, 5), "encode_s": round(t_encode, 2),
                    "l2": "no flush: inputs larger than L2", "parity": "bit-exact vs originals before timing"},
