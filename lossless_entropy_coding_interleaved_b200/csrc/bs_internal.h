@@ -35,9 +35,10 @@ inline uint64_t payload_bytes(uint64_t n_c, uint32_t n_words, bool nib_stored) {
 }
 
 // Decode-kernel geometry: a warp decodes `chains` chunks at once (independent state chains
-// per lane), and a CTA of `warps` warps covers warps*chains chunks of one tensor. The
-// default precisions use 24 warps of 2 chains; the others 20 warps of 2 (ns = 12 tables
-// leave room for 40 rings).
+// per lane), and a CTA of `warps` warps covers warps*chains chunks of one tensor. Kind RANS
+// at the default precisions uses 24 warps of 2 chains, kind JOINT at nj = 13 28 warps of 2
+// (kWarpsJoint below), and the other precisions 20 warps of 2 (ns = 12 tables leave room
+// for 40 rings).
 // Each chunk's 16-bit word stream goes through its own shared-memory ring of kRingBytes,
 // in quarters of kQuarterBytes (one 16-byte cp.async per lane fills a quarter), and its
 // nibble words through a ring of kNibRingBlocks blocks (128 bytes each).
