@@ -378,12 +378,20 @@ def run_ours(a):
     clocks = _Clocks(smi_index)
     time.sleep(0.3)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+    # a container and outputs that fit in L2 (the small workloads) would be timed from the
+    # cache: write a buffer of twice the L2 size before each step, outside its events, and
+    # time the sum of the steps' events instead of the whole loop
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = (torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev)
+                 if coded + out_bytes < 2 * l2_bytes else None)
     barrier()
     torch.cuda.synchronize()
     l0 = bs.launch_counter()
     g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     g0.record(stream)
     for k in range(a.steps):
+        if flush_buf is not None:
+            flush_buf.fill_(k & 0xFF)
         ev[k][0].record(stream)
         step()
         ev[k][1].record(stream)
@@ -392,8 +400,8 @@ def run_ours(a):
     barrier()
     launches = bs.launch_counter() - l0
     clk = clocks.stop()
-    total_ms = g0.elapsed_time(g1)
     step_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
+    total_ms = g0.elapsed_time(g1) if flush_buf is None else sum(step_ms)
     plan.check()
     total_ms = ranks.max(total_ms)
     value = world * a.steps * out_bytes / (total_ms * 1e-3) / 1e9
@@ -482,7 +490,9 @@ def run_ours(a):
                    "entropy_bits_per_weight": round(h_per_w, 5),
                    "overhead_pct_vs_entropy": round(100 * (bf16_coded * 8 / bf16_n / h_per_w - 1), 4),
                    "parallelism": f"replicas x{world} (no collective on the data path)",
-                   "l2": "no flush: inputs larger than L2 (container and outputs are GBs)",
+                   "l2": ("no flush: inputs larger than L2 (container and outputs are GBs)" if flush_buf is None
+                          else f"flushed: {2 * l2_bytes >> 20} MiB written before each step, outside its "
+                               "events; value from the sum of the step times"),
                    "parity": parity_how, "encode_s": round(t_encode, 2),
                    "log2_chunk": a.log2_chunk,
                    "batches": ("one bs_decode_batch of every tensor" if batches is None else
