@@ -54,3 +54,36 @@ def test_plan_without_gpu_fails_loudly():
         pytest.skip("a GPU is present")
     with pytest.raises(bs.BsError):
         bs.Plan(b"\0" * 64)
+
+
+def _golden(name):
+    hexs = []
+    with open(os.path.join(ROOT, "tests", "golden", name)) as fh:
+        for line in fh:
+            hexs.append(line.split("#", 1)[0])
+    return bytes.fromhex("".join("".join(hexs).split()))
+
+
+def test_library_parses_the_joint_golden_on_host():
+    # FORMAT.md section 8.3, derived by hand: the library's parser takes it, and the workspace
+    # holds the error block and one JOINT table of 2^13 slots of 8 bytes
+    import lossless_entropy_coding_interleaved_b200 as bs
+    c = _golden("joint_two_weights.hex")
+    assert bs.workspace_bytes(c) == 256 + (8 << 13)
+
+
+def test_library_refuses_what_the_oracle_refuses():
+    # the malformed JOINT containers the oracle's pins refuse (tests/test_oracle_joint.py):
+    # the library's own parser must refuse each of them too
+    import struct
+    import lossless_entropy_coding_interleaved_b200 as bs
+    c = _golden("joint_two_weights.hex")
+    d, m = 64, 224
+    edits = [(d + 4, "<B", 7), (d + 4, "<B", 14), (d + 5, "<B", 3), (d + 6, "<B", 1), (d + 0, "<B", 4),
+             (m + 0, "<H", 0), (m + 2, "<H", 1), (m + 8, "<H", 1016), (m + 4, "<H", 4096), (m + 6, "<H", 0),
+             (m + 6, "<H", 4095), (d + 40, "<Q", 16)]
+    for off, fmt, v in edits:
+        b = bytearray(c)
+        struct.pack_into(fmt, b, off, v)
+        with pytest.raises(bs.BsError):
+            bs.workspace_bytes(bytes(b))
