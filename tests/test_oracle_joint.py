@@ -173,3 +173,28 @@ def test_too_many_pairs_for_the_precision_is_stored():
     for nj, kind in ((10, oracle.KIND_STORED), (11, oracle.KIND_JOINT)):
         arr = _roundtrip([("w", w, "bf16")], nj=nj, force_rans=True)
         assert oracle.info(arr, 0)["kind"] == kind, nj
+
+
+try:
+    from hypothesis import given, settings, strategies as st
+except ImportError:  # pragma: no cover
+    given = None
+
+if given is not None:
+    @settings(max_examples=60, deadline=None)
+    @given(st.integers(1, 5000), st.integers(1, 4096), st.integers(0, 2 ** 32 - 1),
+           st.sampled_from(["factored", "joint"]), st.sampled_from([8, 12, 16]))
+    def test_random_tensors_round_trip(n, alphabet, seed, model, log2_chunk):
+        # words drawn from a random alphabet of up to 4096 patterns, some of them skewed:
+        # every container validates and decodes back, and the coded size obeys Gibbs
+        rng = np.random.default_rng(seed)
+        pool = rng.integers(0, 1 << 16, size=alphabet, dtype=np.uint32).astype(np.uint16)
+        p = rng.dirichlet(np.full(alphabet, 0.3))
+        w = pool[rng.choice(alphabet, size=n, p=p)]
+        arr = np.frombuffer(oracle.encode([("w", w, "bf16")], model=model, log2_chunk=log2_chunk,
+                                          force_rans=True), np.uint8)
+        assert oracle.validate(arr) == 1
+        assert np.array_equal(oracle.decode(arr, 0), w)
+        ti = oracle.info(arr, 0)
+        if ti["kind"] in (oracle.KIND_JOINT, oracle.KIND_RANS):
+            assert 8.0 * ti["coded_bytes"] >= conditional_entropy_bits(w)
