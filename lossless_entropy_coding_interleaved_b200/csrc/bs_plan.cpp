@@ -368,7 +368,8 @@ bs_status DecodeBatch::flush_bin(Bin& b, void* stream) {
     const uint32_t chains = chains_of(b.mode), max_warps = max_warps_of(b.mode);
     p.warps = launch_warps(b.chunks, max_warps, chains, sms_);
     // Every item rounds up to whole CTAs. If that pushes a launch that would fit one wave into
-    // a second one, widen the CTAs until it fits again (or the shape is the largest).
+    // a second one, widen the CTAs until it fits again. A launch that needs more than one wave
+    // even at the largest shape (many small tensors: each takes a CTA) keeps its shape.
     auto ctas_at = [&](uint32_t warps) {
         uint64_t n = 0;
         for (uint32_t k = 0; k < p.n_items; ++k) {
@@ -378,7 +379,8 @@ bs_status DecodeBatch::flush_bin(Bin& b, void* stream) {
         }
         return n;
     };
-    while (p.warps < max_warps && ctas_at(p.warps) > sms_) ++p.warps;
+    if (ctas_at(p.warps) > sms_ && ctas_at(max_warps) <= sms_)
+        while (ctas_at(p.warps) > sms_) ++p.warps;
     const uint64_t per_cta = uint64_t(p.warps) * chains;
     uint64_t ctas = 0;
     for (uint32_t k = 0; k < p.n_items; ++k) {
