@@ -98,6 +98,8 @@ def lib():
         L.bso_lane_encode.argtypes = [P, u32, P, P, u32, u32, P, u32, ctypes.POINTER(u32), P, P,
                                       ctypes.POINTER(u32)]
         L.bso_lane_decode.argtypes = [P, u32, P, P, u32, u32, u32, P, u32, P, u32, P, ctypes.POINTER(u32)]
+        L.bso_joint_lane_encode.argtypes = [P, u32, P, u32, ctypes.POINTER(u32), P, P, ctypes.POINTER(u32)]
+        L.bso_joint_lane_decode.argtypes = [P, u32, u32, P, u32, P, u32, P, ctypes.POINTER(u32)]
         L.bso_fw_bytes.argtypes = [u64, u64]
         L.bso_fw_bytes.restype = u64
         L.bso_fw_table.argtypes = [P, u64, P, ctypes.POINTER(u32)]
@@ -109,7 +111,8 @@ def lib():
         L.bso_checksum.argtypes = [P, u64, u32]
         L.bso_checksum.restype = u64
         for fn in ("bso_encode", "bso_validate", "bso_tensor_info_get", "bso_decode", "bso_decode_chunks",
-                   "bso_quantise", "bso_choose_routes", "bso_lane_encode", "bso_lane_decode", "bso_fw_table",
+                   "bso_quantise", "bso_choose_routes", "bso_lane_encode", "bso_lane_decode",
+                   "bso_joint_lane_encode", "bso_joint_lane_decode", "bso_fw_table",
                    "bso_fw_encode", "bso_fw_parse", "bso_fw_decode"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -268,6 +271,40 @@ def lane_decode(Fs, ns, route, Fh, nh, state, words, nibbles, S):
     fin = ctypes.c_uint32()
     st = lib().bso_lane_decode(_ptr(Fs), ns, _ptr(route), _ptr(Fhb), nr, nh, state, _ptr(wd), wd.size, _ptr(nb), S,
                                _ptr(out), ctypes.byref(fin))
+    return st, out[:S].copy(), fin.value
+
+
+def joint_lane_encode(Fj, nj, words):
+    """One lane of the JOINT kind: returns (start_state, words, tags) for the pair table
+    Fj[4096] of precision nj. The low nibbles of ``words`` do not enter the state."""
+    Fj = np.ascontiguousarray(Fj, dtype=np.uint32)
+    assert Fj.size == 4096
+    w = np.ascontiguousarray(words, dtype=np.uint16)
+    S = w.size
+    wo = np.zeros(max(S, 1), np.uint16)
+    tg = np.zeros(max(S, 1), np.uint32)
+    st_out = ctypes.c_uint32()
+    nw = ctypes.c_uint32()
+    st = lib().bso_joint_lane_encode(_ptr(Fj), nj, _ptr(w), S, ctypes.byref(st_out), _ptr(wo), _ptr(tg),
+                                     ctypes.byref(nw))
+    if st:
+        raise OracleError(st, "joint_lane_encode")
+    return st_out.value, wo[: nw.value].copy(), tg[: nw.value].copy()
+
+
+def joint_lane_decode(Fj, nj, state, words, nibbles, S):
+    """Returns (status, decoded words, final state) of one JOINT lane."""
+    Fj = np.ascontiguousarray(Fj, dtype=np.uint32)
+    assert Fj.size == 4096
+    wd = np.ascontiguousarray(words, dtype=np.uint16)
+    nb = np.ascontiguousarray(nibbles, dtype=np.uint8)
+    assert nb.size >= S
+    if nb.size == 0:
+        nb = np.zeros(1, np.uint8)
+    out = np.zeros(max(S, 1), np.uint16)
+    fin = ctypes.c_uint32()
+    st = lib().bso_joint_lane_decode(_ptr(Fj), nj, state, _ptr(wd), wd.size, _ptr(nb), S, _ptr(out),
+                                     ctypes.byref(fin))
     return st, out[:S].copy(), fin.value
 
 

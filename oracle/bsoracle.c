@@ -397,6 +397,73 @@ int bso_lane_decode(const uint32_t* Fs, uint32_t ns, const uint8_t* route, const
     return BSO_OK;
 }
 
+/* The JOINT kind, one lane: the pair table Fj[4096] is given directly (sum 2^nj,
+ * 8 <= nj <= 13). Encoding and the tags are as for bso_lane_encode; only the pair
+ * j = w >> 4 goes through the state. */
+static int joint_model_from_table(model_t* m, const uint32_t* Fj, uint32_t nj) {
+    memset(m, 0, sizeof(*m));
+    if (nj < 8 || nj > 13) return BSO_E_ARG;
+    uint64_t sum = 0;
+    for (int j = 0; j < JOINT_PAIRS; j++) { m->Fj[j] = Fj[j]; sum += Fj[j]; }
+    if (sum != (1u << nj)) return BSO_E_ARG;
+    m->joint = 1;
+    m->nj = nj;
+    return joint_build(m);
+}
+
+int bso_joint_lane_encode(const uint32_t* Fj, uint32_t nj, const uint16_t* w, uint32_t S, uint32_t* state_out,
+                          uint16_t* words_out, uint32_t* tags_out, uint32_t* n_words_out) {
+    model_t* m = (model_t*)calloc(1, sizeof(model_t));
+    if (!m) return BSO_E_NOMEM;
+    int st = joint_model_from_table(m, Fj, nj);
+    for (uint32_t t = 0; !st && t < S; t++)
+        if (m->Fj[w[t] >> 4] == 0) st = BSO_E_ARG;
+    uint8_t* em = (uint8_t*)malloc(S ? S : 1);
+    uint16_t* wd = (uint16_t*)malloc(sizeof(uint16_t) * (S ? S : 1));
+    if (!st && (!em || !wd)) st = BSO_E_NOMEM;
+    if (!st) {
+        *state_out = lane_encode(m, w, S, em, wd);
+        uint32_t k = 0;
+        for (uint32_t t = 0; t < S; t++)
+            if (em[t]) { words_out[k] = wd[t]; tags_out[k] = t; k++; }
+        *n_words_out = k;
+    }
+    free(em);
+    free(wd);
+    model_free(m);
+    free(m);
+    return st;
+}
+
+/* Decode S weights of one JOINT lane from `state`, taking words in order; nib[t] is the
+ * low nibble of weight t. BSO_E_CORRUPT unless the lane ends at L with every word used. */
+int bso_joint_lane_decode(const uint32_t* Fj, uint32_t nj, uint32_t state, const uint16_t* words, uint32_t n_words,
+                          const uint8_t* nib, uint32_t S, uint16_t* out, uint32_t* final_state) {
+    model_t* m = (model_t*)calloc(1, sizeof(model_t));
+    if (!m) return BSO_E_NOMEM;
+    int st = joint_model_from_table(m, Fj, nj);
+    if (st) { model_free(m); free(m); return st; }
+    uint32_t x = state, pos = 0;
+    int bad = x < STATE_L;
+    for (uint32_t t = 0; t < S; t++) {
+        uint32_t slot = x & ((1u << nj) - 1u);
+        uint32_t j = m->j_of_slot[slot];
+        x = m->Fj[j] * (x >> nj) + (slot - m->cum_j[j]);
+        if (x < STATE_L) {
+            uint32_t wd = 0;
+            if (pos < n_words) wd = words[pos]; else bad = 1;
+            pos++;
+            x = (x << 16) | wd;
+        }
+        out[t] = (uint16_t)((j << 4) | (nib[t] & 15u));
+    }
+    *final_state = x;
+    model_free(m);
+    free(m);
+    if (bad || x != STATE_L || pos != n_words) return BSO_E_CORRUPT;
+    return BSO_OK;
+}
+
 /* ------------------------------------------------------------------ */
 /* Encoder of one BF16 tensor, FORMAT.md sections 3, 4.3-4.5, 6       */
 /* ------------------------------------------------------------------ */

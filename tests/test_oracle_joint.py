@@ -9,6 +9,8 @@ What pins it:
 * Gibbs' inequality and the 0.5% overhead gate against the empirical entropy;
 * every malformed JOINT field is refused.
 """
+import itertools
+import math
 import os
 import struct
 
@@ -51,6 +53,78 @@ def test_golden_encode_and_decode():
     assert np.array_equal(oracle.decode(want, 0), w)
     ti = oracle.info(want, 0)
     assert (ti["kind"], ti["ns"], ti["nh"], ti["n_routes"], ti["nib_mode"]) == (oracle.KIND_JOINT, 13, 0, 0, 0x10)
+
+
+# Single-lane JOINT models for the brute force: (nj, {pair j: Fj}). The first has power-of-two
+# frequencies, so lane states land exactly on the renormalisation bound Fj << (32 - nj) and an
+# off-by-one comparison there breaks the round trip; the second codes two pairs of frequency 1
+# at the largest precision; the third has frequencies with no common power of two.
+TINY_JOINT = [
+    (8, {1016: 128, 1017: 64, 3000: 64}),
+    (13, {1016: 8190, 1017: 1, 2047: 1}),
+    (10, {5: 700, 1016: 300, 4095: 24}),
+]
+L = 1 << 16
+
+
+@pytest.mark.parametrize("mi", range(len(TINY_JOINT)))
+def test_bruteforce_tiny_joint_alphabets(mi):
+    """Every sequence of length <= 8 over three pairs: decode inverts encode, the lane ends at
+    L, at most one word leaves per step, and the code length log2(start state) + 16 * words
+    is 16 + sum log2(2^nj / F) within the rANS rounding bound log2(1 + 2^(nj - 16)) per step."""
+    nj, freqs = TINY_JOINT[mi]
+    Fj = np.zeros(4096, np.uint32)
+    for j, f in freqs.items():
+        Fj[j] = f
+    assert Fj.sum() == 1 << nj
+    pairs = sorted(freqs)
+    n_seq = 0
+    for S in range(0, 9):
+        for seq in itertools.product(pairs, repeat=S):
+            words = np.array([(j << 4) | ((5 * t + 3) & 15) for t, j in enumerate(seq)], np.uint16)
+            x0, wd, tags = oracle.joint_lane_encode(Fj, nj, words)
+            assert L <= x0 < (1 << 32)
+            assert np.all(np.diff(tags.astype(np.int64)) > 0)
+            st, out, fin = oracle.joint_lane_decode(Fj, nj, x0, wd, words & 15, S)
+            assert st == 0 and fin == L
+            assert np.array_equal(out, words)
+            ideal = sum(nj - math.log2(freqs[j]) for j in seq)
+            got = math.log2(x0) + 16 * wd.size
+            assert abs(got - 16 - ideal) <= 1e-6 + S * math.log2(1 + 2.0 ** (nj - 16)), (seq, got, ideal)
+            n_seq += 1
+    assert n_seq == sum(3 ** k for k in range(9))
+
+
+def test_joint_lane_hits_the_bound_exactly():
+    # Under the first model pair 1016 has frequency 128 of 2^8 and cumulative 0, so encoding it
+    # maps x to (x / 128) * 256 + x % 128, which doubles a state that is a multiple of 128.
+    # From L = 2^16, fifteen weights reach 2^31 = 128 << (32 - 8), the bound itself, so the
+    # sixteenth (step 0) must emit the low word 0 and continue from 2^15, ending at 2^16.
+    nj, freqs = TINY_JOINT[0]
+    Fj = np.zeros(4096, np.uint32)
+    for j, f in freqs.items():
+        Fj[j] = f
+    words = np.full(16, 1016 << 4, np.uint16)
+    x0, wd, tags = oracle.joint_lane_encode(Fj, nj, words)
+    assert wd.tolist() == [0] and tags.tolist() == [0]
+    assert x0 == 1 << 16
+    # fifteen weights stay below the bound and emit nothing
+    x15, wd15, _ = oracle.joint_lane_encode(Fj, nj, words[:15])
+    assert x15 == 1 << 31 and wd15.size == 0
+    st, out, fin = oracle.joint_lane_decode(Fj, nj, x0, wd, words & 15, 16)
+    assert st == 0 and fin == L and np.array_equal(out, words)
+
+
+def test_joint_lane_refuses_bad_tables():
+    Fj = np.zeros(4096, np.uint32)
+    Fj[7] = 255                       # sums to 255, not 2^8
+    with pytest.raises(oracle.OracleError):
+        oracle.joint_lane_encode(Fj, 8, np.array([7 << 4], np.uint16))
+    Fj[7] = 256
+    with pytest.raises(oracle.OracleError):   # a pair of frequency 0
+        oracle.joint_lane_encode(Fj, 8, np.array([8 << 4], np.uint16))
+    with pytest.raises(oracle.OracleError):   # precision outside 8..13
+        oracle.joint_lane_encode(Fj, 7, np.array([7 << 4], np.uint16))
 
 
 def test_every_pattern_round_trips():

@@ -1,7 +1,10 @@
 """Pins of the oracle against facts that do not come from the oracle itself.
 
-* FORMAT.md section 8: two containers derived by hand (tests/golden/one_weight.hex with
-  constant nibbles, tests/golden/two_weights.hex with stored nibbles).
+* Containers derived by hand: one weight with constant nibbles (tests/golden/one_weight.hex),
+  two weights with stored nibbles (tests/golden/two_weights.hex), and sixteen weights whose
+  lanes emit different words at the same steps, which fixes the (step, lane) order of the
+  interleaved stream (tests/golden/interleave_sixteen.hex and, for kind JOINT,
+  tests/golden/joint_interleave_sixteen.hex).
 * The NVLC model card's field split and bitwise reconstruction: every 16-bit pattern
   round-trips (this covers +-0, subnormals, +-inf and NaN payloads).
 * rANS exactness: brute force over tiny alphabets, where the decode must invert the
@@ -50,6 +53,60 @@ def test_golden_decode(golden_dir, fname, words, size, nib_mode):
     ti = oracle.info(c, 0)
     assert (ti["kind"], ti["ns"], ti["nh"], ti["n_chunks"], ti["name"], ti["nib_mode"]) == (0, 11, 5, 1, "w", nib_mode)
     assert oracle.decode(c, 0).tolist() == words
+
+
+# ---------------------------------------------------------------- the interleaved stream
+# Sixteen weights whose lanes 0 and 1 emit different words at the same steps (0 and 4), derived
+# by hand in the comments of tests/golden/interleave_sixteen.hex (kind RANS, ns 1, nh 3) and
+# tests/golden/joint_interleave_sixteen.hex (kind JOINT, nj 12).
+SIXTEEN = np.array([0x3F80 + 16 * h for h in range(8)] + [0x4000 + 16 * h for h in range(8)], np.uint16)
+INTERLEAVE = [("interleave_sixteen.hex", dict(ns=1, nh=3), 768, [0x00010000, 0x00010008],
+               [0x4321, 0xCBA9], [0x0765, 0x0FED]),
+              ("joint_interleave_sixteen.hex", dict(model="joint", nj=12), 576, [0x00010043, 0x000108CB],
+               [0x2107, 0xA90F], [0x6500, 0xED00])]
+
+
+def _chunk0(c):
+    ti = oracle.info(c, 0)
+    e = ti["data_offset"]
+    off = int.from_bytes(c[e:e + 8], "little")
+    nw = int.from_bytes(c[e + 8:e + 12], "little")
+    return off, nw
+
+
+@pytest.mark.parametrize("fname,kw,size,states,step0,step4", INTERLEAVE)
+def test_interleave_golden_encode_and_decode(golden_dir, fname, kw, size, states, step0, step4):
+    want = _golden_bytes(os.path.join(golden_dir, fname))
+    assert len(want) == size
+    assert oracle.encode([("w", SIXTEEN, "bf16")], force_rans=True, **kw) == want
+    assert np.array_equal(oracle.decode(want, 0), SIXTEEN)
+    off, nw = _chunk0(want)
+    st = np.frombuffer(want[off:off + 128], "<u4")
+    words = np.frombuffer(want[off + 128:off + 128 + 2 * nw], "<u2")
+    assert nw == 64 and st[:2].tolist() == states and set(st[2:].tolist()) == {0x00010000}
+    # (step, lane) order: step 0's 32 words, then step 4's
+    assert words[:2].tolist() == step0 and words[32:34].tolist() == step4
+    assert not words[2:32].any() and not words[34:].any()
+
+
+@pytest.mark.parametrize("fname,kw,size,states,step0,step4", INTERLEAVE)
+def test_interleave_order_is_what_decodes(golden_dir, fname, kw, size, states, step0, step4):
+    # Any other order of the same words fails: lane order swapped within a step, or the two
+    # steps' blocks swapped. Each variant either fails the end check or decodes other weights.
+    c = _golden_bytes(os.path.join(golden_dir, fname))
+    off, nw = _chunk0(c)
+    w0 = off + 128
+    words = bytearray(c[w0:w0 + 2 * nw])
+    lanes = words[2:4] + words[0:2] + words[4:]
+    steps = words[64:] + words[:64]
+    for variant in (lanes, steps):
+        bad = c[:w0] + bytes(variant) + c[w0 + 2 * nw:]
+        try:
+            out = oracle.decode(bad, 0)
+        except oracle.OracleError as e:
+            assert e.code == oracle.E_CORRUPT
+        else:
+            assert not np.array_equal(out, SIXTEEN)
 
 
 def test_checksum_published_splitmix64_outputs():
