@@ -178,3 +178,25 @@ def test_bad_arguments():
     assert e.value.code == bs.E_ARG
     with pytest.raises(bs.BsError):
         bs.Plan(c[:-16], device="cuda:0")
+
+
+def _golden(name):
+    import os
+    hexs = []
+    with open(os.path.join(os.path.dirname(__file__), "golden", name)) as fh:
+        for line in fh:
+            hexs.append(line.split("#", 1)[0])
+    return bytes.fromhex("".join("".join(hexs).split()))
+
+
+@pytest.mark.parametrize("name", ["one_weight.hex", "two_weights.hex", "interleave_sixteen.hex",
+                                  "joint_two_weights.hex", "joint_interleave_sixteen.hex"])
+def test_hand_derived_containers(name):
+    # the containers derived by hand in the golden files' comments, decoded on the device;
+    # the interleave pair fixes the (step, lane) order in which the warp takes the words
+    c = _golden(name)
+    want = oracle.decode(c, 0)
+    plan, outs = _decode_all(c, 1)
+    assert np.array_equal(outs[0].reshape(-1), want.reshape(-1))
+    if "sixteen" in name:
+        assert outs[0].reshape(-1).tolist() == [0x3F80 + 16 * h for h in range(8)] + [0x4000 + 16 * h for h in range(8)]
