@@ -8,8 +8,10 @@
  *   - the decoded symbol selects the distribution of the 7-bit fraction (here a table over
  *     its top three bits; the low four bits are kept verbatim);
  *   - the fields are recombined bitwise, so the output is byte-identical to the original.
- * The container layout (interleaved 32-lane chunks, tables, raw spans, checksum) is
- * specified in FORMAT.md in this repository.
+ * The container (BF16RANS version 2: interleaved 32-lane chunks, quantised tables, raw
+ * spans, a per-tensor checksum) is this library's own design; the card gives no byte layout.
+ * Each declaration below names the passage that defines its operation, or says that it is
+ * this library's design.
  *
  * Conventions
  *  - Every function returns a bs_status, and nothing throws across the ABI.
@@ -37,7 +39,7 @@ extern "C" {
 typedef enum {
     BS_OK = 0,
     BS_E_ARG = 1,          /* null pointer, bad index, misaligned buffer, bad size */
-    BS_E_FORMAT = 2,       /* the container fails validation (FORMAT.md section 5) */
+    BS_E_FORMAT = 2,       /* the container fails validation (bad magic, offsets, tables, sizes) */
     BS_E_VERSION = 3,      /* unknown magic version */
     BS_E_SIZE = 4,         /* an output or workspace buffer is the wrong size */
     BS_E_CUDA = 5,         /* a CUDA runtime call failed (the CUDA error is kept, see bs_last_cuda_error) */
@@ -55,23 +57,26 @@ typedef struct {
     uint64_t out_bytes;   /* size of the decoded tensor: 2*n_elems, or n_elems for RAW */
     uint64_t coded_bytes; /* RANS: model + chunk table + chunk payloads (padded); else out_bytes */
     uint64_t n_chunks;    /* RANS only */
-    uint64_t checksum;    /* FORMAT.md section 7, of the original tensor */
+    uint64_t checksum;    /* of the original tensor: sum of splitmix64((i << 16) | w[i]) mod 2^64 */
     uint64_t shape[8];
     uint32_t kind;        /* BS_KIND_* */
     uint32_t ndim;
-    uint32_t ns, nh, n_routes, log2_chunk; /* RANS model parameters (FORMAT.md section 2); JOINT: ns = nj, nh = n_routes = 0 */
+    uint32_t ns, nh, n_routes, log2_chunk; /* RANS: s-table and h-table precisions, routes, chunk; JOINT: ns = nj, nh = n_routes = 0 */
     const char* name;     /* not NUL-terminated; points into the plan */
     uint32_t name_bytes;
     uint32_t nib_mode;    /* RANS: 0 = nibbles stored, 0x10 + c = every low nibble is c */
 } bs_tensor_info;
 
 /* Bytes of device workspace that bs_plan needs for this container: the decode
- * tables of every RANS tensor plus a 256-byte error block. h_container must hold the
- * whole container. Returns 0 if the container does not validate. */
+ * tables of every coded tensor plus a 256-byte error block. h_container must hold the
+ * whole container. Returns 0 if the container does not validate. This library's design. */
 size_t bs_plan_workspace_bytes(const void* h_container, size_t container_bytes);
 
 /*
  * bs_plan: parse and validate a container, build its decode tables and upload them.
+ * Source: the per-tensor model of the NVLC card's field-split paragraph (each tensor carries
+ * its own quantised frequency tables; here they are expanded into slot tables for the
+ * decode). Validation, the workspace and the plan object are this library's design.
  *
  *   h_container      host copy of the whole container (read only during the call), or
  *                    NULL: the plan then reads the header, directory, models and chunk
@@ -84,18 +89,21 @@ size_t bs_plan_workspace_bytes(const void* h_container, size_t container_bytes);
  *   stream           the tables are uploaded with cudaMemcpyAsync on this stream
  *   out              receives the plan
  *
- * Validation follows FORMAT.md section 5: a bad header gives BS_E_FORMAT or
- * BS_E_VERSION, and a short workspace gives BS_E_SIZE.
+ * Validation checks every offset, size, table sum and start state before any device work: a
+ * bad container gives BS_E_FORMAT or BS_E_VERSION, and a short workspace gives BS_E_SIZE.
  */
 bs_status bs_plan(const void* h_container, size_t container_bytes, const void* d_container, void* d_workspace,
                   size_t workspace_bytes, void* stream, bs_plan_t** out);
 
 /* As bs_plan_workspace_bytes, reading the metadata from device memory (synchronous
- * copies on stream). Returns 0 if the container does not validate. */
+ * copies on stream). Returns 0 if the container does not validate. This library's design. */
 size_t bs_plan_workspace_bytes_device(const void* d_container, size_t container_bytes, void* stream);
 
+/* Frees the plan's host memory. The caller's device buffers are untouched. */
 void bs_plan_destroy(bs_plan_t* plan);
 
+/* The directory as parsed (this library's design): tensor count, and one entry's metadata.
+ * BS_E_ARG for a NULL pointer or an index out of range. */
 bs_status bs_tensor_count(const bs_plan_t* plan, int32_t* n);
 bs_status bs_tensor_info_get(const bs_plan_t* plan, int32_t idx, bs_tensor_info* out);
 
@@ -103,15 +111,21 @@ bs_status bs_tensor_info_get(const bs_plan_t* plan, int32_t idx, bs_tensor_info*
  * bs_decode_tensor: decode tensor idx into d_out (device, 16-byte aligned, out_bytes =
  * the tensor's out_bytes; otherwise BS_E_SIZE / BS_E_ARG). The work is enqueued on stream
  * and the call returns at once.
- *  - RANS: the interleaved rANS decode kernel, with one warp per 32-lane chunk.
+ * Source: the NVLC card's field-split paragraph. The sign+exponent symbol is rANS-decoded
+ * with the tensor's model, it selects the fraction's distribution, the fraction is decoded
+ * with it, and the fields are recombined bitwise into the original word; non-BF16 spans come
+ * back verbatim from the residual stream. The 32 interleaved lanes per chunk are this
+ * library's reading of the card's "lane-oriented streams" (runtime streams paragraph).
+ *  - RANS and JOINT: the interleaved rANS decode kernel, with one warp-lane per rANS state.
  *  - STORED and RAW: a vectorised copy kernel.
  */
 bs_status bs_decode_tensor(const bs_plan_t* plan, int32_t idx, void* d_out, size_t out_bytes, void* stream);
 
 /*
- * bs_decode_batch: decode n tensors in one pass. All the RANS tensors go in a single
- * kernel launch per CTA shape (more than 500 of them are split across launches), and STORED/RAW
- * tensors in one copy launch. idx[k] goes to d_out[k], of out_bytes[k] bytes.
+ * bs_decode_batch: decode n tensors in one pass: the operation of bs_decode_tensor for each.
+ * The batching is this library's design. All the coded tensors of one kernel instance go in a
+ * single launch (more than 500 of them are split across launches), and STORED/RAW tensors in
+ * one copy launch. idx[k] goes to d_out[k], of out_bytes[k] bytes.
  *  - The outputs must not overlap.
  *  - idx, d_out and out_bytes are host arrays, read during the call.
  */
@@ -122,7 +136,8 @@ bs_status bs_decode_batch(const bs_plan_t* plan, const int32_t* idx, void* const
  * bs_decode_ranges: decode parts of tensors, in whole chunks, in one pass (the launches of
  * bs_decode_batch). It serves callers that decode a checkpoint in batches of a fixed size,
  * say 1 GB of output at a time, where one batch may end inside a tensor and the next one
- * continue it.
+ * continue it. The operation is bs_decode_tensor's; cutting at chunk boundaries is this
+ * library's design.
  *  - Range k decodes elements [begin, begin + count) of tensor idx (bytes for RAW) into
  *    d_out, which receives exactly those words: out_bytes = 2 * count (RAW: count).
  *  - RANS and JOINT tensors: begin must be a multiple of the tensor's chunk size
@@ -147,7 +162,7 @@ bs_status bs_decode_ranges(const bs_plan_t* plan, const bs_range* ranges, int32_
 
 /*
  * bs_decode_geometry: how the decode kernel splits tensor idx on the current device, for
- * callers that cut their decode into batches (bs_decode_ranges).
+ * callers that cut their decode into batches (bs_decode_ranges). This library's design.
  *  - *chunks_per_cta receives the chunks one CTA takes at the kernel's largest shape. All of
  *    a CTA's chunks come from one tensor, so a range whose chunk count is not a multiple of
  *    it leaves its last CTA part-filled. STORED and RAW tensors give 0.
@@ -161,8 +176,9 @@ bs_status bs_decode_ranges(const bs_plan_t* plan, const bs_range* ranges, int32_
 bs_status bs_decode_geometry(const bs_plan_t* plan, int32_t idx, uint32_t* chunks_per_cta, uint32_t* ctas_per_wave);
 
 /*
- * bs_verify_tensor: compute the FORMAT.md section 7 checksum of a decoded tensor on the
- * device and compare it with the stored one. The check is the analogue of the per-tensor
+ * bs_verify_tensor: compute the per-tensor checksum (sum over i of splitmix64((i << 16) |
+ * w[i]) mod 2^64; bytes for RAW) of a decoded tensor on the device and compare it with the
+ * stored one. The check is the analogue of the per-tensor
  * md5 that the "Gemma 2 9B Instruct -- Lossless Compressed" card ("What lossless
  * means") runs at decompression.
  *  - d_scratch: 16 device bytes, 8-byte aligned, owned by the caller.
@@ -173,7 +189,9 @@ bs_status bs_verify_tensor(const bs_plan_t* plan, int32_t idx, const void* d_out
                            void* d_scratch, void* stream, uint64_t* got);
 
 /*
- * bs_check: synchronise stream, then read and clear the plan's device error word.
+ * bs_check: synchronise stream, then read and clear the plan's device error word. The check
+ * behind it is this library's design: every rANS lane of a chunk must end in the state L the
+ * encoder started from, having consumed exactly the chunk's words.
  * Returns BS_E_CORRUPT if any decode since the last check found a corrupt chunk. In
  * that case *first_bad (if not NULL) is (tensor_index << 40) | chunk_index of the
  * smallest such pair, and -1 otherwise.
@@ -213,8 +231,9 @@ bs_status bs_decode_tensor_noalloc(const void* h_container, size_t container_byt
                                    int32_t idx, void* d_out, size_t out_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------
- * Encoder on the device. It produces the canonical container of FORMAT.md section 4.6,
- * byte-identical to any other encoder that follows FORMAT.md section 6. The card's
+ * Encoder on the device. It produces the canonical container (header, directory, names, then
+ * each tensor's model, chunk table and chunks), byte-identical to any other encoder that
+ * follows the container's integer rules (quantiser, routes, pad word, STORED fallback). The card's
  * compressor ("bigsmall compress" on the "Gemma 2 9B Instruct -- Lossless Compressed"
  * card, "Want to compress your own model?") is the user-facing counterpart.
  *
@@ -247,7 +266,7 @@ typedef struct {
     uint32_t nh;          /* 3..5 with ns + nh <= 16, default 5 */
     uint32_t max_routes;  /* 0..15, default 15 */
     uint32_t force_rans;  /* 1: never fall back to STORED (tests only) */
-    uint32_t model;       /* 0: factored RANS model (ns, nh, routes); 1: JOINT (FORMAT.md section 1) */
+    uint32_t model;       /* 0: factored RANS model (ns, nh, routes); 1: JOINT (one table over (s, h)) */
     uint32_t nj;          /* JOINT precision, 8..13, default 13 */
 } bs_enc_params;
 
@@ -341,11 +360,11 @@ bs_status bs_streamer_check(bs_streamer_t* s, void* stream, int64_t* first_bad);
 void bs_streamer_destroy(bs_streamer_t* s);
 
 /* ------------------------------------------------------------------------------------
- * Fixed-width lane layout ("FW layout", FORMAT.md section 10): a runtime form of one BF16
+ * Fixed-width lane layout ("FW layout"): a runtime form of one BF16
  * tensor whose decode is a few bitwise operations per weight. The "Qwen3.8-27B-BF16-NVLC-
  * Lossless" card says its GPU runtime derives fixed-width, lane-oriented streams from the
  * rANS files once at initialisation (its Fixed7/Compact11 runtime, about 11.36 bits per
- * weight resident). The card gives no layout; section 10 is this library's:
+ * weight resident). The card gives no layout; this one is this library's:
  *   - a 4-bit code per weight for the tensor's 16 most frequent sign+exponent symbols;
  *   - the 7-bit fraction in two planes;
  *   - an exception list of (position, word) for the other symbols.
@@ -416,6 +435,7 @@ typedef struct {
  * d_err as for bs_fw_decode. Enqueued on stream. */
 bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_t batch, uint32_t* d_err, void* stream);
 
+/* Diagnostics (this library's design). */
 const char* bs_status_str(bs_status s);
 int bs_last_cuda_error(void); /* the cudaError_t behind the last BS_E_CUDA on this thread */
 /* Kernel launches libbs has made in this process (all threads); a diagnostic counter. */

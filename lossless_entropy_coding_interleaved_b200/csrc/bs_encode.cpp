@@ -1,6 +1,6 @@
 // bs_encode.cpp -- host side of the device encoder (include/bs.h, bs_encoder_*).
 //
-// It implements FORMAT.md section 6 (quantiser, route rule, joint model, pad word, STORED
+// It implements the container's integer encoder rules (quantiser, route rule, joint model, pad word, STORED
 // fallback)
 // and the canonical layout of section 4.6 from that document. It shares no code with the
 // oracle. The statistics come from histogram_kernel and the per-chunk word counts from the
@@ -32,7 +32,7 @@ void put_u64(uint8_t* p, uint64_t v) { std::memcpy(p, &v, 8); }
 void put_u32(uint8_t* p, uint32_t v) { std::memcpy(p, &v, 4); }
 void put_u16(uint8_t* p, uint16_t v) { std::memcpy(p, &v, 2); }
 
-// FORMAT.md section 6, quantiser: proportional rounding with a floor of one slot per present
+// Quantiser: proportional rounding with a floor of one slot per present
 // symbol, then one-slot moves in the direction of the sum, chosen by the first-order change
 // of sum(c * log q) (c/(2q+1) to add, c/(2q-1) to remove), lowest index on ties.
 bool quantise(const uint64_t* c, int K, uint32_t M, uint32_t* q) {
@@ -74,7 +74,7 @@ bool quantise(const uint64_t* c, int K, uint32_t M, uint32_t* q) {
     return true;
 }
 
-// FORMAT.md section 6, routes: Pearson's statistic of the fraction's top three bits against
+// Routes: Pearson's statistic of the fraction's top three bits against
 // the uniform distribution, chi2 * n_e = 8 * sum c^2 - n_e^2. Exponents with chi2 > 256
 // compete, the largest chi2 (lower exponent on ties) win up to max_routes, numbered in
 // ascending exponent.
@@ -120,9 +120,9 @@ struct EncTensor {
     bool candidate = false;         // a BF16 tensor with weights: try RANS
     uint64_t n_chunks = 0;
     uint32_t n_routes = 0;
-    uint32_t nib_mode = 0;          // FORMAT.md section 3: 0 = stored, 0x10 + c = constant c
+    uint32_t nib_mode = 0;          // 0 = stored nibble words, 0x10 + c = every low nibble is c
     uint16_t pad_word = 0;
-    std::vector<uint8_t> model;     // FORMAT.md 4.3
+    std::vector<uint8_t> model;     // the serialised model section
     std::vector<uint32_t> tables;   // encode tables (bs_internal.h)
     std::vector<uint32_t> n_words;  // per chunk, from the count pass
     uint64_t checksum = 0;
@@ -158,7 +158,7 @@ bool build_model(EncTensor& T, const bs_enc_params& P, const unsigned long long*
             only = u;
         }
     T.nib_mode = seen == 1 ? 0x10u | static_cast<uint32_t>(only) : 0u;
-    if (P.model == 1) { // FORMAT.md section 6, joint model; section 3, its pad word
+    if (P.model == 1) { // joint model: Fj = quantise(pair counts, 2^nj); the pad pair has the largest Fj
         std::vector<uint64_t> cj(hist, hist + kJointPairs);
         std::vector<uint32_t> Fj(kJointPairs);
         if (!quantise(cj.data(), kJointPairs, 1u << P.nj, Fj.data())) return false;
@@ -169,7 +169,7 @@ bool build_model(EncTensor& T, const bs_enc_params& P, const unsigned long long*
         }
         T.pad_word = static_cast<uint16_t>(j_pad << 4);
         T.n_routes = 0;
-        T.model.assign(4 + 4ull * n_pairs, 0); // FORMAT.md 4.3b
+        T.model.assign(4 + 4ull * n_pairs, 0); // n_pairs, reserved, then (j, Fj) pairs
         uint8_t* m = T.model.data();
         put_u16(m, static_cast<uint16_t>(n_pairs));
         uint64_t o = 4;
@@ -212,7 +212,7 @@ bool build_model(EncTensor& T, const bs_enc_params& P, const unsigned long long*
             if (row[h] > row[h_pad]) h_pad = h;
     }
     T.pad_word = static_cast<uint16_t>((s_pad << 7) | (h_pad << 4));
-    // model bytes (FORMAT.md 4.3)
+    // model bytes: n_present, reserved, (s, Fs) pairs, route[256], the route tables
     uint32_t n_present = 0;
     for (int s = 0; s < 512; ++s) n_present += Fs[s] != 0;
     T.model.assign(260 + 4ull * n_present + 16ull * R, 0);
@@ -384,7 +384,7 @@ bs_status bs_encoder_run(bs_encoder_t* enc, void* d_scratch_v, size_t scratch_by
         ce = cudaMemcpyAsync(hist.data(), d_hist, 8ull * kHistBins, cudaMemcpyDeviceToHost, s);
         if (ce == cudaSuccess) ce = cudaStreamSynchronize(s);
         if (ce != cudaSuccess) return enc_cuda(ce);
-        if (P.model == 1) { // FORMAT.md section 6: more distinct pairs than 2^nj slots -> STORED
+        if (P.model == 1) { // more distinct pairs than 2^nj slots: no JOINT table, so STORED
             uint32_t n_pairs = 0;
             for (uint32_t j = 0; j < kJointPairs; ++j) n_pairs += hist[j] != 0;
             if (n_pairs > (1u << P.nj)) {
@@ -415,7 +415,7 @@ bs_status bs_encoder_run(bs_encoder_t* enc, void* d_scratch_v, size_t scratch_by
     }
     ce = cudaStreamSynchronize(s);
     if (ce != cudaSuccess) return enc_cuda(ce);
-    // STORED fallback and canonical layout (FORMAT.md 4.6)
+    // STORED fallback and canonical layout (header, directory, names, then each tensor's sections)
     uint64_t names_bytes = 0;
     for (size_t k = 0; k < enc->t.size(); ++k) {
         EncTensor& T = enc->t[k];

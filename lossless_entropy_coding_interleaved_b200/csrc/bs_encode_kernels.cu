@@ -1,17 +1,17 @@
-// bs_encode_kernels.cu -- sm_100a kernels of the container encoder (FORMAT.md sections 3, 6).
+// bs_encode_kernels.cu -- sm_100a kernels of the container encoder: histograms and the lane encode.
 //
 // histogram_kernel: per-tensor counts of the pairs j = w >> 4 = (s << 3) | h (sign+exponent
 // symbol s, the fraction's top three bits h) and of the low nibbles. The s counts and the
 // (exponent, h) counts that the factored model needs are sums of pair counts, and the JOINT
-// model uses the pair counts as they are (FORMAT.md section 6). The counts go into per-CTA
+// model uses the pair counts as they are. The counts go into per-CTA
 // shared memory, then into global 64-bit bins.
 //
 // encode_kernel: one warp per chunk, lane j holds rANS state j (32-bit). It walks its
-// steps backwards from L = 2^16 as FORMAT.md section 2 specifies: each weight renormalises
+// steps backwards from L = 2^16: each weight renormalises
 // at most once (one 16-bit word) and is one step of the product alphabet (s, h). The count
 // pass records how many words each chunk emits. The write pass places the words of step t
 // (lane order) just before those of step t+1, starting from the end of the chunk's word
-// area. That is the interleaved order of FORMAT.md section 3, with no staging buffer. The
+// area. That is the interleaved (step, lane) order of the word stream, with no staging buffer. The
 // write pass also stores the nibble words when the tensor keeps them.
 #include <cuda_runtime.h>
 
@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(kEncWarps * 32) encode_kernel(const __grid_con
 #pragma unroll
             for (int k = 0; k < 8; ++k) v[k] = (i0 + k < nc) ? in[i0 + k] : it.pad_word;
         }
-        if (p.write && it.nib_stored) { // FORMAT.md section 3: step k's nibble at 4*(k >> 1) + 16*(k & 1)
+        if (p.write && it.nib_stored) { // step k's nibble sits at bit 4*(k >> 1) + 16*(k & 1)
             uint32_t nib = 0;
 #pragma unroll
             for (int k = 0; k < 8; ++k) nib |= static_cast<uint32_t>(v[k] & 15u) << (4 * (k >> 1) + 16 * (k & 1));
@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kEncWarps * 32) encode_kernel(const __grid_con
             }
             if (emit) x >>= 16;
             const uint32_t r = x % Q;
-            if (it.joint) x = ((x / Q) << P) + cs + r; // FORMAT.md section 2, the JOINT kind
+            if (it.joint) x = ((x / Q) << P) + cs + r; // the JOINT kind: x = (x / Fj) * 2^nj + cum(j) + x % Fj
             else x = ((x / Q) << P) + ((cs + r / qh) << nh) + ch + r % qh;
         }
     }

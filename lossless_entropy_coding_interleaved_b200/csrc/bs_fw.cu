@@ -1,4 +1,4 @@
-// bs_fw.cu -- the fixed-width lane layout (FORMAT.md section 10) on sm_100a: the device
+// bs_fw.cu -- the fixed-width lane layout on sm_100a: the device
 // transcoder from BF16 words, the decode kernel, and their C ABI (include/bs.h).
 //
 // The "Qwen3.8-27B-BF16-NVLC-Lossless" card says its GPU runtime derives fixed-width,

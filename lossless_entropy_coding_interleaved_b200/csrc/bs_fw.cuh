@@ -1,5 +1,6 @@
 // bs_fw.cuh -- definitions shared by the kernels of the fixed-width lane layout
-// (FORMAT.md section 10): the decode in bs_fw.cu and the fused GEMV in bs_fw_gemv.cu.
+// (4-bit sign+exponent codes, 7-bit fractions, exceptions): the decode in bs_fw.cu and the fused
+// GEMV in bs_fw_gemv.cu.
 // Nothing here is shared with the oracle.
 #pragma once
 
@@ -20,7 +21,7 @@ constexpr uint64_t kFwMaxElems = 1ull << 40;
 
 __host__ __device__ inline uint64_t up16(uint64_t v) { return (v + 15) & ~uint64_t(15); }
 
-// FORMAT.md section 10, byte layout: section offsets from the start of the layout.
+// Byte layout: section offsets from the start of the layout.
 struct FwOffsets {
     uint64_t a, b, c, tile_exc, exc_pos, exc_word, total;
 };

@@ -1,5 +1,5 @@
 // bs_fw_gemv.cu -- y = W x for a weight matrix W held in the fixed-width lane layout
-// (FORMAT.md section 10). W is decoded in registers on its way to the multiply, so no dense
+// (4-bit codes, 7-bit fractions, exceptions). W is decoded in registers on its way to the multiply, so no dense
 // copy of it is ever written.
 //
 // This is the operand path that the "Qwen3.8-27B-BF16-NVLC-Lossless" card describes for its

@@ -13,7 +13,8 @@ namespace bs {
 
 inline uint64_t up256(uint64_t v) { return (v + 255) & ~uint64_t(255); }
 
-// Parse and validate a container held in host memory (FORMAT.md sections 4-5).
+// Parse and validate a container held in host memory (byte layout and validation rules of
+// the BF16RANS container, version 2).
 bs_status parse_host_container(const uint8_t* h, uint64_t len, std::vector<Tensor>& out);
 
 // Bytes of the decode workspace: the error block, then each RANS tensor's tables.
@@ -32,7 +33,8 @@ bs_status build_workspace(std::vector<Tensor>& ts, std::vector<uint8_t>& image);
 // and launches every bin on flush().
 // The decode kernel instance (and CTA shape) of a coded tensor.
 inline DecodeMode decode_mode_of(const Tensor& t) {
-    if (t.kind == BS_KIND_JOINT) return t.ns == kDefaultNj ? DecodeMode::Joint : DecodeMode::JointGeneric;
+    if (t.kind == BS_KIND_JOINT)
+        return t.joint_compact ? DecodeMode::JointCompact : t.ns == kDefaultNj ? DecodeMode::Joint : DecodeMode::JointGeneric;
     return is_default_precision(t.ns, t.nh) ? DecodeMode::Default : DecodeMode::Generic;
 }
 
@@ -60,7 +62,7 @@ class DecodeBatch {
     bs_status flush_copy(void* stream);
     unsigned long long* err_;
     uint32_t sms_ = 148;
-    Bin bins_[4];
+    Bin bins_[kDecodeModes];
     std::unique_ptr<CopyParams> cp_;
 };
 

@@ -12,23 +12,32 @@
 
 namespace bs {
 
-// FORMAT.md sections 2-4 (version 2)
+// The BF16RANS container, version 2: 32 lanes per chunk, 32-bit states in [2^16, 2^32),
+// 64-byte header, 144-byte directory entries
 constexpr uint32_t kFormatVersion = 2;
 constexpr uint32_t kLanes = 32;
 constexpr uint32_t kStateL = 1u << 16;
 constexpr uint32_t kHeaderBytes = 64;
 constexpr uint32_t kDirEntryBytes = 144;
 constexpr uint32_t kMaxNs = 12, kMinNh = 3, kMaxNh = 5, kMaxPrecision = 16, kMaxRoutes = 15;
-// The JOINT kind (FORMAT.md sections 1-2): one table over the 4096 pairs j = (s << 3) | h,
+// The JOINT kind: one table over the 4096 pairs j = (s << 3) | h,
 // precision nj. Its decode table (2^nj entries of 8 bytes) sits at offset 0 of shared
 // memory, and the rings follow at kJointRegion.
 constexpr uint32_t kJointPairs = 4096, kMinNj = 8, kMaxNj = 13;
 constexpr uint32_t kJointRegion = 8u << kMaxNj;
+// A JOINT tensor whose frequencies are all below 256 (every large tensor of normally
+// distributed weights) gets 4-byte slot entries instead: F in byte 0, the slot's rank in
+// byte 1, bits 16-19 zero and the pair j in bits 20-31 (so the high half is the word j << 4).
+// A random 4-byte gather of 32 lanes costs about 3.5 shared-memory wavefronts against about
+// 6 for the 8-byte one. The table region is then at most 32 KiB.
+constexpr uint32_t kCompactMaxF = 255;
+constexpr uint32_t kJoint4Region = 4u << kMaxNj;
+inline uint32_t joint4_table_bytes(uint32_t nj) { return 4u << nj; }
 inline bool is_coded(uint32_t kind) { return kind == BS_KIND_RANS || kind == BS_KIND_JOINT; }
 // joint table entry for slot (cum(j) + k): .x = F | (word << 16) with word = j << 4, .y = k
 inline uint32_t joint_table_bytes(uint32_t nj) { return 8u << nj; }
 // Bytes of a chunk payload: 32 start states, the nibble words when stored, the 16-bit
-// words, padded to 16 (FORMAT.md section 4.5).
+// words, padded to 16.
 inline uint64_t payload_bytes(uint64_t n_c, uint32_t n_words, bool nib_stored) {
     const uint64_t blocks = (n_c + 255) / 256;
     return (128 + (nib_stored ? 128 * blocks : 0) + 2ull * n_words + 15) & ~uint64_t(15);
@@ -86,6 +95,10 @@ inline uint32_t joint_smem_bytes(uint32_t warps, uint32_t chains) {
     return kJointRegion + warps * chains * (kRingBytes + kNibRingBytes);
 }
 
+inline uint32_t joint4_smem_bytes(uint32_t warps, uint32_t chains) {
+    return kJoint4Region + warps * chains * (kRingBytes + kNibRingBytes);
+}
+
 // Workspace layout: a 256-byte error block, then 256-aligned tables per RANS tensor.
 constexpr uint64_t kErrBlockBytes = 256;
 
@@ -96,7 +109,8 @@ struct Tensor {
     uint64_t checksum = 0, coded_bytes = 0;
     uint64_t shape[8] = {0};
     std::string name;
-    std::vector<uint8_t> model; // RANS: the model section (FORMAT.md 4.3)
+    std::vector<uint8_t> model; // coded kinds: the model section as stored
+    uint32_t joint_compact = 0; // JOINT: 4-byte slot entries (every frequency <= kCompactMaxF)
     uint64_t ws_offset = 0;   // RANS: byte offset of the decode tables in the workspace
     uint32_t table_bytes = 0; // RANS: bytes of s-table + compact fraction rows (multiple of 16)
 };
@@ -213,14 +227,19 @@ void count_launch();
 // Which decode_kernel instance a launch uses: the default precisions (ns 11, nh 5), any
 // other factored precisions, or the JOINT kind.
 // JOINT at nj = 13 (the default) has a compile-time instance; other nj use a generic one.
-enum class DecodeMode { Default = 0, Generic = 1, Joint = 2, JointGeneric = 3 };
+// JointCompact: JOINT with 4-byte slot entries, any nj.
+enum class DecodeMode { Default = 0, Generic = 1, Joint = 2, JointGeneric = 3, JointCompact = 4 };
+constexpr int kDecodeModes = 5;
+constexpr int kWarpsJoint4 = 28, kChainsJoint4 = 2;
 constexpr uint32_t kDefaultNj = 13;
 // The largest CTA shape of each mode (small launches take fewer warps, see launch_warps).
 inline uint32_t max_warps_of(DecodeMode m) {
-    return m == DecodeMode::Default ? kWarpsDefault : m == DecodeMode::Joint ? kWarpsJoint : kWarpsGeneric;
+    return m == DecodeMode::Default ? kWarpsDefault : m == DecodeMode::Joint ? kWarpsJoint
+         : m == DecodeMode::JointCompact ? kWarpsJoint4 : kWarpsGeneric;
 }
 inline uint32_t chains_of(DecodeMode m) {
-    return m == DecodeMode::Default ? kChainsDefault : m == DecodeMode::Joint ? kChainsJoint : kChainsGeneric;
+    return m == DecodeMode::Default ? kChainsDefault : m == DecodeMode::Joint ? kChainsJoint
+         : m == DecodeMode::JointCompact ? kChainsJoint4 : kChainsGeneric;
 }
 int launch_decode(const DecodeParams& p, DecodeMode mode, uint32_t smem_bytes, void* stream);
 int launch_copy(const CopyParams& p, void* stream);

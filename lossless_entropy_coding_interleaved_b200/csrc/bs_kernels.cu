@@ -7,12 +7,13 @@
 //   - s selects the fraction's distribution (here over the fraction's top three bits h;
 //     the low four bits u are stored verbatim) and h is decoded with it;
 //   - w = (s << 7) | (h << 4) | u is rebuilt bitwise.
-// Layout and parameters: FORMAT.md (version 2) sections 2-4.
+// Layout and parameters: the BF16RANS container, version 2.
 //
 // Mapping onto the B200:
 //  * One warp decodes two 32-lane chunks at once (two independent dependency chains per
 //    lane hide the latency of the table lookups). Lane j holds rANS state j of each chunk,
-//    a 32-bit state. Under the octet map of FORMAT.md section 3, a lane owns 8 contiguous
+//    a 32-bit state. Under the octet map (weight i of a chunk goes to lane (i >> 3) & 31 at
+//    step 8 * (i >> 8) + (i & 7)), a lane owns 8 contiguous
 //    output weights per 8 steps. Those leave as one 16-byte store, so a warp writes 512
 //    contiguous bytes per chunk.
 //  * One weight is one state update: the P-bit slot gives the s-entry (its high ns bits)
@@ -81,9 +82,10 @@ struct Chain {
 // NS/NH > 0: compile-time precisions (the default container); 0: read from the item.
 // SHAPE_FROM_PARAMS: the launch's warps per CTA come from the parameters (small launches);
 // otherwise the CTA has WARPS warps, a compile-time constant (measured 3% faster).
-// JOINT: the JOINT kind (FORMAT.md sections 1-2): one table of 2^nj slots (nj = item.ns),
+// JOINT: the JOINT kind: one table of 2^nj slots over the pairs (s, h) (nj = item.ns),
 // one lookup and one multiply-add per weight.
-template <int WARPS, int CHAINS, int NS, int NH, bool SHAPE_FROM_PARAMS, bool JOINT>
+// JOINT 2: the JOINT kind with 4-byte slot entries (F | rank << 8 | j << 20), any nj.
+template <int WARPS, int CHAINS, int NS, int NH, bool SHAPE_FROM_PARAMS, int JOINT>
 __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int kChains = CHAINS;
     // dynamic smem: [fraction rows, one copy per lane][s-table][rings], or for JOINT
@@ -106,7 +108,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
     const uint32_t ns = NS > 0 ? NS : it.ns, nh = NH > 0 ? NH : it.nh, P = ns + nh;
 
     if (JOINT) { // stage the joint table as it is
-        const uint32_t jb = 8u << ns;
+        const uint32_t jb = (JOINT == 2 ? 4u : 8u) << ns;
         uint4* jdst = reinterpret_cast<uint4*>(smem);
         for (uint32_t k = tid; k < jb / 16u; k += blockDim.x) jdst[k] = __ldg(it.tables + k);
     } else { // stage the tables: the s-table as it is, each fraction entry once per lane
@@ -130,7 +132,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
 
     const bool nib_stored = it.nib_mode == 0;
     const uint32_t raw_const = (it.nib_mode & 15u) * 0x11111111u;
-    const uint32_t rings = JOINT ? kJointRegion : kHRegion + s_region_bytes(ns); // a multiple of kRingBytes
+    const uint32_t rings = JOINT == 2 ? kJoint4Region : JOINT ? kJointRegion : kHRegion + s_region_bytes(ns); // a multiple of kRingBytes
     const uint32_t ring_off = rings + (warp * kChains) * kRingBytes;       // this warp's first word ring
     const uint32_t nring_off = rings + warps * kChains * kRingBytes + (warp * kChains) * kNibRingBytes;
     const uint32_t smem_base = smem_u32(smem);
@@ -164,7 +166,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
         nb = max(nb, (h.nc + 255u) >> 8);
     }
 
-    const uint32_t smask8 = ((1u << ns) - 1u) << 3, hmask7 = ((1u << nh) - 1u) << 7; // JOINT: smask8 masks the slot
+    const uint32_t smask8 = ((1u << ns) - 1u) << (JOINT == 2 ? 2 : 3), hmask7 = ((1u << nh) - 1u) << 7; // JOINT: smask8 masks the slot
     const uint32_t lt = lanemask_lt(), lane4 = lane << 2;
     const uint32_t mul2 = p.mul2, mul65536 = p.mul65536;
 
@@ -235,7 +237,17 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
             uint2 se[kChains];
             uint32_t fe[kChains], xn[kChains], m[kChains], w[kChains];
             bool need[kChains];
-            if (JOINT) { // the slot's entry: F and the word's (s, h) part in .x, the rank in .y
+            if (JOINT == 2) { // the slot's 4-byte entry: F, rank, and the word in the high half
+#pragma unroll
+                for (int k = 0; k < kChains; ++k)
+                    se[k].x = *reinterpret_cast<const uint32_t*>(smem + ((c[k].x << 2) & smask8));
+#pragma unroll
+                for (int k = 0; k < kChains; ++k) {
+                    xn[k] = (se[k].x & 0xFFu) * (c[k].x >> ns) + __byte_perm(se[k].x, 0u, 0x4441);
+                    need[k] = xn[k] < kStateL;
+                    fe[k] = 0;
+                }
+            } else if (JOINT) { // the slot's entry: F and the word's (s, h) part in .x, the rank in .y
 #pragma unroll
                 for (int k = 0; k < kChains; ++k)
                     se[k] = *reinterpret_cast<const uint2*>(smem + ((c[k].x << 3) & smask8));
@@ -290,7 +302,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
                 }
             }
         }
-        // the low nibbles of the pairs (FORMAT.md section 3: pair p at bits 4p and 16+4p)
+        // the low nibbles of the pairs (pair p of a block has its nibbles at bits 4p and 16+4p)
 #pragma unroll
         for (int k = 0; k < kChains; ++k)
 #pragma unroll
@@ -386,7 +398,8 @@ __global__ void __launch_bounds__(256) copy_kernel(const __grid_constant__ CopyP
     for (uint64_t k = nv * 16 + threadIdx.x; k < len; k += blockDim.x) dst[k] = src[k];
 }
 
-// FORMAT.md section 7: splitmix64 output for state v.
+// The per-tensor checksum: the sum of splitmix64 outputs mix64((i << 16) | w[i]); mix64 is
+// splitmix64's output for state v.
 __device__ __forceinline__ unsigned long long mix64(unsigned long long v) {
     unsigned long long z = v + 0x9E3779B97F4A7C15ull;
     z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
@@ -419,7 +432,7 @@ int max_dynamic_smem() {
     return v;
 }
 
-template <int WARPS, int CHAINS, int NS, int NH, bool SHAPE_FROM_PARAMS, bool JOINT>
+template <int WARPS, int CHAINS, int NS, int NH, bool SHAPE_FROM_PARAMS, int JOINT>
 static int launch_decode_shape(const DecodeParams& p, uint32_t smem_bytes, cudaStream_t s) {
     auto kernel = decode_kernel<WARPS, CHAINS, NS, NH, SHAPE_FROM_PARAMS, JOINT>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes));
@@ -429,7 +442,7 @@ static int launch_decode_shape(const DecodeParams& p, uint32_t smem_bytes, cudaS
     return cudaGetLastError();
 }
 
-template <int WARPS, int CHAINS, int NS, int NH, bool JOINT>
+template <int WARPS, int CHAINS, int NS, int NH, int JOINT>
 static int launch_decode_t(const DecodeParams& p, uint32_t smem_bytes, cudaStream_t s) {
     if (p.warps < 1 || p.warps > WARPS) return cudaErrorInvalidValue;
     return p.warps == WARPS ? launch_decode_shape<WARPS, CHAINS, NS, NH, false, JOINT>(p, smem_bytes, s)
@@ -440,10 +453,11 @@ int launch_decode(const DecodeParams& p, DecodeMode mode, uint32_t smem_bytes, v
     if (p.total_ctas == 0) return cudaSuccess;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (mode) {
-    case DecodeMode::Default: return launch_decode_t<kWarpsDefault, kChainsDefault, 11, 5, false>(p, smem_bytes, s);
-    case DecodeMode::Joint: return launch_decode_t<kWarpsJoint, kChainsJoint, 13, 5, true>(p, smem_bytes, s);
-    case DecodeMode::JointGeneric: return launch_decode_t<kWarpsGeneric, kChainsGeneric, 0, 5, true>(p, smem_bytes, s);
-    default: return launch_decode_t<kWarpsGeneric, kChainsGeneric, 0, 0, false>(p, smem_bytes, s);
+    case DecodeMode::Default: return launch_decode_t<kWarpsDefault, kChainsDefault, 11, 5, 0>(p, smem_bytes, s);
+    case DecodeMode::Joint: return launch_decode_t<kWarpsJoint, kChainsJoint, 13, 5, 1>(p, smem_bytes, s);
+    case DecodeMode::JointGeneric: return launch_decode_t<kWarpsGeneric, kChainsGeneric, 0, 5, 1>(p, smem_bytes, s);
+    case DecodeMode::JointCompact: return launch_decode_t<kWarpsJoint4, kChainsJoint4, 0, 5, 2>(p, smem_bytes, s);
+    default: return launch_decode_t<kWarpsGeneric, kChainsGeneric, 0, 0, 0>(p, smem_bytes, s);
     }
 }
 

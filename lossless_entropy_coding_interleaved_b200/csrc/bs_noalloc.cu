@@ -167,7 +167,7 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
     cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
     if (!b || !d_container || idx < 0) return BS_E_ARG;
     if (reinterpret_cast<uintptr_t>(d_container) & 15u) return BS_E_ARG;
-    // --- validate the header and this tensor in place (FORMAT.md sections 4-5) ---
+    // --- validate the header and this tensor in place (the container's validation rules) ---
     if (len < kHeaderBytes || std::memcmp(b, "BF16RANS", 8) != 0) return BS_E_FORMAT;
     if (rd32(b + 8) != kFormatVersion) return BS_E_VERSION;
     if (rd32(b + 12) != kHeaderBytes || rd32(b + 20) != kDirEntryBytes || rd64(b + 56) != 0) return BS_E_FORMAT;
@@ -228,7 +228,7 @@ extern "C" bs_status bs_decode_tensor_noalloc(const void* h_container_v, size_t 
     const uint8_t* m = b + model_off;
     const uint32_t n_present = joint ? 0 : rd16(m);
     uint32_t n_pairs = 0;
-    if (joint) { // FORMAT.md section 4.3b
+    if (joint) { // the JOINT model: n_pairs, reserved, then (j, Fj) with j ascending
         n_pairs = rd16(m);
         if (n_pairs < 1 || n_pairs > kJointPairs || rd16(m + 2) != 0 || model_bytes != 4 + 4ull * n_pairs)
             return BS_E_FORMAT;

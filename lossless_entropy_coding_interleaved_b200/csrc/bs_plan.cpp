@@ -1,7 +1,7 @@
 // bs_plan.cpp -- host side of libbs: container parsing and validation, decode-table
 // construction, and the C ABI of include/bs.h. The GPU work lives in bs_kernels.cu.
 //
-// The container is the one FORMAT.md specifies. This parser is written against that
+// The container is BF16RANS version 2. This parser is written against that
 // document. It shares no code with the oracle (oracle/bsoracle.c).
 #include <cuda_runtime.h>
 
@@ -82,7 +82,8 @@ struct Reader {
     }
 };
 
-// FORMAT.md sections 4-5. Fills `out` with every tensor, or returns the first error.
+// Byte layout and validation rules of the container. Fills `out` with every tensor, or returns
+// the first error.
 bs_status parse(Reader& rd, std::vector<Tensor>& out) {
     const uint64_t len = rd.len;
     uint8_t hdr[kHeaderBytes];
@@ -170,7 +171,7 @@ bs_status parse(Reader& rd, std::vector<Tensor>& out) {
         t.model.resize(t.model_bytes);
         if (!rd.read(t.model_offset, t.model_bytes, t.model.data())) return fail(BS_E_FORMAT);
         const uint8_t* m = t.model.data();
-        if (joint) { // FORMAT.md section 4.3b
+        if (joint) { // the JOINT model: n_pairs, reserved, then (j, Fj) with j ascending
             const uint32_t n_pairs = get_u16(m);
             if (n_pairs < 1 || n_pairs > kJointPairs || get_u16(m + 2) != 0) return BS_E_FORMAT;
             if (t.model_bytes != 4 + 4ull * n_pairs) return BS_E_FORMAT;
@@ -225,7 +226,13 @@ bs_status parse(Reader& rd, std::vector<Tensor>& out) {
             if (off % 16 || get_u32(e + 12) != 0 || !inside(off, bytes, len)) return BS_E_FORMAT;
             t.coded_bytes += bytes;
         }
-        t.table_bytes = joint ? joint_table_bytes(t.ns) : table_bytes_for(t.ns, t.nh, t.n_routes);
+        if (joint) {
+            uint32_t max_f = 0;
+            for (uint32_t i = 0; i < get_u16(t.model.data()); ++i) max_f = std::max<uint32_t>(max_f, get_u16(t.model.data() + 6 + 4 * i));
+            t.joint_compact = max_f <= kCompactMaxF;
+        }
+        t.table_bytes = !joint ? table_bytes_for(t.ns, t.nh, t.n_routes)
+                      : t.joint_compact ? joint4_table_bytes(t.ns) : joint_table_bytes(t.ns);
         out.push_back(std::move(t));
     }
     return BS_OK;
@@ -243,8 +250,12 @@ void build_tables(const Tensor& t, uint8_t* dst) {
         for (uint32_t i = 0; i < n_pairs; ++i) {
             const uint32_t j = get_u16(m + 4 + 4 * i), q = get_u16(m + 6 + 4 * i);
             for (uint32_t k = 0; k < q; ++k) {
-                jt[2 * (cum + k)] = q | ((j << 4) << 16);
-                jt[2 * (cum + k) + 1] = k;
+                if (t.joint_compact) { // F | rank << 8 | j << 20 (q <= 255, so k < 255)
+                    jt[cum + k] = q | (k << 8) | (j << 20);
+                } else {
+                    jt[2 * (cum + k)] = q | ((j << 4) << 16);
+                    jt[2 * (cum + k) + 1] = k;
+                }
             }
             cum += q;
         }
@@ -311,8 +322,9 @@ bs_status bs::build_workspace(std::vector<Tensor>& ts, std::vector<uint8_t>& ima
     uint64_t pos = kErrBlockBytes;
     for (Tensor& t : ts) {
         if (!is_coded(t.kind)) continue;
-        const uint32_t need = t.kind == BS_KIND_JOINT ? joint_smem_bytes(kWarpsJoint, kChainsJoint)
-                                                      : smem_bytes_for(t.ns, t.nh);
+        const uint32_t need = t.kind != BS_KIND_JOINT ? smem_bytes_for(t.ns, t.nh)
+                            : t.joint_compact ? joint4_smem_bytes(kWarpsJoint4, kChainsJoint4)
+                                              : joint_smem_bytes(kWarpsJoint, kChainsJoint);
         if (static_cast<int>(need) > smem_cap) return BS_E_UNSUPPORTED;
         t.ws_offset = pos;
         build_tables(t, image.data() + pos);
@@ -342,7 +354,7 @@ void bs::fill_tensor_info(const Tensor& t, bs_tensor_info* o) {
 }
 
 bs_status DecodeBatch::init() {
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < kDecodeModes; ++k) {
         bins_[k].p.reset(new (std::nothrow) DecodeParams);
         if (!bins_[k].p) return BS_E_NOMEM;
         bins_[k].mode = static_cast<DecodeMode>(k);
@@ -391,8 +403,9 @@ bs_status DecodeBatch::flush_bin(Bin& b, void* stream) {
     }
     p.total_ctas = static_cast<uint32_t>(ctas); // at most 2^31 / 8 + kMaxDecodeItems (see add)
     const bool joint = b.mode == DecodeMode::Joint || b.mode == DecodeMode::JointGeneric;
-    const uint32_t smem = joint ? joint_smem_bytes(p.warps, chains)
-                                                      : kHRegion + b.s_region + p.warps * chains * (kRingBytes + kNibRingBytes);
+    const uint32_t smem = b.mode == DecodeMode::JointCompact ? joint4_smem_bytes(p.warps, chains)
+                        : joint ? joint_smem_bytes(p.warps, chains)
+                                : kHRegion + b.s_region + p.warps * chains * (kRingBytes + kNibRingBytes);
     const int e = launch_decode(p, b.mode, smem, stream);
     p.n_items = 0;
     p.total_ctas = 0;
