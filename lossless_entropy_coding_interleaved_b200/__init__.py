@@ -11,7 +11,7 @@ The method is the one in the paragraph after the accounting table of the
   - the sign+exponent symbol is rANS-decoded with a per-tensor model;
   - that symbol selects the 7-bit fraction's distribution;
   - the fields are recombined bitwise.
-The byte layout is FORMAT.md.
+The byte layout is the BF16RANS container, version 2.
 """
 from __future__ import annotations
 
@@ -65,7 +65,7 @@ class _EncParams(ctypes.Structure):
 
 
 class FwInfo(ctypes.Structure):
-    """bs_fw_info: the header of a fixed-width lane layout (FORMAT.md section 10)."""
+    """bs_fw_info: the header of a fixed-width lane layout (4-bit codes, 7-bit fractions, exceptions)."""
     _fields_ = [("n_elems", ctypes.c_uint64), ("n_tiles", ctypes.c_uint64), ("n_exc", ctypes.c_uint64),
                 ("total_bytes", ctypes.c_uint64), ("table", ctypes.c_uint16 * 16)]
 
@@ -209,8 +209,8 @@ def _info_dict(ti: _Info) -> dict:
 
 def _container_names(h: np.ndarray) -> list:
     """Tensor names in directory order, read from a container that already passed
-    validation (FORMAT.md 4.1: n_tensors at 16, dir_offset at 24, names_offset at 32;
-    4.2: 144-byte entries with name_offset at 8 and name_bytes at 12)."""
+    validation (header: n_tensors at byte 16, dir_offset at 24, names_offset at 32; directory:
+    144-byte entries with name_offset at 8 and name_bytes at 12)."""
     hdr = h[:64].tobytes()
     nt = int.from_bytes(hdr[16:20], "little")
     d0, n0 = int.from_bytes(hdr[24:32], "little"), int.from_bytes(hdr[32:40], "little")
@@ -387,7 +387,7 @@ class Plan:
         return cpc.value, wave.value
 
     def to_fw(self, idx: int, scratch: torch.Tensor | None = None, stream=None):
-        """The fixed-width lane layout (FORMAT.md section 10) of BF16 tensor idx, built on the
+        """The fixed-width lane layout of BF16 tensor idx, built on the
         device from the container, as the runtime of the NVLC card derives its streams from
         the rANS files at start-up. The tensor is decoded (bs_decode_tensor) into `scratch`
         (or a temporary), checked (bs_check), then transcoded (bs_fw_measure, bs_fw_write).

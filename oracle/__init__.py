@@ -7,7 +7,7 @@ two share no code.
 What it computes: the method paragraph of the "Qwen3.8-27B-BF16-NVLC-Lossless" model
 card, which splits each BF16 word into sign, exponent and fraction, codes the
 sign+exponent symbol with a per-tensor rANS model, and lets that symbol select the
-fraction's distribution. The byte layout and every parameter come from FORMAT.md
+fraction's distribution. The byte layout and every parameter are those of the BF16RANS
 (version 2: the fraction's top three bits are coded, its low four bits kept verbatim).
 The arithmetic lives in ``bsoracle.c``. This module only marshals arguments through
 ctypes.
@@ -134,7 +134,7 @@ def encode(items, log2_chunk: int = 16, ns: int = 11, nh: int = 5, max_routes: i
     """items: sequence of (name, array, kind) with kind "bf16" (uint16 words, any shape)
     or "raw" (uint8 bytes). model "factored" codes BF16 tensors as kind RANS (ns, nh, routes),
     "joint" as kind JOINT (one table over (s, h) of precision nj). Returns the container
-    bytes (FORMAT.md section 4.6)."""
+    bytes (canonical layout: header, directory, names, then each tensor's sections)."""
     assert model in ("factored", "joint")
     keep = []
     arr_items = (_Item * max(1, len(items)))()
@@ -243,7 +243,7 @@ def _tables(Fs, route, Fh):
 
 
 def lane_encode(Fs, ns, route, Fh, nh, words):
-    """One lane (FORMAT.md sections 2-3): returns (start_state, words, tags). The low
+    """One lane of kind RANS: returns (start_state, words, tags). The low
     nibbles of ``words`` do not enter the state; the caller keeps them."""
     Fs, route, Fhb, nr = _tables(Fs, route, Fh)
     w = np.ascontiguousarray(words, dtype=np.uint16)
@@ -313,13 +313,14 @@ def mix64(v: int) -> int:
 
 
 def checksum(a: np.ndarray) -> int:
-    """FORMAT.md section 7 checksum of uint16 words or uint8 bytes."""
+    """The per-tensor checksum, sum of splitmix64 outputs over (i << 16) | w[i] (uint16 words) or
+    (i << 8) | b[i] (uint8 bytes), mod 2^64."""
     a = np.ascontiguousarray(a).reshape(-1)
     return int(lib().bso_checksum(_ptr(a), a.size, 2 if a.dtype == np.uint8 else 0))
 
 
 # ------------------------------------------------------------ fixed-width lane layout
-# FORMAT.md section 10; the arithmetic is in fworacle.c.
+# The fixed-width lane layout; the arithmetic is in fworacle.c.
 def fw_bytes(n_elems: int, n_exc: int) -> int:
     """Size of the FW layout of n_elems weights with n_exc escapes."""
     return int(lib().bso_fw_bytes(n_elems, n_exc))

@@ -1,6 +1,6 @@
 /*
  * bsoracle.c -- the oracle: a plain, slow, CPU-only encoder and decoder for the
- * BF16RANS container (FORMAT.md). It is TEST INFRASTRUCTURE. Only the tests, the
+ * BF16RANS container, version 2. It is TEST INFRASTRUCTURE. Only the tests, the
  * smoke check and the CPU-baseline leg of bench.py may load it. The GPU library
  * never calls it, and it shares no source with the GPU library.
  *
@@ -12,16 +12,19 @@
  *     table over the fraction's top three bits, with the low four bits verbatim);
  *   - the fields are recombined bitwise;
  *   - a residual stream keeps non-BF16 bytes verbatim (RAW kind here).
- * The card gives no byte layout, rANS parameters, interleaving or quantiser. Those
- * come from FORMAT.md (version 2), and each function says which section it follows.
+ * The card gives no byte layout, rANS parameters, interleaving or quantiser. Those are
+ * this project's container (BF16RANS version 2), and each function states the rule it
+ * follows: 32-bit states in [2^16, 2^32), 16-bit renormalisation words, 32 lanes per
+ * chunk under the octet map, words interleaved in (step, lane) order, the integer
+ * quantiser and route rule, and the byte layout.
  *
- * The JOINT kind (FORMAT.md sections 1-2, 4.3b) codes the pair (s, h) with one table
- * instead of the factored s-model and routes; model_t.joint selects it.
+ * The JOINT kind codes the pair (s, h) with one table of 2^nj slots instead of the
+ * factored s-model and routes; model_t.joint selects it.
  *
  * Pins (tests/test_oracle_*.py):
  *   - round trip on every 16-bit pattern;
  *   - brute force over tiny alphabets;
- *   - the hand-derived container in FORMAT.md section 8;
+ *   - hand-derived containers (the .hex files under tests/golden, each with its derivation);
  *   - Gibbs' inequality and a stated overhead bound against the empirical entropy;
  *   - closed forms of the quantiser.
  *
@@ -44,7 +47,7 @@ enum {
 };
 
 enum { KIND_RANS = 0, KIND_STORED = 1, KIND_RAW = 2, KIND_JOINT = 3 };
-#define JOINT_PAIRS 4096 /* (s << 3) | h, FORMAT.md section 1 */
+#define JOINT_PAIRS 4096 /* j = (s << 3) | h */
 
 /* RANS and JOINT tensors carry chunks of interleaved rANS lanes. */
 static int is_coded(uint32_t kind) { return kind == KIND_RANS || kind == KIND_JOINT; }
@@ -52,7 +55,7 @@ static int is_coded(uint32_t kind) { return kind == KIND_RANS || kind == KIND_JO
 #define LANES 32
 #define HEADER_BYTES 64
 #define DIR_ENTRY_BYTES 144
-#define STATE_L 65536u /* 2^16, FORMAT.md section 2 */
+#define STATE_L 65536u /* L = 2^16: the encoder's start state and the decoder's end state */
 #define FORMAT_VERSION 2
 
 /* ------------------------------------------------------------------ */
@@ -77,7 +80,7 @@ static void wr_u16(uint8_t* p, uint16_t v) { p[0] = (uint8_t)(v & 0xFF); p[1] = 
 static uint64_t align16(uint64_t v) { return (v + 15u) & ~(uint64_t)15u; }
 
 /* ------------------------------------------------------------------ */
-/* Checksum, FORMAT.md section 7: splitmix64 output for state v        */
+/* Checksum: sum of splitmix64 outputs; mix64 = the output for state v */
 /* ------------------------------------------------------------------ */
 uint64_t bso_mix64(uint64_t v) {
     uint64_t z = v + 0x9E3779B97F4A7C15ULL;
@@ -100,7 +103,7 @@ uint64_t bso_checksum(const void* data, uint64_t n, uint32_t kind) {
 }
 
 /* ------------------------------------------------------------------ */
-/* Quantiser, FORMAT.md section 6                                     */
+/* Quantiser: proportional with a floor of 1, fixed one unit at a time */
 /* ------------------------------------------------------------------ */
 /* Is a/b > c/d ?  (all non-negative; b, d > 0) */
 static int ratio_gt(uint64_t a, uint64_t b, uint64_t c, uint64_t d) {
@@ -145,7 +148,7 @@ int bso_quantise(const uint64_t* c, uint32_t K, uint32_t M, uint32_t* q) {
 
 
 /* ------------------------------------------------------------------ */
-/* Route choice, FORMAT.md section 6                                  */
+/* Route choice: Pearson statistic of the top fraction bits            */
 /* ------------------------------------------------------------------ */
 /* ceh: 256*8 counts of the fraction's top three bits, row e = exponent. Writes
  * route[256] and the ascending exponent list route_e[0..n_routes-1]. */
@@ -193,7 +196,7 @@ int bso_choose_routes(const uint64_t* ceh, uint32_t max_routes, uint8_t* route, 
 }
 
 /* ------------------------------------------------------------------ */
-/* Per-tensor model, FORMAT.md sections 1-2                           */
+/* Per-tensor model: s-model, routes and h tables, or the pair table    */
 /* ------------------------------------------------------------------ */
 typedef struct {
     uint32_t ns, nh, n_routes;
@@ -219,7 +222,7 @@ static void model_free(model_t* m) {
     m->j_of_slot = NULL;
 }
 
-/* FORMAT.md section 1, joint model: cumulative frequencies and the slot -> pair lookup */
+/* Joint model: cum(j) = Fj[0] + ... + Fj[j-1] and the slot -> pair lookup */
 static int joint_build(model_t* m) {
     uint32_t acc = 0;
     for (int j = 0; j < JOINT_PAIRS; j++) { m->cum_j[j] = acc; acc += m->Fj[j]; }
@@ -267,7 +270,7 @@ static int model_build_lookups(model_t* m) {
 }
 
 /* ------------------------------------------------------------------ */
-/* One lane, FORMAT.md sections 2-3                                   */
+/* One lane: encode backwards from L, at most one word per step       */
 /* ------------------------------------------------------------------ */
 /* Encode the lane's S weights (given in decode order) backwards from x = L. Only the
  * fields s and h go through the state; the nibbles are stored apart.
@@ -275,7 +278,7 @@ static int model_build_lookups(model_t* m) {
 static uint32_t lane_encode(const model_t* m, const uint16_t* w, uint32_t S, uint8_t* emitted, uint16_t* word) {
     uint32_t x = STATE_L;
     uint32_t P = m->ns + m->nh;
-    if (m->joint) { /* FORMAT.md section 2, the JOINT kind: Q = Fj[j] out of 2^nj */
+    if (m->joint) { /* the JOINT kind: Q = Fj[j] out of 2^nj */
         for (uint32_t tt = S; tt-- > 0;) {
             uint32_t j = w[tt] >> 4;
             uint64_t Q = m->Fj[j];
@@ -465,7 +468,7 @@ int bso_joint_lane_decode(const uint32_t* Fj, uint32_t nj, uint32_t state, const
 }
 
 /* ------------------------------------------------------------------ */
-/* Encoder of one BF16 tensor, FORMAT.md sections 3, 4.3-4.5, 6       */
+/* Encoder of one BF16 tensor: model, chunks, lanes, payloads          */
 /* ------------------------------------------------------------------ */
 typedef struct {
     uint8_t* model; /* serialized model, model_bytes long */
@@ -476,7 +479,7 @@ typedef struct {
     uint32_t* chunk_words;
     uint64_t coded_total; /* model + 16*n_chunks + sum chunk bytes */
     uint32_t n_routes;
-    uint32_t nib_mode; /* FORMAT.md section 3: 0 = stored, 0x10 + c = constant c */
+    uint32_t nib_mode; /* 0 = stored nibble words, 0x10 + c = every low nibble is c */
 } rans_blob_t;
 
 static void blob_free(rans_blob_t* b) {
@@ -489,10 +492,11 @@ static void blob_free(rans_blob_t* b) {
     memset(b, 0, sizeof(*b));
 }
 
-/* local weight index of (step t, lane j): FORMAT.md section 3 */
+/* local weight index of (step t, lane j) under the octet map: block t >> 3, lane j, weight t & 7 */
 static uint64_t octet_index(uint32_t t, uint32_t j) { return ((uint64_t)(t >> 3) << 8) + 8u * j + (t & 7u); }
 
-/* bit position of the nibble of step t inside its lane's block word: FORMAT.md section 3 */
+/* bit position of the nibble of step t inside its lane's block word: pair (t & 7) >> 1 at bit 4p,
+ * the odd step 16 bits higher */
 static uint32_t nibble_shift(uint32_t t) { return 4u * ((t & 7u) >> 1) + 16u * (t & 1u); }
 
 static int encode_rans(const uint16_t* w, uint64_t n, uint32_t log2_chunk, uint32_t ns, uint32_t nh,
@@ -513,7 +517,7 @@ static int encode_rans(const uint16_t* w, uint64_t n, uint32_t log2_chunk, uint3
         cj[w[i] >> 4]++;
     }
     uint16_t pad;
-    if (joint) { /* FORMAT.md section 6, joint model; section 3, its pad word */
+    if (joint) { /* Fj = quantise(pair counts, 2^nj); the pad pair has the largest Fj, lowest j on ties */
         m->joint = 1;
         m->nj = nj;
         if ((st = bso_quantise(cj, JOINT_PAIRS, 1u << nj, m->Fj))) goto done;
@@ -524,7 +528,7 @@ static int encode_rans(const uint16_t* w, uint64_t n, uint32_t log2_chunk, uint3
         pad = (uint16_t)(j_pad << 4);
         uint32_t n_pairs = 0;
         for (int j = 0; j < JOINT_PAIRS; j++) if (m->Fj[j]) n_pairs++;
-        out->model_bytes = 4 + 4ull * n_pairs; /* FORMAT.md section 4.3b */
+        out->model_bytes = 4 + 4ull * n_pairs; /* n_pairs, reserved, (j, Fj) pairs */
         out->model = (uint8_t*)calloc(1, out->model_bytes);
         if (!out->model) { st = BSO_E_NOMEM; goto done; }
         wr_u16(out->model, (uint16_t)n_pairs);
@@ -630,7 +634,7 @@ done:
 }
 
 /* ------------------------------------------------------------------ */
-/* Container writer, FORMAT.md section 4.6                            */
+/* Container writer: header, directory, names, then each tensor        */
 /* ------------------------------------------------------------------ */
 typedef struct {
     uint32_t kind;     /* 0: BF16 words (RANS or STORED chosen by the encoder); 2: RAW bytes */
@@ -671,7 +675,7 @@ int bso_encode(const bso_item* items, uint32_t n_items, const bso_params* p, uin
         if (it->kind == 2) { kinds[k] = KIND_RAW; continue; }
         if (it->n_elems > (1ull << 40)) { st = BSO_E_ARG; goto fail; }
         if (it->n_elems == 0) { kinds[k] = KIND_STORED; continue; }
-        if (p->joint) { /* FORMAT.md section 6: more distinct pairs than 2^nj slots -> STORED */
+        if (p->joint) { /* more distinct pairs than 2^nj slots: no JOINT table, so STORED */
             const uint16_t* w = (const uint16_t*)it->data;
             uint8_t* seen = (uint8_t*)calloc(JOINT_PAIRS, 1);
             uint32_t n_pairs = 0;
@@ -781,7 +785,7 @@ fail:
 void bso_free(void* p) { free(p); }
 
 /* ------------------------------------------------------------------ */
-/* Parser and validation, FORMAT.md sections 4-5                      */
+/* Parser and validation of the byte layout                           */
 /* ------------------------------------------------------------------ */
 typedef struct {
     uint32_t kind, ndim, log2_chunk, lanes, ns, nh, n_routes, name_offset, name_bytes, nib_mode;
@@ -852,7 +856,7 @@ static int parse_entry(const uint8_t* b, uint64_t len, uint32_t idx, bso_tensor_
     if (ti->n_chunks != (ti->n_elems + C - 1) / C || ti->data_bytes != 16 * ti->n_chunks) return BSO_E_FORMAT;
     if (ti->model_offset % 16 || !in_bounds(ti->model_offset, ti->model_bytes, len)) return BSO_E_FORMAT;
     const uint8_t* mm = b + ti->model_offset;
-    if (ti->kind == KIND_JOINT) { /* FORMAT.md section 4.3b */
+    if (ti->kind == KIND_JOINT) { /* n_pairs, reserved, then (j, Fj) with j ascending, sum 2^nj */
         if (ti->model_bytes < 8) return BSO_E_FORMAT;
         uint32_t n_pairs = rd_u16(mm);
         if (n_pairs < 1 || n_pairs > JOINT_PAIRS || rd_u16(mm + 2) != 0) return BSO_E_FORMAT;
@@ -945,7 +949,7 @@ static int load_model(const uint8_t* b, const bso_tensor_info* ti, model_t* m) {
 }
 
 /* ------------------------------------------------------------------ */
-/* Decoder, FORMAT.md sections 2-3                                    */
+/* Decoder: lanes in ascending order take the words, step by step     */
 /* ------------------------------------------------------------------ */
 /* Decode chunk c of a RANS tensor into out (its weights only). Returns BSO_E_CORRUPT
  * when the stream is inconsistent. Every loop is bounded by the chunk's weight count. */
@@ -971,7 +975,7 @@ static int decode_chunk(const uint8_t* b, const bso_tensor_info* ti, const model
     for (uint32_t t = 0; t < S; t++) {
         for (uint32_t j = 0; j < LANES; j++) { /* lanes in ascending order take words */
             uint32_t s, h;
-            if (m->joint) { /* FORMAT.md section 2, the JOINT kind */
+            if (m->joint) { /* the JOINT kind: x = Fj[j] * (x >> nj) + slot - cum(j) */
                 uint32_t slot = x[j] & ((1u << m->nj) - 1u);
                 uint32_t pj = m->j_of_slot[slot];
                 s = pj >> 3;
@@ -1038,7 +1042,7 @@ int bso_decode_chunks(const uint8_t* b, uint64_t len, uint32_t idx, uint64_t c0,
     return st;
 }
 
-/* Whole tensor, then the checksum of FORMAT.md section 7: a mismatch is BSO_E_CORRUPT
+/* Whole tensor, then the per-tensor checksum: a mismatch is BSO_E_CORRUPT
  * with *bad_chunk = -1 (no single chunk is to blame). */
 int bso_decode(const uint8_t* b, uint64_t len, uint32_t idx, void* out, uint64_t out_bytes, int64_t* bad_chunk) {
     bso_tensor_info ti;

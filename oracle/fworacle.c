@@ -1,5 +1,5 @@
 /*
- * fworacle.c -- the oracle for the fixed-width lane layout (FORMAT.md section 10): a plain, slow,
+ * fworacle.c -- the oracle for the fixed-width lane layout: a plain, slow,
  * CPU-only encoder and decoder. It is TEST INFRASTRUCTURE. Only the tests, the smoke
  * check and the CPU-baseline leg of bench.py may load it. The GPU library never calls it,
  * and it shares no source with the GPU library.
@@ -8,10 +8,12 @@
  * "Qwen3.8-27B-BF16-NVLC-Lossless" card says its GPU runtime derives from the rANS files at
  * initialisation (its Fixed7/Compact11 runtime; the runtime accounting table gives the
  * resident codes plus metadata at about 11.36 bits per weight). The card gives no layout,
- * so the one here is FORMAT.md section 10, and each function says which part it follows.
+ * so the one here is this project's, and each function states the part it follows: a
+ * 16-entry code table, planes A (4-bit codes), B (low nibbles) and C (top fraction bits) per
+ * 256-weight tile, and an exception list.
  *
  * Pins (tests/test_fw_oracle.py):
- *   - the two hand-derived layouts of sections 10.1 and 10.2;
+ *   - two hand-derived layouts (tests/golden/lane_*.hex);
  *   - a round trip on every 16-bit pattern;
  *   - the size formula checked against a count of escapes done in the test;
  *   - the code table checked against a sort done in the test;
@@ -56,7 +58,7 @@ static void put_le(uint8_t* p, uint32_t bytes, uint64_t v) {
 }
 
 /* A bit field of `width` bits starting at bit `bit` of a little-endian byte array
- * (bit b is bit b % 8 of byte b / 8). The u32 planes of section 10 are little-endian, so
+ * (bit b is bit b % 8 of byte b / 8). The layout's u32 planes are little-endian, so
  * bit k of lane j's word is bit 32j + k of the plane's bytes. */
 static void set_bits(uint8_t* base, uint64_t bit, uint32_t width, uint32_t value) {
     for (uint32_t b = 0; b < width; ++b)

@@ -1,4 +1,4 @@
-"""Pins of the fixed-width lane layout oracle (oracle/fworacle.c, FORMAT.md section 10).
+"""Pins of the fixed-width lane layout oracle (oracle/fworacle.c).
 
 What pins it (each independent of the oracle's own code):
 * the two layouts of sections 10.1 and 10.2, derived by hand (tests/golden/lane_*.hex);

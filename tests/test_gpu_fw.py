@@ -1,4 +1,4 @@
-"""GPU parity of the fixed-width lane layout (FORMAT.md section 10) through the C ABI.
+"""GPU parity of the fixed-width lane layout through the C ABI.
 
 * The device transcoder (bs_fw_measure + bs_fw_write) must produce the oracle's bytes
   exactly.

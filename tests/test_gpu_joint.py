@@ -1,4 +1,4 @@
-"""GPU parity of the JOINT kind (FORMAT.md sections 1-2, 4.3b) through the C ABI.
+"""GPU parity of the JOINT kind (one table over the pairs (s, h)) through the C ABI.
 
 * Containers the oracle encodes decode bit-exact on the device, against the originals and
   against the oracle's own decode: nj = 13 (the compile-time kernel instance) and 8..12

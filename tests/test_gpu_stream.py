@@ -143,7 +143,7 @@ def test_bad_arguments(model):
 
 
 def _chunk_offset(h: np.ndarray, tensor: int, chunk: int) -> int:
-    # FORMAT.md 4.1 (dir_offset at 24), 4.2 (data_offset at 48), 4.4 (16-byte chunk entries)
+    # header: dir_offset at byte 24; directory entry: data_offset at 48; 16-byte chunk entries
     dir_off = int(h[24:32].view(np.uint64)[0])
     e = dir_off + 144 * tensor
     data_off = int(h[e + 48:e + 56].view(np.uint64)[0])

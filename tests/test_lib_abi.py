@@ -65,7 +65,7 @@ def _golden(name):
 
 
 def test_library_parses_the_joint_golden_on_host():
-    # FORMAT.md section 8.3, derived by hand: the library's parser takes it, and the workspace
+    # the two-weight JOINT container derived by hand: the library's parser takes it, and the workspace
     # holds the error block and one JOINT table of 2^13 slots of 8 bytes
     import lossless_entropy_coding_interleaved_b200 as bs
     c = _golden("joint_two_weights.hex")

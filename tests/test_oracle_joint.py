@@ -1,8 +1,9 @@
-"""Pins of the oracle's JOINT kind (FORMAT.md sections 1-2, 4.3b, 8.3): one quantised table
+"""Pins of the oracle's JOINT kind: one quantised table
 over the pairs j = (s << 3) | h, decoded with one lookup per weight.
 
 What pins it:
-* the container of section 8.3, derived by hand (tests/golden/joint_two_weights.hex);
+* two containers derived by hand (tests/golden/joint_two_weights.hex and, for the word order,
+  tests/golden/joint_interleave_sixteen.hex);
 * every 16-bit pattern and a size sweep round-trip;
 * a closed form: pairs with power-of-two frequencies cost exactly log2(2^nj / F) bits each,
   so the word count is fixed up to the lanes' start and end states;

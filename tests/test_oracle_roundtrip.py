@@ -121,7 +121,7 @@ def _container():
 def test_fault_payload_bitflips_are_detected():
     # A flip that desynchronises a lane fails the end check (E_CORRUPT from the chunk).
     # A flip inside a near-uniform fraction can change one weight and stay in sync; the
-    # tensor checksum (FORMAT.md section 7) catches those. Flips in padding change nothing.
+    # per-tensor checksum catches those. Flips in padding change nothing.
     w, c = _container()
     ti = oracle.info(bytes(c), 0)
     first_chunk = int.from_bytes(c[ti["data_offset"]:ti["data_offset"] + 8], "little")

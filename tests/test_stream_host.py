@@ -25,7 +25,7 @@ def _u64(h, off):
 
 
 def _coded_range(h, k):
-    """[begin, end) of the bytes tensor k's decode reads, from the FORMAT.md directory and
+    """[begin, end) of the bytes tensor k's decode reads, from the container directory and
     chunk table: the chunk table or raw data, and every chunk's payload (section 4.5:
     128 bytes of states, 128 bytes of nibble words per 256-weight block when stored, the
     16-bit words, padded to 16 bytes)."""
