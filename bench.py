@@ -55,7 +55,7 @@ def _args():
     ap.add_argument("--cpu-threads", type=int, default=0, help="oracle threads (0: all host cores)")
     ap.add_argument("--batch", type=int, default=1, help="gemv mode: tokens per product (1..8)")
     ap.add_argument("--model", choices=["joint", "factored"], default="joint",
-                    help="rANS model of the container: joint (one table over (s, h), FORMAT.md kind JOINT; "
+                    help="rANS model of the container: joint (one table over (s, h), kind JOINT; "
                          "the default) or factored (s-model plus exponent routes, kind RANS)")
     ap.add_argument("--mode", choices=["model", "layerwise", "stream", "fw", "gemv"], default="model",
                     help="model: one bs_decode_batch of every tensor per step (the default line); "
@@ -87,20 +87,37 @@ def _peak_hbm():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def _traffic_per_weight(profile="decode_kernel_gemma2_9b.md", sources=("bs_kernels.cu", "bs_internal.h")):
-    """DRAM bytes per weight of a kernel from its committed ncu summary, if the kernel
-    sources still hash to what was profiled; else None."""
+# DRAM traffic per decoded weight of each timed kernel: dram__bytes_read.sum +
+# dram__bytes_write.sum of one ncu capture, over the weights that launch decoded. Each entry
+# keeps the hash of the kernel's sources at capture time (comments and blank lines removed);
+# the figure is reported only while the sources still hash to it, else traffic is null.
+_TRAFFIC = {
+    "decode_kernel": (("bs_kernels.cu", "bs_internal.h"), None, None),
+    "fw_decode_kernel": (("bs_fw.cu", "bs_fw.cuh"), None, None),
+}
+
+
+def _source_hash(files):
+    """sha256 prefix of the given csrc files with comments and blank lines removed."""
     import hashlib
+    import re
     csrc = os.path.join(ROOT, "lossless_entropy_coding_interleaved_b200", "csrc")
+    text = ""
+    for f in files:
+        src = open(os.path.join(csrc, f)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        text += "\n".join(l.rstrip() for l in src.splitlines() if l.strip()) + "\n"
+    return hashlib.sha256(text.encode()).hexdigest()[:16]
+
+
+def _traffic_per_weight(kernel="decode_kernel"):
+    """DRAM bytes per weight of a kernel from its capture, if its sources are unchanged; else None."""
+    files, want, tpw = _TRAFFIC[kernel]
     try:
-        src = b"".join(open(os.path.join(csrc, f), "rb").read() for f in sources)
-        lines = open(os.path.join(ROOT, "profiles", profile)).read().splitlines()
+        return tpw if want is not None and _source_hash(files) == want else None
     except OSError:
         return None
-    kv = dict(l.split(": ", 1) for l in lines if l.startswith(("kernel_sha256: ", "traffic_bytes_per_weight: ")))
-    if kv.get("kernel_sha256") != hashlib.sha256(src).hexdigest()[:16]:
-        return None
-    return float(kv["traffic_bytes_per_weight"])
 
 
 def _workload_desc(name, layers):
@@ -134,8 +151,13 @@ def _word_histograms(originals, specs, dev):
 
 # ------------------------------------------------------------------ oracle on host cores
 def _oracle_sample(workload, threads, model="joint"):
-    """The bounded CPU sample: layer 0 of the workload, generated and encoded on the host by
-    the oracle, then decoded by the oracle with `threads` threads over its chunks."""
+    """The bounded CPU sample: layer 0 of the workload (the whole of a one-tensor or one-layer
+    workload), generated and encoded on the host by the oracle, then decoded by the oracle in
+    chunk ranges (at most 16 chunks each) spread over `threads` host threads.
+
+    Returns (n, desc, run_once, check). run_once(pool, every=1) decodes every `every`-th
+    chunk range (every=1: the whole sample, including its STORED tensors) and returns
+    (seconds, weights decoded)."""
     import numpy as np
     import oracle
     import synthetic as S
@@ -146,29 +168,87 @@ def _oracle_sample(workload, threads, model="joint"):
     c = np.frombuffer(oracle.encode([(s.name, a, "bf16") for s, a in zip(specs, arrs)], model=model), np.uint8)
     infos = [oracle.info(c, k) for k in range(len(specs))]
     outs = [np.zeros(i["n_elems"], np.uint16) for i in infos]
+    coded = (oracle.KIND_RANS, oracle.KIND_JOINT)
+    # ranges of at most 16 chunks, fewer when the sample is small, so that every thread has work
+    total = sum(i["n_chunks"] for i in infos if i["kind"] in coded)
+    span = max(1, min(16, total // (4 * max(1, threads))))
     tasks = []
     for k, i in enumerate(infos):
-        if i["kind"] in (oracle.KIND_RANS, oracle.KIND_JOINT):
-            step = max(1, i["n_chunks"] // max(1, threads))
-            tasks += [(k, c0, min(c0 + step, i["n_chunks"])) for c0 in range(0, i["n_chunks"], step)]
+        if i["kind"] in coded:
+            tasks += [(k, c0, min(c0 + span, i["n_chunks"])) for c0 in range(0, i["n_chunks"], span)]
     n = sum(a.size for a in arrs)
-    desc = (f"oracle decode of layer 0 of {workload} ({len(specs)} tensors, {n} weights), "
-            f"{len(tasks)} chunk ranges over {threads} host threads")
+    desc = (f"oracle decode of layer 0 of {workload} ({len(specs)} tensors, {n} weights) in {len(tasks)} "
+            f"chunk ranges of at most {span} chunks")
 
-    def run_once(pool):
+    def weights(k, c0, c1):
+        C = 1 << infos[k]["log2_chunk"]
+        return min(c1 * C, infos[k]["n_elems"]) - c0 * C
+
+    def run_once(pool, every=1):
+        sub = tasks[::every]
         t0 = time.perf_counter()
-        futs = [pool.submit(oracle.decode_chunks, c, k, c0, c1, outs[k]) for k, c0, c1 in tasks]
-        for k, i in enumerate(infos):
-            if i["kind"] not in (oracle.KIND_RANS, oracle.KIND_JOINT):
-                outs[k][:] = oracle.decode(c, k).reshape(-1)
+        futs = [pool.submit(oracle.decode_chunks, c, k, c0, c1, outs[k]) for k, c0, c1 in sub]
+        if every == 1:
+            for k, i in enumerate(infos):
+                if i["kind"] not in coded:
+                    outs[k][:] = oracle.decode(c, k).reshape(-1)
         assert all(f.result() == 0 for f in futs)
-        return time.perf_counter() - t0
+        sec = time.perf_counter() - t0
+        return sec, (n if every == 1 else sum(weights(*t) for t in sub))
 
     def check():
         for a, o in zip(arrs, outs):
             assert np.array_equal(a.reshape(-1), o), "oracle sample decode mismatch"
 
     return n, desc, run_once, check
+
+
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+CPU_PASSES = 5
+CPU_WORKLOADS = ("tensor_1m", "gemma2_layer", "gemma2_9b")
+
+
+def _cpu_baseline(workload, threads, model, passes=CPU_PASSES):
+    """The oracle on the host cores: for each of the three dense workloads' samples (layer 0
+    of the checkpoint), the median of `passes` timed decodes on `threads` threads and on one
+    thread (one thread decodes every 8th chunk range of the larger samples, which bounds its
+    time). The headline value is the all-core figure on `workload`'s sample."""
+    per = {}
+    head = None
+    for wl in dict.fromkeys(CPU_WORKLOADS + (workload,)):
+        if wl not in ("tensor_1m", "gemma2_layer", "gemma2_9b", "qwen_27b_scale"):
+            continue
+        n, desc, run_once, check = _oracle_sample(wl, threads, model)
+        every1 = 1 if n <= (1 << 22) else 8
+        with cf.ThreadPoolExecutor(threads) as pool:
+            run_once(pool)
+            check()
+            allc = [run_once(pool) for _ in range(passes)]
+        with cf.ThreadPoolExecutor(1) as one:
+            run_once(one, every1)
+            single = [run_once(one, every1) for _ in range(passes)]
+        gbs = lambda runs: 2 * statistics.median(w / sec for sec, w in runs) / 1e9
+        per[wl] = {"all_cores_gbs": round(gbs(allc), 3), "single_thread_gbs": round(gbs(single), 3),
+                   "weights": n, "single_thread_share": f"1/{every1} of the chunk ranges"}
+        if wl == workload:
+            head = (gbs(allc), desc)
+    if head is None:
+        return None
+    return {"value": round(head[0], 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": head[1] + f"; median of {passes} passes over {threads} host threads",
+            "single_thread": per[workload]["single_thread_gbs"], "cpu_model": _cpu_model(),
+            "nproc": os.cpu_count(), "passes": passes, "stat": "median", "per_workload": per}
 
 
 def _cpu_threads(req):
@@ -256,16 +336,19 @@ def run_reference(a):
         for _ in range(a.warmup):
             run_once(pool)
         check()
-        ts = [run_once(pool) for _ in range(a.steps)]
-    sec = sum(ts)
-    value = 2 * n * a.steps / sec / 1e9
+        ts = [run_once(pool)[0] for _ in range(a.steps)]
+    # the median step, as the GPU arm's cpu_baseline leg reports it
+    med = statistics.median(ts)
+    value = 2 * n / med / 1e9
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": a.gpus,
-            "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(1e3 * sec / a.steps, 3),
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(1e3 * med, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32",
             "data": "synthetic", "config": {"workload": a.workload, "description": desc, "n_weights": n_all,
-                                            "step": "one bounded sample per step: " + sample},
+                                            "step": "one bounded sample per step: " + sample,
+                                            "stat": "median step time"},
             "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample + f"; median of {a.steps} passes over {threads} host threads",
+                             "cpu_model": _cpu_model(), "nproc": os.cpu_count()},
             "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -466,14 +549,7 @@ def run_ours(a):
 
     cpu = None
     if rank == 0 and not a.no_cpu_baseline:
-        threads = _cpu_threads(a.cpu_threads)
-        n_s, sample, run_once, check = _oracle_sample(a.workload, threads, a.model)
-        with cf.ThreadPoolExecutor(threads) as pool:
-            run_once(pool)
-            check()
-            sec = run_once(pool)
-        cpu = {"value": round(2 * n_s / sec / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
-               "sample": sample}
+        cpu = _cpu_baseline(a.workload, _cpu_threads(a.cpu_threads), a.model)
 
     ranks.close()
     if rank != 0:
@@ -501,12 +577,12 @@ def run_ours(a):
                                f"{max(1, a.batch_streams)} stream(s) in turn"),
                    "words": "BF16 bit patterns; rANS state arithmetic in u32",
                    "model": ("joint: one rANS table over (sign+exponent, top 3 fraction bits), nj = 13 "
-                             "(FORMAT.md kind JOINT)" if a.model == "joint" else
-                             "factored: s-model (ns = 11) and exponent routes (nh = 5) (FORMAT.md kind RANS)")},
+                             "(kind JOINT)" if a.model == "joint" else
+                             "factored: s-model (ns = 11) and exponent routes (nh = 5) (kind RANS)")},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": (None if tpw is None else int(tpw * bf16_n)),
-                     "traffic_source": "profiles/decode_kernel_gemma2_9b.md (8-layer capture, scaled by weights)",
+                     "traffic_source": "ncu capture of this kernel on the first 8 layers, scaled by weights",
                      "kernel": "decode_kernel", "per_launch_bytes": int(coded + out_bytes),
                      "launch_ms_mean": round(mean_step, 4)},
         "e2e": e2e,
@@ -531,7 +607,7 @@ def _groups(names):
 def _group_ranges(h: "np.ndarray", names):
     """Per layer group, the contiguous container bytes its tensors use and its member indices.
 
-    FORMAT.md 4.2 and 4.6: the canonical layout writes each tensor's sections (RANS: model,
+    The canonical layout writes each tensor's sections (RANS: model,
     chunk table, chunks; else the data) in directory order, each tensor starting at its
     model_offset (RANS) or data_offset. A group's tensors are consecutive, so its bytes run
     from its first tensor's start to the next group's start (or the end of the container)."""
@@ -936,7 +1012,7 @@ def run_fw(a):
     value = world * a.steps * out_bytes / (total_ms * 1e-3) / 1e9
     peak, peak_kind = _peak_hbm()
     achieved = (fw_bytes + out_bytes) / (mean_step * 1e-3) / 1e9
-    tpw = _traffic_per_weight("fw_decode_kernel_gemma2_9b.md", ("bs_fw.cu", "bs_fw.cuh"))
+    tpw = _traffic_per_weight("fw_decode_kernel")
 
     # end to end: every layout copied in from pinned host memory and every output copied back,
     # per layer group on three streams so that the copies of one group overlap the others
@@ -1014,7 +1090,7 @@ def run_fw(a):
         "scaling": "weak", "vs_baseline": None, "dtype": "u32",
         "data": "synthetic (seeded device draws, synthetic/ recipe)",
         "config": {"workload": a.workload, "description": desc, "n_weights": n, "tensors": len(specs),
-                   "layout": "fixed-width lane layout (FORMAT.md section 10)",
+                   "layout": "fixed-width lane layout: 4-bit sign+exponent codes, the 7-bit fraction, exceptions",
                    "fw_bytes": int(fw_bytes), "decoded_bytes": int(out_bytes), "escapes": int(n_exc),
                    "bits_per_weight": round(8 * fw_bytes / n, 5), "transcode_s": round(t_transcode, 3),
                    "parallelism": f"replicas x{world} (no collective on the data path)",
@@ -1023,7 +1099,7 @@ def run_fw(a):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": (None if tpw is None else int(tpw * n)),
-                     "traffic_source": "profiles/fw_decode_kernel_gemma2_9b.md (capture scaled by weights)",
+                     "traffic_source": "ncu capture of this kernel, scaled by weights",
                      "kernel": "fw_decode_kernel", "per_launch_bytes": int(fw_bytes + out_bytes),
                      "launch_ms_mean": round(mean_step, 4)},
         "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": int(launches), "clocks": clk}), flush=True)
