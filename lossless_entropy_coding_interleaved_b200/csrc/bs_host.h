@@ -13,8 +13,34 @@ namespace bs {
 
 inline uint64_t up256(uint64_t v) { return (v + 255) & ~uint64_t(255); }
 
-// Parse and validate a container held in host memory (byte layout and validation rules of
-// the BF16RANS container, version 2).
+// ---- Validation (bs_validate.cpp): one copy of each rule for every host path ----
+struct HeaderInfo {
+    uint32_t n_tensors = 0;
+    uint64_t dir = 0, names = 0, names_bytes = 0;
+};
+// The 64-byte header of a container of len bytes: magic, version, sizes, reserved field,
+// 16-byte aligned directory and names inside the container. BS_E_SIZE if total_bytes != len.
+bs_status check_header(const uint8_t* hdr, uint64_t len, HeaderInfo* h);
+// One 144-byte directory entry: fills t's directory fields and the name's place in the names
+// section, and checks every field that needs no other section (kind, shape, chunking,
+// precisions, section bounds and alignment).
+bs_status check_entry(const uint8_t* d, uint64_t len, const HeaderInfo& h, Tensor* t, uint32_t* name_off,
+                      uint32_t* name_len);
+// The model section (t->model_bytes bytes at m) of a coded entry that passed check_entry:
+// ascending symbols or pairs, nonzero frequencies, table sums, routes. Sets t->table_bytes
+// and, for JOINT, t->joint_compact.
+bs_status check_model(const uint8_t* m, Tensor* t);
+// The chunk table (16 * n_chunks bytes at ct): aligned payloads inside the container, zero
+// reserved words. Sets t->coded_bytes.
+bs_status check_chunk_table(const uint8_t* ct, uint64_t len, Tensor* t);
+// Expand the model (at m) of a coded tensor that passed check_model into its decode tables,
+// t.table_bytes bytes at dst.
+void build_tables(const Tensor& t, const uint8_t* m, uint8_t* dst);
+// Dynamic shared memory of a decode launch of this mode and shape (s_region: the largest
+// s-table region of a factored launch).
+uint32_t decode_smem_bytes(DecodeMode mode, uint32_t warps, uint32_t chains, uint32_t s_region);
+
+// Parse and validate a container held in host memory.
 bs_status parse_host_container(const uint8_t* h, uint64_t len, std::vector<Tensor>& out);
 
 // Bytes of the decode workspace: the error block, then each RANS tensor's tables.

@@ -39,23 +39,7 @@ namespace {
 
 bs_status cuda_fail(cudaError_t e) { return cuda_status(static_cast<int>(e)); }
 
-uint64_t get_u64(const uint8_t* p) {
-    uint64_t v;
-    std::memcpy(&v, p, 8);
-    return v;
-}
-uint32_t get_u32(const uint8_t* p) {
-    uint32_t v;
-    std::memcpy(&v, p, 4);
-    return v;
-}
-uint16_t get_u16(const uint8_t* p) {
-    uint16_t v;
-    std::memcpy(&v, p, 2);
-    return v;
-}
 bool inside(uint64_t off, uint64_t bytes, uint64_t len) { return off <= len && bytes <= len - off; }
-uint64_t up16(uint64_t v) { return (v + 15) & ~uint64_t(15); }
 
 // Reads container bytes from a host copy or, without one, from device memory.
 struct Reader {
@@ -82,212 +66,48 @@ struct Reader {
     }
 };
 
-// Byte layout and validation rules of the container. Fills `out` with every tensor, or returns
-// the first error.
+// Reads and validates the whole container (the rules are in bs_validate.cpp). Fills `out`
+// with every tensor, or returns the first error.
 bs_status parse(Reader& rd, std::vector<Tensor>& out) {
     const uint64_t len = rd.len;
     uint8_t hdr[kHeaderBytes];
     auto fail = [&](bs_status st) { return rd.cuda_error ? BS_E_CUDA : st; };
     if (len < kHeaderBytes || !rd.read(0, kHeaderBytes, hdr)) return fail(BS_E_FORMAT);
-    const uint8_t* b = hdr;
-    if (std::memcmp(b, "BF16RANS", 8) != 0) return BS_E_FORMAT;
-    if (get_u32(b + 8) != kFormatVersion) return BS_E_VERSION;
-    if (get_u32(b + 12) != kHeaderBytes || get_u32(b + 20) != kDirEntryBytes || get_u64(b + 56) != 0)
-        return BS_E_FORMAT;
-    if (get_u64(b + 48) != len) return BS_E_SIZE;
-    const uint32_t nt = get_u32(b + 16);
-    const uint64_t dir = get_u64(b + 24), names = get_u64(b + 32), names_bytes = get_u64(b + 40);
-    if (dir % 16 || names % 16) return BS_E_FORMAT;
-    if (!inside(dir, uint64_t(kDirEntryBytes) * nt, len) || !inside(names, names_bytes, len)) return BS_E_FORMAT;
+    HeaderInfo h;
+    bs_status st = check_header(hdr, len, &h);
+    if (st != BS_OK) return st;
     std::vector<uint8_t> dbuf, nbuf, tbuf;
     try {
-        dbuf.resize(uint64_t(kDirEntryBytes) * nt);
-        nbuf.resize(names_bytes);
+        dbuf.resize(uint64_t(kDirEntryBytes) * h.n_tensors);
+        nbuf.resize(h.names_bytes);
     } catch (...) {
         return BS_E_NOMEM;
     }
-    if (!rd.read(dir, dbuf.size(), dbuf.data()) || !rd.read(names, names_bytes, nbuf.data())) return fail(BS_E_FORMAT);
+    if (!rd.read(h.dir, dbuf.size(), dbuf.data()) || !rd.read(h.names, h.names_bytes, nbuf.data()))
+        return fail(BS_E_FORMAT);
     out.clear();
-    out.reserve(nt);
-    for (uint32_t k = 0; k < nt; ++k) {
-        const uint8_t* d = dbuf.data() + uint64_t(kDirEntryBytes) * k;
+    out.reserve(h.n_tensors);
+    for (uint32_t k = 0; k < h.n_tensors; ++k) {
         Tensor t;
-        t.kind = d[0];
-        t.ndim = d[1];
-        t.log2_chunk = d[2];
-        t.lanes = d[3];
-        t.ns = d[4];
-        t.nh = d[5];
-        t.n_routes = d[6];
-        t.nib_mode = d[7];
-        if (get_u64(d + 72) != 0) return BS_E_FORMAT;
-        const uint32_t name_off = get_u32(d + 8), name_len = get_u32(d + 12);
-        t.n_elems = get_u64(d + 16);
-        t.n_chunks = get_u64(d + 24);
-        t.model_offset = get_u64(d + 32);
-        t.model_bytes = get_u64(d + 40);
-        t.data_offset = get_u64(d + 48);
-        t.data_bytes = get_u64(d + 56);
-        t.checksum = get_u64(d + 64);
-        for (int i = 0; i < 8; ++i) t.shape[i] = get_u64(d + 80 + 8 * i);
-        if (t.kind > BS_KIND_JOINT || t.ndim > 8) return BS_E_FORMAT;
-        if (!is_coded(t.kind) && t.nib_mode != 0) return BS_E_FORMAT;
-        if (uint64_t(name_off) + name_len > names_bytes) return BS_E_FORMAT;
+        uint32_t name_off = 0, name_len = 0;
+        st = check_entry(dbuf.data() + uint64_t(kDirEntryBytes) * k, len, h, &t, &name_off, &name_len);
+        if (st != BS_OK) return st;
         t.name.assign(reinterpret_cast<const char*>(nbuf.data() + name_off), name_len);
-        unsigned __int128 prod = 1;
-        for (uint32_t i = 0; i < t.ndim; ++i) {
-            prod *= t.shape[i];
-            if (prod > (static_cast<unsigned __int128>(1) << 64)) return BS_E_FORMAT;
-        }
-        for (uint32_t i = t.ndim; i < 8; ++i)
-            if (t.shape[i] != 0) return BS_E_FORMAT;
-        if (prod != t.n_elems) return BS_E_FORMAT;
-        if (t.data_offset % 16 || !inside(t.data_offset, t.data_bytes, len)) return BS_E_FORMAT;
-        if (!is_coded(t.kind)) {
-            if (t.kind == BS_KIND_STORED && t.n_elems > (1ull << 62)) return BS_E_FORMAT;
-            const uint64_t want = t.kind == BS_KIND_STORED ? 2 * t.n_elems : t.n_elems;
-            if (t.data_bytes != want) return BS_E_FORMAT;
-            t.coded_bytes = want;
-            out.push_back(std::move(t));
-            continue;
-        }
-        // RANS and JOINT
-        const bool joint = t.kind == BS_KIND_JOINT;
-        if (t.lanes != kLanes || t.log2_chunk < 8 || t.log2_chunk > 24) return BS_E_FORMAT;
-        if (joint) {
-            if (t.ns < kMinNj || t.ns > kMaxNj || t.nh != 0 || t.n_routes != 0) return BS_E_FORMAT;
-        } else if (t.ns < 1 || t.ns > kMaxNs || t.nh < kMinNh || t.nh > kMaxNh || t.ns + t.nh > kMaxPrecision ||
-                   t.n_routes > kMaxRoutes) {
-            return BS_E_FORMAT;
-        }
-        if (t.nib_mode != 0 && (t.nib_mode & 0xF0u) != 0x10u) return BS_E_FORMAT;
-        if (t.n_elems == 0 || t.n_elems > (1ull << 40)) return BS_E_FORMAT;
-        const uint64_t C = 1ull << t.log2_chunk;
-        if (t.n_chunks != (t.n_elems + C - 1) / C || t.data_bytes != 16 * t.n_chunks) return BS_E_FORMAT;
-        const uint64_t model_min = joint ? 8 : 264, model_max = joint ? 4 + 4 * kJointPairs : 260 + 4 * 512 + 16 * kMaxRoutes;
-        if (t.model_offset % 16 || !inside(t.model_offset, t.model_bytes, len) || t.model_bytes < model_min ||
-            t.model_bytes > model_max)
-            return BS_E_FORMAT;
-        t.model.resize(t.model_bytes);
-        if (!rd.read(t.model_offset, t.model_bytes, t.model.data())) return fail(BS_E_FORMAT);
-        const uint8_t* m = t.model.data();
-        if (joint) { // the JOINT model: n_pairs, reserved, then (j, Fj) with j ascending
-            const uint32_t n_pairs = get_u16(m);
-            if (n_pairs < 1 || n_pairs > kJointPairs || get_u16(m + 2) != 0) return BS_E_FORMAT;
-            if (t.model_bytes != 4 + 4ull * n_pairs) return BS_E_FORMAT;
-            uint64_t sumj = 0;
-            int prevj = -1;
-            for (uint32_t i = 0; i < n_pairs; ++i) {
-                const int j = get_u16(m + 4 + 4 * i);
-                const uint32_t q = get_u16(m + 6 + 4 * i);
-                if (j <= prevj || j >= static_cast<int>(kJointPairs) || q == 0) return BS_E_FORMAT;
-                prevj = j;
-                sumj += q;
+        if (is_coded(t.kind)) {
+            try {
+                t.model.resize(t.model_bytes);
+                tbuf.resize(t.data_bytes);
+            } catch (...) {
+                return BS_E_NOMEM;
             }
-            if (sumj != (1ull << t.ns)) return BS_E_FORMAT;
+            if (!rd.read(t.model_offset, t.model_bytes, t.model.data())) return fail(BS_E_FORMAT);
+            if ((st = check_model(t.model.data(), &t)) != BS_OK) return st;
+            if (!rd.read(t.data_offset, t.data_bytes, tbuf.data())) return fail(BS_E_FORMAT);
+            if ((st = check_chunk_table(tbuf.data(), len, &t)) != BS_OK) return st;
         }
-        const uint32_t n_present = joint ? 0 : get_u16(m);
-        if (!joint) {
-        if (n_present < 1 || n_present > 512) return BS_E_FORMAT;
-        if (t.model_bytes != 260 + 4ull * n_present + 16ull * t.n_routes) return BS_E_FORMAT;
-        uint64_t sum = 0;
-        int prev = -1;
-        for (uint32_t i = 0; i < n_present; ++i) {
-            const int s = get_u16(m + 4 + 4 * i);
-            const uint32_t q = get_u16(m + 6 + 4 * i);
-            if (s <= prev || s > 511 || q == 0) return BS_E_FORMAT;
-            prev = s;
-            sum += q;
-        }
-        if (sum != (1ull << t.ns)) return BS_E_FORMAT;
-        const uint8_t* route = m + 4 + 4 * n_present;
-        for (int e = 0; e < 256; ++e)
-            if (route[e] != 0xFF && route[e] >= t.n_routes) return BS_E_FORMAT;
-        for (uint32_t r = 0; r < t.n_routes; ++r) {
-            sum = 0;
-            for (int h = 0; h < 8; ++h) sum += get_u16(route + 256 + 16 * r + 2 * h);
-            if (sum != (1ull << t.nh)) return BS_E_FORMAT;
-        }
-        }
-        (void)n_present;
-        try {
-            tbuf.resize(t.data_bytes);
-        } catch (...) {
-            return BS_E_NOMEM;
-        }
-        if (!rd.read(t.data_offset, t.data_bytes, tbuf.data())) return fail(BS_E_FORMAT);
-        t.coded_bytes = t.model_bytes + t.data_bytes;
-        for (uint64_t c = 0; c < t.n_chunks; ++c) {
-            const uint8_t* e = tbuf.data() + 16 * c;
-            const uint64_t off = get_u64(e);
-            const uint32_t nw = get_u32(e + 8);
-            const uint64_t nc = std::min<uint64_t>(C, t.n_elems - c * C);
-            const uint64_t bytes = payload_bytes(nc, nw, t.nib_mode == 0);
-            if (off % 16 || get_u32(e + 12) != 0 || !inside(off, bytes, len)) return BS_E_FORMAT;
-            t.coded_bytes += bytes;
-        }
-        if (joint) {
-            uint32_t max_f = 0;
-            for (uint32_t i = 0; i < get_u16(t.model.data()); ++i) max_f = std::max<uint32_t>(max_f, get_u16(t.model.data() + 6 + 4 * i));
-            t.joint_compact = max_f <= kCompactMaxF;
-        }
-        t.table_bytes = !joint ? table_bytes_for(t.ns, t.nh, t.n_routes)
-                      : t.joint_compact ? joint4_table_bytes(t.ns) : joint_table_bytes(t.ns);
         out.push_back(std::move(t));
     }
     return BS_OK;
-}
-
-// Expand one tensor's model into the decode tables (layout in bs_internal.h): the s-table,
-// then the compact fraction rows with the UNIFORM row last. For JOINT, one entry per slot:
-// .x = F | ((j << 4) << 16), .y = the slot's rank k within its pair.
-void build_tables(const Tensor& t, uint8_t* dst) {
-    const uint8_t* m = t.model.data();
-    if (t.kind == BS_KIND_JOINT) {
-        const uint32_t n_pairs = get_u16(m);
-        uint32_t* jt = reinterpret_cast<uint32_t*>(dst);
-        uint32_t cum = 0;
-        for (uint32_t i = 0; i < n_pairs; ++i) {
-            const uint32_t j = get_u16(m + 4 + 4 * i), q = get_u16(m + 6 + 4 * i);
-            for (uint32_t k = 0; k < q; ++k) {
-                if (t.joint_compact) { // F | rank << 8 | j << 20 (q <= 255, so k < 255)
-                    jt[cum + k] = q | (k << 8) | (j << 20);
-                } else {
-                    jt[2 * (cum + k)] = q | ((j << 4) << 16);
-                    jt[2 * (cum + k) + 1] = k;
-                }
-            }
-            cum += q;
-        }
-        return;
-    }
-    const uint32_t n_present = get_u16(m);
-    const uint8_t* route = m + 4 + 4 * n_present;
-    const uint32_t Mh = 1u << t.nh;
-    auto frow = [&](uint32_t s) -> uint32_t {
-        const uint8_t r = route[s & 0xFF];
-        return frow_field(r == 0xFF ? t.n_routes : r, t.nh);
-    };
-    uint32_t* st = reinterpret_cast<uint32_t*>(dst);
-    uint32_t cum = 0;
-    for (uint32_t i = 0; i < n_present; ++i) {
-        const uint32_t s = get_u16(m + 4 + 4 * i), q = get_u16(m + 6 + 4 * i);
-        for (uint32_t k = 0; k < q; ++k) {
-            st[2 * (cum + k)] = q | (k << 16);
-            st[2 * (cum + k) + 1] = (s << 7) | (frow(s) << 16);
-        }
-        cum += q;
-    }
-    uint32_t* ht = reinterpret_cast<uint32_t*>(dst + (8u << t.ns));
-    for (uint32_t r = 0; r <= t.n_routes; ++r) {
-        uint32_t* row = ht + r * Mh;
-        cum = 0;
-        for (uint32_t h = 0; h < 8; ++h) {
-            const uint32_t q = (r == t.n_routes) ? Mh / 8 : get_u16(route + 256 + 16 * r + 2 * h);
-            for (uint32_t k = 0; k < q; ++k) row[cum + k] = h_entry(h, q, k);
-            cum += q;
-        }
-    }
 }
 
 } // namespace
@@ -322,12 +142,11 @@ bs_status bs::build_workspace(std::vector<Tensor>& ts, std::vector<uint8_t>& ima
     uint64_t pos = kErrBlockBytes;
     for (Tensor& t : ts) {
         if (!is_coded(t.kind)) continue;
-        const uint32_t need = t.kind != BS_KIND_JOINT ? smem_bytes_for(t.ns, t.nh)
-                            : t.joint_compact ? joint4_smem_bytes(kWarpsJoint4, kChainsJoint4)
-                                              : joint_smem_bytes(kWarpsJoint, kChainsJoint);
+        const DecodeMode mode = decode_mode_of(t);
+        const uint32_t need = decode_smem_bytes(mode, max_warps_of(mode), chains_of(mode), s_region_bytes(t.ns));
         if (static_cast<int>(need) > smem_cap) return BS_E_UNSUPPORTED;
         t.ws_offset = pos;
-        build_tables(t, image.data() + pos);
+        build_tables(t, t.model.data(), image.data() + pos);
         pos += up256(t.table_bytes);
     }
     std::memset(image.data() + 8, 0xFF, 8); // error block: flags = 0, first_bad = all ones
@@ -402,10 +221,7 @@ bs_status DecodeBatch::flush_bin(Bin& b, void* stream) {
         ctas += (n_chunks + per_cta - 1) / per_cta;
     }
     p.total_ctas = static_cast<uint32_t>(ctas); // at most 2^31 / 8 + kMaxDecodeItems (see add)
-    const bool joint = b.mode == DecodeMode::Joint || b.mode == DecodeMode::JointGeneric;
-    const uint32_t smem = b.mode == DecodeMode::JointCompact ? joint4_smem_bytes(p.warps, chains)
-                        : joint ? joint_smem_bytes(p.warps, chains)
-                                : kHRegion + b.s_region + p.warps * chains * (kRingBytes + kNibRingBytes);
+    const uint32_t smem = decode_smem_bytes(b.mode, p.warps, chains, b.s_region);
     const int e = launch_decode(p, b.mode, smem, stream);
     p.n_items = 0;
     p.total_ctas = 0;

@@ -875,7 +875,7 @@ static int parse_entry(const uint8_t* b, uint64_t len, uint32_t idx, bso_tensor_
     }
     if (ti->model_bytes < 264) return BSO_E_FORMAT;
     uint32_t n_present = rd_u16(mm);
-    if (n_present < 1 || n_present > 512) return BSO_E_FORMAT;
+    if (n_present < 1 || n_present > 512 || rd_u16(mm + 2) != 0) return BSO_E_FORMAT;
     if (ti->model_bytes != 260 + 4ull * n_present + 16ull * ti->n_routes) return BSO_E_FORMAT;
     uint64_t sum = 0;
     int prev = -1;

@@ -87,3 +87,26 @@ def test_library_refuses_what_the_oracle_refuses():
         struct.pack_into(fmt, b, off, v)
         with pytest.raises(bs.BsError):
             bs.workspace_bytes(bytes(b))
+
+
+def test_library_refuses_nonzero_reserved_fields_and_unaligned_names():
+    # the same rules as the oracle's: a nonzero reserved field (the RANS model's second u16,
+    # the directory entry's reserved u64, the header's) and a names section off a 16-byte
+    # boundary make the container invalid, for the planner and for the no-alloc entry point
+    import struct
+    import numpy as np
+    import lossless_entropy_coding_interleaved_b200 as bs
+    import oracle
+    w = (np.arange(3000, dtype=np.uint16) % 97) + 0x3C00
+    c = oracle.encode([("a", w, "bf16")], force_rans=True)
+    ti = oracle.info(c, 0)
+    dir_off = int.from_bytes(c[24:32], "little")
+    edits = [(ti["model_offset"] + 2, "<H", 1), (dir_off + 72, "<Q", 1), (56, "<Q", 1), (32, "<Q", 208 + 8)]
+    for off, fmt, v in edits:
+        b = bytearray(c)
+        struct.pack_into(fmt, b, off, v)
+        with pytest.raises(bs.BsError) as e:
+            bs.workspace_bytes(bytes(b))
+        assert e.value.code == bs.E_FORMAT
+        with pytest.raises(oracle.OracleError):
+            oracle.validate(bytes(b))

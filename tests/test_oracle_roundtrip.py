@@ -180,3 +180,17 @@ def test_fault_table_sum_and_offsets():
     bad[ti["data_offset"]] ^= 0x04                         # unaligned chunk offset
     with pytest.raises(oracle.OracleError):
         oracle.validate(bytes(bad))
+
+
+def test_fault_reserved_fields():
+    # a nonzero reserved field makes a container invalid: the RANS model's second u16, the
+    # directory entry's reserved u64, the header's reserved u64
+    _, c = _container()
+    ti = oracle.info(bytes(c), 0)
+    dir_off = int.from_bytes(bytes(c[24:32]), "little")
+    for off in (ti["model_offset"] + 2, dir_off + 72, 56):
+        bad = bytearray(c)
+        bad[off] = 1
+        with pytest.raises(oracle.OracleError) as e:
+            oracle.validate(bytes(bad))
+        assert e.value.code == oracle.E_FORMAT

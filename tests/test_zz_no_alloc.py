@@ -79,3 +79,33 @@ def test_noalloc_reports_corrupt_chunk_and_oversized_tables():
     with pytest.raises(bs.BsError) as e:
         bs.decode_noalloc(bytes(bad), d_big, 0, out)
     assert e.value.code == bs.E_FORMAT
+
+
+@pytest.mark.parametrize("model,compact", [("joint", True), ("joint", False), ("factored", None)])
+def test_noalloc_matches_regular_decode_for_each_table_kind(model, compact):
+    # Both entry points validate with the same rules and build their tables with the same
+    # builder; the no-alloc one keeps them in the static array. Checked on two calls in a row
+    # for the JOINT tables with 4-byte entries (every frequency at most 255) and 8-byte ones,
+    # and for the largest factored tables (ns = 12, 15 routes).
+    rng = np.random.default_rng(3)
+    if model == "factored":
+        w = np.concatenate([((e << 7) | ((np.arange(20000) % 3) << 4) | (np.arange(20000) % 16)).astype(np.uint16)
+                            for e in range(100, 116)])
+        c = oracle.encode([("t", w, "bf16")], ns=12, nh=4, max_routes=15, log2_chunk=12)
+        assert oracle.info(c, 0)["n_routes"] == 15
+    else:
+        x = rng.standard_normal(300_000).astype(np.float32) * 0.02
+        w = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16).copy()
+        if not compact:
+            w[::3] = 0x3F80                    # one pair takes a third of the slots: F above 255
+        c = oracle.encode([("t", w, "bf16")], model="joint", log2_chunk=12)
+    plan = bs.Plan(c, device="cuda:0")
+    want = plan.decode(0)
+    for _ in range(2):
+        got = plan.empty_output(0)
+        got.fill_(0x55)
+        bs.decode_noalloc(c, plan.d_container, 0, got)
+        torch.cuda.synchronize()
+        assert torch.equal(got, want)
+    assert np.array_equal(S.words_numpy(want).reshape(-1), w)
+    plan.check()
