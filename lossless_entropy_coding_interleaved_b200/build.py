@@ -17,9 +17,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libbs.so")
-SOURCES = ["bs_kernels.cu", "bs_encode_kernels.cu", "bs_noalloc.cu", "bs_fw.cu", "bs_fw_gemv.cu", "bs_plan.cpp", "bs_encode.cpp",
+SOURCES = ["bs_kernels.cu", "bs_joint4.cu", "bs_encode_kernels.cu", "bs_noalloc.cu", "bs_fw.cu", "bs_fw_gemv.cu", "bs_plan.cpp", "bs_validate.cpp", "bs_encode.cpp",
            "bs_stream.cpp"]
-HEADERS = ["bs_internal.h", "bs_host.h", "bs_fw.cuh", os.path.join(ROOT, "include", "bs.h")]
+HEADERS = ["bs_internal.h", "bs_device.cuh", "bs_host.h", "bs_fw.cuh", os.path.join(ROOT, "include", "bs.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",

@@ -26,8 +26,8 @@ constexpr uint32_t kMaxNs = 12, kMinNh = 3, kMaxNh = 5, kMaxPrecision = 16, kMax
 constexpr uint32_t kJointPairs = 4096, kMinNj = 8, kMaxNj = 13;
 constexpr uint32_t kJointRegion = 8u << kMaxNj;
 // A JOINT tensor whose frequencies are all below 256 (every large tensor of normally
-// distributed weights) gets 4-byte slot entries instead: F in byte 0, the slot's rank in
-// byte 1, bits 16-19 zero and the pair j in bits 20-31 (so the high half is the word j << 4).
+// distributed weights) gets 4-byte slot entries instead: the word j << 4 in the low half
+// (its low nibble zero), the slot's rank in byte 2 and F in byte 3.
 // A random 4-byte gather of 32 lanes costs about 3.5 shared-memory wavefronts against about
 // 6 for the 8-byte one. The table region is then at most 32 KiB.
 constexpr uint32_t kCompactMaxF = 255;
@@ -230,7 +230,9 @@ void count_launch();
 // JointCompact: JOINT with 4-byte slot entries, any nj.
 enum class DecodeMode { Default = 0, Generic = 1, Joint = 2, JointGeneric = 3, JointCompact = 4 };
 constexpr int kDecodeModes = 5;
-constexpr int kWarpsJoint4 = 28, kChainsJoint4 = 2;
+// JOINT with 4-byte entries: 32 warps of 2 chunks at 64 registers a thread; the 32 KiB table
+// and 64 rings of each kind take 192 KiB of shared memory.
+constexpr int kWarpsJoint4 = 32, kChainsJoint4 = 2;
 constexpr uint32_t kDefaultNj = 13;
 // The largest CTA shape of each mode (small launches take fewer warps, see launch_warps).
 inline uint32_t max_warps_of(DecodeMode m) {
@@ -242,6 +244,7 @@ inline uint32_t chains_of(DecodeMode m) {
          : m == DecodeMode::JointCompact ? kChainsJoint4 : kChainsGeneric;
 }
 int launch_decode(const DecodeParams& p, DecodeMode mode, uint32_t smem_bytes, void* stream);
+int launch_decode_joint4(const DecodeParams& p, uint32_t smem_bytes, void* stream); // bs_joint4.cu
 int launch_copy(const CopyParams& p, void* stream);
 int launch_checksum(const void* data, uint64_t n, int raw_bytes, unsigned long long* d_sum, void* stream);
 int max_dynamic_smem();

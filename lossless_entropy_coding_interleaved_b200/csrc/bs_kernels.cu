@@ -41,27 +41,10 @@
 
 #include <cstdint>
 
+#include "bs_device.cuh"
 #include "bs_internal.h"
 
 namespace bs {
-
-__device__ __forceinline__ uint32_t lanemask_lt() {
-    uint32_t m;
-    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-    return m;
-}
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// cp.async of up to 16 bytes (the rest of the 16-byte destination is zero-filled).
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
 // One chunk in flight on a warp: lane j holds state j.
 // Only what the step loop needs stays in registers; the rest (the rings' offsets, the block
@@ -84,8 +67,8 @@ struct Chain {
 // otherwise the CTA has WARPS warps, a compile-time constant (measured 3% faster).
 // JOINT: the JOINT kind: one table of 2^nj slots over the pairs (s, h) (nj = item.ns),
 // one lookup and one multiply-add per weight.
-// JOINT 2: the JOINT kind with 4-byte slot entries (F | rank << 8 | j << 20), any nj.
-template <int WARPS, int CHAINS, int NS, int NH, bool SHAPE_FROM_PARAMS, int JOINT>
+// (JOINT tensors with 4-byte slot entries have a kernel of their own, bs_joint4.cu.)
+template <int WARPS, int CHAINS, int NS, int NH, bool SHAPE_FROM_PARAMS, bool JOINT>
 __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int kChains = CHAINS;
     // dynamic smem: [fraction rows, one copy per lane][s-table][rings], or for JOINT
@@ -94,21 +77,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
     __shared__ int s_item;
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
 
-    if (tid == 0) { // the item whose CTA range holds this block
-        int lo = 0, hi = static_cast<int>(p.n_items) - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (p.item[mid].cta_begin <= blockIdx.x) lo = mid;
-            else hi = mid - 1;
-        }
-        s_item = lo;
-    }
+    if (tid == 0) find_item(p, &s_item); // the item whose CTA range holds this block
     __syncthreads();
     const DecodeItem& it = p.item[s_item];
     const uint32_t ns = NS > 0 ? NS : it.ns, nh = NH > 0 ? NH : it.nh, P = ns + nh;
 
     if (JOINT) { // stage the joint table as it is
-        const uint32_t jb = (JOINT == 2 ? 4u : 8u) << ns;
+        const uint32_t jb = 8u << ns;
         uint4* jdst = reinterpret_cast<uint4*>(smem);
         for (uint32_t k = tid; k < jb / 16u; k += blockDim.x) jdst[k] = __ldg(it.tables + k);
     } else { // stage the tables: the s-table as it is, each fraction entry once per lane
@@ -132,7 +107,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
 
     const bool nib_stored = it.nib_mode == 0;
     const uint32_t raw_const = (it.nib_mode & 15u) * 0x11111111u;
-    const uint32_t rings = JOINT == 2 ? kJoint4Region : JOINT ? kJointRegion : kHRegion + s_region_bytes(ns); // a multiple of kRingBytes
+    const uint32_t rings = JOINT ? kJointRegion : kHRegion + s_region_bytes(ns); // a multiple of kRingBytes
     const uint32_t ring_off = rings + (warp * kChains) * kRingBytes;       // this warp's first word ring
     const uint32_t nring_off = rings + warps * kChains * kRingBytes + (warp * kChains) * kNibRingBytes;
     const uint32_t smem_base = smem_u32(smem);
@@ -166,7 +141,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
         nb = max(nb, (h.nc + 255u) >> 8);
     }
 
-    const uint32_t smask8 = ((1u << ns) - 1u) << (JOINT == 2 ? 2 : 3), hmask7 = ((1u << nh) - 1u) << 7; // JOINT: smask8 masks the slot
+    const uint32_t smask8 = ((1u << ns) - 1u) << 3, hmask7 = ((1u << nh) - 1u) << 7; // JOINT: smask8 masks the slot
     const uint32_t lt = lanemask_lt(), lane4 = lane << 2;
     const uint32_t mul2 = p.mul2, mul65536 = p.mul65536;
 
@@ -237,17 +212,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_cons
             uint2 se[kChains];
             uint32_t fe[kChains], xn[kChains], m[kChains], w[kChains];
             bool need[kChains];
-            if (JOINT == 2) { // the slot's 4-byte entry: F, rank, and the word in the high half
-#pragma unroll
-                for (int k = 0; k < kChains; ++k)
-                    se[k].x = *reinterpret_cast<const uint32_t*>(smem + ((c[k].x << 2) & smask8));
-#pragma unroll
-                for (int k = 0; k < kChains; ++k) {
-                    xn[k] = (se[k].x & 0xFFu) * (c[k].x >> ns) + __byte_perm(se[k].x, 0u, 0x4441);
-                    need[k] = xn[k] < kStateL;
-                    fe[k] = 0;
-                }
-            } else if (JOINT) { // the slot's entry: F and the word's (s, h) part in .x, the rank in .y
+            if (JOINT) { // the slot's entry: F and the word's (s, h) part in .x, the rank in .y
 #pragma unroll
                 for (int k = 0; k < kChains; ++k)
                     se[k] = *reinterpret_cast<const uint2*>(smem + ((c[k].x << 3) & smask8));
@@ -432,7 +397,7 @@ int max_dynamic_smem() {
     return v;
 }
 
-template <int WARPS, int CHAINS, int NS, int NH, bool SHAPE_FROM_PARAMS, int JOINT>
+template <int WARPS, int CHAINS, int NS, int NH, bool SHAPE_FROM_PARAMS, bool JOINT>
 static int launch_decode_shape(const DecodeParams& p, uint32_t smem_bytes, cudaStream_t s) {
     auto kernel = decode_kernel<WARPS, CHAINS, NS, NH, SHAPE_FROM_PARAMS, JOINT>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes));
@@ -442,7 +407,7 @@ static int launch_decode_shape(const DecodeParams& p, uint32_t smem_bytes, cudaS
     return cudaGetLastError();
 }
 
-template <int WARPS, int CHAINS, int NS, int NH, int JOINT>
+template <int WARPS, int CHAINS, int NS, int NH, bool JOINT>
 static int launch_decode_t(const DecodeParams& p, uint32_t smem_bytes, cudaStream_t s) {
     if (p.warps < 1 || p.warps > WARPS) return cudaErrorInvalidValue;
     return p.warps == WARPS ? launch_decode_shape<WARPS, CHAINS, NS, NH, false, JOINT>(p, smem_bytes, s)
@@ -453,11 +418,11 @@ int launch_decode(const DecodeParams& p, DecodeMode mode, uint32_t smem_bytes, v
     if (p.total_ctas == 0) return cudaSuccess;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (mode) {
-    case DecodeMode::Default: return launch_decode_t<kWarpsDefault, kChainsDefault, 11, 5, 0>(p, smem_bytes, s);
-    case DecodeMode::Joint: return launch_decode_t<kWarpsJoint, kChainsJoint, 13, 5, 1>(p, smem_bytes, s);
-    case DecodeMode::JointGeneric: return launch_decode_t<kWarpsGeneric, kChainsGeneric, 0, 5, 1>(p, smem_bytes, s);
-    case DecodeMode::JointCompact: return launch_decode_t<kWarpsJoint4, kChainsJoint4, 0, 5, 2>(p, smem_bytes, s);
-    default: return launch_decode_t<kWarpsGeneric, kChainsGeneric, 0, 0, 0>(p, smem_bytes, s);
+    case DecodeMode::Default: return launch_decode_t<kWarpsDefault, kChainsDefault, 11, 5, false>(p, smem_bytes, s);
+    case DecodeMode::Joint: return launch_decode_t<kWarpsJoint, kChainsJoint, 13, 5, true>(p, smem_bytes, s);
+    case DecodeMode::JointGeneric: return launch_decode_t<kWarpsGeneric, kChainsGeneric, 0, 5, true>(p, smem_bytes, s);
+    case DecodeMode::JointCompact: return launch_decode_joint4(p, smem_bytes, stream);
+    default: return launch_decode_t<kWarpsGeneric, kChainsGeneric, 0, 0, false>(p, smem_bytes, s);
     }
 }
 

@@ -162,12 +162,17 @@ def test_decode_geometry():
     items = [("joint", w, "bf16"), ("u", np.arange(1 << 16, dtype=np.uint32).astype(np.uint16), "bf16")]
     plan = bs.Plan(oracle.encode(items, model="joint"), device="cuda:0")
     assert plan.info(1)["kind"] == bs.KIND_STORED
-    assert plan.decode_geometry(0) == (56, sms)       # JOINT: 28 warps of 2 chunks, one CTA per SM
+    assert plan.decode_geometry(0) == (64, sms)       # JOINT, 4-byte entries: 32 warps of 2 chunks, one CTA per SM
     assert plan.decode_geometry(1) == (0, sms)
     fplan = bs.Plan(oracle.encode(items[:1]), device="cuda:0")
     assert fplan.decode_geometry(0) == (48, sms)      # RANS, default precisions: 24 warps of 2
     gplan = bs.Plan(oracle.encode(items[:1], ns=10, nh=4), device="cuda:0")
     assert gplan.decode_geometry(0) == (40, sms)      # other precisions: 20 warps of 2
+    # a JOINT tensor with a pair of frequency above 255 keeps 8-byte entries: 28 warps of 2
+    skew = np.full(5000, 0x3F80, np.uint16)
+    skew[::7] = 0x3F90
+    jplan = bs.Plan(oracle.encode([("skew", skew, "bf16")], model="joint", force_rans=True), device="cuda:0")
+    assert jplan.info(0)["kind"] == bs.KIND_JOINT and jplan.decode_geometry(0) == (56, sms)
     with pytest.raises(bs.BsError) as e:
         plan.decode_geometry(2)
     assert e.value.code == bs.E_ARG
