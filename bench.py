@@ -52,6 +52,9 @@ def _args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-modes", action="store_true",
+                    help="model mode on the 9B checkpoint: skip the layer-by-layer and 27B-scale 1 GB-batch "
+                         "measurements that the default line carries under 'modes'")
     ap.add_argument("--cpu-threads", type=int, default=0, help="oracle threads (0: all host cores)")
     ap.add_argument("--batch", type=int, default=1, help="gemv mode: tokens per product (1..8)")
     ap.add_argument("--model", choices=["joint", "factored"], default="joint",
@@ -377,6 +380,85 @@ def run_fw_reference(a):
         flush=True)
 
 
+# ------------------------------------------------------------------ the other decode modes
+def _mode_layerwise(plan, outs, infos, stream, steps, ranks):
+    """The same checkpoint decoded layer by layer: one bs_decode_batch per layer group per
+    step, on one stream, container and outputs in HBM. Returns the measurement as a dict."""
+    gid = _groups(plan.names)
+    members = [[k for k in range(plan.n_tensors) if gid[k] == g] for g in range(max(gid) + 1)]
+    coded = sum(i["coded_bytes"] for i in infos)
+    out_bytes = sum(i["out_bytes"] for i in infos)
+
+    def step():
+        for m in members:
+            plan.decode_batch(m, [outs[k] for k in m], stream=stream)
+
+    for _ in range(3):
+        step()
+    ms = ranks.max(_timed(stream, steps, step, ranks.barrier))
+    plan.check()
+    peak, _ = _peak_hbm()
+    achieved = (coded + out_bytes) * steps / (ms * 1e-3) / 1e9
+    return {"value": round(ranks.world * steps * out_bytes / (ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+            "ms_per_step": round(ms / steps, 4), "steps": steps, "groups": len(members),
+            "calls_per_step": len(members), "roofline_frac": round(achieved / peak, 4),
+            "how": "one bs_decode_batch per layer group (42 layers + the embedding), one stream"}
+
+
+def _mode_batches(workload, batch_gb, model, dev, stream, steps, ranks):
+    """A checkpoint decoded in batches of whole chunks holding at most batch_gb GB of output and
+    one kernel wave each (bs_decode_ranges), one stream. The originals are freed after the
+    histograms, and every tensor's checksum is verified on the device before timing."""
+    import torch
+
+    import lossless_entropy_coding_interleaved_b200 as bs
+    import synthetic as S
+    specs, n, _ = _workload_desc(workload, None)
+    originals = [(s.name, S.generate(s, dev)) for s in specs]
+    d_c, _ = bs.encode(originals, model=model)
+    hist = _word_histograms(originals, specs, dev)
+    del originals
+    torch.cuda.empty_cache()
+    plan = bs.Plan(d_container=d_c)
+    outs = [plan.empty_output(k) for k in range(plan.n_tensors)]
+    infos = [plan.info(k) for k in range(plan.n_tensors)]
+    coded = sum(i["coded_bytes"] for i in infos)
+    out_bytes = sum(i["out_bytes"] for i in infos)
+    bf16_n = sum(i["n_elems"] for i in infos if i["kind"] != bs.KIND_RAW)
+    bf16_coded = sum(i["coded_bytes"] for i in infos if i["kind"] != bs.KIND_RAW)
+    hbits = 0.0
+    for cnt, numel in hist:
+        c = cnt[cnt > 0].to(torch.float64)
+        hbits += float(-(c * torch.log2(c / numel)).sum())
+    batches = _chunk_batches(plan, infos, outs, batch_gb)
+
+    def step():
+        for b in batches:
+            plan.decode_ranges(b, stream=stream)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    plan.check()
+    for k in range(plan.n_tensors):
+        plan.verify(k, outs[k])                  # raises on any mismatch
+    ms = ranks.max(_timed(stream, steps, step, ranks.barrier))
+    plan.check()
+    peak, _ = _peak_hbm()
+    achieved = (coded + out_bytes) * steps / (ms * 1e-3) / 1e9
+    res = {"value": round(ranks.world * steps * out_bytes / (ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+           "ms_per_step": round(ms / steps, 4), "steps": steps, "workload": workload, "n_weights": n,
+           "batches": len(batches), "batch_gb": batch_gb, "roofline_frac": round(achieved / peak, 4),
+           "bits_per_weight": round(bf16_coded * 8 / bf16_n, 5),
+           "overhead_pct_vs_entropy": round(100 * (bf16_coded * 8 / hbits - 1), 4),
+           "parity": "every tensor's checksum verified on the device before timing",
+           "how": f"one bs_decode_ranges call per batch of at most {batch_gb} GB of output and one kernel "
+                  "wave, in container order, one stream"}
+    del plan, outs, d_c
+    torch.cuda.empty_cache()
+    return res
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(a):
     import torch
@@ -404,6 +486,7 @@ def run_ours(a):
         originals = None
         torch.cuda.empty_cache()
     plan = bs.Plan(d_container=d_c)
+    container_bytes = int(d_c.numel())
     outs = [plan.empty_output(k) for k in range(plan.n_tensors)]
     idx = list(range(plan.n_tensors))
     infos = [plan.info(k) for k in idx]
@@ -547,6 +630,17 @@ def run_ours(a):
                        "Plan.decode_batch, its tensors copied back out; three streams overlap the groups"}
         del h_c, h_outs
 
+    # the other two decode modes of the target, beside the whole-model number: the same 9B
+    # checkpoint layer by layer, and the 27B-scale checkpoint in 1 GB batches
+    modes = None
+    if (not a.no_modes and a.workload == "gemma2_9b" and a.layers is None and a.batch_gb is None
+            and a.log2_chunk == 16):
+        modes = {"layerwise": _mode_layerwise(plan, outs, infos, stream, a.steps, ranks)}
+        del plan, outs, d_c
+        torch.cuda.empty_cache()
+        modes["qwen_27b_scale_1gb_batches"] = _mode_batches("qwen_27b_scale", 1.0, a.model, dev, stream,
+                                                            max(5, a.steps // 2), ranks)
+
     cpu = None
     if rank == 0 and not a.no_cpu_baseline:
         cpu = _cpu_baseline(a.workload, _cpu_threads(a.cpu_threads), a.model)
@@ -560,7 +654,7 @@ def run_ours(a):
         "scaling": "weak", "vs_baseline": None, "dtype": "u32",
         "data": "synthetic (seeded device draws, synthetic/ recipe)",
         "config": {"workload": a.workload, "description": desc, "n_weights": n, "tensors": len(specs),
-                   "container_bytes": int(d_c.numel()), "coded_bytes": int(coded),
+                   "container_bytes": container_bytes, "coded_bytes": int(coded),
                    "decoded_bytes": int(out_bytes),
                    "bits_per_weight": round(bf16_coded * 8 / bf16_n, 5),
                    "entropy_bits_per_weight": round(h_per_w, 5),
@@ -590,6 +684,8 @@ def run_ours(a):
         "gpu_launches": int(launches),
         "clocks": clk,
     }
+    if modes is not None:
+        line["modes"] = modes
     print(json.dumps(line), flush=True)
 
 
