@@ -435,6 +435,21 @@ typedef struct {
  * d_err as for bs_fw_decode. Enqueued on stream. */
 bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_t batch, uint32_t* d_err, void* stream);
 
+/* Y = X W^T for a batch of tokens on the tensor cores, W in the FW layout: the same products as
+ * bs_fw_gemv (the same items, Y[b][r] = sum_k W[r][k] X[b][k]) for batches too large for the
+ * CUDA cores. Source: the NVLC card's runtime keeps the compressed weights resident and no
+ * decoded-weight cache (its runtime accounting and DGX Spark tables); the kernel is this
+ * library's. Each CTA decodes 128 rows of W, one 256-wide slice of K at a time, into shared
+ * memory in the tensor cores' operand layout and multiplies them with up to 64 tokens
+ * (tcgen05.mma, BF16 operands, FP32 accumulation in tensor memory); larger batches take
+ * several CTAs per row block, each decoding its rows again.
+ *   rows must be a multiple of 128 and cols of 256 (else BS_E_ARG); batch is 1..2^20.
+ *   d_err: as for bs_fw_decode; bit 1 means that a wait inside the kernel ran out (the
+ *          outputs of that CTA are then not written).
+ * The FP32 sums follow the tensor cores' order, so they may differ from bs_fw_gemv's in the
+ * last bits. Enqueued on stream. */
+bs_status bs_fw_gemm(int32_t n, const bs_fw_gemv_item* items, uint32_t batch, uint32_t* d_err, void* stream);
+
 /* Diagnostics (this library's design). */
 const char* bs_status_str(bs_status s);
 int bs_last_cuda_error(void); /* the cudaError_t behind the last BS_E_CUDA on this thread */

@@ -135,7 +135,8 @@ def _load():
     L.bs_fw_parse.argtypes = [P, sz, sz, ctypes.POINTER(FwInfo)]
     L.bs_fw_decode.argtypes = [i32, P, P, P, P, P, P]
     L.bs_fw_gemv.argtypes = [i32, ctypes.POINTER(FwGemvItem), ctypes.c_uint32, P, P]
-    for fn in ("bs_fw_measure", "bs_fw_write", "bs_fw_parse", "bs_fw_decode", "bs_fw_gemv"):
+    L.bs_fw_gemm.argtypes = [i32, ctypes.POINTER(FwGemvItem), ctypes.c_uint32, P, P]
+    for fn in ("bs_fw_measure", "bs_fw_write", "bs_fw_parse", "bs_fw_decode", "bs_fw_gemv", "bs_fw_gemm"):
         getattr(L, fn).restype = ctypes.c_int
     for fn in ("bs_streamer_create", "bs_streamer_group_count", "bs_streamer_tensor_info_get", "bs_streamer_prefetch", "bs_streamer_acquire",
                "bs_streamer_release", "bs_streamer_get_stats", "bs_streamer_check"):
@@ -160,7 +161,8 @@ EXPORTS = ("bs_plan_workspace_bytes", "bs_plan_workspace_bytes_device", "bs_plan
            "bs_streamer_create", "bs_streamer_group_count", "bs_streamer_tensor_info_get", "bs_streamer_prefetch",
            "bs_streamer_acquire",
            "bs_streamer_release", "bs_streamer_get_stats", "bs_streamer_check", "bs_streamer_destroy",
-           "bs_fw_scratch_bytes", "bs_fw_measure", "bs_fw_write", "bs_fw_parse", "bs_fw_decode", "bs_fw_gemv")
+           "bs_fw_scratch_bytes", "bs_fw_measure", "bs_fw_write", "bs_fw_parse", "bs_fw_decode", "bs_fw_gemv",
+           "bs_fw_gemm")
 
 
 def decode_noalloc(container, d_container: torch.Tensor, idx: int, out: torch.Tensor, stream=None) -> torch.Tensor:
@@ -596,6 +598,36 @@ def fw_decode(fws, infos, outs, err: torch.Tensor, stream=None):
     with torch.cuda.device(err.device):
         _check(lib.bs_fw_decode(n, p_fw, inf, p_out, sizes, err.data_ptr(), _stream(stream)), "fw_decode")
     return outs
+
+
+def _fw_products(products, max_batch):
+    n = len(products)
+    arr = (FwGemvItem * max(n, 1))()
+    batch = None
+    for k, (fw, info, rows, cols, x, y) in enumerate(products):
+        b = 1 if x.dim() == 1 else x.shape[0]
+        assert batch in (None, b), "every product of one call has the same batch"
+        batch = b
+        assert max_batch is None or b <= max_batch
+        assert x.is_cuda and x.is_contiguous() and x.element_size() == 2 and x.numel() == b * cols
+        assert y.is_cuda and y.is_contiguous() and y.dtype == torch.float32 and y.numel() == b * rows
+        arr[k].d_fw = fw.data_ptr()
+        arr[k].info = info
+        arr[k].rows, arr[k].cols = rows, cols
+        arr[k].d_x = x.data_ptr()
+        arr[k].d_y = y.data_ptr()
+    return n, arr, batch or 1
+
+
+def fw_gemm(products, err: torch.Tensor, stream=None):
+    """bs_fw_gemm: as fw_gemv, on the tensor cores, for any batch (rows a multiple of 128):
+    products is a sequence of (fw, info, rows, cols, x [batch, cols] BF16, y [batch, rows] float32).
+    err: a zeroed int32 CUDA tensor of one element. Enqueued on the stream."""
+    n, arr, batch = _fw_products(products, None)
+    assert err.is_cuda and err.dtype == torch.int32 and err.numel() >= 1
+    with torch.cuda.device(err.device):
+        _check(lib.bs_fw_gemm(n, arr, batch, err.data_ptr(), _stream(stream)), "fw_gemm")
+    return [p[5] for p in products]
 
 
 def fw_gemv(products, err: torch.Tensor, stream=None):

@@ -17,7 +17,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libbs.so")
-SOURCES = ["bs_kernels.cu", "bs_joint4.cu", "bs_encode_kernels.cu", "bs_noalloc.cu", "bs_fw.cu", "bs_fw_gemv.cu", "bs_plan.cpp", "bs_validate.cpp", "bs_encode.cpp",
+SOURCES = ["bs_kernels.cu", "bs_joint4.cu", "bs_encode_kernels.cu", "bs_noalloc.cu", "bs_fw.cu", "bs_fw_gemv.cu", "bs_fw_gemm.cu", "bs_plan.cpp", "bs_validate.cpp", "bs_encode.cpp",
            "bs_stream.cpp"]
 HEADERS = ["bs_internal.h", "bs_device.cuh", "bs_host.h", "bs_fw.cuh", os.path.join(ROOT, "include", "bs.h")]
 

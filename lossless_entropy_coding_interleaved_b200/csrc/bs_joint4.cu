@@ -21,8 +21,9 @@
 //    each take a warp instruction every other cycle). The lane-prefix mask of the ballot is
 //    a multiply-add (m * 2^(32 - lane) keeps the bits below the lane) rather than an AND on
 //    the busier ALU pipe; its multiplier, like the renormalisation's 2^16 and 2, comes from
-//    the launch parameters so that it stays a multiply. Multiplies-high are not used: they
-//    run at a lower rate than the shifts they would replace (measured).
+//    the launch parameters so that it stays a multiply. The table is read by slot index, so
+//    the address scaling folds into the load. Multiplies-high are not used: they run at a
+//    lower rate than the shifts they would replace (measured).
 //  * Each chunk's word stream flows through its own 2 KiB ring of four 512-byte quarters, and
 //    its nibble words through a 512-byte ring of four blocks, both filled by cp.async. The
 //    upkeep between two pairs of blocks (16 steps) has no branch: at most two quarters per
@@ -126,7 +127,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) joint4_decode_kernel(const __gr
     const uint32_t lt_mul = lane ? 1u << (32 - lane) : 0u; // m * lt_mul keeps the bits of m below this lane
     const uint32_t lane4 = lane << 2, lane16 = lane << 4;
     const uint32_t mul2 = p.mul2, mul65536 = p.mul65536;
-    const uint32_t tmask = (4u << nj) - 4u;
+    const uint32_t jmask = (1u << nj) - 1u;
 
     // Request the 16-byte units [b, b + 16) of chain k's word stream with b < end, b = fb + i*512
     // + lane*16, into its ring.
@@ -202,7 +203,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) joint4_decode_kernel(const __gr
 #pragma unroll
             for (int k = 0; k < kChains4; ++k) { // the slot's entry
                 q[k] = c[k].x >> nj;
-                e[k] = *reinterpret_cast<const uint32_t*>(smem + ((c[k].x << 2) & tmask));
+                e[k] = reinterpret_cast<const uint32_t*>(smem)[c[k].x & jmask]; // a scaled-index load
             }
 #pragma unroll
             for (int k = 0; k < kChains4; ++k)
