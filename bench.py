@@ -58,6 +58,9 @@ def _args():
     ap.add_argument("--cpu-threads", type=int, default=0, help="oracle threads (0: all host cores)")
     ap.add_argument("--batch", type=int, default=1,
                     help="gemv mode: tokens per product (1..8 on the CUDA cores, more on the tensor cores)")
+    ap.add_argument("--product", choices=["auto", "cuda", "tensor"], default="auto",
+                    help="gemv mode: the CUDA-core product (bs_fw_gemv, batch 1..8), the tensor-core one "
+                         "(bs_fw_gemm), or auto: tensor cores above batch 8")
     ap.add_argument("--model", choices=["joint", "factored"], default="joint",
                     help="rANS model of the container: joint (one table over (s, h), kind JOINT; "
                          "the default) or factored (s-model plus exponent routes, kind RANS)")
@@ -96,7 +99,9 @@ def _peak_hbm():
 # keeps the hash of the kernel's sources at capture time (comments and blank lines removed);
 # the figure is reported only while the sources still hash to it, else traffic is null.
 _TRAFFIC = {
-    "decode_kernel": (("bs_kernels.cu", "bs_internal.h"), None, None),
+    # joint4_decode_kernel, first 8 layers of the 9B checkpoint: 2.0910 GB read + 3.1208 GB
+    # written for 1,585,561,600 weights
+    "joint4_decode_kernel": (("bs_joint4.cu", "bs_device.cuh", "bs_internal.h"), "d8127505dd5bd2be", 3.28706),
     "fw_decode_kernel": (("bs_fw.cu", "bs_fw.cuh"), None, None),
 }
 
@@ -115,7 +120,7 @@ def _source_hash(files):
     return hashlib.sha256(text.encode()).hexdigest()[:16]
 
 
-def _traffic_per_weight(kernel="decode_kernel"):
+def _traffic_per_weight(kernel="joint4_decode_kernel"):
     """DRAM bytes per weight of a kernel from its capture, if its sources are unchanged; else None."""
     files, want, tpw = _TRAFFIC[kernel]
     try:
@@ -382,17 +387,31 @@ def run_fw_reference(a):
 
 
 # ------------------------------------------------------------------ the other decode modes
-def _mode_layerwise(plan, outs, infos, stream, steps, ranks):
+def _mode_layerwise(plan, outs, infos, stream, steps, ranks, n_streams=1):
     """The same checkpoint decoded layer by layer: one bs_decode_batch per layer group per
-    step, on one stream, container and outputs in HBM. Returns the measurement as a dict."""
+    step, container and outputs in HBM, on one stream or, with n_streams = 2, on two streams
+    in turn (as a consumer that double-buffers layers issues them; two layers' CTAs can then
+    share the SMs). Returns the measurement as a dict."""
+    import torch
     gid = _groups(plan.names)
     members = [[k for k in range(plan.n_tensors) if gid[k] == g] for g in range(max(gid) + 1)]
     coded = sum(i["coded_bytes"] for i in infos)
     out_bytes = sum(i["out_bytes"] for i in infos)
+    side = [torch.cuda.Stream(device=stream.device) for _ in range(n_streams)] if n_streams > 1 else []
 
     def step():
-        for m in members:
-            plan.decode_batch(m, [outs[k] for k in m], stream=stream)
+        if not side:
+            for m in members:
+                plan.decode_batch(m, [outs[k] for k in m], stream=stream)
+            return
+        start = torch.cuda.Event()
+        start.record(stream)
+        for s_ in side:
+            s_.wait_event(start)
+        for i, m in enumerate(members):
+            plan.decode_batch(m, [outs[k] for k in m], stream=side[i % len(side)])
+        for s_ in side:
+            stream.wait_stream(s_)
 
     for _ in range(3):
         step()
@@ -403,7 +422,8 @@ def _mode_layerwise(plan, outs, infos, stream, steps, ranks):
     return {"value": round(ranks.world * steps * out_bytes / (ms * 1e-3) / 1e9, 3), "unit": "GB/s",
             "ms_per_step": round(ms / steps, 4), "steps": steps, "groups": len(members),
             "calls_per_step": len(members), "roofline_frac": round(achieved / peak, 4),
-            "how": "one bs_decode_batch per layer group (42 layers + the embedding), one stream"}
+            "how": "one bs_decode_batch per layer group (42 layers + the embedding), "
+                   + ("one stream" if not side else f"{n_streams} streams in turn")}
 
 
 def _mode_batches(workload, batch_gb, model, dev, stream, steps, ranks):
@@ -636,7 +656,8 @@ def run_ours(a):
     modes = None
     if (not a.no_modes and a.workload == "gemma2_9b" and a.layers is None and a.batch_gb is None
             and a.log2_chunk == 16):
-        modes = {"layerwise": _mode_layerwise(plan, outs, infos, stream, a.steps, ranks)}
+        modes = {"layerwise": _mode_layerwise(plan, outs, infos, stream, a.steps, ranks),
+                 "layerwise_two_streams": _mode_layerwise(plan, outs, infos, stream, a.steps, ranks, 2)}
         del plan, outs, d_c
         torch.cuda.empty_cache()
         modes["qwen_27b_scale_1gb_batches"] = _mode_batches("qwen_27b_scale", 1.0, a.model, dev, stream,
@@ -678,7 +699,10 @@ def run_ours(a):
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": (None if tpw is None else int(tpw * bf16_n)),
                      "traffic_source": "ncu capture of this kernel on the first 8 layers, scaled by weights",
-                     "kernel": "decode_kernel", "per_launch_bytes": int(coded + out_bytes),
+                     "kernel": ("joint4_decode_kernel (with decode_kernel for the JOINT tensors whose "
+                                "frequencies exceed 255: the 168 RMSNorm vectors, 0.3% of the step)"
+                                if a.model == "joint" else "decode_kernel"),
+                     "per_launch_bytes": int(coded + out_bytes),
                      "launch_ms_mean": round(mean_step, 4)},
         "e2e": e2e,
         "cpu_baseline": cpu,
@@ -1261,9 +1285,12 @@ def run_gemv(a):
     stream = torch.cuda.current_stream()
 
     # batches above 8 go to the tensor cores (bs_fw_gemm), batches 1..8 to the CUDA cores
-    product = bs.fw_gemm if batch > 8 else bs.fw_gemv
-    kernel = "fw_gemm_kernel" if batch > 8 else "fw_gemv_kernel"
-    if batch > 8 and any(rows % 128 for c in calls for _, rows, _ in c):
+    tensor = a.product == "tensor" or (a.product == "auto" and batch > 8)
+    if not tensor and batch > 8:
+        raise SystemExit("bench: the CUDA-core product takes batches of 1..8")
+    product = bs.fw_gemm if tensor else bs.fw_gemv
+    kernel = "fw_gemm_kernel" if tensor else "fw_gemv_kernel"
+    if tensor and any(rows % 128 for c in calls for _, rows, _ in c):
         raise SystemExit("bench: the tensor-core product needs rows in multiples of 128")
 
     def fused_pass():
@@ -1285,7 +1312,7 @@ def run_gemv(a):
         for (k, rows, cols), y in zip(c, yy):
             wf = dense[k].view(torch.bfloat16).view(rows, cols).double()
             ref = xf @ wf.t()
-            tol = (4.0 if batch > 8 else 2.0) * cols * 2.0 ** -24 * (xf.abs() @ wf.abs().t() + 64.0 * xf.abs().max())
+            tol = (4.0 if tensor else 2.0) * cols * 2.0 ** -24 * (xf.abs() @ wf.abs().t() + 64.0 * xf.abs().max())
             worst = max(worst, float(((y.double() - ref).abs() / tol).max()))
     if int(err.item()) != 0 or not worst <= 1.0:
         raise SystemExit(f"bench: fused GEMV out of tolerance (worst {worst:.3g} of the bound) or error flag set")
@@ -1366,7 +1393,7 @@ def run_gemv(a):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded device draws, synthetic/ recipe)",
         "config": {"workload": a.workload, "description": desc, "batch": batch, "matrices": len(specs),
                    "product": ("tensor cores: W decoded tile by tile into shared memory, tcgen05.mma (bs_fw_gemm)"
-                               if batch > 8 else "CUDA cores: W decoded in registers, fp32 FMA (bs_fw_gemv)"),
+                               if tensor else "CUDA cores: W decoded in registers, fp32 FMA (bs_fw_gemv)"),
                    "calls_per_step": len(calls), "n_weights": int(n_w), "fw_bytes": int(fw_bytes),
                    "bits_per_weight": round(8 * fw_bytes / n_w, 5),
                    "dense_cublas_ms_per_step": round(ms_dense / a.steps, 4),

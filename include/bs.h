@@ -443,7 +443,11 @@ bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_t batch, ui
  * memory in the tensor cores' operand layout and multiplies them with up to 64 tokens
  * (tcgen05.mma, BF16 operands, FP32 accumulation in tensor memory); larger batches take
  * several CTAs per row block, each decoding its rows again.
- *   rows must be a multiple of 128 and cols of 256 (else BS_E_ARG); batch is 1..2^20.
+ *   rows must be a multiple of 128 and cols of 256 (else BS_E_ARG); batch is 1..2^20; a matrix
+ *   of 2^32 / 128 tiles or more gives BS_E_SIZE.
+ *   A matrix with too few 128-row blocks to fill the GPU has its K range split over several
+ *   CTAs that add their parts into Y with atomic FP32 adds (Y is zeroed first, on stream), so
+ *   the last bits of such a product can differ from run to run.
  *   d_err: as for bs_fw_decode; bit 1 means that a wait inside the kernel ran out (the
  *          outputs of that CTA are then not written).
  * The FP32 sums follow the tensor cores' order, so they may differ from bs_fw_gemv's in the

@@ -135,3 +135,16 @@ def test_gemm_corrupt_tile_exc_is_flagged():
     torch.cuda.synchronize()
     assert int(err.item()) == 1
     assert torch.isfinite(y).all()
+
+
+def test_gemm_without_and_with_k_split():
+    # 297 row blocks fill the GPU (one CTA each, the sums written directly); 3 row blocks with
+    # a long K are split over many CTAs that add their parts with atomics
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    batch = 16
+    for rows, cols in ((128 * (2 * sms + 1), 256), (384, 256 * 56)):
+        w = _gauss(rows * cols, seed=rows).reshape(rows, cols)
+        x = _gauss(batch * cols, seed=cols, scale=1.0).reshape(batch, cols)
+        (y,), err, _ = _run([(w, x)], batch)
+        assert err == 0
+        _check(w, x, y)
