@@ -10,10 +10,14 @@
 // 11.4 instead of 16 bits per weight is the whole gain, so it runs on the CUDA cores (fp32
 // accumulation) and not on the tensor cores.
 //
-// Work split: a warp owns whole rows of W (row r covers tiles r*cols/256 .. +cols/256) and
-// walks them in the groups of 4 tiles of bs_fw.cu, through the same 3-slot cp.async ring.
+// Work split: the rows of W are shared evenly among the item's CTAs, whole rows each (row r
+// covers tiles r*cols/256 .. +cols/256). Inside a CTA the tiles of its rows, taken row after
+// row, are shared evenly among the 8 warps, so that no warp has more than one tile more than
+// another however few rows the CTA has (with whole rows per warp, a projection of 3584 rows
+// would leave 1.5 rows per warp and a quarter of the warps idle for the last row). A warp
+// walks its tiles in groups of up to 8 tiles inside one row, through a 3-slot cp.async ring.
 // Per tile and lane, the 8 decoded weights meet 8 entries of x (one 16-byte load per batch
-// row, served by L1/L2 since every warp reads the same x).
+// row; x is staged in shared memory when it is small, else served by L1/L2).
 //
 // Escapes: an escaped weight decodes to (table[0] << 7) | fraction, which is wrong only in its
 // sign and exponent. Lane e of the warp holds the group's e-th exception and adds
@@ -21,7 +25,9 @@
 // that owns the weight. Each slot carries the next group's tile_exc entries, so a group's
 // exception loads are issued one group early.
 //
-// Each row's sum is reduced over the warp (fixed order, no atomics) and written in fp32.
+// Each row piece's sum is reduced over the warp. A row held whole by one warp is written
+// directly; the pieces of a row split between warps are added in shared memory, in warp order,
+// once the CTA is done. So every output is a fixed sum (no atomics), written in fp32.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -45,7 +51,7 @@ struct FwGemvItem {
     uint32_t rows, cols;
     uint32_t n_exc;
     uint32_t cta_begin; // first CTA of this item in the launch
-    uint32_t ctas;      // CTAs of this item
+    uint32_t ctas;      // CTAs of this item (at most its rows)
     uint16_t table[16];
     uint32_t pad;
 };
@@ -80,13 +86,19 @@ struct GemvSlot {
 };
 template <int GROUP>
 constexpr uint32_t gemv_smem() { return 1024 + kGemvWarps * kFwStages * GemvSlot<GROUP>::bytes; }
+// x is staged in shared memory, once per CTA, when its batch rows take at most this many bytes:
+// then two CTAs still fit on an SM, and every load of x (the 16-byte loads of each tile and the
+// scattered loads of the escape corrections) is a shared-memory load.
+constexpr uint32_t kGemvXsMax = 32768;
 
-// One group's exception list as lane e holds it: entry e's column offset in the group and its
-// word, the count, and (for the path with more than 32) where each tile's entries start,
-// two 16-bit offsets per word.
+// One group's exception list as lane e holds it: the start of entry e's tile in the group
+// (gpos) and the entry's position byte and word as loaded (pos, word), the count, and (for the
+// path with more than 32) where each tile's entries start, two 16-bit offsets per word. The
+// position byte and the word are loaded one group before they are used and are not touched
+// until then, so the loads' latency hides behind a whole group of work.
 template <int GROUP>
 struct GemvExc {
-    uint32_t cnt = 0, e0 = 0, gpos = 0, word = 0;
+    uint32_t cnt = 0, e0 = 0, gpos = 0, pos = 0, word = 0;
     uint32_t d[(GROUP + 1) / 2] = {};
     __device__ uint32_t tile_of(uint32_t e) const {
         uint32_t t = 0;
@@ -96,13 +108,15 @@ struct GemvExc {
     }
 };
 
-// Batches above 2 are held to 2 CTAs per SM (at most 128 registers); 1-2 need fewer anyway.
-template <int BATCH, int GROUP>
-__global__ void __launch_bounds__(kGemvWarps * 32, BATCH <= 2 ? 1 : 2) fw_gemv_kernel(const __grid_constant__ FwGemvParams p) {
+// Two CTAs per SM (at most 128 registers a thread).
+// XS: x is copied into shared memory after the ring (kGemvXsMax bytes at most).
+template <int BATCH, int GROUP, bool XS>
+__global__ void __launch_bounds__(kGemvWarps * 32, 2) fw_gemv_kernel(const __grid_constant__ FwGemvParams p) {
     using Slot = GemvSlot<GROUP>;
     extern __shared__ __align__(16) uint8_t smem[];
     uint32_t* pair_tab = reinterpret_cast<uint32_t*>(smem);
     __shared__ int s_item;
+    __shared__ float s_first[kGemvWarps][BATCH], s_last[kGemvWarps][BATCH];
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
     if (tid == 0) {
         int lo = 0, hi = static_cast<int>(p.n_items) - 1;
@@ -117,38 +131,51 @@ __global__ void __launch_bounds__(kGemvWarps * 32, BATCH <= 2 ? 1 : 2) fw_gemv_k
     const FwGemvItem& it = p.item[s_item];
     for (uint32_t k = tid; k < 256; k += kGemvWarps * 32)
         pair_tab[k] = (uint32_t(it.table[k & 15u]) << 7) | (uint32_t(it.table[k >> 4]) << 23);
+    uint16_t* xs = reinterpret_cast<uint16_t*>(smem + 1024 + kGemvWarps * kFwStages * Slot::bytes);
+    if (XS) { // BATCH * cols BF16 values, a multiple of 256, in 16-byte pieces
+        const uint4* src = reinterpret_cast<const uint4*>(it.x);
+        for (uint32_t k = tid; k < BATCH * (it.cols >> 3); k += kGemvWarps * 32) reinterpret_cast<uint4*>(xs)[k] = __ldg(src + k);
+    }
     __syncthreads();
 
     const uint32_t rows = it.rows, cols = it.cols, tpr = cols >> 8; // tiles per row
-    const uint32_t gpr = (tpr + GROUP - 1) / GROUP;                 // groups per row
     const uint64_t nt = uint64_t(rows) * tpr;
     const uint32_t n_exc = it.n_exc;
     const FwOffsets o = fw_offsets(nt, n_exc);
     const uint8_t* fw = it.fw;
     const uint8_t* EP = fw + o.exc_pos;
     const uint16_t* EW = reinterpret_cast<const uint16_t*>(fw + o.exc_word);
-    const uint16_t* x = it.x;
+    const uint16_t* x = XS ? xs : it.x;
     const uint32_t esc_base = uint32_t(it.table[0]) << 7; // an escape decodes to this | its fraction
     const uint32_t cw0 = (3u * lane) >> 2, csh = (24u * lane) & 31u, cw1 = csh > 8 ? cw0 + 1 : cw0;
-    const uint32_t wg = (blockIdx.x - it.cta_begin) * kGemvWarps + warp; // warp within the item
-    const uint32_t nw = it.ctas * kGemvWarps;
-    const uint32_t my_rows = wg < rows ? (rows - wg + nw - 1) / nw : 0u;
-    const uint32_t groups = my_rows * gpr;
+    // The CTA's rows [r_begin, r_end) (whole rows, the item's rows shared evenly among its CTAs)
+    // and this warp's tiles [tb, te): the CTA's tiles, row after row, split evenly among its
+    // warps. Tile indices fit in 32 bits (a layout has at most 2^32 tiles).
+    const uint32_t cta = blockIdx.x - it.cta_begin;
+    const uint32_t r_begin = static_cast<uint32_t>(uint64_t(rows) * cta / it.ctas);
+    const uint32_t r_end = static_cast<uint32_t>(uint64_t(rows) * (cta + 1) / it.ctas);
+    const uint64_t cta_tiles = uint64_t(r_end - r_begin) * tpr;
+    auto warp_begin = [&](uint32_t w) { return r_begin * tpr + static_cast<uint32_t>(cta_tiles * w / kGemvWarps); };
+    const uint32_t tb = warp_begin(warp), te = warp_begin(warp + 1);
     uint8_t* wsm = smem + 1024 + warp * kFwStages * Slot::bytes;
     const uint32_t wsm_s = static_cast<uint32_t>(__cvta_generic_to_shared(wsm));
 
-    // The warp's groups in order: row wg, then wg + nw, ...; within a row, gi = 0 .. gpr-1
-    // covers tiles GROUP gi onwards. A Grp is one group's place; next() steps to the following
-    // one. The loop keeps the places of groups k .. k+3 in a rolling window. Tile indices fit
-    // in 32 bits (a layout has at most 2^32 tiles).
+    // The warp walks its tiles in groups: runs of at most GROUP tiles that stay inside one row.
+    // A Grp is one group's place (tiles k .. k+n-1 of row `row`, that is from tile
+    // row * tpr + k on; n = 0 past the end); next() steps to the following one. The loop keeps
+    // the places of groups j .. j+2 in a rolling window and works out j+3's when it needs it.
     struct Grp {
-        uint32_t row, gi;
+        uint32_t row, k, n;
     };
-    auto next = [&](Grp g) { return g.gi + 1 < gpr ? Grp{g.row, g.gi + 1} : Grp{g.row + nw, 0u}; };
-    auto tile0 = [&](Grp g) { return g.row * tpr + GROUP * g.gi; };
-    auto ntiles = [&](Grp g) {
-        const uint32_t left = tpr - GROUP * g.gi;
-        return left < GROUP ? left : static_cast<uint32_t>(GROUP);
+    auto tile0 = [&](Grp g) { return g.row * tpr + g.k; };
+    auto ntiles = [&](Grp g) { return g.n; };
+    auto run = [&](uint32_t row, uint32_t k) {
+        const uint32_t t = row * tpr + k, left = min(tpr - k, te - t);
+        return Grp{row, k, t < te ? min(left, static_cast<uint32_t>(GROUP)) : 0u};
+    };
+    auto next = [&](Grp g) {
+        if (g.n == 0) return g;
+        return g.k + g.n == tpr ? run(g.row + 1, 0u) : run(g.row, g.k + g.n);
     };
     // this lane's 16-byte share of a group's plane bytes, and of its exception arrays
     const uint8_t* gA = fw + o.a + 16 * lane;
@@ -207,7 +234,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32, BATCH <= 2 ? 1 : 2) fw_gemv_k
 #pragma unroll
         for (int g = 0; g < GROUP; g += 2) e.d[g >> 1] = (te[g] - te[0]) | ((te[g + 1] - te[0]) << 16);
         if (lane < e.cnt) {
-            e.gpos = (e.tile_of(lane) << 8) + EPl[e.e0];
+            e.gpos = e.tile_of(lane) << 8;
+            e.pos = EPl[e.e0];
             e.word = EWl[e.e0];
         }
         return e;
@@ -222,27 +250,28 @@ __global__ void __launch_bounds__(kGemvWarps * 32, BATCH <= 2 ? 1 : 2) fw_gemv_k
     float acc[BATCH];
 #pragma unroll
     for (int b = 0; b < BATCH; ++b) acc[b] = 0.f;
-    // places of groups k, k+1, k+2, k+3, and the slots of groups k and k+2
-    Grp g0{wg, 0u};
-    Grp g1 = next(g0), g2 = next(g1), g3 = next(g2);
+    // places of groups j, j+1, j+2, j+3, and the slots of groups j and j+2
+    Grp g0 = run(tb / tpr, tb % tpr);
+    Grp g1 = next(g0), g2 = next(g1);
     uint32_t slot_k = 0, slot_k2 = 2 * Slot::bytes; // byte offsets in the warp's ring
     // group 0's tile_exc entries go to slot 2 (free until group 2 is queued), as the oldest
     // commit, so that the first wait below covers them
-    if (groups > 0 && lane <= ntiles(g0)) fw_cp4(wsm_s + 2 * Slot::bytes + Slot::TE + 4 * lane, gT + 4 * uint64_t(tile0(g0)));
+    if (g0.n > 0 && lane <= g0.n) fw_cp4(wsm_s + 2 * Slot::bytes + Slot::TE + 4 * lane, gT + 4 * uint64_t(tile0(g0)));
     fw_commit();
-    issue(groups > 0, g0, groups > 1, g1, wsm_s);
-    issue(groups > 1, g1, groups > 2, g2, wsm_s + Slot::bytes);
+    issue(g0.n > 0, g0, g1.n > 0, g1, wsm_s);
+    issue(g1.n > 0, g1, g2.n > 0, g2, wsm_s + Slot::bytes);
     fw_wait_older();
     __syncwarp();
-    GemvExc<GROUP> cur = load_exc(groups > 0, g0, reinterpret_cast<const uint32_t*>(wsm + 2 * Slot::bytes + Slot::TE));
-    for (uint32_t k = 0; k < groups; ++k) {
-        issue(k + 2 < groups, g2, k + 3 < groups, g3, wsm_s + slot_k2);
-        fw_wait_older(); // group k has landed
+    GemvExc<GROUP> cur = load_exc(g0.n > 0, g0, reinterpret_cast<const uint32_t*>(wsm + 2 * Slot::bytes + Slot::TE));
+    while (g0.n > 0) {
+        const Grp g3 = next(g2);
+        issue(g2.n > 0, g2, g3.n > 0, g3, wsm_s + slot_k2);
+        fw_wait_older(); // group j has landed
         __syncwarp();
         const uint8_t* sl = wsm + slot_k;
-        const GemvExc<GROUP> nxt = load_exc(k + 1 < groups, g1, reinterpret_cast<const uint32_t*>(sl + Slot::TE));
-        const uint32_t gi = g0.gi, ng = ntiles(g0), row = g0.row;
-        const uint32_t col0 = gi * GROUP * kFwTile; // column of the group's first weight
+        const GemvExc<GROUP> nxt = load_exc(g1.n > 0, g1, reinterpret_cast<const uint32_t*>(sl + Slot::TE));
+        const uint32_t ng = g0.n, row = g0.row;
+        const uint32_t col0 = g0.k * kFwTile; // column of the group's first weight
         const uint32_t* sa = reinterpret_cast<const uint32_t*>(sl + Slot::A) + lane;
         const uint32_t* sb = reinterpret_cast<const uint32_t*>(sl + Slot::B) + lane;
         const uint32_t* sc0 = reinterpret_cast<const uint32_t*>(sl + Slot::C) + cw0;
@@ -252,7 +281,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32, BATCH <= 2 ? 1 : 2) fw_gemv_k
             const uint4 w = fw_octet(pair_tab, sa[32 * g], sb[32 * g], sc0[24 * g], sc1[24 * g], csh);
 #pragma unroll
             for (int b = 0; b < BATCH; ++b) {
-                const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xg + b * cols + 256 * g));
+                const uint4* xp = reinterpret_cast<const uint4*>(xg + b * cols + 256 * g);
+                const uint4 xv = XS ? *xp : __ldg(xp);
                 float s = acc[b];
                 s = fma_bf16x2(w.x, xv.x, s);
                 s = fma_bf16x2(w.y, xv.y, s);
@@ -267,16 +297,24 @@ __global__ void __launch_bounds__(kGemvWarps * 32, BATCH <= 2 ? 1 : 2) fw_gemv_k
         } else {
             for (uint32_t g = 0; g < ng; ++g) tile(static_cast<int>(g));
         }
-        if (lane < cur.cnt) correct(acc, col0 + cur.gpos, cur.word);
+        if (lane < cur.cnt) correct(acc, col0 + cur.gpos + cur.pos, cur.word);
         for (uint32_t e = lane + 32; e < cur.cnt; e += 32) // a group with more than 32 escapes
             correct(acc, col0 + (cur.tile_of(e) << 8) + EP[cur.e0 + e], EW[cur.e0 + e]);
-        if (gi + 1 == gpr) { // the row is complete
+        const bool row_end = g0.k + ng == tpr;
+        if (row_end || tile0(g0) + ng == te) { // the warp's piece of this row is complete
+            // a row that the warp holds whole is stored; a piece that starts inside the row
+            // goes to s_first, a piece that starts the row and ends inside it to s_last
+            const bool starts = row * tpr >= tb;
 #pragma unroll
             for (int b = 0; b < BATCH; ++b) {
                 float s = acc[b];
 #pragma unroll
                 for (int d = 16; d > 0; d >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, d);
-                if (lane == 0) it.y[size_t(b) * rows + row] = s;
+                if (lane == 0) {
+                    if (starts && row_end) it.y[size_t(b) * rows + row] = s;
+                    else if (!starts) s_first[warp][b] = s;
+                    else s_last[warp][b] = s;
+                }
                 acc[b] = 0.f;
             }
         }
@@ -285,11 +323,34 @@ __global__ void __launch_bounds__(kGemvWarps * 32, BATCH <= 2 ? 1 : 2) fw_gemv_k
         g0 = g1;
         g1 = g2;
         g2 = g3;
-        g3 = next(g3);
         slot_k = slot_k == 2 * Slot::bytes ? 0u : slot_k + Slot::bytes;
         slot_k2 = slot_k2 == 2 * Slot::bytes ? 0u : slot_k2 + Slot::bytes;
     }
     fw_wait<0>();
+    // Rows split among the CTA's warps: the warp whose piece starts the row adds, in warp
+    // order, the pieces of the following warps that start inside it (warps with no tiles are
+    // passed over), so every output is one fixed sum.
+    __syncthreads();
+    if (tid < kGemvWarps) {
+        const uint32_t w = tid, wb = warp_begin(w), we = warp_begin(w + 1);
+        if (we > wb) {
+            const uint32_t rl = (we - 1) / tpr; // the row of the warp's last tile
+            if (rl * tpr >= wb && we < (rl + 1) * tpr) {
+                float sum[BATCH];
+#pragma unroll
+                for (int b = 0; b < BATCH; ++b) sum[b] = s_last[w][b];
+                for (uint32_t v = w + 1; v < kGemvWarps; ++v) {
+                    const uint32_t vb = warp_begin(v), ve = warp_begin(v + 1);
+                    if (ve == vb) continue;
+                    if (vb / tpr != rl) break;
+#pragma unroll
+                    for (int b = 0; b < BATCH; ++b) sum[b] += s_first[v][b];
+                }
+#pragma unroll
+                for (int b = 0; b < BATCH; ++b) it.y[size_t(b) * rows + rl] = sum[b];
+            }
+        }
+    }
 }
 
 // The group size of a product: the largest of 8, 7 and 4 that divides the row's tile count,
@@ -299,30 +360,30 @@ inline int gemv_group_for(uint32_t cols) {
     return tpr % 8 == 0 ? 8 : tpr % 7 == 0 ? 7 : tpr % 4 == 0 ? 4 : 8;
 }
 
-// The kernel instance for (batch, group), its shared memory, and the CTAs that fit on an SM.
+// The kernel instance for (batch, group, x staged or not) and its shared memory, without x.
 struct GemvKernel {
     void (*fn)(const FwGemvParams);
     uint32_t smem;
 };
 template <int BATCH, int GROUP>
-GemvKernel gemv_kernel_of() {
-    return {fw_gemv_kernel<BATCH, GROUP>, gemv_smem<GROUP>()};
+GemvKernel gemv_kernel_of(bool xs) {
+    return {xs ? fw_gemv_kernel<BATCH, GROUP, true> : fw_gemv_kernel<BATCH, GROUP, false>, gemv_smem<GROUP>()};
 }
 template <int GROUP>
-GemvKernel gemv_kernel_b(uint32_t batch) {
+GemvKernel gemv_kernel_b(uint32_t batch, bool xs) {
     switch (batch) {
-    case 1: return gemv_kernel_of<1, GROUP>();
-    case 2: return gemv_kernel_of<2, GROUP>();
-    case 3: return gemv_kernel_of<3, GROUP>();
-    case 4: return gemv_kernel_of<4, GROUP>();
-    case 5: return gemv_kernel_of<5, GROUP>();
-    case 6: return gemv_kernel_of<6, GROUP>();
-    case 7: return gemv_kernel_of<7, GROUP>();
-    default: return gemv_kernel_of<8, GROUP>();
+    case 1: return gemv_kernel_of<1, GROUP>(xs);
+    case 2: return gemv_kernel_of<2, GROUP>(xs);
+    case 3: return gemv_kernel_of<3, GROUP>(xs);
+    case 4: return gemv_kernel_of<4, GROUP>(xs);
+    case 5: return gemv_kernel_of<5, GROUP>(xs);
+    case 6: return gemv_kernel_of<6, GROUP>(xs);
+    case 7: return gemv_kernel_of<7, GROUP>(xs);
+    default: return gemv_kernel_of<8, GROUP>(xs);
     }
 }
-GemvKernel gemv_kernel(uint32_t batch, int group) {
-    return group == 7 ? gemv_kernel_b<7>(batch) : group == 4 ? gemv_kernel_b<4>(batch) : gemv_kernel_b<8>(batch);
+GemvKernel gemv_kernel(uint32_t batch, int group, bool xs) {
+    return group == 7 ? gemv_kernel_b<7>(batch, xs) : group == 4 ? gemv_kernel_b<4>(batch, xs) : gemv_kernel_b<8>(batch, xs);
 }
 
 } // namespace
@@ -348,18 +409,21 @@ extern "C" bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     // One wave per group size: as many CTAs as fit on the GPU at once, shared among the
-    // items in proportion to their rows (a warp per row at a time, at least one row per warp),
-    // so that every warp walks many rows and its copy ring stays full. Items whose rows split
+    // items in proportion to their rows (at least one row per CTA). Items whose rows split
     // differently into groups run as separate launches.
     std::vector<FwGemvParams> params(1);
     FwGemvParams& p = params[0];
     p.err = d_err;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     for (int group : {8, 7, 4}) {
-        const GemvKernel kern = gemv_kernel(batch, group);
-        bool any = false;
-        for (int32_t k = 0; k < n && !any; ++k) any = items[k].info.n_elems && gemv_group_for(items[k].cols) == group;
-        if (!any) continue;
+        uint32_t max_cols = 0;
+        for (int32_t k = 0; k < n; ++k)
+            if (items[k].info.n_elems && gemv_group_for(items[k].cols) == group) max_cols = std::max(max_cols, items[k].cols);
+        if (max_cols == 0) continue;
+        const uint64_t x_bytes = uint64_t(2) * batch * max_cols;
+        const bool xs = x_bytes <= kGemvXsMax;
+        GemvKernel kern = gemv_kernel(batch, group, xs);
+        if (xs) kern.smem += static_cast<uint32_t>(x_bytes);
         cudaError_t e = cudaFuncSetAttribute(kern.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kern.smem));
         int per_sm = 0;
@@ -380,8 +444,7 @@ extern "C" bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_
                 const bs_fw_gemv_item& g = items[k];
                 if (g.info.n_elems == 0 || gemv_group_for(g.cols) != group) continue;
                 const uint64_t share = std::max<uint64_t>(1, wave * g.rows / std::max<uint64_t>(rows_here, 1));
-                const uint32_t c =
-                    static_cast<uint32_t>(std::min<uint64_t>(share, (g.rows + kGemvWarps - 1) / kGemvWarps));
+                const uint32_t c = static_cast<uint32_t>(std::min<uint64_t>(share, g.rows)); // a row at least per CTA
                 if (ctas + c >= (1ull << 31)) break;
                 FwGemvItem& it = p.item[p.n_items++];
                 it.fw = static_cast<const uint8_t*>(g.d_fw);

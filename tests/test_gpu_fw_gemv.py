@@ -74,6 +74,29 @@ def test_gemv_matches_oracle(rows, cols, batch):
     assert np.all(np.abs(y - ref) <= tol), float(np.max(np.abs(y - ref) / tol))
 
 
+@pytest.mark.parametrize("rows,cols", [(3584, 4096), (3584, 14336)])
+def test_gemv_rows_split_between_warps_are_exact_sums(rows, cols):
+    # o- and down-projection shapes: a CTA holds 12-13 rows and its 8 warps share their tiles,
+    # so most warps end inside a row and hand their piece to the warp that starts it; the
+    # outputs are fixed sums, the same bits on every call
+    batch = 2
+    w = _gauss(rows * cols, seed=rows ^ cols).reshape(rows, cols)
+    x = _gauss(batch * cols, seed=77, scale=1.0).reshape(batch, cols)
+    (y,), err, items = _run([(w, x)], batch)
+    assert err == 0
+    blob = oracle.fw_encode(w)
+    ref = oracle.fw_gemv(blob, rows, cols, x)
+    assert np.all(np.abs(y - ref) <= _tolerance(w, x, oracle.fw_info(blob)["table"][0]))
+    fw, info, _, _, xd, _ = items[0]
+    for _ in range(3):
+        y2 = torch.empty((batch, rows), dtype=torch.float32, device="cuda")
+        e2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+        bs.fw_gemv([(fw, info, rows, cols, xd, y2)], e2)
+        torch.cuda.synchronize()
+        assert int(e2.item()) == 0
+        assert np.array_equal(y2.cpu().numpy().view(np.uint32), y.astype(np.float32).view(np.uint32))
+
+
 def test_gemv_many_escapes_per_group():
     rows, cols = 40, 1024
     w = _gauss(rows * cols, seed=3, scale=1.0).reshape(rows, cols)
