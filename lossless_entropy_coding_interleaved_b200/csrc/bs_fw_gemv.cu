@@ -15,7 +15,7 @@
 // row, are shared evenly among the 8 warps, so that no warp has more than one tile more than
 // another however few rows the CTA has (with whole rows per warp, a projection of 3584 rows
 // would leave 1.5 rows per warp and a quarter of the warps idle for the last row). A warp
-// walks its tiles in groups of up to 8 tiles inside one row, through a 3-slot cp.async ring.
+// walks its tiles in groups of up to 14 or 16 tiles inside one row, through a 2-slot cp.async ring.
 // Per tile and lane, the 8 decoded weights meet 8 entries of x (one 16-byte load per batch
 // row; x is staged in shared memory when it is small, else served by L1/L2).
 //
@@ -76,36 +76,32 @@ __device__ __forceinline__ float fma_bf16x2(uint32_t w, uint32_t x, float acc) {
     return acc;
 }
 
-// A warp walks its rows in groups of GROUP tiles. One slot of its ring: plane A and B words
+// A warp walks its tiles in groups of up to GROUP tiles through a ring of two slots: while it
+// works on one group, the copies of the next are in flight. One slot: plane A and B words
 // (128 B per tile each), plane C (96 B per tile), and the tile_exc entries of the warp's
-// NEXT group (GROUP + 1 of them).
+// NEXT group (GROUP + 1 of them). Groups of 14 or 16 tiles keep the per-group work (copy
+// issue, exception list, bookkeeping) small per tile.
+constexpr int kGemvStages = 2;
 template <int GROUP>
 struct GemvSlot {
     static constexpr uint32_t A = 0, B = 128 * GROUP, C = 256 * GROUP, TE = 352 * GROUP;
     static constexpr uint32_t bytes = TE + ((4 * (GROUP + 1) + 15) / 16) * 16;
 };
 template <int GROUP>
-constexpr uint32_t gemv_smem() { return 1024 + kGemvWarps * kFwStages * GemvSlot<GROUP>::bytes; }
+constexpr uint32_t gemv_smem() { return 1024 + kGemvWarps * kGemvStages * GemvSlot<GROUP>::bytes; }
 // x is staged in shared memory, once per CTA, when its batch rows take at most this many bytes:
 // then two CTAs still fit on an SM, and every load of x (the 16-byte loads of each tile and the
 // scattered loads of the escape corrections) is a shared-memory load.
 constexpr uint32_t kGemvXsMax = 32768;
 
-// One group's exception list as lane e holds it: the start of entry e's tile in the group
-// (gpos) and the entry's position byte and word as loaded (pos, word), the count, and (for the
-// path with more than 32) where each tile's entries start, two 16-bit offsets per word. The
-// position byte and the word are loaded one group before they are used and are not touched
-// until then, so the loads' latency hides behind a whole group of work.
-template <int GROUP>
+// One group's exception list as the lanes hold it: the count, the index of its first entry, and
+// for entries lane and lane + 32 the start of the entry's tile in the group (gpos) and its
+// position byte and word as loaded (pos, word). The bytes and words are loaded one group
+// before they are used and are not touched until then, so the loads' latency hides behind a
+// whole group of work.
 struct GemvExc {
-    uint32_t cnt = 0, e0 = 0, gpos = 0, pos = 0, word = 0;
-    uint32_t d[(GROUP + 1) / 2] = {};
-    __device__ uint32_t tile_of(uint32_t e) const {
-        uint32_t t = 0;
-#pragma unroll
-        for (int g = 1; g < GROUP; ++g) t += e >= ((d[g >> 1] >> (16 * (g & 1))) & 0xFFFFu);
-        return t;
-    }
+    uint32_t cnt = 0, e0 = 0;
+    uint32_t gpos[2] = {0, 0}, pos[2] = {0, 0}, word[2] = {0, 0};
 };
 
 // Two CTAs per SM (at most 128 registers a thread).
@@ -118,6 +114,12 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) fw_gemv_kernel(const __gri
     __shared__ int s_item;
     __shared__ float s_first[kGemvWarps][BATCH], s_last[kGemvWarps][BATCH];
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
+    // Programmatic dependent launch: the next kernel of the stream may be scheduled as soon as
+    // every CTA of this one has started, so its CTAs take over the SMs that this one leaves
+    // and set up while this one finishes. Nothing is read from global memory before the wait
+    // below, which returns once the kernels before this one have completed and their writes
+    // are visible; until then only the kernel parameters are used.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (tid == 0) {
         int lo = 0, hi = static_cast<int>(p.n_items) - 1;
         while (lo < hi) {
@@ -131,12 +133,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) fw_gemv_kernel(const __gri
     const FwGemvItem& it = p.item[s_item];
     for (uint32_t k = tid; k < 256; k += kGemvWarps * 32)
         pair_tab[k] = (uint32_t(it.table[k & 15u]) << 7) | (uint32_t(it.table[k >> 4]) << 23);
-    uint16_t* xs = reinterpret_cast<uint16_t*>(smem + 1024 + kGemvWarps * kFwStages * Slot::bytes);
-    if (XS) { // BATCH * cols BF16 values, a multiple of 256, in 16-byte pieces
-        const uint4* src = reinterpret_cast<const uint4*>(it.x);
-        for (uint32_t k = tid; k < BATCH * (it.cols >> 3); k += kGemvWarps * 32) reinterpret_cast<uint4*>(xs)[k] = __ldg(src + k);
-    }
-    __syncthreads();
+    uint16_t* xs = reinterpret_cast<uint16_t*>(smem + 1024 + kGemvWarps * kGemvStages * Slot::bytes);
 
     const uint32_t rows = it.rows, cols = it.cols, tpr = cols >> 8; // tiles per row
     const uint64_t nt = uint64_t(rows) * tpr;
@@ -145,6 +142,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) fw_gemv_kernel(const __gri
     const uint8_t* fw = it.fw;
     const uint8_t* EP = fw + o.exc_pos;
     const uint16_t* EW = reinterpret_cast<const uint16_t*>(fw + o.exc_word);
+    const uint32_t* TE = reinterpret_cast<const uint32_t*>(fw + o.tile_exc);
     const uint16_t* x = XS ? xs : it.x;
     const uint32_t esc_base = uint32_t(it.table[0]) << 7; // an escape decodes to this | its fraction
     const uint32_t cw0 = (3u * lane) >> 2, csh = (24u * lane) & 31u, cw1 = csh > 8 ? cw0 + 1 : cw0;
@@ -157,7 +155,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) fw_gemv_kernel(const __gri
     const uint64_t cta_tiles = uint64_t(r_end - r_begin) * tpr;
     auto warp_begin = [&](uint32_t w) { return r_begin * tpr + static_cast<uint32_t>(cta_tiles * w / kGemvWarps); };
     const uint32_t tb = warp_begin(warp), te = warp_begin(warp + 1);
-    uint8_t* wsm = smem + 1024 + warp * kFwStages * Slot::bytes;
+    uint8_t* wsm = smem + 1024 + warp * kGemvStages * Slot::bytes;
     const uint32_t wsm_s = static_cast<uint32_t>(__cvta_generic_to_shared(wsm));
 
     // The warp walks its tiles in groups: runs of at most GROUP tiles that stay inside one row.
@@ -182,8 +180,6 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) fw_gemv_kernel(const __gri
     const uint8_t* gB = fw + o.b + 16 * lane;
     const uint8_t* gC = fw + o.c + 16 * lane;
     const uint8_t* gT = fw + o.tile_exc + 4 * lane;
-    const uint8_t* EPl = EP + lane;
-    const uint16_t* EWl = EW + lane;
     const uint16_t* xl = x + 8 * lane;
     // Queue the copies of a group (place g; h is the next group's place) into the slot at
     // shared address `slot`. Every call commits one cp.async group, empty or not.
@@ -205,9 +201,11 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) fw_gemv_kernel(const __gri
         }
         fw_commit();
     };
-    // A group's exception list (its tile_exc entries at ste): checked, then lane e loads entry e.
+    // A group's exception list (its tile_exc entries at ste): checked, then lane e loads
+    // entries e and e + 32. An entry's tile is the number of the group's later tiles whose
+    // first entry is at or before it.
     auto load_exc = [&](bool live, Grp place, const uint32_t* ste) {
-        GemvExc<GROUP> e;
+        GemvExc e;
         if (!live) return e;
         const uint32_t ng = ntiles(place);
         uint32_t te[GROUP + 1];
@@ -232,11 +230,16 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) fw_gemv_kernel(const __gri
         e.cnt = te[GROUP] - te[0];
         e.e0 = te[0];
 #pragma unroll
-        for (int g = 0; g < GROUP; g += 2) e.d[g >> 1] = (te[g] - te[0]) | ((te[g + 1] - te[0]) << 16);
-        if (lane < e.cnt) {
-            e.gpos = e.tile_of(lane) << 8;
-            e.pos = EPl[e.e0];
-            e.word = EWl[e.e0];
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t ei = te[0] + lane + 32 * h;
+            if (ei < te[GROUP]) {
+                uint32_t t = 0;
+#pragma unroll
+                for (int g = 1; g < GROUP; ++g) t += ei >= te[g];
+                e.gpos[h] = t << 8;
+                e.pos[h] = EP[ei];
+                e.word[h] = EW[ei];
+            }
         }
         return e;
     };
@@ -250,26 +253,33 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) fw_gemv_kernel(const __gri
     float acc[BATCH];
 #pragma unroll
     for (int b = 0; b < BATCH; ++b) acc[b] = 0.f;
-    // places of groups j, j+1, j+2, j+3, and the slots of groups j and j+2
+    // places of groups j and j+1, and the slot of group j (byte offset in the warp's ring)
     Grp g0 = run(tb / tpr, tb % tpr);
-    Grp g1 = next(g0), g2 = next(g1);
-    uint32_t slot_k = 0, slot_k2 = 2 * Slot::bytes; // byte offsets in the warp's ring
-    // group 0's tile_exc entries go to slot 2 (free until group 2 is queued), as the oldest
+    Grp g1 = next(g0);
+    uint32_t slot_k = 0;
+    // group 0's tile_exc entries go to slot 1 (free until group 1 is queued), as the oldest
     // commit, so that the first wait below covers them
-    if (g0.n > 0 && lane <= g0.n) fw_cp4(wsm_s + 2 * Slot::bytes + Slot::TE + 4 * lane, gT + 4 * uint64_t(tile0(g0)));
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (g0.n > 0 && lane <= g0.n) fw_cp4(wsm_s + Slot::bytes + Slot::TE + 4 * lane, gT + 4 * uint64_t(tile0(g0)));
     fw_commit();
     issue(g0.n > 0, g0, g1.n > 0, g1, wsm_s);
-    issue(g1.n > 0, g1, g2.n > 0, g2, wsm_s + Slot::bytes);
-    fw_wait_older();
+    // x is staged while the first group's copies are in flight
+    if (XS) { // BATCH * cols BF16 values, a multiple of 256, in 16-byte pieces
+        const uint4* src = reinterpret_cast<const uint4*>(it.x);
+        for (uint32_t k = tid; k < BATCH * (cols >> 3); k += kGemvWarps * 32) reinterpret_cast<uint4*>(xs)[k] = __ldg(src + k);
+    }
+    __syncthreads(); // the pair table and x are in place
+    fw_wait<1>();
     __syncwarp();
-    GemvExc<GROUP> cur = load_exc(g0.n > 0, g0, reinterpret_cast<const uint32_t*>(wsm + 2 * Slot::bytes + Slot::TE));
+    GemvExc cur = load_exc(g0.n > 0, g0, reinterpret_cast<const uint32_t*>(wsm + Slot::bytes + Slot::TE));
+    __syncwarp(); // every lane has read slot 1 before its first fill
     while (g0.n > 0) {
-        const Grp g3 = next(g2);
-        issue(g2.n > 0, g2, g3.n > 0, g3, wsm_s + slot_k2);
-        fw_wait_older(); // group j has landed
+        const Grp g2 = next(g1);
+        issue(g1.n > 0, g1, g2.n > 0, g2, wsm_s + (slot_k ^ Slot::bytes));
+        fw_wait<1>(); // all but the copies just queued: group j has landed
         __syncwarp();
         const uint8_t* sl = wsm + slot_k;
-        const GemvExc<GROUP> nxt = load_exc(g1.n > 0, g1, reinterpret_cast<const uint32_t*>(sl + Slot::TE));
+        const GemvExc nxt = load_exc(g1.n > 0, g1, reinterpret_cast<const uint32_t*>(sl + Slot::TE));
         const uint32_t ng = g0.n, row = g0.row;
         const uint32_t col0 = g0.k * kFwTile; // column of the group's first weight
         const uint32_t* sa = reinterpret_cast<const uint32_t*>(sl + Slot::A) + lane;
@@ -297,9 +307,14 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) fw_gemv_kernel(const __gri
         } else {
             for (uint32_t g = 0; g < ng; ++g) tile(static_cast<int>(g));
         }
-        if (lane < cur.cnt) correct(acc, col0 + cur.gpos + cur.pos, cur.word);
-        for (uint32_t e = lane + 32; e < cur.cnt; e += 32) // a group with more than 32 escapes
-            correct(acc, col0 + (cur.tile_of(e) << 8) + EP[cur.e0 + e], EW[cur.e0 + e]);
+        if (lane < cur.cnt) correct(acc, col0 + cur.gpos[0] + cur.pos[0], cur.word[0]);
+        if (lane + 32 < cur.cnt) correct(acc, col0 + cur.gpos[1] + cur.pos[1], cur.word[1]);
+        for (uint32_t e = lane + 64; e < cur.cnt; e += 32) { // a group with more than 64 escapes
+            const uint32_t ei = cur.e0 + e, t0 = tile0(g0);
+            uint32_t t = 0; // its tile, from the tile_exc entries checked in load_exc
+            for (uint32_t g = 1; g < ng; ++g) t += ei >= TE[t0 + g];
+            correct(acc, col0 + (t << 8) + EP[ei], EW[ei]);
+        }
         const bool row_end = g0.k + ng == tpr;
         if (row_end || tile0(g0) + ng == te) { // the warp's piece of this row is complete
             // a row that the warp holds whole is stored; a piece that starts inside the row
@@ -322,9 +337,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) fw_gemv_kernel(const __gri
         cur = nxt;
         g0 = g1;
         g1 = g2;
-        g2 = g3;
-        slot_k = slot_k == 2 * Slot::bytes ? 0u : slot_k + Slot::bytes;
-        slot_k2 = slot_k2 == 2 * Slot::bytes ? 0u : slot_k2 + Slot::bytes;
+        slot_k ^= Slot::bytes;
     }
     fw_wait<0>();
     // Rows split among the CTA's warps: the warp whose piece starts the row adds, in warp
@@ -353,12 +366,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) fw_gemv_kernel(const __gri
     }
 }
 
-// The group size of a product: the largest of 8, 7 and 4 that divides the row's tile count,
-// so that every group is whole (else 8, with a shorter last group per row).
-inline int gemv_group_for(uint32_t cols) {
-    const uint32_t tpr = cols / 256;
-    return tpr % 8 == 0 ? 8 : tpr % 7 == 0 ? 7 : tpr % 4 == 0 ? 4 : 8;
-}
+// The group size of a product: 14 when it divides the row's tile count, else 16 (groups are cut
+// at row ends, so any row length works).
+inline int gemv_group_for(uint32_t cols) { return (cols / 256) % 14 == 0 ? 14 : 16; }
 
 // The kernel instance for (batch, group, x staged or not) and its shared memory, without x.
 struct GemvKernel {
@@ -383,7 +393,7 @@ GemvKernel gemv_kernel_b(uint32_t batch, bool xs) {
     }
 }
 GemvKernel gemv_kernel(uint32_t batch, int group, bool xs) {
-    return group == 7 ? gemv_kernel_b<7>(batch, xs) : group == 4 ? gemv_kernel_b<4>(batch, xs) : gemv_kernel_b<8>(batch, xs);
+    return group == 14 ? gemv_kernel_b<14>(batch, xs) : gemv_kernel_b<16>(batch, xs);
 }
 
 } // namespace
@@ -415,7 +425,7 @@ extern "C" bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_
     FwGemvParams& p = params[0];
     p.err = d_err;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    for (int group : {8, 7, 4}) {
+    for (int group : {16, 14}) {
         uint32_t max_cols = 0;
         for (int32_t k = 0; k < n; ++k)
             if (items[k].info.n_elems && gemv_group_for(items[k].cols) == group) max_cols = std::max(max_cols, items[k].cols);
@@ -459,9 +469,19 @@ extern "C" bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_
                 ctas += c;
             }
             if (p.n_items == 0) continue;
-            kern.fn<<<static_cast<uint32_t>(ctas), kGemvWarps * 32, kern.smem, s>>>(p);
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(static_cast<uint32_t>(ctas));
+            cfg.blockDim = dim3(kGemvWarps * 32);
+            cfg.dynamicSmemBytes = kern.smem;
+            cfg.stream = s;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization; // see the kernel's wait
+            attr[0].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            e = cudaLaunchKernelEx(&cfg, kern.fn, p);
             count_launch();
-            e = cudaGetLastError();
+            if (e == cudaSuccess) e = cudaGetLastError();
             if (e != cudaSuccess) return cuda_status(e);
         }
     }
