@@ -21,6 +21,7 @@ bit-exact against the originals before timing. The JSON line carries:
 from __future__ import annotations
 
 import argparse
+import functools
 import concurrent.futures as cf
 import json
 import math
@@ -1288,7 +1289,9 @@ def run_gemv(a):
     tensor = a.product == "tensor" or (a.product == "auto" and batch > 8)
     if not tensor and batch > 8:
         raise SystemExit("bench: the CUDA-core product takes batches of 1..8")
-    product = bs.fw_gemm if tensor else bs.fw_gemv
+    # the layouts are written once, before the pass, and stay resident: the CUDA-core product
+    # may start copying them while the kernel before it finishes
+    product = bs.fw_gemm if tensor else functools.partial(bs.fw_gemv, layouts_resident=True)
     kernel = "fw_gemm_kernel" if tensor else "fw_gemv_kernel"
     if tensor and any(rows % 128 for c in calls for _, rows, _ in c):
         raise SystemExit("bench: the tensor-core product needs rows in multiples of 128")

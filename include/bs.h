@@ -432,8 +432,18 @@ typedef struct {
     float* d_y;
 } bs_fw_gemv_item;
 /* Computes every item's product, up to 384 items per launch; batch is 1..8 for all items.
- * d_err as for bs_fw_decode. Enqueued on stream. */
-bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_t batch, uint32_t* d_err, void* stream);
+ * d_err as for bs_fw_decode. Enqueued on stream.
+ * Each launch may be scheduled while the kernel before it on the stream is finishing
+ * (programmatic dependent launch): its CTAs take the SMs that kernel leaves. Without flags it
+ * reads and writes no global memory before that kernel has completed, so stream order holds
+ * as for any launch.
+ * flags: 0, or BS_FW_LAYOUTS_RESIDENT: the caller states that no work still in flight on the
+ * stream writes any item's layout (d_fw), as for weights written once and kept resident. The
+ * kernel then starts copying the layouts as soon as it is scheduled; it still waits for the
+ * preceding kernel to complete before it reads x or writes y or d_err. Other bits: BS_E_ARG. */
+#define BS_FW_LAYOUTS_RESIDENT 1u
+bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_t batch, uint32_t flags, uint32_t* d_err,
+                     void* stream);
 
 /* Y = X W^T for a batch of tokens on the tensor cores, W in the FW layout: the same products as
  * bs_fw_gemv (the same items, Y[b][r] = sum_k W[r][k] X[b][k]) for batches too large for the

@@ -25,6 +25,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbs.so")
 
 OK, E_ARG, E_FORMAT, E_VERSION, E_SIZE, E_CUDA, E_CORRUPT, E_NOMEM, E_UNSUPPORTED = range(9)
+FW_LAYOUTS_RESIDENT = 1  # bs_fw_gemv flag: no work in flight writes the layouts
 KIND_RANS, KIND_STORED, KIND_RAW, KIND_JOINT = 0, 1, 2, 3
 
 
@@ -134,7 +135,7 @@ def _load():
     L.bs_fw_write.argtypes = [P, u64, P, sz, ctypes.POINTER(FwInfo), P, sz, P]
     L.bs_fw_parse.argtypes = [P, sz, sz, ctypes.POINTER(FwInfo)]
     L.bs_fw_decode.argtypes = [i32, P, P, P, P, P, P]
-    L.bs_fw_gemv.argtypes = [i32, ctypes.POINTER(FwGemvItem), ctypes.c_uint32, P, P]
+    L.bs_fw_gemv.argtypes = [i32, ctypes.POINTER(FwGemvItem), ctypes.c_uint32, ctypes.c_uint32, P, P]
     L.bs_fw_gemm.argtypes = [i32, ctypes.POINTER(FwGemvItem), ctypes.c_uint32, P, P]
     for fn in ("bs_fw_measure", "bs_fw_write", "bs_fw_parse", "bs_fw_decode", "bs_fw_gemv", "bs_fw_gemm"):
         getattr(L, fn).restype = ctypes.c_int
@@ -630,11 +631,13 @@ def fw_gemm(products, err: torch.Tensor, stream=None):
     return [p[5] for p in products]
 
 
-def fw_gemv(products, err: torch.Tensor, stream=None):
+def fw_gemv(products, err: torch.Tensor, stream=None, layouts_resident: bool = False):
     """bs_fw_gemv: products is a sequence of (fw, info, rows, cols, x, y) with fw the layout of
     W (rows x cols), x a BF16 CUDA tensor [batch, cols] (or [cols]) and y a float32 CUDA
     tensor [batch, rows] (or [rows]); every x has the same batch (1..8). err: a zeroed int32
-    CUDA tensor of one element. Enqueued on the stream."""
+    CUDA tensor of one element. Enqueued on the stream. layouts_resident: BS_FW_LAYOUTS_RESIDENT,
+    a statement that no work in flight on the stream writes the layouts (resident weights), so
+    that their copies may start before the preceding kernel has finished."""
     n = len(products)
     arr = (FwGemvItem * max(n, 1))()
     batch = None
@@ -651,5 +654,6 @@ def fw_gemv(products, err: torch.Tensor, stream=None):
         arr[k].d_y = y.data_ptr()
     assert err.is_cuda and err.dtype == torch.int32 and err.numel() >= 1
     with torch.cuda.device(err.device):
-        _check(lib.bs_fw_gemv(n, arr, batch or 1, err.data_ptr(), _stream(stream)), "fw_gemv")
+        _check(lib.bs_fw_gemv(n, arr, batch or 1, FW_LAYOUTS_RESIDENT if layouts_resident else 0, err.data_ptr(),
+                              _stream(stream)), "fw_gemv")
     return [p[5] for p in products]

@@ -58,7 +58,7 @@ struct FwGemvItem {
 static_assert(sizeof(FwGemvItem) == 80, "FwGemvItem layout");
 struct FwGemvParams {
     uint32_t n_items;
-    uint32_t pad;
+    uint32_t layouts_resident; // BS_FW_LAYOUTS_RESIDENT: copy W before the dependency wait
     unsigned int* err; // device: bit 0 = an exception list failed its checks
     FwGemvItem item[kGemvMaxItems];
 };
@@ -116,9 +116,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) fw_gemv_kernel(const __gri
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
     // Programmatic dependent launch: the next kernel of the stream may be scheduled as soon as
     // every CTA of this one has started, so its CTAs take over the SMs that this one leaves
-    // and set up while this one finishes. Nothing is read from global memory before the wait
-    // below, which returns once the kernels before this one have completed and their writes
-    // are visible; until then only the kernel parameters are used.
+    // and set up while this one finishes. The wait below returns once the kernels before this
+    // one have completed and their writes are visible. Before it only the kernel parameters
+    // are used, and, when the caller has stated that no work in flight writes the layouts,
+    // the first group's copies of W are queued.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (tid == 0) {
         int lo = 0, hi = static_cast<int>(p.n_items) - 1;
@@ -259,10 +260,11 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) fw_gemv_kernel(const __gri
     uint32_t slot_k = 0;
     // group 0's tile_exc entries go to slot 1 (free until group 1 is queued), as the oldest
     // commit, so that the first wait below covers them
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (!p.layouts_resident) asm volatile("griddepcontrol.wait;" ::: "memory");
     if (g0.n > 0 && lane <= g0.n) fw_cp4(wsm_s + Slot::bytes + Slot::TE + 4 * lane, gT + 4 * uint64_t(tile0(g0)));
     fw_commit();
     issue(g0.n > 0, g0, g1.n > 0, g1, wsm_s);
+    if (p.layouts_resident) asm volatile("griddepcontrol.wait;" ::: "memory");
     // x is staged while the first group's copies are in flight
     if (XS) { // BATCH * cols BF16 values, a multiple of 256, in 16-byte pieces
         const uint4* src = reinterpret_cast<const uint4*>(it.x);
@@ -402,9 +404,10 @@ GemvKernel gemv_kernel(uint32_t batch, int group, bool xs) {
 using namespace bs;
 using namespace bs::fw;
 
-extern "C" bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_t batch, uint32_t* d_err,
-                                void* stream) {
+extern "C" bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_t batch, uint32_t flags,
+                                uint32_t* d_err, void* stream) {
     if (n < 0 || !d_err || (n > 0 && !items) || batch < 1 || batch > kGemvMaxBatch) return BS_E_ARG;
+    if (flags & ~BS_FW_LAYOUTS_RESIDENT) return BS_E_ARG;
     for (int32_t k = 0; k < n; ++k) {
         const bs_fw_gemv_item& g = items[k];
         if (!fw_info_ok(g.info) || uint64_t(g.rows) * g.cols != g.info.n_elems) return BS_E_ARG;
@@ -424,6 +427,7 @@ extern "C" bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_
     std::vector<FwGemvParams> params(1);
     FwGemvParams& p = params[0];
     p.err = d_err;
+    p.layouts_resident = (flags & BS_FW_LAYOUTS_RESIDENT) ? 1u : 0u;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     for (int group : {16, 14}) {
         uint32_t max_cols = 0;

@@ -196,3 +196,44 @@ def test_gemv_special_weights_follow_ieee():
     fin = np.isfinite(ref)
     tol = _tolerance(w, x, oracle.fw_info(oracle.fw_encode(w))["table"][0])
     assert np.all(np.abs(y[fin] - ref[fin]) <= tol[fin])
+
+
+@pytest.mark.parametrize("resident", [False, True])
+def test_gemv_back_to_back_calls_keep_stream_order(resident):
+    # A call may be scheduled while the one before it on the stream finishes. Here the second
+    # call's y is the first call's x (the same bytes), so the second must not write before the
+    # first has read; a third call then writes its y over the same bytes, so the last writer
+    # must win. Results are compared bit for bit with the calls made one at a time.
+    cols, rows1, rows2 = 3584, 4096, 1792  # y2 (1792 fp32) takes exactly x1's 3584 BF16 words
+    w1 = _gauss(rows1 * cols, seed=101).reshape(rows1, cols)
+    w2 = _gauss(rows2 * cols, seed=102).reshape(rows2, cols)
+    w3 = _gauss(rows2 * cols, seed=103).reshape(rows2, cols)
+    x1 = _dev(_gauss(cols, seed=104, scale=1.0))
+    x2 = _dev(_gauss(cols, seed=105, scale=1.0))
+    fws = [bs.fw_transcode(_dev(w.reshape(-1))) for w in (w1, w2, w3)]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def call(k, rows, x, y):
+        fw, info = fws[k]
+        bs.fw_gemv([(fw, info, rows, cols, x.view(1, cols), y.view(1, rows))], err, layouts_resident=resident)
+
+    alone = []
+    for k, rows, x in ((0, rows1, x1), (1, rows2, x2), (2, rows2, x2)):
+        y = torch.empty(rows, dtype=torch.float32, device="cuda")
+        call(k, rows, x, y)
+        torch.cuda.synchronize()
+        alone.append(y.clone())
+    shared = torch.empty(cols, dtype=torch.int16, device="cuda")   # x1, then y2 and y3
+    y1 = torch.empty(rows1, dtype=torch.float32, device="cuda")
+    for _ in range(20):
+        shared.copy_(x1)
+        call(0, rows1, shared, y1)
+        call(1, rows2, x2, shared.view(torch.float32))
+        torch.cuda.synchronize()
+        assert torch.equal(y1.view(torch.int32), alone[0].view(torch.int32))
+        assert torch.equal(shared.view(torch.float32).view(torch.int32), alone[1].view(torch.int32))
+        call(1, rows2, x2, shared.view(torch.float32))
+        call(2, rows2, x2, shared.view(torch.float32))
+        torch.cuda.synchronize()
+        assert torch.equal(shared.view(torch.float32).view(torch.int32), alone[2].view(torch.int32))
+    assert int(err.item()) == 0

@@ -110,3 +110,13 @@ def test_library_refuses_nonzero_reserved_fields_and_unaligned_names():
         assert e.value.code == bs.E_FORMAT
         with pytest.raises(oracle.OracleError):
             oracle.validate(bytes(b))
+
+
+def test_fw_gemv_refuses_unknown_flags_before_any_launch():
+    # argument checks run on the host before any CUDA call, so they work without a GPU
+    import lossless_entropy_coding_interleaved_b200 as bs
+    item = bs.FwGemvItem()
+    err = ctypes.c_uint32(0)
+    call = lambda flags: bs.lib.bs_fw_gemv(0, ctypes.byref(item), 1, flags, ctypes.addressof(err), None)
+    assert call(2) == bs.E_ARG and call(0x80000000) == bs.E_ARG
+    assert bs.lib.bs_fw_gemv(0, ctypes.byref(item), 9, 0, ctypes.addressof(err), None) == bs.E_ARG  # batch 1..8
