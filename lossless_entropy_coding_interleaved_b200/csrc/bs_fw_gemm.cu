@@ -10,28 +10,33 @@
 // accumulators in tensor memory).
 //
 // Work split ("swap AB": the weight rows are the MMA's M, the tokens its N):
-//  * A CTA owns 128 rows of W and up to 64 tokens and walks K in 256-wide slices (one FW tile
-//    of each row). The slice kb + 1's plane bytes (A, B, C: 352 bytes a tile), its tile_exc
-//    entries and the tokens' X slice are copied into shared memory with cp.async while slice
-//    kb is decoded, so the HBM reads run a slice ahead of the work (45 KiB in flight a CTA).
-//  * Its 16 warps decode slice kb from shared memory into the A stage (BF16, K-major, the
-//    128-byte swizzle of the MMA's canonical layout) and patch in its exceptions. A tile's
-//    exception entries are loaded into registers (four lanes a tile, up to 8 each) before the
-//    decode, so their latency hides behind it.
+//  * A CTA owns 128 rows of W and up to 64 tokens and walks its K range in slices of 128
+//    columns: half an FW tile of each row. A slice's plane bytes (A, B, C: 176 bytes a row),
+//    its tiles' tile_exc entries and the tokens' X slice are copied with cp.async into one of
+//    four slots, three slices ahead of the decode (about 70 KiB in flight a CTA). Each copying
+//    thread's cp.async completion arrives on the slot's mbarrier.
+//  * 16 warps decode a slice from its slot into one of two A stages (BF16, K-major, the
+//    128-byte swizzle of the MMA's canonical layout), patch in its exceptions, and arrive on
+//    the stage's mbarrier. A tile's exception entries are loaded into registers (four lanes a
+//    row, up to 3 each, the rest of a tile's entries read from memory) when its first half is
+//    decoded and serve both halves.
+//  * A 17th warp issues each slice's 8 MMAs (M = 128, N = tokens, K = 16 each) into a 128 x N
+//    FP32 accumulator in tensor memory once the stage is written, and commits them to the
+//    slot's completion barrier. That one barrier frees both the A stage (rewritten two slices
+//    later) and the slot (refilled with the slice three ahead). So the decode of a slice,
+//    the MMAs of the one before and the copies of the next three all overlap, with no
+//    barrier across the CTA inside the loop.
 //  * A matrix with too few row blocks to fill the GPU splits its K range over several CTAs
 //    per row block (up to about two CTAs per SM in all); they add their parts into Y, which
 //    bs_fw_gemm zeroes first, with atomic FP32 adds (so the sum's order, and its last bits,
 //    can differ between runs).
-//  * One thread issues the slice's 16 MMAs (M = 128, N = tokens, K = 16 each) into a 128 x N
-//    FP32 accumulator in tensor memory and commits them to an mbarrier. The A stage is
-//    rewritten only after that commit has arrived; at these N the MMAs take a small fraction
-//    of a slice's time, so one A stage suffices and the shared memory goes to the copies.
 //  * The epilogue reads the accumulator with tcgen05.ld (warps 0-7; warp w reads lanes
 //    32(w % 4)..+31, that is 32 rows of W, and 32 tokens from column 32(w / 4)) and writes
 //    Y[token][row] in FP32, 128 contiguous bytes per warp and token.
-//  * Every wait on an mbarrier is bounded. A wait that runs out sets bit 1 of the error word,
-//    skips the remaining work and still frees the tensor memory. A tile_exc entry out of order
-//    or past n_exc sets bit 0 and skips that tile's exceptions.
+//  * Every wait on an mbarrier is bounded. A wait that runs out, or sees that another thread's
+//    has, sets the CTA's abort flag and bit 1 of the error word; the threads then skip the
+//    remaining work and the tensor memory is still freed. A tile_exc entry out of order or
+//    past n_exc sets bit 0 and skips that tile's exceptions.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -47,25 +52,26 @@ namespace bs {
 namespace {
 using namespace fw;
 
-constexpr int kGemmWarps = 16;
-constexpr int kGemmThreads = kGemmWarps * 32;
-constexpr uint32_t kBM = 128;                     // rows of W per CTA: the MMA's M
-constexpr uint32_t kMaxNt = 64;                   // tokens per CTA: the MMA's N (a multiple of 16)
-constexpr uint32_t kAtomA = kBM * 128;            // one 64-wide K atom of the A stage (16 KiB)
-constexpr uint32_t kStageA = 4 * kAtomA;          // 128 rows x 256 K x 2 B
-constexpr uint32_t kStageB = 4 * kMaxNt * 128;    // up to 64 tokens x 256 K x 2 B
-// One slot of copied plane bytes: A and B planes (128 B a tile), C (96 B a tile), and each
-// tile's two tile_exc entries (8 B a tile).
-constexpr uint32_t kPlA = 0, kPlB = kBM * 128, kPlC = 2 * kBM * 128, kPlTE = kPlC + kBM * 96;
-constexpr uint32_t kSlot = kPlTE + kBM * 8;       // 46,080 B
-constexpr uint32_t kHead = 2048;                  // pair table, mbarrier, tensor-memory address
-// + 1 KiB of slack to align the A stage; then A, two B stages, two plane slots
-constexpr uint32_t kGemmSmem = kHead + 1024 + kStageA + 2 * kStageB + 2 * kSlot;
+constexpr uint32_t kDecWarps = 16;                  // warps that copy and decode
+constexpr uint32_t kDecThreads = kDecWarps * 32;
+constexpr uint32_t kGemmThreads = kDecThreads + 32;  // + the warp that issues the MMAs
+constexpr uint32_t kBM = 128;                        // rows of W per CTA: the MMA's M
+constexpr uint32_t kMaxNt = 64;                      // tokens per CTA: the MMA's N (a multiple of 16)
+constexpr uint32_t kAtomA = kBM * 128;               // one 64-wide K atom of an A stage (16 KiB)
+constexpr uint32_t kStageA = 2 * kAtomA;             // 128 rows x 128 K x 2 B
+constexpr uint32_t kSlots = 4;                       // copy slots: slices in flight + the one decoded
+// One slot: the half-tile plane bytes of the CTA's 128 rows (A and B 64 B, C 48 B a row), their
+// tiles' two tile_exc entries (8 B a row) and the tokens' X slice (N x 128 K x 2 B, swizzled).
+constexpr uint32_t kPlA = 0, kPlB = kBM * 64, kPlC = 2 * kBM * 64, kPlTE = kPlC + kBM * 48, kPlX = kPlTE + kBM * 8;
+constexpr uint32_t kSlotBytes = kPlX + kMaxNt * 256; // 39 KiB
+static_assert(kPlX % 1024 == 0 && kSlotBytes % 1024 == 0, "the swizzled X atoms start on 1 KiB");
+constexpr uint32_t kHead = 1024 + 128;               // pair table, mbarriers, tensor-memory address
+constexpr uint32_t kGemmSmem = kHead + 1024 + 2 * kStageA + kSlots * kSlotBytes; // + slack for 1 KiB alignment
 static_assert(kGemmSmem <= 232448, "shared memory of one CTA");
 constexpr uint32_t kTmemCols = 64;
-constexpr uint32_t kSpinLimit = 1u << 24;
+constexpr uint32_t kSpinLimit = 1u << 20;             // polls of an mbarrier wait (each up to 1 us)
 constexpr int kGemmMaxItems = 320;
-constexpr uint32_t kExcRegs = 8;                  // exception entries a lane holds in registers
+constexpr uint32_t kExcRegs = 3;                     // exception entries a lane holds in registers
 
 struct FwGemmItem {
     const uint8_t* fw;  // device: the layout of W
@@ -76,7 +82,7 @@ struct FwGemmItem {
     uint32_t cta_begin; // first CTA of this item in the launch
     uint32_t row_tiles; // rows / 128
     uint16_t ksplit;    // CTAs that share a row block's K range, each adding its part into Y
-    uint16_t kper;      // 256-wide K slices per such CTA
+    uint16_t kper;      // 256-wide K tiles per such CTA
     uint16_t table[16];
 };
 static_assert(sizeof(FwGemmItem) == 80, "FwGemmItem layout");
@@ -99,14 +105,27 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 __device__ __forceinline__ void mbar_init(uint32_t addr, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(addr), "r"(count) : "memory");
 }
-// Waits for the completion of the barrier's phase of this parity; false if it ran out.
-__device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity) {
+__device__ __forceinline__ void mbar_arrive(uint32_t addr) {
+    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}" ::"r"(addr) : "memory");
+}
+// The barrier's arrival for this thread fires once all of the thread's earlier cp.async copies
+// have landed (the barrier's count includes it).
+__device__ __forceinline__ void mbar_arrive_cp_async(uint32_t addr) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(addr) : "memory");
+}
+// Waits for the completion of the barrier's phase of this parity. Gives up, sets the CTA's
+// abort flag and returns false after kSpinLimit polls (about a second), or within 64 polls of
+// another thread giving up.
+__device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity, volatile int* abort_flag) {
     for (uint32_t i = 0; i < kSpinLimit; ++i) {
         uint32_t done;
-        asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        // the thread may sleep up to 1 us inside one poll, waking as soon as the phase completes
+        asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 1000;\n selp.u32 %0, 1, 0, p;\n}"
                      : "=r"(done) : "r"(addr), "r"(parity) : "memory");
         if (done) return true;
+        if ((i & 63u) == 63u && *abort_flag) return false;
     }
+    *abort_flag = 1;
     return false;
 }
 
@@ -120,19 +139,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
         s_abort = 0;
     }
     __syncthreads();
+    volatile int* abort_flag = &s_abort;
     const FwGemmItem& it = p.item[s_item];
     uint32_t* pair_tab = reinterpret_cast<uint32_t*>(smem);
     for (uint32_t k = tid; k < 256; k += kGemmThreads)
         pair_tab[k] = (uint32_t(it.table[k & 15u]) << 7) | (uint32_t(it.table[k >> 4]) << 23);
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t mbar = sbase + 1024;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 1040);
+    // mbarriers: slot_full[4] (the copies of a slot have landed: one arrival a copying thread),
+    // a_full[2] (an A stage is written: one arrival a decoding thread), mma_done[4] (the MMAs
+    // of the slice in a slot have completed: the commit)
+    const uint32_t bar_slot = sbase + 1024, bar_a = bar_slot + 8 * kSlots, bar_mma = bar_a + 16;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 1024 + 8 * (2 * kSlots + 2));
     const uint32_t sA = (sbase + kHead + 1023u) & ~1023u; // 1 KiB aligned, as the swizzle needs
+    const uint32_t sS = sA + 2 * kStageA;                  // slot k at sS + k * kSlotBytes
+    uint8_t* const gA = smem + (sA - sbase);
     if (tid == 0) {
-        mbar_init(mbar, 1);
+        for (uint32_t k = 0; k < kSlots; ++k) {
+            mbar_init(bar_slot + 8 * k, kDecThreads);
+            mbar_init(bar_mma + 8 * k, 1);
+        }
+        mbar_init(bar_a, kDecThreads);
+        mbar_init(bar_a + 8, kDecThreads);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) { // 64 columns of tensor memory: the 128 x (at most 64) FP32 accumulator
+    if (warp == kDecWarps) { // 64 columns of tensor memory: the 128 x (at most 64) FP32 accumulator
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(kTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -149,187 +179,218 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
     const uint32_t row0 = (rt % it.row_tiles) * kBM;
     const uint32_t nt = p.nt, tok0 = (rt / it.row_tiles) * nt, batch = p.batch;
     const uint32_t kbeg = kpart * it.kper, kend = min(tpr, kbeg + it.kper);
+    // the CTA's slices: half tiles, slice q is half q & 1 of tile kbeg + q / 2
+    const uint32_t nsl = kbeg < kend ? 2 * (kend - kbeg) : 0u;
     const bool split = it.ksplit > 1;
     const uint64_t n_tiles = uint64_t(rows) * tpr;
     const FwOffsets o = fw_offsets(n_tiles, it.n_exc);
     const uint8_t* fw = it.fw;
-    const uint8_t* EP = fw + o.exc_pos;
-    const uint16_t* EW = reinterpret_cast<const uint16_t*>(fw + o.exc_word);
-    const uint32_t cw0 = (3u * lane) >> 2, csh = (24u * lane) & 31u, cw1 = csh > 8 ? cw0 + 1 : cw0;
-    // M = 128, N = nt, BF16 x BF16 -> FP32, both operands K-major
-    const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((nt >> 3) << 17) | ((kBM >> 4) << 24);
-    const uint32_t sB0 = sA + kStageA, bbytes = 4 * nt * 128;      // B stages: sB0 + s * bbytes
-    const uint32_t sP0 = sB0 + 2 * bbytes;                           // plane slots: sP0 + s * kSlot
-    uint8_t* const pA = smem + (sA - sbase);
-
-    // The copies of a slice, split over the threads so that each thread's share has the same
-    // place in every slice: A and B plane pieces (16 bytes, 8 a tile, contiguous in the slot)
-    // at piece tid + kGemmThreads i, C plane pieces (6 a tile) likewise, and tile_exc entries.
-    // A slice kb's source is the same plus kb * 128 (A, B) or kb * 96 (C) bytes.
-    constexpr uint32_t kPiecesAB = kBM * 8 / kGemmThreads, kPiecesC = (kBM * 6 + kGemmThreads - 1) / kGemmThreads;
-    static_assert(kBM * 8 % kGemmThreads == 0, "pieces per thread");
-    uint32_t offAB[kPiecesAB], offC[kPiecesC]; // byte offsets of slice 0's pieces in the planes
-#pragma unroll
-    for (uint32_t i = 0; i < kPiecesAB; ++i) {
-        const uint32_t c = tid + kGemmThreads * i;
-        offAB[i] = (row0 + (c >> 3)) * tpr * 128u + (c & 7u) * 16u;
-    }
-#pragma unroll
-    for (uint32_t i = 0; i < kPiecesC; ++i) {
-        const uint32_t c = min(tid + kGemmThreads * i, kBM * 6 - 1); // the guard below skips the clamped ones
-        offC[i] = (row0 + c / 6) * tpr * 96u + (c % 6) * 16u;
-    }
-    const uint8_t* const planeA = fw + o.a;
-    const uint8_t* const planeB = fw + o.b;
-    const uint8_t* const planeC = fw + o.c;
-    const uint8_t* const tex = fw + o.tile_exc;
-
-    // Queue the copies of slice kb into plane slot kb & 1 and B stage kb & 1 (tokens past the
-    // batch read as 0).
-    auto issue = [&](uint32_t kb) {
-        const uint32_t sp = sP0 + (kb & 1u) * kSlot, sb = sB0 + (kb & 1u) * bbytes;
-#pragma unroll
-        for (uint32_t i = 0; i < kPiecesAB; ++i) {
-            const uint32_t c = tid + kGemmThreads * i;
-            cp_async16(sp + kPlA + 16 * c, planeA + offAB[i] + kb * 128u, 16u);
-            cp_async16(sp + kPlB + 16 * c, planeB + offAB[i] + kb * 128u, 16u);
-        }
-#pragma unroll
-        for (uint32_t i = 0; i < kPiecesC; ++i)
-            if (tid + kGemmThreads * i < kBM * 6)
-                cp_async16(sp + kPlC + 16 * (tid + kGemmThreads * i), planeC + offC[i] + kb * 96u, 16u);
-        if (tid < 2 * kBM) { // tile_exc[T] and tile_exc[T + 1] of row tid >> 1
-            const uint64_t T = uint64_t(row0 + (tid >> 1)) * tpr + kb + (tid & 1u);
-            fw_cp4(sp + kPlTE + 4 * tid, tex + 4 * T);
-        }
-        for (uint32_t id = tid; id < nt * 32; id += kGemmThreads) { // X: 16-byte chunks c of token t
-            const uint32_t t = id >> 5, c = id & 31u, tok = tok0 + t;
-            const uint32_t dst = sb + (c >> 3) * (nt * 128) + t * 128 + (((c & 7u) ^ (t & 7u)) << 4);
-            const uint16_t* src = tok < batch ? it.x + uint64_t(tok) * K + kb * 256 + c * 8 : it.x;
-            cp_async16(dst, src, tok < batch ? 16u : 0u);
-        }
-        cp_async_commit();
-    };
-
     bool ok = true;
-    if (kbeg < kend) issue(kbeg);
-    for (uint32_t kb = kbeg; kb < kend && ok; ++kb) {
-        const uint32_t s = kb & 1u, it_k = kb - kbeg; // it_k: this CTA's slice count so far
-        const uint32_t sp = sP0 + s * kSlot, sb = sB0 + s * bbytes;
-        const uint8_t* slot = smem + (sp - sbase);
-        cp_async_wait<0>(); // slice kb's copies (the only group in flight)
-        __syncthreads();
-        // this lane's share of the exceptions of row (lane & 7) of the warp's 8: entries
-        // e0 + 8 (lane >> 3) .. +7, as (position << 16) | word
-        constexpr uint32_t kRowsW = kBM / kGemmWarps; // 8 rows a warp
+
+    if (tid < kDecThreads) {
+        const uint8_t* EP = fw + o.exc_pos;
+        const uint16_t* EW = reinterpret_cast<const uint16_t*>(fw + o.exc_word);
+        // The copies of a slice, split over the threads so that each thread's share has the
+        // same place in every slice: A and B plane pieces (16 bytes, 4 a row), C pieces (3 a
+        // row), tile_exc entries (2 a row) and X pieces (16 a token). Slice q's plane source
+        // is slice 0's plus 64 q (A, B) or 48 q (C) bytes: the half tiles of a row are
+        // contiguous in each plane.
+        constexpr uint32_t kPcAB = kBM * 4 / kDecThreads, kPcC = (kBM * 3 + kDecThreads - 1) / kDecThreads;
+        constexpr uint32_t kPcTE = (kBM * 2 + kDecThreads - 1) / kDecThreads, kPcX = kMaxNt * 16 / kDecThreads;
+        static_assert(kBM * 4 % kDecThreads == 0 && kMaxNt * 16 % kDecThreads == 0, "pieces");
+        uint64_t srcAB[kPcAB], srcC[kPcC], srcTE[kPcTE];
+#pragma unroll
+        for (uint32_t i = 0; i < kPcAB; ++i) {
+            const uint32_t c = tid + kDecThreads * i;
+            srcAB[i] = (uint64_t(row0 + (c >> 2)) * tpr + kbeg) * 128u + 16u * (c & 3u);
+        }
+#pragma unroll
+        for (uint32_t i = 0; i < kPcC; ++i) {
+            const uint32_t c = min(tid + kDecThreads * i, kBM * 3 - 1); // the clamped ones are not copied
+            srcC[i] = (uint64_t(row0 + c / 3u) * tpr + kbeg) * 96u + 16u * (c % 3u);
+        }
+#pragma unroll
+        for (uint32_t i = 0; i < kPcTE; ++i) {
+            const uint32_t c = min(tid + kDecThreads * i, kBM * 2 - 1); // likewise
+            srcTE[i] = uint64_t(row0 + (c >> 1)) * tpr + kbeg + (c & 1u);
+        }
+        // X pieces: 16-byte chunk c of token t, at a swizzled place of the slot; tokens past
+        // the batch are zero-filled, pieces past nt tokens are not copied
+        uint32_t dstX[kPcX];
+        uint64_t srcX[kPcX];
+        uint32_t bytesX = 0, liveX = 0; // bit i: piece i reads 16 bytes; piece i is copied
+#pragma unroll
+        for (uint32_t i = 0; i < kPcX; ++i) {
+            const uint32_t id = tid + kDecThreads * i, t = id >> 4, c = id & 15u, tok = tok0 + t;
+            dstX[i] = kPlX + (c >> 3) * (nt * 128) + t * 128 + (((c & 7u) ^ (t & 7u)) << 4);
+            srcX[i] = tok < batch ? uint64_t(tok) * K + kbeg * 256 + c * 8 : 0;
+            bytesX |= (tok < batch ? 1u : 0u) << i;
+            liveX |= (t < nt ? 1u : 0u) << i;
+        }
+        const uint8_t* const planeA = fw + o.a;
+        const uint8_t* const planeB = fw + o.b;
+        const uint8_t* const planeC = fw + o.c;
+        const uint8_t* const tex = fw + o.tile_exc;
+        auto issue = [&](uint32_t q) {
+            const uint32_t sp = sS + (q % kSlots) * kSlotBytes;
+#pragma unroll
+            for (uint32_t i = 0; i < kPcAB; ++i) {
+                cp_async16(sp + kPlA + 16 * (tid + kDecThreads * i), planeA + srcAB[i] + 64u * q, 16u);
+                cp_async16(sp + kPlB + 16 * (tid + kDecThreads * i), planeB + srcAB[i] + 64u * q, 16u);
+            }
+#pragma unroll
+            for (uint32_t i = 0; i < kPcC; ++i)
+                cp_async16_if(tid + kDecThreads * i < kBM * 3, sp + kPlC + 16 * (tid + kDecThreads * i),
+                              planeC + srcC[i] + 48u * q, 16u);
+#pragma unroll
+            for (uint32_t i = 0; i < kPcTE; ++i)
+                if (tid + kDecThreads * i < kBM * 2) fw_cp4(sp + kPlTE + 4 * (tid + kDecThreads * i), tex + 4 * (srcTE[i] + (q >> 1)));
+#pragma unroll
+            for (uint32_t i = 0; i < kPcX; ++i)
+                cp_async16_if((liveX >> i) & 1u, sp + dstX[i], it.x + srcX[i] + 128u * q, ((bytesX >> i) & 1u) * 16u);
+            mbar_arrive_cp_async(bar_slot + 8 * (q % kSlots));
+        };
+        // decode: warp w writes rows 8w .. 8w+7, two at a time (lanes 0-15 and 16-31), lane
+        // octet j = lane & 15 of the half tile
+        const uint32_t j = lane & 15u, rsub = lane >> 4;
+        const uint32_t cw0 = (3u * j) >> 2, csh = (24u * j) & 31u, cw1 = csh > 8 ? cw0 + 1 : cw0;
+        // exceptions: lane holds entries e0 + kExcRegs (lane >> 3) .. of row er's tile, as
+        // (position << 16) | word, the first nex of them valid
+        constexpr uint32_t kRowsW = kBM / kDecWarps; // 8 rows a warp
         const uint32_t er = warp * kRowsW + (lane & (kRowsW - 1u));
-        const uint32_t* te = reinterpret_cast<const uint32_t*>(slot + kPlTE) + 2 * er;
-        const uint32_t e0 = te[0], e1 = te[1];
-        const bool e_ok = e0 <= e1 && e1 <= it.n_exc;
-        if (!e_ok && lane < kRowsW) atomicOr(p.err, 1u);
-        const uint32_t ebeg = e0 + kExcRegs * (lane / kRowsW), eend = e_ok ? e1 : e0;
-        uint32_t ex[kExcRegs];
+        uint32_t ex[kExcRegs], nex[kExcRegs];
+        uint32_t e0 = 0, eend = 0, ne0 = 0, neend = 0, n_ex = 0, n_nex = 0;
+        // checks a tile's tile_exc pair and queues the loads of this lane's share of its entries
+        auto load_exc = [&](uint32_t t0, uint32_t t1) {
+            const bool e_ok = t0 <= t1 && t1 <= it.n_exc;
+            if (!e_ok && lane < kRowsW) atomicOr(p.err, 1u);
+            ne0 = t0;
+            neend = e_ok ? t1 : t0;
+            const uint32_t ebeg = t0 + kExcRegs * (lane / kRowsW);
+            n_nex = ebeg < neend ? min(neend - ebeg, kExcRegs) : 0u;
 #pragma unroll
-        for (uint32_t i = 0; i < kExcRegs; ++i)
-            ex[i] = ebeg + i < eend ? (uint32_t(__ldg(EP + ebeg + i)) << 16) | __ldg(EW + ebeg + i) : 0xFFFFFFFFu;
-        // the planes of this warp's 8 tiles, read from the slot before anything waits
-        uint32_t pa[kRowsW], pb[kRowsW], pc0[kRowsW], pc1[kRowsW];
+            for (uint32_t i = 0; i < kExcRegs; ++i)
+                nex[i] = i < n_nex ? (uint32_t(__ldg(EP + ebeg + i)) << 16) | __ldg(EW + ebeg + i) : 0u;
+        };
+
+        for (uint32_t q = 0; q + 1 < kSlots && q < nsl; ++q) issue(q); // slices 0 .. kSlots - 2
+        for (uint32_t q = 0; q < nsl && ok; ++q) {
+            const uint32_t s = q % kSlots, st = q & 1u, h = q & 1u;
+            const uint8_t* slot = smem + (sS - sbase) + s * kSlotBytes;
+            if (!mbar_wait(bar_slot + 8 * s, (q / kSlots) & 1u, abort_flag)) { ok = false; break; }
+            if (h == 0) { // a new tile: its exception entries, both halves use them
+                const uint32_t* te = reinterpret_cast<const uint32_t*>(slot + kPlTE) + 2 * er;
+                load_exc(te[0], te[1]);
 #pragma unroll
-        for (uint32_t i = 0; i < kRowsW; ++i) {
-            const uint32_t r = warp * kRowsW + i;
-            pa[i] = *reinterpret_cast<const uint32_t*>(slot + kPlA + r * 128 + 4 * lane);
-            pb[i] = *reinterpret_cast<const uint32_t*>(slot + kPlB + r * 128 + 4 * lane);
-            const uint32_t* cp = reinterpret_cast<const uint32_t*>(slot + kPlC + r * 96);
-            pc0[i] = cp[cw0];
-            pc1[i] = cp[cw1];
-        }
-        // the MMAs of slice kb - 1 read the A stage and B stage s ^ 1: one thread waits for
-        // them, then slice kb + 1 is queued into the other slot and stage
-        if (tid == 0 && it_k >= 1 && !mbar_wait(mbar, (it_k - 1) & 1u)) {
-            atomicOr(p.err, 2u);
-            s_abort = 1;
-        }
-        __syncthreads();
-        if (kb + 1 < kend) issue(kb + 1);
-        // decode: warp w writes rows 8w .. 8w+7, lane j its 8 weights (chunk j of the row)
-#pragma unroll
-        for (uint32_t i = 0; i < kRowsW; ++i) {
-            const uint32_t r = warp * kRowsW + i;
-            const uint4 w = fw_octet(pair_tab, pa[i], pb[i], pc0[i], pc1[i], csh);
-            *reinterpret_cast<uint4*>(pA + (lane >> 3) * kAtomA + r * 128 + (((lane & 7u) ^ (r & 7u)) << 4)) = w;
-        }
-        __syncwarp();
-#pragma unroll
-        for (uint32_t i = 0; i < kExcRegs; ++i) {
-            if (ex[i] != 0xFFFFFFFFu) {
-                const uint32_t pos = ex[i] >> 16, j = pos >> 3;
-                *reinterpret_cast<uint16_t*>(pA + (j >> 3) * kAtomA + er * 128 + (((j & 7u) ^ (er & 7u)) << 4) +
-                                             2 * (pos & 7u)) = static_cast<uint16_t>(ex[i]);
+                for (uint32_t i = 0; i < kExcRegs; ++i) ex[i] = nex[i];
+                e0 = ne0;
+                eend = neend;
+                n_ex = n_nex;
             }
-        }
-        if (lane < kRowsW) // a tile with more than 32 exceptions: the rest, straight from memory
-            for (uint32_t e = e0 + (32 / kRowsW) * kExcRegs; e < eend; ++e) {
-                const uint32_t pos = __ldg(EP + e), j = pos >> 3;
-                *reinterpret_cast<uint16_t*>(pA + (j >> 3) * kAtomA + er * 128 + (((j & 7u) ^ (er & 7u)) << 4) +
-                                             2 * (pos & 7u)) = __ldg(EW + e);
+            uint32_t pa[4], pb[4], pc0[4], pc1[4];
+#pragma unroll
+            for (uint32_t i = 0; i < 4; ++i) {
+                const uint32_t r = warp * kRowsW + 2 * i + rsub;
+                pa[i] = *reinterpret_cast<const uint32_t*>(slot + kPlA + r * 64 + 4 * j);
+                pb[i] = *reinterpret_cast<const uint32_t*>(slot + kPlB + r * 64 + 4 * j);
+                const uint32_t* cp = reinterpret_cast<const uint32_t*>(slot + kPlC + r * 48);
+                pc0[i] = cp[cw0];
+                pc1[i] = cp[cw1];
             }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); // the stage is read by the tensor cores
-        __syncthreads();
-        if (s_abort) {
-            ok = false;
-            break;
+            // A stage st was last read by the MMAs of slice q - 2
+            if (q >= 2 && !mbar_wait(bar_mma + 8 * ((q - 2) % kSlots), ((q - 2) / kSlots) & 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            uint8_t* const stA = gA + st * kStageA;
+#pragma unroll
+            for (uint32_t i = 0; i < 4; ++i) {
+                const uint32_t r = warp * kRowsW + 2 * i + rsub;
+                const uint4 w = fw_octet(pair_tab, pa[i], pb[i], pc0[i], pc1[i], csh);
+                *reinterpret_cast<uint4*>(stA + (j >> 3) * kAtomA + r * 128 + (((j & 7u) ^ (r & 7u)) << 4)) = w;
+            }
+            __syncwarp();
+            // the exceptions of this half: positions 128 h .. 128 h + 127 of the tile
+#pragma unroll
+            for (uint32_t i = 0; i < kExcRegs; ++i) {
+                if (i >= n_ex) break;
+                const uint32_t pos = ex[i] >> 16;
+                if ((pos >> 7) == h) {
+                    const uint32_t jj = (pos >> 3) & 15u;
+                    *reinterpret_cast<uint16_t*>(stA + (jj >> 3) * kAtomA + er * 128 + (((jj & 7u) ^ (er & 7u)) << 4) +
+                                                 2 * (pos & 7u)) = static_cast<uint16_t>(ex[i]);
+                }
+            }
+            if (lane < kRowsW) // a tile with more than 32 exceptions: the rest, straight from memory
+                for (uint32_t e = e0 + (32 / kRowsW) * kExcRegs; e < eend; ++e) {
+                    const uint32_t pos = __ldg(EP + e);
+                    if ((pos >> 7) != h) continue;
+                    const uint32_t jj = (pos >> 3) & 15u;
+                    *reinterpret_cast<uint16_t*>(stA + (jj >> 3) * kAtomA + er * 128 + (((jj & 7u) ^ (er & 7u)) << 4) +
+                                                 2 * (pos & 7u)) = __ldg(EW + e);
+                }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); // read by the tensor cores
+            mbar_arrive(bar_a + 8 * st);
+            // refill: slice q + kSlots - 2 goes into the slot of slice q - 2, whose MMAs have
+            // completed (waited for above); slice q - 1's MMAs may still be running
+            const uint32_t qn = q + kSlots - 2;
+            if (qn < nsl && qn >= kSlots - 1) issue(qn);
         }
-        if (tid == 0) {
+        asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (tid == kDecThreads) {
+        // the MMA thread: M = 128, N = nt, BF16 x BF16 -> FP32, both operands K-major
+        const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((nt >> 3) << 17) | ((kBM >> 4) << 24);
+        for (uint32_t q = 0; q < nsl; ++q) {
+            const uint32_t st = q & 1u, s = q % kSlots;
+            if (!mbar_wait(bar_a + 8 * st, (q >> 1) & 1u, abort_flag)) { ok = false; break; }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint32_t a0 = sA + st * kStageA, b0 = sS + s * kSlotBytes + kPlX;
 #pragma unroll
-            for (uint32_t kk = 0; kk < 16; ++kk) { // K = 16 per MMA: atom kk / 4, 32 bytes per step inside it
-                const uint64_t ad = sw128_desc(sA + (kk >> 2) * kAtomA + (kk & 3u) * 32);
-                const uint64_t bd = sw128_desc(sb + (kk >> 2) * (nt * 128) + (kk & 3u) * 32);
-                const uint32_t acc = (it_k | kk) != 0;
+            for (uint32_t kk = 0; kk < 8; ++kk) { // K = 16 per MMA: atom kk / 4, 32 bytes per step inside it
+                const uint64_t ad = sw128_desc(a0 + (kk >> 2) * kAtomA + (kk & 3u) * 32);
+                const uint64_t bd = sw128_desc(b0 + (kk >> 2) * (nt * 128) + (kk & 3u) * 32);
+                const uint32_t acc = (q | kk) != 0;
                 asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
                              " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}"
                              ::"r"(tmem), "l"(ad), "l"(bd), "r"(idesc), "r"(acc) : "memory");
             }
-            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_mma + 8 * s)
                          : "memory");
         }
     }
-    cp_async_wait<0>();
     // The last commit covers every MMA before it.
-    if (ok && kbeg < kend) {
-        if (!mbar_wait(mbar, (kend - kbeg - 1) & 1u)) {
-            atomicOr(p.err, 2u);
-            ok = false;
-        }
-    }
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    if (ok && kbeg < kend && warp < 8) {
-        // warp w reads tensor-memory lanes 32 (w % 4) .. +31 (rows of W) and columns (tokens)
-        // 32 (w / 4) .. +31 of the accumulator
-        const uint32_t quarter = warp & 3u, half = warp >> 2;
-        const uint32_t row = row0 + quarter * 32 + lane;
-        for (uint32_t cb = half * 32; cb < half * 32 + 32 && cb < nt; cb += 16) {
-            uint32_t v[16];
-            const uint32_t taddr = tmem + ((quarter * 32) << 16) + cb;
-            asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-                         : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-                           "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-                         : "r"(taddr));
-            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    if (warp < 8 && nsl > 0) {
+        ok = ok && !*abort_flag && mbar_wait(bar_mma + 8 * ((nsl - 1) % kSlots), ((nsl - 1) / kSlots) & 1u, abort_flag);
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        if (ok) {
+            // warp w reads tensor-memory lanes 32 (w % 4) .. +31 (rows of W) and columns (tokens)
+            // 32 (w / 4) .. +31 of the accumulator
+            const uint32_t quarter = warp & 3u, half = warp >> 2;
+            const uint32_t row = row0 + quarter * 32 + lane;
+            for (uint32_t cb = half * 32; cb < half * 32 + 32 && cb < nt; cb += 16) {
+                uint32_t v[16];
+                const uint32_t taddr = tmem + ((quarter * 32) << 16) + cb;
+                asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+                             : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                               "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+                             : "r"(taddr));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-            for (uint32_t q = 0; q < 16; ++q) {
-                const uint32_t tok = tok0 + cb + q;
-                if (tok < batch) {
-                    float* dst = it.y + uint64_t(tok) * rows + row;
-                    if (split) atomicAdd(dst, __uint_as_float(v[q])); // Y was zeroed; parts add up
-                    else *dst = __uint_as_float(v[q]);
+                for (uint32_t q = 0; q < 16; ++q) {
+                    const uint32_t tok = tok0 + cb + q;
+                    if (tok < batch) {
+                        float* dst = it.y + uint64_t(tok) * rows + row;
+                        if (split) atomicAdd(dst, __uint_as_float(v[q])); // Y was zeroed; parts add up
+                        else *dst = __uint_as_float(v[q]);
+                    }
                 }
             }
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
-    if (warp == 0)
+    if (tid == 0 && *abort_flag) atomicOr(p.err, 2u);
+    if (warp == kDecWarps)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
 }
 
