@@ -449,15 +449,17 @@ bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_t batch, ui
  * bs_fw_gemv (the same items, Y[b][r] = sum_k W[r][k] X[b][k]) for batches too large for the
  * CUDA cores. Source: the NVLC card's runtime keeps the compressed weights resident and no
  * decoded-weight cache (its runtime accounting and DGX Spark tables); the kernel is this
- * library's. Each CTA decodes 128 rows of W, one 256-wide slice of K at a time, into shared
- * memory in the tensor cores' operand layout and multiplies them with up to 64 tokens
- * (tcgen05.mma, BF16 operands, FP32 accumulation in tensor memory); larger batches take
- * several CTAs per row block, each decoding its rows again.
+ * library's. W is decoded in blocks of 128 rows, 128 columns of K at a time, into shared
+ * memory in the tensor cores' operand layout and multiplied with up to 64 tokens
+ * (tcgen05.mma, BF16 operands, FP32 accumulation in tensor memory); larger batches decode
+ * each row block once per 64 tokens.
  *   rows must be a multiple of 128 and cols of 256 (else BS_E_ARG); batch is 1..2^20; a matrix
  *   of 2^32 / 128 tiles or more gives BS_E_SIZE.
- *   A matrix with too few 128-row blocks to fill the GPU has its K range split over several
- *   CTAs that add their parts into Y with atomic FP32 adds (Y is zeroed first, on stream), so
- *   the last bits of such a product can differ from run to run.
+ *   The work (row blocks x K tiles x token blocks) is shared evenly by one wave of CTAs, so a
+ *   row block's K range can be split between CTAs. Every item's Y is zeroed first (on stream)
+ *   and split row blocks add their parts with atomic FP32 adds; a part sum over two CTAs does
+ *   not depend on their order, but one over three or more (small launches) can differ in its
+ *   last bits from run to run.
  *   d_err: as for bs_fw_decode; bit 1 means that a wait inside the kernel ran out (the
  *          outputs of that CTA are then not written).
  * The FP32 sums follow the tensor cores' order, so they may differ from bs_fw_gemv's in the

@@ -10,8 +10,8 @@
 // accumulators in tensor memory).
 //
 // Work split ("swap AB": the weight rows are the MMA's M, the tokens its N):
-//  * A CTA owns 128 rows of W and up to 64 tokens and walks its K range in slices of 128
-//    columns: half an FW tile of each row. A slice's plane bytes (A, B, C: 176 bytes a row),
+//  * A segment's 128 rows of W and up to 64 tokens are walked in slices of 128 columns: half
+//    an FW tile of each row. A slice's plane bytes (A, B, C: 176 bytes a row),
 //    its tiles' tile_exc entries and the tokens' X slice are copied with cp.async into one of
 //    four slots, three slices ahead of the decode (about 70 KiB in flight a CTA). Each copying
 //    thread's cp.async completion arrives on the slot's mbarrier.
@@ -26,10 +26,15 @@
 //    later) and the slot (refilled with the slice three ahead). So the decode of a slice,
 //    the MMAs of the one before and the copies of the next three all overlap, with no
 //    barrier across the CTA inside the loop.
-//  * A matrix with too few row blocks to fill the GPU splits its K range over several CTAs
-//    per row block (up to about two CTAs per SM in all); they add their parts into Y, which
-//    bs_fw_gemm zeroes first, with atomic FP32 adds (so the sum's order, and its last bits,
-//    can differ between runs).
+//  * Stream-K work split: a launch's units (item, token tile, 128-row block, FW tile) are shared
+//    evenly by one wave of CTAs, one per SM, so no SM idles through a partial last wave. A
+//    CTA walks its units as runs of one row block's tiles (segments). Segment g accumulates in
+//    tensor-memory accumulator g & 1, so the read-out of one segment overlaps the MMAs of the
+//    next. A segment that covers its row block's whole K range stores its sums; one that
+//    covers part of it adds them into Y (zeroed by bs_fw_gemm first) with atomic FP32 adds. A
+//    row block split between two CTAs gets two such parts, whose sum does not depend on their
+//    order; one split among three or more CTAs (tiny launches) can differ in its last bits
+//    from run to run.
 //  * The epilogue reads the accumulator with tcgen05.ld (warps 0-7; warp w reads lanes
 //    32(w % 4)..+31, that is 32 rows of W, and 32 tokens from column 32(w / 4)) and writes
 //    Y[token][row] in FP32, 128 contiguous bytes per warp and token.
@@ -65,34 +70,44 @@ constexpr uint32_t kSlots = 4;                       // copy slots: slices in fl
 constexpr uint32_t kPlA = 0, kPlB = kBM * 64, kPlC = 2 * kBM * 64, kPlTE = kPlC + kBM * 48, kPlX = kPlTE + kBM * 8;
 constexpr uint32_t kSlotBytes = kPlX + kMaxNt * 256; // 39 KiB
 static_assert(kPlX % 1024 == 0 && kSlotBytes % 1024 == 0, "the swizzled X atoms start on 1 KiB");
-constexpr uint32_t kHead = 1024 + 128;               // pair table, mbarriers, tensor-memory address
+constexpr uint32_t kMaxSegs = 64;                     // segments (runs of one row block's tiles) a CTA
+constexpr uint32_t kTabs = 2;                         // pair tables a CTA holds (items it spans)
+// pair tables, mbarriers, tensor-memory address
+constexpr uint32_t kHead = kTabs * 1024 + 128;
 constexpr uint32_t kGemmSmem = kHead + 1024 + 2 * kStageA + kSlots * kSlotBytes; // + slack for 1 KiB alignment
-static_assert(kGemmSmem <= 232448, "shared memory of one CTA");
-constexpr uint32_t kTmemCols = 64;
+static_assert(kGemmSmem + kMaxSegs * 32 + 64 <= 232448, "shared memory of one CTA");
+constexpr uint32_t kTmemCols = 128;                   // two 128 x 64 FP32 accumulators
 constexpr uint32_t kSpinLimit = 1u << 20;             // polls of an mbarrier wait (each up to 1 us)
 constexpr int kGemmMaxItems = 320;
-constexpr uint32_t kExcRegs = 3;                     // exception entries a lane holds in registers
+constexpr uint32_t kExcRegs = 3;                      // exception entries a lane holds in registers
 
 struct FwGemmItem {
-    const uint8_t* fw;  // device: the layout of W
-    const uint16_t* x;  // device: BF16 [batch][cols]
-    float* y;           // device: FP32 [batch][rows]
+    const uint8_t* fw;   // device: the layout of W
+    const uint16_t* x;   // device: BF16 [batch][cols]
+    float* y;            // device: FP32 [batch][rows], zeroed before the launch
     uint32_t rows, cols;
     uint32_t n_exc;
-    uint32_t cta_begin; // first CTA of this item in the launch
-    uint32_t row_tiles; // rows / 128
-    uint16_t ksplit;    // CTAs that share a row block's K range, each adding its part into Y
-    uint16_t kper;      // 256-wide K tiles per such CTA
+    uint32_t unit_begin; // first unit of this item in the launch
+    uint32_t row_tiles;  // rows / 128
+    uint32_t pad;
     uint16_t table[16];
 };
 static_assert(sizeof(FwGemmItem) == 80, "FwGemmItem layout");
 struct FwGemmParams {
     uint32_t n_items;
     uint32_t batch;       // tokens
-    uint32_t nt;          // tokens per CTA: min(64, batch rounded up to 16)
+    uint32_t nt;          // tokens per token tile: min(64, batch rounded up to 16)
     uint32_t token_tiles; // ceil(batch / nt)
+    uint32_t units;       // units of the launch: (item, token tile, row block, tile), in that order
+    uint32_t ctas;        // CTA c takes units [c * units / ctas, (c + 1) * units / ctas)
     unsigned int* err;    // bit 0: an exception list failed its checks; bit 1: an mbarrier wait ran out
     FwGemmItem item[kGemmMaxItems];
+};
+
+// A run of consecutive units of one (item, token tile, row block): tiles kt0 .. kt0 + n - 1 of
+// the row block, slices q0 .. q0 + 2n - 1 of the CTA.
+struct GemmSeg {
+    uint32_t item, row0, tok0, kt0, n, q0, tab, full; // full: the run covers the whole K range
 };
 
 // Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzle: rows of 128
@@ -131,28 +146,65 @@ __device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity, volati
 
 __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_constant__ FwGemmParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
-    __shared__ int s_item;
-    __shared__ int s_abort;
+    __shared__ GemmSeg s_seg[kMaxSegs];
+    __shared__ int s_nseg, s_abort;
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
+    const uint32_t nt = p.nt, batch = p.batch;
     if (tid == 0) {
-        find_item(p, &s_item);
+        // this CTA's units, cut into segments; the host keeps every CTA within kMaxSegs
+        // segments and kTabs items
         s_abort = 0;
+        const uint32_t u0 = static_cast<uint32_t>(uint64_t(p.units) * blockIdx.x / p.ctas);
+        const uint32_t u1 = static_cast<uint32_t>(uint64_t(p.units) * (blockIdx.x + 1) / p.ctas);
+        int k = 0, hi = static_cast<int>(p.n_items) - 1;
+        while (k < hi) { // the item holding u0
+            const int mid = (k + hi + 1) >> 1;
+            if (p.item[mid].unit_begin <= u0) k = mid;
+            else hi = mid - 1;
+        }
+        uint32_t n = 0, q = 0, tab = 0, u = u0;
+        int first_item = k;
+        while (u < u1 && n < kMaxSegs) {
+            while (k + 1 < static_cast<int>(p.n_items) && p.item[k + 1].unit_begin <= u) ++k;
+            const FwGemmItem& it = p.item[k];
+            const uint32_t tpr = it.cols >> 8, l = u - it.unit_begin, per_tt = it.row_tiles * tpr;
+            const uint32_t tt = l / per_tt, rb = (l % per_tt) / tpr, kt = l % tpr;
+            const uint32_t len = min(u1 - u, tpr - kt);
+            if (k != first_item) tab = 1;
+            s_seg[n] = GemmSeg{static_cast<uint32_t>(k), rb * kBM, tt * nt, kt, len, q, tab, (kt == 0 && len == tpr) ? 1u : 0u};
+            ++n;
+            q += 2 * len;
+            u += len;
+        }
+        if (u < u1) s_abort = 1; // more runs than kMaxSegs: the host's bound was not kept
+        s_nseg = static_cast<int>(n);
     }
     __syncthreads();
     volatile int* abort_flag = &s_abort;
-    const FwGemmItem& it = p.item[s_item];
-    uint32_t* pair_tab = reinterpret_cast<uint32_t*>(smem);
-    for (uint32_t k = tid; k < 256; k += kGemmThreads)
-        pair_tab[k] = (uint32_t(it.table[k & 15u]) << 7) | (uint32_t(it.table[k >> 4]) << 23);
+    const uint32_t nseg = static_cast<uint32_t>(s_nseg);
+    const uint32_t nsl = nseg ? s_seg[nseg - 1].q0 + 2 * s_seg[nseg - 1].n : 0u; // the CTA's slices
+    // pair table t (t < kTabs): the first segment's item, and the next item if the CTA spans two
+    for (uint32_t t = 0; t < kTabs && nseg > 0; ++t) {
+        uint32_t item = s_seg[0].item;
+        for (uint32_t g = 0; g < nseg; ++g)
+            if (s_seg[g].tab == t) { item = s_seg[g].item; break; }
+        uint32_t* pt = reinterpret_cast<uint32_t*>(smem) + 256 * t;
+        const FwGemmItem& it = p.item[item];
+        for (uint32_t k = tid; k < 256; k += kGemmThreads)
+            pt[k] = (uint32_t(it.table[k & 15u]) << 7) | (uint32_t(it.table[k >> 4]) << 23);
+    }
     const uint32_t sbase = smem_u32(smem);
     // mbarriers: slot_full[4] (the copies of a slot have landed: one arrival a copying thread),
     // a_full[2] (an A stage is written: one arrival a decoding thread), mma_done[4] (the MMAs
-    // of the slice in a slot have completed: the commit)
-    const uint32_t bar_slot = sbase + 1024, bar_a = bar_slot + 8 * kSlots, bar_mma = bar_a + 16;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 1024 + 8 * (2 * kSlots + 2));
+    // of the slice in a slot have completed: the commit), d_free[2] (an accumulator has been
+    // read out: one arrival an epilogue thread)
+    const uint32_t bar_slot = sbase + kTabs * 1024, bar_a = bar_slot + 8 * kSlots, bar_mma = bar_a + 16;
+    const uint32_t bar_d = bar_mma + 8 * kSlots;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTabs * 1024 + 8 * (2 * kSlots + 4));
     const uint32_t sA = (sbase + kHead + 1023u) & ~1023u; // 1 KiB aligned, as the swizzle needs
     const uint32_t sS = sA + 2 * kStageA;                  // slot k at sS + k * kSlotBytes
     uint8_t* const gA = smem + (sA - sbase);
+    constexpr uint32_t kEpiThreads = 8 * 32;               // warps 0-7 read the accumulators out
     if (tid == 0) {
         for (uint32_t k = 0; k < kSlots; ++k) {
             mbar_init(bar_slot + 8 * k, kDecThreads);
@@ -160,9 +212,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
         }
         mbar_init(bar_a, kDecThreads);
         mbar_init(bar_a + 8, kDecThreads);
+        mbar_init(bar_d, kEpiThreads);
+        mbar_init(bar_d + 8, kEpiThreads);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == kDecWarps) { // 64 columns of tensor memory: the 128 x (at most 64) FP32 accumulator
+    if (warp == kDecWarps) { // tensor memory: two 128 x (at most 64) FP32 accumulators
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(kTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -171,83 +225,82 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
-
-    const uint32_t rows = it.rows, K = it.cols, tpr = K >> 8;
-    // CTA (row block, token block, K part): K parts innermost, so a row block's parts run together
-    const uint32_t local = blockIdx.x - it.cta_begin;
-    const uint32_t kpart = local % it.ksplit, rt = local / it.ksplit;
-    const uint32_t row0 = (rt % it.row_tiles) * kBM;
-    const uint32_t nt = p.nt, tok0 = (rt / it.row_tiles) * nt, batch = p.batch;
-    const uint32_t kbeg = kpart * it.kper, kend = min(tpr, kbeg + it.kper);
-    // the CTA's slices: half tiles, slice q is half q & 1 of tile kbeg + q / 2
-    const uint32_t nsl = kbeg < kend ? 2 * (kend - kbeg) : 0u;
-    const bool split = it.ksplit > 1;
-    const uint64_t n_tiles = uint64_t(rows) * tpr;
-    const FwOffsets o = fw_offsets(n_tiles, it.n_exc);
-    const uint8_t* fw = it.fw;
     bool ok = true;
 
     if (tid < kDecThreads) {
-        const uint8_t* EP = fw + o.exc_pos;
-        const uint16_t* EW = reinterpret_cast<const uint16_t*>(fw + o.exc_word);
-        // The copies of a slice, split over the threads so that each thread's share has the
-        // same place in every slice: A and B plane pieces (16 bytes, 4 a row), C pieces (3 a
-        // row), tile_exc entries (2 a row) and X pieces (16 a token). Slice q's plane source
-        // is slice 0's plus 64 q (A, B) or 48 q (C) bytes: the half tiles of a row are
-        // contiguous in each plane.
+        // Reads segment g's accumulator (g & 1) out into Y: warp w (w < 8) reads tensor-memory
+        // lanes 32 (w % 4) .. +31 (rows of W) and columns (tokens) 32 (w / 4) .. +31. A
+        // segment that covers its row block's whole K range stores; the others add their part.
+        auto epilogue = [&](uint32_t g) {
+            if (warp >= 8) return;
+            const GemmSeg sg = s_seg[g];
+            const FwGemmItem& it = p.item[sg.item];
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint32_t quarter = warp & 3u, half = warp >> 2;
+            const uint32_t row = sg.row0 + quarter * 32 + lane;
+            for (uint32_t cb = half * 32; cb < half * 32 + 32 && cb < nt; cb += 16) {
+                uint32_t v[16];
+                const uint32_t taddr = tmem + ((quarter * 32) << 16) + (g & 1u) * 64 + cb;
+                asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+                             : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                               "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+                             : "r"(taddr));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                for (uint32_t q = 0; q < 16; ++q) {
+                    const uint32_t tok = sg.tok0 + cb + q;
+                    if (tok < batch) {
+                        float* dst = it.y + uint64_t(tok) * it.rows + row;
+                        if (sg.full) *dst = __uint_as_float(v[q]);
+                        else atomicAdd(dst, __uint_as_float(v[q])); // Y was zeroed; parts add up
+                    }
+                }
+            }
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            mbar_arrive(bar_d + 8 * (g & 1u));
+        };
+
+        // The copies of slice q, split over the threads: A and B plane pieces (16 bytes, 4 a
+        // row), C pieces (3 a row), tile_exc entries (2 a row) and X pieces (16 a token, placed
+        // in the 128-byte swizzle; tokens past the batch are zero-filled, pieces past nt
+        // tokens are not copied).
         constexpr uint32_t kPcAB = kBM * 4 / kDecThreads, kPcC = (kBM * 3 + kDecThreads - 1) / kDecThreads;
         constexpr uint32_t kPcTE = (kBM * 2 + kDecThreads - 1) / kDecThreads, kPcX = kMaxNt * 16 / kDecThreads;
         static_assert(kBM * 4 % kDecThreads == 0 && kMaxNt * 16 % kDecThreads == 0, "pieces");
-        uint64_t srcAB[kPcAB], srcC[kPcC], srcTE[kPcTE];
-#pragma unroll
-        for (uint32_t i = 0; i < kPcAB; ++i) {
-            const uint32_t c = tid + kDecThreads * i;
-            srcAB[i] = (uint64_t(row0 + (c >> 2)) * tpr + kbeg) * 128u + 16u * (c & 3u);
-        }
-#pragma unroll
-        for (uint32_t i = 0; i < kPcC; ++i) {
-            const uint32_t c = min(tid + kDecThreads * i, kBM * 3 - 1); // the clamped ones are not copied
-            srcC[i] = (uint64_t(row0 + c / 3u) * tpr + kbeg) * 96u + 16u * (c % 3u);
-        }
-#pragma unroll
-        for (uint32_t i = 0; i < kPcTE; ++i) {
-            const uint32_t c = min(tid + kDecThreads * i, kBM * 2 - 1); // likewise
-            srcTE[i] = uint64_t(row0 + (c >> 1)) * tpr + kbeg + (c & 1u);
-        }
-        // X pieces: 16-byte chunk c of token t, at a swizzled place of the slot; tokens past
-        // the batch are zero-filled, pieces past nt tokens are not copied
-        uint32_t dstX[kPcX];
-        uint64_t srcX[kPcX];
-        uint32_t bytesX = 0, liveX = 0; // bit i: piece i reads 16 bytes; piece i is copied
-#pragma unroll
-        for (uint32_t i = 0; i < kPcX; ++i) {
-            const uint32_t id = tid + kDecThreads * i, t = id >> 4, c = id & 15u, tok = tok0 + t;
-            dstX[i] = kPlX + (c >> 3) * (nt * 128) + t * 128 + (((c & 7u) ^ (t & 7u)) << 4);
-            srcX[i] = tok < batch ? uint64_t(tok) * K + kbeg * 256 + c * 8 : 0;
-            bytesX |= (tok < batch ? 1u : 0u) << i;
-            liveX |= (t < nt ? 1u : 0u) << i;
-        }
-        const uint8_t* const planeA = fw + o.a;
-        const uint8_t* const planeB = fw + o.b;
-        const uint8_t* const planeC = fw + o.c;
-        const uint8_t* const tex = fw + o.tile_exc;
+        uint32_t gi = 0; // the segment of the slice being queued
         auto issue = [&](uint32_t q) {
+            while (q >= s_seg[gi].q0 + 2 * s_seg[gi].n) ++gi;
+            const GemmSeg sg = s_seg[gi];
+            const FwGemmItem& it = p.item[sg.item];
+            const uint32_t tpr = it.cols >> 8, qq = q - sg.q0, kt = sg.kt0 + (qq >> 1), h = qq & 1u;
+            const FwOffsets o = fw_offsets(uint64_t(it.rows) * tpr, it.n_exc);
             const uint32_t sp = sS + (q % kSlots) * kSlotBytes;
+            const uint64_t tile0 = uint64_t(sg.row0) * tpr + kt; // the tile of the block's first row
 #pragma unroll
             for (uint32_t i = 0; i < kPcAB; ++i) {
-                cp_async16(sp + kPlA + 16 * (tid + kDecThreads * i), planeA + srcAB[i] + 64u * q, 16u);
-                cp_async16(sp + kPlB + 16 * (tid + kDecThreads * i), planeB + srcAB[i] + 64u * q, 16u);
+                const uint32_t c = tid + kDecThreads * i;
+                const uint64_t src = (tile0 + uint64_t(c >> 2) * tpr) * 128u + 64u * h + 16u * (c & 3u);
+                cp_async16(sp + kPlA + 16 * c, it.fw + o.a + src, 16u);
+                cp_async16(sp + kPlB + 16 * c, it.fw + o.b + src, 16u);
             }
 #pragma unroll
-            for (uint32_t i = 0; i < kPcC; ++i)
-                cp_async16_if(tid + kDecThreads * i < kBM * 3, sp + kPlC + 16 * (tid + kDecThreads * i),
-                              planeC + srcC[i] + 48u * q, 16u);
+            for (uint32_t i = 0; i < kPcC; ++i) {
+                const uint32_t c = tid + kDecThreads * i, cc = min(c, kBM * 3 - 1);
+                const uint64_t src = (tile0 + uint64_t(cc / 3u) * tpr) * 96u + 48u * h + 16u * (cc % 3u);
+                cp_async16_if(c < kBM * 3, sp + kPlC + 16 * c, it.fw + o.c + src, 16u);
+            }
 #pragma unroll
-            for (uint32_t i = 0; i < kPcTE; ++i)
-                if (tid + kDecThreads * i < kBM * 2) fw_cp4(sp + kPlTE + 4 * (tid + kDecThreads * i), tex + 4 * (srcTE[i] + (q >> 1)));
+            for (uint32_t i = 0; i < kPcTE; ++i) {
+                const uint32_t c = tid + kDecThreads * i;
+                if (c < kBM * 2) fw_cp4(sp + kPlTE + 4 * c, it.fw + o.tile_exc + 4 * (tile0 + uint64_t(c >> 1) * tpr + (c & 1u)));
+            }
 #pragma unroll
-            for (uint32_t i = 0; i < kPcX; ++i)
-                cp_async16_if((liveX >> i) & 1u, sp + dstX[i], it.x + srcX[i] + 128u * q, ((bytesX >> i) & 1u) * 16u);
+            for (uint32_t i = 0; i < kPcX; ++i) {
+                const uint32_t id = tid + kDecThreads * i, t = id >> 4, c = id & 15u, tok = sg.tok0 + t;
+                const uint32_t dst = sp + kPlX + (c >> 3) * (nt * 128) + t * 128 + (((c & 7u) ^ (t & 7u)) << 4);
+                const uint16_t* src = tok < batch ? it.x + uint64_t(tok) * it.cols + kt * 256 + h * 128 + c * 8 : it.x;
+                cp_async16_if(t < nt, dst, src, tok < batch ? 16u : 0u);
+            }
             mbar_arrive_cp_async(bar_slot + 8 * (q % kSlots));
         };
         // decode: warp w writes rows 8w .. 8w+7, two at a time (lanes 0-15 and 16-31), lane
@@ -255,37 +308,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
         const uint32_t j = lane & 15u, rsub = lane >> 4;
         const uint32_t cw0 = (3u * j) >> 2, csh = (24u * j) & 31u, cw1 = csh > 8 ? cw0 + 1 : cw0;
         // exceptions: lane holds entries e0 + kExcRegs (lane >> 3) .. of row er's tile, as
-        // (position << 16) | word, the first nex of them valid
+        // (position << 16) | word, the first n_ex of them valid
         constexpr uint32_t kRowsW = kBM / kDecWarps; // 8 rows a warp
         const uint32_t er = warp * kRowsW + (lane & (kRowsW - 1u));
-        uint32_t ex[kExcRegs], nex[kExcRegs];
-        uint32_t e0 = 0, eend = 0, ne0 = 0, neend = 0, n_ex = 0, n_nex = 0;
-        // checks a tile's tile_exc pair and queues the loads of this lane's share of its entries
-        auto load_exc = [&](uint32_t t0, uint32_t t1) {
-            const bool e_ok = t0 <= t1 && t1 <= it.n_exc;
-            if (!e_ok && lane < kRowsW) atomicOr(p.err, 1u);
-            ne0 = t0;
-            neend = e_ok ? t1 : t0;
-            const uint32_t ebeg = t0 + kExcRegs * (lane / kRowsW);
-            n_nex = ebeg < neend ? min(neend - ebeg, kExcRegs) : 0u;
-#pragma unroll
-            for (uint32_t i = 0; i < kExcRegs; ++i)
-                nex[i] = i < n_nex ? (uint32_t(__ldg(EP + ebeg + i)) << 16) | __ldg(EW + ebeg + i) : 0u;
-        };
-
+        uint32_t ex[kExcRegs];
+        uint32_t e0 = 0, eend = 0, n_ex = 0;
+        uint32_t gd = 0;                  // the segment of the slice being decoded
+        uint32_t epi_next = 0;            // the next segment to read out
         for (uint32_t q = 0; q + 1 < kSlots && q < nsl; ++q) issue(q); // slices 0 .. kSlots - 2
         for (uint32_t q = 0; q < nsl && ok; ++q) {
-            const uint32_t s = q % kSlots, st = q & 1u, h = q & 1u;
+            while (q >= s_seg[gd].q0 + 2 * s_seg[gd].n) ++gd;
+            const GemmSeg sg = s_seg[gd];
+            const FwGemmItem& it = p.item[sg.item];
+            const uint32_t s = q % kSlots, st = q & 1u, h = (q - sg.q0) & 1u;
             const uint8_t* slot = smem + (sS - sbase) + s * kSlotBytes;
             if (!mbar_wait(bar_slot + 8 * s, (q / kSlots) & 1u, abort_flag)) { ok = false; break; }
+            const FwOffsets o = fw_offsets(uint64_t(it.rows) * (it.cols >> 8), it.n_exc);
+            const uint8_t* EP = it.fw + o.exc_pos;
+            const uint16_t* EW = reinterpret_cast<const uint16_t*>(it.fw + o.exc_word);
             if (h == 0) { // a new tile: its exception entries, both halves use them
                 const uint32_t* te = reinterpret_cast<const uint32_t*>(slot + kPlTE) + 2 * er;
-                load_exc(te[0], te[1]);
+                const uint32_t t0 = te[0], t1 = te[1];
+                const bool e_ok = t0 <= t1 && t1 <= it.n_exc;
+                if (!e_ok && lane < kRowsW) atomicOr(p.err, 1u);
+                e0 = t0;
+                eend = e_ok ? t1 : t0;
+                const uint32_t ebeg = t0 + kExcRegs * (lane / kRowsW);
+                n_ex = ebeg < eend ? min(eend - ebeg, kExcRegs) : 0u;
 #pragma unroll
-                for (uint32_t i = 0; i < kExcRegs; ++i) ex[i] = nex[i];
-                e0 = ne0;
-                eend = neend;
-                n_ex = n_nex;
+                for (uint32_t i = 0; i < kExcRegs; ++i)
+                    ex[i] = i < n_ex ? (uint32_t(__ldg(EP + ebeg + i)) << 16) | __ldg(EW + ebeg + i) : 0u;
             }
             uint32_t pa[4], pb[4], pc0[4], pc1[4];
 #pragma unroll
@@ -297,12 +349,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
                 pc0[i] = cp[cw0];
                 pc1[i] = cp[cw1];
             }
-            // A stage st was last read by the MMAs of slice q - 2
+            // A stage st was last read by the MMAs of slice q - 2; once they have completed, a
+            // segment that ended with slice q - 2 or before can be read out
             if (q >= 2 && !mbar_wait(bar_mma + 8 * ((q - 2) % kSlots), ((q - 2) / kSlots) & 1u, abort_flag)) {
                 ok = false;
                 break;
             }
+            while (q >= 2 && epi_next < nseg && s_seg[epi_next].q0 + 2 * s_seg[epi_next].n <= q - 1) epilogue(epi_next++);
             uint8_t* const stA = gA + st * kStageA;
+            const uint32_t* pair_tab = reinterpret_cast<const uint32_t*>(smem) + 256 * sg.tab;
 #pragma unroll
             for (uint32_t i = 0; i < 4; ++i) {
                 const uint32_t r = warp * kRowsW + 2 * i + rsub;
@@ -321,7 +376,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
                                                  2 * (pos & 7u)) = static_cast<uint16_t>(ex[i]);
                 }
             }
-            if (lane < kRowsW) // a tile with more than 32 exceptions: the rest, straight from memory
+            if (lane < kRowsW) // a tile with more exceptions than the lanes hold: the rest, from memory
                 for (uint32_t e = e0 + (32 / kRowsW) * kExcRegs; e < eend; ++e) {
                     const uint32_t pos = __ldg(EP + e);
                     if ((pos >> 7) != h) continue;
@@ -337,54 +392,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
             if (qn < nsl && qn >= kSlots - 1) issue(qn);
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
+        // the segments not yet read out: after the last slice's MMAs
+        if (ok && nsl > 0 && warp < 8) {
+            ok = !*abort_flag && mbar_wait(bar_mma + 8 * ((nsl - 1) % kSlots), ((nsl - 1) / kSlots) & 1u, abort_flag);
+            while (ok && epi_next < nseg) epilogue(epi_next++);
+        }
     } else if (tid == kDecThreads) {
-        // the MMA thread: M = 128, N = nt, BF16 x BF16 -> FP32, both operands K-major
+        // the MMA thread: M = 128, N = nt, BF16 x BF16 -> FP32, both operands K-major;
+        // segment g accumulates into accumulator g & 1, which segment g - 2's read-out frees
         const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((nt >> 3) << 17) | ((kBM >> 4) << 24);
+        uint32_t g = 0;
         for (uint32_t q = 0; q < nsl; ++q) {
-            const uint32_t st = q & 1u, s = q % kSlots;
+            while (q >= s_seg[g].q0 + 2 * s_seg[g].n) ++g;
+            const uint32_t st = q & 1u, s = q % kSlots, first = q == s_seg[g].q0;
+            if (first && g >= 2 && !mbar_wait(bar_d + 8 * (g & 1u), ((g - 2) >> 1) & 1u, abort_flag)) { ok = false; break; }
             if (!mbar_wait(bar_a + 8 * st, (q >> 1) & 1u, abort_flag)) { ok = false; break; }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const uint32_t a0 = sA + st * kStageA, b0 = sS + s * kSlotBytes + kPlX;
+            const uint32_t a0 = sA + st * kStageA, b0 = sS + s * kSlotBytes + kPlX, d = tmem + (g & 1u) * 64;
 #pragma unroll
             for (uint32_t kk = 0; kk < 8; ++kk) { // K = 16 per MMA: atom kk / 4, 32 bytes per step inside it
                 const uint64_t ad = sw128_desc(a0 + (kk >> 2) * kAtomA + (kk & 3u) * 32);
                 const uint64_t bd = sw128_desc(b0 + (kk >> 2) * (nt * 128) + (kk & 3u) * 32);
-                const uint32_t acc = (q | kk) != 0;
+                const uint32_t acc = !(first && kk == 0);
                 asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
                              " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}"
-                             ::"r"(tmem), "l"(ad), "l"(bd), "r"(idesc), "r"(acc) : "memory");
+                             ::"r"(d), "l"(ad), "l"(bd), "r"(idesc), "r"(acc) : "memory");
             }
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_mma + 8 * s)
                          : "memory");
-        }
-    }
-    // The last commit covers every MMA before it.
-    if (warp < 8 && nsl > 0) {
-        ok = ok && !*abort_flag && mbar_wait(bar_mma + 8 * ((nsl - 1) % kSlots), ((nsl - 1) / kSlots) & 1u, abort_flag);
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        if (ok) {
-            // warp w reads tensor-memory lanes 32 (w % 4) .. +31 (rows of W) and columns (tokens)
-            // 32 (w / 4) .. +31 of the accumulator
-            const uint32_t quarter = warp & 3u, half = warp >> 2;
-            const uint32_t row = row0 + quarter * 32 + lane;
-            for (uint32_t cb = half * 32; cb < half * 32 + 32 && cb < nt; cb += 16) {
-                uint32_t v[16];
-                const uint32_t taddr = tmem + ((quarter * 32) << 16) + cb;
-                asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-                             : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-                               "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-                             : "r"(taddr));
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-                for (uint32_t q = 0; q < 16; ++q) {
-                    const uint32_t tok = tok0 + cb + q;
-                    if (tok < batch) {
-                        float* dst = it.y + uint64_t(tok) * rows + row;
-                        if (split) atomicAdd(dst, __uint_as_float(v[q])); // Y was zeroed; parts add up
-                        else *dst = __uint_as_float(v[q]);
-                    }
-                }
-            }
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -430,32 +465,21 @@ extern "C" bs_status bs_fw_gemm(int32_t n, const bs_fw_gemv_item* items, uint32_
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int32_t k = 0;
     while (k < n) {
-        // the items of one launch; K is split where the row blocks alone would not give about
-        // two CTAs per SM
-        int32_t k1 = k;
-        uint64_t blocks = 0;
-        for (uint32_t m = 0; k1 < n && m < static_cast<uint32_t>(kGemmMaxItems); ++k1) {
-            if (items[k1].info.n_elems == 0) continue;
-            blocks += uint64_t(items[k1].rows / kBM) * p.token_tiles;
-            ++m;
-        }
-        const uint64_t want = 2ull * static_cast<uint64_t>(sms);
+        // The items of one launch and their units (token tile, row block, tile). The units are
+        // shared evenly by one wave of CTAs (one per SM), so a CTA's range may start or end
+        // inside a row block; those parts add into Y, which is zeroed first. A CTA holds at
+        // most kMaxSegs runs and two items: launches with small items use more CTAs.
         p.n_items = 0;
-        uint64_t ctas = 0;
-        for (; k < k1; ++k) {
+        uint64_t units = 0;
+        uint32_t min_units = ~0u, min_tpr = ~0u;
+        for (; k < n && p.n_items < static_cast<uint32_t>(kGemmMaxItems); ++k) {
             const bs_fw_gemv_item& g = items[k];
             if (g.info.n_elems == 0) continue;
             const uint32_t tpr = g.cols / 256;
-            uint32_t ksplit = blocks >= want ? 1u : static_cast<uint32_t>(std::min<uint64_t>((want + blocks - 1) / blocks, tpr));
-            ksplit = std::max<uint32_t>(1u, std::min<uint32_t>(ksplit, 0xFFFFu));
-            const uint32_t kper = (tpr + ksplit - 1) / ksplit;
-            ksplit = (tpr + kper - 1) / kper; // no empty part
-            const uint64_t c = uint64_t(g.rows / kBM) * p.token_tiles * ksplit;
-            if (ctas + c >= (1ull << 31) || kper > 0xFFFFu) return BS_E_SIZE;
-            if (ksplit > 1) { // the parts add into Y
-                e = cudaMemsetAsync(g.d_y, 0, sizeof(float) * uint64_t(batch) * g.rows, s);
-                if (e != cudaSuccess) return cuda_status(e);
-            }
+            const uint64_t u = uint64_t(g.rows / kBM) * p.token_tiles * tpr;
+            if (units + u >= (1ull << 31)) break;
+            e = cudaMemsetAsync(g.d_y, 0, sizeof(float) * uint64_t(batch) * g.rows, s);
+            if (e != cudaSuccess) return cuda_status(e);
             FwGemmItem& it = p.item[p.n_items++];
             it.fw = static_cast<const uint8_t*>(g.d_fw);
             it.x = static_cast<const uint16_t*>(g.d_x);
@@ -463,14 +487,23 @@ extern "C" bs_status bs_fw_gemm(int32_t n, const bs_fw_gemv_item* items, uint32_
             it.rows = g.rows;
             it.cols = g.cols;
             it.n_exc = static_cast<uint32_t>(g.info.n_exc);
-            it.cta_begin = static_cast<uint32_t>(ctas);
+            it.unit_begin = static_cast<uint32_t>(units);
             it.row_tiles = g.rows / kBM;
-            it.ksplit = static_cast<uint16_t>(ksplit);
-            it.kper = static_cast<uint16_t>(kper);
+            it.pad = 0;
             std::memcpy(it.table, g.info.table, sizeof(it.table));
-            ctas += c;
+            units += u;
+            min_units = std::min<uint32_t>(min_units, static_cast<uint32_t>(u));
+            min_tpr = std::min(min_tpr, tpr);
         }
         if (p.n_items == 0) continue;
+        // one CTA per SM, unless a CTA's share (at most ceil(units / ctas)) would exceed the
+        // smallest item's units (so that a CTA spans at most two items) or give more than
+        // kMaxSegs runs (a share of L units over rows of at least min_tpr tiles makes at most
+        // L / min_tpr + 3 runs)
+        const uint64_t bound = std::max<uint64_t>(1, std::min<uint64_t>(min_units, uint64_t(kMaxSegs - 4) * min_tpr));
+        const uint64_t ctas = std::max<uint64_t>(std::min<uint64_t>(static_cast<uint64_t>(sms), units), (units + bound - 1) / bound);
+        p.units = static_cast<uint32_t>(units);
+        p.ctas = static_cast<uint32_t>(ctas);
         fw_gemm_kernel<<<static_cast<uint32_t>(ctas), kGemmThreads, kGemmSmem, s>>>(p);
         count_launch();
         e = cudaGetLastError();
