@@ -267,42 +267,79 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
         constexpr uint32_t kPcAB = kBM * 4 / kDecThreads, kPcC = (kBM * 3 + kDecThreads - 1) / kDecThreads;
         constexpr uint32_t kPcTE = (kBM * 2 + kDecThreads - 1) / kDecThreads, kPcX = kMaxNt * 16 / kDecThreads;
         static_assert(kBM * 4 % kDecThreads == 0 && kMaxNt * 16 % kDecThreads == 0, "pieces");
-        uint32_t gi = 0; // the segment of the slice being queued
-        auto issue = [&](uint32_t q) {
-            while (q >= s_seg[gi].q0 + 2 * s_seg[gi].n) ++gi;
-            const GemmSeg sg = s_seg[gi];
+        // The sources of this thread's pieces for the first slice of segment gi (slice q0 + qq
+        // of the segment adds 64 qq bytes for A and B, 48 qq for C, 4 (qq / 2) for tile_exc and
+        // 128 qq elements for X), worked out once a segment.
+        uint32_t gi = 0, gi_end = 0, gi_q0 = 0; // the segment of the slice being queued, its slices
+        const uint8_t* srcA[kPcAB];
+        const uint8_t* srcC[kPcC];
+        const uint8_t* srcT[kPcTE];
+        const uint16_t* srcX[kPcX];
+        uint64_t gapB = 0;               // plane B's offset from plane A
+        uint32_t bytesX = 0, liveX = 0;  // bit i: X piece i reads 16 bytes; piece i is copied
+        auto seg_sources = [&](uint32_t g) {
+            const GemmSeg sg = s_seg[g];
             const FwGemmItem& it = p.item[sg.item];
-            const uint32_t tpr = it.cols >> 8, qq = q - sg.q0, kt = sg.kt0 + (qq >> 1), h = qq & 1u;
+            const uint32_t tpr = it.cols >> 8;
             const FwOffsets o = fw_offsets(uint64_t(it.rows) * tpr, it.n_exc);
-            const uint32_t sp = sS + (q % kSlots) * kSlotBytes;
-            const uint64_t tile0 = uint64_t(sg.row0) * tpr + kt; // the tile of the block's first row
+            const uint64_t tile0 = uint64_t(sg.row0) * tpr + sg.kt0; // the block's first row's tile
+            gapB = o.b - o.a;
 #pragma unroll
             for (uint32_t i = 0; i < kPcAB; ++i) {
                 const uint32_t c = tid + kDecThreads * i;
-                const uint64_t src = (tile0 + uint64_t(c >> 2) * tpr) * 128u + 64u * h + 16u * (c & 3u);
-                cp_async16(sp + kPlA + 16 * c, it.fw + o.a + src, 16u);
-                cp_async16(sp + kPlB + 16 * c, it.fw + o.b + src, 16u);
+                srcA[i] = it.fw + o.a + (tile0 + uint64_t(c >> 2) * tpr) * 128u + 16u * (c & 3u);
             }
 #pragma unroll
             for (uint32_t i = 0; i < kPcC; ++i) {
-                const uint32_t c = tid + kDecThreads * i, cc = min(c, kBM * 3 - 1);
-                const uint64_t src = (tile0 + uint64_t(cc / 3u) * tpr) * 96u + 48u * h + 16u * (cc % 3u);
-                cp_async16_if(c < kBM * 3, sp + kPlC + 16 * c, it.fw + o.c + src, 16u);
+                const uint32_t cc = min(tid + kDecThreads * i, kBM * 3 - 1); // the clamped ones are not copied
+                srcC[i] = it.fw + o.c + (tile0 + uint64_t(cc / 3u) * tpr) * 96u + 16u * (cc % 3u);
+            }
+#pragma unroll
+            for (uint32_t i = 0; i < kPcTE; ++i) {
+                const uint32_t cc = min(tid + kDecThreads * i, kBM * 2 - 1); // likewise
+                srcT[i] = it.fw + o.tile_exc + 4 * (tile0 + uint64_t(cc >> 1) * tpr + (cc & 1u));
+            }
+            bytesX = 0;
+            liveX = 0;
+#pragma unroll
+            for (uint32_t i = 0; i < kPcX; ++i) {
+                const uint32_t id = tid + kDecThreads * i, t = id >> 4, c = id & 15u, tok = sg.tok0 + t;
+                srcX[i] = tok < batch ? it.x + uint64_t(tok) * it.cols + sg.kt0 * 256 + c * 8 : it.x;
+                bytesX |= (tok < batch ? 1u : 0u) << i;
+                liveX |= (t < nt ? 1u : 0u) << i;
+            }
+            gi_q0 = sg.q0;
+            gi_end = sg.q0 + 2 * sg.n;
+        };
+        auto issue = [&](uint32_t q) {
+            while (q >= gi_end) seg_sources(++gi);
+            const uint32_t qq = q - gi_q0;
+            const uint32_t sp = sS + (q % kSlots) * kSlotBytes;
+#pragma unroll
+            for (uint32_t i = 0; i < kPcAB; ++i) {
+                const uint32_t c = tid + kDecThreads * i;
+                cp_async16(sp + kPlA + 16 * c, srcA[i] + 64u * qq, 16u);
+                cp_async16(sp + kPlB + 16 * c, srcA[i] + gapB + 64u * qq, 16u);
+            }
+#pragma unroll
+            for (uint32_t i = 0; i < kPcC; ++i) {
+                const uint32_t c = tid + kDecThreads * i;
+                cp_async16_if(c < kBM * 3, sp + kPlC + 16 * c, srcC[i] + 48u * qq, 16u);
             }
 #pragma unroll
             for (uint32_t i = 0; i < kPcTE; ++i) {
                 const uint32_t c = tid + kDecThreads * i;
-                if (c < kBM * 2) fw_cp4(sp + kPlTE + 4 * c, it.fw + o.tile_exc + 4 * (tile0 + uint64_t(c >> 1) * tpr + (c & 1u)));
+                if (c < kBM * 2) fw_cp4(sp + kPlTE + 4 * c, srcT[i] + 4 * (qq >> 1));
             }
 #pragma unroll
             for (uint32_t i = 0; i < kPcX; ++i) {
-                const uint32_t id = tid + kDecThreads * i, t = id >> 4, c = id & 15u, tok = sg.tok0 + t;
+                const uint32_t id = tid + kDecThreads * i, t = id >> 4, c = id & 15u;
                 const uint32_t dst = sp + kPlX + (c >> 3) * (nt * 128) + t * 128 + (((c & 7u) ^ (t & 7u)) << 4);
-                const uint16_t* src = tok < batch ? it.x + uint64_t(tok) * it.cols + kt * 256 + h * 128 + c * 8 : it.x;
-                cp_async16_if(t < nt, dst, src, tok < batch ? 16u : 0u);
+                cp_async16_if((liveX >> i) & 1u, dst, srcX[i] + 128u * qq, ((bytesX >> i) & 1u) * 16u);
             }
             mbar_arrive_cp_async(bar_slot + 8 * (q % kSlots));
         };
+        if (nsl > 0) seg_sources(0);
         // decode: warp w writes rows 8w .. 8w+7, two at a time (lanes 0-15 and 16-31), lane
         // octet j = lane & 15 of the half tile
         const uint32_t j = lane & 15u, rsub = lane >> 4;
@@ -313,23 +350,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
         const uint32_t er = warp * kRowsW + (lane & (kRowsW - 1u));
         uint32_t ex[kExcRegs];
         uint32_t e0 = 0, eend = 0, n_ex = 0;
-        uint32_t gd = 0;                  // the segment of the slice being decoded
+        // the segment of the slice being decoded: its first slice and end, its item's exception
+        // arrays, exception count and pair table, worked out once a segment
+        uint32_t gd = 0, gd_q0 = 0, gd_end = 0, gd_nexc = 0;
+        const uint8_t* EP = nullptr;
+        const uint16_t* EW = nullptr;
+        const uint32_t* pair_tab = nullptr;
+        auto seg_decode = [&](uint32_t g) {
+            const GemmSeg sg = s_seg[g];
+            const FwGemmItem& it = p.item[sg.item];
+            const FwOffsets o = fw_offsets(uint64_t(it.rows) * (it.cols >> 8), it.n_exc);
+            EP = it.fw + o.exc_pos;
+            EW = reinterpret_cast<const uint16_t*>(it.fw + o.exc_word);
+            gd_nexc = it.n_exc;
+            pair_tab = reinterpret_cast<const uint32_t*>(smem) + 256 * sg.tab;
+            gd_q0 = sg.q0;
+            gd_end = sg.q0 + 2 * sg.n;
+        };
+        if (nsl > 0) seg_decode(0);
         uint32_t epi_next = 0;            // the next segment to read out
         for (uint32_t q = 0; q + 1 < kSlots && q < nsl; ++q) issue(q); // slices 0 .. kSlots - 2
         for (uint32_t q = 0; q < nsl && ok; ++q) {
-            while (q >= s_seg[gd].q0 + 2 * s_seg[gd].n) ++gd;
-            const GemmSeg sg = s_seg[gd];
-            const FwGemmItem& it = p.item[sg.item];
-            const uint32_t s = q % kSlots, st = q & 1u, h = (q - sg.q0) & 1u;
+            while (q >= gd_end) seg_decode(++gd);
+            const uint32_t s = q % kSlots, st = q & 1u, h = (q - gd_q0) & 1u;
             const uint8_t* slot = smem + (sS - sbase) + s * kSlotBytes;
             if (!mbar_wait(bar_slot + 8 * s, (q / kSlots) & 1u, abort_flag)) { ok = false; break; }
-            const FwOffsets o = fw_offsets(uint64_t(it.rows) * (it.cols >> 8), it.n_exc);
-            const uint8_t* EP = it.fw + o.exc_pos;
-            const uint16_t* EW = reinterpret_cast<const uint16_t*>(it.fw + o.exc_word);
             if (h == 0) { // a new tile: its exception entries, both halves use them
                 const uint32_t* te = reinterpret_cast<const uint32_t*>(slot + kPlTE) + 2 * er;
                 const uint32_t t0 = te[0], t1 = te[1];
-                const bool e_ok = t0 <= t1 && t1 <= it.n_exc;
+                const bool e_ok = t0 <= t1 && t1 <= gd_nexc;
                 if (!e_ok && lane < kRowsW) atomicOr(p.err, 1u);
                 e0 = t0;
                 eend = e_ok ? t1 : t0;
@@ -357,7 +406,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
             }
             while (q >= 2 && epi_next < nseg && s_seg[epi_next].q0 + 2 * s_seg[epi_next].n <= q - 1) epilogue(epi_next++);
             uint8_t* const stA = gA + st * kStageA;
-            const uint32_t* pair_tab = reinterpret_cast<const uint32_t*>(smem) + 256 * sg.tab;
 #pragma unroll
             for (uint32_t i = 0; i < 4; ++i) {
                 const uint32_t r = warp * kRowsW + 2 * i + rsub;

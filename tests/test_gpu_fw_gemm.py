@@ -148,3 +148,20 @@ def test_gemm_without_and_with_k_split():
         (y,), err, _ = _run([(w, x)], batch)
         assert err == 0
         _check(w, x, y)
+
+
+def test_gemm_items_of_different_shapes_and_tables_in_one_call():
+    # one launch shares the (row block, tile) units of all items evenly among its CTAs, so a CTA
+    # can cover the end of one item and the start of the next, with a different code table and
+    # row length; rows of a single tile (cols 256) make many short runs per CTA
+    batch = 24
+    shapes = [(384, 256), (1280, 3584), (256, 1024), (640, 256), (128, 7168)]
+    scales = [0.02, 1.0, 0.003, 0.5, 0.05]
+    ws = [_gauss(r * c, seed=100 + k, scale=sc).reshape(r, c) for k, ((r, c), sc) in enumerate(zip(shapes, scales))]
+    xs = [_gauss(batch * c, seed=200 + k, scale=1.0).reshape(batch, c) for k, (_, c) in enumerate(shapes)]
+    tables = {tuple(oracle.fw_info(oracle.fw_encode(w))["table"]) for w in ws}
+    assert len(tables) >= 3
+    ys, err, _ = _run(list(zip(ws, xs)), batch)
+    assert err == 0
+    for w, x, y in zip(ws, xs, ys):
+        _check(w, x, y)
