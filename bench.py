@@ -61,7 +61,7 @@ def _args():
                     help="gemv mode: tokens per product (1..8 on the CUDA cores, more on the tensor cores)")
     ap.add_argument("--product", choices=["auto", "cuda", "tensor"], default="auto",
                     help="gemv mode: the CUDA-core product (bs_fw_gemv, batch 1..8), the tensor-core one "
-                         "(bs_fw_gemm), or auto: tensor cores above batch 8")
+                         "(bs_fw_gemm), or auto: tensor cores above batch 4, where they become the faster")
     ap.add_argument("--model", choices=["joint", "factored"], default="joint",
                     help="rANS model of the container: joint (one table over (s, h), kind JOINT; "
                          "the default) or factored (s-model plus exponent routes, kind RANS)")
@@ -1285,8 +1285,10 @@ def run_gemv(a):
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
 
-    # batches above 8 go to the tensor cores (bs_fw_gemm), batches 1..8 to the CUDA cores
-    tensor = a.product == "tensor" or (a.product == "auto" and batch > 8)
+    # batches 1..4 go to the CUDA cores (bs_fw_gemv), larger ones to the tensor cores
+    # (bs_fw_gemm): on the 9B pass the CUDA-core product takes 4.4 / 5.6 / 6.5 / 7.7 ms at
+    # batch 1 / 2 / 3 / 4 and 15 ms at 8, the tensor-core one about 8.7 ms at any batch up to 16
+    tensor = a.product == "tensor" or (a.product == "auto" and batch > 4)
     if not tensor and batch > 8:
         raise SystemExit("bench: the CUDA-core product takes batches of 1..8")
     # the layouts are written once, before the pass, and stay resident: the CUDA-core product
