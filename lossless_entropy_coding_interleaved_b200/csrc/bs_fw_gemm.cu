@@ -4,28 +4,28 @@
 //
 // This is the operand path of the "Qwen3.8-27B-BF16-NVLC-Lossless" card's runtime (compressed
 // weights resident, no persistent decoded-weight cache; its runtime accounting and DGX Spark
-// tables) for batches of tokens too large for the CUDA-core product of bs_fw_gemv.cu: at 9 or
-// more tokens a product needs more multiply-adds per weight byte than the CUDA cores give, so
-// the multiply goes to the 5th-generation tensor cores (tcgen05, BF16 operands, FP32
-// accumulators in tensor memory).
+// tables) for batches of tokens too large for the CUDA-core product of bs_fw_gemv.cu: each token
+// adds a multiply-add per weight there (on the 9B-shaped pass it passes this kernel's time at
+// about 5 tokens), so the multiply goes to the 5th-generation tensor cores (tcgen05, BF16
+// operands, FP32 accumulators in tensor memory).
 //
 // Work split ("swap AB": the weight rows are the MMA's M, the tokens its N):
 //  * A segment's 128 rows of W and up to 64 tokens are walked in slices of 128 columns: half
 //    an FW tile of each row. A slice's plane bytes (A, B, C: 176 bytes a row),
 //    its tiles' tile_exc entries and the tokens' X slice are copied with cp.async into one of
-//    four slots, three slices ahead of the decode (about 70 KiB in flight a CTA). Each copying
-//    thread's cp.async completion arrives on the slot's mbarrier.
+//    four slots, two slices ahead of the decode. Each copying thread's cp.async completion
+//    arrives on the slot's mbarrier.
 //  * 16 warps decode a slice from its slot into one of two A stages (BF16, K-major, the
 //    128-byte swizzle of the MMA's canonical layout), patch in its exceptions, and arrive on
 //    the stage's mbarrier. A tile's exception entries are loaded into registers (four lanes a
 //    row, up to 3 each, the rest of a tile's entries read from memory) when its first half is
-//    decoded and serve both halves.
+//    decoded, and serve both halves.
 //  * A 17th warp issues each slice's 8 MMAs (M = 128, N = tokens, K = 16 each) into a 128 x N
 //    FP32 accumulator in tensor memory once the stage is written, and commits them to the
 //    slot's completion barrier. That one barrier frees both the A stage (rewritten two slices
-//    later) and the slot (refilled with the slice three ahead). So the decode of a slice,
-//    the MMAs of the one before and the copies of the next three all overlap, with no
-//    barrier across the CTA inside the loop.
+//    later) and the slot (refilled with the slice two ahead). So the decode of a slice, the
+//    MMAs of the one before and the copies of the next two all overlap, with no barrier
+//    across the CTA inside the loop.
 //  * Stream-K work split: a launch's units (item, token tile, 128-row block, FW tile) are shared
 //    evenly by one wave of CTAs, one per SM, so no SM idles through a partial last wave. A
 //    CTA walks its units as runs of one row block's tiles (segments). Segment g accumulates in
@@ -35,7 +35,7 @@
 //    row block split between two CTAs gets two such parts, whose sum does not depend on their
 //    order; one split among three or more CTAs (tiny launches) can differ in its last bits
 //    from run to run.
-//  * The epilogue reads the accumulator with tcgen05.ld (warps 0-7; warp w reads lanes
+//  * The read-out uses tcgen05.ld (warps 0-7; warp w reads lanes
 //    32(w % 4)..+31, that is 32 rows of W, and 32 tokens from column 32(w / 4)) and writes
 //    Y[token][row] in FP32, 128 contiguous bytes per warp and token.
 //  * Every wait on an mbarrier is bounded. A wait that runs out, or sees that another thread's
