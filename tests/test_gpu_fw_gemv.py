@@ -104,7 +104,7 @@ def test_gemv_many_escapes_per_group():
     x = _gauss(2 * cols, seed=4, scale=1.0).reshape(2, cols)
     (y,), err, items = _run([(w, x)], 2)
     assert err == 0
-    assert items[0][1].n_exc > 32 * rows          # far more than 32 escapes per group of 4 tiles
+    assert items[0][1].n_exc > 64 * rows          # far more than 64 escapes per group (a row here)
     ref = oracle.fw_gemv(oracle.fw_encode(w), rows, cols, x)
     finite = np.isfinite(ref)
     assert np.array_equal(np.isfinite(y), finite)
