@@ -35,9 +35,10 @@
 //    row block split between two CTAs gets two such parts, whose sum does not depend on their
 //    order; one split among three or more CTAs (tiny launches) can differ in its last bits
 //    from run to run.
-//  * The read-out uses tcgen05.ld (warps 0-7; warp w reads lanes
-//    32(w % 4)..+31, that is 32 rows of W, and 32 tokens from column 32(w / 4)) and writes
-//    Y[token][row] in FP32, 128 contiguous bytes per warp and token.
+//  * Four more warps read the accumulators out with tcgen05.ld (warp w reads lanes
+//    32(w % 4)..+31, that is 32 rows of W, and every token column) once an extra commit after
+//    a segment's last slice has arrived, and write Y[token][row] in FP32, 128 contiguous bytes
+//    per warp and token; the decoding warps never wait for it.
 //  * Every wait on an mbarrier is bounded. A wait that runs out, or sees that another thread's
 //    has, sets the CTA's abort flag and bit 1 of the error word; the threads then skip the
 //    remaining work and the tensor memory is still freed. A tile_exc entry out of order or
@@ -59,7 +60,8 @@ using namespace fw;
 
 constexpr uint32_t kDecWarps = 16;                  // warps that copy and decode
 constexpr uint32_t kDecThreads = kDecWarps * 32;
-constexpr uint32_t kGemmThreads = kDecThreads + 32;  // + the warp that issues the MMAs
+constexpr uint32_t kEpiWarps = 4;                    // warps that read the accumulators out
+constexpr uint32_t kGemmThreads = kDecThreads + 32 + kEpiWarps * 32; // + the MMA warp, + those
 constexpr uint32_t kBM = 128;                        // rows of W per CTA: the MMA's M
 constexpr uint32_t kMaxNt = 64;                      // tokens per CTA: the MMA's N (a multiple of 16)
 constexpr uint32_t kAtomA = kBM * 128;               // one 64-wide K atom of an A stage (16 KiB)
@@ -197,14 +199,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
     // mbarriers: slot_full[4] (the copies of a slot have landed: one arrival a copying thread),
     // a_full[2] (an A stage is written: one arrival a decoding thread), mma_done[4] (the MMAs
     // of the slice in a slot have completed: the commit), d_free[2] (an accumulator has been
-    // read out: one arrival an epilogue thread)
+    // read out: one arrival an epilogue thread), seg_done[2] (the MMAs of a segment have
+    // completed: an extra commit after its last slice)
     const uint32_t bar_slot = sbase + kTabs * 1024, bar_a = bar_slot + 8 * kSlots, bar_mma = bar_a + 16;
-    const uint32_t bar_d = bar_mma + 8 * kSlots;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTabs * 1024 + 8 * (2 * kSlots + 4));
+    const uint32_t bar_d = bar_mma + 8 * kSlots, bar_seg = bar_d + 16;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTabs * 1024 + 8 * (2 * kSlots + 6));
     const uint32_t sA = (sbase + kHead + 1023u) & ~1023u; // 1 KiB aligned, as the swizzle needs
     const uint32_t sS = sA + 2 * kStageA;                  // slot k at sS + k * kSlotBytes
     uint8_t* const gA = smem + (sA - sbase);
-    constexpr uint32_t kEpiThreads = 8 * 32;               // warps 0-7 read the accumulators out
+    constexpr uint32_t kEpiThreads = kEpiWarps * 32;
+    constexpr uint32_t kEpiWarp0 = kDecWarps + 1;          // the read-out warps follow the MMA warp
     if (tid == 0) {
         for (uint32_t k = 0; k < kSlots; ++k) {
             mbar_init(bar_slot + 8 * k, kDecThreads);
@@ -214,6 +218,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
         mbar_init(bar_a + 8, kDecThreads);
         mbar_init(bar_d, kEpiThreads);
         mbar_init(bar_d + 8, kEpiThreads);
+        mbar_init(bar_seg, 1);
+        mbar_init(bar_seg + 8, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kDecWarps) { // tensor memory: two 128 x (at most 64) FP32 accumulators
@@ -228,38 +234,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
     bool ok = true;
 
     if (tid < kDecThreads) {
-        // Reads segment g's accumulator (g & 1) out into Y: warp w (w < 8) reads tensor-memory
-        // lanes 32 (w % 4) .. +31 (rows of W) and columns (tokens) 32 (w / 4) .. +31. A
-        // segment that covers its row block's whole K range stores; the others add their part.
-        auto epilogue = [&](uint32_t g) {
-            if (warp >= 8) return;
-            const GemmSeg sg = s_seg[g];
-            const FwGemmItem& it = p.item[sg.item];
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const uint32_t quarter = warp & 3u, half = warp >> 2;
-            const uint32_t row = sg.row0 + quarter * 32 + lane;
-            for (uint32_t cb = half * 32; cb < half * 32 + 32 && cb < nt; cb += 16) {
-                uint32_t v[16];
-                const uint32_t taddr = tmem + ((quarter * 32) << 16) + (g & 1u) * 64 + cb;
-                asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-                             : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-                               "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-                             : "r"(taddr));
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-                for (uint32_t q = 0; q < 16; ++q) {
-                    const uint32_t tok = sg.tok0 + cb + q;
-                    if (tok < batch) {
-                        float* dst = it.y + uint64_t(tok) * it.rows + row;
-                        if (sg.full) *dst = __uint_as_float(v[q]);
-                        else atomicAdd(dst, __uint_as_float(v[q])); // Y was zeroed; parts add up
-                    }
-                }
-            }
-            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-            mbar_arrive(bar_d + 8 * (g & 1u));
-        };
-
         // The copies of slice q, split over the threads: A and B plane pieces (16 bytes, 4 a
         // row), C pieces (3 a row), tile_exc entries (2 a row) and X pieces (16 a token, placed
         // in the 128-byte swizzle; tokens past the batch are zero-filled, pieces past nt
@@ -368,7 +342,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
             gd_end = sg.q0 + 2 * sg.n;
         };
         if (nsl > 0) seg_decode(0);
-        uint32_t epi_next = 0;            // the next segment to read out
         for (uint32_t q = 0; q + 1 < kSlots && q < nsl; ++q) issue(q); // slices 0 .. kSlots - 2
         for (uint32_t q = 0; q < nsl && ok; ++q) {
             while (q >= gd_end) seg_decode(++gd);
@@ -404,7 +377,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
                 ok = false;
                 break;
             }
-            while (q >= 2 && epi_next < nseg && s_seg[epi_next].q0 + 2 * s_seg[epi_next].n <= q - 1) epilogue(epi_next++);
             uint8_t* const stA = gA + st * kStageA;
 #pragma unroll
             for (uint32_t i = 0; i < 4; ++i) {
@@ -440,10 +412,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
             if (qn < nsl && qn >= kSlots - 1) issue(qn);
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
-        // the segments not yet read out: after the last slice's MMAs
-        if (ok && nsl > 0 && warp < 8) {
-            ok = !*abort_flag && mbar_wait(bar_mma + 8 * ((nsl - 1) % kSlots), ((nsl - 1) / kSlots) & 1u, abort_flag);
-            while (ok && epi_next < nseg) epilogue(epi_next++);
+    } else if (warp >= kEpiWarp0) {
+        // The read-out warps: warp w reads tensor-memory lanes 32 (w % 4) .. +31 (rows of W) and
+        // every token column of segment g's accumulator (g & 1) once the segment's MMAs have
+        // completed, and writes Y. A segment that covers its row block's whole K range stores;
+        // the others add their part. The accumulator is then free for segment g + 2.
+        const uint32_t quarter = warp & 3u;
+        for (uint32_t g = 0; g < nseg && ok; ++g) {
+            if (!mbar_wait(bar_seg + 8 * (g & 1u), (g >> 1) & 1u, abort_flag)) { ok = false; break; }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const GemmSeg sg = s_seg[g];
+            const FwGemmItem& it = p.item[sg.item];
+            const uint32_t row = sg.row0 + quarter * 32 + lane;
+            for (uint32_t cb = 0; cb < nt; cb += 16) {
+                uint32_t v[16];
+                const uint32_t taddr = tmem + ((quarter * 32) << 16) + (g & 1u) * 64 + cb;
+                asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+                             : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                               "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+                             : "r"(taddr));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                for (uint32_t q = 0; q < 16; ++q) {
+                    const uint32_t tok = sg.tok0 + cb + q;
+                    if (tok < batch) {
+                        float* dst = it.y + uint64_t(tok) * it.rows + row;
+                        if (sg.full) *dst = __uint_as_float(v[q]);
+                        else atomicAdd(dst, __uint_as_float(v[q])); // Y was zeroed; parts add up
+                    }
+                }
+            }
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            mbar_arrive(bar_d + 8 * (g & 1u));
         }
     } else if (tid == kDecThreads) {
         // the MMA thread: M = 128, N = nt, BF16 x BF16 -> FP32, both operands K-major;
@@ -468,6 +468,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fw_gemm_kernel(const __grid_c
             }
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_mma + 8 * s)
                          : "memory");
+            if (q + 1 == s_seg[g].q0 + 2 * s_seg[g].n) // the segment's last slice: tell the read-out warps
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_seg + 8 * (g & 1u))
+                             : "memory");
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
