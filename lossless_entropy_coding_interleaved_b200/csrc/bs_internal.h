@@ -45,15 +45,17 @@ inline uint64_t payload_bytes(uint64_t n_c, uint32_t n_words, bool nib_stored) {
 
 // Decode-kernel geometry: a warp decodes `chains` chunks at once (independent state chains
 // per lane), and a CTA of `warps` warps covers warps*chains chunks of one tensor. Kind RANS
-// at the default precisions uses 24 warps of 2 chains, kind JOINT at nj = 13 28 warps of 2
-// (kWarpsJoint below), and the other precisions 20 warps of 2 (ns = 12 tables leave room
-// for 40 rings).
+// at the default precisions uses 24 warps of 2 chains; kind JOINT at nj = 13 uses 32 warps of
+// 2 with 4-byte table entries (kWarpsJoint4, bs_joint4.cu) and 28 warps of 2 with 8-byte ones
+// (kWarpsJoint below); the other precisions use 20 warps of 2 (ns = 12 tables leave room for
+// 40 rings).
 // Each chunk's 16-bit word stream goes through its own shared-memory ring of kRingBytes,
 // in quarters of kQuarterBytes (one 16-byte cp.async per lane fills a quarter), and its
 // nibble words through a ring of kNibRingBlocks blocks (128 bytes each).
 constexpr int kWarpsDefault = 24, kChainsDefault = 2, kWarpsGeneric = 20, kChainsGeneric = 2;
-// JOINT at the default precision (nj = 13): the table takes the first 64 KiB, then 56 rings of
-// each kind (204 KiB in all). 28 warps hold 72 registers a thread, the most that fits.
+// JOINT at the default precision (nj = 13) with 8-byte entries (a pair frequency above 255):
+// the table takes the first 64 KiB, then 56 rings of each kind (204 KiB in all). 28 warps
+// hold 72 registers a thread, the most that fits.
 constexpr int kWarpsJoint = 28, kChainsJoint = 2;
 inline bool is_default_precision(uint32_t ns, uint32_t nh) { return ns == 11 && nh == 5; }
 inline int warps_for(uint32_t ns, uint32_t nh) { return is_default_precision(ns, nh) ? kWarpsDefault : kWarpsGeneric; }
