@@ -15,7 +15,7 @@
 // row, are shared evenly among the 8 warps, so that no warp has more than one tile more than
 // another however few rows the CTA has (with whole rows per warp, a projection of 3584 rows
 // would leave 1.5 rows per warp and a quarter of the warps idle for the last row). A warp
-// walks its tiles in groups of up to 14 or 16 tiles inside one row, through a 2-slot cp.async ring.
+// walks its tiles in groups of up to 10, 14 or 16 tiles inside one row, through a 2-slot cp.async ring.
 // Per tile and lane, the 8 decoded weights meet 8 entries of x (one 16-byte load per batch
 // row; x is staged in shared memory when it is small, else served by L1/L2).
 //
@@ -79,7 +79,7 @@ __device__ __forceinline__ float fma_bf16x2(uint32_t w, uint32_t x, float acc) {
 // A warp walks its tiles in groups of up to GROUP tiles through a ring of two slots: while it
 // works on one group, the copies of the next are in flight. One slot: plane A and B words
 // (128 B per tile each), plane C (96 B per tile), and the tile_exc entries of the warp's
-// NEXT group (GROUP + 1 of them). Groups of 14 or 16 tiles keep the per-group work (copy
+// NEXT group (GROUP + 1 of them). Groups of 10 to 16 tiles keep the per-group work (copy
 // issue, exception list, bookkeeping) small per tile.
 constexpr int kGemvStages = 2;
 template <int GROUP>
@@ -368,9 +368,13 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) fw_gemv_kernel(const __gri
     }
 }
 
-// The group size of a product: 14 when it divides the row's tile count, else 16 (groups are cut
-// at row ends, so any row length works).
-inline int gemv_group_for(uint32_t cols) { return (cols / 256) % 14 == 0 ? 14 : 16; }
+// The group size of a product: 16, 14 or 10 when it divides the row's tile count (rows of 16,
+// 14, 56 tiles in the 9B-shaped model, 20 and 100 in the 27B-shaped one), so that every group
+// is whole; else 16 (groups are cut at row ends, so any row length works).
+inline int gemv_group_for(uint32_t cols) {
+    const uint32_t tpr = cols / 256;
+    return tpr % 16 == 0 ? 16 : tpr % 14 == 0 ? 14 : tpr % 10 == 0 ? 10 : 16;
+}
 
 // The kernel instance for (batch, group, x staged or not) and its shared memory, without x.
 struct GemvKernel {
@@ -395,7 +399,7 @@ GemvKernel gemv_kernel_b(uint32_t batch, bool xs) {
     }
 }
 GemvKernel gemv_kernel(uint32_t batch, int group, bool xs) {
-    return group == 14 ? gemv_kernel_b<14>(batch, xs) : gemv_kernel_b<16>(batch, xs);
+    return group == 14 ? gemv_kernel_b<14>(batch, xs) : group == 10 ? gemv_kernel_b<10>(batch, xs) : gemv_kernel_b<16>(batch, xs);
 }
 
 } // namespace
@@ -429,7 +433,7 @@ extern "C" bs_status bs_fw_gemv(int32_t n, const bs_fw_gemv_item* items, uint32_
     p.err = d_err;
     p.layouts_resident = (flags & BS_FW_LAYOUTS_RESIDENT) ? 1u : 0u;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    for (int group : {16, 14}) {
+    for (int group : {16, 14, 10}) {
         uint32_t max_cols = 0;
         for (int32_t k = 0; k < n; ++k)
             if (items[k].info.n_elems && gemv_group_for(items[k].cols) == group) max_cols = std::max(max_cols, items[k].cols);
