@@ -97,6 +97,19 @@ def test_gemv_rows_split_between_warps_are_exact_sums(rows, cols):
         assert np.array_equal(y2.cpu().numpy().view(np.uint32), y.astype(np.float32).view(np.uint32))
 
 
+@pytest.mark.parametrize("batch", [2, 4, 5, 6, 7])
+def test_gemv_every_batch_instance(batch):
+    # one kernel instance per batch size; rows of 20 tiles (cols 5120) take groups of 10
+    rows, cols = 200, 5120
+    w = _gauss(rows * cols, seed=55).reshape(rows, cols)
+    x = _gauss(batch * cols, seed=56 + batch, scale=1.0).reshape(batch, cols)
+    (y,), err, items = _run([(w, x)], batch)
+    assert err == 0 and items[0][1].n_exc > 0
+    blob = oracle.fw_encode(w)
+    ref = oracle.fw_gemv(blob, rows, cols, x)
+    assert np.all(np.abs(y - ref) <= _tolerance(w, x, oracle.fw_info(blob)["table"][0]))
+
+
 def test_gemv_many_escapes_per_group():
     rows, cols = 40, 1024
     w = _gauss(rows * cols, seed=3, scale=1.0).reshape(rows, cols)
