@@ -20,12 +20,13 @@ def _layer_key(name: str):
     return name.split(".")[1] if name.startswith("layers.") else "misc"
 
 
-@pytest.fixture(scope="module")
-def model():
-    """Four full-shape Gemma-2-9B layers plus the edge mix, as one host container."""
+@pytest.fixture(scope="module", params=["factored", "joint"])
+def model(request):
+    """Four full-shape Gemma-2-9B layers plus the edge mix, as one host container, in kind
+    RANS (the factored model) and in kind JOINT (the bench's default)."""
     specs = S.workload("gemma2_9b", layers=4) + S.workload("edge_mix")
     dev = [(s.name, S.generate(s, "cuda:0")) for s in specs]
-    _, h_c = bs.encode(dev, host_copy=True)
+    _, h_c = bs.encode(dev, host_copy=True, model=request.param)
     del dev
     torch.cuda.empty_cache()
     return specs, h_c
