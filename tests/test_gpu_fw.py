@@ -177,11 +177,13 @@ def test_position_past_tensor_is_flagged_and_contained():
     assert np.array_equal(got[:256 * 4], w[:256 * 4])
 
 
-def test_layout_from_container_matches_oracle():
-    # the runtime path: rANS container -> decode on the device -> FW layout on the device
+@pytest.mark.parametrize("model", ["factored", "joint"])
+def test_layout_from_container_matches_oracle(model):
+    # the runtime path: rANS container (kind RANS or JOINT) -> decode on the device -> FW
+    # layout on the device
     specs = [s for s in S.workload("edge_mix") if not s.is_raw]
     arrs = [S.words_numpy(S.generate(s, "cpu")) for s in specs]
-    c = oracle.encode([(s.name, a, "bf16") for s, a in zip(specs, arrs)])
+    c = oracle.encode([(s.name, a, "bf16") for s, a in zip(specs, arrs)], model=model)
     plan = bs.Plan(c, device="cuda:0")
     for k, a in enumerate(arrs):
         fw, info = plan.to_fw(k)
