@@ -104,6 +104,9 @@ _TRAFFIC = {
     # written for 1,585,561,600 weights
     "joint4_decode_kernel": (("bs_joint4.cu", "bs_device.cuh", "bs_internal.h"), "d8127505dd5bd2be", 3.28706),
     "fw_decode_kernel": (("bs_fw.cu", "bs_fw.cuh"), None, None),
+    # fw_gemv_kernel, batch 1, the gate/up call of the 9B checkpoint's layer 0 (two 14336 x
+    # 3584 matrices): 148.79 MB read + 3.63 MB written for 102,760,448 weights
+    "fw_gemv_kernel": (("bs_fw_gemv.cu", "bs_fw.cuh"), "12b694d32f782e9f", 1.48328),
 }
 
 
@@ -1392,6 +1395,7 @@ def run_gemv(a):
     ranks.close()
     if rank != 0:
         return
+    gemv_tpw = _traffic_per_weight("fw_gemv_kernel") if (not tensor and batch == 1) else None
     print(json.dumps({
         "metric": GEMV_METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True, "scaling": "weak",
@@ -1408,7 +1412,10 @@ def run_gemv(a):
                    "parallelism": f"replicas x{world} (no collective on the data path)",
                    "l2": "no flush: the layouts (GBs) are larger than L2"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": (None if gemv_tpw is None else int(gemv_tpw * n_w)),
+                     "traffic_source": ("ncu capture of this kernel at batch 1 on one gate/up call, scaled by weights"
+                                        if gemv_tpw is not None else None),
                      "kernel": kernel, "per_step_bytes": int(fw_bytes + xy_bytes),
                      "tflops": round(2.0 * n_w * batch / (step_ms * 1e-3) / 1e12, 2),
                      "launches_per_step": int(launches_per_pass)},
